@@ -1,0 +1,223 @@
+"""Seeded synthetic inputs for the activation-sparse gated FFN.
+
+This module only draws and quantises input tensors.  It holds none of the
+method's arithmetic (no gate, no activation, no selection, no projection), so
+that both the fp64 oracle and the CUDA path can be fed from it without sharing
+any code with each other.
+
+Every tensor is drawn from ``numpy.random.default_rng([seed, tensor_id])``
+(PCG64 seeded through SeedSequence) in float32, scaled, and then rounded to the
+operand dtype (bf16 by round-to-nearest-even through torch, or kept in fp32).
+
+Tensor ids: x = 0, W_gate = 1, W_up = 2, W_down = 3, A = 4, B = 5, bias = 6,
+nnz draw = 7, exact-grid sparsity pattern of A = 8.
+
+Weight scales follow N(0, 1/fan_in): fan_in = d for W_gate, W_up and A, r for
+B, and d_ff for W_down (the down projection sums over the d_ff neurons).  All
+weights are stored neuron-major, i.e. W_gate, W_up and W_down are [d_ff][d]
+row-major; row j belongs to neuron j.  A is [d][r] and B is [r][d_ff], so the
+low-rank gate is x·A·B.
+
+Workload recipes (the activation statistics that the pages' trained models
+produce, stood in for by Gaussian draws):
+
+* ``tiny_fp32``: d=256, d_ff=1024, T=64, fp32, ReLU, bias -1.2816 per neuron
+  (P(N(0,1) > 1.2816) = 0.1000, about 90 % zeros), threshold 0, C = 128.
+* ``decode_bf16``: d=4096, d_ff=14336, T in {1, 4, 8}, bf16, same gate
+  statistics (about 90 % zeros), C = 32.
+* ``lopa_bf16``: low-rank gate with r = d/8 = 512 (rank ratio 1/8 of the
+  LoPA page), A ~ N(0, 1/d), B ~ N(0, 1/r) so x·A·B has unit variance; bias
+  -1.2816 (about 90 % zeros); T = 32; C = 32.
+* ``prefill_bf16``: d=2048, d_ff=8192, T=4096.  Per-token activity
+  nnz_t = min(d_ff, round(exp(ln 60 + xi_t))), xi_t ~ N(0, 1) (lognormal,
+  median 60, mean 60·e^0.5 = 98.9, i.e. about 98.8 % sparsity).  Realised by
+  x_t = s_t·z_t with z_t ~ N(0, I), bias -beta (beta = 3) and
+  s_t = beta / Phi^-1(1 - min(nnz_t/d_ff, 0.45)), so that
+  P(g_tj > 0) = min(nnz_t/d_ff, 0.45).  C = 8, so heavy tokens overflow.
+* ``wina_bf16``: d=4096, d_ff=14336, T=32, SiLU, no bias, keep the top
+  k = round(0.35·14336) = 5018 neurons per token, C = 128.
+
+The optional ``exact_grid`` flag quantises every operand to a coarse dyadic
+grid (x to multiples of 2^-4, weights to k·2^-e with |k| <= 255, the bias to
+the 2^-14 accumulator grid) so that every fp32 partial sum of the gate and up
+projections is exact in any order; parity runs use it to demand bit-exact
+TwELL values as well as indices.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+from statistics import NormalDist
+from typing import Optional
+
+import numpy as np
+import torch
+
+TID_X, TID_WGATE, TID_WUP, TID_WDOWN, TID_A, TID_B, TID_BIAS, TID_NNZ, TID_APAT = range(9)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    d_model: int
+    d_ff: int
+    tokens: int
+    dtype: str = "bf16"          # "bf16" or "fp32"
+    mode: str = "relu_threshold"  # or "wina_topk"
+    act: str = "relu"            # "relu" or "silu"
+    rank: int = 0                # 0 = dense gate
+    bias: Optional[float] = -1.2816
+    threshold: float = 0.0
+    k: int = 0
+    tile_capacity: int = 32
+    x_kind: str = "gauss"        # "gauss" or "lognormal_nnz"
+    beta: float = 3.0            # prefill bias magnitude
+    nnz_mu: float = math.log(60.0)
+    nnz_sigma: float = 1.0
+    nnz_cap_frac: float = 0.45
+    exact_grid: bool = False
+    seed: int = 0
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", 256, 1024, 64, dtype="fp32", tile_capacity=128),
+    "decode_bf16": Workload("decode_bf16", 4096, 14336, 8, tile_capacity=32),
+    "lopa_bf16": Workload("lopa_bf16", 4096, 14336, 32, rank=512, tile_capacity=32),
+    "prefill_bf16": Workload("prefill_bf16", 2048, 8192, 4096, tile_capacity=8,
+                             x_kind="lognormal_nnz", bias=None),
+    "wina_bf16": Workload("wina_bf16", 4096, 14336, 32, mode="wina_topk", act="silu",
+                          bias=None, k=5018, tile_capacity=128),
+}
+
+
+def _rng(seed: int, tid: int) -> np.random.Generator:
+    return np.random.default_rng([int(seed), int(tid)])
+
+
+def _normal(seed: int, tid: int, shape, scale: float) -> np.ndarray:
+    a = _rng(seed, tid).standard_normal(int(np.prod(shape)), dtype=np.float32)
+    a *= np.float32(scale)
+    return a.reshape(shape)
+
+
+def _to_dtype(a: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    if dtype == "bf16":
+        return t.to(torch.bfloat16)
+    if dtype == "fp32":
+        return t.clone()
+    raise ValueError(dtype)
+
+
+def _grid(a: np.ndarray, e: int, kmax: int = 255) -> np.ndarray:
+    """Quantise to integer multiples of 2^-e with |k| <= kmax (exact in bf16)."""
+    k = np.clip(np.rint(a.astype(np.float64) * (2.0 ** e)), -kmax, kmax)
+    return (k / (2.0 ** e)).astype(np.float32)
+
+
+def _grid_exp(std: float) -> int:
+    """Grid exponent e such that a N(0, std^2) draw spans about +-16 grid units
+    per standard deviation (and fits |k| <= 255 with a 16-sigma margin)."""
+    return int(round(math.log2(16.0 / std)))
+
+
+@dataclass
+class Inputs:
+    """Host tensors for one workload.  Weights are neuron-major [d_ff][d]."""
+    wl: Workload
+    x: torch.Tensor
+    W_gate: Optional[torch.Tensor]
+    A: Optional[torch.Tensor]
+    B: Optional[torch.Tensor]
+    W_up: torch.Tensor
+    W_down: torch.Tensor
+    bias: Optional[torch.Tensor]          # fp32 [d_ff] or None
+    nnz_target: Optional[np.ndarray] = None
+    extra: dict = field(default_factory=dict)
+
+
+def token_scales(wl: Workload, T: Optional[int] = None) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token activity targets and x scales of the lognormal-nnz recipe."""
+    T = wl.tokens if T is None else T
+    xi = _normal(wl.seed, TID_NNZ, (T,), 1.0).astype(np.float64)
+    nnz = np.minimum(wl.d_ff, np.rint(np.exp(wl.nnz_mu + wl.nnz_sigma * xi)))
+    nnz = np.maximum(nnz, 1.0)
+    p = np.minimum(nnz / wl.d_ff, wl.nnz_cap_frac)
+    inv = NormalDist()
+    s = np.array([wl.beta / inv.inv_cdf(1.0 - pi) for pi in p])
+    return nnz.astype(np.int64), s
+
+
+def make_inputs(wl: Workload, T: Optional[int] = None, weights_only: bool = False,
+                x_only: bool = False) -> Inputs:
+    """Draw the seeded tensors of ``wl`` (optionally with a different token count)."""
+    T = wl.tokens if T is None else T
+    d, F, r, seed = wl.d_model, wl.d_ff, wl.rank, wl.seed
+    eg = wl.exact_grid
+
+    # activations
+    nnz = None
+    x = None
+    if not weights_only:
+        if wl.x_kind == "gauss":
+            xa = _normal(seed, TID_X, (T, d), 1.0)
+            if eg:
+                xa = _grid(xa, 4)
+        elif wl.x_kind == "lognormal_nnz":
+            nnz, s = token_scales(wl, T)
+            xa = _normal(seed, TID_X, (T, d), 1.0) * s[:, None].astype(np.float32)
+            if eg:
+                # x_t = s_t·z_t on the 2^-3 grid (s_t reaches about 24)
+                xa = _grid(xa, 3, kmax=4095)
+        else:
+            raise ValueError(wl.x_kind)
+        x = _to_dtype(xa, wl.dtype)
+    if x_only:
+        return Inputs(wl, x, None, None, None, None, None, None, nnz)
+
+    def wmat(tid, shape, fan_in):
+        std = 1.0 / math.sqrt(fan_in)
+        a = _normal(seed, tid, shape, std)
+        if eg:
+            a = _grid(a, _grid_exp(std))
+        return _to_dtype(a, wl.dtype)
+
+    W_gate = A = B = None
+    if r == 0:
+        W_gate = wmat(TID_WGATE, (F, d), d)
+    else:
+        if eg:
+            # exact-grid low-rank gate: every column of A holds 8 entries of
+            # +-1/2 and zeros elsewhere, so each z = x·A is a sum of 8 grid
+            # values, exact in fp32 and on the 2^-5 grid after bf16 rounding.
+            rng = _rng(seed, TID_APAT)
+            Aa = np.zeros((d, r), dtype=np.float32)
+            for c in range(r):
+                rows = rng.choice(d, size=8, replace=False)
+                Aa[rows, c] = rng.choice(np.array([-0.5, 0.5], dtype=np.float32), size=8)
+            A = _to_dtype(Aa, wl.dtype)
+        else:
+            A = wmat(TID_A, (d, r), d)
+        B = wmat(TID_B, (r, F), r)
+    W_up = wmat(TID_WUP, (F, d), d)
+    W_down = wmat(TID_WDOWN, (F, d), F)
+
+    bias = None
+    if wl.x_kind == "lognormal_nnz":
+        bias = torch.full((F,), -wl.beta, dtype=torch.float32)
+    elif wl.bias is not None:
+        b = wl.bias
+        if eg:
+            b = round(b * 2.0 ** 14) / 2.0 ** 14
+        bias = torch.full((F,), b, dtype=torch.float32)
+    return Inputs(wl, x, W_gate, A, B, W_up, W_down, bias, nnz)
+
+
+def to_f64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:
+    """Exact decode of a bf16/fp32 tensor to a float64 numpy array."""
+    if t is None:
+        return None
+    return t.detach().to("cpu").to(torch.float64).numpy()
