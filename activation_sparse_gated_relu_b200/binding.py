@@ -1,0 +1,283 @@
+"""ctypes binding of libsffn.so: the same entry points as include/sffn.h.
+
+Argument marshalling only.  Every step of the forward runs in the library's
+CUDA kernels; if the library is missing this module raises instead of falling
+back to anything else.  PyTorch supplies device memory and the stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsffn.so")
+
+# status codes (include/sffn.h)
+SFFN_OK, SFFN_ERR_INVALID_ARG, SFFN_ERR_UNSUPPORTED, SFFN_ERR_ALLOC, SFFN_ERR_CUDA, \
+    SFFN_ERR_TIMEOUT, SFFN_ERR_DEVICE, SFFN_ERR_NO_DEVICE = range(8)
+SFFN_BF16, SFFN_FP32 = 0, 1
+SFFN_MODE_RELU_THRESHOLD, SFFN_MODE_WINA_TOPK = 0, 1
+SFFN_ACT_RELU, SFFN_ACT_SILU = 0, 1
+SFFN_PATH_AUTO, SFFN_PATH_ROWS, SFFN_PATH_TILES = 0, 1, 2
+SFFN_FLAG_DEBUG_GATE = 1
+
+
+class sffn_desc(ctypes.Structure):
+    _fields_ = [
+        ("d_model", ctypes.c_int), ("d_ff", ctypes.c_int), ("max_tokens", ctypes.c_int),
+        ("rank", ctypes.c_int), ("dtype", ctypes.c_int), ("mode", ctypes.c_int),
+        ("act", ctypes.c_int), ("threshold", ctypes.c_float), ("k", ctypes.c_int),
+        ("tile_capacity", ctypes.c_int), ("path", ctypes.c_int), ("flags", ctypes.c_uint),
+        ("W_gate", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+        ("W_up", ctypes.c_void_p), ("W_down", ctypes.c_void_p), ("gate_bias", ctypes.c_void_p),
+    ]
+
+
+class sffn_stats(ctypes.Structure):
+    _fields_ = [("n_overflow", ctypes.c_int), ("n_launches", ctypes.c_int), ("path", ctypes.c_int),
+                ("epoch", ctypes.c_uint)]
+
+
+class SffnError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})" if what else status_string(status))
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsffn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m activation_sparse_gated_relu_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, ip, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int
+    lib.sffn_create.argtypes = [ctypes.POINTER(sffn_desc), vp, ctypes.POINTER(vp)]
+    lib.sffn_create.restype = st
+    lib.sffn_forward.argtypes = [vp, vp, ip, vp, vp]
+    lib.sffn_forward.restype = st
+    lib.sffn_forward_host.argtypes = [vp, vp, ip, vp, vp]
+    lib.sffn_forward_host.restype = st
+    lib.sffn_destroy.argtypes = [vp]
+    lib.sffn_destroy.restype = st
+    lib.sffn_status_string.argtypes = [st]
+    lib.sffn_status_string.restype = ctypes.c_char_p
+    lib.sffn_read_status.argtypes = [vp, vp]
+    lib.sffn_read_status.restype = st
+    lib.sffn_debug_twell.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                     ctypes.POINTER(vp), ctypes.POINTER(ip), ctypes.POINTER(ip)]
+    lib.sffn_debug_twell.restype = st
+    lib.sffn_debug_gate.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.sffn_debug_gate.restype = st
+    lib.sffn_debug_norms.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.sffn_debug_norms.restype = st
+    lib.sffn_get_stats.argtypes = [vp, vp, ctypes.POINTER(sffn_stats)]
+    lib.sffn_get_stats.restype = st
+    lib.sffn_timing_begin.argtypes = [vp, ip]
+    lib.sffn_timing_begin.restype = st
+    lib.sffn_timing_end.argtypes = [vp, ip, vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ip),
+                                    ctypes.POINTER(ip)]
+    lib.sffn_timing_end.restype = st
+    lib.sffn_version.argtypes = []
+    lib.sffn_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load_library().sffn_status_string(int(s)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != SFFN_OK:
+        raise SffnError(status, what)
+
+
+# ----------------------------------------------------------------- raw entry points
+def sffn_create(desc: sffn_desc, stream: int = 0) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(load_library().sffn_create(ctypes.byref(desc), ctypes.c_void_p(stream), ctypes.byref(h)),
+           "sffn_create")
+    return h
+
+
+def sffn_forward(h, x_ptr: int, T: int, out_ptr: int, stream: int = 0) -> None:
+    _check(load_library().sffn_forward(h, ctypes.c_void_p(x_ptr), int(T), ctypes.c_void_p(out_ptr),
+                                       ctypes.c_void_p(stream)), "sffn_forward")
+
+
+def sffn_forward_host(h, x_ptr: int, T: int, out_ptr: int, stream: int = 0) -> None:
+    _check(load_library().sffn_forward_host(h, ctypes.c_void_p(x_ptr), int(T),
+                                            ctypes.c_void_p(out_ptr), ctypes.c_void_p(stream)),
+           "sffn_forward_host")
+
+
+def sffn_destroy(h) -> None:
+    _check(load_library().sffn_destroy(h), "sffn_destroy")
+
+
+def sffn_read_status(h, stream: int = 0) -> int:
+    return load_library().sffn_read_status(h, ctypes.c_void_p(stream))
+
+
+def sffn_get_stats(h, stream: int = 0) -> sffn_stats:
+    st = sffn_stats()
+    _check(load_library().sffn_get_stats(h, ctypes.c_void_p(stream), ctypes.byref(st)), "sffn_get_stats")
+    return st
+
+
+def sffn_timing_begin(h, max_forwards: int) -> None:
+    _check(load_library().sffn_timing_begin(h, int(max_forwards)), "sffn_timing_begin")
+
+
+def sffn_timing_end(h) -> dict:
+    """{label: (total_ms, launches)} over the forwards timed since sffn_timing_begin."""
+    n_max = 16
+    names = (ctypes.c_char * 32 * n_max)()
+    ms = (ctypes.c_float * n_max)()
+    cnt = (ctypes.c_int * n_max)()
+    n = ctypes.c_int()
+    _check(load_library().sffn_timing_end(h, n_max, ctypes.cast(names, ctypes.c_void_p), ms, cnt,
+                                          ctypes.byref(n)), "sffn_timing_end")
+    return {names[i].value.decode(): (float(ms[i]), int(cnt[i])) for i in range(min(n.value, n_max))}
+
+
+def sffn_version() -> str:
+    return load_library().sffn_version().decode()
+
+
+# ----------------------------------------------------------------- torch convenience
+class _CudaView:
+    """Zero-copy __cuda_array_interface__ view of library-owned device memory."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+def _view(ptr: int, shape, typestr: str, torch_dtype=None):
+    import torch
+    t = torch.as_tensor(_CudaView(ptr, shape, typestr), device="cuda")
+    if torch_dtype is not None:
+        t = t.view(torch_dtype)
+    return t.clone()
+
+
+_DTYPE = {"bf16": SFFN_BF16, "fp32": SFFN_FP32}
+_MODE = {"relu_threshold": SFFN_MODE_RELU_THRESHOLD, "wina_topk": SFFN_MODE_WINA_TOPK}
+_ACT = {"relu": SFFN_ACT_RELU, "silu": SFFN_ACT_SILU}
+_PATH = {"auto": SFFN_PATH_AUTO, "rows": SFFN_PATH_ROWS, "tiles": SFFN_PATH_TILES}
+
+
+class SparseFFN:
+    """A handle over device tensors (the tensors are kept alive by the object).
+
+    Weights are neuron-major [d_ff][d_model] (W_down is down_proj.weight^T);
+    A is [d_model][rank], B is [rank][d_ff]; bias is fp32 [d_ff].
+    """
+
+    def __init__(self, W_up, W_down, *, W_gate=None, A=None, B=None, bias=None,
+                 mode: str = "relu_threshold", act: str = "relu", threshold: float = 0.0,
+                 k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
+                 debug_gate: bool = False, stream: Optional[int] = None):
+        import torch
+        self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias) if t is not None]
+        dt = W_up.dtype
+        if dt not in (torch.bfloat16, torch.float32):
+            raise TypeError("operands must be bf16 or fp32")
+        self.dtype = "bf16" if dt == torch.bfloat16 else "fp32"
+        F, d = W_up.shape
+        self.d_model, self.d_ff, self.max_tokens = d, F, max_tokens
+        desc = sffn_desc()
+        desc.d_model, desc.d_ff, desc.max_tokens = d, F, max_tokens
+        desc.rank = 0 if A is None else A.shape[1]
+        desc.dtype = _DTYPE[self.dtype]
+        desc.mode = _MODE[mode]
+        desc.act = _ACT[act]
+        desc.threshold = float(threshold)
+        desc.k = int(k)
+        desc.tile_capacity = int(tile_capacity)
+        desc.path = _PATH[path]
+        desc.flags = SFFN_FLAG_DEBUG_GATE if debug_gate else 0
+        ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        desc.W_gate, desc.A, desc.B = ptr(W_gate), ptr(A), ptr(B)
+        desc.W_up, desc.W_down, desc.gate_bias = ptr(W_up), ptr(W_down), ptr(bias)
+        self.desc = desc
+        self.h = sffn_create(desc, self._stream(stream))
+
+    @staticmethod
+    def _stream(stream: Optional[int]) -> int:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if stream is None else int(stream)
+
+    def forward(self, x, out=None, stream: Optional[int] = None):
+        import torch
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
+        sffn_forward(self.h, x.data_ptr(), T, out.data_ptr(), self._stream(stream))
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, x_host, out_host=None, stream: Optional[int] = None):
+        import torch
+        T = x_host.shape[0]
+        if out_host is None:
+            out_host = torch.empty((T, self.d_model), dtype=torch.float32, pin_memory=True)
+        sffn_forward_host(self.h, x_host.data_ptr(), T, out_host.data_ptr(), self._stream(stream))
+        return out_host
+
+    def twell(self, T: int) -> dict:
+        """Copies of the last forward's TwELL records and overflow flags."""
+        lib = load_library()
+        vp = ctypes.c_void_p
+        c, i, v, o = vp(), vp(), vp(), vp()
+        nt, cap = ctypes.c_int(), ctypes.c_int()
+        _check(lib.sffn_debug_twell(self.h, ctypes.byref(c), ctypes.byref(i), ctypes.byref(v),
+                                    ctypes.byref(o), ctypes.byref(nt), ctypes.byref(cap)), "twell")
+        P, C = nt.value, cap.value
+        import torch
+        vt = ("<u2", torch.bfloat16) if self.dtype == "bf16" else ("<f4", None)
+        return {"count": _view(c.value, (T, P), "<i2"), "idx": _view(i.value, (T, P, C), "<i2"),
+                "val": _view(v.value, (T, P, C), vt[0], vt[1]),
+                "overflow_epoch": _view(o.value, (T,), "<u4")}
+
+    def gate_debug(self, T: int):
+        g = ctypes.c_void_p()
+        _check(load_library().sffn_debug_gate(self.h, ctypes.byref(g)), "gate_debug")
+        return _view(g.value, (T, self.d_ff), "<f4")
+
+    def norms(self):
+        n = ctypes.c_void_p()
+        _check(load_library().sffn_debug_norms(self.h, ctypes.byref(n)), "norms")
+        return _view(n.value, (self.d_ff,), "<f4")
+
+    def stats(self, stream: Optional[int] = None) -> sffn_stats:
+        return sffn_get_stats(self.h, self._stream(stream))
+
+    def timing_begin(self, max_forwards: int) -> None:
+        sffn_timing_begin(self.h, max_forwards)
+
+    def timing_end(self) -> dict:
+        return sffn_timing_end(self.h)
+
+    def read_status(self, stream: Optional[int] = None) -> int:
+        return sffn_read_status(self.h, self._stream(stream))
+
+    def close(self) -> None:
+        if getattr(self, "h", None) is not None and self.h.value:
+            sffn_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

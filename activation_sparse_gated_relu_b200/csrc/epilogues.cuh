@@ -1,0 +1,384 @@
+// Epilogues of the tensor-core tile kernel.  In every one of them the 128
+// epilogue threads hold one accumulator row each (a neuron, a low-rank
+// coordinate or an output column) and 16 consecutive columns (tokens) at a
+// time, read from TMEM with tcgen05.ld.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace sffn {
+
+enum : int { ACT_RELU = 0, ACT_SILU = 1 };
+
+__device__ __forceinline__ float act_fn(float g, int act) {
+  return act == ACT_RELU ? fmaxf(g, 0.0f) : g / (1.0f + expf(-g));
+}
+
+// ------------------------------------------------------------------ TwELL
+// TwELL emission for one chunk of 16 tokens, shared by the tensor-core gate
+// and the fp32 SIMT gate.  Called by 128 threads (4 full warps); thread etid
+// owns neuron j of tile p = j / 128 (j % 128 == etid) and holds g (pre-bias)
+// for tokens t0..t0+15.  Kept neurons are compacted per token with warp
+// ballots: the rank of neuron j among the kept neurons of its tile is the
+// popcount of the kept bits of lower lanes in lower warps and in its own warp,
+// which is its slot (ascending neuron order).
+struct TwellParams {
+  const float* bias;  // [F] or null
+  float tau;
+  int act;
+  int T, F, n_tiles, C;
+  int16_t* count;     // [T][n_tiles]
+  int16_t* idx;       // [T][n_tiles][C]
+  void* val;          // [T][n_tiles][C] bf16 or fp32
+  int val_f32;
+  uint32_t* ovf;      // [T]: = epoch iff the token overflows in this forward
+  uint32_t epoch;
+  uint32_t* umask;    // [ceil(T/8)][n_tiles][4] union of kept bits per 8-token block, or null
+  float* gdebug;      // [T][F] dense gate (debug), or null
+};
+
+__device__ __forceinline__ void twell_chunk(const TwellParams& o, const float* g, int j, int t0, int etid,
+                                            uint32_t* masks /*[4][16]*/) {
+  const int w = etid >> 5, lane = etid & 31;
+  const int p = j >> 7;
+  const float b = o.bias ? o.bias[j] : 0.0f;
+  float a[16];
+  uint32_t keep = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float gv = g[i] + b;
+    a[i] = act_fn(gv, o.act);
+    const bool in = (t0 + i) < o.T;
+    const bool k = in && fabsf(a[i]) > o.tau;
+    keep |= (k ? 1u : 0u) << i;
+    if (o.gdebug && in) o.gdebug[(size_t)(t0 + i) * o.F + j] = gv;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, k);
+    if (lane == 0) masks[w * 16 + i] = bal;
+  }
+  if (o.umask) {
+    const uint32_t u0 = __ballot_sync(0xFFFFFFFFu, (keep & 0x00FFu) != 0);
+    const uint32_t u1 = __ballot_sync(0xFFFFFFFFu, (keep & 0xFF00u) != 0);
+    if (lane == 0) {
+      const int blk = t0 >> 3;
+      if (t0 < o.T) o.umask[((size_t)blk * o.n_tiles + p) * 4 + w] = u0;
+      if (t0 + 8 < o.T) o.umask[((size_t)(blk + 1) * o.n_tiles + p) * 4 + w] = u1;
+    }
+  }
+  named_bar_sync(1, 128);
+  const uint32_t lt = lanemask_lt();
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const int t = t0 + i;
+    if (t >= o.T) break;
+    const uint32_t m0 = masks[i], m1 = masks[16 + i], m2 = masks[32 + i], m3 = masks[48 + i];
+    const int c0 = __popc(m0), c1 = __popc(m1), c2 = __popc(m2), c3 = __popc(m3);
+    const int total = c0 + c1 + c2 + c3;
+    const uint32_t mw = w == 0 ? m0 : w == 1 ? m1 : w == 2 ? m2 : m3;
+    const int pre = (w > 0 ? c0 : 0) + (w > 1 ? c1 : 0) + (w > 2 ? c2 : 0) + __popc(mw & lt);
+    const size_t base = ((size_t)t * o.n_tiles + p) * o.C;
+    if (((keep >> i) & 1u) && pre < o.C) {
+      o.idx[base + pre] = (int16_t)j;
+      if (o.val_f32)
+        reinterpret_cast<float*>(o.val)[base + pre] = a[i];
+      else
+        reinterpret_cast<__nv_bfloat16*>(o.val)[base + pre] = __float2bfloat16_rn(a[i]);
+    }
+    if (etid >= total && etid < o.C) {
+      o.idx[base + etid] = -1;
+      if (o.val_f32)
+        reinterpret_cast<float*>(o.val)[base + etid] = 0.0f;
+      else
+        reinterpret_cast<__nv_bfloat16*>(o.val)[base + etid] = __float2bfloat16_rn(0.0f);
+    }
+    if (etid == 0) {
+      o.count[(size_t)t * o.n_tiles + p] = (int16_t)total;
+      if (total > o.C) o.ovf[t] = o.epoch;
+    }
+  }
+}
+
+struct EpiGateTwell {
+  static constexpr int N_ACC = 1;
+  using Params = TwellParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t* scratch) {
+    uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);
+    const int j = m0 + etid;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.T) break;
+      float g[16];
+      tmem_ld16(tmem + c, g);
+      twell_chunk(o, g, j, n0 + c, etid, masks + ((c >> 4) & 1) * 64);
+    }
+  }
+};
+
+// ------------------------------------------------------------------- WINA
+// Dense activation and score for the per-token top-k: v = round(sigma(g+b)),
+// s = |sigma(g+b)|·n_j, both [T][F].
+struct WinaParams {
+  const float* bias;
+  int act, T, F;
+  const float* norms;
+  void* vdense;       // [T][F] bf16 or fp32
+  int val_f32;
+  float* scores;      // [T][F]
+};
+
+__device__ __forceinline__ void wina_chunk(const WinaParams& o, const float* g, int j, int t0) {
+  const float b = o.bias ? o.bias[j] : 0.0f;
+  const float n = o.norms[j];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int t = t0 + i;
+    if (t < o.T) {
+      const float a = act_fn(g[i] + b, o.act);
+      const size_t off = (size_t)t * o.F + j;
+      if (o.val_f32)
+        reinterpret_cast<float*>(o.vdense)[off] = a;
+      else
+        reinterpret_cast<__nv_bfloat16*>(o.vdense)[off] = __float2bfloat16_rn(a);
+      o.scores[off] = fabsf(a) * n;
+    }
+  }
+}
+
+struct EpiWina {
+  static constexpr int N_ACC = 1;
+  using Params = WinaParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int j = m0 + etid;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.T) break;
+      float g[16];
+      tmem_ld16(tmem + c, g);
+      wina_chunk(o, g, j, n0 + c);
+    }
+  }
+};
+
+// ------------------------------------------------------- low-rank gate: z
+// z = round_bf16(x·A).  The tile's rows are rank coordinates r, its columns
+// tokens.  With a split K the partial sums are added into zacc (fp32, zero
+// between forwards) and the last CTA of the row tile rounds, stores z and
+// clears zacc and its ticket.
+struct ZParams {
+  int T, R, splits;
+  float* zacc;             // [maxT][R]
+  __nv_bfloat16* z;        // [maxT][R]
+  int* tickets;            // [R/128]
+};
+
+struct EpiLowRankZ {
+  static constexpr int N_ACC = 1;
+  using Params = ZParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t* scratch) {
+    const int r = m0 + etid;
+    const bool rin = r < o.R;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.T) break;
+      float g[16];
+      tmem_ld16(tmem + c, g);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = n0 + c + i;
+        if (t < o.T && rin) {
+          if (o.splits == 1)
+            o.z[(size_t)t * o.R + r] = __float2bfloat16_rn(g[i]);
+          else
+            atomicAdd(&o.zacc[(size_t)t * o.R + r], g[i]);
+        }
+      }
+    }
+    if (o.splits == 1) return;
+    int* last = reinterpret_cast<int*>(scratch);
+    __threadfence();
+    named_bar_sync(1, 128);
+    if (etid == 0) *last = (atomicAdd(&o.tickets[blockIdx.x * gridDim.y + blockIdx.y], 1) == o.splits - 1);
+    named_bar_sync(1, 128);
+    if (*last) {
+      __threadfence();
+      const int tend = min(o.T, n0 + BN);
+      if (rin) {
+        for (int t = n0; t < tend; ++t) {
+          float* p = &o.zacc[(size_t)t * o.R + r];
+          o.z[(size_t)t * o.R + r] = __float2bfloat16_rn(__ldcg(p));
+          *p = 0.0f;
+        }
+      }
+      if (etid == 0) o.tickets[blockIdx.x * gridDim.y + blockIdx.y] = 0;
+    }
+  }
+};
+
+// -------------------------------------------------- dense fallback: h rows
+// Overflow tokens ([TwELL] hybrid routing): both accumulators hold g (col 0)
+// and u (col BN) for the gathered overflow rows.  h = keep ? bf16(a)·u : 0 is
+// written as a bf16 pair (hi + lo, hi = bf16(h), lo = bf16(h - hi)) so the
+// tensor-core down projection loses no more than 2^-16 relative of h.
+struct HParams {
+  const float* bias;
+  float tau;
+  int act, F;
+  const int* n_rows_dev;    // number of valid rows (overflow count)
+  int n_rows;               // used when n_rows_dev is null
+  const int* row_map;       // output row of gathered row o (or null: identity)
+  __nv_bfloat16* h_hi;      // [maxT][F]
+  __nv_bfloat16* h_lo;
+  int val_f32;              // stored value rounding: 0 bf16
+};
+
+__device__ __forceinline__ void store_h(const HParams& o, int row, int j, float h) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+  const size_t off = (size_t)row * o.F + j;
+  o.h_hi[off] = hi;
+  o.h_lo[off] = lo;
+}
+
+struct EpiFallbackH {
+  static constexpr int N_ACC = 2;
+  using Params = HParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int n_rows = o.n_rows_dev ? *o.n_rows_dev : o.n_rows;
+    const int j = m0 + etid;
+    const float b = o.bias ? o.bias[j] : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= n_rows) break;
+      float g[16], u[16];
+      tmem_ld16(tmem + c, g);
+      tmem_ld16(tmem + BN + c, u);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = n0 + c + i;
+        if (r < n_rows) {
+          const float a = act_fn(g[i] + b, o.act);
+          const bool keep = fabsf(a) > o.tau;
+          const float v = __bfloat162float(__float2bfloat16_rn(a));
+          store_h(o, o.row_map ? o.row_map[r] : r, j, keep ? v * u[i] : 0.0f);
+        }
+      }
+    }
+  }
+};
+
+// ------------------------------------------- tile path: h from TwELL values
+// Non-overflow tokens on the tile path: the accumulator holds u for a
+// 128-neuron tile; the kept values come from the token's TwELL record, which
+// is scattered into a shared [32 tokens][128 neurons] table, 32 tokens at a
+// time.  Overflow tokens are skipped (their rows come from the fallback).
+struct TwellHParams {
+  int T, F, n_tiles, C;
+  const int16_t* count;
+  const int16_t* idx;
+  const __nv_bfloat16* val;
+  const uint32_t* ovf;
+  uint32_t epoch;
+  __nv_bfloat16* h_hi;
+  __nv_bfloat16* h_lo;
+};
+
+struct EpiTwellH {
+  static constexpr int N_ACC = 1;
+  using Params = TwellHParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t* scratch) {
+    uint16_t* tab = reinterpret_cast<uint16_t*>(scratch);            // [32][128]
+    int* live = reinterpret_cast<int*>(scratch + 32 * 128 * 2);        // [32]
+    const int p = m0 >> 7, j = m0 + etid;
+    HParams hp;
+    hp.F = o.F;
+    hp.h_hi = o.h_hi;
+    hp.h_lo = o.h_lo;
+#pragma unroll 1
+    for (int c32 = 0; c32 < BN; c32 += 32) {
+      if (n0 + c32 >= o.T) break;
+      for (int e = etid; e < 32 * 128 / 2; e += 128) reinterpret_cast<uint32_t*>(tab)[e] = 0u;
+      if (etid < 32) {
+        const int t = n0 + c32 + etid;
+        live[etid] = (t < o.T && o.ovf[t] != o.epoch) ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      {
+        const int tl = etid >> 2, q = etid & 3;
+        const int t = n0 + c32 + tl;
+        if (live[tl]) {
+          const size_t rec = (size_t)t * o.n_tiles + p;
+          const int cnt = min((int)o.count[rec], o.C);
+          for (int s = q; s < cnt; s += 4) {
+            const int jj = o.idx[rec * o.C + s] - m0;
+            if (jj >= 0 && jj < 128)
+              tab[tl * 128 + jj] = reinterpret_cast<const uint16_t*>(o.val)[rec * o.C + s];
+          }
+        }
+      }
+      named_bar_sync(1, 128);
+#pragma unroll 1
+      for (int c = 0; c < 32; c += 16) {
+        if (c32 + c >= BN) break;
+        float u[16];
+        tmem_ld16(tmem + c32 + c, u);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int tl = c + i;
+          if (live[tl]) {
+            const float v = __uint_as_float((uint32_t)tab[tl * 128 + etid] << 16);
+            store_h(hp, n0 + c32 + tl, j, v * u[i]);
+          }
+        }
+      }
+      named_bar_sync(1, 128);
+    }
+  }
+};
+
+// -------------------------------------------------- down projection output
+// D^T tile: rows are output columns (m0 + etid), columns are h rows.  With a
+// split K the partial sums are added into out (zeroed by the router).
+struct OutParams {
+  float* out;          // [T][d]
+  int d;
+  const int* n_rows_dev;
+  int n_rows;
+  const int* row_map;  // out row of h row r (null: identity)
+  int atomic;
+};
+
+struct EpiDownOut {
+  static constexpr int N_ACC = 1;
+  using Params = OutParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int n_rows = o.n_rows_dev ? *o.n_rows_dev : o.n_rows;
+    const int col = m0 + etid;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= n_rows) break;
+      float y[16];
+      tmem_ld16(tmem + c, y);
+      if (col < o.d) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = n0 + c + i;
+          if (r < n_rows) {
+            const int row = o.row_map ? o.row_map[r] : r;
+            float* dst = &o.out[(size_t)row * o.d + col];
+            if (o.atomic)
+              atomicAdd(dst, y[i]);
+            else
+              *dst = y[i];
+          }
+        }
+      }
+    }
+  }
+};
+
+}  // namespace sffn

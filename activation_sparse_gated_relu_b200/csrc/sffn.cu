@@ -1,0 +1,852 @@
+// C ABI of the activation-sparse gated FFN forward (see include/sffn.h):
+// argument validation, workspace, TMA tensor maps and the launch sequence.
+//
+// Launch sequence of one bf16 forward (all on the caller's stream):
+//   gate    tensor-core tile kernel, epilogue = TwELL emission (threshold) or
+//           dense value + score (WINA, then the top-k kernel emits TwELL);
+//           low-rank gate = two tile kernels (z = bf16(x·A) split over K, then
+//           g = z·B with the TwELL epilogue)
+//   router  overflow list, per-block live masks, gathers, output zeroing
+//   ROWS    fused SIMT up x down over the kept rows (non-overflow tokens)
+//   TILES   tensor-core u per tile with h from TwELL (non-overflow tokens)
+//   dense   tensor-core recompute of g and u for overflow tokens -> h
+//   down    tensor-core y = h·W_down for the h rows (overflow rows on ROWS,
+//           all rows on TILES)
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/sffn.h"
+#include "epilogues.cuh"
+#include "simt.cuh"
+#include "tc_gemm.cuh"
+
+using namespace sffn;
+
+#define SFFN_VERSION_STRING "sffn 0.1.0 (sm_100a)"
+
+namespace {
+
+constexpr int kNumSMsFallback = 148;
+constexpr int kMaxMarks = 12;
+enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
+                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_COUNT };
+const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
+                                          "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
+                                          "fallback_f32"};
+constexpr int kMaxTokensLimit = 16384;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][inner] matrix, box = 64 x box_rows,
+// 128-byte swizzle (the K-major operand layout of the tile kernel).
+bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int pick_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
+int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+template <int BN, class Epi>
+cudaError_t launch_tc_bn(dim3 grid, cudaStream_t st, const CUtensorMap& a0, const CUtensorMap& b0,
+                         const CUtensorMap& a1, const CUtensorMap& b1, const TcArgs& args,
+                         const typename Epi::Params& ep) {
+  k_tc_gemm<BN, Epi><<<grid, TC_THREADS, TcCfg<BN>::SMEM, st>>>(a0, b0, a1, b1, args, ep);
+  return cudaGetLastError();
+}
+
+template <class Epi>
+cudaError_t launch_tc(int BN, dim3 grid, cudaStream_t st, const CUtensorMap& a0, const CUtensorMap& b0,
+                      const CUtensorMap& a1, const CUtensorMap& b1, const TcArgs& args,
+                      const typename Epi::Params& ep) {
+  switch (BN) {
+    case 16: return launch_tc_bn<16, Epi>(grid, st, a0, b0, a1, b1, args, ep);
+    case 32: return launch_tc_bn<32, Epi>(grid, st, a0, b0, a1, b1, args, ep);
+    case 64: return launch_tc_bn<64, Epi>(grid, st, a0, b0, a1, b1, args, ep);
+    case 128: return launch_tc_bn<128, Epi>(grid, st, a0, b0, a1, b1, args, ep);
+    default: return launch_tc_bn<256, Epi>(grid, st, a0, b0, a1, b1, args, ep);
+  }
+}
+
+template <class Epi>
+cudaError_t set_tc_attrs() {
+  cudaError_t e = cudaSuccess;
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<16, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<16>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<32, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<32>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<64, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<128, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<128>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<256, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<256>::SMEM);
+  return e;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct sffn_handle {
+  sffn_desc desc;
+  int dev = 0, n_sm = kNumSMsFallback;
+  int d = 0, F = 0, P = 0, R = 0, C = 0, maxT = 0, esize = 2;
+  bool f32 = false, wina = false, lowrank = false;
+  uint32_t epoch = 0;
+  // workspace
+  int16_t* count = nullptr;
+  int16_t* idx = nullptr;
+  void* val = nullptr;
+  uint32_t* ovf = nullptr;
+  uint32_t* umask = nullptr;
+  int* ovf_list = nullptr;
+  int* ovf_count = nullptr;
+  uint8_t* blk_live = nullptr;
+  __nv_bfloat16* xo = nullptr;
+  __nv_bfloat16* h_hi = nullptr;
+  __nv_bfloat16* h_lo = nullptr;
+  float* scores = nullptr;
+  void* vdense = nullptr;
+  float* norms = nullptr;
+  __nv_bfloat16* z = nullptr;
+  __nv_bfloat16* zo = nullptr;
+  float* zacc = nullptr;
+  int* tickets = nullptr;
+  __nv_bfloat16* At = nullptr;
+  __nv_bfloat16* Bt = nullptr;
+  __nv_bfloat16* WdT = nullptr;
+  float* gdebug = nullptr;
+  uint32_t* status = nullptr;
+  void* xstage = nullptr;
+  float* ostage = nullptr;
+  // A-operand tensor maps (box 64 x 128)
+  CUtensorMap tmWgate, tmWup, tmWdT, tmAt, tmBt;
+  int last_T = 0, last_path = 0, last_launches = 0;
+  int rows_nslot = 0, rows_lcap = 0, rows_smem = 0;
+  // per-kernel timing (sffn_timing_begin/end)
+  bool tm_on = false;
+  int tm_max = 0, tm_n = 0, tm_cur = -1;
+  std::vector<cudaEvent_t> tm_ev;   // [tm_max][kMaxMarks + 1]
+  std::vector<int> tm_lab;          // [tm_max][kMaxMarks]
+  std::vector<int> tm_nk;           // [tm_max]
+};
+
+namespace {
+
+void timing_free(sffn_handle* h);
+
+void free_handle(sffn_handle* h) {
+  if (!h) return;
+  timing_free(h);
+  void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->umask, h->ovf_list, h->ovf_count, h->blk_live,
+                  h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zacc,
+                  h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  delete h;
+}
+
+template <typename T>
+bool dalloc(T** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  void* q = nullptr;
+  if (cudaMalloc(&q, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  *p = static_cast<T*>(q);
+  return true;
+}
+
+void tmark(sffn_handle* h, cudaStream_t st, int label) {
+  if (!h->tm_on || h->tm_cur < 0) return;
+  const int f = h->tm_cur, i = h->tm_nk[f];
+  if (i >= kMaxMarks) return;
+  cudaEventRecord(h->tm_ev[(size_t)f * (kMaxMarks + 1) + i], st);
+  h->tm_lab[(size_t)f * kMaxMarks + i] = label;
+  h->tm_nk[f] = i + 1;
+}
+
+void tmark_begin(sffn_handle* h) {
+  h->tm_cur = -1;
+  if (h->tm_on && h->tm_n < h->tm_max) {
+    h->tm_cur = h->tm_n++;
+    h->tm_nk[h->tm_cur] = 0;
+  }
+}
+
+void tmark_end(sffn_handle* h, cudaStream_t st) {
+  if (!h->tm_on || h->tm_cur < 0) return;
+  const int f = h->tm_cur;
+  cudaEventRecord(h->tm_ev[(size_t)f * (kMaxMarks + 1) + h->tm_nk[f]], st);
+  h->tm_cur = -1;
+}
+
+void timing_free(sffn_handle* h) {
+  for (cudaEvent_t e : h->tm_ev)
+    if (e) cudaEventDestroy(e);
+  h->tm_ev.clear();
+  h->tm_lab.clear();
+  h->tm_nk.clear();
+  h->tm_on = false;
+  h->tm_max = h->tm_n = 0;
+  h->tm_cur = -1;
+}
+
+sffn_status validate(const sffn_desc* d) {
+  if (!d) return SFFN_ERR_INVALID_ARG;
+  if (d->d_model <= 0 || d->d_ff <= 0 || d->max_tokens <= 0 || d->rank < 0) return SFFN_ERR_INVALID_ARG;
+  if (d->dtype != SFFN_BF16 && d->dtype != SFFN_FP32) return SFFN_ERR_INVALID_ARG;
+  if (d->mode != SFFN_MODE_RELU_THRESHOLD && d->mode != SFFN_MODE_WINA_TOPK) return SFFN_ERR_INVALID_ARG;
+  if (d->act != SFFN_ACT_RELU && d->act != SFFN_ACT_SILU) return SFFN_ERR_INVALID_ARG;
+  if (d->path < SFFN_PATH_AUTO || d->path > SFFN_PATH_TILES) return SFFN_ERR_INVALID_ARG;
+  const int C = d->tile_capacity;
+  if (C != 8 && C != 16 && C != 32 && C != 64 && C != 128) return SFFN_ERR_INVALID_ARG;
+  if (d->mode == SFFN_MODE_RELU_THRESHOLD && (!(d->threshold >= 0.0f) || !std::isfinite(d->threshold)))
+    return SFFN_ERR_INVALID_ARG;
+  if (d->mode == SFFN_MODE_WINA_TOPK && (d->k < 0 || d->k > d->d_ff)) return SFFN_ERR_INVALID_ARG;
+  if (!d->W_up || !d->W_down) return SFFN_ERR_INVALID_ARG;
+  if (d->rank == 0 && (!d->W_gate || d->A || d->B)) return SFFN_ERR_INVALID_ARG;
+  if (d->rank > 0 && (d->W_gate || !d->A || !d->B)) return SFFN_ERR_INVALID_ARG;
+  const void* ptrs[] = {d->W_gate, d->A, d->B, d->W_up, d->W_down, d->gate_bias};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return SFFN_ERR_INVALID_ARG;
+  if (d->d_model % 8 != 0) return SFFN_ERR_UNSUPPORTED;
+  if (d->d_ff % 128 != 0 || d->d_ff > 32767) return SFFN_ERR_UNSUPPORTED;
+  if (d->max_tokens > kMaxTokensLimit) return SFFN_ERR_UNSUPPORTED;
+  if (d->d_model > 4096) return SFFN_ERR_UNSUPPORTED;
+  if (d->mode == SFFN_MODE_WINA_TOPK && C != 128) return SFFN_ERR_UNSUPPORTED;
+  if (d->rank > 0 && (d->dtype != SFFN_BF16 || d->rank % 64 != 0 || d->rank > 4096)) return SFFN_ERR_UNSUPPORTED;
+  if (d->dtype == SFFN_FP32 && d->d_ff > 8192) return SFFN_ERR_UNSUPPORTED;
+  if ((d->flags & SFFN_FLAG_DEBUG_GATE) && d->rank > 0) return SFFN_ERR_UNSUPPORTED;
+  return SFFN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sffn_version(void) { return SFFN_VERSION_STRING; }
+
+const char* sffn_status_string(sffn_status s) {
+  switch (s) {
+    case SFFN_OK: return "ok";
+    case SFFN_ERR_INVALID_ARG: return "invalid argument";
+    case SFFN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SFFN_ERR_ALLOC: return "device allocation failed";
+    case SFFN_ERR_CUDA: return "CUDA error";
+    case SFFN_ERR_TIMEOUT: return "device-side wait timed out";
+    case SFFN_ERR_DEVICE: return "device-side range check failed";
+    case SFFN_ERR_NO_DEVICE: return "no usable sm_100 device";
+  }
+  return "unknown status";
+}
+
+sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** out) {
+  if (!out) return SFFN_ERR_INVALID_ARG;
+  *out = nullptr;
+  sffn_status vs = validate(desc);
+  if (vs != SFFN_OK) return vs;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_NO_DEVICE;
+  }
+  int major = 0, nsm = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10) return SFFN_ERR_NO_DEVICE;
+  if (!get_encode()) return SFFN_ERR_CUDA;
+
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  sffn_handle* h = new (std::nothrow) sffn_handle();
+  if (!h) return SFFN_ERR_ALLOC;
+  h->desc = *desc;
+  h->dev = dev;
+  h->n_sm = nsm > 0 ? nsm : kNumSMsFallback;
+  h->d = desc->d_model;
+  h->F = desc->d_ff;
+  h->P = desc->d_ff / 128;
+  h->R = desc->rank;
+  h->C = desc->tile_capacity;
+  h->maxT = desc->max_tokens;
+  h->f32 = desc->dtype == SFFN_FP32;
+  h->esize = h->f32 ? 4 : 2;
+  h->wina = desc->mode == SFFN_MODE_WINA_TOPK;
+  h->lowrank = desc->rank > 0;
+  const size_t T = (size_t)h->maxT, d = (size_t)h->d, F = (size_t)h->F, P = (size_t)h->P, C = (size_t)h->C;
+  const size_t nblk = (T + 7) / 8;
+  bool ok = true;
+  ok = ok && dalloc(&h->count, T * P * 2);
+  ok = ok && dalloc(&h->idx, T * P * C * 2);
+  ok = ok && dalloc(&h->val, T * P * C * h->esize);
+  ok = ok && dalloc(&h->ovf, T * 4);
+  ok = ok && dalloc(&h->umask, nblk * P * 16);
+  ok = ok && dalloc(&h->ovf_list, T * 4);
+  ok = ok && dalloc(&h->ovf_count, 16);
+  ok = ok && dalloc(&h->blk_live, nblk);
+  ok = ok && dalloc(&h->status, 16);
+  ok = ok && dalloc(&h->xstage, T * d * h->esize);
+  ok = ok && dalloc(&h->ostage, T * d * 4);
+  if (!h->f32) {
+    ok = ok && dalloc(&h->xo, T * d * 2);
+    ok = ok && dalloc(&h->h_hi, T * F * 2);
+    ok = ok && dalloc(&h->h_lo, T * F * 2);
+    ok = ok && dalloc(&h->WdT, d * F * 2);
+  }
+  if (h->wina) {
+    ok = ok && dalloc(&h->scores, T * F * 4);
+    ok = ok && dalloc(&h->vdense, T * F * h->esize);
+    ok = ok && dalloc(&h->norms, F * 4);
+  }
+  if (h->lowrank) {
+    const size_t R = (size_t)h->R;
+    ok = ok && dalloc(&h->z, T * R * 2);
+    ok = ok && dalloc(&h->zo, T * R * 2);
+    ok = ok && dalloc(&h->zacc, T * R * 4);
+    ok = ok && dalloc(&h->tickets, (R / 128 + 1) * (T / 16 + 2) * 4);
+    ok = ok && dalloc(&h->At, R * d * 2);
+    ok = ok && dalloc(&h->Bt, F * R * 2);
+  }
+  if (desc->flags & SFFN_FLAG_DEBUG_GATE) ok = ok && dalloc(&h->gdebug, T * F * 4);
+  if (!ok) {
+    free_handle(h);
+    return SFFN_ERR_ALLOC;
+  }
+  cudaError_t e = cudaSuccess;
+  e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
+  e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
+  e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
+  if (h->lowrank) {
+    e = e ? e : cudaMemsetAsync(h->zacc, 0, T * (size_t)h->R * 4, st);
+    e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * (T / 16 + 2) * 4, st);
+  }
+  // create-time derived data
+  const dim3 tb(32, 8);
+  if (!e && !h->f32) {
+    k_transpose_bf16<<<dim3(cdiv(d, 32), cdiv(F, 32)), tb, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(desc->W_down), h->WdT, (int)F, (int)d);
+    e = cudaGetLastError();
+  }
+  if (!e && h->lowrank) {
+    const int R = h->R;
+    k_transpose_bf16<<<dim3(cdiv(R, 32), cdiv(d, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->A),
+                                                                    h->At, (int)d, R);
+    k_transpose_bf16<<<dim3(cdiv(F, 32), cdiv(R, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->B),
+                                                                    h->Bt, R, (int)F);
+    e = cudaGetLastError();
+  }
+  if (!e && h->wina) {
+    if (h->f32)
+      k_row_norms<float><<<cdiv(F, 8), 256, 0, st>>>(static_cast<const float*>(desc->W_down), (int)F, (int)d,
+                                                      h->norms);
+    else
+      k_row_norms<__nv_bfloat16><<<cdiv(F, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->W_down),
+                                                             (int)F, (int)d, h->norms);
+    e = cudaGetLastError();
+  }
+  // kernel attributes and A-operand tensor maps
+  if (!e && !h->f32) {
+    e = e ? e : set_tc_attrs<EpiGateTwell>();
+    e = e ? e : set_tc_attrs<EpiWina>();
+    e = e ? e : set_tc_attrs<EpiLowRankZ>();
+    e = e ? e : set_tc_attrs<EpiFallbackH>();
+    e = e ? e : set_tc_attrs<EpiTwellH>();
+    e = e ? e : set_tc_attrs<EpiDownOut>();
+    bool mok = true;
+    if (!h->lowrank) mok = mok && make_map(&h->tmWgate, desc->W_gate, h->d, h->F, 128);
+    mok = mok && make_map(&h->tmWup, desc->W_up, h->d, h->F, 128);
+    mok = mok && make_map(&h->tmWdT, h->WdT, h->F, h->d, 128);
+    if (h->lowrank) {
+      mok = mok && make_map(&h->tmAt, h->At, h->d, h->R, 128);
+      mok = mok && make_map(&h->tmBt, h->Bt, h->R, h->F, 128);
+    }
+    if (!mok) {
+      free_handle(h);
+      return SFFN_ERR_CUDA;
+    }
+    // fused up x down: ring slots and list capacity from the shared memory budget
+    int max_smem = 0;
+    cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    int nslot = 16, lcap = 1024;
+    while (nslot > 2 && RowsSmem::make(h->d, h->P, nslot, 256).total > max_smem) --nslot;
+    while (lcap > 64 && RowsSmem::make(h->d, h->P, nslot, lcap).total > max_smem) lcap -= 64;
+    h->rows_nslot = nslot;
+    h->rows_lcap = lcap;
+    h->rows_smem = RowsSmem::make(h->d, h->P, nslot, lcap).total;
+    e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
+  }
+  if (!e && h->wina) {
+    const int tk_smem = (int)(F * 4 + 32 * 256 * 4 + P * 4);
+    e = cudaFuncSetAttribute(k_wina_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, tk_smem);
+  }
+  if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(T * 4));
+  if (!e && h->f32) {
+    e = cudaFuncSetAttribute(k_rows_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)((d + 2 * P * C) * 4));
+    e = e ? e : cudaFuncSetAttribute(k_fallback_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)((d + F) * 4));
+  }
+  if (!e) e = cudaStreamSynchronize(st);
+  if (e) {
+    cudaGetLastError();
+    free_handle(h);
+    return SFFN_ERR_CUDA;
+  }
+  *out = h;
+  return SFFN_OK;
+}
+
+sffn_status sffn_destroy(sffn_handle* h) {
+  if (!h) return SFFN_OK;
+  cudaDeviceSynchronize();
+  free_handle(h);
+  return SFFN_OK;
+}
+
+static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out, cudaStream_t st) {
+  const sffn_desc& D = h->desc;
+  const int d = h->d, F = h->F, P = h->P;
+  int launches = 0;
+  const uint32_t epoch = h->epoch;
+  const int BN = pick_bn(T);
+  const int ntile_tok = cdiv(T, BN);
+  CUtensorMap mx, mxo, mhi, mlo, mz, mzo;
+  bool mok = make_map(&mx, x, d, T, BN) && make_map(&mxo, h->xo, d, h->maxT, BN) &&
+             make_map(&mhi, h->h_hi, F, h->maxT, BN) && make_map(&mlo, h->h_lo, F, h->maxT, BN);
+  if (h->lowrank)
+    mok = mok && make_map(&mz, h->z, h->R, h->maxT, BN) && make_map(&mzo, h->zo, h->R, h->maxT, BN);
+  if (!mok) return SFFN_ERR_CUDA;
+
+  int path = D.path;
+  if (path == SFFN_PATH_AUTO) path = (T <= 8 || T > 256) ? SFFN_PATH_ROWS : SFFN_PATH_TILES;
+  if (h->wina) path = SFFN_PATH_TILES;  // the top-k kernel writes no union masks
+  const bool rows = path == SFFN_PATH_ROWS;
+  const int nblk = cdiv(T, 8);
+  const int rows_split = rows ? std::max(1, h->n_sm / nblk) : 1;
+  // down projection split over d_ff so that its grid covers the SMs
+  const int m_tiles_down = cdiv(d, 128);
+  const int est_rows_tiles = rows ? 1 : ntile_tok;
+  const int kb_down = cdiv(F, 64);
+  const int sk_down = std::max(1, std::min(kb_down / 4, cdiv(h->n_sm, m_tiles_down * est_rows_tiles)));
+
+  cudaError_t e = cudaSuccess;
+  TwellParams tw;
+  tw.bias = D.gate_bias;
+  tw.tau = h->wina ? 0.f : D.threshold;
+  tw.act = D.act;
+  tw.T = T;
+  tw.F = F;
+  tw.n_tiles = P;
+  tw.C = h->C;
+  tw.count = h->count;
+  tw.idx = h->idx;
+  tw.val = h->val;
+  tw.val_f32 = 0;
+  tw.ovf = h->ovf;
+  tw.epoch = epoch;
+  tw.umask = rows ? h->umask : nullptr;
+  tw.gdebug = h->gdebug;
+
+  // ---------------------------------------------------------------- gate
+  const CUtensorMap* gateA = &h->tmWgate;
+  const CUtensorMap* gateB = &mx;
+  int gate_kb = cdiv(d, 64);
+  if (h->lowrank) {
+    // z = bf16(x·A): rows are rank coordinates, split over d
+    const int mt = cdiv(h->R, 128);
+    const int sk = std::max(1, std::min(cdiv(d, 64), cdiv(h->n_sm, mt * ntile_tok)));
+    TcArgs za{};
+    za.n_phase = 1;
+    za.kb_total[0] = cdiv(d, 64);
+    za.n_rows = T;
+    za.status = h->status;
+    ZParams zp{T, h->R, sk, h->zacc, h->z, h->tickets};
+    tmark(h, st, L_GATE_Z);
+    e = launch_tc<EpiLowRankZ>(BN, dim3(mt, ntile_tok, sk), st, h->tmAt, mx, h->tmAt, mx, za, zp);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+    gateA = &h->tmBt;
+    gateB = &mz;
+    gate_kb = cdiv(h->R, 64);
+  }
+  TcArgs ga{};
+  ga.n_phase = 1;
+  ga.kb_total[0] = gate_kb;
+  ga.n_rows = T;
+  ga.status = h->status;
+  if (h->wina) {
+    WinaParams wp{D.gate_bias, D.act, T, F, h->norms, h->vdense, 0, h->scores};
+    tmark(h, st, L_GATE);
+    e = launch_tc<EpiWina>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, wp);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+    TopkArgs ta{h->scores, h->vdense, 0, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
+    tmark(h, st, L_WINA_TOPK);
+    k_wina_topk<<<T, 1024, (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st>>>(ta);
+    ++launches;
+    if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  } else {
+    tmark(h, st, L_GATE);
+    e = launch_tc<EpiGateTwell>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, tw);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+  }
+
+  // -------------------------------------------------------------- router
+  RouterArgs ra{};
+  ra.T = T;
+  ra.ovf = h->ovf;
+  ra.epoch = epoch;
+  ra.ovf_list = h->ovf_list;
+  ra.ovf_count = h->ovf_count;
+  ra.blk_live = h->blk_live;
+  ra.x = static_cast<const uint4*>(x);
+  ra.xo = reinterpret_cast<uint4*>(h->xo);
+  ra.d_vec = d / 8;
+  ra.z = h->lowrank ? reinterpret_cast<const uint4*>(h->z) : nullptr;
+  ra.zo = reinterpret_cast<uint4*>(h->zo);
+  ra.r_vec = h->R / 8;
+  ra.out = reinterpret_cast<float4*>(out);
+  ra.d4 = d / 4;
+  ra.zero_mode = (!rows || rows_split > 1) ? 1 : (sk_down > 1 ? 2 : 0);
+  const int router_ctas = std::max(1, std::min(h->n_sm, cdiv((long long)T * d / 4, 4096)));
+  tmark(h, st, L_ROUTER);
+  k_router<<<router_ctas, 1024, (size_t)T * 4, st>>>(ra);
+  ++launches;
+  if (cudaGetLastError()) return SFFN_ERR_CUDA;
+
+  // ------------------------------------------ non-overflow tokens
+  if (rows) {
+    RowsArgs rw{};
+    rw.x = static_cast<const __nv_bfloat16*>(x);
+    rw.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
+    rw.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
+    rw.count = h->count;
+    rw.idx = h->idx;
+    rw.val = static_cast<const __nv_bfloat16*>(h->val);
+    rw.umask = reinterpret_cast<const uint4*>(h->umask);
+    rw.blk_live = h->blk_live;
+    rw.out = out;
+    rw.T = T;
+    rw.d = d;
+    rw.F = F;
+    rw.n_tiles = P;
+    rw.C = h->C;
+    rw.atomic = rows_split > 1 ? 1 : 0;
+    rw.nslot = h->rows_nslot;
+    rw.lcap = h->rows_lcap;
+    rw.status = h->status;
+    tmark(h, st, L_UPDOWN_ROWS);
+    k_rows<<<dim3(rows_split, nblk), RW_THREADS, h->rows_smem, st>>>(rw);
+    ++launches;
+    if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  } else {
+    TcArgs ua{};
+    ua.n_phase = 1;
+    ua.kb_total[0] = cdiv(d, 64);
+    ua.n_rows = T;
+    ua.status = h->status;
+    TwellHParams hp{T, F, P, h->C, h->count, h->idx, static_cast<const __nv_bfloat16*>(h->val), h->ovf, epoch,
+                    h->h_hi, h->h_lo};
+    tmark(h, st, L_TILE_H);
+    e = launch_tc<EpiTwellH>(BN, dim3(P, ntile_tok, 1), st, h->tmWup, mx, h->tmWup, mx, ua, hp);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+  }
+
+  // ------------------------------------- dense channel for overflow tokens
+  if (!h->wina) {
+    TcArgs fa{};
+    fa.n_phase = 2;
+    fa.kb_total[0] = h->lowrank ? cdiv(h->R, 64) : cdiv(d, 64);
+    fa.kb_total[1] = cdiv(d, 64);
+    fa.n_rows = T;
+    fa.n_rows_dev = h->ovf_count;
+    fa.status = h->status;
+    HParams hp{};
+    hp.bias = D.gate_bias;
+    hp.tau = D.threshold;
+    hp.act = D.act;
+    hp.F = F;
+    hp.n_rows_dev = h->ovf_count;
+    hp.n_rows = T;
+    hp.row_map = rows ? nullptr : h->ovf_list;
+    hp.h_hi = h->h_hi;
+    hp.h_lo = h->h_lo;
+    const CUtensorMap& a0 = h->lowrank ? h->tmBt : h->tmWgate;
+    const CUtensorMap& b0 = h->lowrank ? mzo : mxo;
+    tmark(h, st, L_FALLBACK_H);
+    e = launch_tc<EpiFallbackH>(BN, dim3(P, ntile_tok, 1), st, a0, b0, h->tmWup, mxo, fa, hp);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+  }
+
+  // ----------------------------------------------------- down projection
+  {
+    TcArgs da{};
+    da.n_phase = 2;
+    da.acc_same = 1;
+    da.kb_total[0] = kb_down;
+    da.kb_total[1] = kb_down;
+    da.n_rows = T;
+    da.n_rows_dev = rows ? h->ovf_count : nullptr;
+    da.status = h->status;
+    OutParams op{};
+    op.out = out;
+    op.d = d;
+    op.n_rows_dev = rows ? h->ovf_count : nullptr;
+    op.n_rows = T;
+    op.row_map = rows ? h->ovf_list : nullptr;
+    op.atomic = sk_down > 1 ? 1 : 0;
+    tmark(h, st, L_DOWN);
+    e = launch_tc<EpiDownOut>(BN, dim3(m_tiles_down, ntile_tok, sk_down), st, h->tmWdT, mhi, h->tmWdT, mlo, da,
+                              op);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+  }
+  h->last_path = path;
+  h->last_launches = launches;
+  return SFFN_OK;
+}
+
+static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out, cudaStream_t st) {
+  const sffn_desc& D = h->desc;
+  const int d = h->d, F = h->F, P = h->P;
+  const uint32_t epoch = h->epoch;
+  int launches = 0;
+  GateF32Args ga{};
+  ga.x = static_cast<const float*>(x);
+  ga.W_gate = static_cast<const float*>(D.W_gate);
+  ga.d = d;
+  ga.wina = h->wina ? 1 : 0;
+  ga.tw.bias = D.gate_bias;
+  ga.tw.tau = D.threshold;
+  ga.tw.act = D.act;
+  ga.tw.T = T;
+  ga.tw.F = F;
+  ga.tw.n_tiles = P;
+  ga.tw.C = h->C;
+  ga.tw.count = h->count;
+  ga.tw.idx = h->idx;
+  ga.tw.val = h->val;
+  ga.tw.val_f32 = 1;
+  ga.tw.ovf = h->ovf;
+  ga.tw.epoch = epoch;
+  ga.tw.umask = nullptr;
+  ga.tw.gdebug = h->gdebug;
+  ga.wp = WinaParams{D.gate_bias, D.act, T, F, h->norms, h->vdense, 1, h->scores};
+  tmark(h, st, L_GATE_F32);
+  k_gate_f32<<<dim3(P, cdiv(T, 16)), 128, 0, st>>>(ga);
+  ++launches;
+  if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  if (h->wina) {
+    TopkArgs ta{h->scores, h->vdense, 1, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
+    tmark(h, st, L_WINA_TOPK);
+    k_wina_topk<<<T, 1024, (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st>>>(ta);
+    ++launches;
+    if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  }
+  RouterArgs ra{};
+  ra.T = T;
+  ra.ovf = h->ovf;
+  ra.epoch = epoch;
+  ra.ovf_list = h->ovf_list;
+  ra.ovf_count = h->ovf_count;
+  ra.blk_live = h->blk_live;
+  ra.zero_mode = 0;
+  tmark(h, st, L_ROUTER);
+  k_router<<<1, 1024, (size_t)T * 4, st>>>(ra);
+  ++launches;
+  RowsF32Args rf{static_cast<const float*>(x), static_cast<const float*>(D.W_up), static_cast<const float*>(D.W_down),
+                 h->count, h->idx, static_cast<const float*>(h->val), h->ovf, epoch, out, T, d, P, h->C};
+  tmark(h, st, L_ROWS_F32);
+  k_rows_f32<<<T, 256, (size_t)(d + 2 * P * h->C) * 4, st>>>(rf);
+  ++launches;
+  if (!h->wina) {
+    FallbackF32Args fa{static_cast<const float*>(x), static_cast<const float*>(D.W_gate),
+                       static_cast<const float*>(D.W_up), static_cast<const float*>(D.W_down), D.gate_bias,
+                       D.threshold, D.act, h->ovf_list, h->ovf_count, out, d, F};
+    tmark(h, st, L_FALLBACK_F32);
+    k_fallback_f32<<<T, 256, (size_t)(d + F) * 4, st>>>(fa);
+    ++launches;
+  }
+  if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  h->last_path = SFFN_PATH_ROWS;
+  h->last_launches = launches;
+  return SFFN_OK;
+}
+
+sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (T < 0 || T > h->maxT) return SFFN_ERR_INVALID_ARG;
+  if (T == 0) return SFFN_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  ++h->epoch;
+  if (h->epoch == 0) ++h->epoch;  // 0 marks "never overflowed"
+  h->last_T = T;
+  tmark_begin(h);
+  const sffn_status r = h->f32 ? forward_f32(h, x, T, out, st) : forward_bf16(h, x, T, out, st);
+  tmark_end(h, st);
+  return r;
+}
+
+sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards) {
+  if (!h || max_forwards <= 0 || max_forwards > 100000) return SFFN_ERR_INVALID_ARG;
+  timing_free(h);
+  const size_t nev = (size_t)max_forwards * (kMaxMarks + 1);
+  h->tm_ev.assign(nev, nullptr);
+  for (size_t i = 0; i < nev; ++i) {
+    if (cudaEventCreate(&h->tm_ev[i]) != cudaSuccess) {
+      cudaGetLastError();
+      timing_free(h);
+      return SFFN_ERR_CUDA;
+    }
+  }
+  h->tm_lab.assign((size_t)max_forwards * kMaxMarks, 0);
+  h->tm_nk.assign(max_forwards, 0);
+  h->tm_max = max_forwards;
+  h->tm_n = 0;
+  h->tm_on = true;
+  return SFFN_OK;
+}
+
+sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], float* total_ms, int* launches,
+                            int* n_kernels) {
+  if (!h || !h->tm_on) return SFFN_ERR_INVALID_ARG;
+  double acc[L_COUNT] = {0};
+  int cnt[L_COUNT] = {0};
+  sffn_status rs = SFFN_OK;
+  for (int f = 0; f < h->tm_n && rs == SFFN_OK; ++f) {
+    const int nk = h->tm_nk[f];
+    cudaEvent_t* ev = &h->tm_ev[(size_t)f * (kMaxMarks + 1)];
+    if (cudaEventSynchronize(ev[nk]) != cudaSuccess) {
+      rs = SFFN_ERR_CUDA;
+      break;
+    }
+    for (int i = 0; i < nk; ++i) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) {
+        rs = SFFN_ERR_CUDA;
+        break;
+      }
+      const int lab = h->tm_lab[(size_t)f * kMaxMarks + i];
+      acc[lab] += ms;
+      cnt[lab] += 1;
+    }
+  }
+  int n = 0;
+  for (int l = 0; l < L_COUNT; ++l) {
+    if (!cnt[l]) continue;
+    if (n < max_kernels) {
+      if (names) {
+        std::strncpy(names[n], kLabelNames[l], 31);
+        names[n][31] = 0;
+      }
+      if (total_ms) total_ms[n] = (float)acc[l];
+      if (launches) launches[n] = cnt[l];
+    }
+    ++n;
+  }
+  if (n_kernels) *n_kernels = n;
+  timing_free(h);
+  cudaGetLastError();
+  return rs;
+}
+
+sffn_status sffn_forward_host(sffn_handle* h, const void* x_host, int T, float* out_host, void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (T < 0 || T > h->maxT) return SFFN_ERR_INVALID_ARG;
+  if (T == 0) return SFFN_OK;
+  if (!x_host || !out_host) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const size_t xb = (size_t)T * h->d * h->esize, ob = (size_t)T * h->d * 4;
+  if (cudaMemcpyAsync(h->xstage, x_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess) return SFFN_ERR_CUDA;
+  sffn_status s = sffn_forward(h, h->xstage, T, h->ostage, cuda_stream);
+  if (s != SFFN_OK) return s;
+  if (cudaMemcpyAsync(out_host, h->ostage, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SFFN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SFFN_ERR_CUDA;
+  return SFFN_OK;
+}
+
+sffn_status sffn_read_status(sffn_handle* h, void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint32_t w = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SFFN_ERR_CUDA;
+  if (cudaMemcpy(&w, h->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFFN_ERR_CUDA;
+  if (w) cudaMemset(h->status, 0, 4);
+  if (w & DEV_ERR_TIMEOUT) return SFFN_ERR_TIMEOUT;
+  if (w & DEV_ERR_RANGE) return SFFN_ERR_DEVICE;
+  return SFFN_OK;
+}
+
+sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_t** idx, const void** val,
+                             const uint32_t** overflow, int* n_tiles, int* tile_capacity) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (count) *count = h->count;
+  if (idx) *idx = h->idx;
+  if (val) *val = h->val;
+  if (overflow) *overflow = h->ovf;
+  if (n_tiles) *n_tiles = h->P;
+  if (tile_capacity) *tile_capacity = h->C;
+  return SFFN_OK;
+}
+
+sffn_status sffn_debug_gate(sffn_handle* h, const float** g) {
+  if (!h || !g) return SFFN_ERR_INVALID_ARG;
+  if (!h->gdebug) return SFFN_ERR_UNSUPPORTED;
+  *g = h->gdebug;
+  return SFFN_OK;
+}
+
+sffn_status sffn_debug_norms(sffn_handle* h, const float** norms) {
+  if (!h || !norms) return SFFN_ERR_INVALID_ARG;
+  if (!h->norms) return SFFN_ERR_UNSUPPORTED;
+  *norms = h->norms;
+  return SFFN_OK;
+}
+
+sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st) {
+  if (!h || !st) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  int n = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SFFN_ERR_CUDA;
+  if (cudaMemcpy(&n, h->ovf_count, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFFN_ERR_CUDA;
+  st->n_overflow = n;
+  st->n_launches = h->last_launches;
+  st->path = h->last_path;
+  st->epoch = h->epoch;
+  return SFFN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,769 @@
+// SIMT kernels: the overflow router, the fused sparse up x down pass over
+// kept rows, the WINA per-token top-k, the fp32 path and create-time helpers.
+#pragma once
+
+#include "epilogues.cuh"
+#include "ptx.cuh"
+
+namespace sffn {
+
+// Exclusive scan of one int per thread over the whole block (<= 32 warps).
+// warp_tot: shared scratch of >= 33 ints.  Returns the exclusive prefix and
+// sets *total (all threads).  Contains __syncthreads.
+__device__ __forceinline__ int block_scan_excl(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? warp_tot[lane] : 0;
+    int ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+      if (lane >= o) ti += n;
+    }
+    if (lane < nw) warp_tot[lane] = ti - t;
+    if (lane == 31) warp_tot[32] = ti;
+  }
+  __syncthreads();
+  const int excl = warp_tot[warp] + inc - v;
+  *total = warp_tot[32];
+  __syncthreads();
+  return excl;
+}
+
+// ---------------------------------------------------------------- router
+// Hybrid routing ([TwELL] "Hybrid 應對非均勻稀疏"): a token whose TwELL record
+// overflowed in some tile goes whole to the dense channel.  Every CTA ranks
+// the overflow tokens itself (the flags are few), CTA 0 publishes the list,
+// the count and the per-8-token-block live masks, and all CTAs gather the
+// overflow rows of x (and z) and zero the output rows that are accumulated
+// with atomics afterwards.
+struct RouterArgs {
+  int T;
+  const uint32_t* ovf;
+  uint32_t epoch;
+  int* ovf_list;           // [maxT]
+  int* ovf_count;          // [1]
+  uint8_t* blk_live;       // [ceil(T/8)]: bit i = token 8b+i < T and not overflow
+  const uint4* x;          // [T][d] bf16 as 16-byte vectors, or null (no gather)
+  uint4* xo;               // [maxT][d]
+  int d_vec;               // d / 8
+  const uint4* z;          // [T][R] bf16, or null
+  uint4* zo;
+  int r_vec;               // R / 8
+  float4* out;             // [T][d] fp32
+  int d4;                  // d / 4
+  int zero_mode;           // 0: none, 1: all T rows, 2: overflow rows only
+};
+
+__global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
+  extern __shared__ int rs_list[];   // [T]
+  __shared__ int scan_tmp[33];
+  int base = 0;
+  for (int c = 0; c < a.T; c += blockDim.x) {
+    const int t = c + threadIdx.x;
+    const int f = (t < a.T && a.ovf[t] == a.epoch) ? 1 : 0;
+    int tot;
+    const int ex = block_scan_excl(f, scan_tmp, &tot);
+    if (f) rs_list[base + ex] = t;
+    base += tot;
+  }
+  __syncthreads();
+  const int n_o = base;
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < n_o; i += blockDim.x) a.ovf_list[i] = rs_list[i];
+    if (threadIdx.x == 0) *a.ovf_count = n_o;
+    const int nb = (a.T + 7) >> 3;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+      uint32_t m = 0;
+      for (int i = 0; i < 8; ++i) {
+        const int t = b * 8 + i;
+        if (t < a.T && a.ovf[t] != a.epoch) m |= 1u << i;
+      }
+      a.blk_live[b] = (uint8_t)m;
+    }
+  }
+  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long gstride = (long long)gridDim.x * blockDim.x;
+  if (a.x) {
+    const long long n = (long long)n_o * a.d_vec;
+    for (long long e = gtid; e < n; e += gstride) {
+      const int o = (int)(e / a.d_vec), v = (int)(e % a.d_vec);
+      a.xo[(size_t)o * a.d_vec + v] = a.x[(size_t)rs_list[o] * a.d_vec + v];
+    }
+  }
+  if (a.z) {
+    const long long n = (long long)n_o * a.r_vec;
+    for (long long e = gtid; e < n; e += gstride) {
+      const int o = (int)(e / a.r_vec), v = (int)(e % a.r_vec);
+      a.zo[(size_t)o * a.r_vec + v] = a.z[(size_t)rs_list[o] * a.r_vec + v];
+    }
+  }
+  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (a.zero_mode == 1) {
+    const long long n = (long long)a.T * a.d4;
+    for (long long e = gtid; e < n; e += gstride) a.out[e] = zero4;
+  } else if (a.zero_mode == 2) {
+    const long long n = (long long)n_o * a.d4;
+    for (long long e = gtid; e < n; e += gstride) {
+      const int o = (int)(e / a.d4), v = (int)(e % a.d4);
+      a.out[(size_t)rs_list[o] * a.d4 + v] = zero4;
+    }
+  }
+}
+
+// ------------------------------------------------- fused sparse up x down
+// [TwELL] "TwELL 減掉轉換開銷": one pass computes both projections for the kept
+// (token, neuron) pairs and never stores h.  One CTA works on a block of 8
+// tokens and a contiguous range of the block's union of kept neurons (ranked
+// tile by tile from the union masks the gate epilogue wrote), so that every
+// CTA streams the same number of W_up / W_down rows.  A producer thread
+// stages each kept neuron's W_up and W_down rows (contiguous, neuron-major)
+// into a shared-memory ring with 1-D bulk copies (thread 0 refills the slots
+// a batch has released right after the batch's closing barrier, so no
+// producer warp takes registers from the consumers); 16 warps compute
+// u_tj = <W_up[j], x_t> (4 warps per neuron, warp-shuffle reduction), form
+// h_tj = v_tj·u_tj in registers and add h_tj·W_down[j] into per-thread
+// accumulators that own 8 output columns for each of the 8 tokens.  The
+// partial y goes to out with plain stores (one CTA per block) or vector
+// atomics (a block split over several CTAs).
+constexpr int RW_CW = 16;                    // warps (all consume; thread 0 also issues copies)
+constexpr int RW_THREADS = RW_CW * 32;
+constexpr int RW_NB = 4;                     // neurons per consumer batch
+constexpr int RW_WPN = RW_CW / RW_NB;        // warps per neuron in the up phase
+
+struct RowsArgs {
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* W_up;
+  const __nv_bfloat16* W_down;
+  const int16_t* count;
+  const int16_t* idx;
+  const __nv_bfloat16* val;
+  const uint4* umask;        // [n_blk][n_tiles] 128-bit union masks
+  const uint8_t* blk_live;
+  float* out;
+  int T, d, F, n_tiles, C;
+  int atomic;
+  int nslot, lcap;
+  uint32_t* status;
+};
+
+struct RowsSmem {
+  // byte offsets inside the dynamic shared memory
+  int xs, ring, bars, tpre, nid, lmask, lval, nid2, lmask2, lval2, part, misc, total;
+  __host__ __device__ static RowsSmem make(int d, int n_tiles, int nslot, int lcap) {
+    RowsSmem s;
+    int o = 0;
+    s.xs = o;    o += 8 * d * 2;
+    s.ring = o;  o += nslot * 4 * d;
+    s.bars = o;  o += (nslot * 8 + 15) & ~15;
+    s.tpre = o;  o += ((n_tiles + 1) * 4 + 15) & ~15;
+    s.nid = o;   o += lcap * 4;
+    s.lmask = o; o += lcap * 4;
+    s.lval = o;  o += lcap * 16;
+    s.nid2 = o;  o += lcap * 4;
+    s.lmask2 = o; o += lcap * 4;
+    s.lval2 = o; o += lcap * 16;
+    s.part = o;  o += RW_NB * RW_WPN * 8 * 4;
+    s.misc = o;  o += 64 * 4;
+    s.total = o;
+    return s;
+  }
+};
+
+__device__ __forceinline__ uint32_t word4(const uint4& m, int q) {
+  return q == 0 ? m.x : q == 1 ? m.y : q == 2 ? m.z : m.w;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+}
+
+__global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const RowsSmem L = RowsSmem::make(a.d, a.n_tiles, a.nslot, a.lcap);
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sm + L.xs);
+  uint8_t* ring = sm + L.ring;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
+  int* tpre = reinterpret_cast<int*>(sm + L.tpre);
+  int* nid = reinterpret_cast<int*>(sm + L.nid);
+  uint32_t* lmask = reinterpret_cast<uint32_t*>(sm + L.lmask);
+  uint4* lval = reinterpret_cast<uint4*>(sm + L.lval);
+  int* nid2 = reinterpret_cast<int*>(sm + L.nid2);
+  uint32_t* lmask2 = reinterpret_cast<uint32_t*>(sm + L.lmask2);
+  uint4* lval2 = reinterpret_cast<uint4*>(sm + L.lval2);
+  float* part = reinterpret_cast<float*>(sm + L.part);
+  int* misc = reinterpret_cast<int*>(sm + L.misc);
+  volatile int* abort_flag = misc + 40;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int P = a.n_tiles, b = blockIdx.y, S = gridDim.x, s = blockIdx.x;
+  const int tb0 = b * 8;
+  const uint32_t live = a.blk_live[b];
+  const int d = a.d, nv = d >> 3;
+  const uint32_t row_bytes = (uint32_t)d * 2u;
+  const uint4* um = a.umask + (size_t)b * P;
+
+  // 1. union counts per tile -> exclusive prefix tpre[0..P]
+  if (warp == 0) {
+    int run = 0;
+    for (int p0 = 0; p0 < P; p0 += 32) {
+      const int p = p0 + lane;
+      int c = 0;
+      if (p < P) {
+        const uint4 m = um[p];
+        c = __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
+      }
+      int inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      if (p < P) tpre[p] = run + inc - c;
+      run += __shfl_sync(0xFFFFFFFFu, inc, 31);
+    }
+    if (lane == 0) tpre[P] = run;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < a.nslot; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // 2. the block's x rows (zero beyond T)
+  for (int e = tid; e < 8 * nv; e += blockDim.x) {
+    const int row = e / nv, v = e - row * nv;
+    const int t = tb0 + row;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (t < a.T) val = reinterpret_cast<const uint4*>(a.x + (size_t)t * d)[v];
+    reinterpret_cast<uint4*>(xs + (size_t)row * d)[v] = val;
+  }
+  __syncthreads();
+  const int U = tpre[P];
+  const int r0 = (int)((long long)U * s / S), r1 = (int)((long long)U * (s + 1) / S);
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+
+  int gi = 0;  // running ring index (uniform)
+  for (int c0 = r0; c0 < r1; c0 += a.lcap) {
+    const int c1 = min(r1, c0 + a.lcap), Lc = c1 - c0;
+    // a. neuron ids of ranks [c0, c1)
+    for (int p = tid; p < P; p += blockDim.x) {
+      const int lo = tpre[p], hi = tpre[p + 1];
+      if (hi <= c0 || lo >= c1) continue;
+      const uint4 m4 = um[p];
+      int rank = lo;
+      for (int q = 0; q < 4; ++q) {
+        uint32_t m = word4(m4, q);
+        while (m) {
+          const int bit = __ffs(m) - 1;
+          m &= m - 1;
+          if (rank >= c0 && rank < c1) nid[rank - c0] = p * 128 + q * 32 + bit;
+          ++rank;
+        }
+      }
+    }
+    for (int e = tid; e < Lc; e += blockDim.x) {
+      lmask[e] = 0u;
+      lval[e] = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    // b. scatter the TwELL values of the block's live tokens
+    for (int e = tid; e < 8 * P; e += blockDim.x) {
+      const int i = e & 7, p = e >> 3;
+      if (!((live >> i) & 1u)) continue;
+      const int lo = tpre[p], hi = tpre[p + 1];
+      if (hi <= c0 || lo >= c1) continue;
+      const size_t rec = (size_t)(tb0 + i) * P + p;
+      const int cnt = min((int)a.count[rec], a.C);
+      const uint4 m4 = um[p];
+      for (int sl = 0; sl < cnt; ++sl) {
+        const int bit = (int)a.idx[rec * a.C + sl] - p * 128;
+        if (bit < 0 || bit >= 128) {
+          atomicOr(a.status, DEV_ERR_RANGE);
+          continue;
+        }
+        const int q = bit >> 5;
+        int below = __popc(word4(m4, q) & ((1u << (bit & 31)) - 1u));
+        if (q > 0) below += __popc(m4.x);
+        if (q > 1) below += __popc(m4.y);
+        if (q > 2) below += __popc(m4.z);
+        const int rank = lo + below;
+        if (rank >= c0 && rank < c1) {
+          reinterpret_cast<uint16_t*>(&lval[rank - c0])[i] =
+              reinterpret_cast<const uint16_t*>(a.val)[rec * a.C + sl];
+          atomicOr(&lmask[rank - c0], 1u << i);
+        }
+      }
+    }
+    __syncthreads();
+    // c. drop neurons that only overflow tokens kept
+    int L2;
+    {
+      const int per = (Lc + blockDim.x - 1) / blockDim.x;
+      const int e0 = min(Lc, tid * per), e1 = min(Lc, e0 + per);
+      int cnt = 0;
+      for (int e = e0; e < e1; ++e) cnt += lmask[e] ? 1 : 0;
+      int tot;
+      int o = block_scan_excl(cnt, misc, &tot);
+      for (int e = e0; e < e1; ++e) {
+        if (lmask[e]) {
+          nid2[o] = nid[e];
+          lmask2[o] = lmask[e];
+          lval2[o] = lval[e];
+          ++o;
+        }
+      }
+      L2 = tot;
+    }
+    __syncthreads();
+    // d. stream the rows through the ring
+    auto issue = [&](int i) {  // thread 0 only: entry i of this chunk -> its slot
+      const int gs = gi + i, slot = gs % a.nslot;
+      uint8_t* dst = ring + (size_t)slot * 4 * d;
+      const size_t row = (size_t)nid2[i] * d;
+      mbar_expect_tx(&full[slot], 2u * row_bytes);
+      bulk_g2s(dst, a.W_up + row, row_bytes, &full[slot]);
+      bulk_g2s(dst + row_bytes, a.W_down + row, row_bytes, &full[slot]);
+    };
+    if (tid == 0) {
+      const int pro = min(L2, a.nslot);
+      for (int i = 0; i < pro; ++i) issue(i);
+    }
+    for (int i0 = 0; i0 < L2; i0 += RW_NB) {
+      // up: 4 warps per neuron, each over a quarter of the row
+      {
+        const int n = i0 + warp / RW_WPN, q = warp % RW_WPN;
+        if (n < L2) {
+          const int gs = gi + n, slot = gs % a.nslot;
+          if (mbar_wait(&full[slot], (gs / a.nslot) & 1, abort_flag, a.status)) {
+            const uint32_t m = lmask2[n];
+            const uint4* wr = reinterpret_cast<const uint4*>(ring + (size_t)slot * 4 * d);
+            float u[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) u[t] = 0.f;
+            const int v0 = q * nv / RW_WPN, v1 = (q + 1) * nv / RW_WPN;
+            for (int v = v0 + lane; v < v1; v += 32) {
+              float w[8];
+              bf16x8_to_f32(wr[v], w);
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                if ((m >> t) & 1u) {
+                  float xv[8];
+                  bf16x8_to_f32(reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v], xv);
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) u[t] = fmaf(w[k], xv[k], u[t]);
+                }
+              }
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              if ((m >> t) & 1u) {
+                float r = u[t];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+                if (lane == 0) part[((n - i0) * RW_WPN + q) * 8 + t] = r;
+              }
+            }
+          }
+        }
+      }
+      __syncthreads();
+      // down: every thread owns 8 columns for the 8 tokens
+      const int nb = min(RW_NB, L2 - i0);
+      for (int nn = 0; nn < nb; ++nn) {
+        const int n = i0 + nn, gs = gi + n, slot = gs % a.nslot;
+        if (!mbar_wait(&full[slot], (gs / a.nslot) & 1, abort_flag, a.status)) break;
+        const uint32_t m = lmask2[n];
+        float h[8];
+        float vf[8];
+        bf16x8_to_f32(lval2[n], vf);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          float uu = 0.f;
+          if ((m >> t) & 1u) {
+#pragma unroll
+            for (int q = 0; q < RW_WPN; ++q) uu += part[(nn * RW_WPN + q) * 8 + t];
+          }
+          h[t] = vf[t] * uu;
+        }
+        if (tid < nv) {
+          const uint4* wr = reinterpret_cast<const uint4*>(ring + (size_t)slot * 4 * d + row_bytes);
+          float w[8];
+          bf16x8_to_f32(wr[tid], w);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if ((m >> t) & 1u) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) acc[t][k] = fmaf(h[t], w[k], acc[t][k]);
+            }
+          }
+        }
+      }
+      __syncthreads();
+      // the batch's slots are free: refill them with the entries nslot ahead
+      if (tid == 0 && !*abort_flag) {
+        for (int nn = 0; nn < nb; ++nn) {
+          const int i = i0 + nn + a.nslot;
+          if (i < L2) issue(i);
+        }
+      }
+    }
+    gi += L2;
+    __syncthreads();
+    if (*abort_flag) break;
+  }
+  // drain any copies still in flight (only after an abort)
+  if (tid == 0 && *abort_flag) {
+    for (int k = 0; k < a.nslot && k < gi; ++k) {
+      const int last = gi - 1 - k;
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&full[last % a.nslot], (last / a.nslot) & 1)) {
+        if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) break;
+      }
+    }
+  }
+  // 4. write the block's partial y
+  if (tid < nv && !*abort_flag) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if ((live >> t) & 1u) {
+        float4* dst = reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d + tid * 8);
+        const float4 v0 = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+        const float4 v1 = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
+        if (a.atomic) {
+          atomicAdd(dst, v0);
+          atomicAdd(dst + 1, v1);
+        } else {
+          dst[0] = v0;
+          dst[1] = v1;
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ WINA top-k
+// [WINA] section 3.1 / section 2: per token keep the k largest scores
+// s_tj = |a_tj|·n_j, equal scores going to the smaller index, and write the
+// kept neurons as TwELL.  Scores are non-negative, so their fp32 bit patterns
+// order like the values: a 4-pass 8-bit radix select finds the k-th largest
+// pattern K and how many entries equal to K are kept; tie ranks follow index
+// order through per-tile counts.  One CTA (1024 threads) per token.
+struct TopkArgs {
+  const float* scores;   // [T][F]
+  const void* vdense;    // [T][F] bf16 or fp32
+  int val_f32;
+  int T, F, k, n_tiles, C;
+  int16_t* count;
+  int16_t* idx;
+  void* val;
+  uint32_t* ovf;
+  uint32_t epoch;
+};
+
+__global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
+  extern __shared__ uint32_t tk_keys[];   // [F] then [32][256] histograms then [n_tiles] tie prefix
+  uint32_t* hist = tk_keys + a.F;
+  int* eqpre = reinterpret_cast<int*>(hist + 32 * 256);
+  __shared__ int scan_tmp[33];
+  __shared__ uint32_t sel[4];  // prefix, remaining
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* sc = a.scores + (size_t)t * a.F;
+  for (int j = tid; j < a.F; j += blockDim.x) tk_keys[j] = __float_as_uint(sc[j]);
+  const int k = a.k;
+  const bool keep_all = k >= a.F, keep_none = k <= 0;
+  uint32_t prefix = 0, mask = 0;
+  int rem = k;
+  if (!keep_all && !keep_none) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int e = tid; e < 32 * 256; e += blockDim.x) hist[e] = 0;
+      __syncthreads();
+      for (int j = tid; j < a.F; j += blockDim.x) {
+        const uint32_t key = tk_keys[j];
+        if ((key & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key >> shift) & 255u)], 1u);
+      }
+      __syncthreads();
+      // bins in descending order: suffix sums over bins 255..0 (threads 0..255 = bin 255-tid)
+      int c = 0;
+      if (tid < 256) {
+        const int bin = 255 - tid;
+        for (int w = 0; w < 32; ++w) c += (int)hist[w * 256 + bin];
+      }
+      int tot;
+      const int ex = block_scan_excl(tid < 256 ? c : 0, scan_tmp, &tot);
+      if (tid < 256 && ex < rem && ex + c >= rem) {
+        sel[0] = (uint32_t)(255 - tid);
+        sel[1] = (uint32_t)(rem - ex);
+      }
+      __syncthreads();
+      prefix |= sel[0] << shift;
+      mask |= 255u << shift;
+      rem = (int)sel[1];
+      __syncthreads();
+    }
+  }
+  // tie prefix over tiles: number of keys equal to K in lower tiles
+  const uint32_t K = prefix;
+  for (int p = warp; p < a.n_tiles; p += 32) {
+    int c = 0;
+    for (int q = 0; q < 4; ++q) c += __popc(__ballot_sync(0xFFFFFFFFu, tk_keys[p * 128 + q * 32 + lane] == K));
+    if (lane == 0) eqpre[p] = c;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int p = 0; p < a.n_tiles; ++p) {
+      const int c = eqpre[p];
+      eqpre[p] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = lanemask_lt();
+  for (int p = warp; p < a.n_tiles; p += 32) {
+    int run = 0, ties = eqpre[p];
+    const size_t rec = (size_t)t * a.n_tiles + p;
+    for (int q = 0; q < 4; ++q) {
+      const int j = p * 128 + q * 32 + lane;
+      const uint32_t key = tk_keys[j];
+      const uint32_t eqb = __ballot_sync(0xFFFFFFFFu, key == K);
+      const int tie_rank = ties + __popc(eqb & lt);
+      const bool keep = keep_all || (!keep_none && (key > K || (key == K && tie_rank < rem)));
+      ties += __popc(eqb);
+      const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
+      const int slot = run + __popc(kb & lt);
+      if (keep && slot < a.C) {
+        a.idx[rec * a.C + slot] = (int16_t)j;
+        if (a.val_f32)
+          reinterpret_cast<float*>(a.val)[rec * a.C + slot] =
+              reinterpret_cast<const float*>(a.vdense)[(size_t)t * a.F + j];
+        else
+          reinterpret_cast<__nv_bfloat16*>(a.val)[rec * a.C + slot] =
+              reinterpret_cast<const __nv_bfloat16*>(a.vdense)[(size_t)t * a.F + j];
+      }
+      run += __popc(kb);
+    }
+    for (int sl = run + lane; sl < a.C; sl += 32) {
+      a.idx[rec * a.C + sl] = -1;
+      if (a.val_f32)
+        reinterpret_cast<float*>(a.val)[rec * a.C + sl] = 0.f;
+      else
+        reinterpret_cast<__nv_bfloat16*>(a.val)[rec * a.C + sl] = __float2bfloat16_rn(0.f);
+    }
+    if (lane == 0) {
+      a.count[rec] = (int16_t)run;
+      if (run > a.C) a.ovf[t] = a.epoch;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- fp32 path
+// The fp32 configuration has no full-precision tensor-core MMA, so its gate
+// is a SIMT tile: 128 threads = the 128 neurons of one tile, 16 tokens, the
+// tokens' x staged in shared memory 256 columns at a time.  The same TwELL
+// (or WINA score) emission as the tensor-core epilogue follows.
+struct GateF32Args {
+  const float* x;       // [T][d]
+  const float* W_gate;  // [F][d]
+  int d;
+  int wina;             // 0: TwELL emission, 1: WINA dense value + score
+  TwellParams tw;
+  WinaParams wp;
+};
+
+__global__ void __launch_bounds__(128) k_gate_f32(const GateF32Args a) {
+  __shared__ __align__(16) float xs[16][256];
+  __shared__ uint32_t masks[2][64];
+  const int p = blockIdx.x, t0 = blockIdx.y * 16;
+  const int etid = threadIdx.x, j = p * 128 + etid;
+  const int T = a.wina ? a.wp.T : a.tw.T;
+  float g[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) g[i] = 0.f;
+  const float* wrow = a.W_gate + (size_t)j * a.d;
+  for (int k0 = 0; k0 < a.d; k0 += 256) {
+    const int kn = min(256, a.d - k0);
+    __syncthreads();
+    for (int e = etid; e < 16 * 256; e += 128) {
+      const int i = e >> 8, kk = e & 255;
+      const int t = t0 + i;
+      xs[i][kk] = (t < T && kk < kn) ? a.x[(size_t)t * a.d + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+    for (int kk = 0; kk < kn; ++kk) {
+      const float w = wrow[k0 + kk];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) g[i] = fmaf(w, xs[i][kk], g[i]);
+    }
+  }
+  if (a.wina)
+    wina_chunk(a.wp, g, j, t0);
+  else
+    twell_chunk(a.tw, g, j, t0, etid, masks[0]);
+}
+
+// Sparse up x down for one fp32 token per CTA: its TwELL neurons are gathered
+// into shared memory, one warp per neuron computes u = <W_up[j], x_t> and
+// h = v·u, then every thread adds h·W_down[j] into its own output columns.
+struct RowsF32Args {
+  const float* x;
+  const float* W_up;
+  const float* W_down;
+  const int16_t* count;
+  const int16_t* idx;
+  const float* val;
+  const uint32_t* ovf;
+  uint32_t epoch;
+  float* out;
+  int T, d, n_tiles, C;
+};
+
+__global__ void __launch_bounds__(256) k_rows_f32(const RowsF32Args a) {
+  extern __shared__ float rf_smem[];   // xs[d], then hj[cap], then jj[cap] (int)
+  const int t = blockIdx.x;
+  if (t >= a.T || a.ovf[t] == a.epoch) return;
+  const int cap = a.n_tiles * a.C;
+  float* xs = rf_smem;
+  float* hv = xs + a.d;
+  int* jj = reinterpret_cast<int*>(hv + cap);
+  __shared__ int scan_tmp[33];
+  __shared__ int n_keep;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < a.d; i += blockDim.x) xs[i] = a.x[(size_t)t * a.d + i];
+  // gather the kept list in tile order (ascending j)
+  int base = 0;
+  for (int p0 = 0; p0 < a.n_tiles; p0 += blockDim.x) {
+    const int p = p0 + tid;
+    const int c = p < a.n_tiles ? min((int)a.count[(size_t)t * a.n_tiles + p], a.C) : 0;
+    int tot;
+    const int ex = block_scan_excl(c, scan_tmp, &tot);
+    for (int sl = 0; sl < c; ++sl) {
+      const size_t r = ((size_t)t * a.n_tiles + p) * a.C + sl;
+      jj[base + ex + sl] = a.idx[r];
+      hv[base + ex + sl] = a.val[r];
+    }
+    base += tot;
+  }
+  if (tid == 0) n_keep = base;
+  __syncthreads();
+  const int nk = n_keep;
+  for (int e = warp; e < nk; e += blockDim.x / 32) {
+    const float* wr = a.W_up + (size_t)jj[e] * a.d;
+    float u = 0.f;
+    for (int i = lane; i < a.d; i += 32) u = fmaf(wr[i], xs[i], u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xFFFFFFFFu, u, o);
+    if (lane == 0) hv[e] = hv[e] * u;
+  }
+  __syncthreads();
+  for (int i = tid; i < a.d; i += blockDim.x) {
+    float y = 0.f;
+    for (int e = 0; e < nk; ++e) y = fmaf(hv[e], a.W_down[(size_t)jj[e] * a.d + i], y);
+    a.out[(size_t)t * a.d + i] = y;
+  }
+}
+
+// Dense fallback for one fp32 overflow token per CTA: every neuron is
+// recomputed (gate, activation, threshold, up), h is kept in shared memory and
+// the down projection follows.
+struct FallbackF32Args {
+  const float* x;
+  const float* W_gate;
+  const float* W_up;
+  const float* W_down;
+  const float* bias;
+  float tau;
+  int act;
+  const int* ovf_list;
+  const int* ovf_count;
+  float* out;
+  int d, F;
+};
+
+__global__ void __launch_bounds__(256) k_fallback_f32(const FallbackF32Args a) {
+  extern __shared__ float ff_smem[];   // xs[d], h[F]
+  const int o = blockIdx.x;
+  if (o >= *a.ovf_count) return;
+  const int t = a.ovf_list[o];
+  float* xs = ff_smem;
+  float* h = xs + a.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < a.d; i += blockDim.x) xs[i] = a.x[(size_t)t * a.d + i];
+  __syncthreads();
+  for (int j = warp; j < a.F; j += blockDim.x / 32) {
+    const float* wg = a.W_gate + (size_t)j * a.d;
+    const float* wu = a.W_up + (size_t)j * a.d;
+    float g = 0.f, u = 0.f;
+    for (int i = lane; i < a.d; i += 32) {
+      g = fmaf(wg[i], xs[i], g);
+      u = fmaf(wu[i], xs[i], u);
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      g += __shfl_xor_sync(0xFFFFFFFFu, g, s);
+      u += __shfl_xor_sync(0xFFFFFFFFu, u, s);
+    }
+    if (lane == 0) {
+      const float av = act_fn(g + (a.bias ? a.bias[j] : 0.f), a.act);
+      h[j] = fabsf(av) > a.tau ? av * u : 0.f;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < a.d; i += blockDim.x) {
+    float y = 0.f;
+    for (int j = 0; j < a.F; ++j) {
+      const float hj = h[j];
+      if (hj != 0.f) y = fmaf(hj, a.W_down[(size_t)j * a.d + i], y);
+    }
+    a.out[(size_t)t * a.d + i] = y;
+  }
+}
+
+// ------------------------------------------------------------- create time
+// out[c][r] = in[r][c] for a rows x cols bf16 matrix (32x32 tiles).
+__global__ void k_transpose_bf16(const __nv_bfloat16* in, __nv_bfloat16* out, int rows, int cols) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+// n_j = ||W_down[j,:]||_2, accumulated in fp64 and rounded to fp32 ([WINA] 3.1).
+template <typename Tw>
+__global__ void k_row_norms(const Tw* W, int F, int d, float* norms) {
+  const int j = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= F) return;
+  double s = 0.0;
+  for (int i = lane; i < d; i += 32) {
+    const double v = (double)(float)W[(size_t)j * d + i];
+    s += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if (lane == 0) norms[j] = (float)sqrt(s);
+}
+
+}  // namespace sffn

@@ -1,0 +1,194 @@
+// Tensor-core tile kernel for sm_100a: TMA -> shared memory -> tcgen05.mma ->
+// TMEM -> epilogue.  One CTA computes D[128 x BN] = A[m0:m0+128, K] ·
+// B[n0:n0+BN, K]^T for one or two GEMM phases (two accumulators, or one that
+// both phases add into), over a K range that may be split across gridDim.z.
+//
+// Warp roles (192 threads): warps 0-3 run the epilogue (warp w reads TMEM
+// lanes 32w..32w+31, one accumulator row per thread), warp 4 issues the TMA
+// loads, warp 5 owns TMEM and issues the MMAs.  Every wait is bounded; on a
+// timeout the CTA records DEV_ERR_TIMEOUT, drains its own copies and MMAs,
+// frees TMEM and returns.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace sffn {
+
+constexpr int TC_THREADS = 192;
+constexpr int TC_BM = 128;           // rows per tile (TMEM lanes)
+constexpr int TC_BK = 64;            // bf16 elements per 128-byte swizzled row
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
+
+template <int BN>
+struct TcCfg {
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 12 ? 12 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
+  static constexpr int EPI_SMEM = 9 * 1024;
+  static constexpr int SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + EPI_SMEM;
+};
+
+__host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
+  return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : n <= 256 ? 256u : 512u;
+}
+
+struct TcArgs {
+  int n_phase;          // 1 or 2
+  int acc_same;         // 1: both phases accumulate into one accumulator
+  int kb_total[2];      // 64-wide K blocks of each phase (before the split)
+  int n_rows;           // valid B rows (columns of D); CTAs with n0 >= n_rows exit
+  const int* n_rows_dev;  // if set, the valid B row count is read from the device
+  uint32_t* status;
+};
+
+// Epilogue contract:
+//   struct Epi { struct Params; static constexpr int N_ACC;
+//     __device__ static void run(const Params&, uint32_t tmem, int m0, int n0,
+//                                int split, int etid, uint8_t* scratch); };
+// run() is called by the 128 epilogue threads (etid 0..127) once the
+// accumulators are complete; accumulator a lives at TMEM column a*BN.
+
+template <int BN, class Epi>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
+          const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
+          const TcArgs args, const typename Epi::Params ep) {
+  using Cfg = TcCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr uint32_t NCOLS = tmem_cols_for(Epi::N_ACC * BN);
+  constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, BN);
+
+  const int m0 = blockIdx.x * TC_BM;
+  const int n0 = blockIdx.y * BN;
+  const int n_rows = args.n_rows_dev ? *args.n_rows_dev : args.n_rows;
+  if (n0 >= n_rows) return;  // uniform: the whole CTA leaves before any setup
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * TC_A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* scratch = smem + STAGES * Cfg::STAGE_BYTES + 256;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, NCOLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&mA0);
+    tma_prefetch_desc(&mB0);
+    if (args.n_phase > 1) {
+      tma_prefetch_desc(&mA1);
+      tma_prefetch_desc(&mB1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int S = gridDim.z, sk = blockIdx.z;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------------- TMA producer
+      int it = 0;
+      bool ok = true;
+      for (int ph = 0; ph < args.n_phase && ok; ++ph) {
+        const CUtensorMap* ma = ph == 0 ? &mA0 : &mA1;
+        const CUtensorMap* mb = ph == 0 ? &mB0 : &mB1;
+        const int kb0 = (int)((long long)args.kb_total[ph] * sk / S);
+        const int kb1 = (int)((long long)args.kb_total[ph] * (sk + 1) / S);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES, f = it / STAGES;
+          if (f > 0 && !mbar_wait(&empty[s], (f - 1) & 1, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], Cfg::STAGE_BYTES);
+          tma_load_2d(sA + s * TC_A_BYTES, ma, &full[s], kb * TC_BK, m0);
+          tma_load_2d(sB + s * Cfg::B_BYTES, mb, &full[s], kb * TC_BK, n0);
+        }
+      }
+      // Drain: the last fill of every stage has landed before the CTA can exit.
+      for (int s = 0; s < STAGES && s < it; ++s) {
+        const int last = s + STAGES * ((it - 1 - s) / STAGES);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&full[s], (last / STAGES) & 1)) {
+          if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+            atomicOr(args.status, DEV_ERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA issuer
+      int it = 0;
+      bool ok = true;
+      for (int ph = 0; ph < args.n_phase && ok; ++ph) {
+        const uint32_t dcol = args.acc_same ? 0u : (uint32_t)(ph * BN);
+        const int kb0 = (int)((long long)args.kb_total[ph] * sk / S);
+        const int kb1 = (int)((long long)args.kb_total[ph] * (sk + 1) / S);
+        bool first = (ph == 0) || !args.acc_same;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES, f = it / STAGES;
+          if (!mbar_wait(&full[s], f & 1, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sdesc_k_sw128(smem_u32(sA + s * TC_A_BYTES));
+          const uint64_t bd = sdesc_k_sw128(smem_u32(sB + s * Cfg::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k) {
+            tc_mma(tmem + dcol, ad + 2u * k, bd + 2u * k, IDESC, (first && k == 0) ? 0u : 1u);
+          }
+          first = false;
+          tc_commit(&empty[s]);
+        }
+      }
+      // An accumulator whose K range is empty stays unwritten: only happens
+      // when the split exceeds the K blocks, which the host never launches.
+      tc_commit(accf);
+      if (!ok) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(accf, 0)) {
+          if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    if (mbar_wait(accf, 0, abort_flag, args.status) && !*abort_flag) {
+      tc_fence_after();
+      Epi::template run<BN>(ep, tmem + ((uint32_t)(warp * 32) << 16), m0, n0, sk, threadIdx.x, scratch);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NCOLS);
+  }
+}
+
+}  // namespace sffn

@@ -1,0 +1,195 @@
+/*
+ * sffn.h — activation-sparse gated FFN forward for NVIDIA B200 (sm_100a).
+ *
+ * The library computes, for T tokens x_t (rows of x),
+ *
+ *     g   = W_gate x_t + b            (dense gate)   or   z = bf16(x_t A), g = z B + b   (low-rank gate)
+ *     a   = sigma(g)                  sigma = ReLU or SiLU
+ *     keep_j  iff |a_j| > threshold   (relu-threshold mode)   or   j in top-k of |a_j|·||W_down[j,:]||_2 (wina-topk mode)
+ *     v_j = round_to_operand_dtype(a_j)            (the TwELL value)
+ *     u_j = <W_up[j,:], x_t>          only for kept j
+ *     y_t = sum_{kept j} (v_j u_j) W_down[j,:]
+ *
+ * Sources (web pages, cited by title and section):
+ *   - gated FFN structure and the low-rank (rank ratio 1/8) gate:
+ *     "Meta FAIR and Inria's LoPA Gating Hits 3.31x Real GPU Speedup for LLM
+ *     Inference", section "How LoPA Gating Restructures FFN Computation";
+ *   - ReLU sparsity, the TwELL format written in the gate epilogue, the fused
+ *     up/down pass that never stores h, and routing of highly active tokens
+ *     to a dense tensor-core channel: "Sparser, Faster, Lighter Transformer
+ *     Language Models" (news article), sections "稀疏不等於提速",
+ *     "TwELL 減掉轉換開銷" and "Hybrid 應對非均勻稀疏";
+ *   - the WINA score |hidden value| x ||weight column||_2 and per-token top-K:
+ *     WINA framework explainer, sections 3.1 and 2.
+ *
+ * Layouts (all row-major, all pointers are DEVICE pointers, 16-byte aligned):
+ *   x       [T][d_model]          operand dtype (bf16 or fp32)
+ *   W_gate  [d_ff][d_model]       neuron-major: row j is neuron j (PyTorch Linear weight)
+ *   A       [d_model][rank]       low-rank gate factor (x·A)
+ *   B       [rank][d_ff]          low-rank gate factor (z·B)
+ *   W_up    [d_ff][d_model]       neuron-major (PyTorch Linear weight of up_proj)
+ *   W_down  [d_ff][d_model]       neuron-major: row j is neuron j's output row,
+ *                                 i.e. the transpose of PyTorch's down_proj.weight
+ *   gate_bias [d_ff] fp32 (optional)
+ *   out     [T][d_model] fp32
+ *
+ * TwELL (tile-wise ELLPACK) as written by the gate epilogue, one record per
+ * (token t, tile p) where a tile is 128 consecutive neurons:
+ *   count[t][p]        int16: the TRUE number kept in the tile (may exceed C)
+ *   idx[t][p][0..C)    int16: kept global neuron indices, ascending; pad -1
+ *   val[t][p][0..C)    operand dtype: v of the kept neurons; pad +0.0
+ * A token overflows iff some tile of it keeps more than C neurons; it is then
+ * computed whole by the dense tensor-core fallback.  y does not depend on C.
+ *
+ * Ownership: the caller owns x, out and all weights.  Weights are borrowed
+ * and must stay valid and unchanged for the life of the handle (the handle
+ * keeps derived copies made at create time: a transposed W_down for the
+ * tensor-core down projection, transposed low-rank factors, WINA norms).
+ * The handle owns its workspace (TwELL, routing lists, scratch, status word).
+ *
+ * Errors: argument and shape errors are returned before any launch and leave
+ * no side effect.  Launch failures return SFFN_ERR_CUDA.  Device-side problems
+ * (a bounded wait that expired, an index out of range) are recorded in the
+ * handle's device status word, which sffn_read_status() returns (and clears).
+ * sffn_forward never blocks the host.  One handle serves one forward at a time
+ * on one stream (not re-entrant); distinct handles are independent.
+ */
+#ifndef SFFN_H
+#define SFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SFFN_OK = 0,
+  SFFN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad enum       */
+  SFFN_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d_ff % 128 != 0) */
+  SFFN_ERR_ALLOC = 3,         /* device allocation failed                          */
+  SFFN_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed       */
+  SFFN_ERR_TIMEOUT = 5,       /* a device-side bounded wait expired                */
+  SFFN_ERR_DEVICE = 6,        /* a device-side range check failed                  */
+  SFFN_ERR_NO_DEVICE = 7      /* no usable sm_100 device                           */
+} sffn_status;
+
+typedef enum { SFFN_BF16 = 0, SFFN_FP32 = 1 } sffn_dtype;
+typedef enum { SFFN_MODE_RELU_THRESHOLD = 0, SFFN_MODE_WINA_TOPK = 1 } sffn_mode;
+typedef enum { SFFN_ACT_RELU = 0, SFFN_ACT_SILU = 1 } sffn_act;
+
+/* How the kept (token, neuron) pairs of non-overflow tokens are computed.
+ *   ROWS : the fused SIMT up x down kernel streams only the kept rows of W_up
+ *          and W_down, per block of 8 tokens (best when few tokens share a
+ *          neuron: decode at T <= 8, sparse prefill);
+ *   TILES: tensor-core up and down over every 128-neuron tile that some token
+ *          keeps, with the non-kept entries of h zeroed (best when the union
+ *          of kept neurons covers most tiles: WINA, T in 16..256).
+ *   AUTO : ROWS for T <= 8 or T > 256 in relu-threshold mode, TILES otherwise. */
+typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sffn_path;
+
+/* desc.flags */
+#define SFFN_FLAG_DEBUG_GATE 1u   /* keep the dense fp32 gate g[T][d_ff] of the last forward */
+
+typedef struct sffn_desc {
+  int d_model;          /* d: multiple of 8, 8..4096 (ROWS path needs d <= 4096)   */
+  int d_ff;             /* F: multiple of 128, <= 32767 (int16 TwELL indices)      */
+  int max_tokens;       /* workspace is sized for T <= max_tokens                  */
+  int rank;             /* 0: dense W_gate; > 0: low-rank A,B (bf16 only), %64==0  */
+  sffn_dtype dtype;     /* operand dtype; out is always fp32                       */
+  sffn_mode mode;
+  sffn_act act;
+  float threshold;      /* relu-threshold: keep iff |sigma(g)| > threshold (>= 0)  */
+  int k;                /* wina-topk: neurons kept per token, 0..d_ff              */
+  int tile_capacity;    /* C: 8, 16, 32, 64 or 128                                 */
+  int path;             /* sffn_path                                               */
+  unsigned flags;       /* SFFN_FLAG_*                                             */
+  const void* W_gate;   /* [d_ff][d_model]  (NULL iff rank > 0)                    */
+  const void* A;        /* [d_model][rank]  (NULL iff rank == 0)                   */
+  const void* B;        /* [rank][d_ff]     (NULL iff rank == 0)                   */
+  const void* W_up;     /* [d_ff][d_model]                                         */
+  const void* W_down;   /* [d_ff][d_model]                                         */
+  const float* gate_bias; /* [d_ff] fp32 or NULL                                   */
+} sffn_desc;
+
+typedef struct sffn_handle sffn_handle;
+
+/* Validate desc, allocate the workspace for max_tokens, build the TMA tensor
+ * maps and the create-time derived data (transposed W_down; transposed A and
+ * B; WINA norms), all on `cuda_stream` (a cudaStream_t, NULL = legacy default
+ * stream).  Synchronises the stream before returning.  On error *out is NULL
+ * and nothing stays allocated. */
+sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** out);
+
+/* y = FFN(x) for T tokens, asynchronously on `cuda_stream`.  x: [T][d_model]
+ * device, operand dtype; out: [T][d_model] fp32 device, fully overwritten.
+ * 0 <= T <= max_tokens; T == 0 returns SFFN_OK and launches nothing.  Must not
+ * overlap another forward of the same handle. */
+sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void* cuda_stream);
+
+/* Same as sffn_forward but x and out are HOST buffers: copies x to the
+ * handle's device staging buffer, runs the forward and copies y back, all on
+ * `cuda_stream`, then synchronises it.  Page-locked host memory makes the
+ * copies asynchronous DMA. */
+sffn_status sffn_forward_host(sffn_handle* h, const void* x_host, int T, float* out_host,
+                              void* cuda_stream);
+
+/* Free everything the handle owns.  NULL is accepted (SFFN_OK). */
+sffn_status sffn_destroy(sffn_handle* h);
+
+const char* sffn_status_string(sffn_status s);
+
+/* Synchronise `cuda_stream`, then return and clear the device status word
+ * (SFFN_OK, SFFN_ERR_TIMEOUT or SFFN_ERR_DEVICE). */
+sffn_status sffn_read_status(sffn_handle* h, void* cuda_stream);
+
+/* Device views of the last forward's TwELL and overflow flags (valid until the
+ * next forward or destroy).  count: int16 [T][n_tiles]; idx: int16
+ * [T][n_tiles][C]; val: operand dtype [T][n_tiles][C]; overflow: uint32 [T],
+ * equal to sffn_stats.epoch iff the token took the dense channel in the last
+ * forward.  Test and bench use. */
+sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_t** idx,
+                             const void** val, const uint32_t** overflow, int* n_tiles,
+                             int* tile_capacity);
+
+/* Device view of the dense fp32 gate g[T][d_ff] of the last forward (only
+ * with SFFN_FLAG_DEBUG_GATE; dense gate only).  Test use. */
+sffn_status sffn_debug_gate(sffn_handle* h, const float** g);
+
+/* Device view of the WINA norms n_j (fp32 [d_ff]), wina-topk mode only. */
+sffn_status sffn_debug_norms(sffn_handle* h, const float** norms);
+
+/* Counters of the last forward, copied to the host (synchronises the stream):
+ * number of overflow tokens, the number of kernel launches it made, the path
+ * taken and the forward's epoch (see sffn_debug_twell). */
+typedef struct sffn_stats {
+  int n_overflow;
+  int n_launches;
+  int path;             /* the sffn_path actually taken (ROWS or TILES) */
+  unsigned epoch;       /* overflow[t] == epoch marks the last forward's overflow tokens */
+} sffn_stats;
+sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st);
+
+/* Per-kernel device timing (bench use).  Between sffn_timing_begin and
+ * sffn_timing_end every forward records a CUDA event on its own stream before
+ * each kernel launch and after the last one; no work is skipped or added.
+ * max_forwards bounds the forwards recorded (later ones are not timed). */
+sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards);
+
+/* Synchronise the recorded events and report, per kernel label (a short
+ * name such as "gate" or "updown_rows", NUL-terminated, at most 31 chars), the
+ * summed device time in ms and the number of launches timed.  At most
+ * max_kernels labels are written; *n_kernels receives how many exist.
+ * Timing is off afterwards. */
+sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], float* total_ms,
+                            int* launches, int* n_kernels);
+
+/* Library version string. */
+const char* sffn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFFN_H */

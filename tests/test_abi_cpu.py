@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads,
+exports every entry point include/sffn.h declares, and rejects bad arguments
+before touching CUDA."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from activation_sparse_gated_relu_b200 import binding as B
+from activation_sparse_gated_relu_b200.build import HEADER, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return B.load_library()
+
+
+def _declared_symbols() -> set[str]:
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"\b(sffn_[a-z_]+)\s*\(", text))
+
+
+def test_header_declares_the_north_star_calls():
+    syms = _declared_symbols()
+    assert {"sffn_create", "sffn_forward", "sffn_destroy"} <= syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (sffn_\w+)", out))
+    missing = _declared_symbols() - exported
+    assert not missing, missing
+    for s in _declared_symbols():
+        assert hasattr(lib, s)
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert B.status_string(s) and B.status_string(s) != "unknown status"
+    assert B.status_string(99) == "unknown status"
+    assert "sm_100a" in B.sffn_version()
+
+
+def _desc(**kw):
+    d = B.sffn_desc()
+    d.d_model, d.d_ff, d.max_tokens, d.rank = 4096, 14336, 8, 0
+    d.dtype, d.mode, d.act = B.SFFN_BF16, B.SFFN_MODE_RELU_THRESHOLD, B.SFFN_ACT_RELU
+    d.threshold, d.k, d.tile_capacity, d.path, d.flags = 0.0, 0, 32, 0, 0
+    fake = 0x7F0000000000  # 16-byte aligned, never dereferenced by validation
+    d.W_gate, d.W_up, d.W_down, d.gate_bias = fake, fake + 0x100, fake + 0x200, fake + 0x300
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def _create(lib, d):
+    h = ctypes.c_void_p()
+    s = lib.sffn_create(ctypes.byref(d) if d is not None else None, None, ctypes.byref(h))
+    return s, h
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d_ff=14335), B.SFFN_ERR_UNSUPPORTED),           # not a multiple of 128
+    (dict(d_ff=32768), B.SFFN_ERR_UNSUPPORTED),           # int16 indices
+    (dict(d_model=4100), B.SFFN_ERR_UNSUPPORTED),         # d % 8
+    (dict(d_model=8192), B.SFFN_ERR_UNSUPPORTED),
+    (dict(d_model=0), B.SFFN_ERR_INVALID_ARG),
+    (dict(max_tokens=0), B.SFFN_ERR_INVALID_ARG),
+    (dict(max_tokens=1 << 20), B.SFFN_ERR_UNSUPPORTED),
+    (dict(tile_capacity=24), B.SFFN_ERR_INVALID_ARG),
+    (dict(dtype=7), B.SFFN_ERR_INVALID_ARG),
+    (dict(mode=3), B.SFFN_ERR_INVALID_ARG),
+    (dict(act=5), B.SFFN_ERR_INVALID_ARG),
+    (dict(path=9), B.SFFN_ERR_INVALID_ARG),
+    (dict(threshold=-1.0), B.SFFN_ERR_INVALID_ARG),
+    (dict(threshold=float("nan")), B.SFFN_ERR_INVALID_ARG),
+    (dict(W_up=None), B.SFFN_ERR_INVALID_ARG),
+    (dict(W_gate=None), B.SFFN_ERR_INVALID_ARG),         # dense gate needs W_gate
+    (dict(W_gate=0x7F0000000008), B.SFFN_ERR_INVALID_ARG),  # misaligned
+    (dict(rank=512), B.SFFN_ERR_INVALID_ARG),             # W_gate given with rank > 0
+    (dict(mode=1, k=20000), B.SFFN_ERR_INVALID_ARG),      # k > d_ff
+    (dict(mode=1, k=100, tile_capacity=32), B.SFFN_ERR_UNSUPPORTED),  # WINA needs C = 128
+])
+def test_create_rejects_bad_descriptors(lib, kw, want):
+    s, h = _create(lib, _desc(**kw))
+    assert s == want, (kw, B.status_string(s))
+    assert h.value is None
+
+
+def test_create_lowrank_rules(lib):
+    fake = 0x7F0000001000
+    ok = dict(rank=512, W_gate=None, A=fake, B=fake + 0x100)
+    assert _create(lib, _desc(**ok))[0] in (B.SFFN_ERR_NO_DEVICE, B.SFFN_OK)
+    assert _create(lib, _desc(**{**ok, "rank": 100}))[0] == B.SFFN_ERR_UNSUPPORTED
+    assert _create(lib, _desc(**{**ok, "dtype": B.SFFN_FP32}))[0] == B.SFFN_ERR_UNSUPPORTED
+    assert _create(lib, _desc(**{**ok, "B": None}))[0] == B.SFFN_ERR_INVALID_ARG
+
+
+def test_null_arguments(lib):
+    h = ctypes.c_void_p()
+    assert lib.sffn_create(None, None, ctypes.byref(h)) == B.SFFN_ERR_INVALID_ARG
+    d = _desc()
+    assert lib.sffn_create(ctypes.byref(d), None, None) == B.SFFN_ERR_INVALID_ARG
+    assert lib.sffn_destroy(None) == B.SFFN_OK
+    assert lib.sffn_forward(None, None, 1, None, None) == B.SFFN_ERR_INVALID_ARG
+    assert lib.sffn_forward_host(None, None, 1, None, None) == B.SFFN_ERR_INVALID_ARG
+    assert lib.sffn_read_status(None, None) == B.SFFN_ERR_INVALID_ARG
+    assert lib.sffn_get_stats(None, None, None) == B.SFFN_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="a GPU is present")
+def test_valid_descriptor_without_gpu_reports_no_device(lib):
+    s, h = _create(lib, _desc())
+    assert s == B.SFFN_ERR_NO_DEVICE and h.value is None
+
+
+def test_binding_raises_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(ImportError):
+        B.load_library(str(tmp_path / "missing.so"))
