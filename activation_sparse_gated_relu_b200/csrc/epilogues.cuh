@@ -33,7 +33,7 @@ struct TwellParams {
   int val_f32;
   uint32_t* ovf;      // [T]: = epoch iff the token overflows in this forward
   uint32_t epoch;
-  uint32_t* umask;    // [ceil(T/8)][n_tiles][4] union of kept bits per 8-token block, or null
+  uint32_t* kmask;    // [T][n_tiles][4] kept bits of every (token, tile), or null
   float* gdebug;      // [T][F] dense gate (debug), or null
 };
 
@@ -55,16 +55,11 @@ __device__ __forceinline__ void twell_chunk(const TwellParams& o, const float* g
     const uint32_t bal = __ballot_sync(0xFFFFFFFFu, k);
     if (lane == 0) masks[w * 16 + i] = bal;
   }
-  if (o.umask) {
-    const uint32_t u0 = __ballot_sync(0xFFFFFFFFu, (keep & 0x00FFu) != 0);
-    const uint32_t u1 = __ballot_sync(0xFFFFFFFFu, (keep & 0xFF00u) != 0);
-    if (lane == 0) {
-      const int blk = t0 >> 3;
-      if (t0 < o.T) o.umask[((size_t)blk * o.n_tiles + p) * 4 + w] = u0;
-      if (t0 + 8 < o.T) o.umask[((size_t)(blk + 1) * o.n_tiles + p) * 4 + w] = u1;
-    }
-  }
   named_bar_sync(1, 128);
+  if (o.kmask && etid < 64) {
+    const int i = etid & 15, ww = etid >> 4;
+    if (t0 + i < o.T) o.kmask[((size_t)(t0 + i) * o.n_tiles + p) * 4 + ww] = masks[ww * 16 + i];
+  }
   const uint32_t lt = lanemask_lt();
 #pragma unroll 4
   for (int i = 0; i < 16; ++i) {

@@ -25,6 +25,7 @@
 
 #include "../../include/sffn.h"
 #include "epilogues.cuh"
+#include "rows_mma.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 
@@ -127,6 +128,7 @@ struct sffn_handle {
   void* val = nullptr;
   uint32_t* ovf = nullptr;
   uint32_t* umask = nullptr;
+  uint32_t* kmask = nullptr;
   int* ovf_list = nullptr;
   int* ovf_count = nullptr;
   uint8_t* blk_live = nullptr;
@@ -151,6 +153,9 @@ struct sffn_handle {
   CUtensorMap tmWgate, tmWup, tmWdT, tmAt, tmBt;
   int last_T = 0, last_path = 0, last_launches = 0;
   int rows_nslot = 0, rows_lcap = 0, rows_smem = 0;
+  int rows_cs = 1, rows_max_ctas = 0;  // cluster size of the split fused kernel, co-resident CTAs
+  bool rows_ok = false;                // the fused row kernel supports this shape
+  __nv_bfloat16* zero_row = nullptr;   // 2 KB of zeros: row chunks of padding neurons
   // per-kernel timing (sffn_timing_begin/end)
   bool tm_on = false;
   int tm_max = 0, tm_n = 0, tm_cur = -1;
@@ -166,9 +171,10 @@ void timing_free(sffn_handle* h);
 void free_handle(sffn_handle* h) {
   if (!h) return;
   timing_free(h);
-  void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->umask, h->ovf_list, h->ovf_count, h->blk_live,
+  void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->umask, h->kmask, h->ovf_list, h->ovf_count, h->blk_live,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zacc,
-                  h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage};
+                  h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
+                  h->zero_row};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -310,6 +316,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   ok = ok && dalloc(&h->val, T * P * C * h->esize);
   ok = ok && dalloc(&h->ovf, T * 4);
   ok = ok && dalloc(&h->umask, nblk * P * 16);
+  ok = ok && dalloc(&h->kmask, T * P * 16);
   ok = ok && dalloc(&h->ovf_list, T * 4);
   ok = ok && dalloc(&h->ovf_count, 16);
   ok = ok && dalloc(&h->blk_live, nblk);
@@ -321,6 +328,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     ok = ok && dalloc(&h->h_hi, T * F * 2);
     ok = ok && dalloc(&h->h_lo, T * F * 2);
     ok = ok && dalloc(&h->WdT, d * F * 2);
+    ok = ok && dalloc(&h->zero_row, 2048);
   }
   if (h->wina) {
     ok = ok && dalloc(&h->scores, T * F * 4);
@@ -345,6 +353,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
   e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
+  if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, 2048, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->zacc, 0, T * (size_t)h->R * 4, st);
     e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * (T / 16 + 2) * 4, st);
@@ -396,19 +405,47 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     // fused up x down: ring slots and list capacity from the shared memory budget
     int max_smem = 0;
     cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    int nslot = 16, lcap = 1024;
-    while (nslot > 2 && RowsSmem::make(h->d, h->P, nslot, 256).total > max_smem) --nslot;
-    while (lcap > 64 && RowsSmem::make(h->d, h->P, nslot, lcap).total > max_smem) lcap -= 64;
-    h->rows_nslot = nslot;
+    int lcap = 512;
+    while (lcap > 64 && RowsSmem::make(h->P, lcap).total > max_smem) lcap -= 64;
+    h->rows_nslot = RW_NS;
     h->rows_lcap = lcap;
-    h->rows_smem = RowsSmem::make(h->d, h->P, nslot, lcap).total;
+    h->rows_smem = RowsSmem::make(h->P, lcap).total;
+    // the ring doubles as the [8][d] fp32 partial-output buffer
+    h->rows_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXC * RW_CHUNK &&
+                 (long long)RW_NS * RowsSmem::STAGE >= 32LL * h->d && h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
+    // largest cluster (4, else 2) whose co-resident CTAs still cover almost every SM
+    h->rows_cs = 1;
+    h->rows_max_ctas = h->n_sm;
+    for (int cs = 4; cs >= 2 && !e; cs /= 2) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((h->n_sm / cs) * cs, 1, 1);
+      cfg.blockDim = dim3(RW_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = h->rows_smem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = cs;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, k_rows, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      if (ncl * cs >= h->n_sm - 8) {
+        h->rows_cs = cs;
+        h->rows_max_ctas = ncl * cs;
+        break;
+      }
+    }
   }
   if (!e && h->wina) {
     const int tk_smem = (int)(F * 4 + 32 * 256 * 4 + P * 4);
     e = cudaFuncSetAttribute(k_wina_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, tk_smem);
   }
-  if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(T * 4));
+  if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, router_smem_bytes((int)T));
   if (!e && h->f32) {
     e = cudaFuncSetAttribute(k_rows_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)((d + 2 * P * C) * 4));
@@ -447,11 +484,18 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   if (!mok) return SFFN_ERR_CUDA;
 
   int path = D.path;
-  if (path == SFFN_PATH_AUTO) path = (T <= 8 || T > 256) ? SFFN_PATH_ROWS : SFFN_PATH_TILES;
-  if (h->wina) path = SFFN_PATH_TILES;  // the top-k kernel writes no union masks
+  if (path == SFFN_PATH_AUTO) path = (h->rows_ok && (T <= 8 || T > 256)) ? SFFN_PATH_ROWS : SFFN_PATH_TILES;
+  if (h->wina) path = SFFN_PATH_TILES;  // the top-k kernel writes no per-token keep masks
+  if (path == SFFN_PATH_ROWS && !h->rows_ok) return SFFN_ERR_UNSUPPORTED;
   const bool rows = path == SFFN_PATH_ROWS;
   const int nblk = cdiv(T, 8);
-  const int rows_split = rows ? std::max(1, h->n_sm / nblk) : 1;
+  int rows_split = rows ? std::max(1, h->n_sm / nblk) : 1;
+  int rows_cs = 1;
+  if (rows_split > 1) {  // split blocks: clusters of rows_cs CTAs, all resident at once
+    rows_cs = h->rows_cs;
+    rows_split = std::min(rows_split, std::max(1, h->rows_max_ctas / nblk));
+    rows_split = std::max(rows_cs, (rows_split / rows_cs) * rows_cs);
+  }
   // down projection split over d_ff so that its grid covers the SMs
   const int m_tiles_down = cdiv(d, 128);
   const int est_rows_tiles = rows ? 1 : ntile_tok;
@@ -473,7 +517,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   tw.val_f32 = 0;
   tw.ovf = h->ovf;
   tw.epoch = epoch;
-  tw.umask = rows ? h->umask : nullptr;
+  tw.kmask = rows ? h->kmask : nullptr;
   tw.gdebug = h->gdebug;
 
   // ---------------------------------------------------------------- gate
@@ -529,6 +573,9 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   ra.ovf_list = h->ovf_list;
   ra.ovf_count = h->ovf_count;
   ra.blk_live = h->blk_live;
+  ra.kmask = reinterpret_cast<const uint4*>(h->kmask);
+  ra.umask = rows ? reinterpret_cast<uint4*>(h->umask) : nullptr;
+  ra.P = P;
   ra.x = static_cast<const uint4*>(x);
   ra.xo = reinterpret_cast<uint4*>(h->xo);
   ra.d_vec = d / 8;
@@ -540,7 +587,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   ra.zero_mode = (!rows || rows_split > 1) ? 1 : (sk_down > 1 ? 2 : 0);
   const int router_ctas = std::max(1, std::min(h->n_sm, cdiv((long long)T * d / 4, 4096)));
   tmark(h, st, L_ROUTER);
-  k_router<<<router_ctas, 1024, (size_t)T * 4, st>>>(ra);
+  k_router<<<router_ctas, 1024, (size_t)router_smem_bytes(T), st>>>(ra);
   ++launches;
   if (cudaGetLastError()) return SFFN_ERR_CUDA;
 
@@ -550,6 +597,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     rw.x = static_cast<const __nv_bfloat16*>(x);
     rw.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
     rw.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
+    rw.zero_row = h->zero_row;
     rw.count = h->count;
     rw.idx = h->idx;
     rw.val = static_cast<const __nv_bfloat16*>(h->val);
@@ -566,9 +614,23 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     rw.lcap = h->rows_lcap;
     rw.status = h->status;
     tmark(h, st, L_UPDOWN_ROWS);
-    k_rows<<<dim3(rows_split, nblk), RW_THREADS, h->rows_smem, st>>>(rw);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows_split, nblk, 1);
+    cfg.blockDim = dim3(RW_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = h->rows_smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = rows_cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = rows_cs > 1 ? 1 : 0;
     ++launches;
-    if (cudaGetLastError()) return SFFN_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, k_rows, rw) != cudaSuccess) {
+      cudaGetLastError();
+      return SFFN_ERR_CUDA;
+    }
   } else {
     TcArgs ua{};
     ua.n_phase = 1;
@@ -661,7 +723,7 @@ static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out,
   ga.tw.val_f32 = 1;
   ga.tw.ovf = h->ovf;
   ga.tw.epoch = epoch;
-  ga.tw.umask = nullptr;
+  ga.tw.kmask = nullptr;
   ga.tw.gdebug = h->gdebug;
   ga.wp = WinaParams{D.gate_bias, D.act, T, F, h->norms, h->vdense, 1, h->scores};
   tmark(h, st, L_GATE_F32);
@@ -684,7 +746,7 @@ static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out,
   ra.blk_live = h->blk_live;
   ra.zero_mode = 0;
   tmark(h, st, L_ROUTER);
-  k_router<<<1, 1024, (size_t)T * 4, st>>>(ra);
+  k_router<<<1, 1024, (size_t)router_smem_bytes(T), st>>>(ra);
   ++launches;
   RowsF32Args rf{static_cast<const float*>(x), static_cast<const float*>(D.W_up), static_cast<const float*>(D.W_down),
                  h->count, h->idx, static_cast<const float*>(h->val), h->ovf, epoch, out, T, d, P, h->C};

@@ -42,10 +42,12 @@ __device__ __forceinline__ int block_scan_excl(int v, int* warp_tot, int* total)
 // ---------------------------------------------------------------- router
 // Hybrid routing ([TwELL] "Hybrid 應對非均勻稀疏"): a token whose TwELL record
 // overflowed in some tile goes whole to the dense channel.  Every CTA ranks
-// the overflow tokens itself (the flags are few), CTA 0 publishes the list,
-// the count and the per-8-token-block live masks, and all CTAs gather the
-// overflow rows of x (and z) and zero the output rows that are accumulated
-// with atomics afterwards.
+// the overflow tokens itself (the flags are few) and keeps them as a bit set;
+// CTA 0 publishes the overflow list, its count and the per-8-token-block live
+// masks; all CTAs then gather the overflow rows of x (and z), build the union
+// of kept neurons of every (8-token block, tile) over the block's live tokens
+// from the gate epilogue's per-token keep masks, and zero the output rows that
+// are accumulated with atomics afterwards.
 struct RouterArgs {
   int T;
   const uint32_t* ovf;
@@ -53,6 +55,9 @@ struct RouterArgs {
   int* ovf_list;           // [maxT]
   int* ovf_count;          // [1]
   uint8_t* blk_live;       // [ceil(T/8)]: bit i = token 8b+i < T and not overflow
+  const uint4* kmask;      // [T][P] kept bits per (token, tile), or null
+  uint4* umask;            // [ceil(T/8)][P] union over the block's live tokens
+  int P;
   const uint4* x;          // [T][d] bf16 as 16-byte vectors, or null (no gather)
   uint4* xo;               // [maxT][d]
   int d_vec;               // d / 8
@@ -64,13 +69,18 @@ struct RouterArgs {
   int zero_mode;           // 0: none, 1: all T rows, 2: overflow rows only
 };
 
+__host__ __device__ inline int router_smem_bytes(int T) { return T * 4 + ((T + 31) / 32) * 4; }
+
 __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
-  extern __shared__ int rs_list[];   // [T]
+  extern __shared__ int rs_list[];   // [T] overflow list, then [ceil(T/32)] overflow bits
+  uint32_t* obits = reinterpret_cast<uint32_t*>(rs_list + a.T);
   __shared__ int scan_tmp[33];
   int base = 0;
   for (int c = 0; c < a.T; c += blockDim.x) {
     const int t = c + threadIdx.x;
     const int f = (t < a.T && a.ovf[t] == a.epoch) ? 1 : 0;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, f);
+    if ((threadIdx.x & 31) == 0 && t < a.T) obits[t >> 5] = bal;
     int tot;
     const int ex = block_scan_excl(f, scan_tmp, &tot);
     if (f) rs_list[base + ex] = t;
@@ -78,21 +88,33 @@ __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
   }
   __syncthreads();
   const int n_o = base;
+  const int nb = (a.T + 7) >> 3;
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < n_o; i += blockDim.x) a.ovf_list[i] = rs_list[i];
     if (threadIdx.x == 0) *a.ovf_count = n_o;
-    const int nb = (a.T + 7) >> 3;
     for (int b = threadIdx.x; b < nb; b += blockDim.x) {
-      uint32_t m = 0;
-      for (int i = 0; i < 8; ++i) {
-        const int t = b * 8 + i;
-        if (t < a.T && a.ovf[t] != a.epoch) m |= 1u << i;
-      }
-      a.blk_live[b] = (uint8_t)m;
+      const int valid = min(8, a.T - b * 8);
+      const uint32_t ob = (obits[(b * 8) >> 5] >> ((b * 8) & 31)) & 0xFFu;
+      a.blk_live[b] = (uint8_t)(((1u << valid) - 1u) & ~ob);
     }
   }
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long gstride = (long long)gridDim.x * blockDim.x;
+  if (a.umask) {
+    const long long n = (long long)nb * a.P;
+    for (long long e = gtid; e < n; e += gstride) {
+      const int b = (int)(e / a.P), p = (int)(e % a.P);
+      const int valid = min(8, a.T - b * 8);
+      const uint32_t ob = (obits[(b * 8) >> 5] >> ((b * 8) & 31)) & 0xFFu;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < valid; ++i) {
+        if ((ob >> i) & 1u) continue;
+        const uint4 m = a.kmask[(size_t)(b * 8 + i) * a.P + p];
+        u.x |= m.x; u.y |= m.y; u.z |= m.z; u.w |= m.w;
+      }
+      a.umask[e] = u;
+    }
+  }
   if (a.x) {
     const long long n = (long long)n_o * a.d_vec;
     for (long long e = gtid; e < n; e += gstride) {
@@ -116,342 +138,6 @@ __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
     for (long long e = gtid; e < n; e += gstride) {
       const int o = (int)(e / a.d4), v = (int)(e % a.d4);
       a.out[(size_t)rs_list[o] * a.d4 + v] = zero4;
-    }
-  }
-}
-
-// ------------------------------------------------- fused sparse up x down
-// [TwELL] "TwELL 減掉轉換開銷": one pass computes both projections for the kept
-// (token, neuron) pairs and never stores h.  One CTA works on a block of 8
-// tokens and a contiguous range of the block's union of kept neurons (ranked
-// tile by tile from the union masks the gate epilogue wrote), so that every
-// CTA streams the same number of W_up / W_down rows.  A producer thread
-// stages each kept neuron's W_up and W_down rows (contiguous, neuron-major)
-// into a shared-memory ring with 1-D bulk copies (thread 0 refills the slots
-// a batch has released right after the batch's closing barrier, so no
-// producer warp takes registers from the consumers); 16 warps compute
-// u_tj = <W_up[j], x_t> (4 warps per neuron, warp-shuffle reduction), form
-// h_tj = v_tj·u_tj in registers and add h_tj·W_down[j] into per-thread
-// accumulators that own 8 output columns for each of the 8 tokens.  The
-// partial y goes to out with plain stores (one CTA per block) or vector
-// atomics (a block split over several CTAs).
-constexpr int RW_CW = 16;                    // warps (all consume; thread 0 also issues copies)
-constexpr int RW_THREADS = RW_CW * 32;
-constexpr int RW_NB = 4;                     // neurons per consumer batch
-constexpr int RW_WPN = RW_CW / RW_NB;        // warps per neuron in the up phase
-
-struct RowsArgs {
-  const __nv_bfloat16* x;
-  const __nv_bfloat16* W_up;
-  const __nv_bfloat16* W_down;
-  const int16_t* count;
-  const int16_t* idx;
-  const __nv_bfloat16* val;
-  const uint4* umask;        // [n_blk][n_tiles] 128-bit union masks
-  const uint8_t* blk_live;
-  float* out;
-  int T, d, F, n_tiles, C;
-  int atomic;
-  int nslot, lcap;
-  uint32_t* status;
-};
-
-struct RowsSmem {
-  // byte offsets inside the dynamic shared memory
-  int xs, ring, bars, tpre, nid, lmask, lval, nid2, lmask2, lval2, part, misc, total;
-  __host__ __device__ static RowsSmem make(int d, int n_tiles, int nslot, int lcap) {
-    RowsSmem s;
-    int o = 0;
-    s.xs = o;    o += 8 * d * 2;
-    s.ring = o;  o += nslot * 4 * d;
-    s.bars = o;  o += (nslot * 8 + 15) & ~15;
-    s.tpre = o;  o += ((n_tiles + 1) * 4 + 15) & ~15;
-    s.nid = o;   o += lcap * 4;
-    s.lmask = o; o += lcap * 4;
-    s.lval = o;  o += lcap * 16;
-    s.nid2 = o;  o += lcap * 4;
-    s.lmask2 = o; o += lcap * 4;
-    s.lval2 = o; o += lcap * 16;
-    s.part = o;  o += RW_NB * RW_WPN * 8 * 4;
-    s.misc = o;  o += 64 * 4;
-    s.total = o;
-    return s;
-  }
-};
-
-__device__ __forceinline__ uint32_t word4(const uint4& m, int q) {
-  return q == 0 ? m.x : q == 1 ? m.y : q == 2 ? m.z : m.w;
-}
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
-  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-}
-
-__global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  const RowsSmem L = RowsSmem::make(a.d, a.n_tiles, a.nslot, a.lcap);
-  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sm + L.xs);
-  uint8_t* ring = sm + L.ring;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
-  int* tpre = reinterpret_cast<int*>(sm + L.tpre);
-  int* nid = reinterpret_cast<int*>(sm + L.nid);
-  uint32_t* lmask = reinterpret_cast<uint32_t*>(sm + L.lmask);
-  uint4* lval = reinterpret_cast<uint4*>(sm + L.lval);
-  int* nid2 = reinterpret_cast<int*>(sm + L.nid2);
-  uint32_t* lmask2 = reinterpret_cast<uint32_t*>(sm + L.lmask2);
-  uint4* lval2 = reinterpret_cast<uint4*>(sm + L.lval2);
-  float* part = reinterpret_cast<float*>(sm + L.part);
-  int* misc = reinterpret_cast<int*>(sm + L.misc);
-  volatile int* abort_flag = misc + 40;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int P = a.n_tiles, b = blockIdx.y, S = gridDim.x, s = blockIdx.x;
-  const int tb0 = b * 8;
-  const uint32_t live = a.blk_live[b];
-  const int d = a.d, nv = d >> 3;
-  const uint32_t row_bytes = (uint32_t)d * 2u;
-  const uint4* um = a.umask + (size_t)b * P;
-
-  // 1. union counts per tile -> exclusive prefix tpre[0..P]
-  if (warp == 0) {
-    int run = 0;
-    for (int p0 = 0; p0 < P; p0 += 32) {
-      const int p = p0 + lane;
-      int c = 0;
-      if (p < P) {
-        const uint4 m = um[p];
-        c = __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
-      }
-      int inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-        if (lane >= o) inc += n;
-      }
-      if (p < P) tpre[p] = run + inc - c;
-      run += __shfl_sync(0xFFFFFFFFu, inc, 31);
-    }
-    if (lane == 0) tpre[P] = run;
-  }
-  if (tid == 0) {
-    for (int i = 0; i < a.nslot; ++i) mbar_init(&full[i], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  // 2. the block's x rows (zero beyond T)
-  for (int e = tid; e < 8 * nv; e += blockDim.x) {
-    const int row = e / nv, v = e - row * nv;
-    const int t = tb0 + row;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (t < a.T) val = reinterpret_cast<const uint4*>(a.x + (size_t)t * d)[v];
-    reinterpret_cast<uint4*>(xs + (size_t)row * d)[v] = val;
-  }
-  __syncthreads();
-  const int U = tpre[P];
-  const int r0 = (int)((long long)U * s / S), r1 = (int)((long long)U * (s + 1) / S);
-
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
-
-  int gi = 0;  // running ring index (uniform)
-  for (int c0 = r0; c0 < r1; c0 += a.lcap) {
-    const int c1 = min(r1, c0 + a.lcap), Lc = c1 - c0;
-    // a. neuron ids of ranks [c0, c1)
-    for (int p = tid; p < P; p += blockDim.x) {
-      const int lo = tpre[p], hi = tpre[p + 1];
-      if (hi <= c0 || lo >= c1) continue;
-      const uint4 m4 = um[p];
-      int rank = lo;
-      for (int q = 0; q < 4; ++q) {
-        uint32_t m = word4(m4, q);
-        while (m) {
-          const int bit = __ffs(m) - 1;
-          m &= m - 1;
-          if (rank >= c0 && rank < c1) nid[rank - c0] = p * 128 + q * 32 + bit;
-          ++rank;
-        }
-      }
-    }
-    for (int e = tid; e < Lc; e += blockDim.x) {
-      lmask[e] = 0u;
-      lval[e] = make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    // b. scatter the TwELL values of the block's live tokens
-    for (int e = tid; e < 8 * P; e += blockDim.x) {
-      const int i = e & 7, p = e >> 3;
-      if (!((live >> i) & 1u)) continue;
-      const int lo = tpre[p], hi = tpre[p + 1];
-      if (hi <= c0 || lo >= c1) continue;
-      const size_t rec = (size_t)(tb0 + i) * P + p;
-      const int cnt = min((int)a.count[rec], a.C);
-      const uint4 m4 = um[p];
-      for (int sl = 0; sl < cnt; ++sl) {
-        const int bit = (int)a.idx[rec * a.C + sl] - p * 128;
-        if (bit < 0 || bit >= 128) {
-          atomicOr(a.status, DEV_ERR_RANGE);
-          continue;
-        }
-        const int q = bit >> 5;
-        int below = __popc(word4(m4, q) & ((1u << (bit & 31)) - 1u));
-        if (q > 0) below += __popc(m4.x);
-        if (q > 1) below += __popc(m4.y);
-        if (q > 2) below += __popc(m4.z);
-        const int rank = lo + below;
-        if (rank >= c0 && rank < c1) {
-          reinterpret_cast<uint16_t*>(&lval[rank - c0])[i] =
-              reinterpret_cast<const uint16_t*>(a.val)[rec * a.C + sl];
-          atomicOr(&lmask[rank - c0], 1u << i);
-        }
-      }
-    }
-    __syncthreads();
-    // c. drop neurons that only overflow tokens kept
-    int L2;
-    {
-      const int per = (Lc + blockDim.x - 1) / blockDim.x;
-      const int e0 = min(Lc, tid * per), e1 = min(Lc, e0 + per);
-      int cnt = 0;
-      for (int e = e0; e < e1; ++e) cnt += lmask[e] ? 1 : 0;
-      int tot;
-      int o = block_scan_excl(cnt, misc, &tot);
-      for (int e = e0; e < e1; ++e) {
-        if (lmask[e]) {
-          nid2[o] = nid[e];
-          lmask2[o] = lmask[e];
-          lval2[o] = lval[e];
-          ++o;
-        }
-      }
-      L2 = tot;
-    }
-    __syncthreads();
-    // d. stream the rows through the ring
-    auto issue = [&](int i) {  // thread 0 only: entry i of this chunk -> its slot
-      const int gs = gi + i, slot = gs % a.nslot;
-      uint8_t* dst = ring + (size_t)slot * 4 * d;
-      const size_t row = (size_t)nid2[i] * d;
-      mbar_expect_tx(&full[slot], 2u * row_bytes);
-      bulk_g2s(dst, a.W_up + row, row_bytes, &full[slot]);
-      bulk_g2s(dst + row_bytes, a.W_down + row, row_bytes, &full[slot]);
-    };
-    if (tid == 0) {
-      const int pro = min(L2, a.nslot);
-      for (int i = 0; i < pro; ++i) issue(i);
-    }
-    for (int i0 = 0; i0 < L2; i0 += RW_NB) {
-      // up: 4 warps per neuron, each over a quarter of the row
-      {
-        const int n = i0 + warp / RW_WPN, q = warp % RW_WPN;
-        if (n < L2) {
-          const int gs = gi + n, slot = gs % a.nslot;
-          if (mbar_wait(&full[slot], (gs / a.nslot) & 1, abort_flag, a.status)) {
-            const uint32_t m = lmask2[n];
-            const uint4* wr = reinterpret_cast<const uint4*>(ring + (size_t)slot * 4 * d);
-            float u[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) u[t] = 0.f;
-            const int v0 = q * nv / RW_WPN, v1 = (q + 1) * nv / RW_WPN;
-            for (int v = v0 + lane; v < v1; v += 32) {
-              float w[8];
-              bf16x8_to_f32(wr[v], w);
-#pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                if ((m >> t) & 1u) {
-                  float xv[8];
-                  bf16x8_to_f32(reinterpret_cast<const uint4*>(xs + (size_t)t * d)[v], xv);
-#pragma unroll
-                  for (int k = 0; k < 8; ++k) u[t] = fmaf(w[k], xv[k], u[t]);
-                }
-              }
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              if ((m >> t) & 1u) {
-                float r = u[t];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
-                if (lane == 0) part[((n - i0) * RW_WPN + q) * 8 + t] = r;
-              }
-            }
-          }
-        }
-      }
-      __syncthreads();
-      // down: every thread owns 8 columns for the 8 tokens
-      const int nb = min(RW_NB, L2 - i0);
-      for (int nn = 0; nn < nb; ++nn) {
-        const int n = i0 + nn, gs = gi + n, slot = gs % a.nslot;
-        if (!mbar_wait(&full[slot], (gs / a.nslot) & 1, abort_flag, a.status)) break;
-        const uint32_t m = lmask2[n];
-        float h[8];
-        float vf[8];
-        bf16x8_to_f32(lval2[n], vf);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          float uu = 0.f;
-          if ((m >> t) & 1u) {
-#pragma unroll
-            for (int q = 0; q < RW_WPN; ++q) uu += part[(nn * RW_WPN + q) * 8 + t];
-          }
-          h[t] = vf[t] * uu;
-        }
-        if (tid < nv) {
-          const uint4* wr = reinterpret_cast<const uint4*>(ring + (size_t)slot * 4 * d + row_bytes);
-          float w[8];
-          bf16x8_to_f32(wr[tid], w);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            if ((m >> t) & 1u) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) acc[t][k] = fmaf(h[t], w[k], acc[t][k]);
-            }
-          }
-        }
-      }
-      __syncthreads();
-      // the batch's slots are free: refill them with the entries nslot ahead
-      if (tid == 0 && !*abort_flag) {
-        for (int nn = 0; nn < nb; ++nn) {
-          const int i = i0 + nn + a.nslot;
-          if (i < L2) issue(i);
-        }
-      }
-    }
-    gi += L2;
-    __syncthreads();
-    if (*abort_flag) break;
-  }
-  // drain any copies still in flight (only after an abort)
-  if (tid == 0 && *abort_flag) {
-    for (int k = 0; k < a.nslot && k < gi; ++k) {
-      const int last = gi - 1 - k;
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&full[last % a.nslot], (last / a.nslot) & 1)) {
-        if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) break;
-      }
-    }
-  }
-  // 4. write the block's partial y
-  if (tid < nv && !*abort_flag) {
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      if ((live >> t) & 1u) {
-        float4* dst = reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d + tid * 8);
-        const float4 v0 = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
-        const float4 v1 = make_float4(acc[t][4], acc[t][5], acc[t][6], acc[t][7]);
-        if (a.atomic) {
-          atomicAdd(dst, v0);
-          atomicAdd(dst + 1, v1);
-        } else {
-          dst[0] = v0;
-          dst[1] = v1;
-        }
-      }
     }
   }
 }

@@ -93,10 +93,21 @@ def test_single_heavy_token_overflows():
 
 
 def test_ragged_dims_and_threshold():
-    # d not a multiple of 64 (ragged K block), a positive threshold, one tile
-    inp = synth.make_inputs(small(tokens=11, d_model=200, d_ff=128, threshold=0.25))
-    check(inp, path="rows")
+    # d not a multiple of 64 (ragged K block of the gate), a positive threshold, one tile
+    inp = synth.make_inputs(small(tokens=11, d_model=208, d_ff=128, threshold=0.25))
     check(inp, path="tiles")
+    inp = synth.make_inputs(small(tokens=11, d_model=768, d_ff=128, threshold=0.25))
+    check(inp, path="rows")
+
+
+def test_row_path_shape_rule():
+    # the fused row kernel needs d % 256 == 0; AUTO then takes the tile path
+    inp = synth.make_inputs(small(tokens=6, d_model=200, d_ff=256))
+    st = check(inp)
+    assert st["path"] == SFFN_PATH_TILES
+    from activation_sparse_gated_relu_b200 import SffnError
+    with pytest.raises(SffnError):
+        check(inp, path="rows")
 
 
 def test_silu_threshold_and_no_bias():
