@@ -20,6 +20,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -912,3 +913,142 @@ sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free low-rank gate -> TwELL.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// gate: code embedded in a runtime that owns all device memory (a serving
+// engine with a pre-planned pool, a plugin host that hands out fixed buffers)
+// and code on a latency-critical path, where cudaMalloc may synchronise the
+// device or fail when memory is reserved or fragmented.  For them this entry
+// point computes z = bf16(x·A) and the TwELL records of sigma(z·B + b) with
+// the same kernels as sffn_forward, but keeps its scratch (the split-K fp32
+// accumulator of z, its per-tile tickets, z itself and a status word) in
+// file-scope device arrays of fixed size that every GPU loading this library
+// holds until the process exits.  It calls no allocator: inputs and outputs
+// come from the caller.
+namespace {
+
+constexpr int kNaMaxT = 64, kNaMaxD = 4096, kNaMaxR = 1024, kNaMaxF = 16384;
+constexpr int kNaTickets = (kNaMaxR / 128) * (kNaMaxT / 16);
+
+static __device__ __align__(256) float g_na_zacc[kNaMaxT * kNaMaxR];
+static __device__ __align__(256) __nv_bfloat16 g_na_z[kNaMaxT * kNaMaxR];
+static __device__ __align__(256) int g_na_tickets[kNaTickets];
+static __device__ __align__(256) uint32_t g_na_status[4];
+
+struct NaScratch {
+  float* zacc = nullptr;
+  __nv_bfloat16* z = nullptr;
+  int* tickets = nullptr;
+  uint32_t* status = nullptr;
+  bool ready = false;
+};
+constexpr int kNaMaxDevices = 64;
+NaScratch g_na_dev[kNaMaxDevices];
+std::mutex g_na_mu;
+
+// Device addresses of the scratch arrays for the current device (looked up
+// once per device; the host-side names of the arrays are not device addresses).
+sffn_status na_setup(int dev, NaScratch** out) {
+  if (dev < 0 || dev >= kNaMaxDevices) return SFFN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_na_mu);
+  NaScratch& s = g_na_dev[dev];
+  if (!s.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_na_zacc) != cudaSuccess) goto fail;
+    s.zacc = static_cast<float*>(p);
+    if (cudaGetSymbolAddress(&p, g_na_z) != cudaSuccess) goto fail;
+    s.z = static_cast<__nv_bfloat16*>(p);
+    if (cudaGetSymbolAddress(&p, g_na_tickets) != cudaSuccess) goto fail;
+    s.tickets = static_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, g_na_status) != cudaSuccess) goto fail;
+    s.status = static_cast<uint32_t*>(p);
+    if (set_tc_attrs<EpiLowRankZ>() != cudaSuccess || set_tc_attrs<EpiGateTwell>() != cudaSuccess) goto fail;
+    s.ready = true;
+  }
+  *out = &s;
+  return SFFN_OK;
+fail:
+  cudaGetLastError();
+  return SFFN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_model, const void* A_t, int rank,
+                                                  const void* B_t, int d_ff, const float* gate_bias, int act,
+                                                  float threshold, int tile_capacity, int16_t* count, int16_t* idx,
+                                                  void* val, uint32_t* overflow, void* cuda_stream) {
+  if (!x || !A_t || !B_t || !count || !idx || !val || !overflow) return SFFN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(A_t) || !aligned16(B_t)) return SFFN_ERR_INVALID_ARG;
+  if (gate_bias && (reinterpret_cast<uintptr_t>(gate_bias) & 3u)) return SFFN_ERR_INVALID_ARG;
+  if (act != SFFN_ACT_RELU && act != SFFN_ACT_SILU) return SFFN_ERR_INVALID_ARG;
+  if (!(threshold >= 0.0f) || !std::isfinite(threshold)) return SFFN_ERR_INVALID_ARG;
+  const int C = tile_capacity;
+  if (C != 8 && C != 16 && C != 32 && C != 64 && C != 128) return SFFN_ERR_INVALID_ARG;
+  if (T < 0 || d_model <= 0 || rank <= 0 || d_ff <= 0) return SFFN_ERR_INVALID_ARG;
+  if (T == 0) return SFFN_OK;
+  // the scratch arrays bound the problem size
+  if (T > kNaMaxT || d_model > kNaMaxD || rank > kNaMaxR || d_ff > kNaMaxF) return SFFN_ERR_UNSUPPORTED;
+  if (d_model % 8 != 0 || rank % 64 != 0 || d_ff % 128 != 0) return SFFN_ERR_UNSUPPORTED;
+  int dev = 0, major = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_NO_DEVICE;
+  }
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10) return SFFN_ERR_NO_DEVICE;
+  NaScratch* sc = nullptr;
+  sffn_status ss = na_setup(dev, &sc);
+  if (ss != SFFN_OK) return ss;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const int P = d_ff / 128, BN = pick_bn(T), ntile = cdiv(T, BN), mt = cdiv(rank, 128);
+  const int sk = std::max(1, std::min(cdiv(d_model, 64), cdiv(nsm > 0 ? nsm : kNumSMsFallback, mt * ntile)));
+  // the split-K accumulator, the tickets and the caller's overflow flags start at zero
+  cudaError_t e = cudaMemsetAsync(sc->zacc, 0, (size_t)T * rank * sizeof(float), st);
+  e = e ? e : cudaMemsetAsync(sc->tickets, 0, sizeof(int) * kNaTickets, st);
+  e = e ? e : cudaMemsetAsync(overflow, 0, (size_t)T * sizeof(uint32_t), st);
+  if (e) {
+    cudaGetLastError();
+    return SFFN_ERR_CUDA;
+  }
+  CUtensorMap mAt, mx, mBt, mz;
+  if (!make_map(&mAt, A_t, d_model, rank, 128) || !make_map(&mx, x, d_model, T, BN) ||
+      !make_map(&mBt, B_t, rank, d_ff, 128) || !make_map(&mz, sc->z, rank, T, BN))
+    return SFFN_ERR_CUDA;
+  TcArgs za{};
+  za.n_phase = 1;
+  za.kb_total[0] = cdiv(d_model, 64);
+  za.n_rows = T;
+  za.status = sc->status;
+  ZParams zp{T, rank, sk, sc->zacc, sc->z, sc->tickets};
+  if (launch_tc<EpiLowRankZ>(BN, dim3(mt, ntile, sk), st, mAt, mx, mAt, mx, za, zp) != cudaSuccess)
+    return SFFN_ERR_CUDA;
+  TcArgs ga{};
+  ga.n_phase = 1;
+  ga.kb_total[0] = cdiv(rank, 64);
+  ga.n_rows = T;
+  ga.status = sc->status;
+  TwellParams tw;
+  tw.bias = gate_bias;
+  tw.tau = threshold;
+  tw.act = act;
+  tw.T = T;
+  tw.F = d_ff;
+  tw.n_tiles = P;
+  tw.C = C;
+  tw.count = count;
+  tw.idx = idx;
+  tw.val = val;
+  tw.val_f32 = 0;
+  tw.ovf = overflow;
+  tw.epoch = 1;
+  tw.kmask = nullptr;
+  tw.gdebug = nullptr;
+  if (launch_tc<EpiGateTwell>(BN, dim3(P, ntile, 1), st, mBt, mz, mBt, mz, ga, tw) != cudaSuccess)
+    return SFFN_ERR_CUDA;
+  return SFFN_OK;
+}

@@ -185,6 +185,32 @@ sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards);
 sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], float* total_ms,
                             int* launches, int* n_kernels);
 
+/* Allocation-free low-rank gate (no counterpart in the pages: an interface
+ * convenience).  For callers that must not allocate device memory where they
+ * run: code inside a runtime that owns all device memory (a pre-planned pool,
+ * a plugin host with fixed buffers) or on a latency-critical path, where
+ * cudaMalloc can synchronise the device or fail.  It computes the same TwELL
+ * records as the low-rank gate of sffn_forward: z = bf16(x·A), g = z·B + b,
+ * keep iff |sigma(g)| > threshold.  Inputs (device, 16-byte aligned):
+ *   x [T][d_model] bf16; A_t [rank][d_model] bf16 (A transposed);
+ *   B_t [d_ff][rank] bf16 (B transposed); gate_bias [d_ff] fp32 or NULL.
+ * Outputs (device): count [T][d_ff/128] int16, idx [T][d_ff/128][C] int16,
+ *   val [T][d_ff/128][C] bf16 (TwELL as described above), overflow [T]
+ *   uint32: 1 iff the token overflows some tile, else 0.
+ * Limits: T <= 64, d_model <= 4096 (multiple of 8), rank <= 1024 (multiple of
+ * 64), d_ff <= 16384 (multiple of 128); larger sizes return
+ * SFFN_ERR_UNSUPPORTED before anything runs.  Scratch lives in fixed device
+ * arrays inside this library (about 400 KB per GPU, held until the process
+ * exits); the first call on a device looks their addresses up, so make that
+ * call before any stream capture.  Every call shares that scratch and clears
+ * what must start at zero, so calls that overlap on the GPU (two streams, two
+ * threads) race and must be serialised by the caller.  Asynchronous on
+ * cuda_stream; no allocation, no host synchronisation. */
+sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_model, const void* A_t, int rank,
+                                       const void* B_t, int d_ff, const float* gate_bias, int act,
+                                       float threshold, int tile_capacity, int16_t* count, int16_t* idx,
+                                       void* val, uint32_t* overflow, void* cuda_stream);
+
 /* Library version string. */
 const char* sffn_version(void);
 
