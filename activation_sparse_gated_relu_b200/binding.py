@@ -79,7 +79,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_debug_norms.restype = st
     lib.sffn_get_stats.argtypes = [vp, vp, ctypes.POINTER(sffn_stats)]
     lib.sffn_get_stats.restype = st
-    lib.sffn_timing_begin.argtypes = [vp, ip]
+    lib.sffn_timing_begin.argtypes = [vp, ip, ip]
     lib.sffn_timing_begin.restype = st
     lib.sffn_timing_end.argtypes = [vp, ip, vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ip),
                                     ctypes.POINTER(ip)]
@@ -132,8 +132,8 @@ def sffn_get_stats(h, stream: int = 0) -> sffn_stats:
     return st
 
 
-def sffn_timing_begin(h, max_forwards: int) -> None:
-    _check(load_library().sffn_timing_begin(h, int(max_forwards)), "sffn_timing_begin")
+def sffn_timing_begin(h, max_forwards: int, stride: int = 1) -> None:
+    _check(load_library().sffn_timing_begin(h, int(max_forwards), int(stride)), "sffn_timing_begin")
 
 
 def sffn_timing_end(h) -> dict:
@@ -262,8 +262,8 @@ class SparseFFN:
     def stats(self, stream: Optional[int] = None) -> sffn_stats:
         return sffn_get_stats(self.h, self._stream(stream))
 
-    def timing_begin(self, max_forwards: int) -> None:
-        sffn_timing_begin(self.h, max_forwards)
+    def timing_begin(self, max_forwards: int, stride: int = 1) -> None:
+        sffn_timing_begin(self.h, max_forwards, stride)
 
     def timing_end(self) -> dict:
         return sffn_timing_end(self.h)

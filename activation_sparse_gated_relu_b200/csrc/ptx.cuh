@@ -207,6 +207,13 @@ __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
   return v;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Wait until the grids this one depends on (launched earlier on the stream)
+// have completed and their writes are visible; a no-op without the launch
+// attribute.  Every kernel calls it before touching data that an earlier
+// kernel writes or reads.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -135,11 +135,12 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = a.n_tiles, b = blockIdx.y, S = gridDim.x, s = blockIdx.x;
   const int tb0 = b * 8;
-  const uint32_t live = a.blk_live[b];
   const int d = a.d;
   const int nchunk = (d + RW_CHUNK - 1) / RW_CHUNK;
   const int spg = 2 * nchunk;        // stages per group: up chunks, then down chunks
 
+  griddep_wait();  // union masks and live masks come from the router
+  const uint32_t live = a.blk_live[b];
   // 1. union masks of the block, barriers
   for (int p = tid; p < P; p += blockDim.x) ums[p] = a.umask[(size_t)b * P + p];
   if (tid == 0) {
@@ -399,8 +400,13 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     const int q0 = (int)(n4 * rank / CS), q1 = (int)(n4 * (rank + 1) / CS);
     const int width = q1 - q0;
     const uint32_t red_s = smem_u32(red);
-    for (int e = tid; e < 8 * width; e += blockDim.x) {
-      const int t = e / width, q = q0 + (e - t * width);
+    // clusters start their slices at different columns, so that at any moment
+    // they add into different L2 lines
+    const int nclu = (int)((gridDim.x * gridDim.y) / CS);
+    const int cid = (int)((blockIdx.y * gridDim.x + blockIdx.x) / CS);
+    const int rot = (int)(((long long)cid * width) / max(1, nclu));
+    for (int e0 = tid; e0 < 8 * width; e0 += blockDim.x) {
+      const int t = e0 / width, q = q0 + (e0 - t * width + rot) % width;
       if (!((live >> t) & 1u)) continue;
       const uint32_t off = (uint32_t)((t * n4 + q) * 16);
       float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);

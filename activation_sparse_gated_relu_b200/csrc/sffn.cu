@@ -81,12 +81,42 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows,
 int pick_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// Launch with programmatic dependent launch: the kernel may be scheduled while
+// the previous kernel on the stream drains; it calls griddepcontrol.wait before
+// touching data an earlier kernel writes or reads.  cluster_x > 1 also sets
+// the thread-block cluster size.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = cluster_x;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
+}
+
 template <int BN, class Epi>
 cudaError_t launch_tc_bn(dim3 grid, cudaStream_t st, const CUtensorMap& a0, const CUtensorMap& b0,
                          const CUtensorMap& a1, const CUtensorMap& b1, const TcArgs& args,
                          const typename Epi::Params& ep) {
-  k_tc_gemm<BN, Epi><<<grid, TC_THREADS, TcCfg<BN>::SMEM, st>>>(a0, b0, a1, b1, args, ep);
-  return cudaGetLastError();
+  return launch_pdl(k_tc_gemm<BN, Epi>, grid, dim3(TC_THREADS), TcCfg<BN>::SMEM, st, 1, a0, b0, a1, b1, args, ep);
 }
 
 template <class Epi>
@@ -159,7 +189,7 @@ struct sffn_handle {
   __nv_bfloat16* zero_row = nullptr;   // 2 KB of zeros: row chunks of padding neurons
   // per-kernel timing (sffn_timing_begin/end)
   bool tm_on = false;
-  int tm_max = 0, tm_n = 0, tm_cur = -1;
+  int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
   std::vector<cudaEvent_t> tm_ev;   // [tm_max][kMaxMarks + 1]
   std::vector<int> tm_lab;          // [tm_max][kMaxMarks]
   std::vector<int> tm_nk;           // [tm_max]
@@ -204,7 +234,7 @@ void tmark(sffn_handle* h, cudaStream_t st, int label) {
 
 void tmark_begin(sffn_handle* h) {
   h->tm_cur = -1;
-  if (h->tm_on && h->tm_n < h->tm_max) {
+  if (h->tm_on && (h->tm_seen++ % h->tm_stride) == 0 && h->tm_n < h->tm_max) {
     h->tm_cur = h->tm_n++;
     h->tm_nk[h->tm_cur] = 0;
   }
@@ -556,9 +586,9 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     if (e) return SFFN_ERR_CUDA;
     TopkArgs ta{h->scores, h->vdense, 0, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
     tmark(h, st, L_WINA_TOPK);
-    k_wina_topk<<<T, 1024, (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st>>>(ta);
     ++launches;
-    if (cudaGetLastError()) return SFFN_ERR_CUDA;
+    if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st, 1, ta))
+      return SFFN_ERR_CUDA;
   } else {
     tmark(h, st, L_GATE);
     e = launch_tc<EpiGateTwell>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, tw);
@@ -588,9 +618,9 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   ra.zero_mode = (!rows || rows_split > 1) ? 1 : (sk_down > 1 ? 2 : 0);
   const int router_ctas = std::max(1, std::min(h->n_sm, cdiv((long long)T * d / 4, 4096)));
   tmark(h, st, L_ROUTER);
-  k_router<<<router_ctas, 1024, (size_t)router_smem_bytes(T), st>>>(ra);
   ++launches;
-  if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_router, dim3(router_ctas), dim3(1024), (size_t)router_smem_bytes(T), st, 1, ra))
+    return SFFN_ERR_CUDA;
 
   // ------------------------------------------ non-overflow tokens
   if (rows) {
@@ -615,23 +645,9 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     rw.lcap = h->rows_lcap;
     rw.status = h->status;
     tmark(h, st, L_UPDOWN_ROWS);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(rows_split, nblk, 1);
-    cfg.blockDim = dim3(RW_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = h->rows_smem;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = rows_cs;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = rows_cs > 1 ? 1 : 0;
     ++launches;
-    if (cudaLaunchKernelEx(&cfg, k_rows, rw) != cudaSuccess) {
-      cudaGetLastError();
+    if (launch_pdl(k_rows, dim3(rows_split, nblk, 1), dim3(RW_THREADS), (size_t)h->rows_smem, st, rows_cs, rw))
       return SFFN_ERR_CUDA;
-    }
   } else {
     TcArgs ua{};
     ua.n_phase = 1;
@@ -728,15 +744,14 @@ static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out,
   ga.tw.gdebug = h->gdebug;
   ga.wp = WinaParams{D.gate_bias, D.act, T, F, h->norms, h->vdense, 1, h->scores};
   tmark(h, st, L_GATE_F32);
-  k_gate_f32<<<dim3(P, cdiv(T, 16)), 128, 0, st>>>(ga);
   ++launches;
-  if (cudaGetLastError()) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_gate_f32, dim3(P, cdiv(T, 16)), dim3(128), 0, st, 1, ga)) return SFFN_ERR_CUDA;
   if (h->wina) {
     TopkArgs ta{h->scores, h->vdense, 1, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
     tmark(h, st, L_WINA_TOPK);
-    k_wina_topk<<<T, 1024, (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st>>>(ta);
     ++launches;
-    if (cudaGetLastError()) return SFFN_ERR_CUDA;
+    if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st, 1, ta))
+      return SFFN_ERR_CUDA;
   }
   RouterArgs ra{};
   ra.T = T;
@@ -747,22 +762,21 @@ static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out,
   ra.blk_live = h->blk_live;
   ra.zero_mode = 0;
   tmark(h, st, L_ROUTER);
-  k_router<<<1, 1024, (size_t)router_smem_bytes(T), st>>>(ra);
   ++launches;
+  if (launch_pdl(k_router, dim3(1), dim3(1024), (size_t)router_smem_bytes(T), st, 1, ra)) return SFFN_ERR_CUDA;
   RowsF32Args rf{static_cast<const float*>(x), static_cast<const float*>(D.W_up), static_cast<const float*>(D.W_down),
                  h->count, h->idx, static_cast<const float*>(h->val), h->ovf, epoch, out, T, d, P, h->C};
   tmark(h, st, L_ROWS_F32);
-  k_rows_f32<<<T, 256, (size_t)(d + 2 * P * h->C) * 4, st>>>(rf);
   ++launches;
+  if (launch_pdl(k_rows_f32, dim3(T), dim3(256), (size_t)(d + 2 * P * h->C) * 4, st, 1, rf)) return SFFN_ERR_CUDA;
   if (!h->wina) {
     FallbackF32Args fa{static_cast<const float*>(x), static_cast<const float*>(D.W_gate),
                        static_cast<const float*>(D.W_up), static_cast<const float*>(D.W_down), D.gate_bias,
                        D.threshold, D.act, h->ovf_list, h->ovf_count, out, d, F};
     tmark(h, st, L_FALLBACK_F32);
-    k_fallback_f32<<<T, 256, (size_t)(d + F) * 4, st>>>(fa);
     ++launches;
+    if (launch_pdl(k_fallback_f32, dim3(T), dim3(256), (size_t)(d + F) * 4, st, 1, fa)) return SFFN_ERR_CUDA;
   }
-  if (cudaGetLastError()) return SFFN_ERR_CUDA;
   h->last_path = SFFN_PATH_ROWS;
   h->last_launches = launches;
   return SFFN_OK;
@@ -783,9 +797,11 @@ sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void*
   return r;
 }
 
-sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards) {
-  if (!h || max_forwards <= 0 || max_forwards > 100000) return SFFN_ERR_INVALID_ARG;
+sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards, int stride) {
+  if (!h || max_forwards <= 0 || max_forwards > 100000 || stride <= 0) return SFFN_ERR_INVALID_ARG;
   timing_free(h);
+  h->tm_stride = stride;
+  h->tm_seen = 0;
   const size_t nev = (size_t)max_forwards * (kMaxMarks + 1);
   h->tm_ev.assign(nev, nullptr);
   for (size_t i = 0; i < nev; ++i) {

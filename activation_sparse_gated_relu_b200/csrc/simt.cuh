@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
   extern __shared__ int rs_list[];   // [T] overflow list, then [ceil(T/32)] overflow bits
   uint32_t* obits = reinterpret_cast<uint32_t*>(rs_list + a.T);
   __shared__ int scan_tmp[33];
+  griddep_wait();
   int base = 0;
   for (int c = 0; c < a.T; c += blockDim.x) {
     const int t = c + threadIdx.x;
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
   int* eqpre = reinterpret_cast<int*>(hist + 32 * 256);
   __shared__ int scan_tmp[33];
   __shared__ uint32_t sel[4];  // prefix, remaining
+  griddep_wait();
   const int t = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* sc = a.scores + (size_t)t * a.F;
@@ -275,6 +277,7 @@ struct GateF32Args {
 __global__ void __launch_bounds__(128) k_gate_f32(const GateF32Args a) {
   __shared__ __align__(16) float xs[16][256];
   __shared__ uint32_t masks[2][64];
+  griddep_wait();
   const int p = blockIdx.x, t0 = blockIdx.y * 16;
   const int etid = threadIdx.x, j = p * 128 + etid;
   const int T = a.wina ? a.wp.T : a.tw.T;
@@ -321,6 +324,7 @@ struct RowsF32Args {
 
 __global__ void __launch_bounds__(256) k_rows_f32(const RowsF32Args a) {
   extern __shared__ float rf_smem[];   // xs[d], then hj[cap], then jj[cap] (int)
+  griddep_wait();
   const int t = blockIdx.x;
   if (t >= a.T || a.ovf[t] == a.epoch) return;
   const int cap = a.n_tiles * a.C;
@@ -383,6 +387,7 @@ struct FallbackF32Args {
 
 __global__ void __launch_bounds__(256) k_fallback_f32(const FallbackF32Args a) {
   extern __shared__ float ff_smem[];   // xs[d], h[F]
+  griddep_wait();
   const int o = blockIdx.x;
   if (o >= *a.ovf_count) return;
   const int t = a.ovf_list[o];

@@ -61,6 +61,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
 
   const int m0 = blockIdx.x * TC_BM;
   const int n0 = blockIdx.y * BN;
+  if (args.n_rows_dev) griddep_wait();  // the row count comes from an earlier kernel
   const int n_rows = args.n_rows_dev ? *args.n_rows_dev : args.n_rows;
   if (n0 >= n_rows) return;  // uniform: the whole CTA leaves before any setup
 
@@ -103,6 +104,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // inputs and outputs may belong to earlier kernels on the stream
 
   const int S = gridDim.z, sk = blockIdx.z;
 

@@ -172,10 +172,11 @@ typedef struct sffn_stats {
 sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st);
 
 /* Per-kernel device timing (bench use).  Between sffn_timing_begin and
- * sffn_timing_end every forward records a CUDA event on its own stream before
- * each kernel launch and after the last one; no work is skipped or added.
- * max_forwards bounds the forwards recorded (later ones are not timed). */
-sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards);
+ * sffn_timing_end every stride-th forward records a CUDA event on its own
+ * stream before each kernel launch and after the last one; no work is skipped
+ * or added.  max_forwards bounds the forwards recorded (later ones are not
+ * timed). */
+sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards, int stride);
 
 /* Synchronise the recorded events and report, per kernel label (a short
  * name such as "gate" or "updown_rows", NUL-terminated, at most 31 chars), the

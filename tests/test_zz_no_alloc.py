@@ -93,7 +93,12 @@ def test_noalloc_matches_forward_gaussian_within_band():
         count, idx, val, ovf = _call(f, inp, T, C)
         same = (count == ref.count) & (idx == ref.idx).all(-1)
         assert np.all(same | amb_tile)
-        close = np.abs(val - ref.val) <= 2.0 ** -7 * np.abs(ref.val)
+        # same tolerance as the parity tests: one rounding of the stored bf16
+        # value plus twice the gate's decision band at that neuron (z is summed
+        # with split-K atomics, so a z coordinate at a bf16 rounding midpoint
+        # may round either way between two runs)
+        band = res.band[np.arange(T)[:, None, None], np.maximum(ref.idx, 0)]
+        close = np.abs(val - ref.val) <= 2.0 ** -7 * np.abs(ref.val) + 2 * band
         assert np.all(close.all(-1) | amb_tile)
 
 
