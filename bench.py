@@ -44,7 +44,7 @@ TIMING_STRIDE = 8
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {
     "gate": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
-    "updown_rows": ["simt.cuh", "ptx.cuh"],
+    "updown_rows": ["rows_mma.cuh", "ptx.cuh"],
 }
 
 
