@@ -109,6 +109,65 @@ struct EpiGateTwell {
   }
 };
 
+// Stream-K gate: a tile whose K blocks are shared by n_pieces CTAs.  Each
+// CTA stores its fp32 partial of the 128 x BN tile in its piece slot, and the
+// CTA that completes the tile's ticket adds the pieces in ascending K order
+// (the same order on every forward, so the sum is reproducible) and emits
+// TwELL from the sum.  A tile held by one CTA goes straight to TwELL.
+constexpr int SK_MAX_PIECES = 4;  // CTAs that may share one tile
+
+struct GateSKParams {
+  TwellParams tw;
+  float* part;   // [tiles x token tiles][SK_MAX_PIECES][BN][128] fp32
+  int* tick;     // [tiles x token tiles], zero between forwards
+};
+
+struct EpiGateTwellSK {
+  static constexpr int N_ACC = 2;  // a CTA's range touches at most two tiles
+  static constexpr bool STREAMK = true;
+  using Params = GateSKParams;
+  template <int BN>
+  __device__ static void run_piece(const Params& o, uint32_t tmem, int m0, int n0, int piece, int n_pieces,
+                                   int etid, uint8_t* scratch) {
+    if (n_pieces == 1) {
+      named_bar_sync(1, 128);  // an earlier piece's threads are done with the masks
+      EpiGateTwell::run<BN>(o.tw, tmem, m0, n0, 0, etid, scratch);
+      return;
+    }
+    const int slot = (m0 >> 7) * (int)gridDim.y + (int)blockIdx.y;
+    float* base = o.part + (size_t)slot * SK_MAX_PIECES * BN * 128;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.tw.T) break;
+      float g[16];
+      tmem_ld16(tmem + c, g);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) __stcg(&base[((size_t)piece * BN + c + i) * 128 + etid], g[i]);
+    }
+    int* last = reinterpret_cast<int*>(scratch + 1024);
+    __threadfence();
+    named_bar_sync(1, 128);
+    if (etid == 0) *last = atomicAdd(&o.tick[slot], 1) == n_pieces - 1;
+    named_bar_sync(1, 128);
+    if (!*last) return;
+    __threadfence();
+    uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.tw.T) break;
+      float g[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) g[i] = __ldcg(&base[(size_t)(c + i) * 128 + etid]);
+      for (int q = 1; q < n_pieces; ++q) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) g[i] += __ldcg(&base[((size_t)q * BN + c + i) * 128 + etid]);
+      }
+      twell_chunk(o.tw, g, m0 + etid, n0 + c, etid, masks + ((c >> 4) & 1) * 64);
+    }
+    if (etid == 0) o.tick[slot] = 0;
+  }
+};
+
 // ------------------------------------------------------------------- WINA
 // Dense activation and score for the per-token top-k: v = round(sigma(g+b)),
 // s = |sigma(g+b)|·n_j, both [T][F].

@@ -3,8 +3,10 @@
 // stores h in global memory).
 //
 // One CTA (16 warps) takes a block of 8 tokens and a contiguous range of the
-// block's union of kept neurons, ranked tile by tile from the router's union
-// masks, so that every CTA streams the same number of rows.  Neurons are
+// block's union of kept neurons, ranked tile by tile from the union of the
+// live (non-overflow) tokens' keep masks, so that every CTA streams the same
+// number of rows.  CTA 0 of each block also routes the block's overflow
+// tokens to the dense channel (list, count, gathered rows).  Neurons are
 // processed in groups of 16.  A group's W_up rows and then its W_down rows
 // (contiguous, neuron-major) pass through a ring of shared-memory stages, one
 // stage = the same 1024-column chunk of the 16 rows (16 KB... 32 KB), each
@@ -27,8 +29,8 @@
 //         the whole CTA.
 // At the end the per-CTA partial y goes to out: plain stores when one CTA
 // owns the block, otherwise summed over the CTAs of a thread-block cluster
-// through distributed shared memory and added with vector atomics (each CTA
-// of the cluster owns one column slice).
+// through distributed shared memory (each CTA of the cluster owns one column
+// slice) and added into out by bulk reduce-add copies, one per live token.
 #pragma once
 
 #include "ptx.cuh"
@@ -52,8 +54,17 @@ struct RowsArgs {
   const int16_t* count;
   const int16_t* idx;
   const __nv_bfloat16* val;
-  const uint4* umask;        // [n_blk][n_tiles] 128-bit union masks (live tokens only)
-  const uint8_t* blk_live;
+  const uint4* kmask;        // [T][n_tiles] 128-bit keep masks from the gate epilogue
+  const uint32_t* ovf;       // [T] overflow epochs
+  uint32_t epoch;
+  // overflow routing (CTA 0 of every block): compacted list, count, gathered rows
+  int* ovf_list;
+  int* ovf_count;
+  uint4* xo;                 // [T][d / 8] gathered x rows of overflow tokens
+  const uint4* z;            // low-rank z rows to gather (or null)
+  uint4* zo;
+  int r_vec;
+  int zero_ovf_rows;         // zero out's rows of overflow tokens (split down adds into them)
   float* out;
   int T, d, F, n_tiles, C;
   int atomic;
@@ -139,14 +150,50 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   const int nchunk = (d + RW_CHUNK - 1) / RW_CHUNK;
   const int spg = 2 * nchunk;        // stages per group: up chunks, then down chunks
 
-  griddep_wait();  // union masks and live masks come from the router
-  const uint32_t live = a.blk_live[b];
-  // 1. union masks of the block, barriers
-  for (int p = tid; p < P; p += blockDim.x) ums[p] = a.umask[(size_t)b * P + p];
-  if (tid == 0) {
-    for (int i = 0; i < RW_NS; ++i) mbar_init(&full[i], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
+  griddep_wait();  // keep masks, TwELL and overflow epochs come from the gate
+  // 1. live tokens of the block (valid, not overflowing) and the union of
+  // their keep masks, tile by tile; barriers
+  uint4 km[8];
+  if (tid < P) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      km[i] = tb0 + i < a.T ? a.kmask[(size_t)(tb0 + i) * P + tid] : make_uint4(0, 0, 0, 0);
+  }
+  if (warp == 0) {
+    const int t = tb0 + lane;
+    const bool v = lane < 8 && t < a.T;
+    const bool o = v && a.ovf[t] == a.epoch;
+    const uint32_t vb = __ballot_sync(0xFFFFFFFFu, v), obb = __ballot_sync(0xFFFFFFFFu, o);
+    if (lane == 0) {
+      misc[50] = (int)(vb & ~obb);
+      misc[51] = (int)obb;
+      misc[52] = 0;
+      for (int i = 0; i < RW_NS; ++i) mbar_init(&full[i], 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+  }
+  __syncthreads();
+  const uint32_t live = (uint32_t)misc[50], obits = (uint32_t)misc[51];
+  if (tid < P) {
+    uint4 u = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((live >> i) & 1u) {
+        u.x |= km[i].x;
+        u.y |= km[i].y;
+        u.z |= km[i].z;
+        u.w |= km[i].w;
+      }
+    ums[tid] = u;
+  }
+  // overflow routing ([TwELL] hybrid): CTA 0 of the block ranks the block's
+  // overflow tokens after those of earlier blocks, lists them and gathers
+  // their rows for the dense channel; the last block writes the count
+  if (s == 0) {
+    int before = 0;
+    for (int t = tid; t < tb0; t += blockDim.x) before += a.ovf[t] == a.epoch ? 1 : 0;
+    if (before) atomicAdd(&misc[52], before);
   }
   // x^T fragments of this warp's k steps (16(w + 16 j) in every chunk), in
   // registers; zero beyond T
@@ -167,6 +214,25 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       }
   }
   __syncthreads();
+  if (s == 0 && (obits != 0u || b == (int)gridDim.y - 1)) {
+    const int base = misc[52];
+    if (b == (int)gridDim.y - 1 && tid == 0) *a.ovf_count = base + __popc(obits);
+    const int dv = d >> 3, d4 = d >> 2;
+    int o = base;
+    for (int i = 0; i < 8; ++i) {
+      if (!((obits >> i) & 1u)) continue;
+      const int t = tb0 + i;
+      if (tid == 0) a.ovf_list[o] = t;
+      const uint4* xr = reinterpret_cast<const uint4*>(a.x) + (size_t)t * dv;
+      for (int v = tid; v < dv; v += blockDim.x) a.xo[(size_t)o * dv + v] = xr[v];
+      if (a.z)
+        for (int v = tid; v < a.r_vec; v += blockDim.x) a.zo[(size_t)o * a.r_vec + v] = a.z[(size_t)t * a.r_vec + v];
+      if (a.zero_ovf_rows)
+        for (int v = tid; v < d4; v += blockDim.x)
+          reinterpret_cast<float4*>(a.out)[(size_t)t * d4 + v] = make_float4(0.f, 0.f, 0.f, 0.f);
+      ++o;
+    }
+  }
   // 2. exclusive prefix of the tile union counts
   if (warp == 0) {
     int run = 0;
@@ -395,18 +461,17 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   const uint32_t CS = cluster_nctarank();
   const int n4 = d >> 2;
   if (a.atomic && CS > 1) {
+    // the cluster's CTAs sum their partials over distributed shared memory,
+    // each one column slice, into a slice buffer behind red; the bulk-copy
+    // engine then adds each live token's slice row into out at L2
     cluster_sync();
     const uint32_t rank = cluster_ctarank();
     const int q0 = (int)(n4 * rank / CS), q1 = (int)(n4 * (rank + 1) / CS);
     const int width = q1 - q0;
     const uint32_t red_s = smem_u32(red);
-    // clusters start their slices at different columns, so that at any moment
-    // they add into different L2 lines
-    const int nclu = (int)((gridDim.x * gridDim.y) / CS);
-    const int cid = (int)((blockIdx.y * gridDim.x + blockIdx.x) / CS);
-    const int rot = (int)(((long long)cid * width) / max(1, nclu));
+    float4* slice = reinterpret_cast<float4*>(red + 8 * d);
     for (int e0 = tid; e0 < 8 * width; e0 += blockDim.x) {
-      const int t = e0 / width, q = q0 + (e0 - t * width + rot) % width;
+      const int t = e0 / width, q = q0 + (e0 - t * width);
       if (!((live >> t) & 1u)) continue;
       const uint32_t off = (uint32_t)((t * n4 + q) * 16);
       float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -414,20 +479,30 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
         const float4 v = ld_shared_cluster_f4(mapa_shared(red_s + off, r));
         sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
       }
-      if (okall) atomicAdd(reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d) + q, sum);
+      slice[e0] = sum;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid < 8 && ((live >> tid) & 1u) && okall) {
+      bulk_reduce_add_f32(a.out + (size_t)(tb0 + tid) * d + 4 * q0, slice + tid * width, (uint32_t)width * 16u);
+      bulk_commit();
+      bulk_wait_all();
     }
     cluster_sync();
+  } else if (a.atomic) {
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid < 8 && ((live >> tid) & 1u) && okall) {
+      bulk_reduce_add_f32(a.out + (size_t)(tb0 + tid) * d, red + tid * d, (uint32_t)d * 4u);
+      bulk_commit();
+      bulk_wait_all();
+    }
   } else {
     __syncthreads();
     for (int e = tid; e < 8 * n4; e += blockDim.x) {
       const int t = e / n4, q = e - t * n4;
       if (!((live >> t) & 1u) || !okall) continue;
-      const float4 v = reinterpret_cast<const float4*>(red)[t * n4 + q];
-      float4* dst = reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d) + q;
-      if (a.atomic)
-        atomicAdd(dst, v);
-      else
-        *dst = v;
+      reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d)[q] = reinterpret_cast<const float4*>(red)[t * n4 + q];
     }
   }
 }

@@ -5,9 +5,11 @@
 //   gate    tensor-core tile kernel, epilogue = TwELL emission (threshold) or
 //           dense value + score (WINA, then the top-k kernel emits TwELL);
 //           low-rank gate = two tile kernels (z = bf16(x·A) split over K, then
-//           g = z·B with the TwELL epilogue)
-//   router  overflow list, per-block live masks, gathers, output zeroing
-//   ROWS    fused SIMT up x down over the kept rows (non-overflow tokens)
+//           g = z·B with the TwELL epilogue, stream-K over the SMs)
+//   router  (TILES only) overflow list, gathers, output zeroing
+//   ROWS    fused up x down over the kept rows of each 8-token block
+//           (non-overflow tokens; the kernel also routes the overflow tokens,
+//           and the gate zeroes out when the kernel adds partial sums into it)
 //   TILES   tensor-core u per tile with h from TwELL (non-overflow tokens)
 //   dense   tensor-core recompute of g and u for overflow tokens -> h
 //   down    tensor-core y = h·W_down for the h rows (overflow rows on ROWS,
@@ -80,6 +82,25 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows,
 
 int pick_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Stream-K grid for a GEMM of m_tiles tiles x kb K blocks: the largest CTA
+// count up to n_sm (and above m_tiles) whose ranges hold at most kb units, so
+// that a CTA touches at most two tiles, and that splits no tile over more
+// than max_pieces CTAs.  0 if there is none.
+int streamk_grid(int m_tiles, int kb, int n_sm, int max_pieces) {
+  const long long U = (long long)m_tiles * kb;
+  for (int G = n_sm; G > m_tiles; --G) {
+    if (U < G || cdiv(U, G) > kb) continue;
+    bool ok = true;
+    for (int p = 0; p < m_tiles && ok; ++p) {
+      const int sa = streamk_owner((long long)p * kb, U, G);
+      const int sb = streamk_owner((long long)p * kb + kb - 1, U, G);
+      ok = sb - sa + 1 <= max_pieces;
+    }
+    if (ok) return G;
+  }
+  return 0;
+}
 
 // Launch with programmatic dependent launch: the kernel may be scheduled while
 // the previous kernel on the stream drains; it calls griddepcontrol.wait before
@@ -158,11 +179,9 @@ struct sffn_handle {
   int16_t* idx = nullptr;
   void* val = nullptr;
   uint32_t* ovf = nullptr;
-  uint32_t* umask = nullptr;
   uint32_t* kmask = nullptr;
   int* ovf_list = nullptr;
   int* ovf_count = nullptr;
-  uint8_t* blk_live = nullptr;
   __nv_bfloat16* xo = nullptr;
   __nv_bfloat16* h_hi = nullptr;
   __nv_bfloat16* h_lo = nullptr;
@@ -187,6 +206,10 @@ struct sffn_handle {
   int rows_cs = 1, rows_max_ctas = 0;  // cluster size of the split fused kernel, co-resident CTAs
   bool rows_ok = false;                // the fused row kernel supports this shape
   __nv_bfloat16* zero_row = nullptr;   // 2 KB of zeros: row chunks of padding neurons
+  // stream-K gate (fewer neuron tiles than SMs, T <= 64): CTA count, partials, tickets
+  int sk_grid = 0, sk_bn = 0;
+  float* skpart = nullptr;
+  int* sktick = nullptr;
   // per-kernel timing (sffn_timing_begin/end)
   bool tm_on = false;
   int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
@@ -202,10 +225,10 @@ void timing_free(sffn_handle* h);
 void free_handle(sffn_handle* h) {
   if (!h) return;
   timing_free(h);
-  void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->umask, h->kmask, h->ovf_list, h->ovf_count, h->blk_live,
+  void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zacc,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->zero_row};
+                  h->zero_row, h->skpart, h->sktick};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -340,17 +363,14 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   h->wina = desc->mode == SFFN_MODE_WINA_TOPK;
   h->lowrank = desc->rank > 0;
   const size_t T = (size_t)h->maxT, d = (size_t)h->d, F = (size_t)h->F, P = (size_t)h->P, C = (size_t)h->C;
-  const size_t nblk = (T + 7) / 8;
   bool ok = true;
   ok = ok && dalloc(&h->count, T * P * 2);
   ok = ok && dalloc(&h->idx, T * P * C * 2);
   ok = ok && dalloc(&h->val, T * P * C * h->esize);
   ok = ok && dalloc(&h->ovf, T * 4);
-  ok = ok && dalloc(&h->umask, nblk * P * 16);
   ok = ok && dalloc(&h->kmask, T * P * 16);
   ok = ok && dalloc(&h->ovf_list, T * 4);
   ok = ok && dalloc(&h->ovf_count, 16);
-  ok = ok && dalloc(&h->blk_live, nblk);
   ok = ok && dalloc(&h->status, 16);
   ok = ok && dalloc(&h->xstage, T * d * h->esize);
   ok = ok && dalloc(&h->ostage, T * d * 4);
@@ -376,6 +396,17 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     ok = ok && dalloc(&h->Bt, F * R * 2);
   }
   if (desc->flags & SFFN_FLAG_DEBUG_GATE) ok = ok && dalloc(&h->gdebug, T * F * 4);
+  // stream-K gate for the low-rank second GEMM (short K): with the dense gate's
+  // long K, one CTA per tile streams W_gate faster than split tiles do
+  if (!h->f32 && !h->wina && h->lowrank && (int)P < h->n_sm) {
+    const int gate_kb = cdiv(h->R, 64);
+    h->sk_grid = streamk_grid((int)P, gate_kb, h->n_sm, SK_MAX_PIECES);
+    if (h->sk_grid) {
+      h->sk_bn = pick_bn((int)std::min<size_t>(T, 64));
+      ok = ok && dalloc(&h->skpart, P * SK_MAX_PIECES * (size_t)h->sk_bn * 128 * 4);
+      ok = ok && dalloc(&h->sktick, P * 4);
+    }
+  }
   if (!ok) {
     free_handle(h);
     return SFFN_ERR_ALLOC;
@@ -385,6 +416,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
   if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, 2048, st);
+  if (h->sktick) e = e ? e : cudaMemsetAsync(h->sktick, 0, P * 4, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->zacc, 0, T * (size_t)h->R * 4, st);
     e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * (T / 16 + 2) * 4, st);
@@ -416,6 +448,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   // kernel attributes and A-operand tensor maps
   if (!e && !h->f32) {
     e = e ? e : set_tc_attrs<EpiGateTwell>();
+    e = e ? e : set_tc_attrs<EpiGateTwellSK>();
     e = e ? e : set_tc_attrs<EpiWina>();
     e = e ? e : set_tc_attrs<EpiLowRankZ>();
     e = e ? e : set_tc_attrs<EpiFallbackH>();
@@ -441,9 +474,10 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     h->rows_nslot = RW_NS;
     h->rows_lcap = lcap;
     h->rows_smem = RowsSmem::make(h->P, lcap).total;
-    // the ring doubles as the [8][d] fp32 partial-output buffer
+    // the ring doubles as the [8][d] fp32 partial-output buffer and its cluster slice
     h->rows_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXC * RW_CHUNK &&
-                 (long long)RW_NS * RowsSmem::STAGE >= 32LL * h->d && h->rows_smem <= max_smem;
+                 (long long)RW_NS * RowsSmem::STAGE >= 48LL * h->d && h->P <= RW_THREADS &&
+                 h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
     // largest cluster (4, else 2) whose co-resident CTAs still cover almost every SM
     h->rows_cs = 1;
@@ -578,6 +612,10 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   ga.kb_total[0] = gate_kb;
   ga.n_rows = T;
   ga.status = h->status;
+  if (rows && rows_split > 1) {  // the split fused kernel adds its partials into out
+    ga.zero_out = reinterpret_cast<float4*>(out);
+    ga.zero_n4 = (long long)T * d / 4;
+  }
   if (h->wina) {
     WinaParams wp{D.gate_bias, D.act, T, F, h->norms, h->vdense, 0, h->scores};
     tmark(h, st, L_GATE);
@@ -591,36 +629,42 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
       return SFFN_ERR_CUDA;
   } else {
     tmark(h, st, L_GATE);
-    e = launch_tc<EpiGateTwell>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, tw);
+    if (h->sk_grid && T <= 64) {
+      // fewer neuron tiles than SMs: spread the K blocks over every SM
+      ga.m_tiles = P;
+      GateSKParams sp{tw, h->skpart, h->sktick};
+      e = launch_tc<EpiGateTwellSK>(BN, dim3(h->sk_grid, 1, 1), st, *gateA, *gateB, *gateA, *gateB, ga, sp);
+    } else {
+      e = launch_tc<EpiGateTwell>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, tw);
+    }
     ++launches;
     if (e) return SFFN_ERR_CUDA;
   }
 
   // -------------------------------------------------------------- router
-  RouterArgs ra{};
-  ra.T = T;
-  ra.ovf = h->ovf;
-  ra.epoch = epoch;
-  ra.ovf_list = h->ovf_list;
-  ra.ovf_count = h->ovf_count;
-  ra.blk_live = h->blk_live;
-  ra.kmask = reinterpret_cast<const uint4*>(h->kmask);
-  ra.umask = rows ? reinterpret_cast<uint4*>(h->umask) : nullptr;
-  ra.P = P;
-  ra.x = static_cast<const uint4*>(x);
-  ra.xo = reinterpret_cast<uint4*>(h->xo);
-  ra.d_vec = d / 8;
-  ra.z = h->lowrank ? reinterpret_cast<const uint4*>(h->z) : nullptr;
-  ra.zo = reinterpret_cast<uint4*>(h->zo);
-  ra.r_vec = h->R / 8;
-  ra.out = reinterpret_cast<float4*>(out);
-  ra.d4 = d / 4;
-  ra.zero_mode = (!rows || rows_split > 1) ? 1 : (sk_down > 1 ? 2 : 0);
-  const int router_ctas = std::max(1, std::min(h->n_sm, cdiv((long long)T * d / 4, 4096)));
-  tmark(h, st, L_ROUTER);
-  ++launches;
-  if (launch_pdl(k_router, dim3(router_ctas), dim3(1024), (size_t)router_smem_bytes(T), st, 1, ra))
-    return SFFN_ERR_CUDA;
+  // (the fused row kernel does its own routing: only the tile path needs this)
+  if (!rows) {
+    RouterArgs ra{};
+    ra.T = T;
+    ra.ovf = h->ovf;
+    ra.epoch = epoch;
+    ra.ovf_list = h->ovf_list;
+    ra.ovf_count = h->ovf_count;
+    ra.x = static_cast<const uint4*>(x);
+    ra.xo = reinterpret_cast<uint4*>(h->xo);
+    ra.d_vec = d / 8;
+    ra.z = h->lowrank ? reinterpret_cast<const uint4*>(h->z) : nullptr;
+    ra.zo = reinterpret_cast<uint4*>(h->zo);
+    ra.r_vec = h->R / 8;
+    ra.out = reinterpret_cast<float4*>(out);
+    ra.d4 = d / 4;
+    ra.zero_all = 1;
+    const int router_ctas = std::max(1, std::min(h->n_sm, cdiv((long long)T * d / 4, 4096)));
+    tmark(h, st, L_ROUTER);
+    ++launches;
+    if (launch_pdl(k_router, dim3(router_ctas), dim3(1024), (size_t)router_smem_bytes(T), st, 1, ra))
+      return SFFN_ERR_CUDA;
+  }
 
   // ------------------------------------------ non-overflow tokens
   if (rows) {
@@ -632,8 +676,16 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     rw.count = h->count;
     rw.idx = h->idx;
     rw.val = static_cast<const __nv_bfloat16*>(h->val);
-    rw.umask = reinterpret_cast<const uint4*>(h->umask);
-    rw.blk_live = h->blk_live;
+    rw.kmask = reinterpret_cast<const uint4*>(h->kmask);
+    rw.ovf = h->ovf;
+    rw.epoch = epoch;
+    rw.ovf_list = h->ovf_list;
+    rw.ovf_count = h->ovf_count;
+    rw.xo = reinterpret_cast<uint4*>(h->xo);
+    rw.z = h->lowrank ? reinterpret_cast<const uint4*>(h->z) : nullptr;
+    rw.zo = reinterpret_cast<uint4*>(h->zo);
+    rw.r_vec = h->R / 8;
+    rw.zero_ovf_rows = rows_split == 1 && sk_down > 1 ? 1 : 0;
     rw.out = out;
     rw.T = T;
     rw.d = d;
@@ -759,8 +811,7 @@ static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out,
   ra.epoch = epoch;
   ra.ovf_list = h->ovf_list;
   ra.ovf_count = h->ovf_count;
-  ra.blk_live = h->blk_live;
-  ra.zero_mode = 0;
+  ra.zero_all = 0;
   tmark(h, st, L_ROUTER);
   ++launches;
   if (launch_pdl(k_router, dim3(1), dim3(1024), (size_t)router_smem_bytes(T), st, 1, ra)) return SFFN_ERR_CUDA;

@@ -40,24 +40,19 @@ __device__ __forceinline__ int block_scan_excl(int v, int* warp_tot, int* total)
 }
 
 // ---------------------------------------------------------------- router
-// Hybrid routing ([TwELL] "Hybrid 應對非均勻稀疏"): a token whose TwELL record
-// overflowed in some tile goes whole to the dense channel.  Every CTA ranks
-// the overflow tokens itself (the flags are few) and keeps them as a bit set;
-// CTA 0 publishes the overflow list, its count and the per-8-token-block live
-// masks; all CTAs then gather the overflow rows of x (and z), build the union
-// of kept neurons of every (8-token block, tile) over the block's live tokens
-// from the gate epilogue's per-token keep masks, and zero the output rows that
-// are accumulated with atomics afterwards.
+// Hybrid routing ([TwELL] "Hybrid 應對非均勻稀疏") for the tile path and the
+// fp32 path: a token whose TwELL record overflowed in some tile goes whole to
+// the dense channel.  Every CTA ranks the overflow tokens itself (the flags
+// are few); CTA 0 publishes the overflow list and its count; all CTAs then
+// gather the overflow rows of x (and z) and, if asked, zero the output that
+// later kernels accumulate into.  (The fused row kernel routes its own
+// blocks.)
 struct RouterArgs {
   int T;
   const uint32_t* ovf;
   uint32_t epoch;
   int* ovf_list;           // [maxT]
   int* ovf_count;          // [1]
-  uint8_t* blk_live;       // [ceil(T/8)]: bit i = token 8b+i < T and not overflow
-  const uint4* kmask;      // [T][P] kept bits per (token, tile), or null
-  uint4* umask;            // [ceil(T/8)][P] union over the block's live tokens
-  int P;
   const uint4* x;          // [T][d] bf16 as 16-byte vectors, or null (no gather)
   uint4* xo;               // [maxT][d]
   int d_vec;               // d / 8
@@ -66,22 +61,19 @@ struct RouterArgs {
   int r_vec;               // R / 8
   float4* out;             // [T][d] fp32
   int d4;                  // d / 4
-  int zero_mode;           // 0: none, 1: all T rows, 2: overflow rows only
+  int zero_all;            // zero all T rows of out
 };
 
-__host__ __device__ inline int router_smem_bytes(int T) { return T * 4 + ((T + 31) / 32) * 4; }
+__host__ __device__ inline int router_smem_bytes(int T) { return T * 4; }
 
 __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
-  extern __shared__ int rs_list[];   // [T] overflow list, then [ceil(T/32)] overflow bits
-  uint32_t* obits = reinterpret_cast<uint32_t*>(rs_list + a.T);
+  extern __shared__ int rs_list[];   // [T] overflow list
   __shared__ int scan_tmp[33];
   griddep_wait();
   int base = 0;
   for (int c = 0; c < a.T; c += blockDim.x) {
     const int t = c + threadIdx.x;
     const int f = (t < a.T && a.ovf[t] == a.epoch) ? 1 : 0;
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, f);
-    if ((threadIdx.x & 31) == 0 && t < a.T) obits[t >> 5] = bal;
     int tot;
     const int ex = block_scan_excl(f, scan_tmp, &tot);
     if (f) rs_list[base + ex] = t;
@@ -89,33 +81,12 @@ __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
   }
   __syncthreads();
   const int n_o = base;
-  const int nb = (a.T + 7) >> 3;
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < n_o; i += blockDim.x) a.ovf_list[i] = rs_list[i];
     if (threadIdx.x == 0) *a.ovf_count = n_o;
-    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
-      const int valid = min(8, a.T - b * 8);
-      const uint32_t ob = (obits[(b * 8) >> 5] >> ((b * 8) & 31)) & 0xFFu;
-      a.blk_live[b] = (uint8_t)(((1u << valid) - 1u) & ~ob);
-    }
   }
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long gstride = (long long)gridDim.x * blockDim.x;
-  if (a.umask) {
-    const long long n = (long long)nb * a.P;
-    for (long long e = gtid; e < n; e += gstride) {
-      const int b = (int)(e / a.P), p = (int)(e % a.P);
-      const int valid = min(8, a.T - b * 8);
-      const uint32_t ob = (obits[(b * 8) >> 5] >> ((b * 8) & 31)) & 0xFFu;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      for (int i = 0; i < valid; ++i) {
-        if ((ob >> i) & 1u) continue;
-        const uint4 m = a.kmask[(size_t)(b * 8 + i) * a.P + p];
-        u.x |= m.x; u.y |= m.y; u.z |= m.z; u.w |= m.w;
-      }
-      a.umask[e] = u;
-    }
-  }
   if (a.x) {
     const long long n = (long long)n_o * a.d_vec;
     for (long long e = gtid; e < n; e += gstride) {
@@ -130,16 +101,9 @@ __global__ void __launch_bounds__(1024) k_router(const RouterArgs a) {
       a.zo[(size_t)o * a.r_vec + v] = a.z[(size_t)rs_list[o] * a.r_vec + v];
     }
   }
-  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (a.zero_mode == 1) {
+  if (a.zero_all) {
     const long long n = (long long)a.T * a.d4;
-    for (long long e = gtid; e < n; e += gstride) a.out[e] = zero4;
-  } else if (a.zero_mode == 2) {
-    const long long n = (long long)n_o * a.d4;
-    for (long long e = gtid; e < n; e += gstride) {
-      const int o = (int)(e / a.d4), v = (int)(e % a.d4);
-      a.out[(size_t)rs_list[o] * a.d4 + v] = zero4;
-    }
+    for (long long e = gtid; e < n; e += gstride) a.out[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 

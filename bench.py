@@ -2,14 +2,20 @@
 """Throughput of the activation-sparse gated FFN forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload decode_bf16|lopa_bf16|wina_bf16|prefill_bf16|tiny_fp32]
 
-One step = one forward of the whole hot path (gate GEMM with the TwELL
-epilogue, overflow routing, fused sparse up x down, dense-channel launches)
-over one batch of the decode workload: d_model=4096, d_ff=14336, 8 tokens,
-bf16, ReLU gate with bias -1.2816 (about 90 % zeros), tile capacity 32.
-Inputs are seeded synthetic tensors already resident in HBM.  Three copies of
-the weights (1.06 GB) and 16 input batches rotate between steps, so no step
-finds its weights in the 126 MB L2.
+One step = one forward of the whole hot path over one batch of synthetic
+tokens: gate GEMM with the TwELL epilogue (dense, low-rank or WINA top-k),
+overflow routing, the sparse up x down of the non-overflow tokens and the
+dense channel of the overflow tokens.  The default workload is decode:
+d_model=4096, d_ff=14336, 8 tokens, bf16, ReLU gate with bias -1.2816 (about
+90 % zeros), tile capacity 32.  The other workloads are the low-rank gate
+(rank 512, 32 tokens), WINA top-k (k = 5018 of 14336, SiLU, 32 tokens),
+sparse prefill (d_model=2048, d_ff=8192, 4096 tokens, ~99 % zeros with
+heavy-tailed per-token activity, tile capacity 8) and a tiny fp32 case.
+Inputs are seeded synthetic tensors already resident in HBM.  Several copies
+of the weights rotate between steps, so that no step finds its weights in
+the 126 MB L2.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
 (the forward has no exchange step), the timed region is bracketed by a
@@ -23,7 +29,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import sys
@@ -36,15 +41,37 @@ if ROOT not in sys.path:
 
 METRIC = "sparse gated-FFN tokens/s and achieved HBM GB/s vs peak at 90%/99% sparsity"
 UNIT = "tokens/s"
-WORKLOAD = "decode_bf16"
-TOKENS = 8
-N_WEIGHT_SETS = 3
-N_X_BATCHES = 16
+DEFAULT_WORKLOAD = "decode_bf16"
+# tokens per step, rotating weight copies, x batches, default timed steps
+BENCH_SHAPES = {
+    "decode_bf16": (8, 3, 16, 2000),
+    "lopa_bf16": (32, 2, 16, 1000),
+    "wina_bf16": (32, 2, 16, 1000),
+    "prefill_bf16": (4096, 4, 3, 300),
+    "tiny_fp32": (64, 1, 4, 1000),
+}
+SPARSITY = {
+    "decode_bf16": "relu gate bias -1.2816 (~90% zeros)",
+    "lopa_bf16": "low-rank gate r=512, relu, bias -1.2816 (~90% zeros)",
+    "wina_bf16": "silu gate, WINA top-k k=5018 (65% dropped)",
+    "prefill_bf16": "relu gate, heavy-tailed per-token nnz (mean ~99 dropped of 8192)",
+    "tiny_fp32": "relu gate bias -1.2816 (~90% zeros)",
+}
 TIMING_STRIDE = 8
+REF_BUDGET_S = 90.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {
     "gate": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
+    "gate_lowrank_z": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
+    "tile_h": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
+    "fallback_h": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
+    "down": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "updown_rows": ["rows_mma.cuh", "ptx.cuh"],
+    "router": ["simt.cuh", "ptx.cuh"],
+    "wina_topk": ["simt.cuh", "ptx.cuh"],
+    "gate_f32": ["simt.cuh", "epilogues.cuh", "ptx.cuh"],
+    "rows_f32": ["simt.cuh", "ptx.cuh"],
+    "fallback_f32": ["simt.cuh", "ptx.cuh"],
 }
 
 
@@ -163,10 +190,11 @@ def cpu_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_timing(inp, budget_s: float, steps: int = 0):
-    """Time the fp64 oracle on the workload's token batch: operands decoded to
-    fp64 once, then whole oracle forwards (gate, selection, TwELL pack, sparse
-    up/down) until the budget is spent (or for `steps` forwards)."""
+def oracle_timing(inp, T: int, budget_s: float, steps: int = 0):
+    """Time the fp64 oracle on T-token batches of the workload: operands
+    decoded to fp64 once, then whole oracle forwards (gate, selection, TwELL
+    pack, sparse up/down, dense channel) until the budget is spent (or for
+    `steps` forwards)."""
     import numpy as np
     import oracle
     f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
@@ -176,7 +204,7 @@ def oracle_timing(inp, budget_s: float, steps: int = 0):
     xs = f(inp.x)
     n, tokens, t0 = 0, 0, time.perf_counter()
     while True:
-        x = xs[(n * TOKENS) % xs.shape[0]:][:TOKENS]
+        x = xs[(n * T) % xs.shape[0]:][:T]
         oracle.forward(np.ascontiguousarray(x), W["W_up"], W["W_down"], W_gate=W["W_gate"], A=W["A"],
                        B=W["B"], bias=W["bias"], dtype=wl.dtype, mode=wl.mode, act=wl.act,
                        threshold=wl.threshold, k=wl.k, C=wl.tile_capacity)
@@ -188,18 +216,126 @@ def oracle_timing(inp, budget_s: float, steps: int = 0):
     return tokens / el, n, el
 
 
-def config_dict(wl, T: int, sets: int = N_WEIGHT_SETS) -> dict:
+def weight_bytes(wl) -> int:
+    es = 4 if wl.dtype == "fp32" else 2
+    gate = (wl.d_model + wl.d_ff) * wl.rank if wl.rank else wl.d_ff * wl.d_model
+    return (gate + 2 * wl.d_ff * wl.d_model) * es
+
+
+def config_dict(wl, T: int, sets: int, x_batches: int) -> dict:
     return {"workload": f"{wl.name}: d_model={wl.d_model} d_ff={wl.d_ff} tokens={T} {wl.dtype} "
-                        f"{wl.act} gate bias={wl.bias} (~90% zeros) tile_capacity={wl.tile_capacity}",
+                        f"{SPARSITY.get(wl.name, '')} tile_capacity={wl.tile_capacity}",
             "tokens_per_step": T, "d_model": wl.d_model, "d_ff": wl.d_ff,
             "l2": f"inputs larger than L2: {sets} rotating weight copies "
-                  f"({sets * 3 * wl.d_model * wl.d_ff * 2 / 1e9:.2f} GB) and {N_X_BATCHES} x batches",
+                  f"({sets * weight_bytes(wl) / 1e9:.2f} GB) and {x_batches} x batches"
+                  if sets * weight_bytes(wl) > 126e6 else
+                  f"weights ({weight_bytes(wl) / 1e6:.1f} MB) are L2-resident: this workload is launch-bound",
             "parallelism": "replicas (one independent forward per GPU)"}
 
 
+def kernel_work(wl, T: int, path: str, st: dict) -> dict:
+    """Algorithmic HBM bytes and FLOPs of one launch of each kernel of the
+    forward, from the workload's sizes and the realised sparsity of the batch
+    (st: union = distinct kept neurons of the live tokens, nnz = their kept
+    (token, neuron) pairs, n_overflow).  Bytes count what the method must
+    move (weights read once, x, out, TwELL written and read); FLOPs exclude
+    the dense work the method avoids and the dense channel's recomputed gate."""
+    d, F, R = wl.d_model, wl.d_ff, wl.rank
+    P, C = F // 128, wl.tile_capacity
+    es = 4 if wl.dtype == "fp32" else 2
+    twell = T * P * (2 + C * (2 + es))
+    kmask = T * P * 16
+    xb, yb = T * d * es, T * d * 4
+    n_o, U, nnz = st["n_overflow"], st["union"], st["nnz"]
+    fp32 = wl.dtype == "fp32"
+    w = {}
+    g = "gate_f32" if fp32 else "gate"
+    if R:
+        w["gate_lowrank_z"] = {"bytes": d * R * es + xb + T * R * es, "flops": 2 * T * d * R}
+        w[g] = {"bytes": R * F * es + T * R * es + twell + kmask, "flops": 2 * T * R * F}
+    elif wl.mode == "wina_topk":
+        w[g] = {"bytes": F * d * es + xb + T * F * (es + 4) + F * 4, "flops": 2 * T * d * F}
+        w["wina_topk"] = {"bytes": T * F * (es + 4) + twell, "flops": 0}
+    else:
+        w[g] = {"bytes": F * d * es + xb + twell + (0 if fp32 else kmask), "flops": 2 * T * d * F}
+    sparse = {"bytes": U * 2 * d * es + xb + yb + twell, "flops": 4 * nnz * d}
+    dense_in = 2 * F * d * es if n_o else 0      # W_gate and W_up, read once if any token overflows
+    if fp32:
+        w["router"] = {"bytes": T * 4, "flops": 0}
+        w["rows_f32"] = sparse
+        w["fallback_f32"] = {"bytes": dense_in + (F * d * es if n_o else 0), "flops": 4 * n_o * d * F}
+    elif path == "rows":
+        w["updown_rows"] = {"bytes": sparse["bytes"] + kmask, "flops": sparse["flops"]}
+        if wl.mode != "wina_topk":
+            w["fallback_h"] = {"bytes": dense_in + n_o * F * 4, "flops": 2 * n_o * d * F}
+        w["down"] = {"bytes": (F * d * es + n_o * F * 4 + n_o * d * 4) if n_o else 0, "flops": 2 * n_o * F * d}
+    else:
+        w["router"] = {"bytes": yb + 2 * n_o * d * es, "flops": 0}
+        w["tile_h"] = {"bytes": F * d * es + xb + twell + T * F * 4, "flops": 2 * T * d * F}
+        if wl.mode != "wina_topk":
+            w["fallback_h"] = {"bytes": dense_in + n_o * F * 4, "flops": 2 * n_o * d * F}
+        w["down"] = {"bytes": F * d * es + T * F * 4 + yb, "flops": 2 * T * F * d}
+    return w
+
+
+def step_work(wl, T: int, st: dict) -> tuple[int, int]:
+    """Algorithmic bytes and FLOPs of one whole forward."""
+    d, F, R = wl.d_model, wl.d_ff, wl.rank
+    P, C = F // 128, wl.tile_capacity
+    es = 4 if wl.dtype == "fp32" else 2
+    twell = T * P * (2 + C * (2 + es))
+    gate_w = (d * R + R * F) * es if R else F * d * es
+    gate_f = 2 * T * (d * R + R * F) if R else 2 * T * d * F
+    n_o = st["n_overflow"]
+    byts = gate_w + st["union"] * 2 * d * es + T * d * es + T * d * 4 + 2 * twell
+    if n_o:
+        byts += 2 * F * d * es
+    flops = gate_f + 4 * st["nnz"] * d + 4 * n_o * d * F
+    return int(byts), int(flops)
+
+
+def roofline_of(work: dict, ms: float, peaks: dict, peak_src: str) -> dict:
+    """Roofline of one kernel: bound = the resource whose ideal time for the
+    kernel's algorithmic work is longer (HBM bytes at the copy peak, or bf16
+    tensor FLOPs at the sustained GEMM peak, the kernel being timed inside a
+    long run of steps)."""
+    hbm, tc = peaks["hbm_gbs"], peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_hbm = work["bytes"] / (hbm * 1e9)
+    t_tc = work["flops"] / (tc * 1e12)
+    src = "measured" if peak_src == "measured" else "fallback"
+    if t_tc > t_hbm:
+        a = work["flops"] / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(a, 2), "peak": tc, "unit": "TFLOP/s",
+                "frac": round(a / tc, 4), "algorithmic_flops": int(work["flops"]),
+                "peak_source": f"{src} (bf16_tflops_sustained)"}
+    a = work["bytes"] / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(a, 1), "peak": hbm, "unit": "GB/s", "frac": round(a / hbm, 4),
+            "algorithmic_bytes": int(work["bytes"]), "peak_source": f"{src} (hbm_gbs)"}
+
+
 # ---------------------------------------------------------------- our arm
+def batch_sparsity(ffn, T: int, C: int) -> dict:
+    """Realised sparsity of the last forward, from its TwELL records: the
+    distinct kept neurons of the live (non-overflow) tokens, their kept pairs,
+    the 8-token-block unions summed (rows the fused kernel gathers) and the
+    overflow count."""
+    import torch
+    tw = ffn.twell(T)
+    cnt = tw["count"].long()
+    ovf = (cnt > C).any(dim=1)
+    live = ~ovf
+    n = torch.minimum(cnt, torch.tensor(C, device=cnt.device))
+    used = (torch.arange(C, device=cnt.device)[None, None, :] < n[:, :, None]) & live[:, None, None]
+    idx = tw["idx"].long()
+    tok = torch.arange(T, device=cnt.device)[:, None, None].expand_as(idx)
+    kept_idx, kept_tok = idx[used], tok[used]
+    blocks = torch.zeros(((T + 7) // 8, ffn.d_ff), dtype=torch.bool, device=cnt.device)
+    blocks[kept_tok // 8, kept_idx] = True
+    return {"union": int(torch.unique(kept_idx).numel()), "nnz": int(kept_idx.numel()),
+            "block_rows": int(blocks.sum()), "n_overflow": int(ovf.sum())}
+
+
 def run_ours(args) -> None:
-    import numpy as np
     import torch
 
     import synth
@@ -220,24 +356,25 @@ def run_ours(args) -> None:
     barrier(world)
     load_library()
 
-    wl = synth.WORKLOADS[WORKLOAD]
-    T = TOKENS
-    inp = synth.make_inputs(wl, T=T * N_X_BATCHES)
+    wl = synth.WORKLOADS[args.workload]
+    T, _, NXB, _ = BENCH_SHAPES[args.workload]
+    NS = args.weight_sets
+    inp = synth.make_inputs(wl, T=T * NXB)
     dev = lambda t: None if t is None else t.to("cuda")  # noqa: E731
     sets = []
-    for s in range(args.weight_sets):
-        ws = {k: dev(getattr(inp, k)) for k in ("W_gate", "W_up", "W_down", "bias")}
-        ffn = SparseFFN(ws["W_up"], ws["W_down"], W_gate=ws["W_gate"], bias=ws["bias"],
+    for s in range(NS):
+        ws = {k: dev(getattr(inp, k)) for k in ("W_gate", "A", "B", "W_up", "W_down", "bias")}
+        ffn = SparseFFN(ws["W_up"], ws["W_down"], W_gate=ws["W_gate"], A=ws["A"], B=ws["B"], bias=ws["bias"],
+                        mode=wl.mode, act=wl.act, threshold=wl.threshold, k=wl.k,
                         tile_capacity=wl.tile_capacity, max_tokens=T)
         sets.append((ws, ffn))
     xall = dev(inp.x)
-    xb = [xall[i * T:(i + 1) * T].contiguous() for i in range(N_X_BATCHES)]
-    NS = args.weight_sets
+    xb = [xall[i * T:(i + 1) * T].contiguous() for i in range(NXB)]
     outs = [torch.empty((T, wl.d_model), dtype=torch.float32, device="cuda") for _ in range(NS)]
     stream = torch.cuda.current_stream()
 
     def step(i):
-        sets[i % NS][1].forward(xb[i % N_X_BATCHES], outs[i % NS])
+        sets[i % NS][1].forward(xb[i % NXB], outs[i % NS])
 
     for i in range(args.warmup):
         step(i)
@@ -274,90 +411,84 @@ def run_ours(args) -> None:
         assert ffn.read_status() == SFFN_OK
     tot_ms, tot_units = aggregate(elapsed, float(T * args.steps), world)
 
-    # ------------------------------------------------- algorithmic bytes
-    # per x batch: union of kept neurons (from the forward's TwELL records)
+    # ---------------------------------- algorithmic work of the batches
     ffn0 = sets[0][1]
-    unions, twell_bytes = [], []
-    P, C = wl.d_ff // 128, wl.tile_capacity
-    for b in range(N_X_BATCHES):
+    sp = []
+    for b in range(NXB):
         ffn0.forward(xb[b], outs[0])
-        tw = ffn0.twell(T)
-        n = torch.minimum(tw["count"].long(), torch.tensor(C, device="cuda"))
-        used = torch.arange(C, device="cuda")[None, None, :] < n[:, :, None]
-        idx = tw["idx"].long()[used]
-        unions.append(int(torch.unique(idx).numel()))
-    union = float(np.mean(unions))
-    d, F, es = wl.d_model, wl.d_ff, 2
-    twell = T * P * (2 + C * (2 + es))
-    nblk = math.ceil(T / 8)
-    bytes_gate = F * d * es + T * d * es + twell + nblk * P * 16
-    bytes_rows = union * 2 * d * es + T * d * es + T * d * 4 + twell + nblk * P * 16
-    bytes_step = F * d * es + union * 2 * d * es + T * d * es + T * d * 4 + 2 * twell
+        sp.append(batch_sparsity(ffn0, T, wl.tile_capacity))
+    st = {k: sum(x[k] for x in sp) / len(sp) for k in sp[0]}
+    path = "rows" if ffn0.stats().path == 1 else "tiles"
+    works = kernel_work(wl, T, path, st)
+    bytes_step, flops_step = step_work(wl, T, st)
 
     peaks, peak_src = load_peaks()
     per = {k: (v[0] / v[1] if v[1] else 0.0) for k, v in kernels.items()}
     dom = max(per, key=lambda k: kernels[k][0]) if per else None
-    alg = {"gate": bytes_gate, "updown_rows": bytes_rows}
     roof = None
-    if dom in alg:
-        achieved = alg[dom] / (per[dom] * 1e-3) / 1e9
-        traffic = profiled_traffic(dom, WORKLOAD)
-        roof = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                "algorithmic_bytes": int(alg[dom]), "ms_per_launch": round(per[dom], 5),
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                else "fallback 6650 GB/s"}
+    if dom in works and per[dom] > 0:
+        roof = roofline_of(works[dom], per[dom], peaks, peak_src)
+        roof.update({"kernel": dom, "traffic": profiled_traffic(dom, args.workload),
+                     "ms_per_launch": round(per[dom], 5)})
     total_kernel_ms = sum(v[0] for v in kernels.values())
-    kern_out = {k: {"ms_per_launch": round(per[k], 5), "launches": kernels[k][1],
-                    "share": round(kernels[k][0] / total_kernel_ms, 4) if total_kernel_ms else None,
-                    **({"achieved_gbs": round(alg[k] / (per[k] * 1e-3) / 1e9, 1),
-                        "frac_of_hbm": round(alg[k] / (per[k] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
-                       if k in alg and per[k] > 0 else {})}
-                for k in kernels}
+    kern_out = {}
+    for k in kernels:
+        e = {"ms_per_launch": round(per[k], 5), "launches": kernels[k][1],
+             "share": round(kernels[k][0] / total_kernel_ms, 4) if total_kernel_ms else None}
+        if k in works and per[k] > 0 and (works[k]["bytes"] or works[k]["flops"]):
+            r = roofline_of(works[k], per[k], peaks, peak_src)
+            e.update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
+        kern_out[k] = e
 
     # ------------------------------------------------------ end to end
     e2e = None
     e2e_steps = 0 if args.no_e2e else max(10, min(args.steps, 400))
     if e2e_steps:
-        xh = [inp.x[i * T:(i + 1) * T].contiguous().pin_memory() for i in range(N_X_BATCHES)]
+        xh = [inp.x[i * T:(i + 1) * T].contiguous().pin_memory() for i in range(NXB)]
         oh = torch.empty((T, wl.d_model), dtype=torch.float32).pin_memory()
         for i in range(3):
-            sets[i % NS][1].forward_host(xh[i % N_X_BATCHES], oh)
+            sets[i % NS][1].forward_host(xh[i % NXB], oh)
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(e2e_steps):
-            sets[i % NS][1].forward_host(xh[i % N_X_BATCHES], oh)
+            sets[i % NS][1].forward_host(xh[i % NXB], oh)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms, e2e_units = aggregate(e0.elapsed_time(e1), float(T * e2e_steps), world)
+        es = 4 if wl.dtype == "fp32" else 2
         e2e = {"value": round(e2e_units / (e2e_ms * 1e-3), 1), "unit": UNIT,
-               "h2d_bytes_per_step": T * wl.d_model * 2, "d2h_bytes_per_step": T * wl.d_model * 4,
+               "h2d_bytes_per_step": T * wl.d_model * es, "d2h_bytes_per_step": T * wl.d_model * 4,
                "api": "sffn_forward_host (pinned host x in, host y out, stream synchronised per step)"}
 
     # --------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu_inp = synth.make_inputs(wl, T=T * 4)
-        v, n, el = oracle_timing(cpu_inp, budget_s=args.cpu_budget)
+        cpu_inp = synth.make_inputs(wl, T=T * min(NXB, 4))
+        v, n, el = oracle_timing(cpu_inp, T, budget_s=args.cpu_budget)
         cpu = {"value": round(v, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n} fp64 oracle forwards of {T}-token batches of the same workload "
                          f"({el:.1f} s; operands decoded to fp64 once, before timing)"}
 
     if rank == 0:
         value = tot_units / (tot_ms * 1e-3)
+        step_s = tot_ms * 1e-3 / args.steps
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_ms / args.steps, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if wl.dtype == "fp32" else "bf16",
             "data": "synthetic (seeded Gaussian x and N(0,1/fan_in) weights)",
-            "config": config_dict(wl, T, NS),
-            "hbm_gbs_step": round(bytes_step * args.steps * world / (tot_ms * 1e-3) / 1e9, 1),
-            "hbm_frac_step": round(bytes_step * args.steps * world / (tot_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "union_active_neurons": union,
-            "algorithmic_bytes_per_step": int(bytes_step),
+            "config": config_dict(wl, T, NS, NXB),
+            "hbm_gbs_step": round(bytes_step * world / step_s / 1e9, 1),
+            "hbm_frac_step": round(bytes_step * world / step_s / 1e9 / peaks["hbm_gbs"], 4),
+            "tflops_step": round(flops_step * world / step_s / 1e12, 2),
+            "sparsity": {k: round(v, 1) for k, v in st.items()},
+            "path": path,
+            "algorithmic_bytes_per_step": bytes_step,
+            "algorithmic_flops_per_step": flops_step,
             "roofline": roof,
             "kernels": kern_out,
             "cpu_baseline": cpu,
@@ -375,23 +506,30 @@ def run_ours(args) -> None:
 
 # ------------------------------------------------------- reference arm
 def run_reference(args) -> None:
+    """The reference arm: the fp64 oracle on the host cores, one T-token
+    forward of the workload per step.  The timed steps are capped so that the
+    whole run stays within a few minutes (the rate does not depend on how
+    many forwards are timed); the line says how many were."""
     rank, _, world = dist_env()
     if rank != 0:
         return
     import synth
-    wl = synth.WORKLOADS[WORKLOAD]
-    T = TOKENS
-    inp = synth.make_inputs(wl, T=T * 4)
-    oracle_timing(inp, 0, steps=max(1, min(args.warmup, 3)))
-    v, n, el = oracle_timing(inp, 0, steps=args.steps)
+    wl = synth.WORKLOADS[args.workload]
+    T, _, NXB, _ = BENCH_SHAPES[args.workload]
+    inp = synth.make_inputs(wl, T=T * min(NXB, 4))
+    _, nw, elw = oracle_timing(inp, T, 0, steps=max(1, min(args.warmup, 3)))
+    per_fwd = elw / nw
+    n_timed = max(1, min(args.steps, int(REF_BUDGET_S / max(per_fwd, 1e-6))))
+    v, n, el = oracle_timing(inp, T, 0, steps=n_timed)
     cores = cpu_threads()
+    sample = (f"{n} fp64 oracle forwards of {T}-token batches (one per step; {args.steps} steps asked, "
+              f"capped at ~{REF_BUDGET_S:.0f} s of host time)")
     line = {
-        "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(wl, T), "impl": "reference",
-        "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{n} fp64 oracle forwards of {T}-token batches (one per step)"},
+        "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world, "steps": n,
+        "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, T, 1, min(NXB, 4)), "impl": "reference",
+        "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -400,17 +538,23 @@ def run_reference(args) -> None:
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default: per workload)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(BENCH_SHAPES), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
-    ap.add_argument("--weight-sets", type=int, default=N_WEIGHT_SETS,
+    ap.add_argument("--weight-sets", type=int, default=None,
                     help="rotating weight copies (fewer only for small profiler captures)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    _, sets, _, steps = BENCH_SHAPES[args.workload]
+    if args.steps is None:
+        args.steps = steps
+    if args.weight_sets is None:
+        args.weight_sets = sets
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -65,3 +65,51 @@ def test_profiled_traffic_requires_matching_sources(tmp_path, monkeypatch):
 def test_warmup_floor():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "1"])
+
+
+def test_work_model_decode_matches_byte_formula():
+    import synth
+    wl = synth.WORKLOADS["decode_bf16"]
+    st = {"union": 8163, "nnz": 12000, "block_rows": 8163, "n_overflow": 0}
+    b, f = bench.step_work(wl, 8, st)
+    P = wl.d_ff // 128
+    twell = 8 * P * (2 + 32 * 4)
+    assert b == wl.d_ff * wl.d_model * 2 + 8163 * 2 * wl.d_model * 2 + 8 * wl.d_model * (2 + 4) + 2 * twell
+    assert f == 2 * 8 * wl.d_model * wl.d_ff + 4 * 12000 * wl.d_model
+    w = bench.kernel_work(wl, 8, "rows", st)
+    assert set(w) == {"gate", "updown_rows", "fallback_h", "down"}
+    # no overflow: the dense channel moves nothing
+    assert w["fallback_h"]["bytes"] == 0 and w["down"]["flops"] == 0
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    r = bench.roofline_of(w["gate"], 0.030, peaks, "measured")
+    assert r["bound"] == "hbm" and abs(r["achieved"] - w["gate"]["bytes"] / 30e-6 / 1e9) < 0.1
+
+
+def test_work_model_prefill_gate_is_tensor_bound():
+    import synth
+    wl = synth.WORKLOADS["prefill_bf16"]
+    st = {"union": 8192, "nnz": 4096 * 99, "block_rows": 300000, "n_overflow": 400}
+    w = bench.kernel_work(wl, 4096, "rows", st)
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    r = bench.roofline_of(w["gate"], 0.2, peaks, "measured")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert w["gate"]["flops"] == 2 * 4096 * 2048 * 8192
+    assert w["fallback_h"]["flops"] == 2 * 400 * 2048 * 8192
+
+
+def test_work_model_tile_path_kernels():
+    import synth
+    for name, extra in (("lopa_bf16", {"gate_lowrank_z", "fallback_h"}), ("wina_bf16", {"wina_topk"})):
+        wl = synth.WORKLOADS[name]
+        st = {"union": 14000, "nnz": 32 * 1400, "block_rows": 4 * 14000, "n_overflow": 1}
+        w = bench.kernel_work(wl, 32, "tiles", st)
+        assert {"gate", "router", "tile_h", "down"} | extra == set(w)
+
+
+def test_reference_arm_tiny_workload(capsys):
+    import json
+    bench.main(["--impl", "reference", "--workload", "tiny_fp32", "--steps", "2", "--warmup", "3"])
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["steps"] == 2 and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["config"]["tokens_per_step"] == 64
