@@ -394,8 +394,10 @@ struct EpiTwellH {
 };
 
 // -------------------------------------------------- down projection output
-// D^T tile: rows are output columns (m0 + etid), columns are h rows.  With a
-// split K the partial sums are added into out (zeroed by the router).
+// D^T tile: rows are output columns (m0 + etid), columns are h rows; every
+// stage multiplies one W_down^T tile by both halves of h (hi and lo) into the
+// one accumulator.  With a split K the partial sums are added into out
+// (zeroed beforehand by the router, the gate or the fused row kernel).
 struct OutParams {
   float* out;          // [T][d]
   int d;
@@ -407,6 +409,7 @@ struct OutParams {
 
 struct EpiDownOut {
   static constexpr int N_ACC = 1;
+  static constexpr bool DUAL_B = true;  // B0 = h_hi, B1 = h_lo, one accumulator
   using Params = OutParams;
   template <int BN>
   __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {

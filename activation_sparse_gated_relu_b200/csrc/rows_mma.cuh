@@ -6,27 +6,31 @@
 // block's union of kept neurons, ranked tile by tile from the union of the
 // live (non-overflow) tokens' keep masks, so that every CTA streams the same
 // number of rows.  CTA 0 of each block also routes the block's overflow
-// tokens to the dense channel (list, count, gathered rows).  Neurons are
-// processed in groups of 16.  A group's W_up rows and then its W_down rows
-// (contiguous, neuron-major) pass through a ring of shared-memory stages, one
-// stage = the same 1024-column chunk of the 16 rows (16 KB... 32 KB), each
-// row chunk brought by a 1-D bulk copy that one of the 16 warps issues, so
-// the copies of a stage go out in parallel; rows are padded by 16 bytes so
-// ldmatrix is free of bank conflicts.  One CTA barrier per stage releases its
-// slot, which the warps refill at once with the stage NS ahead.
+// tokens to the dense channel (list, count, gathered rows).
 //
-// Both contractions are warp-level tensor-core MMAs (m16n8k16, bf16 inputs,
-// fp32 accumulate) on the staged rows:
-//   up:   u[16 neurons][8 tokens] = W_up rows (ldmatrix) · x^T -- warp w takes
+// Neurons are processed in groups of 8.  A group's 8 W_up rows, then its 8
+// W_down rows, pass through a ring of shared-memory stages, one stage = 8
+// whole rows (8 x d bf16), each row brought by one 1-D bulk copy (8 KB at
+// d = 4096: the copy size at which one SM's bulk-copy traffic reaches the HBM
+// rate, where 2 KB pieces fall about a fifth short).  Rows are padded by 16
+// bytes so that ldmatrix is free of bank conflicts.  The warps issue the 8
+// copies of a stage in parallel, and one CTA barrier per stage releases its
+// slot, which is refilled at once with the stage nslot ahead.
+//
+// Both contractions are warp-level tensor-core MMAs (bf16 inputs, fp32
+// accumulate) on the staged rows:
+//   up:   u^T[8 tokens][8 neurons] = x · W_up rows^T (m16n8k16, tokens as M,
+//         padded to 16 with zero rows; rows as N via ldmatrix) -- warp w takes
 //         every 16th 16-wide k step, whose x fragments it keeps in registers;
-//         the 16 warps' partial sums meet in shared memory and every warp
-//         adds them up itself;
+//         the 16 warps' partial sums meet in shared memory and every lane
+//         adds up the 16 partials of its own fragment position;
 //   h:    h_tj = v_tj·u_tj where (t, j) is kept, else 0, split into
 //         hi = bf16(h) and lo = bf16(h - hi) (so the bf16 MMA operand loses at
-//         most 2^-16 of h);
+//         most 2^-16 of h); the up output fragment is exactly the B fragment
+//         of the down product, so h never leaves the registers;
 //   down: y^T[d][8 tokens] += W_down rows^T (ldmatrix.trans) · (h_hi + h_lo)
-//         -- warp w owns every 16th 16-row output tile, held in registers for
-//         the whole CTA.
+//         (m16n8k8, the 8 neurons as K) -- warp w owns every 16th 16-row
+//         output tile, held in registers for the whole CTA.
 // At the end the per-CTA partial y goes to out: plain stores when one CTA
 // owns the block, otherwise summed over the CTAs of a thread-block cluster
 // through distributed shared memory (each CTA of the cluster owns one column
@@ -39,12 +43,10 @@ namespace sffn {
 
 constexpr int RW_WARPS = 16;
 constexpr int RW_THREADS = RW_WARPS * 32;
-constexpr int RW_G = 16;            // neurons per group (MMA M of up, K of down)
-constexpr int RW_CHUNK = 1024;      // columns of a row per stage
-constexpr int RW_MAXC = 4;          // chunks per row: d <= 4096
-constexpr int RW_MAXJ = RW_CHUNK / 256;  // k steps (or output tiles) per warp and chunk
+constexpr int RW_G = 8;             // neurons per group = rows per stage (up N, down K)
+constexpr int RW_MAXJ = 16;         // k steps (up) and output tiles (down) per warp: d <= 4096
 constexpr int RW_DIV = 256;         // d must be a multiple of 16 warps x 16
-constexpr int RW_NS = 6;            // ring stages
+constexpr int RW_NSMAX = 6;         // ring slots at most
 
 struct RowsArgs {
   const __nv_bfloat16* x;
@@ -68,26 +70,27 @@ struct RowsArgs {
   float* out;
   int T, d, F, n_tiles, C;
   int atomic;
-  int nslot, lcap;
+  int nslot, lcap;          // ring slots (<= RW_NSMAX), neuron-id list capacity
   uint32_t* status;
 };
 
 struct RowsSmem {
   // byte offsets inside the dynamic shared memory
-  int ring, bars, tpre, ums, nid, lmask, lval, ured, misc, total;
-  static constexpr int RSTRIDE = RW_CHUNK * 2 + 16;    // padded staged row chunk (bytes)
-  static constexpr int STAGE = RW_G * RSTRIDE;
-  __host__ __device__ static RowsSmem make(int n_tiles, int lcap) {
+  int xs, ring, bars, tpre, ums, nid, lmask, lval, ured, misc, total;
+  __host__ __device__ static int pitch(int d) { return d * 2 + 16; }   // padded staged row (bytes)
+  __host__ __device__ static int stage(int d) { return RW_G * pitch(d); }
+  __host__ __device__ static RowsSmem make(int n_tiles, int lcap, int d, int nslot) {
     RowsSmem s;
     int o = 0;
-    s.ring = o;  o += RW_NS * STAGE;
-    s.bars = o;  o += RW_NS * 8;
+    s.xs = o;    o += stage(d);           // the block's 8 x rows, staged like weight rows
+    s.ring = o;  o += nslot * stage(d);
+    s.bars = o;  o += ((RW_NSMAX + 1) * 8 + 15) & ~15;  // ring slots, then the x rows; keeps 16-B alignment
     s.tpre = o;  o += ((n_tiles + 1) * 4 + 15) & ~15;
     s.ums = o;   o += n_tiles * 16;
     s.nid = o;   o += lcap * 4;
     s.lmask = o; o += lcap * 4;
     s.lval = o;  o += lcap * 16;
-    s.ured = o;  o += RW_WARPS * 32 * 16;
+    s.ured = o;  o += RW_WARPS * 32 * 8;
     s.misc = o;  o += 64 * 4;
     s.total = o;
     return s;
@@ -127,32 +130,58 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// D[16x8] += A[16x8] (row) · B[8x8] (col), bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_1688(float* c, uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
 
 __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
-  const RowsSmem L = RowsSmem::make(a.n_tiles, a.lcap);
-  constexpr int RS = RowsSmem::RSTRIDE, SB = RowsSmem::STAGE;
+  const int d = a.d;
+  const int ns = max(2, min(a.nslot, RW_NSMAX));  // ring slots, all kept in flight
+  const RowsSmem L = RowsSmem::make(a.n_tiles, a.lcap, d, ns);
+  const int RS = RowsSmem::pitch(d), SB = RowsSmem::stage(d);
   uint8_t* ring = sm + L.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint64_t* xbar = full + RW_NSMAX;
   int* tpre = reinterpret_cast<int*>(sm + L.tpre);
   uint4* ums = reinterpret_cast<uint4*>(sm + L.ums);
   int* nid = reinterpret_cast<int*>(sm + L.nid);
   uint32_t* lmask = reinterpret_cast<uint32_t*>(sm + L.lmask);
   uint4* lval = reinterpret_cast<uint4*>(sm + L.lval);
-  float4* ured = reinterpret_cast<float4*>(sm + L.ured);
+  float2* ured = reinterpret_cast<float2*>(sm + L.ured);
   int* misc = reinterpret_cast<int*>(sm + L.misc);
   volatile int* abort_flag = misc + 40;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = a.n_tiles, b = blockIdx.y, S = gridDim.x, s = blockIdx.x;
   const int tb0 = b * 8;
-  const int d = a.d;
-  const int nchunk = (d + RW_CHUNK - 1) / RW_CHUNK;
-  const int spg = 2 * nchunk;        // stages per group: up chunks, then down chunks
+  const int nj = d / RW_DIV;         // k steps (up) and output tiles (down) of each warp
 
   griddep_wait();  // keep masks, TwELL and overflow epochs come from the gate
-  // 1. live tokens of the block (valid, not overflowing) and the union of
-  // their keep masks, tile by tile; barriers
+  // 1. barriers; the block's x rows go out at once as bulk copies into the x
+  // block (staged like weight rows: the up product's A operand comes from
+  // them by ldmatrix), rows beyond T are zeroed; then the live tokens of the
+  // block (valid, not overflowing) and the union of their keep masks, tile
+  // by tile
+  const int nvalid = max(0, min(8, a.T - tb0));
+  if (tid == 0) {
+    for (int i = 0; i < ns; ++i) mbar_init(&full[i], 1);
+    mbar_init(xbar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    mbar_expect_tx(xbar, (uint32_t)(nvalid * d * 2));
+    for (int t = 0; t < nvalid; ++t)
+      bulk_g2s(sm + L.xs + t * RS, a.x + (size_t)(tb0 + t) * d, (uint32_t)d * 2u, xbar);
+  }
+  for (int e = tid; e < (8 - nvalid) * (d >> 3); e += blockDim.x) {
+    const int t = nvalid + e / (d >> 3), v = e % (d >> 3);
+    *reinterpret_cast<uint4*>(sm + L.xs + t * RS + v * 16) = make_uint4(0u, 0u, 0u, 0u);
+  }
   uint4 km[8];
   if (tid < P) {
 #pragma unroll
@@ -168,9 +197,6 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       misc[50] = (int)(vb & ~obb);
       misc[51] = (int)obb;
       misc[52] = 0;
-      for (int i = 0; i < RW_NS; ++i) mbar_init(&full[i], 1);
-      *abort_flag = 0;
-      fence_mbar_init();
     }
   }
   __syncthreads();
@@ -194,24 +220,6 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     int before = 0;
     for (int t = tid; t < tb0; t += blockDim.x) before += a.ovf[t] == a.epoch ? 1 : 0;
     if (before) atomicAdd(&misc[52], before);
-  }
-  // x^T fragments of this warp's k steps (16(w + 16 j) in every chunk), in
-  // registers; zero beyond T
-  uint32_t xb[RW_MAXC][RW_MAXJ][2];
-  {
-    const int t = tb0 + (lane >> 2);
-#pragma unroll
-    for (int c = 0; c < RW_MAXC; ++c)
-#pragma unroll
-      for (int j = 0; j < RW_MAXJ; ++j) {
-        xb[c][j][0] = xb[c][j][1] = 0u;
-        const int k = c * RW_CHUNK + 16 * (warp + RW_WARPS * j);
-        if (k < d && t < a.T) {
-          const uint32_t* xr = reinterpret_cast<const uint32_t*>(a.x + (size_t)t * d + k + 2 * (lane & 3));
-          xb[c][j][0] = xr[0];
-          xb[c][j][1] = xr[4];
-        }
-      }
   }
   __syncthreads();
   if (s == 0 && (obits != 0u || b == (int)gridDim.y - 1)) {
@@ -258,13 +266,11 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   const int U = tpre[P];
   const int r0 = (int)((long long)U * s / S), r1 = (int)((long long)U * (s + 1) / S);
 
-  float acc[RW_MAXC][RW_MAXJ][4];
+  float acc[RW_MAXJ][4];
 #pragma unroll
-  for (int c = 0; c < RW_MAXC; ++c)
+  for (int j = 0; j < RW_MAXJ; ++j)
 #pragma unroll
-    for (int j = 0; j < RW_MAXJ; ++j)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[c][j][k] = 0.f;
+    for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
 
   const uint32_t ring_s = smem_u32(ring);
   int sbase = 0;        // stages of earlier chunks (uniform), for slot and parity
@@ -273,7 +279,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   for (int c0 = r0; c0 < r1; c0 += a.lcap) {
     const int c1 = min(r1, c0 + a.lcap), Lc = c1 - c0;
     const int n_groups = (Lc + RW_G - 1) / RW_G;
-    const int n_stages = n_groups * spg;
+    const int n_stages = n_groups * 2;  // per group: its W_up rows, then its W_down rows
     // a. tiles overlapping [c0, c1): pa holds rank c0, pb holds rank c1 - 1
     for (int p = tid; p < P; p += blockDim.x) {
       if (tpre[p] <= c0 && c0 < tpre[p + 1]) misc[48] = p;
@@ -296,27 +302,25 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       lval[e] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    // c. stage q of this chunk: warp w (lane 0) copies row w's column chunk;
-    // padding rows of W_down stages copy zeros, of W_up stages nothing
+    // c. stage q of this chunk (group q / 2; W_up rows if q is even): warp w
+    // (lane 0) copies row w; padding rows of W_down stages copy zeros, of W_up
+    // stages nothing (their u is never used)
     auto issue_stage = [&](int q) {
-      if (q >= n_stages || lane != 0) return;
-      const int gs = sbase + q, slot = gs % RW_NS;
-      const int g = q / spg, st = q - g * spg;
-      const bool up = st < nchunk;
-      const int ch = up ? st : st - nchunk;
-      const int cols = min(RW_CHUNK, d - ch * RW_CHUNK);
-      const uint32_t bytes = (uint32_t)cols * 2u;
+      if (q >= n_stages || lane != 0 || warp >= RW_G) return;
+      const int gs = sbase + q, slot = gs % ns;
+      const int g = q >> 1;
+      const bool up = (q & 1) == 0;
+      const uint32_t bytes = (uint32_t)d * 2u;
       const int n0 = g * RW_G, nn = min(RW_G, Lc - n0);
       const int nrows = up ? nn : RW_G;
       if (warp == 0) mbar_expect_tx(&full[slot], bytes * (uint32_t)nrows);
       if (warp < nrows) {
-        const __nv_bfloat16* src =
-            warp < nn ? (up ? a.W_up : a.W_down) + (size_t)nid[n0 + warp] * d + ch * RW_CHUNK : a.zero_row;
+        const __nv_bfloat16* src = warp < nn ? (up ? a.W_up : a.W_down) + (size_t)nid[n0 + warp] * d : a.zero_row;
         bulk_g2s(ring + (size_t)slot * SB + warp * RS, src, bytes, &full[slot]);
       }
     };
-    for (int q = 0; q < RW_NS; ++q) issue_stage(q);
-    issued_end = sbase + min(RW_NS, n_stages);
+    for (int q = 0; q < ns; ++q) issue_stage(q);
+    issued_end = sbase + min(ns, n_stages);
     // d. scatter TwELL values of the live tokens: one thread per (slot, token, tile)
     {
       const int n_items = a.C * 8 * (pb - pa + 1);
@@ -341,88 +345,88 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       }
     }
     __syncthreads();
+    if (sbase == 0) mbar_wait(xbar, 0, abort_flag, a.status);  // the x rows have landed
 
-    // e. consume the stages in order; one barrier per stage releases its slot
+    // e. consume the stages in order; one barrier per stage releases its slot.
+    // ldmatrix lanes: 0-7 rows 0-7 at column c, 8-15 rows 0-7 at column c + 8,
+    // 16-31 the same for the warp's next k step (or output tile)
+    const uint32_t lrow = (uint32_t)((lane & 7) * RS + 16 * ((lane >> 3) & 1) + 32 * warp);
+    const uint32_t xsl = smem_u32(sm + L.xs) + lrow;
+    const uint32_t hi_off = (lane >> 4) ? 32u * RW_WARPS : 0u;  // lanes 16-31: the next k step / tile
     for (int g = 0; g < n_groups; ++g) {
       const int n0 = g * RW_G, nn = min(RW_G, Lc - n0);
-      float cu[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
+      uint32_t bh = 0u, bl = 0u;  // h of the group as the down product's B fragment (hi, lo)
 #pragma unroll
-      for (int st = 0; st < 2 * RW_MAXC; ++st) {
-        const bool up = st < RW_MAXC;
-        const int ch = up ? st : st - RW_MAXC;
-        if (ch >= nchunk) continue;
-        const int q = g * spg + (up ? ch : nchunk + ch);
-        const int gs = sbase + q, slot = gs % RW_NS;
-        const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / RW_NS) & 1), abort_flag, a.status);
-        const uint32_t sbs = ring_s + (uint32_t)(slot * SB);
-        if (ok && up) {
-          // A rows = the 16 neurons; lane supplies row (lane & 7) + 8((lane >> 3) & 1)
-          const uint32_t arow = sbs + (uint32_t)(((lane & 7) + 8 * ((lane >> 3) & 1)) * RS);
+      for (int ud = 0; ud < 2; ++ud) {
+        const int q = 2 * g + ud;
+        const int gs = sbase + q, slot = gs % ns;
+        const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
+        const uint32_t sbs = ring_s + (uint32_t)(slot * SB) + lrow;
+        if (ud == 0) {
+          // up: u^T[token][neuron] partial over this warp's k steps
+          float cu[4] = {0.f, 0.f, 0.f, 0.f};
+          if (ok) {
 #pragma unroll
-          for (int j = 0; j < RW_MAXJ; ++j) {
-            const int kk = 16 * (warp + RW_WARPS * j);        // chunk-local k
-            if (ch * RW_CHUNK + kk < d) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4(arow + (kk + 8 * (lane >> 4)) * 2, a0, a1, a2, a3);
-              mma_bf16_16816(cu, a0, a1, a2, a3, xb[ch][j][0], xb[ch][j][1]);
+            for (int j = 0; j < RW_MAXJ; j += 2) {
+              if (j < nj) {
+                const uint32_t off = 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u);
+                uint32_t x0, x1, x2, x3, b0, b1, b2, b3;
+                ldsm_x4(xsl + off, x0, x1, x2, x3);
+                ldsm_x4(sbs + off, b0, b1, b2, b3);
+                mma_bf16_16816(cu, x0, 0u, x1, 0u, b0, b1);
+                if (j + 1 < nj) mma_bf16_16816(cu, x2, 0u, x3, 0u, b2, b3);
+              }
             }
           }
-        } else if (ok) {
-          // A = stored [neuron k][d] rows; lane supplies k = (lane & 7) + 8(lane >> 4)
-          const uint32_t krow = sbs + (uint32_t)(((lane & 7) + 8 * (lane >> 4)) * RS);
-          const int moff = 8 * ((lane >> 3) & 1);
+          ured[warp * 32 + lane] = make_float2(cu[0], cu[1]);
+          __syncthreads();
+          issue_stage(q + ns);  // the W_up slot is free
+          if (q + ns < n_stages) issued_end = sbase + q + ns + 1;
+          // h for (token lane/4, neurons 2(lane%4) and +1): the sum of the 16
+          // warps' partials at this lane's own fragment position
+          const int tn = lane >> 2, r0 = 2 * (lane & 3);
+          float u0 = 0.f, u1 = 0.f;
 #pragma unroll
-          for (int j = 0; j < RW_MAXJ; ++j) {
-            const int mm = 16 * (warp + RW_WARPS * j);        // chunk-local output row
-            if (ch * RW_CHUNK + mm < d) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4_t(krow + (mm + moff) * 2, a0, a1, a2, a3);
-              mma_bf16_16816(acc[ch][j], a0, a1, a2, a3, bh0, bh1);
-              mma_bf16_16816(acc[ch][j], a0, a1, a2, a3, bl0, bl1);
-            }
+          for (int w = 0; w < RW_WARPS; ++w) {
+            const float2 v = ured[w * 32 + lane];
+            u0 += v.x;
+            u1 += v.y;
           }
-        }
-        const bool last_up = up && ch == nchunk - 1;
-        if (last_up) ured[warp * 32 + lane] = make_float4(cu[0], cu[1], cu[2], cu[3]);
-        __syncthreads();
-        // the slot is free: refill it with the stage RW_NS ahead
-        issue_stage(q + RW_NS);
-        if (sbase + q + RW_NS < sbase + n_stages) issued_end = sbase + q + RW_NS + 1;
-        if (last_up) {
-          // h for the group: lane needs neurons k0 = 2(l&3) (+1, +8, +9) of token l>>2;
-          // element (row r, col c) of a warp's partial lives in lane 4(r&7) + (c>>1),
-          // register (c&1) + 2(r>>3)
-          const int tn = lane >> 2, k0 = 2 * (lane & 3);
-          float hv[4];
+          float hv[2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = k0 + (e & 1) + 8 * (e >> 1);
-            const float* pu = reinterpret_cast<const float*>(ured) + (4 * (r & 7) + (tn >> 1)) * 4 + (tn & 1) +
-                              2 * (r >> 3);
-            float u = 0.f;
-#pragma unroll
-            for (int w = 0; w < RW_WARPS; ++w) u += pu[w * 128];
-            const int n = n0 + r;
+          for (int e = 0; e < 2; ++e) {
+            const int r = r0 + e, n = n0 + r;
             float h = 0.f;
             if (r < nn && ((lmask[n] >> tn) & 1u)) {
               const float v = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(&lval[n])[tn] << 16);
-              h = v * u;
+              h = v * (e ? u1 : u0);
             }
             hv[e] = h;
           }
-          uint32_t hb[4], lb[4];
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(hv[0]), h1 = __float2bfloat16_rn(hv[1]);
+          bh = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          bl = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[0] - __bfloat162float(h0))) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[1] - __bfloat162float(h1))) << 16);
+        } else {
+          // down: y^T[d][token] += W_down rows^T · h over the 8 neurons
+          if (ok) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat16 hi = __float2bfloat16_rn(hv[e]);
-            hb[e] = (uint32_t)__bfloat16_as_ushort(hi);
-            lb[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[e] - __bfloat162float(hi)));
+            for (int j = 0; j < RW_MAXJ; j += 2) {
+              if (j < nj) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(sbs + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), a0, a1, a2, a3);
+                mma_bf16_1688(acc[j], a0, a1, bh);
+                mma_bf16_1688(acc[j], a0, a1, bl);
+                if (j + 1 < nj) {
+                  mma_bf16_1688(acc[j + 1], a2, a3, bh);
+                  mma_bf16_1688(acc[j + 1], a2, a3, bl);
+                }
+              }
+            }
           }
-          bh0 = hb[0] | (hb[1] << 16);
-          bh1 = hb[2] | (hb[3] << 16);
-          bl0 = lb[0] | (lb[1] << 16);
-          bl1 = lb[2] | (lb[3] << 16);
-          __syncthreads();  // every warp has read the partials before the next group writes them
+          __syncthreads();
+          issue_stage(q + ns);  // the W_down slot is free
+          if (q + ns < n_stages) issued_end = sbase + q + ns + 1;
         }
       }
     }
@@ -432,10 +436,14 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   }
   // drain copies still in flight (only after an abort): the last fill of every slot
   if (tid == 0 && *abort_flag) {
-    for (int k = 0; k < RW_NS && k < issued_end; ++k) {
+    const uint64_t tx = globaltimer();
+    while (!mbar_try_wait(xbar, 0u)) {
+      if (globaltimer() - tx > SFFN_WAIT_LIMIT_NS) break;
+    }
+    for (int k = 0; k < ns && k < issued_end; ++k) {
       const int last = issued_end - 1 - k;
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&full[last % RW_NS], (uint32_t)((last / RW_NS) & 1))) {
+      while (!mbar_try_wait(&full[last % ns], (uint32_t)((last / ns) & 1))) {
         if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) break;
       }
     }
@@ -443,21 +451,22 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   __syncthreads();
   const bool okall = !*abort_flag;
 
-  // 4. partial y -> red[8][d] (fp32, in the free ring), then out
-  float* red = reinterpret_cast<float*>(ring);
+  // 4. partial y -> red[8][d] (fp32, over the x rows and the free ring; rows
+  // padded by 4 floats, so that the four token rows a warp writes at once
+  // fall in different banks), then out
+  const int RP = d + 4, n4p = RP >> 2;
+  float* red = reinterpret_cast<float*>(sm + L.xs);
 #pragma unroll
-  for (int c = 0; c < RW_MAXC; ++c)
-#pragma unroll
-    for (int j = 0; j < RW_MAXJ; ++j) {
-      const int row = c * RW_CHUNK + 16 * (warp + RW_WARPS * j) + (lane >> 2);
-      if (row < d) {
-        const int t = 2 * (lane & 3);
-        red[t * d + row] = acc[c][j][0];
-        red[(t + 1) * d + row] = acc[c][j][1];
-        red[t * d + row + 8] = acc[c][j][2];
-        red[(t + 1) * d + row + 8] = acc[c][j][3];
-      }
+  for (int j = 0; j < RW_MAXJ; ++j) {
+    const int row = 16 * (warp + RW_WARPS * j) + (lane >> 2);
+    if (j < nj) {
+      const int t = 2 * (lane & 3);
+      red[t * RP + row] = acc[j][0];
+      red[(t + 1) * RP + row] = acc[j][1];
+      red[t * RP + row + 8] = acc[j][2];
+      red[(t + 1) * RP + row + 8] = acc[j][3];
     }
+  }
   const uint32_t CS = cluster_nctarank();
   const int n4 = d >> 2;
   if (a.atomic && CS > 1) {
@@ -469,17 +478,35 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     const int q0 = (int)(n4 * rank / CS), q1 = (int)(n4 * (rank + 1) / CS);
     const int width = q1 - q0;
     const uint32_t red_s = smem_u32(red);
-    float4* slice = reinterpret_cast<float4*>(red + 8 * d);
-    for (int e0 = tid; e0 < 8 * width; e0 += blockDim.x) {
-      const int t = e0 / width, q = q0 + (e0 - t * width);
-      if (!((live >> t) & 1u)) continue;
-      const uint32_t off = (uint32_t)((t * n4 + q) * 16);
-      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (uint32_t r = 0; r < CS; ++r) {
-        const float4 v = ld_shared_cluster_f4(mapa_shared(red_s + off, r));
-        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+    float4* slice = reinterpret_cast<float4*>(red + 8 * RP);
+    // four elements per thread per pass, all their remote loads issued before
+    // any is summed (each load is a cluster round trip)
+    constexpr int RW_MAXCS = 4;
+    for (int base = 0; base < 8 * width; base += 4 * RW_THREADS) {
+      float4 v[4][RW_MAXCS];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e0 = base + u * RW_THREADS + tid;
+        const int t = e0 / width, q = q0 + (e0 - t * width);
+        const bool use = e0 < 8 * width && ((live >> t) & 1u);
+        const uint32_t off = (uint32_t)((t * n4p + q) * 16);
+#pragma unroll
+        for (int r = 0; r < RW_MAXCS; ++r)
+          v[u][r] = use && r < (int)CS ? ld_shared_cluster_f4(mapa_shared(red_s + off, (uint32_t)r))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      slice[e0] = sum;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e0 = base + u * RW_THREADS + tid;
+        if (e0 < 8 * width) {
+          float4 sum = v[u][0];
+#pragma unroll
+          for (int r = 1; r < RW_MAXCS; ++r) {
+            sum.x += v[u][r].x; sum.y += v[u][r].y; sum.z += v[u][r].z; sum.w += v[u][r].w;
+          }
+          slice[e0] = sum;
+        }
+      }
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -493,7 +520,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     fence_proxy_async_smem();
     __syncthreads();
     if (tid < 8 && ((live >> tid) & 1u) && okall) {
-      bulk_reduce_add_f32(a.out + (size_t)(tb0 + tid) * d, red + tid * d, (uint32_t)d * 4u);
+      bulk_reduce_add_f32(a.out + (size_t)(tb0 + tid) * d, red + tid * RP, (uint32_t)d * 4u);
       bulk_commit();
       bulk_wait_all();
     }
@@ -502,7 +529,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     for (int e = tid; e < 8 * n4; e += blockDim.x) {
       const int t = e / n4, q = e - t * n4;
       if (!((live >> t) & 1u) || !okall) continue;
-      reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d)[q] = reinterpret_cast<const float4*>(red)[t * n4 + q];
+      reinterpret_cast<float4*>(a.out + (size_t)(tb0 + t) * d)[q] = reinterpret_cast<const float4*>(red)[t * n4p + q];
     }
   }
 }

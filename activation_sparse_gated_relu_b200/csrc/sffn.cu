@@ -137,7 +137,7 @@ template <int BN, class Epi>
 cudaError_t launch_tc_bn(dim3 grid, cudaStream_t st, const CUtensorMap& a0, const CUtensorMap& b0,
                          const CUtensorMap& a1, const CUtensorMap& b1, const TcArgs& args,
                          const typename Epi::Params& ep) {
-  return launch_pdl(k_tc_gemm<BN, Epi>, grid, dim3(TC_THREADS), TcCfg<BN>::SMEM, st, 1, a0, b0, a1, b1, args, ep);
+  return launch_pdl(k_tc_gemm<BN, Epi>, grid, dim3(TC_THREADS), TcCfgOf<BN, Epi>::SMEM, st, 1, a0, b0, a1, b1, args, ep);
 }
 
 template <class Epi>
@@ -156,11 +156,11 @@ cudaError_t launch_tc(int BN, dim3 grid, cudaStream_t st, const CUtensorMap& a0,
 template <class Epi>
 cudaError_t set_tc_attrs() {
   cudaError_t e = cudaSuccess;
-  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<16, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<16>::SMEM);
-  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<32, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<32>::SMEM);
-  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<64, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<64>::SMEM);
-  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<128, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<128>::SMEM);
-  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<256, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<256>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<16, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfgOf<16, Epi>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<32, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfgOf<32, Epi>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<64, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfgOf<64, Epi>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<128, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfgOf<128, Epi>::SMEM);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gemm<256, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfgOf<256, Epi>::SMEM);
   return e;
 }
 
@@ -205,9 +205,10 @@ struct sffn_handle {
   int rows_nslot = 0, rows_lcap = 0, rows_smem = 0;
   int rows_cs = 1, rows_max_ctas = 0;  // cluster size of the split fused kernel, co-resident CTAs
   bool rows_ok = false;                // the fused row kernel supports this shape
-  __nv_bfloat16* zero_row = nullptr;   // 2 KB of zeros: row chunks of padding neurons
+  __nv_bfloat16* zero_row = nullptr;   // a row of zeros (>= 2 KB): W_down rows of padding neurons
   // stream-K gate (fewer neuron tiles than SMs, T <= 64): CTA count, partials, tickets
   int sk_grid = 0, sk_bn = 0;
+  int gate_stages = 0, down_stages = 0;  // ring depth of the gate and down tile kernels (0: all)
   float* skpart = nullptr;
   int* sktick = nullptr;
   // per-kernel timing (sffn_timing_begin/end)
@@ -379,7 +380,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     ok = ok && dalloc(&h->h_hi, T * F * 2);
     ok = ok && dalloc(&h->h_lo, T * F * 2);
     ok = ok && dalloc(&h->WdT, d * F * 2);
-    ok = ok && dalloc(&h->zero_row, 2048);
+    ok = ok && dalloc(&h->zero_row, std::max<size_t>(2048, d * 2));
   }
   if (h->wina) {
     ok = ok && dalloc(&h->scores, T * F * 4);
@@ -415,7 +416,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
   e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
-  if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, 2048, st);
+  if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, std::max<size_t>(2048, d * 2), st);
   if (h->sktick) e = e ? e : cudaMemsetAsync(h->sktick, 0, P * 4, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->zacc, 0, T * (size_t)h->R * 4, st);
@@ -469,14 +470,17 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     // fused up x down: ring slots and list capacity from the shared memory budget
     int max_smem = 0;
     cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    int lcap = 512;
-    while (lcap > 64 && RowsSmem::make(h->P, lcap).total > max_smem) lcap -= 64;
-    h->rows_nslot = RW_NS;
+    int lcap = 512, ns = RW_NSMAX;
+    auto fits = [&](int l, int n) { return RowsSmem::make(h->P, l, h->d, n).total <= max_smem; };
+    while (ns > 2 && !fits(lcap, ns)) --ns;
+    while (lcap > 64 && !fits(lcap, ns)) lcap -= 64;
+    h->rows_nslot = ns;
     h->rows_lcap = lcap;
-    h->rows_smem = RowsSmem::make(h->P, lcap).total;
-    // the ring doubles as the [8][d] fp32 partial-output buffer and its cluster slice
-    h->rows_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXC * RW_CHUNK &&
-                 (long long)RW_NS * RowsSmem::STAGE >= 48LL * h->d && h->P <= RW_THREADS &&
+    h->rows_smem = RowsSmem::make(h->P, lcap, h->d, ns).total;
+    // the x rows and the ring double as the [8][d] fp32 partial-output buffer and its cluster slice
+    h->rows_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV &&
+                 (long long)(ns + 1) * RowsSmem::stage(h->d) >= 32LL * (h->d + 4) + 16LL * h->d &&
+                 h->P <= RW_THREADS &&
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
     // largest cluster (4, else 2) whose co-resident CTAs still cover almost every SM
@@ -565,7 +569,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   const int m_tiles_down = cdiv(d, 128);
   const int est_rows_tiles = rows ? 1 : ntile_tok;
   const int kb_down = cdiv(F, 64);
-  const int sk_down = std::max(1, std::min(kb_down / 4, cdiv(h->n_sm, m_tiles_down * est_rows_tiles)));
+  const int sk_down = std::max(1, std::min(kb_down / 4, h->n_sm / (m_tiles_down * est_rows_tiles)));
 
   cudaError_t e = cudaSuccess;
   TwellParams tw;
@@ -612,6 +616,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   ga.kb_total[0] = gate_kb;
   ga.n_rows = T;
   ga.status = h->status;
+  ga.stages = h->gate_stages;
   if (rows && rows_split > 1) {  // the split fused kernel adds its partials into out
     ga.zero_out = reinterpret_cast<float4*>(out);
     ga.zero_n4 = (long long)T * d / 4;
@@ -744,10 +749,9 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   // ----------------------------------------------------- down projection
   {
     TcArgs da{};
-    da.n_phase = 2;
-    da.acc_same = 1;
+    da.n_phase = 1;  // each stage multiplies one W_down^T tile by h_hi and h_lo
     da.kb_total[0] = kb_down;
-    da.kb_total[1] = kb_down;
+    da.stages = h->down_stages;
     da.n_rows = T;
     da.n_rows_dev = rows ? h->ovf_count : nullptr;
     da.status = h->status;

@@ -25,10 +25,12 @@ constexpr int TC_BM = 128;           // rows per tile (TMEM lanes)
 constexpr int TC_BK = 64;            // bf16 elements per 128-byte swizzled row
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
 
-template <int BN>
+// NB = B operands per stage: 2 when one A tile multiplies two B tiles into
+// the same accumulator (the hi and lo halves of a split bf16 operand).
+template <int BN, int NB = 1>
 struct TcCfg {
   static constexpr int B_BYTES = BN * TC_BK * 2;
-  static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
+  static constexpr int STAGE_BYTES = TC_A_BYTES + NB * B_BYTES;
   static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
   static constexpr int EPI_SMEM = 9 * 1024;
@@ -49,7 +51,19 @@ struct TcArgs {
   int m_tiles;          // stream-K: M tiles of the flattened unit space
   float4* zero_out;     // if set, the CTAs zero zero_n4 float4 here (after the grid dependency)
   long long zero_n4;
+  int stages;           // ring stages in use (0: all that fit); fewer bound the bytes in flight
 };
+
+template <class E, class = void>
+struct epi_dual_b {
+  static constexpr bool value = false;
+};
+template <class E>
+struct epi_dual_b<E, decltype(void(E::DUAL_B))> {
+  static constexpr bool value = E::DUAL_B;
+};
+template <int BN, class Epi>
+using TcCfgOf = TcCfg<BN, epi_dual_b<Epi>::value ? 2 : 1>;
 
 template <class E, class = void>
 struct epi_streamk {
@@ -82,13 +96,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mB0,
           const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mB1,
           const TcArgs args, const typename Epi::Params ep) {
-  using Cfg = TcCfg<BN>;
-  constexpr int STAGES = Cfg::STAGES;
+  using Cfg = TcCfgOf<BN, Epi>;
+  constexpr bool DUAL = epi_dual_b<Epi>::value;  // phase 0 only: A · (B0 + B1) per stage
+  constexpr int NB = DUAL ? 2 : 1;
+  const int STAGES = args.stages > 0 && args.stages < Cfg::STAGES ? args.stages : Cfg::STAGES;
   constexpr uint32_t NCOLS = tmem_cols_for(Epi::N_ACC * BN);
   constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, BN);
   constexpr bool SKM = epi_streamk<Epi>::value;
   constexpr int NACCF = SKM ? Epi::N_ACC : 1;  // accumulator-complete barriers
-  static_assert(2 * STAGES * 8 + NACCF * 8 + 8 <= 256, "barrier area");
+  static_assert(2 * Cfg::STAGES * 8 + NACCF * 8 + 8 <= 256, "barrier area");
 
   const int m0 = blockIdx.x * TC_BM;
   const int n0 = blockIdx.y * BN;
@@ -137,7 +153,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&mA0);
     tma_prefetch_desc(&mB0);
-    if (args.n_phase > 1) {
+    if (args.n_phase > 1 || DUAL) {
       tma_prefetch_desc(&mA1);
       tma_prefetch_desc(&mB1);
     }
@@ -162,7 +178,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
           if (f > 0 && !mbar_wait(&empty[s], (f - 1) & 1, abort_flag, args.status)) break;
           mbar_expect_tx(&full[s], Cfg::STAGE_BYTES);
           tma_load_2d(sA + s * TC_A_BYTES, &mA0, &full[s], kb * TC_BK, p * TC_BM);
-          tma_load_2d(sB + s * Cfg::B_BYTES, &mB0, &full[s], kb * TC_BK, n0);
+          tma_load_2d(sB + s * NB * Cfg::B_BYTES, &mB0, &full[s], kb * TC_BK, n0);
+          if (DUAL) tma_load_2d(sB + (s * NB + 1) * Cfg::B_BYTES, &mB1, &full[s], kb * TC_BK, n0);
         }
         ok = false;  // the phase loop below is for the tiled modes
       }
@@ -179,7 +196,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
           }
           mbar_expect_tx(&full[s], Cfg::STAGE_BYTES);
           tma_load_2d(sA + s * TC_A_BYTES, ma, &full[s], kb * TC_BK, m0);
-          tma_load_2d(sB + s * Cfg::B_BYTES, mb, &full[s], kb * TC_BK, n0);
+          tma_load_2d(sB + s * NB * Cfg::B_BYTES, mb, &full[s], kb * TC_BK, n0);
+          if (DUAL) tma_load_2d(sB + (s * NB + 1) * Cfg::B_BYTES, &mB1, &full[s], kb * TC_BK, n0);
         }
       }
       // Drain: the last fill of every stage has landed before the CTA can exit.
@@ -218,10 +236,13 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
           }
           tc_fence_after();
           const uint64_t ad = sdesc_k_sw128(smem_u32(sA + s * TC_A_BYTES));
-          const uint64_t bd = sdesc_k_sw128(smem_u32(sB + s * Cfg::B_BYTES));
+          const uint64_t bd = sdesc_k_sw128(smem_u32(sB + s * NB * Cfg::B_BYTES));
+          const uint64_t bd1 = sdesc_k_sw128(smem_u32(sB + (s * NB + 1) * Cfg::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < TC_BK / 16; ++k)
+          for (int k = 0; k < TC_BK / 16; ++k) {
             tc_mma(tmem + (uint32_t)(piece * BN), ad + 2u * k, bd + 2u * k, IDESC, (first && k == 0) ? 0u : 1u);
+            if (DUAL) tc_mma(tmem + (uint32_t)(piece * BN), ad + 2u * k, bd1 + 2u * k, IDESC, 1u);
+          }
           first = false;
           tc_commit(&empty[s]);
         }
@@ -239,10 +260,12 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
           }
           tc_fence_after();
           const uint64_t ad = sdesc_k_sw128(smem_u32(sA + s * TC_A_BYTES));
-          const uint64_t bd = sdesc_k_sw128(smem_u32(sB + s * Cfg::B_BYTES));
+          const uint64_t bd = sdesc_k_sw128(smem_u32(sB + s * NB * Cfg::B_BYTES));
+          const uint64_t bd1 = sdesc_k_sw128(smem_u32(sB + (s * NB + 1) * Cfg::B_BYTES));
 #pragma unroll
           for (int k = 0; k < TC_BK / 16; ++k) {
             tc_mma(tmem + dcol, ad + 2u * k, bd + 2u * k, IDESC, (first && k == 0) ? 0u : 1u);
+            if (DUAL) tc_mma(tmem + dcol, ad + 2u * k, bd1 + 2u * k, IDESC, 1u);
           }
           first = false;
           tc_commit(&empty[s]);
