@@ -32,9 +32,10 @@
 //         (m16n8k8, the 8 neurons as K) -- warp w owns every 16th 16-row
 //         output tile, held in registers for the whole CTA.
 // At the end the per-CTA partial y goes to out: plain stores when one CTA
-// owns the block, otherwise summed over the CTAs of a thread-block cluster
-// through distributed shared memory (each CTA of the cluster owns one column
-// slice) and added into out by bulk reduce-add copies, one per live token.
+// owns the block, otherwise bulk reduce-add copies, one per live token, that
+// the bulk-copy engine adds into out at L2.  (Summing first over a
+// thread-block cluster through distributed shared memory measured slower:
+// its remote loads ran at about 40 GB/s per SM.)
 #pragma once
 
 #include "ptx.cuh"
@@ -467,56 +468,9 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       red[(t + 1) * RP + row + 8] = acc[j][3];
     }
   }
-  const uint32_t CS = cluster_nctarank();
   const int n4 = d >> 2;
-  if (a.atomic && CS > 1) {
-    // the cluster's CTAs sum their partials over distributed shared memory,
-    // each one column slice, into a slice buffer behind red; the bulk-copy
-    // engine then adds each live token's slice row into out at L2
-    cluster_sync();
-    const uint32_t rank = cluster_ctarank();
-    const int q0 = (int)(n4 * rank / CS), q1 = (int)(n4 * (rank + 1) / CS);
-    const int width = q1 - q0;
-    const uint32_t red_s = smem_u32(red);
-    float4* slice = reinterpret_cast<float4*>(red + 8 * RP);
-    // four elements per thread per pass, all their remote loads issued before
-    // any is summed (each load is a cluster round trip)
-    constexpr int RW_MAXCS = 4;
-    for (int base = 0; base < 8 * width; base += 4 * RW_THREADS) {
-      float4 v[4][RW_MAXCS];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e0 = base + u * RW_THREADS + tid;
-        const int t = e0 / width, q = q0 + (e0 - t * width);
-        const bool use = e0 < 8 * width && ((live >> t) & 1u);
-        const uint32_t off = (uint32_t)((t * n4p + q) * 16);
-#pragma unroll
-        for (int r = 0; r < RW_MAXCS; ++r)
-          v[u][r] = use && r < (int)CS ? ld_shared_cluster_f4(mapa_shared(red_s + off, (uint32_t)r))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e0 = base + u * RW_THREADS + tid;
-        if (e0 < 8 * width) {
-          float4 sum = v[u][0];
-#pragma unroll
-          for (int r = 1; r < RW_MAXCS; ++r) {
-            sum.x += v[u][r].x; sum.y += v[u][r].y; sum.z += v[u][r].z; sum.w += v[u][r].w;
-          }
-          slice[e0] = sum;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid < 8 && ((live >> tid) & 1u) && okall) {
-      bulk_reduce_add_f32(a.out + (size_t)(tb0 + tid) * d + 4 * q0, slice + tid * width, (uint32_t)width * 16u);
-      bulk_commit();
-      bulk_wait_all();
-    }
-    cluster_sync();
-  } else if (a.atomic) {
+  if (a.atomic) {
+    // the bulk-copy engine adds each live token's partial row into out at L2
     fence_proxy_async_smem();
     __syncthreads();
     if (tid < 8 && ((live >> tid) & 1u) && okall) {

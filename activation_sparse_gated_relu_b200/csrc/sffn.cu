@@ -203,7 +203,6 @@ struct sffn_handle {
   CUtensorMap tmWgate, tmWup, tmWdT, tmAt, tmBt;
   int last_T = 0, last_path = 0, last_launches = 0;
   int rows_nslot = 0, rows_lcap = 0, rows_smem = 0;
-  int rows_cs = 1, rows_max_ctas = 0;  // cluster size of the split fused kernel, co-resident CTAs
   bool rows_ok = false;                // the fused row kernel supports this shape
   __nv_bfloat16* zero_row = nullptr;   // a row of zeros (>= 2 KB): W_down rows of padding neurons
   // stream-K gate (fewer neuron tiles than SMs, T <= 64): CTA count, partials, tickets
@@ -477,38 +476,12 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     h->rows_nslot = ns;
     h->rows_lcap = lcap;
     h->rows_smem = RowsSmem::make(h->P, lcap, h->d, ns).total;
-    // the x rows and the ring double as the [8][d] fp32 partial-output buffer and its cluster slice
+    // the x rows and the ring double as the [8][d] fp32 partial-output buffer
     h->rows_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV &&
-                 (long long)(ns + 1) * RowsSmem::stage(h->d) >= 32LL * (h->d + 4) + 16LL * h->d &&
+                 (long long)(ns + 1) * RowsSmem::stage(h->d) >= 32LL * (h->d + 4) &&
                  h->P <= RW_THREADS &&
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
-    // largest cluster (4, else 2) whose co-resident CTAs still cover almost every SM
-    h->rows_cs = 1;
-    h->rows_max_ctas = h->n_sm;
-    for (int cs = 4; cs >= 2 && !e; cs /= 2) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((h->n_sm / cs) * cs, 1, 1);
-      cfg.blockDim = dim3(RW_THREADS, 1, 1);
-      cfg.dynamicSmemBytes = h->rows_smem;
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = cs;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int ncl = 0;
-      if (cudaOccupancyMaxActiveClusters(&ncl, k_rows, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        continue;
-      }
-      if (ncl * cs >= h->n_sm - 8) {
-        h->rows_cs = cs;
-        h->rows_max_ctas = ncl * cs;
-        break;
-      }
-    }
   }
   if (!e && h->wina) {
     const int tk_smem = (int)(F * 4 + 32 * 256 * 4 + P * 4);
@@ -559,12 +532,6 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   const bool rows = path == SFFN_PATH_ROWS;
   const int nblk = cdiv(T, 8);
   int rows_split = rows ? std::max(1, h->n_sm / nblk) : 1;
-  int rows_cs = 1;
-  if (rows_split > 1) {  // split blocks: clusters of rows_cs CTAs, all resident at once
-    rows_cs = h->rows_cs;
-    rows_split = std::min(rows_split, std::max(1, h->rows_max_ctas / nblk));
-    rows_split = std::max(rows_cs, (rows_split / rows_cs) * rows_cs);
-  }
   // down projection split over d_ff so that its grid covers the SMs
   const int m_tiles_down = cdiv(d, 128);
   const int est_rows_tiles = rows ? 1 : ntile_tok;
@@ -703,7 +670,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     rw.status = h->status;
     tmark(h, st, L_UPDOWN_ROWS);
     ++launches;
-    if (launch_pdl(k_rows, dim3(rows_split, nblk, 1), dim3(RW_THREADS), (size_t)h->rows_smem, st, rows_cs, rw))
+    if (launch_pdl(k_rows, dim3(rows_split, nblk, 1), dim3(RW_THREADS), (size_t)h->rows_smem, st, 1, rw))
       return SFFN_ERR_CUDA;
   } else {
     TcArgs ua{};
