@@ -92,79 +92,109 @@ __device__ __forceinline__ void twell_chunk(const TwellParams& o, const float* g
   }
 }
 
+// TwELL emission for one 128-neuron tile and up to 32 tokens t0..t0+31 (bf16
+// values), by the 128 threads of four full warps.  It is the same format as
+// twell_chunk, but its phases keep every thread busy and write whole records:
+//   1. thread = neuron: activation, keep bit, bf16 value into a staging
+//      block; warp ballots give each token's 128-bit keep mask;
+//   2. four threads per token, one per 32-bit mask word: each ranks its kept
+//      neurons after the lower words' counts.  The first C ranks go to the
+//      token's staged record (ascending neuron order); pads fill slots at or
+//      after the count.  Count, overflow epoch and keep mask are written
+//      here;
+//   3. the staged [32][C] idx and val records go out as 16-byte vectors.
+// (Thread-per-neuron stores of 2-byte slots kept one warp per scheduler
+// waiting on dependent latencies and flooded L2 with partial writes.)
+constexpr int TW32_VP = 128 + 8;   // padded staged-value row (bf16 elements)
+__host__ __device__ constexpr int twell32_smem(int C) { return 32 * 4 * 4 + 32 * TW32_VP * 2 + 32 * C * 2 * 2; }
+
+__device__ __forceinline__ void twell_tile32(const TwellParams& o, const float* g, int j, int t0, int etid,
+                                             uint8_t* scratch, uint32_t bar_id) {
+  const int w = etid >> 5, lane = etid & 31;
+  const int p = j >> 7, n_in = j & 127;
+  const int C = o.C;
+  uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);                         // [32 tokens][4]
+  uint16_t* vals = reinterpret_cast<uint16_t*>(scratch + 32 * 4 * 4);             // [32][TW32_VP]
+  uint16_t* sidx = reinterpret_cast<uint16_t*>(scratch + 32 * 4 * 4 + 32 * TW32_VP * 2);  // [32][C]
+  uint16_t* sval = sidx + 32 * C;                                                  // [32][C]
+  const float b = o.bias ? o.bias[j] : 0.0f;
+  // 1. thread = neuron
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float gv = g[i] + b;
+    const float a = act_fn(gv, o.act);
+    const bool in = (t0 + i) < o.T;
+    const bool k = in && fabsf(a) > o.tau;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, k);
+    if (lane == 0) masks[i * 4 + w] = bal;
+    vals[i * TW32_VP + n_in] = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+    if (o.gdebug && in) o.gdebug[(size_t)(t0 + i) * o.F + j] = gv;
+  }
+  named_bar_sync(bar_id, 128);
+  // 2. four threads per token
+  {
+    const int tt = etid >> 2, wq = etid & 3, t = t0 + tt;
+    const uint4 m4 = reinterpret_cast<const uint4*>(masks)[tt];
+    const int c0 = __popc(m4.x), c1 = __popc(m4.y), c2 = __popc(m4.z), c3 = __popc(m4.w);
+    const int total = c0 + c1 + c2 + c3;
+    int rank = (wq > 0 ? c0 : 0) + (wq > 1 ? c1 : 0) + (wq > 2 ? c2 : 0);
+    uint32_t m = wq == 0 ? m4.x : wq == 1 ? m4.y : wq == 2 ? m4.z : m4.w;
+    const int q = C >> 2;  // pad slots this thread owns: [wq q, (wq + 1) q)
+    for (int sl = wq * q; sl < (wq + 1) * q; ++sl)
+      if (sl >= total) {
+        sidx[tt * C + sl] = 0xFFFFu;   // -1
+        sval[tt * C + sl] = 0u;        // +0
+      }
+    while (m != 0u && rank < C) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1u;
+      const int n = wq * 32 + bit;
+      sidx[tt * C + rank] = (uint16_t)(p * 128 + n);
+      sval[tt * C + rank] = vals[tt * TW32_VP + n];
+      ++rank;
+    }
+    if (wq == 0 && t < o.T) {
+      o.count[(size_t)t * o.n_tiles + p] = (int16_t)total;
+      if (total > C) o.ovf[t] = o.epoch;
+      if (o.kmask) reinterpret_cast<uint4*>(o.kmask)[(size_t)t * o.n_tiles + p] = m4;
+    }
+  }
+  named_bar_sync(bar_id, 128);
+  // 3. whole records out, 8 slots per 16-byte vector
+  {
+    const int nvec = C >> 3;
+    for (int e = etid; e < 2 * 32 * nvec; e += 128) {
+      const int arr = e / (32 * nvec), r = e - arr * 32 * nvec;
+      const int tt = r / nvec, v = r - tt * nvec, t = t0 + tt;
+      if (t >= o.T) continue;
+      const uint4 val = reinterpret_cast<const uint4*>((arr ? sval : sidx) + tt * C)[v];
+      uint16_t* dst = arr ? reinterpret_cast<uint16_t*>(o.val) : reinterpret_cast<uint16_t*>(o.idx);
+      reinterpret_cast<uint4*>(dst + ((size_t)t * o.n_tiles + p) * C)[v] = val;
+    }
+  }
+  named_bar_sync(bar_id, 128);  // the staging is free for the next call
+}
+
 struct EpiGateTwell {
   static constexpr int N_ACC = 1;
+  static constexpr int EPI_SMEM = twell32_smem(128);
   using Params = TwellParams;
   template <int BN>
   __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t* scratch) {
-    uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);
     const int j = m0 + etid;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = 0; c < BN; c += 32) {
       if (n0 + c >= o.T) break;
-      float g[16];
+      float g[32];
       tmem_ld16(tmem + c, g);
-      twell_chunk(o, g, j, n0 + c, etid, masks + ((c >> 4) & 1) * 64);
-    }
-  }
-};
-
-// Stream-K gate: a tile whose K blocks are shared by n_pieces CTAs.  Each
-// CTA stores its fp32 partial of the 128 x BN tile in its piece slot, and the
-// CTA that completes the tile's ticket adds the pieces in ascending K order
-// (the same order on every forward, so the sum is reproducible) and emits
-// TwELL from the sum.  A tile held by one CTA goes straight to TwELL.
-constexpr int SK_MAX_PIECES = 4;  // CTAs that may share one tile
-
-struct GateSKParams {
-  TwellParams tw;
-  float* part;   // [tiles x token tiles][SK_MAX_PIECES][BN][128] fp32
-  int* tick;     // [tiles x token tiles], zero between forwards
-};
-
-struct EpiGateTwellSK {
-  static constexpr int N_ACC = 2;  // a CTA's range touches at most two tiles
-  static constexpr bool STREAMK = true;
-  using Params = GateSKParams;
-  template <int BN>
-  __device__ static void run_piece(const Params& o, uint32_t tmem, int m0, int n0, int piece, int n_pieces,
-                                   int etid, uint8_t* scratch) {
-    if (n_pieces == 1) {
-      named_bar_sync(1, 128);  // an earlier piece's threads are done with the masks
-      EpiGateTwell::run<BN>(o.tw, tmem, m0, n0, 0, etid, scratch);
-      return;
-    }
-    const int slot = (m0 >> 7) * (int)gridDim.y + (int)blockIdx.y;
-    float* base = o.part + (size_t)slot * SK_MAX_PIECES * BN * 128;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      if (n0 + c >= o.tw.T) break;
-      float g[16];
-      tmem_ld16(tmem + c, g);
+      if (BN > 16) {
+        tmem_ld16(tmem + c + 16, g + 16);
+      } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) __stcg(&base[((size_t)piece * BN + c + i) * 128 + etid], g[i]);
-    }
-    int* last = reinterpret_cast<int*>(scratch + 1024);
-    __threadfence();
-    named_bar_sync(1, 128);
-    if (etid == 0) *last = atomicAdd(&o.tick[slot], 1) == n_pieces - 1;
-    named_bar_sync(1, 128);
-    if (!*last) return;
-    __threadfence();
-    uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      if (n0 + c >= o.tw.T) break;
-      float g[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) g[i] = __ldcg(&base[(size_t)(c + i) * 128 + etid]);
-      for (int q = 1; q < n_pieces; ++q) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) g[i] += __ldcg(&base[((size_t)q * BN + c + i) * 128 + etid]);
+        for (int i = 16; i < 32; ++i) g[i] = 0.f;
       }
-      twell_chunk(o.tw, g, m0 + etid, n0 + c, etid, masks + ((c >> 4) & 1) * 64);
+      twell_tile32(o, g, j, n0 + c, etid, scratch, 1);
     }
-    if (etid == 0) o.tick[slot] = 0;
   }
 };
 

@@ -5,7 +5,8 @@
 //   gate    tensor-core tile kernel, epilogue = TwELL emission (threshold) or
 //           dense value + score (WINA, then the top-k kernel emits TwELL);
 //           low-rank gate = two tile kernels (z = bf16(x·A) split over K, then
-//           g = z·B with the TwELL epilogue, stream-K over the SMs)
+//           g = z·B with the TwELL epilogue); up to 8 tokens: a row-streaming
+//           gate over every SM with the same epilogue
 //   router  (TILES only) overflow list, gathers, output zeroing
 //   ROWS    fused up x down over the kept rows of each 8-token block
 //           (non-overflow tokens; the kernel also routes the overflow tokens,
@@ -28,6 +29,7 @@
 
 #include "../../include/sffn.h"
 #include "epilogues.cuh"
+#include "gate_rows.cuh"
 #include "rows_mma.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -82,25 +84,6 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows,
 
 int pick_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
-
-// Stream-K grid for a GEMM of m_tiles tiles x kb K blocks: the largest CTA
-// count up to n_sm (and above m_tiles) whose ranges hold at most kb units, so
-// that a CTA touches at most two tiles, and that splits no tile over more
-// than max_pieces CTAs.  0 if there is none.
-int streamk_grid(int m_tiles, int kb, int n_sm, int max_pieces) {
-  const long long U = (long long)m_tiles * kb;
-  for (int G = n_sm; G > m_tiles; --G) {
-    if (U < G || cdiv(U, G) > kb) continue;
-    bool ok = true;
-    for (int p = 0; p < m_tiles && ok; ++p) {
-      const int sa = streamk_owner((long long)p * kb, U, G);
-      const int sb = streamk_owner((long long)p * kb + kb - 1, U, G);
-      ok = sb - sa + 1 <= max_pieces;
-    }
-    if (ok) return G;
-  }
-  return 0;
-}
 
 // Launch with programmatic dependent launch: the kernel may be scheduled while
 // the previous kernel on the stream drains; it calls griddepcontrol.wait before
@@ -205,11 +188,12 @@ struct sffn_handle {
   int rows_nslot = 0, rows_lcap = 0, rows_smem = 0;
   bool rows_ok = false;                // the fused row kernel supports this shape
   __nv_bfloat16* zero_row = nullptr;   // a row of zeros (>= 2 KB): W_down rows of padding neurons
-  // stream-K gate (fewer neuron tiles than SMs, T <= 64): CTA count, partials, tickets
-  int sk_grid = 0, sk_bn = 0;
   int gate_stages = 0, down_stages = 0;  // ring depth of the gate and down tile kernels (0: all)
-  float* skpart = nullptr;
-  int* sktick = nullptr;
+  // row-streaming gate for up to 8 tokens: tile staging, tickets, ring slots, shared memory
+  float* gstage = nullptr;
+  int* gtick = nullptr;
+  int gr_nslot = 0, gr_smem = 0;
+  bool gr_ok = false;
   // per-kernel timing (sffn_timing_begin/end)
   bool tm_on = false;
   int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
@@ -228,7 +212,7 @@ void free_handle(sffn_handle* h) {
   void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zacc,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->zero_row, h->skpart, h->sktick};
+                  h->zero_row, h->gstage, h->gtick};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -396,16 +380,9 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     ok = ok && dalloc(&h->Bt, F * R * 2);
   }
   if (desc->flags & SFFN_FLAG_DEBUG_GATE) ok = ok && dalloc(&h->gdebug, T * F * 4);
-  // stream-K gate for the low-rank second GEMM (short K): with the dense gate's
-  // long K, one CTA per tile streams W_gate faster than split tiles do
-  if (!h->f32 && !h->wina && h->lowrank && (int)P < h->n_sm) {
-    const int gate_kb = cdiv(h->R, 64);
-    h->sk_grid = streamk_grid((int)P, gate_kb, h->n_sm, SK_MAX_PIECES);
-    if (h->sk_grid) {
-      h->sk_bn = pick_bn((int)std::min<size_t>(T, 64));
-      ok = ok && dalloc(&h->skpart, P * SK_MAX_PIECES * (size_t)h->sk_bn * 128 * 4);
-      ok = ok && dalloc(&h->sktick, P * 4);
-    }
+  if (!h->f32 && !h->wina && !h->lowrank) {
+    ok = ok && dalloc(&h->gstage, P * 8 * 128 * 4);
+    ok = ok && dalloc(&h->gtick, P * 4);
   }
   if (!ok) {
     free_handle(h);
@@ -416,7 +393,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
   if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, std::max<size_t>(2048, d * 2), st);
-  if (h->sktick) e = e ? e : cudaMemsetAsync(h->sktick, 0, P * 4, st);
+  if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->zacc, 0, T * (size_t)h->R * 4, st);
     e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * (T / 16 + 2) * 4, st);
@@ -448,7 +425,6 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   // kernel attributes and A-operand tensor maps
   if (!e && !h->f32) {
     e = e ? e : set_tc_attrs<EpiGateTwell>();
-    e = e ? e : set_tc_attrs<EpiGateTwellSK>();
     e = e ? e : set_tc_attrs<EpiWina>();
     e = e ? e : set_tc_attrs<EpiLowRankZ>();
     e = e ? e : set_tc_attrs<EpiFallbackH>();
@@ -482,6 +458,15 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
                  h->P <= RW_THREADS &&
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
+    // row-streaming gate: the same staged-row layout, as many ring slots as fit
+    if (h->gstage) {
+      const int gns = 2;
+      h->gr_nslot = gns;
+      h->gr_smem = GateRowsSmem::make(h->d, gns).total;
+      h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem;
+      if (h->gr_ok)
+        e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->gr_smem);
+    }
   }
   if (!e && h->wina) {
     const int tk_smem = (int)(F * 4 + 32 * 256 * 4 + P * 4);
@@ -601,11 +586,21 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
       return SFFN_ERR_CUDA;
   } else {
     tmark(h, st, L_GATE);
-    if (h->sk_grid && T <= 64) {
-      // fewer neuron tiles than SMs: spread the K blocks over every SM
-      ga.m_tiles = P;
-      GateSKParams sp{tw, h->skpart, h->sktick};
-      e = launch_tc<EpiGateTwellSK>(BN, dim3(h->sk_grid, 1, 1), st, *gateA, *gateB, *gateA, *gateB, ga, sp);
+    if (h->gr_ok && T <= 8) {
+      // up to 8 tokens: stream whole W_gate rows over every SM
+      GateRowsArgs gr{};
+      gr.x = static_cast<const __nv_bfloat16*>(x);
+      gr.W_gate = static_cast<const __nv_bfloat16*>(D.W_gate);
+      gr.tw = tw;
+      gr.gstage = h->gstage;
+      gr.tick = h->gtick;
+      gr.zero_out = ga.zero_out;
+      gr.zero_n4 = ga.zero_n4;
+      gr.d = d;
+      gr.nslot = h->gr_nslot;
+      gr.status = h->status;
+      e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS), (size_t)h->gr_smem, st, 1,
+                     gr);
     } else {
       e = launch_tc<EpiGateTwell>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, tw);
     }

@@ -2,12 +2,6 @@
 // TMEM -> epilogue.  One CTA computes D[128 x BN] = A[m0:m0+128, K] ·
 // B[n0:n0+BN, K]^T for one or two GEMM phases (two accumulators, or one that
 // both phases add into), over a K range that may be split across gridDim.z.
-// Stream-K mode (epilogues that declare STREAMK, one phase): the (M tile,
-// 64-wide K block) units are flattened and CTA x of gridDim.x takes the
-// contiguous range [U x / G, U (x+1) / G), so that a GEMM with fewer tiles
-// than SMs still streams its A operand through every SM; each M tile the
-// range touches is one accumulator piece, handed to the epilogue's
-// run_piece with its position among the CTAs that share the tile.
 //
 // Warp roles (192 threads): warps 0-3 run the epilogue (warp w reads TMEM
 // lanes 32w..32w+31, one accumulator row per thread), warp 4 issues the TMA
@@ -26,15 +20,18 @@ constexpr int TC_BK = 64;            // bf16 elements per 128-byte swizzled row
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
 
 // NB = B operands per stage: 2 when one A tile multiplies two B tiles into
-// the same accumulator (the hi and lo halves of a split bf16 operand).
-template <int BN, int NB = 1>
+// the same accumulator (the hi and lo halves of a split bf16 operand).  EPI =
+// the epilogue's shared scratch; the ring takes what is left of 227 KB.
+constexpr int TC_SMEM_BUDGET = 227 * 1024;
+template <int BN, int NB = 1, int EPI = 9 * 1024>
 struct TcCfg {
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = TC_A_BYTES + NB * B_BYTES;
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int EPI_SMEM = (EPI + 127) & ~127;
+  static constexpr int STAGES_RAW = (TC_SMEM_BUDGET - 1024 - 256 - EPI_SMEM) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 12 ? 12 : (STAGES_RAW < 2 ? 2 : STAGES_RAW);
-  static constexpr int EPI_SMEM = 9 * 1024;
   static constexpr int SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + EPI_SMEM;
+  static_assert(SMEM <= TC_SMEM_BUDGET, "shared memory budget");
 };
 
 __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
@@ -48,7 +45,6 @@ struct TcArgs {
   int n_rows;           // valid B rows (columns of D); CTAs with n0 >= n_rows exit
   const int* n_rows_dev;  // if set, the valid B row count is read from the device
   uint32_t* status;
-  int m_tiles;          // stream-K: M tiles of the flattened unit space
   float4* zero_out;     // if set, the CTAs zero zero_n4 float4 here (after the grid dependency)
   long long zero_n4;
   int stages;           // ring stages in use (0: all that fit); fewer bound the bytes in flight
@@ -62,22 +58,16 @@ template <class E>
 struct epi_dual_b<E, decltype(void(E::DUAL_B))> {
   static constexpr bool value = E::DUAL_B;
 };
-template <int BN, class Epi>
-using TcCfgOf = TcCfg<BN, epi_dual_b<Epi>::value ? 2 : 1>;
-
 template <class E, class = void>
-struct epi_streamk {
-  static constexpr bool value = false;
+struct epi_smem {
+  static constexpr int value = 9 * 1024;
 };
 template <class E>
-struct epi_streamk<E, decltype(void(E::STREAMK))> {
-  static constexpr bool value = E::STREAMK;
+struct epi_smem<E, decltype(void(E::EPI_SMEM))> {
+  static constexpr int value = E::EPI_SMEM;
 };
-
-// CTA of a stream-K grid (G CTAs over U units) whose range holds unit u
-__host__ __device__ __forceinline__ int streamk_owner(long long u, long long U, int G) {
-  return (int)(((u + 1) * G - 1) / U);
-}
+template <int BN, class Epi>
+using TcCfgOf = TcCfg<BN, epi_dual_b<Epi>::value ? 2 : 1, epi_smem<Epi>::value>;
 
 // Epilogue contract:
 //   struct Epi { struct Params; static constexpr int N_ACC;
@@ -85,11 +75,6 @@ __host__ __device__ __forceinline__ int streamk_owner(long long u, long long U, 
 //                                int split, int etid, uint8_t* scratch); };
 // run() is called by the 128 epilogue threads (etid 0..127) once the
 // accumulators are complete; accumulator a lives at TMEM column a*BN.
-// A stream-K epilogue (STREAMK = true, N_ACC = pieces a CTA may hold) has
-//   run_piece(const Params&, uint32_t tmem, int m0, int n0, int piece,
-//             int n_pieces, int etid, uint8_t* scratch)
-// called once per M tile of the CTA's range, in tile order: piece is the
-// CTA's rank among the n_pieces CTAs that share the tile (ascending K).
 
 template <int BN, class Epi>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -102,26 +87,13 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
   const int STAGES = args.stages > 0 && args.stages < Cfg::STAGES ? args.stages : Cfg::STAGES;
   constexpr uint32_t NCOLS = tmem_cols_for(Epi::N_ACC * BN);
   constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, BN);
-  constexpr bool SKM = epi_streamk<Epi>::value;
-  constexpr int NACCF = SKM ? Epi::N_ACC : 1;  // accumulator-complete barriers
-  static_assert(2 * Cfg::STAGES * 8 + NACCF * 8 + 8 <= 256, "barrier area");
+  static_assert(2 * Cfg::STAGES * 8 + 8 + 8 <= 256, "barrier area");
 
   const int m0 = blockIdx.x * TC_BM;
   const int n0 = blockIdx.y * BN;
   if (args.n_rows_dev) griddep_wait();  // the row count comes from an earlier kernel
   const int n_rows = args.n_rows_dev ? *args.n_rows_dev : args.n_rows;
   if (n0 >= n_rows) return;  // uniform: the whole CTA leaves before any setup
-  // stream-K range of this CTA: units [u0, u1), unit u = (tile u / KB, block u % KB)
-  const int KB0 = args.kb_total[0];
-  const long long U = SKM ? (long long)args.m_tiles * KB0 : 0;
-  const long long u0 = SKM ? U * blockIdx.x / gridDim.x : 0;
-  const long long u1 = SKM ? U * (blockIdx.x + 1) / gridDim.x : 0;
-  const int pfirst = SKM ? (int)(u0 / KB0) : 0;
-  const int n_piece = SKM ? (u1 > u0 ? (int)((u1 - 1) / KB0) - pfirst + 1 : 0) : 1;
-  if (SKM && (n_piece == 0 || n_piece > NACCF)) {  // the host never launches this
-    if (n_piece > NACCF && threadIdx.x == 0) atomicOr(args.status, DEV_ERR_RANGE);
-    return;
-  }
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,7 +102,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + NACCF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* scratch = smem + STAGES * Cfg::STAGE_BYTES + 256;
 
@@ -142,7 +114,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < NACCF; ++i) mbar_init(&accf[i], 1);
+    mbar_init(accf, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -171,18 +143,6 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       // ------------------------------------------------------- TMA producer
       int it = 0;
       bool ok = true;
-      if constexpr (SKM) {
-        for (long long u = u0; u < u1; ++u, ++it) {
-          const int p = (int)(u / KB0), kb = (int)(u - (long long)p * KB0);
-          const int s = it % STAGES, f = it / STAGES;
-          if (f > 0 && !mbar_wait(&empty[s], (f - 1) & 1, abort_flag, args.status)) break;
-          mbar_expect_tx(&full[s], Cfg::STAGE_BYTES);
-          tma_load_2d(sA + s * TC_A_BYTES, &mA0, &full[s], kb * TC_BK, p * TC_BM);
-          tma_load_2d(sB + s * NB * Cfg::B_BYTES, &mB0, &full[s], kb * TC_BK, n0);
-          if (DUAL) tma_load_2d(sB + (s * NB + 1) * Cfg::B_BYTES, &mB1, &full[s], kb * TC_BK, n0);
-        }
-        ok = false;  // the phase loop below is for the tiled modes
-      }
       for (int ph = 0; ph < args.n_phase && ok; ++ph) {
         const CUtensorMap* ma = ph == 0 ? &mA0 : &mA1;
         const CUtensorMap* mb = ph == 0 ? &mB0 : &mB1;
@@ -217,37 +177,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       // --------------------------------------------------------- MMA issuer
       int it = 0;
       bool ok = true;
-      int piece = 0;
-      if constexpr (SKM) {
-        int pcur = pfirst;
-        bool first = true;
-        for (long long u = u0; u < u1; ++u, ++it) {
-          const int p = (int)(u / KB0);
-          if (p != pcur) {  // the previous tile's piece is complete
-            tc_commit(&accf[piece]);
-            ++piece;
-            pcur = p;
-            first = true;
-          }
-          const int s = it % STAGES, f = it / STAGES;
-          if (!mbar_wait(&full[s], f & 1, abort_flag, args.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t ad = sdesc_k_sw128(smem_u32(sA + s * TC_A_BYTES));
-          const uint64_t bd = sdesc_k_sw128(smem_u32(sB + s * NB * Cfg::B_BYTES));
-          const uint64_t bd1 = sdesc_k_sw128(smem_u32(sB + (s * NB + 1) * Cfg::B_BYTES));
-#pragma unroll
-          for (int k = 0; k < TC_BK / 16; ++k) {
-            tc_mma(tmem + (uint32_t)(piece * BN), ad + 2u * k, bd + 2u * k, IDESC, (first && k == 0) ? 0u : 1u);
-            if (DUAL) tc_mma(tmem + (uint32_t)(piece * BN), ad + 2u * k, bd1 + 2u * k, IDESC, 1u);
-          }
-          first = false;
-          tc_commit(&empty[s]);
-        }
-      }
-      for (int ph = 0; ph < args.n_phase && ok && !SKM; ++ph) {
+      for (int ph = 0; ph < args.n_phase && ok; ++ph) {
         const uint32_t dcol = args.acc_same ? 0u : (uint32_t)(ph * BN);
         const int kb0 = (int)((long long)args.kb_total[ph] * sk / S);
         const int kb1 = (int)((long long)args.kb_total[ph] * (sk + 1) / S);
@@ -273,10 +203,10 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       }
       // An accumulator whose K range is empty stays unwritten: only happens
       // when the split exceeds the K blocks, which the host never launches.
-      tc_commit(&accf[piece]);
+      tc_commit(accf);
       if (!ok) {
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(&accf[piece], 0)) {
+        while (!mbar_try_wait(accf, 0)) {
           if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) break;
         }
       }
@@ -290,17 +220,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
         args.zero_out[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
-    if constexpr (SKM) {
-      for (int pi = 0; pi < n_piece; ++pi) {
-        if (!mbar_wait(&accf[pi], 0, abort_flag, args.status) || *abort_flag) break;
-        tc_fence_after();
-        const int p = pfirst + pi;
-        const int sa = streamk_owner((long long)p * KB0, U, (int)gridDim.x);
-        const int sb = streamk_owner((long long)p * KB0 + KB0 - 1, U, (int)gridDim.x);
-        Epi::template run_piece<BN>(ep, tlane + (uint32_t)(pi * BN), p * TC_BM, n0, (int)blockIdx.x - sa,
-                                    sb - sa + 1, threadIdx.x, scratch);
-      }
-    } else if (mbar_wait(accf, 0, abort_flag, args.status) && !*abort_flag) {
+    if (mbar_wait(accf, 0, abort_flag, args.status) && !*abort_flag) {
       tc_fence_after();
       Epi::template run<BN>(ep, tlane, m0, n0, sk, threadIdx.x, scratch);
     }
