@@ -246,57 +246,77 @@ struct EpiWina {
 
 // ------------------------------------------------------- low-rank gate: z
 // z = round_bf16(x·A).  The tile's rows are rank coordinates r, its columns
-// tokens.  With a split K the partial sums are added into zacc (fp32, zero
-// between forwards) and the last CTA of the row tile rounds, stores z and
-// clears zacc and its ticket.
+// tokens.  With a split K every CTA stores its fp32 partial in its split's
+// slot; the CTA that completes the tile's ticket adds the splits in
+// ascending K order (the same order on every forward, so z is reproducible),
+// rounds and stores z, and clears the ticket.
+constexpr int Z_MAX_SPLITS = 4;  // the last CTA's loads of every split go out at once
+
 struct ZParams {
   int T, R, splits;
-  float* zacc;             // [maxT][R]
+  float* zpart;            // [row tiles x token tiles][splits][BN][128] fp32 (splits > 1)
   __nv_bfloat16* z;        // [maxT][R]
-  int* tickets;            // [R/128]
+  int* tickets;            // [row tiles x token tiles], zero between forwards
 };
 
 struct EpiLowRankZ {
   static constexpr int N_ACC = 1;
   using Params = ZParams;
   template <int BN>
-  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t* scratch) {
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int split, int etid, uint8_t* scratch) {
     const int r = m0 + etid;
     const bool rin = r < o.R;
+    if (o.splits == 1) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 16) {
+        if (n0 + c >= o.T) break;
+        float g[16];
+        tmem_ld16(tmem + c, g);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (n0 + c + i < o.T && rin) o.z[(size_t)(n0 + c + i) * o.R + r] = __float2bfloat16_rn(g[i]);
+      }
+      return;
+    }
+    const int slot = blockIdx.x * gridDim.y + blockIdx.y;
+    float* base = o.zpart + (size_t)slot * o.splits * BN * 128;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 16) {
       if (n0 + c >= o.T) break;
       float g[16];
       tmem_ld16(tmem + c, g);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = n0 + c + i;
-        if (t < o.T && rin) {
-          if (o.splits == 1)
-            o.z[(size_t)t * o.R + r] = __float2bfloat16_rn(g[i]);
-          else
-            atomicAdd(&o.zacc[(size_t)t * o.R + r], g[i]);
-        }
-      }
+      for (int i = 0; i < 16; ++i) __stcg(&base[((size_t)split * BN + c + i) * 128 + etid], g[i]);
     }
-    if (o.splits == 1) return;
     int* last = reinterpret_cast<int*>(scratch);
     __threadfence();
     named_bar_sync(1, 128);
-    if (etid == 0) *last = (atomicAdd(&o.tickets[blockIdx.x * gridDim.y + blockIdx.y], 1) == o.splits - 1);
+    if (etid == 0) *last = atomicAdd(&o.tickets[slot], 1) == o.splits - 1;
     named_bar_sync(1, 128);
-    if (*last) {
-      __threadfence();
-      const int tend = min(o.T, n0 + BN);
-      if (rin) {
-        for (int t = n0; t < tend; ++t) {
-          float* p = &o.zacc[(size_t)t * o.R + r];
-          o.z[(size_t)t * o.R + r] = __float2bfloat16_rn(__ldcg(p));
-          *p = 0.0f;
-        }
+    if (!*last) return;
+    __threadfence();
+    const int tend = min(o.T - n0, BN);
+#pragma unroll 1
+    for (int c = 0; c < tend; c += 16) {
+      float h[Z_MAX_SPLITS][16];
+#pragma unroll
+      for (int q = 0; q < Z_MAX_SPLITS; ++q)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[q][i] = q < o.splits ? __ldcg(&base[((size_t)q * BN + c + i) * 128 + etid]) : 0.f;
+      float g[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {  // splits added in ascending K order
+        g[i] = h[0][i];
+#pragma unroll
+        for (int q = 1; q < Z_MAX_SPLITS; ++q)
+          if (q < o.splits) g[i] += h[q][i];
       }
-      if (etid == 0) o.tickets[blockIdx.x * gridDim.y + blockIdx.y] = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (c + i < tend && rin) o.z[(size_t)(n0 + c + i) * o.R + r] = __float2bfloat16_rn(g[i]);
     }
+    if (etid == 0) o.tickets[slot] = 0;
   }
 };
 
@@ -358,6 +378,51 @@ struct EpiFallbackH {
 // 128-neuron tile; the kept values come from the token's TwELL record, which
 // is scattered into a shared [32 tokens][128 neurons] table, 32 tokens at a
 // time.  Overflow tokens are skipped (their rows come from the fallback).
+// Hybrid routing ([TwELL] "Hybrid 應對非均勻稀疏") for the tile path, done
+// by the epilogue warps of the first tile's CTA before their own tile: the
+// tokens whose TwELL record overflowed go whole to the dense channel, which
+// runs after this kernel.  They are listed in token order and counted, and
+// their x (and z) rows are gathered for the dense channel's B operand.
+struct RouteParams {
+  int* ovf_list;      // [maxT] (null: no routing in this launch)
+  int* ovf_count;     // [1]
+  const uint4* x;     // [T][d/8]
+  uint4* xo;
+  int d_vec;
+  const uint4* z;     // [T][R/8] or null
+  uint4* zo;
+  int r_vec;
+};
+
+__device__ __forceinline__ void route_overflow(const RouteParams& r, const uint32_t* ovf, uint32_t epoch, int T,
+                                               int etid, int* sh /*[8]*/) {
+  const int w = etid >> 5, lane = etid & 31;
+  int base = 0;
+  for (int c = 0; c < T; c += 128) {
+    const int t = c + etid;
+    const bool o = t < T && ovf[t] == epoch;
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, o);
+    if (lane == 0) sh[w] = __popc(bal);
+    named_bar_sync(1, 128);
+    int pre = base;
+    for (int q = 0; q < w; ++q) pre += sh[q];
+    if (o) r.ovf_list[pre + __popc(bal & lanemask_lt())] = t;
+    base += sh[0] + sh[1] + sh[2] + sh[3];
+    named_bar_sync(1, 128);
+  }
+  if (etid == 0) *r.ovf_count = base;
+  // gathers: the list entries this thread wrote are visible to the CTA after the barrier
+  __threadfence_block();
+  named_bar_sync(1, 128);
+  for (int o = 0; o < base; ++o) {
+    const int t = r.ovf_list[o];
+    for (int v = etid; v < r.d_vec; v += 128) r.xo[(size_t)o * r.d_vec + v] = r.x[(size_t)t * r.d_vec + v];
+    if (r.z)
+      for (int v = etid; v < r.r_vec; v += 128) r.zo[(size_t)o * r.r_vec + v] = r.z[(size_t)t * r.r_vec + v];
+  }
+  named_bar_sync(1, 128);
+}
+
 struct TwellHParams {
   int T, F, n_tiles, C;
   const int16_t* count;
@@ -367,6 +432,7 @@ struct TwellHParams {
   uint32_t epoch;
   __nv_bfloat16* h_hi;
   __nv_bfloat16* h_lo;
+  RouteParams route;  // done by the CTA of tile (0, 0) when route.ovf_list is set
 };
 
 struct EpiTwellH {
@@ -377,6 +443,8 @@ struct EpiTwellH {
     uint16_t* tab = reinterpret_cast<uint16_t*>(scratch);            // [32][128]
     int* live = reinterpret_cast<int*>(scratch + 32 * 128 * 2);        // [32]
     const int p = m0 >> 7, j = m0 + etid;
+    if (o.route.ovf_list && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+      route_overflow(o.route, o.ovf, o.epoch, o.T, etid, live);
     HParams hp;
     hp.F = o.F;
     hp.h_hi = o.h_hi;

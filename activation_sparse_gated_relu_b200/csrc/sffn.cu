@@ -7,11 +7,11 @@
 //           low-rank gate = two tile kernels (z = bf16(x·A) split over K, then
 //           g = z·B with the TwELL epilogue); up to 8 tokens: a row-streaming
 //           gate over every SM with the same epilogue
-//   router  (TILES only) overflow list, gathers, output zeroing
 //   ROWS    fused up x down over the kept rows of each 8-token block
 //           (non-overflow tokens; the kernel also routes the overflow tokens,
 //           and the gate zeroes out when the kernel adds partial sums into it)
-//   TILES   tensor-core u per tile with h from TwELL (non-overflow tokens)
+//   TILES   tensor-core u per tile with h from TwELL (non-overflow tokens);
+//           the first tile's CTA routes the overflow tokens, the gate zeroes out
 //   dense   tensor-core recompute of g and u for overflow tokens -> h
 //   down    tensor-core y = h·W_down for the h rows (overflow rows on ROWS,
 //           all rows on TILES)
@@ -84,6 +84,14 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows,
 
 int pick_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// K splits of the z = x·A GEMM: only with one token tile (up to 256 tokens),
+// at most Z_MAX_SPLITS, at least 4 K blocks each, and no more CTAs than SMs
+// (the splits' sum is a serial step at the end, so few long splits beat many)
+int z_splits(int d, int m_tiles, int tok_tiles, int n_sm) {
+  if (tok_tiles != 1) return 1;
+  return std::max(1, std::min({Z_MAX_SPLITS, cdiv(d, 64) / 4, n_sm / m_tiles}));
+}
 
 // Launch with programmatic dependent launch: the kernel may be scheduled while
 // the previous kernel on the stream drains; it calls griddepcontrol.wait before
@@ -173,7 +181,7 @@ struct sffn_handle {
   float* norms = nullptr;
   __nv_bfloat16* z = nullptr;
   __nv_bfloat16* zo = nullptr;
-  float* zacc = nullptr;
+  float* zpart = nullptr;   // split-K partials of z (up to 256 tokens)
   int* tickets = nullptr;
   __nv_bfloat16* At = nullptr;
   __nv_bfloat16* Bt = nullptr;
@@ -210,7 +218,7 @@ void free_handle(sffn_handle* h) {
   if (!h) return;
   timing_free(h);
   void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
-                  h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zacc,
+                  h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zpart,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
                   h->zero_row, h->gstage, h->gtick};
   for (void* p : ptrs)
@@ -374,8 +382,8 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     const size_t R = (size_t)h->R;
     ok = ok && dalloc(&h->z, T * R * 2);
     ok = ok && dalloc(&h->zo, T * R * 2);
-    ok = ok && dalloc(&h->zacc, T * R * 4);
-    ok = ok && dalloc(&h->tickets, (R / 128 + 1) * (T / 16 + 2) * 4);
+    ok = ok && dalloc(&h->zpart, (R / 128 + 1) * Z_MAX_SPLITS * (size_t)pick_bn((int)std::min<size_t>(T, 256)) * 128 * 4);
+    ok = ok && dalloc(&h->tickets, (R / 128 + 1) * 4);
     ok = ok && dalloc(&h->At, R * d * 2);
     ok = ok && dalloc(&h->Bt, F * R * 2);
   }
@@ -395,8 +403,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, std::max<size_t>(2048, d * 2), st);
   if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
   if (h->lowrank) {
-    e = e ? e : cudaMemsetAsync(h->zacc, 0, T * (size_t)h->R * 4, st);
-    e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * (T / 16 + 2) * 4, st);
+    e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * 4, st);
   }
   // create-time derived data
   const dim3 tb(32, 8);
@@ -469,7 +476,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     }
   }
   if (!e && h->wina) {
-    const int tk_smem = (int)(F * 4 + 32 * 256 * 4 + P * 4);
+    const int tk_smem = topk_smem_bytes((int)F, (int)P, (int)C);
     e = cudaFuncSetAttribute(k_wina_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, tk_smem);
   }
   if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, router_smem_bytes((int)T));
@@ -548,13 +555,13 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   if (h->lowrank) {
     // z = bf16(x·A): rows are rank coordinates, split over d
     const int mt = cdiv(h->R, 128);
-    const int sk = std::max(1, std::min(cdiv(d, 64), cdiv(h->n_sm, mt * ntile_tok)));
+    const int sk = z_splits(d, mt, ntile_tok, h->n_sm);
     TcArgs za{};
     za.n_phase = 1;
     za.kb_total[0] = cdiv(d, 64);
     za.n_rows = T;
     za.status = h->status;
-    ZParams zp{T, h->R, sk, h->zacc, h->z, h->tickets};
+    ZParams zp{T, h->R, sk, h->zpart, h->z, h->tickets};
     tmark(h, st, L_GATE_Z);
     e = launch_tc<EpiLowRankZ>(BN, dim3(mt, ntile_tok, sk), st, h->tmAt, mx, h->tmAt, mx, za, zp);
     ++launches;
@@ -569,7 +576,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   ga.n_rows = T;
   ga.status = h->status;
   ga.stages = h->gate_stages;
-  if (rows && rows_split > 1) {  // the split fused kernel adds its partials into out
+  if (!rows || rows_split > 1) {  // later kernels add partial sums into out
     ga.zero_out = reinterpret_cast<float4*>(out);
     ga.zero_n4 = (long long)T * d / 4;
   }
@@ -582,7 +589,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     TopkArgs ta{h->scores, h->vdense, 0, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
     tmark(h, st, L_WINA_TOPK);
     ++launches;
-    if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st, 1, ta))
+    if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)topk_smem_bytes(F, P, h->C), st, 1, ta))
       return SFFN_ERR_CUDA;
   } else {
     tmark(h, st, L_GATE);
@@ -606,31 +613,6 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     }
     ++launches;
     if (e) return SFFN_ERR_CUDA;
-  }
-
-  // -------------------------------------------------------------- router
-  // (the fused row kernel does its own routing: only the tile path needs this)
-  if (!rows) {
-    RouterArgs ra{};
-    ra.T = T;
-    ra.ovf = h->ovf;
-    ra.epoch = epoch;
-    ra.ovf_list = h->ovf_list;
-    ra.ovf_count = h->ovf_count;
-    ra.x = static_cast<const uint4*>(x);
-    ra.xo = reinterpret_cast<uint4*>(h->xo);
-    ra.d_vec = d / 8;
-    ra.z = h->lowrank ? reinterpret_cast<const uint4*>(h->z) : nullptr;
-    ra.zo = reinterpret_cast<uint4*>(h->zo);
-    ra.r_vec = h->R / 8;
-    ra.out = reinterpret_cast<float4*>(out);
-    ra.d4 = d / 4;
-    ra.zero_all = 1;
-    const int router_ctas = std::max(1, std::min(h->n_sm, cdiv((long long)T * d / 4, 4096)));
-    tmark(h, st, L_ROUTER);
-    ++launches;
-    if (launch_pdl(k_router, dim3(router_ctas), dim3(1024), (size_t)router_smem_bytes(T), st, 1, ra))
-      return SFFN_ERR_CUDA;
   }
 
   // ------------------------------------------ non-overflow tokens
@@ -674,7 +656,16 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     ua.n_rows = T;
     ua.status = h->status;
     TwellHParams hp{T, F, P, h->C, h->count, h->idx, static_cast<const __nv_bfloat16*>(h->val), h->ovf, epoch,
-                    h->h_hi, h->h_lo};
+                    h->h_hi, h->h_lo, RouteParams{}};
+    // the first tile's CTA routes the overflow tokens for the dense channel
+    hp.route.ovf_list = h->ovf_list;
+    hp.route.ovf_count = h->ovf_count;
+    hp.route.x = static_cast<const uint4*>(x);
+    hp.route.xo = reinterpret_cast<uint4*>(h->xo);
+    hp.route.d_vec = d / 8;
+    hp.route.z = h->lowrank ? reinterpret_cast<const uint4*>(h->z) : nullptr;
+    hp.route.zo = reinterpret_cast<uint4*>(h->zo);
+    hp.route.r_vec = h->R / 8;
     tmark(h, st, L_TILE_H);
     e = launch_tc<EpiTwellH>(BN, dim3(P, ntile_tok, 1), st, h->tmWup, mx, h->tmWup, mx, ua, hp);
     ++launches;
@@ -768,7 +759,7 @@ static sffn_status forward_f32(sffn_handle* h, const void* x, int T, float* out,
     TopkArgs ta{h->scores, h->vdense, 1, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
     tmark(h, st, L_WINA_TOPK);
     ++launches;
-    if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)(F * 4 + 32 * 256 * 4 + P * 4), st, 1, ta))
+    if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)topk_smem_bytes(F, P, h->C), st, 1, ta))
       return SFFN_ERR_CUDA;
   }
   RouterArgs ra{};
@@ -957,22 +948,22 @@ sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st) {
 // device or fail when memory is reserved or fragmented.  For them this entry
 // point computes z = bf16(x·A) and the TwELL records of sigma(z·B + b) with
 // the same kernels as sffn_forward, but keeps its scratch (the split-K fp32
-// accumulator of z, its per-tile tickets, z itself and a status word) in
+// partials of z, its per-tile tickets, z itself and a status word) in
 // file-scope device arrays of fixed size that every GPU loading this library
 // holds until the process exits.  It calls no allocator: inputs and outputs
 // come from the caller.
 namespace {
 
 constexpr int kNaMaxT = 64, kNaMaxD = 4096, kNaMaxR = 1024, kNaMaxF = 16384;
-constexpr int kNaTickets = (kNaMaxR / 128) * (kNaMaxT / 16);
+constexpr int kNaTickets = kNaMaxR / 128;
 
-static __device__ __align__(256) float g_na_zacc[kNaMaxT * kNaMaxR];
+static __device__ __align__(256) float g_na_zpart[(kNaMaxR / 128) * Z_MAX_SPLITS * kNaMaxT * 128];
 static __device__ __align__(256) __nv_bfloat16 g_na_z[kNaMaxT * kNaMaxR];
 static __device__ __align__(256) int g_na_tickets[kNaTickets];
 static __device__ __align__(256) uint32_t g_na_status[4];
 
 struct NaScratch {
-  float* zacc = nullptr;
+  float* zpart = nullptr;
   __nv_bfloat16* z = nullptr;
   int* tickets = nullptr;
   uint32_t* status = nullptr;
@@ -990,8 +981,8 @@ sffn_status na_setup(int dev, NaScratch** out) {
   NaScratch& s = g_na_dev[dev];
   if (!s.ready) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_na_zacc) != cudaSuccess) goto fail;
-    s.zacc = static_cast<float*>(p);
+    if (cudaGetSymbolAddress(&p, g_na_zpart) != cudaSuccess) goto fail;
+    s.zpart = static_cast<float*>(p);
     if (cudaGetSymbolAddress(&p, g_na_z) != cudaSuccess) goto fail;
     s.z = static_cast<__nv_bfloat16*>(p);
     if (cudaGetSymbolAddress(&p, g_na_tickets) != cudaSuccess) goto fail;
@@ -1039,10 +1030,9 @@ extern "C" sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_mo
   if (ss != SFFN_OK) return ss;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const int P = d_ff / 128, BN = pick_bn(T), ntile = cdiv(T, BN), mt = cdiv(rank, 128);
-  const int sk = std::max(1, std::min(cdiv(d_model, 64), cdiv(nsm > 0 ? nsm : kNumSMsFallback, mt * ntile)));
-  // the split-K accumulator, the tickets and the caller's overflow flags start at zero
-  cudaError_t e = cudaMemsetAsync(sc->zacc, 0, (size_t)T * rank * sizeof(float), st);
-  e = e ? e : cudaMemsetAsync(sc->tickets, 0, sizeof(int) * kNaTickets, st);
+  const int sk = z_splits(d_model, mt, ntile, nsm > 0 ? nsm : kNumSMsFallback);
+  // the split tickets and the caller's overflow flags start at zero
+  cudaError_t e = cudaMemsetAsync(sc->tickets, 0, sizeof(int) * kNaTickets, st);
   e = e ? e : cudaMemsetAsync(overflow, 0, (size_t)T * sizeof(uint32_t), st);
   if (e) {
     cudaGetLastError();
@@ -1057,7 +1047,7 @@ extern "C" sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_mo
   za.kb_total[0] = cdiv(d_model, 64);
   za.n_rows = T;
   za.status = sc->status;
-  ZParams zp{T, rank, sk, sc->zacc, sc->z, sc->tickets};
+  ZParams zp{T, rank, sk, sc->zpart, sc->z, sc->tickets};
   if (launch_tc<EpiLowRankZ>(BN, dim3(mt, ntile, sk), st, mAt, mx, mAt, mx, za, zp) != cudaSuccess)
     return SFFN_ERR_CUDA;
   TcArgs ga{};

@@ -126,17 +126,26 @@ struct TopkArgs {
   uint32_t epoch;
 };
 
+// keys, histograms, tie prefix (padded to 16 bytes), per-warp staged records
+__host__ __device__ inline int topk_smem_bytes(int F, int n_tiles, int C) {
+  return F * 4 + 32 * 256 * 4 + ((n_tiles + 3) & ~3) * 4 + 32 * 3 * C * 2;
+}
+
 __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
-  extern __shared__ uint32_t tk_keys[];   // [F] then [32][256] histograms then [n_tiles] tie prefix
+  extern __shared__ uint32_t tk_keys[];   // [F] keys, [32][256] histograms, [n_tiles] tie prefix, [32] records
   uint32_t* hist = tk_keys + a.F;
   int* eqpre = reinterpret_cast<int*>(hist + 32 * 256);
-  __shared__ int scan_tmp[33];
+  uint16_t* recs = reinterpret_cast<uint16_t*>(eqpre + ((a.n_tiles + 3) & ~3));
+  __shared__ int wtot[32], wpre[32];
   __shared__ uint32_t sel[4];  // prefix, remaining
   griddep_wait();
   const int t = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* sc = a.scores + (size_t)t * a.F;
-  for (int j = tid; j < a.F; j += blockDim.x) tk_keys[j] = __float_as_uint(sc[j]);
+  // F is a multiple of 128: 16-byte loads, several in flight per thread
+#pragma unroll 4
+  for (int j = 4 * tid; j < a.F; j += 4 * blockDim.x)
+    *reinterpret_cast<uint4*>(&tk_keys[j]) = *reinterpret_cast<const uint4*>(&sc[j]);
   const int k = a.k;
   const bool keep_all = k >= a.F, keep_none = k <= 0;
   uint32_t prefix = 0, mask = 0;
@@ -150,16 +159,36 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
         if ((key & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key >> shift) & 255u)], 1u);
       }
       __syncthreads();
-      // bins in descending order: suffix sums over bins 255..0 (threads 0..255 = bin 255-tid)
+      // bins in descending order: four threads per bin (thread group g = bin
+      // 255 - g) add the 32 per-warp counts, then a scan over the groups gives
+      // every bin the number of keys in higher bins
+      const int g = tid >> 2, part = tid & 3, bin = 255 - g;
       int c = 0;
-      if (tid < 256) {
-        const int bin = 255 - tid;
-        for (int w = 0; w < 32; ++w) c += (int)hist[w * 256 + bin];
+      for (int w2 = part; w2 < 32; w2 += 4) c += (int)hist[w2 * 256 + bin];
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, 1);
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, 2);
+      int inc = c;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += n;
       }
-      int tot;
-      const int ex = block_scan_excl(tid < 256 ? c : 0, scan_tmp, &tot);
-      if (tid < 256 && ex < rem && ex + c >= rem) {
-        sel[0] = (uint32_t)(255 - tid);
+      if (lane == 31) wtot[warp] = inc;
+      __syncthreads();
+      if (warp == 0) {
+        const int v = wtot[lane];
+        int vi = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xFFFFFFFFu, vi, o);
+          if (lane >= o) vi += n;
+        }
+        wpre[lane] = vi - v;
+      }
+      __syncthreads();
+      const int ex = wpre[warp] + inc - c;
+      if (part == 0 && ex < rem && ex + c >= rem) {
+        sel[0] = (uint32_t)bin;
         sel[1] = (uint32_t)(rem - ex);
       }
       __syncthreads();
@@ -177,19 +206,44 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
     if (lane == 0) eqpre[p] = c;
   }
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int p = 0; p < a.n_tiles; ++p) {
-      const int c = eqpre[p];
-      eqpre[p] = run;
-      run += c;
+  if (warp == 0) {  // exclusive prefix over the tiles: lane l takes tiles [8l, 8l + 8)
+    int loc[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int p = 8 * lane + i;
+      loc[i] = p < a.n_tiles ? eqpre[p] : 0;
+      sum += loc[i];
+    }
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+      if (lane >= o) inc += n;
+    }
+    int run = inc - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int p = 8 * lane + i;
+      if (p < a.n_tiles) eqpre[p] = run;
+      run += loc[i];
     }
   }
   __syncthreads();
+  // records: each warp stages a tile's record (ascending neuron order, pads
+  // after the count) in shared memory and writes it as 16-byte vectors
   const uint32_t lt = lanemask_lt();
+  uint16_t* ridx = recs + warp * 3 * a.C;                 // [C] idx, then [C] values (2 or 4 bytes)
+  uint16_t* rval = ridx + a.C;
+  const int vb = a.val_f32 ? 4 : 2;
   for (int p = warp; p < a.n_tiles; p += 32) {
     int run = 0, ties = eqpre[p];
     const size_t rec = (size_t)t * a.n_tiles + p;
+    for (int sl = lane; sl < a.C; sl += 32) {
+      ridx[sl] = 0xFFFFu;  // -1
+      rval[sl] = 0u;       // +0
+      if (a.val_f32) rval[a.C + sl] = 0u;
+    }
+    __syncwarp();
     for (int q = 0; q < 4; ++q) {
       const int j = p * 128 + q * 32 + lane;
       const uint32_t key = tk_keys[j];
@@ -200,27 +254,29 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
       const uint32_t kb = __ballot_sync(0xFFFFFFFFu, keep);
       const int slot = run + __popc(kb & lt);
       if (keep && slot < a.C) {
-        a.idx[rec * a.C + slot] = (int16_t)j;
+        ridx[slot] = (uint16_t)j;
         if (a.val_f32)
-          reinterpret_cast<float*>(a.val)[rec * a.C + slot] =
-              reinterpret_cast<const float*>(a.vdense)[(size_t)t * a.F + j];
+          reinterpret_cast<float*>(rval)[slot] = reinterpret_cast<const float*>(a.vdense)[(size_t)t * a.F + j];
         else
-          reinterpret_cast<__nv_bfloat16*>(a.val)[rec * a.C + slot] =
-              reinterpret_cast<const __nv_bfloat16*>(a.vdense)[(size_t)t * a.F + j];
+          rval[slot] = reinterpret_cast<const uint16_t*>(a.vdense)[(size_t)t * a.F + j];
       }
       run += __popc(kb);
     }
-    for (int sl = run + lane; sl < a.C; sl += 32) {
-      a.idx[rec * a.C + sl] = -1;
-      if (a.val_f32)
-        reinterpret_cast<float*>(a.val)[rec * a.C + sl] = 0.f;
-      else
-        reinterpret_cast<__nv_bfloat16*>(a.val)[rec * a.C + sl] = __float2bfloat16_rn(0.f);
+    __syncwarp();
+    const int ni = a.C >> 3, nvv = a.C * vb / 16;  // 16-byte vectors of idx and of values
+    for (int e = lane; e < ni + nvv; e += 32) {
+      if (e < ni) {
+        reinterpret_cast<uint4*>(a.idx + rec * a.C)[e] = reinterpret_cast<const uint4*>(ridx)[e];
+      } else {
+        uint8_t* dst = reinterpret_cast<uint8_t*>(a.val) + rec * a.C * vb;
+        reinterpret_cast<uint4*>(dst)[e - ni] = reinterpret_cast<const uint4*>(rval)[e - ni];
+      }
     }
     if (lane == 0) {
       a.count[rec] = (int16_t)run;
       if (run > a.C) a.ovf[t] = a.epoch;
     }
+    __syncwarp();
   }
 }
 
