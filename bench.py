@@ -61,7 +61,7 @@ TIMING_STRIDE = 8
 REF_BUDGET_S = 90.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {
-    "gate": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
+    "gate": ["gate_rows.cuh", "rows_mma.cuh", "tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "gate_lowrank_z": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "tile_h": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "fallback_h": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
