@@ -21,6 +21,7 @@ SFFN_MODE_RELU_THRESHOLD, SFFN_MODE_WINA_TOPK = 0, 1
 SFFN_ACT_RELU, SFFN_ACT_SILU = 0, 1
 SFFN_PATH_AUTO, SFFN_PATH_ROWS, SFFN_PATH_TILES = 0, 1, 2
 SFFN_FLAG_DEBUG_GATE = 1
+SFFN_FLAG_SEPARATE = 2
 
 
 class sffn_desc(ctypes.Structure):
@@ -185,7 +186,7 @@ class SparseFFN:
     def __init__(self, W_up, W_down, *, W_gate=None, A=None, B=None, bias=None,
                  mode: str = "relu_threshold", act: str = "relu", threshold: float = 0.0,
                  k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
-                 debug_gate: bool = False, stream: Optional[int] = None):
+                 debug_gate: bool = False, separate: bool = False, stream: Optional[int] = None):
         import torch
         self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias) if t is not None]
         dt = W_up.dtype
@@ -204,7 +205,7 @@ class SparseFFN:
         desc.k = int(k)
         desc.tile_capacity = int(tile_capacity)
         desc.path = _PATH[path]
-        desc.flags = SFFN_FLAG_DEBUG_GATE if debug_gate else 0
+        desc.flags = (SFFN_FLAG_DEBUG_GATE if debug_gate else 0) | (SFFN_FLAG_SEPARATE if separate else 0)
         ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         desc.W_gate, desc.A, desc.B = ptr(W_gate), ptr(A), ptr(B)
         desc.W_up, desc.W_down, desc.gate_bias = ptr(W_up), ptr(W_down), ptr(bias)

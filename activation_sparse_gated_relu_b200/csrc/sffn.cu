@@ -29,6 +29,7 @@
 
 #include "../../include/sffn.h"
 #include "epilogues.cuh"
+#include "decode_fused.cuh"
 #include "gate_rows.cuh"
 #include "rows_mma.cuh"
 #include "simt.cuh"
@@ -43,10 +44,10 @@ namespace {
 constexpr int kNumSMsFallback = 148;
 constexpr int kMaxMarks = 12;
 enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
-                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_COUNT };
+                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_COUNT };
 const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
                                           "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
-                                          "fallback_f32"};
+                                          "fallback_f32", "decode_fused"};
 constexpr int kMaxTokensLimit = 16384;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -202,6 +203,11 @@ struct sffn_handle {
   int* gtick = nullptr;
   int gr_nslot = 0, gr_smem = 0;
   bool gr_ok = false;
+  // single persistent launch for T <= 8: dense-channel h, grid barrier, launch shape
+  float* hdense = nullptr;
+  unsigned* gbar = nullptr;
+  int dec_nslot = 0, dec_lcap = 0, dec_smem = 0, dec_grid = 0;
+  bool dec_ok = false;
   // per-kernel timing (sffn_timing_begin/end)
   bool tm_on = false;
   int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
@@ -220,7 +226,7 @@ void free_handle(sffn_handle* h) {
   void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zpart,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->zero_row, h->gstage, h->gtick};
+                  h->zero_row, h->gstage, h->gtick, h->hdense, h->gbar};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -299,6 +305,7 @@ sffn_status validate(const sffn_desc* d) {
   if (d->rank > 0 && (d->dtype != SFFN_BF16 || d->rank % 64 != 0 || d->rank > 4096)) return SFFN_ERR_UNSUPPORTED;
   if (d->dtype == SFFN_FP32 && d->d_ff > 8192) return SFFN_ERR_UNSUPPORTED;
   if ((d->flags & SFFN_FLAG_DEBUG_GATE) && d->rank > 0) return SFFN_ERR_UNSUPPORTED;
+  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE)) return SFFN_ERR_INVALID_ARG;
   return SFFN_OK;
 }
 
@@ -391,6 +398,8 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   if (!h->f32 && !h->wina && !h->lowrank) {
     ok = ok && dalloc(&h->gstage, P * 8 * 128 * 4);
     ok = ok && dalloc(&h->gtick, P * 4);
+    ok = ok && dalloc(&h->hdense, 8 * F * 4);
+    ok = ok && dalloc(&h->gbar, 16);
   }
   if (!ok) {
     free_handle(h);
@@ -402,6 +411,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
   if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, std::max<size_t>(2048, d * 2), st);
   if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
+  if (h->gbar) e = e ? e : cudaMemsetAsync(h->gbar, 0, 16, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * 4, st);
   }
@@ -473,6 +483,21 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem;
       if (h->gr_ok)
         e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->gr_smem);
+      // the single persistent launch: two ring slots, the largest rank list that fits,
+      // and exactly as many CTAs as can be resident at once (its grid barriers need that)
+      int dl = 512;
+      while (dl > 64 && DecodeSmem::make(h->P, h->C, dl, h->d, 2).total > max_smem) dl -= 64;
+      h->dec_nslot = 2;
+      h->dec_lcap = dl;
+      h->dec_smem = DecodeSmem::make(h->P, h->C, dl, h->d, 2).total;
+      h->dec_ok = h->gr_ok && h->rows_ok && h->dec_smem <= max_smem && h->P <= RW_THREADS;
+      if (h->dec_ok && !e) {
+        e = cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, h->dec_smem);
+        int nb = 0;
+        if (!e) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode, RW_THREADS, h->dec_smem);
+        h->dec_grid = nb * h->n_sm;
+        h->dec_ok = !e && nb >= 1;
+      }
     }
   }
   if (!e && h->wina) {
@@ -547,6 +572,34 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   tw.epoch = epoch;
   tw.kmask = rows ? h->kmask : nullptr;
   tw.gdebug = h->gdebug;
+
+  // ---------------------------------------- one persistent launch at T <= 8
+  if (rows && T <= 8 && h->dec_ok && !(D.flags & SFFN_FLAG_SEPARATE)) {
+    DecodeArgs da{};
+    da.x = static_cast<const __nv_bfloat16*>(x);
+    da.W_gate = static_cast<const __nv_bfloat16*>(D.W_gate);
+    da.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
+    da.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
+    da.zero_row = h->zero_row;
+    da.tw = tw;
+    da.gstage = h->gstage;
+    da.gtick = h->gtick;
+    da.gbar = h->gbar;
+    da.ovf_list = h->ovf_list;
+    da.ovf_count = h->ovf_count;
+    da.hdense = h->hdense;
+    da.out = out;
+    da.d = d;
+    da.nslot = h->dec_nslot;
+    da.lcap = h->dec_lcap;
+    da.status = h->status;
+    tmark(h, st, L_DECODE);
+    if (launch_pdl(k_decode, dim3(h->dec_grid), dim3(RW_THREADS), (size_t)h->dec_smem, st, 1, da))
+      return SFFN_ERR_CUDA;
+    h->last_path = SFFN_PATH_ROWS;
+    h->last_launches = 1;
+    return SFFN_OK;
+  }
 
   // ---------------------------------------------------------------- gate
   const CUtensorMap* gateA = &h->tmWgate;

@@ -67,6 +67,7 @@ KERNEL_SOURCES = {
     "fallback_h": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "down": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "updown_rows": ["rows_mma.cuh", "ptx.cuh"],
+    "decode_fused": ["decode_fused.cuh", "rows_mma.cuh", "epilogues.cuh", "ptx.cuh"],
     "router": ["simt.cuh", "ptx.cuh"],
     "wina_topk": ["simt.cuh", "ptx.cuh"],
     "gate_f32": ["simt.cuh", "epilogues.cuh", "ptx.cuh"],
@@ -269,6 +270,11 @@ def kernel_work(wl, T: int, path: str, st: dict) -> dict:
         if wl.mode != "wina_topk":
             w["fallback_h"] = {"bytes": dense_in + n_o * F * 4, "flops": 2 * n_o * d * F}
         w["down"] = {"bytes": (F * d * es + n_o * F * 4 + n_o * d * 4) if n_o else 0, "flops": 2 * n_o * F * d}
+        # the single persistent launch (T <= 8) does all of the above; the gate
+        # TwELL and keep masks stay on chip-near L2 between its phases but are
+        # still written and read, so they count like the separate kernels'
+        w["decode_fused"] = {"bytes": sum(w[k]["bytes"] for k in (g, "updown_rows", "fallback_h", "down")) - xb,
+                             "flops": sum(w[k]["flops"] for k in (g, "updown_rows", "fallback_h", "down"))}
     else:
         w["router"] = {"bytes": yb + 2 * n_o * d * es, "flops": 0}
         w["tile_h"] = {"bytes": F * d * es + xb + twell + T * F * 4, "flops": 2 * T * d * F}

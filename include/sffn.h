@@ -80,9 +80,11 @@ typedef enum { SFFN_MODE_RELU_THRESHOLD = 0, SFFN_MODE_WINA_TOPK = 1 } sffn_mode
 typedef enum { SFFN_ACT_RELU = 0, SFFN_ACT_SILU = 1 } sffn_act;
 
 /* How the kept (token, neuron) pairs of non-overflow tokens are computed.
- *   ROWS : the fused SIMT up x down kernel streams only the kept rows of W_up
+ *   ROWS : the fused up x down kernel streams only the kept rows of W_up
  *          and W_down, per block of 8 tokens (best when few tokens share a
- *          neuron: decode at T <= 8, sparse prefill);
+ *          neuron: decode at T <= 8, sparse prefill).  At T <= 8 with a dense
+ *          threshold gate the whole forward (gate, TwELL, routing, up x down,
+ *          dense channel) runs as one persistent launch;
  *   TILES: tensor-core up and down over every 128-neuron tile that some token
  *          keeps, with the non-kept entries of h zeroed (best when the union
  *          of kept neurons covers most tiles: WINA, T in 16..256).
@@ -91,6 +93,8 @@ typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sff
 
 /* desc.flags */
 #define SFFN_FLAG_DEBUG_GATE 1u   /* keep the dense fp32 gate g[T][d_ff] of the last forward */
+#define SFFN_FLAG_SEPARATE 2u     /* T <= 8: separate gate, up x down and dense-channel launches
+                                     instead of the single persistent launch (diagnostics, tests) */
 
 typedef struct sffn_desc {
   int d_model;          /* d: multiple of 8, 8..4096 (ROWS path needs d <= 4096)   */

@@ -77,7 +77,9 @@ def test_work_model_decode_matches_byte_formula():
     assert b == wl.d_ff * wl.d_model * 2 + 8163 * 2 * wl.d_model * 2 + 8 * wl.d_model * (2 + 4) + 2 * twell
     assert f == 2 * 8 * wl.d_model * wl.d_ff + 4 * 12000 * wl.d_model
     w = bench.kernel_work(wl, 8, "rows", st)
-    assert set(w) == {"gate", "updown_rows", "fallback_h", "down"}
+    assert set(w) == {"gate", "updown_rows", "fallback_h", "down", "decode_fused"}
+    # the single launch moves the step's bytes plus the keep masks written and read
+    assert w["decode_fused"]["bytes"] == b + 2 * 8 * P * 16
     # no overflow: the dense channel moves nothing
     assert w["fallback_h"]["bytes"] == 0 and w["down"]["flops"] == 0
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}

@@ -215,6 +215,24 @@ def test_decode_forced_overflow_same_y(decode_inputs):
     assert b["overflow"] == 0
 
 
+def test_decode_single_launch_and_separate_kernels(decode_inputs):
+    # T <= 8 runs as one persistent launch; the flag keeps the separate
+    # gate, up x down and dense-channel launches, which must agree
+    one = check(decode_inputs, T=8)
+    assert one["launches"] == 1 and one["path"] == SFFN_PATH_ROWS
+    sep = check(decode_inputs, T=8, separate=True)
+    assert sep["launches"] == 4 and sep["path"] == SFFN_PATH_ROWS
+    check(decode_inputs, T=3, C=8, separate=True)
+
+
+@pytest.mark.parametrize("C", [8, 16])
+def test_decode_single_launch_dense_channel(decode_inputs, C):
+    # small capacities make tokens overflow: the single launch's dense channel
+    # (its third phase, after a second grid barrier) computes their outputs
+    st = check(decode_inputs, T=8, C=C)
+    assert st["overflow"] > 0 and st["launches"] == 1
+
+
 def test_lopa_config():
     inp = synth.make_inputs(W["lopa_bf16"])
     st = check(inp)
