@@ -11,14 +11,17 @@
 // staged x block and the partial output registers, and drops the dense
 // channel's launches when no token overflows (the common case at decode).
 //
-//   G  gate: CTA s takes an equal range of 8-neuron groups of W_gate; a
-//      tile's 128 gate values are assembled across CTAs in a staging block
-//      and the CTA completing the tile's ticket emits its TwELL records;
-//   -- grid barrier: every tile emitted (overflow epochs final) --
-//   R  rows: the union of the live tokens' keep masks is ranked and split
-//      into equal ranges; each range's W_up rows then W_down rows stream
-//      through the ring, u and h stay in registers, y accumulates in
-//      registers; CTA 0 lists and counts the overflow tokens;
+//   G  gate: CTA s takes an equal range of 8-neuron groups of W_gate and
+//      writes their gate values (fp32, for the TwELL values) and keep bits
+//      (one byte per token and group);
+//   -- grid barrier: every gate value and keep bit in --
+//   R  rows: every CTA derives the per-tile counts, the overflow tokens and
+//      the union of the live tokens' keep masks from the keep bits, ranks
+//      the union and takes an equal range; its W_up rows then W_down rows
+//      stream through the ring, u and h stay in registers, y accumulates in
+//      registers.  While its first stages are in flight, CTA p writes tile
+//      p's TwELL records (the format's output; nothing here waits for them)
+//      and CTA 0 lists and counts the overflow tokens;
 //   D  dense channel, only if some token overflowed: D1 streams W_gate and
 //      W_up rows over the CTA's gate range and writes h = bf16(sigma(g))·u
 //      of the overflow tokens (0 where not kept); after a second grid
@@ -44,8 +47,8 @@ struct DecodeArgs {
   const __nv_bfloat16* W_down;
   const __nv_bfloat16* zero_row; // >= d bf16 zeros
   TwellParams tw;                // T, F, n_tiles, C, bias, tau, act, TwELL outputs, keep masks, epochs
-  float* gstage;                 // [n_tiles][8][128] gate values of tiles being assembled
-  int* gtick;                    // [n_tiles], zero between forwards
+  float* gstage;                 // [n_tiles][8][128] fp32 gate values (before the bias)
+  uint8_t* kbits;                // [8][d_ff / 8] keep bits, one byte per (token, 8-neuron group)
   unsigned* gbar;                // [2] grid barrier: arrivals, generation
   int* ovf_list;                 // [8]
   int* ovf_count;                // [1]
@@ -56,8 +59,8 @@ struct DecodeArgs {
 };
 
 struct DecodeSmem {
-  int xs, ring, bars, uni, ured, misc, total;
-  // uni: the TwELL staging of G, or the rank bookkeeping of R (never both)
+  int xs, ring, bars, uni, emit, ured, misc, total;
+  // uni: the rank bookkeeping of R; emit: the TwELL staging (8 tokens)
   __host__ __device__ static int rank_bytes(int n_tiles, int lcap) {
     return (((n_tiles + 1) * 4 + 15) & ~15) + n_tiles * 16 + lcap * 4 + lcap * 4 + lcap * 16;
   }
@@ -67,7 +70,8 @@ struct DecodeSmem {
     s.xs = o;      o += RowsSmem::stage(d);
     s.ring = o;    o += nslot * RowsSmem::stage(d);
     s.bars = o;    o += ((RW_NSMAX + 1) * 8 + 15) & ~15;
-    s.uni = o;     o += max(twell32_smem(C), rank_bytes(n_tiles, lcap));
+    s.uni = o;     o += rank_bytes(n_tiles, lcap);
+    s.emit = o;    o += twell_smem(8, C);
     s.ured = o;    o += 2 * RW_WARPS * 32 * 8;
     s.misc = o;    o += 64 * 4;
     s.total = o;
@@ -119,7 +123,6 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   float2* ured = reinterpret_cast<float2*>(sm + L.ured);
   int* misc = reinterpret_cast<int*>(sm + L.misc);
   volatile int* abort_flag = misc + 40;
-  volatile int* done_flag = misc + 41;
   volatile int* bar_ok = misc + 42;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   const int nj = d / RW_DIV;
   const int NG = F / RW_G;
   const int g0 = (int)((long long)NG * s / G), g1 = (int)((long long)NG * (s + 1) / G);
-  constexpr int GPT = 128 / RW_G;
+  constexpr int GPT = 128 / RW_G;  // 8-neuron groups per TwELL tile
   const uint32_t ring_s = smem_u32(ring);
   const uint32_t lrow = (uint32_t)((lane & 7) * RS + 16 * ((lane >> 3) & 1) + 32 * warp);
   const uint32_t hi_off = (lane >> 4) ? 32u * RW_WARPS : 0u;
@@ -231,49 +234,33 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
         issue_rows(gs + ns, a.W_gate, nullptr, RW_G, (g0 + q + ns) * RW_G);
         issued_end = gs + ns + 1;
       }
-      if (warp < 4) {
-        // warp 0 sums the warps' partials into the tile's staging block; the
-        // CTA's last group of a tile takes the tile's ticket
+      if (warp == 0) {
+        // warp 0 sums the warps' partials into the tile's staging block
         const int grp = g0 + q, p = grp / GPT;
-        const bool last_of_tile = q == n_st - 1 || (grp + 1) % GPT == 0;
-        if (warp == 0) {
-          float u0 = 0.f, u1 = 0.f;
+        float u0 = 0.f, u1 = 0.f;
 #pragma unroll
-          for (int w = 0; w < RW_WARPS; ++w) {
-            const float2 v = ub[w * 32 + lane];
-            u0 += v.x;
-            u1 += v.y;
-          }
-          float* gsg = a.gstage + ((size_t)p * 8 + (lane >> 2)) * 128 + (grp % GPT) * RW_G + 2 * (lane & 3);
-          __stcg(gsg, u0);
-          __stcg(gsg + 1, u1);
-          if (last_of_tile) {
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) {
-              const int n_done = grp - max(g0, p * GPT) + 1;
-              *done_flag = atomicAdd(&a.gtick[p], n_done) + n_done == GPT;
-            }
-            __syncwarp();
-          }
+        for (int w = 0; w < RW_WARPS; ++w) {
+          const float2 v = ub[w * 32 + lane];
+          u0 += v.x;
+          u1 += v.y;
         }
-        if (last_of_tile) {
-          named_bar_sync(2, 128);
-          if (*done_flag) {  // the whole tile is in: its TwELL records
-            __threadfence();
-            float g[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) g[i] = i < 8 ? __ldcg(a.gstage + ((size_t)p * 8 + i) * 128 + tid) : 0.f;
-            twell_tile32(a.tw, g, p * 128 + tid, 0, tid, sm + L.uni, 1);
-            if (tid == 0) a.gtick[p] = 0;
-          }
-          named_bar_sync(2, 128);
-        }
+        float* gsg = a.gstage + ((size_t)p * 8 + (lane >> 2)) * 128 + (grp % GPT) * RW_G + 2 * (lane & 3);
+        __stcg(gsg, u0);
+        __stcg(gsg + 1, u1);
+        // keep bits of (token lane/4, neurons 2(lane%4), +1), gathered into one byte per token
+        const int t = lane >> 2, n = grp * RW_G + 2 * (lane & 3);
+        const float b0 = a.tw.bias ? a.tw.bias[n] : 0.f, b1 = a.tw.bias ? a.tw.bias[n + 1] : 0.f;
+        const bool k0 = t < T && fabsf(act_fn(u0 + b0, a.tw.act)) > a.tw.tau;
+        const bool k1 = t < T && fabsf(act_fn(u1 + b1, a.tw.act)) > a.tw.tau;
+        uint32_t bits = ((k0 ? 1u : 0u) | (k1 ? 2u : 0u)) << (2 * (lane & 3));
+        bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 1);
+        bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 2);
+        if ((lane & 3) == 0) a.kbits[(size_t)t * NG + grp] = (uint8_t)bits;
       }
     }
     gsq += n_st;
   }
-  // every tile emitted, every slice of out zeroed
+  // every gate value and keep bit in, every slice of out zeroed
   grid_barrier(a.gbar, abort_flag, a.status, bar_ok);
 
   // ------------------------------------------------------------ R: rows
@@ -282,22 +269,27 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   int* nid = reinterpret_cast<int*>(ums + P);
   uint32_t* lmask = reinterpret_cast<uint32_t*>(nid + a.lcap);
   uint4* lval = reinterpret_cast<uint4*>(lmask + a.lcap);
-  // live tokens (valid, not overflowing) and the union of their keep masks
+  // per (token, tile) keep masks from the keep bits: counts, overflow tokens
+  // ([TwELL] hybrid: a token overflows iff some tile keeps more than C),
+  // then the union of the live (valid, not overflowing) tokens' masks
   uint4 km[8];
+  if (tid == 0) {
+    misc[50] = 0;
+    misc[51] = 0;
+  }
+  __syncthreads();
   if (tid < P) {
+    uint32_t ob = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      km[i] = i < T ? reinterpret_cast<const uint4*>(a.tw.kmask)[(size_t)i * P + tid] : make_uint4(0, 0, 0, 0);
-  }
-  if (warp == 0) {
-    const bool v = lane < 8 && lane < T;
-    const bool o = v && a.tw.ovf[lane] == a.tw.epoch;
-    const uint32_t vb = __ballot_sync(0xFFFFFFFFu, v), obb = __ballot_sync(0xFFFFFFFFu, o);
-    if (lane == 0) {
-      misc[50] = (int)(vb & ~obb);
-      misc[51] = (int)obb;
+    for (int i = 0; i < 8; ++i) {
+      km[i] = i < T ? __ldcg(reinterpret_cast<const uint4*>(a.kbits + (size_t)i * NG) + tid) : make_uint4(0, 0, 0, 0);
+      const int c = __popc(km[i].x) + __popc(km[i].y) + __popc(km[i].z) + __popc(km[i].w);
+      if (c > C) ob |= 1u << i;
     }
+    if (ob) atomicOr(reinterpret_cast<unsigned*>(&misc[51]), ob);
   }
+  __syncthreads();
+  if (tid == 0) misc[50] = (int)(((1u << T) - 1u) & ~(uint32_t)misc[51]);
   __syncthreads();
   const uint32_t live = (uint32_t)misc[50], obits = (uint32_t)misc[51];
   if (tid < P) {
@@ -343,9 +335,21 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     if (lane == 0) tpre[P] = run;
   }
   __syncthreads();
+  // the TwELL records of tile s (and s + G, ...) by warps 0-3, the same
+  // emission as the tile kernels'; the rows phase does not wait for them
+  auto emit_tiles = [&]() {
+    if (warp >= 4) return;
+    for (int p = s; p < P; p += G) {
+      float g[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) g[i] = __ldcg(a.gstage + ((size_t)p * 8 + i) * 128 + tid);
+      twell_tile32<8>(a.tw, g, p * 128 + tid, 0, tid, sm + L.emit, 1);
+    }
+  };
   {
     const int U = tpre[P];
     const int r0 = (int)((long long)U * s / G), r1 = (int)((long long)U * (s + 1) / G);
+    if (r0 >= r1) emit_tiles();  // no rows for this CTA
     for (int c0 = r0; c0 < r1; c0 += a.lcap) {
       const int c1 = min(r1, c0 + a.lcap), Lc = c1 - c0;
       const int n_groups = (Lc + RW_G - 1) / RW_G;
@@ -375,25 +379,18 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
       };
       for (int q = 0; q < ns && q < n_st; ++q) issue_r(q);
       issued_end = gsq + min(ns, n_st);
-      // TwELL values of the live tokens, one thread per (slot, token, tile)
-      for (int e = tid; e < C * 8 * (pb - pa + 1); e += blockDim.x) {
-        const int sl = e % C, rest = e / C;
-        const int i = rest & 7, p = pa + (rest >> 3);
+      if (c0 == r0) emit_tiles();  // while the first stages are in flight
+      // h's bf16 values v = bf16(sigma(g + b)) of the live tokens' kept
+      // pairs of this chunk's neurons: one thread per (neuron, token)
+      for (int e = tid; e < Lc * 8; e += blockDim.x) {
+        const int r = e >> 3, i = e & 7;
+        const int n = nid[r];
         if (!((live >> i) & 1u)) continue;
-        const size_t rec = (size_t)i * P + p;
-        const int cnt = min((int)a.tw.count[rec], C);
-        if (sl >= cnt) continue;
-        const int bit = (int)a.tw.idx[rec * C + sl] - p * 128;
-        if (bit < 0 || bit >= 128) {
-          atomicOr(a.status, DEV_ERR_RANGE);
-          continue;
-        }
-        const int rank = tpre[p] + popc_below(ums[p], bit);
-        if (rank >= c0 && rank < c1) {
-          reinterpret_cast<uint16_t*>(&lval[rank - c0])[i] =
-              reinterpret_cast<const uint16_t*>(a.tw.val)[rec * C + sl];
-          atomicOr(&lmask[rank - c0], 1u << i);
-        }
+        if (!((a.kbits[(size_t)i * NG + (n >> 3)] >> (n & 7)) & 1u)) continue;
+        const float gv = __ldcg(a.gstage + ((size_t)(n >> 7) * 8 + i) * 128 + (n & 127)) +
+                         (a.tw.bias ? a.tw.bias[n] : 0.f);
+        reinterpret_cast<uint16_t*>(&lval[r])[i] = __bfloat16_as_ushort(__float2bfloat16_rn(act_fn(gv, a.tw.act)));
+        atomicOr(&lmask[r], 1u << i);
       }
       __syncthreads();
       for (int g = 0; g < n_groups; ++g) {

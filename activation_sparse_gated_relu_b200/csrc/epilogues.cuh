@@ -92,8 +92,8 @@ __device__ __forceinline__ void twell_chunk(const TwellParams& o, const float* g
   }
 }
 
-// TwELL emission for one 128-neuron tile and up to 32 tokens t0..t0+31 (bf16
-// values), by the 128 threads of four full warps.  It is the same format as
+// TwELL emission for one 128-neuron tile and up to NT (8 or 32) tokens
+// t0..t0+NT-1 (bf16 values), by the 128 threads of four full warps.  It is the same format as
 // twell_chunk, but its phases keep every thread busy and write whole records:
 //   1. thread = neuron: activation, keep bit, bf16 value into a staging
 //      block; warp ballots give each token's 128-bit keep mask;
@@ -102,25 +102,32 @@ __device__ __forceinline__ void twell_chunk(const TwellParams& o, const float* g
 //      token's staged record (ascending neuron order); pads fill slots at or
 //      after the count.  Count, overflow epoch and keep mask are written
 //      here;
-//   3. the staged [32][C] idx and val records go out as 16-byte vectors.
+//   3. the staged [NT][C] idx and val records go out as 16-byte vectors.
 // (Thread-per-neuron stores of 2-byte slots kept one warp per scheduler
 // waiting on dependent latencies and flooded L2 with partial writes.)
 constexpr int TW32_VP = 128 + 8;   // padded staged-value row (bf16 elements)
-__host__ __device__ constexpr int twell32_smem(int C) { return 32 * 4 * 4 + 32 * TW32_VP * 2 + 32 * C * 2 * 2; }
+__host__ __device__ constexpr int twell_smem(int NT, int C) { return NT * 4 * 4 + NT * TW32_VP * 2 + NT * C * 2 * 2; }
+__host__ __device__ constexpr int twell32_smem(int C) { return twell_smem(32, C); }
 
+template <int NT = 32>
 __device__ __forceinline__ void twell_tile32(const TwellParams& o, const float* g, int j, int t0, int etid,
                                              uint8_t* scratch, uint32_t bar_id) {
   const int w = etid >> 5, lane = etid & 31;
   const int p = j >> 7, n_in = j & 127;
   const int C = o.C;
-  uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);                         // [32 tokens][4]
-  uint16_t* vals = reinterpret_cast<uint16_t*>(scratch + 32 * 4 * 4);             // [32][TW32_VP]
-  uint16_t* sidx = reinterpret_cast<uint16_t*>(scratch + 32 * 4 * 4 + 32 * TW32_VP * 2);  // [32][C]
-  uint16_t* sval = sidx + 32 * C;                                                  // [32][C]
+  uint32_t* masks = reinterpret_cast<uint32_t*>(scratch);                         // [NT tokens][4]
+  uint16_t* vals = reinterpret_cast<uint16_t*>(scratch + NT * 4 * 4);             // [NT][TW32_VP]
+  uint16_t* sidx = reinterpret_cast<uint16_t*>(scratch + NT * 4 * 4 + NT * TW32_VP * 2);  // [NT][C]
+  uint16_t* sval = sidx + NT * C;                                                  // [NT][C]
   const float b = o.bias ? o.bias[j] : 0.0f;
+  const int ntok = min(NT, o.T - t0);  // tokens of this call (the rest are masked)
   // 1. thread = neuron
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NT; ++i) {
+    if (i >= ntok) {  // uniform: tokens beyond T keep nothing
+      if (lane == 0) masks[i * 4 + w] = 0u;
+      continue;
+    }
     const float gv = g[i] + b;
     const float a = act_fn(gv, o.act);
     const bool in = (t0 + i) < o.T;
@@ -132,7 +139,7 @@ __device__ __forceinline__ void twell_tile32(const TwellParams& o, const float* 
   }
   named_bar_sync(bar_id, 128);
   // 2. four threads per token
-  {
+  if (etid < 4 * NT && t0 + (etid >> 2) < o.T) {
     const int tt = etid >> 2, wq = etid & 3, t = t0 + tt;
     const uint4 m4 = reinterpret_cast<const uint4*>(masks)[tt];
     const int c0 = __popc(m4.x), c1 = __popc(m4.y), c2 = __popc(m4.z), c3 = __popc(m4.w);
@@ -163,8 +170,8 @@ __device__ __forceinline__ void twell_tile32(const TwellParams& o, const float* 
   // 3. whole records out, 8 slots per 16-byte vector
   {
     const int nvec = C >> 3;
-    for (int e = etid; e < 2 * 32 * nvec; e += 128) {
-      const int arr = e / (32 * nvec), r = e - arr * 32 * nvec;
+    for (int e = etid; e < 2 * NT * nvec; e += 128) {
+      const int arr = e / (NT * nvec), r = e - arr * NT * nvec;
       const int tt = r / nvec, v = r - tt * nvec, t = t0 + tt;
       if (t >= o.T) continue;
       const uint4 val = reinterpret_cast<const uint4*>((arr ? sval : sidx) + tt * C)[v];

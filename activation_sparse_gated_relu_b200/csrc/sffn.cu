@@ -205,6 +205,7 @@ struct sffn_handle {
   bool gr_ok = false;
   // single persistent launch for T <= 8: dense-channel h, grid barrier, launch shape
   float* hdense = nullptr;
+  uint8_t* kbits = nullptr;
   unsigned* gbar = nullptr;
   int dec_nslot = 0, dec_lcap = 0, dec_smem = 0, dec_grid = 0;
   bool dec_ok = false;
@@ -226,7 +227,7 @@ void free_handle(sffn_handle* h) {
   void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zpart,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->zero_row, h->gstage, h->gtick, h->hdense, h->gbar};
+                  h->zero_row, h->gstage, h->gtick, h->hdense, h->kbits, h->gbar};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -399,6 +400,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     ok = ok && dalloc(&h->gstage, P * 8 * 128 * 4);
     ok = ok && dalloc(&h->gtick, P * 4);
     ok = ok && dalloc(&h->hdense, 8 * F * 4);
+    ok = ok && dalloc(&h->kbits, F);
     ok = ok && dalloc(&h->gbar, 16);
   }
   if (!ok) {
@@ -583,7 +585,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     da.zero_row = h->zero_row;
     da.tw = tw;
     da.gstage = h->gstage;
-    da.gtick = h->gtick;
+    da.kbits = h->kbits;
     da.gbar = h->gbar;
     da.ovf_list = h->ovf_list;
     da.ovf_count = h->ovf_count;
