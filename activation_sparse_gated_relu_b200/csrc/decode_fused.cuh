@@ -148,6 +148,12 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     fence_mbar_init();
     mbar_expect_tx(xbar, (uint32_t)(nvalid * d * 2));
     for (int t = 0; t < nvalid; ++t) bulk_g2s(sm + L.xs + t * RS, a.x + (size_t)t * d, (uint32_t)d * 2u, xbar);
+    // the gate's first stages go out with x, ahead of the zeroing below
+    for (int q = 0; q < ns && q < g1 - g0; ++q) {
+      mbar_expect_tx(&full[q], (uint32_t)(RW_G * d * 2));
+      for (int r = 0; r < RW_G; ++r)
+        bulk_g2s(ring + (size_t)q * SB + r * RS, a.W_gate + (size_t)((g0 + q) * RW_G + r) * d, (uint32_t)d * 2u, &full[q]);
+    }
   }
   for (int e = tid; e < (8 - nvalid) * (d >> 3); e += blockDim.x) {
     const int t = nvalid + e / (d >> 3), v = e % (d >> 3);
@@ -219,11 +225,17 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
 
   // ------------------------------------------------------------ G: gate
   {
-    const int n_st = g1 - g0;
-    for (int q = 0; q < ns && q < n_st; ++q) issue_rows(gsq + q, a.W_gate, nullptr, RW_G, (g0 + q) * RW_G);
+    const int n_st = g1 - g0;  // the first ns stages were issued in the setup
     issued_end = gsq + min(ns, n_st);
     for (int q = 0; q < n_st; ++q) {
       const int gs = gsq + q, slot = gs % ns;
+      // warp 0's bias pair for this group, loaded before the wait
+      float b0 = 0.f, b1 = 0.f;
+      if (warp == 0 && a.tw.bias) {
+        const int n = (g0 + q) * RW_G + 2 * (lane & 3);
+        b0 = __ldg(a.tw.bias + n);
+        b1 = __ldg(a.tw.bias + n + 1);
+      }
       const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
       float cu[4];
       up_partial(ring_s + (uint32_t)(slot * SB) + lrow, ok, cu);
@@ -248,8 +260,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
         __stcg(gsg, u0);
         __stcg(gsg + 1, u1);
         // keep bits of (token lane/4, neurons 2(lane%4), +1), gathered into one byte per token
-        const int t = lane >> 2, n = grp * RW_G + 2 * (lane & 3);
-        const float b0 = a.tw.bias ? a.tw.bias[n] : 0.f, b1 = a.tw.bias ? a.tw.bias[n + 1] : 0.f;
+        const int t = lane >> 2;
         const bool k0 = t < T && fabsf(act_fn(u0 + b0, a.tw.act)) > a.tw.tau;
         const bool k1 = t < T && fabsf(act_fn(u1 + b1, a.tw.act)) > a.tw.tau;
         uint32_t bits = ((k0 ? 1u : 0u) | (k1 ? 2u : 0u)) << (2 * (lane & 3));
