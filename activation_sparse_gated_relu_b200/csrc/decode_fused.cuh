@@ -1,38 +1,53 @@
 // The whole forward for one block of up to 8 tokens in one persistent launch
 // ([TwELL] sections "TwELL 減掉轉換開銷" and "Hybrid 應對非均勻稀疏"): the gate
-// with its TwELL emission, the overflow routing, the fused sparse up x down of
-// the non-overflow tokens and the dense channel of the overflow tokens.
+// with its TwELL emission, the overflow flags and the fused sparse up x down
+// of every kept neuron.
 //
-// With one CTA per SM, every phase streams weight rows through the same
-// ring of shared-memory stages (8 whole rows of 8 KB per stage, one bulk copy
-// per row) and computes on warp MMAs, as the separate row-streaming kernels
-// do (gate_rows.cuh, rows_mma.cuh).  Keeping the phases in one launch removes
-// a kernel boundary (grid drain, launch, prologue) between each, shares the
-// staged x block and the partial output registers, and drops the dense
-// channel's launches when no token overflows (the common case at decode).
+// With one CTA per SM, every phase streams whole weight rows through shared-
+// memory stages (8 rows of 8 KB per stage, one bulk copy per row) and
+// computes on warp MMAs, as the separate row-streaming kernels do
+// (gate_rows.cuh, rows_mma.cuh).  There is no grid-wide barrier:
 //
-//   G  gate: CTA s takes an equal range of 8-neuron groups of W_gate and
-//      writes their gate values (fp32, for the TwELL values) and keep bits
-//      (one byte per token and group);
-//   -- grid barrier: every gate value and keep bit in --
-//   R  rows: every CTA derives the per-tile counts, the overflow tokens and
-//      the union of the live tokens' keep masks from the keep bits, ranks
-//      the union and takes an equal range; its W_up rows then W_down rows
-//      stream through the ring, u and h stay in registers, y accumulates in
-//      registers.  While its first stages are in flight, CTA p writes tile
-//      p's TwELL records (the format's output; nothing here waits for them)
-//      and CTA 0 lists and counts the overflow tokens;
-//   D  dense channel, only if some token overflowed: D1 streams W_gate and
-//      W_up rows over the CTA's gate range and writes h = bf16(sigma(g))·u
-//      of the overflow tokens (0 where not kept); after a second grid
-//      barrier, D2 streams W_down rows over the same range and adds
-//      h·W_down into the same partial-output registers;
-//   the partial outputs go into out (zeroed in G, before the first barrier)
-//   by bulk reduce-add copies at L2.
+//   G  CTA s gates an equal range of 8-neuron groups of W_gate through three
+//      slots (the two ring slots and the x block: x sits in registers while
+//      the partial y is not yet live).  Its warp 0 turns each group's gate
+//      values into the TwELL staging block (fp32, shared with the other CTAs
+//      of the tile) and into CTA s's own row list: one record per neuron of
+//      the range that some token keeps (the neuron, its token mask and the 8
+//      tokens' bf16 values bf16(sigma(g + b))), copied to global memory as it
+//      grows.  The list is complete when the range is, with no other CTA's
+//      results.
+//   R  the list's 8-record items go through the two ring slots as a W_up
+//      stage and a W_down stage each, with x back in the x block; u and h
+//      stay in registers, y accumulates in registers.  The first item's
+//      stages are issued while the last gate stages are still in use, so the
+//      stream does not pause between G and R.  Each list is published (its
+//      length, tagged with the forward's epoch, after a release fence), its
+//      owner takes items in small claims, and a CTA whose own list is
+//      exhausted steals half of the largest remainder of another CTA's list:
+//      the work of an SM that gated slowly, or whose range keeps more
+//      neurons, spreads over the others.
+//   y  every CTA zeroes a slice of out when it starts (its publication
+//      announces that too); each CTA's partial y goes into out by bulk
+//      reduce-add copies at L2, eight pieces per token row.
+//   TwELL: while those copies run, warps 4-7 of CTA s write the records of
+//      the tiles [e_lo, e_hi) assigned to it, from the staged gate values of
+//      the CTAs that gated them (complete once those have published).
 //
-// The grid barriers need every CTA resident: the host launches exactly the
-// number of CTAs that fit at once (one per SM), and every wait is bounded
-// (a timeout sets the status word and the CTA gives up instead of hanging).
+// Overflow tokens.  The hybrid format sends a token that keeps more than C
+// neurons of some tile to a dense channel, which computes
+// y = sum_j h_j W_down[j] over all d_ff neurons with h_j = 0 where the token
+// does not keep j.  Here a token's row list has no capacity, so the same sum
+// over the kept neurons is what R computes for every token: an overflow
+// token's dense-channel result comes out of the same stream, and it costs at
+// most its extra kept rows rather than a second pass over all three matrices.
+// The TwELL records and the per-token overflow flags are still written
+// exactly as the format defines them; the flags are the routing's record.
+//
+// The only waits on other CTAs are a steal while some list is not yet
+// published, the zeroed slices of out and the completeness of a tile to
+// write; all CTAs are resident (the host launches one per SM), every wait is
+// bounded, and a timeout sets the status word.
 #pragma once
 
 #include "epilogues.cuh"
@@ -48,109 +63,111 @@ struct DecodeArgs {
   const __nv_bfloat16* zero_row; // >= d bf16 zeros
   TwellParams tw;                // T, F, n_tiles, C, bias, tau, act, TwELL outputs, keep masks, epochs
   float* gstage;                 // [n_tiles][8][128] fp32 gate values (before the bias)
-  uint8_t* kbits;                // [8][d_ff / 8] keep bits, one byte per (token, 8-neuron group)
-  unsigned* gbar;                // [2] grid barrier: arrivals, generation
-  int* ovf_list;                 // [8]
-  int* ovf_count;                // [1]
-  float* hdense;                 // [8][F] h of the overflow tokens (dense channel)
+  int* sched;                    // [decode_sched_ints(n_tiles, grid)] zero before the first launch
+  uint32_t* wl_id;               // [grid][maxr] published records: neuron | token mask << 24
+  uint4* wl_val;                 // [grid][maxr] published records: 8 tokens' bf16 values
+  int maxr;                      // records per list (>= 8 x the most groups a CTA gates)
   float* out;                    // [T][d]
-  int d, nslot, lcap;
+  int d;
   uint32_t* status;
 };
 
+// Scheduler words, in ints from the start of DecodeArgs::sched.  A list
+// length carries the forward's epoch, so a value left by an earlier launch
+// never reads as this launch's, and its owner sets the claim count before it
+// publishes the length: nothing needs resetting between launches.
+struct DecodeSched {
+  int P, G;
+  __host__ __device__ int pub(int v) const { return v; }        // (epoch << 16) | (list length + 1)
+  __host__ __device__ int claim(int v) const { return G + v; }  // items taken from list v
+  __host__ __device__ int total() const { return 2 * G; }
+};
+__host__ __device__ inline int decode_sched_ints(int P, int G) { return DecodeSched{P, G}.total(); }
+
+constexpr int DEC_NS = 2;  // ring slots (the gate also streams through the x block)
+
 struct DecodeSmem {
-  int xs, ring, bars, uni, emit, ured, misc, total;
-  // uni: the rank bookkeeping of R; emit: the TwELL staging (8 tokens)
-  __host__ __device__ static int rank_bytes(int n_tiles, int lcap) {
-    return (((n_tiles + 1) * 4 + 15) & ~15) + n_tiles * 16 + lcap * 4 + lcap * 4 + lcap * 16;
-  }
-  __host__ __device__ static DecodeSmem make(int n_tiles, int C, int lcap, int d, int nslot) {
+  int xs, ring, bars, lid, lval, ib, emit, ured, vcnt, misc, total;
+  __host__ __device__ static DecodeSmem make(int C, int maxr, int d) {
     DecodeSmem s;
     int o = 0;
-    s.xs = o;      o += RowsSmem::stage(d);
-    s.ring = o;    o += nslot * RowsSmem::stage(d);
-    s.bars = o;    o += ((RW_NSMAX + 1) * 8 + 15) & ~15;
-    s.uni = o;     o += rank_bytes(n_tiles, lcap);
-    s.emit = o;    o += twell_smem(8, C);
-    s.ured = o;    o += 2 * RW_WARPS * 32 * 8;
-    s.misc = o;    o += 64 * 4;
+    s.xs = o;    o += RowsSmem::stage(d);
+    s.ring = o;  o += DEC_NS * RowsSmem::stage(d);
+    s.bars = o;  o += ((RW_NSMAX + 1) * 8 + 15) & ~15;
+    s.lid = o;   o += (maxr * 4 + 15) & ~15;       // own list: packed ids
+    s.lval = o;  o += maxr * 16;                   // own list: values
+    s.ib = o;    o += 2 * 8 * 4 + 2 * 8 * 16;      // two item buffers (ids, then values)
+    s.emit = o;  o += twell_smem(8, C);
+    s.ured = o;  o += 2 * RW_WARPS * 32 * 8;
+    s.vcnt = o;  o += RW_THREADS * 4;              // steal scan: list lengths
+    s.misc = o;  o += 64 * 4;
     s.total = o;
     return s;
   }
 };
 
-// Bounded grid-wide barrier over all CTAs of the launch (all resident).
-// Returns false (and records a timeout) if the other CTAs do not arrive.
-__device__ __forceinline__ bool grid_barrier(unsigned* gbar, volatile int* abort_flag, uint32_t* status,
-                                             volatile int* shared_ok) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    __threadfence();
-    const unsigned gen = atomicAdd(&gbar[1], 0u);
-    if (atomicAdd(&gbar[0], 1u) == gridDim.x - 1) {
-      atomicExch(&gbar[0], 0u);
-      __threadfence();
-      atomicAdd(&gbar[1], 1u);
-    } else {
-      const uint64_t t0 = globaltimer();
-      while (atomicAdd(&gbar[1], 0u) == gen) {
-        if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
-          atomicOr(status, DEV_ERR_TIMEOUT);
-          *abort_flag = 1;
-          ok = 0;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    *shared_ok = ok;
-  }
-  __syncthreads();
-  return *shared_ok != 0;
-}
+// misc[] slots
+enum : int {
+  DM_ABORT = 0, DM_CNT = 1, DM_RISS = 2, DM_EMOK = 3, DM_CHV = 4, DM_CHK = 5, DM_CHK1 = 6,
+  DM_VCNT = 7, DM_OWNMORE = 8, DM_RES = 9, DM_LK0 = 12, DM_XLK = 15,
+  DM_RED = 16
+};
 
 __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
-  const int d = a.d, T = a.tw.T, F = a.tw.F, P = a.tw.n_tiles, C = a.tw.C;
-  const int ns = max(2, min(a.nslot, RW_NSMAX));
-  const DecodeSmem L = DecodeSmem::make(P, C, a.lcap, d, ns);
+  const int d = a.d, T = a.tw.T, F = a.tw.F, P = a.tw.n_tiles;
+  const DecodeSmem L = DecodeSmem::make(a.tw.C, a.maxr, d);
   const int RS = RowsSmem::pitch(d), SB = RowsSmem::stage(d);
   uint8_t* ring = sm + L.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* xbar = full + RW_NSMAX;
+  uint32_t* lid = reinterpret_cast<uint32_t*>(sm + L.lid);
+  uint4* lval = reinterpret_cast<uint4*>(sm + L.lval);
+  uint32_t* ib_id = reinterpret_cast<uint32_t*>(sm + L.ib);   // [2][8]
+  uint4* ib_val = reinterpret_cast<uint4*>(sm + L.ib + 64);   // [2][8]
   float2* ured = reinterpret_cast<float2*>(sm + L.ured);
+  int* vcs = reinterpret_cast<int*>(sm + L.vcnt);
   int* misc = reinterpret_cast<int*>(sm + L.misc);
-  volatile int* abort_flag = misc + 40;
-  volatile int* bar_ok = misc + 42;
+  volatile int* abort_flag = misc + DM_ABORT;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, s = blockIdx.x;
+  const DecodeSched S{P, G};
+  int* sc = a.sched;
   const int nj = d / RW_DIV;
   const int NG = F / RW_G;
   const int g0 = (int)((long long)NG * s / G), g1 = (int)((long long)NG * (s + 1) / G);
+  const int n_g = g1 - g0;  // gate stages: stage k < n_g holds W_gate rows of group g0 + k
   constexpr int GPT = 128 / RW_G;  // 8-neuron groups per TwELL tile
   const uint32_t ring_s = smem_u32(ring);
   const uint32_t lrow = (uint32_t)((lane & 7) * RS + 16 * ((lane >> 3) & 1) + 32 * warp);
   const uint32_t hi_off = (lane >> 4) ? 32u * RW_WARPS : 0u;
   const uint32_t xsl = smem_u32(sm + L.xs) + lrow;
-  int gsq = 0;         // stages issued and consumed by earlier phases (slot and parity base)
-  int issued_end = 0;  // stages issued so far (for the drain after an abort)
 
   griddep_wait();  // x, out and the workspace belong to the stream order
   // ---------------------------------------------------------------- setup
+  // The gate streams through three slots, the two ring slots and the x
+  // block: x moves into registers for the gate (the partial y is not live
+  // yet), and the x block's last gate stage hands it back to a second copy of
+  // x for the rows phase, which streams through the two ring slots.
   const int nvalid = min(8, T);
+  const bool x_slot = n_g >= 3;  // the gate uses the x block as a third slot
+  auto g_fills = [&](int sl) { return n_g > sl ? (n_g - sl + 2) / 3 : 0; };    // gate stages in slot sl
+  auto g_last = [&](int sl) { return n_g > sl ? sl + 3 * ((n_g - 1 - sl) / 3) : -1; };
+  auto slot_at = [&](int sl) -> uint8_t* { return sl < 2 ? ring + (size_t)sl * SB : sm + L.xs; };
   if (tid == 0) {
-    for (int i = 0; i < ns; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&full[i], 1);
     mbar_init(xbar, 1);
-    *abort_flag = 0;
+    misc[DM_ABORT] = 0;
+    misc[DM_LK0] = misc[DM_LK0 + 1] = misc[DM_LK0 + 2] = -1;
     fence_mbar_init();
     mbar_expect_tx(xbar, (uint32_t)(nvalid * d * 2));
+    misc[DM_XLK] = 1;
     for (int t = 0; t < nvalid; ++t) bulk_g2s(sm + L.xs + t * RS, a.x + (size_t)t * d, (uint32_t)d * 2u, xbar);
-    // the gate's first stages go out with x, ahead of the zeroing below
-    for (int q = 0; q < ns && q < g1 - g0; ++q) {
+    // the gate's first stages go out with x
+    for (int q = 0; q < 2 && q < n_g; ++q) {
       mbar_expect_tx(&full[q], (uint32_t)(RW_G * d * 2));
+      misc[DM_LK0 + q] = 0;
       for (int r = 0; r < RW_G; ++r)
         bulk_g2s(ring + (size_t)q * SB + r * RS, a.W_gate + (size_t)((g0 + q) * RW_G + r) * d, (uint32_t)d * 2u, &full[q]);
     }
@@ -159,7 +176,8 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     const int t = nvalid + e / (d >> 3), v = e % (d >> 3);
     *reinterpret_cast<uint4*>(sm + L.xs + t * RS + v * 16) = make_uint4(0u, 0u, 0u, 0u);
   }
-  {  // this CTA's slice of out starts at zero: every phase adds into it at the end
+  {  // every CTA adds its partial y into all of out at the end; the list's
+     // publication (below) tells the others this slice is zero
     const long long n4 = (long long)T * d / 4;
     const long long q0 = n4 * s / G, q1 = n4 * (s + 1) / G;
     for (long long e = q0 + tid; e < q1; e += blockDim.x)
@@ -167,17 +185,33 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   }
   __syncthreads();
 
-  // stage of 8 rows of matrix W starting at row r0 (or the given row ids)
-  auto issue_rows = [&](int gs, const __nv_bfloat16* W, const int* rowid, int nrows, int row0) {
+  // gate stage q: 8 consecutive W_gate rows into slot q % 3 (lane 0 of warps 0-7, one row each)
+  auto issue_gate = [&](int q) {
     if (lane != 0 || warp >= RW_G) return;
-    const int slot = gs % ns;
-    if (warp == 0) mbar_expect_tx(&full[slot], (uint32_t)(RW_G * d * 2));
-    const __nv_bfloat16* src =
-        warp < nrows ? W + (size_t)(rowid ? rowid[warp] : row0 + warp) * d : a.zero_row;
-    bulk_g2s(ring + (size_t)slot * SB + warp * RS, src, (uint32_t)d * 2u, &full[slot]);
+    const int sl = q % 3;
+    if (warp == 0) {
+      mbar_expect_tx(&full[sl], (uint32_t)(RW_G * d * 2));
+      misc[DM_LK0 + sl] = (q / 3) & 1;
+    }
+    bulk_g2s(slot_at(sl) + warp * RS, a.W_gate + (size_t)((g0 + q) * RW_G + warp) * d, (uint32_t)d * 2u, &full[sl]);
+  };
+  // rows stage kr: item kr/2's W_up rows (kr even) or W_down rows (kr odd)
+  // from item buffer b into ring slot kr % 2; absent records stream the zero row
+  auto r_par = [&](int kr) { return (uint32_t)((g_fills(kr & 1) + (kr >> 1)) & 1); };
+  auto issue_item = [&](int kr, int b) {
+    if (lane != 0 || warp >= RW_G) return;
+    const int sl = kr & 1;
+    if (warp == 0) {
+      mbar_expect_tx(&full[sl], (uint32_t)(RW_G * d * 2));
+      misc[DM_LK0 + sl] = (int)r_par(kr);
+    }
+    const uint32_t id = ib_id[b * 8 + warp];
+    const __nv_bfloat16* W = (kr & 1) ? a.W_down : a.W_up;
+    const __nv_bfloat16* src = id ? W + (size_t)(id & 0xFFFFFFu) * d : a.zero_row;
+    bulk_g2s(ring + (size_t)sl * SB + warp * RS, src, (uint32_t)d * 2u, &full[sl]);
   };
   // up-style product of a staged stage: the warp's partial of
-  // u^T[token lane/4][neurons 2(lane%4), +1] over its k steps
+  // u^T[token lane/4][rows 2(lane%4), +1] over its k steps, x from the x block
   auto up_partial = [&](uint32_t sbs, bool ok, float* cu) {
     cu[0] = cu[1] = cu[2] = cu[3] = 0.f;
     if (!ok) return;
@@ -193,7 +227,141 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
       }
     }
   };
-  float acc[RW_MAXJ][4];
+  // h as bf16 hi + lo halves (the down product's B fragment)
+  auto split_hilo = [](float h0, float h1, uint32_t& bh, uint32_t& bl) {
+    const __nv_bfloat16 a0 = __float2bfloat16_rn(h0), a1 = __float2bfloat16_rn(h1);
+    bh = (uint32_t)__bfloat16_as_ushort(a0) | ((uint32_t)__bfloat16_as_ushort(a1) << 16);
+    bl = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h0 - __bfloat162float(a0))) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h1 - __bfloat162float(a1))) << 16);
+  };
+  // x into registers for the gate: the A fragments of the warp's k steps
+  uint32_t xr[RW_MAXJ / 2][4];
+  mbar_wait(xbar, 0, abort_flag, a.status);
+#pragma unroll
+  for (int jp = 0; jp < RW_MAXJ / 2; ++jp) {
+    const int j = 2 * jp;
+    if (j < nj) {
+      ldsm_x4(xsl + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), xr[jp][0], xr[jp][1], xr[jp][2], xr[jp][3]);
+    } else {
+      xr[jp][0] = xr[jp][1] = xr[jp][2] = xr[jp][3] = 0u;
+    }
+  }
+  __syncthreads();  // every warp holds x: the x block is the gate's third slot
+  if (x_slot) issue_gate(2);
+
+  // ------------------------------------------------------------ G: gate
+  // warp 0's running state: records in the own list, stages of the first
+  // item already issued
+  int cnt = 0, r_iss = 0;
+  // warp 0 turns group qq's partials (in ured[qq & 1]) into its gate values,
+  // keep decisions and list records
+  auto gate_group = [&](int qq, float b0, float b1) {
+    const float2* ub = ured + (qq & 1) * RW_WARPS * 32;
+    const int grp = g0 + qq, p = grp / GPT;
+    float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < RW_WARPS; ++w) {
+      const float2 v = ub[w * 32 + lane];
+      u0 += v.x;
+      u1 += v.y;
+    }
+    // g^T[token lane/4][rows 2(lane%4), +1] into the tile's staging block
+    const int t = lane >> 2, c = lane & 3;
+    float* gsg = a.gstage + ((size_t)p * 8 + t) * 128 + (grp % GPT) * RW_G + 2 * c;
+    __stcg(gsg, u0);
+    __stcg(gsg + 1, u1);
+    // keep decisions ([TwELL]: |sigma(g + b)| > tau) and the records of the
+    // group's rows that some token keeps, appended in row order
+    const float a0 = act_fn(u0 + b0, a.tw.act), a1 = act_fn(u1 + b1, a.tw.act);
+    const bool k0 = t < T && fabsf(a0) > a.tw.tau, k1 = t < T && fabsf(a1) > a.tw.tau;
+    const uint32_t bal0 = __ballot_sync(0xFFFFFFFFu, k0), bal1 = __ballot_sync(0xFFFFFFFFu, k1);
+    uint32_t ra = 0u;  // row r = 2c' + e is kept by token t' iff bit 4t' + c' of bal_e
+#pragma unroll
+    for (int r = 0; r < RW_G; ++r)
+      if (((((r & 1) ? bal1 : bal0) >> (r >> 1)) & 0x11111111u) != 0u) ra |= 1u << r;
+    if ((ra >> (2 * c)) & 1u)
+      reinterpret_cast<uint16_t*>(&lval[cnt + __popc(ra & ((1u << (2 * c)) - 1u))])[t] =
+          k0 ? __bfloat16_as_ushort(__float2bfloat16_rn(a0)) : (uint16_t)0;
+    if ((ra >> (2 * c + 1)) & 1u)
+      reinterpret_cast<uint16_t*>(&lval[cnt + __popc(ra & ((2u << (2 * c)) - 1u))])[t] =
+          k1 ? __bfloat16_as_ushort(__float2bfloat16_rn(a1)) : (uint16_t)0;
+    if (lane < RW_G && ((ra >> lane) & 1u)) {
+      const uint32_t bal = (lane & 1) ? bal1 : bal0;
+      uint32_t tm = 0u;
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt) tm |= ((bal >> (4 * tt + (lane >> 1))) & 1u) << tt;
+      lid[cnt + __popc(ra & ((1u << lane) - 1u))] = (uint32_t)(grp * RW_G + lane) | (tm << 24);
+    }
+    __syncwarp();
+    if (lane < __popc(ra)) {  // the new records go out now; the publication orders them
+      const int i = cnt + lane;
+      a.wl_id[(size_t)s * a.maxr + i] = lid[i];
+      a.wl_val[(size_t)s * a.maxr + i] = lval[i];
+    }
+    cnt += __popc(ra);
+    __syncwarp();
+  };
+  // warp 0: the first item (own records 0-7) into ring slots 0 and 1 (rows
+  // stages 0 and 1) once their last gate stages are read and the list has it
+  auto early_rows = [&](int q_read) {
+    while (r_iss < 2 && g_last(r_iss) <= q_read && cnt >= 8) {
+      if (lane == 0) {
+        mbar_expect_tx(&full[r_iss], (uint32_t)(RW_G * d * 2));
+        misc[DM_LK0 + r_iss] = (int)r_par(r_iss);
+      }
+      if (lane < RW_G)
+        bulk_g2s(ring + (size_t)r_iss * SB + lane * RS,
+                 (r_iss ? a.W_down : a.W_up) + (size_t)(lid[lane] & 0xFFFFFFu) * d, (uint32_t)d * 2u, &full[r_iss]);
+      ++r_iss;
+    }
+  };
+  for (int q = 0; q < n_g; ++q) {
+    const int sl = q % 3;
+    float b0 = 0.f, b1 = 0.f;  // warp 0's bias pair, loaded before the wait
+    if (warp == 0 && a.tw.bias) {
+      const int n = (g0 + q) * RW_G + 2 * (lane & 3);
+      b0 = __ldg(a.tw.bias + n);
+      b1 = __ldg(a.tw.bias + n + 1);
+    }
+    const bool ok = mbar_wait(&full[sl], (uint32_t)((q / 3) & 1), abort_flag, a.status);
+    // this stage's partials: two chains of MMAs against x in registers
+    float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+    if (ok) {
+      const uint32_t sbs = smem_u32(slot_at(sl)) + lrow;
+#pragma unroll
+      for (int jp = 0; jp < RW_MAXJ / 2; ++jp) {
+        const int j = 2 * jp;
+        if (j < nj) {
+          uint32_t b0r, b1r, b2r, b3r;
+          ldsm_x4(sbs + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), b0r, b1r, b2r, b3r);
+          mma_bf16_16816(ca, xr[jp][0], 0u, xr[jp][1], 0u, b0r, b1r);
+          if (j + 1 < nj) mma_bf16_16816(cb, xr[jp][2], 0u, xr[jp][3], 0u, b2r, b3r);
+        }
+      }
+    }
+    ured[(q & 1) * RW_WARPS * 32 + warp * 32 + lane] = make_float2(ca[0] + cb[0], ca[1] + cb[1]);
+    __syncthreads();
+    // the slot is free: the stream's next gate stage, or x back into the x block
+    if (q + 3 < n_g) {
+      issue_gate(q + 3);
+    } else if (sl == 2 && tid == 0) {
+      mbar_expect_tx(xbar, (uint32_t)(nvalid * d * 2));
+      misc[DM_XLK] = 2;
+      for (int t = 0; t < nvalid; ++t) bulk_g2s(sm + L.xs + t * RS, a.x + (size_t)t * d, (uint32_t)d * 2u, xbar);
+    }
+    if (warp == 0) {
+      early_rows(q);
+      gate_group(q, b0, b1);
+    }
+  }
+  if (n_g > 0 && warp == 0) early_rows(n_g - 1);
+  if (x_slot) {  // the second copy of x: rows of absent tokens are zero again
+    for (int e = tid; e < (8 - nvalid) * (d >> 3); e += blockDim.x) {
+      const int t = nvalid + e / (d >> 3), v = e % (d >> 3);
+      *reinterpret_cast<uint4*>(sm + L.xs + t * RS + v * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  float acc[RW_MAXJ][4];  // the partial y: live from here on
 #pragma unroll
   for (int j = 0; j < RW_MAXJ; ++j)
 #pragma unroll
@@ -215,329 +383,265 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
       }
     }
   };
-  auto split_hilo = [](float h0, float h1, uint32_t& bh, uint32_t& bl) {
-    const __nv_bfloat16 a0 = __float2bfloat16_rn(h0), a1 = __float2bfloat16_rn(h1);
-    bh = (uint32_t)__bfloat16_as_ushort(a0) | ((uint32_t)__bfloat16_as_ushort(a1) << 16);
-    bl = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h0 - __bfloat162float(a0))) |
-         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h1 - __bfloat162float(a1))) << 16);
-  };
-  mbar_wait(xbar, 0, abort_flag, a.status);
+  if (tid == 0) {  // warp 0's totals; the claim state starts on the own list
+    const int items = (cnt + 7) >> 3;
+    misc[DM_CNT] = cnt;
+    misc[DM_RISS] = r_iss;
+    misc[DM_CHV] = s;
+    misc[DM_CHK] = 0;
+    misc[DM_CHK1] = min(items, max(2, (items + 1) >> 1));
+    misc[DM_VCNT] = cnt;
+    misc[DM_OWNMORE] = misc[DM_CHK1] < items;
+  }
+  __syncthreads();
 
-  // ------------------------------------------------------------ G: gate
-  {
-    const int n_st = g1 - g0;  // the first ns stages were issued in the setup
-    issued_end = gsq + min(ns, n_st);
-    for (int q = 0; q < n_st; ++q) {
-      const int gs = gsq + q, slot = gs % ns;
-      // warp 0's bias pair for this group, loaded before the wait
-      float b0 = 0.f, b1 = 0.f;
-      if (warp == 0 && a.tw.bias) {
-        const int n = (g0 + q) * RW_G + 2 * (lane & 3);
-        b0 = __ldg(a.tw.bias + n);
-        b1 = __ldg(a.tw.bias + n + 1);
+  // ------------------------------------------------------ own list, steals
+  const int cnt_own = misc[DM_CNT], r_issued = misc[DM_RISS];
+  const int items_own = (cnt_own + 7) >> 3;
+  const int k_pre = min(items_own, max(2, (items_own + 1) >> 1));  // items the owner keeps outright
+  const uint32_t epoch = a.tw.epoch;
+  // Publication of the own list (its length, tagged with the epoch, after the
+  // claim count and a release fence that also covers the records, the gate
+  // values and the zeroed slice of out).  It comes after the first item's
+  // stages are under way, or before the first claim or steal.
+  bool published = false;   // uniform
+  bool all_seen = false;    // uniform: a steal scan found every list published
+  auto publish = [&]() {
+    if (tid == 0) {
+      sc[S.claim(s)] = k_pre;
+      fence_acq_rel_gpu();
+      atomicExch(sc + S.pub(s), (int)(((epoch & 0xFFFFu) << 16) | (uint32_t)(cnt_own + 1)));
+    }
+    published = true;
+  };
+
+  // The next item into item buffer `buf` (block-wide; false when no list
+  // anywhere has work left).  The items of the current claim come first
+  // (one barrier); then own items, one per claim; then the largest published
+  // remainder, half of it per steal.  Only tid 0 writes the claim state in
+  // misc, between barriers.
+  auto acquire = [&](int buf) -> bool {
+    if (misc[DM_CHK] >= misc[DM_CHK1]) {
+      if (__syncthreads_or(*abort_flag)) return false;
+      if (!published) publish();
+      if (tid == 0) {
+        int got = 0;
+        if (misc[DM_OWNMORE]) {
+          const int c = atomicAdd(sc + S.claim(s), 1);
+          if (c < items_own) {
+            misc[DM_CHV] = s;
+            misc[DM_CHK] = c;
+            misc[DM_CHK1] = c + 1;
+            misc[DM_VCNT] = cnt_own;
+            got = 1;
+          } else {
+            misc[DM_OWNMORE] = 0;
+          }
+        }
+        misc[DM_RES] = got;
       }
-      const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
-      float cu[4];
-      up_partial(ring_s + (uint32_t)(slot * SB) + lrow, ok, cu);
-      float2* ub = ured + (q & 1) * RW_WARPS * 32;
-      ub[warp * 32 + lane] = make_float2(cu[0], cu[1]);
       __syncthreads();
-      if (q + ns < n_st) {
-        issue_rows(gs + ns, a.W_gate, nullptr, RW_G, (g0 + q + ns) * RW_G);
-        issued_end = gs + ns + 1;
+      if (!misc[DM_RES]) {
+        uint64_t t0 = 0;
+        if (tid == 0) t0 = globaltimer();
+        for (;;) {
+          int key = -1;
+          bool unpub = false;
+          if (tid < G && tid != s) {
+            const uint32_t pv = (uint32_t)ld_acquire_gpu(sc + S.pub(tid));
+            const int len = (int)(pv & 0xFFFFu) - 1;
+            if ((pv >> 16) != (epoch & 0xFFFFu) || len < 0) {
+              unpub = true;  // not yet published in this launch
+            } else {
+              vcs[tid] = len;
+              const int rem = ((len + 7) >> 3) - __ldcg(sc + S.claim(tid));
+              if (rem > 0) key = (rem << 9) | tid;
+            }
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) key = max(key, __shfl_xor_sync(0xFFFFFFFFu, key, o));
+          if (lane == 0) misc[DM_RED + warp] = key;
+          const int n_unpub = __syncthreads_count(unpub);
+          if (tid == 0) {
+            int best = -1;
+            for (int w = 0; w < RW_WARPS; ++w) best = max(best, misc[DM_RED + w]);
+            int res = 0;  // 0: look again, 1: claimed, 2: no work left (3: and every list seen)
+            if (best >= 0) {
+              const int v = best & 511, vc = vcs[v], it = (vc + 7) >> 3;
+              const int m = max(1, (best >> 9) >> 1);
+              const int c = atomicAdd(sc + S.claim(v), m);
+              if (c < it) {
+                misc[DM_CHV] = v;
+                misc[DM_CHK] = c;
+                misc[DM_CHK1] = min(c + m, it);
+                misc[DM_VCNT] = vc;
+                res = 1;
+              }
+            } else if (n_unpub > 0) {  // lists still being gated: wait for them, bounded
+              if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+                atomicOr(a.status, DEV_ERR_TIMEOUT);
+                *abort_flag = 1;
+                res = 2;
+              } else {
+                __nanosleep(256);
+              }
+            } else {
+              res = 3;
+            }
+            misc[DM_RES] = res;
+          }
+          __syncthreads();
+          if (misc[DM_RES] != 0) break;
+        }
+        if (misc[DM_RES] >= 2) {
+          all_seen = misc[DM_RES] == 3;
+          return false;
+        }
       }
-      if (warp == 0) {
-        // warp 0 sums the warps' partials into the tile's staging block
-        const int grp = g0 + q, p = grp / GPT;
+    }
+    const int v = misc[DM_CHV], k = misc[DM_CHK], vc = misc[DM_VCNT];
+    if (tid < RW_G) {
+      const int i = k * RW_G + tid;
+      uint32_t id = 0u;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (i < vc) {
+        if (v == s) {
+          id = lid[i];
+          val = lval[i];
+        } else {
+          id = __ldcg(a.wl_id + (size_t)v * a.maxr + i);
+          val = __ldcg(a.wl_val + (size_t)v * a.maxr + i);
+        }
+      }
+      ib_id[buf * 8 + tid] = id;
+      ib_val[buf * 8 + tid] = val;
+    }
+    __syncthreads();  // the item buffer is complete; every thread has read the claim state
+    if (tid == 0) misc[DM_CHK] = k + 1;  // read again only after the loop's next barrier
+    return true;
+  };
+
+  // ------------------------------------------------------------ R: rows
+  // rows stage 2i is item i's W_up stage, 2i + 1 its W_down stage
+  const bool have_first = acquire(0);
+  if (have_first)
+    for (int r = r_issued; r < 2; ++r) issue_item(r, 0);  // those G did not issue
+  if (x_slot) mbar_wait(xbar, 1, abort_flag, a.status);  // the second copy of x
+  if (have_first) {
+    int kr = 0, cur = 0;
+    __syncthreads();  // the claim state acquire(0) left
+    bool have_next = acquire(1);
+    for (;;) {
+      uint32_t bh, bl;
+      {  // W_up stage: u of the item's rows, then h = v·u where the token keeps the row
+        const int sl = kr & 1;
+        const bool ok = mbar_wait(&full[sl], r_par(kr), abort_flag, a.status);
+        float cu[4];
+        up_partial(ring_s + (uint32_t)(sl * SB) + lrow, ok, cu);
+        ured[warp * 32 + lane] = make_float2(cu[0], cu[1]);
+        __syncthreads();
+        if (have_next) issue_item(kr + 2, cur ^ 1);
         float u0 = 0.f, u1 = 0.f;
 #pragma unroll
         for (int w = 0; w < RW_WARPS; ++w) {
-          const float2 v = ub[w * 32 + lane];
+          const float2 v = ured[w * 32 + lane];
           u0 += v.x;
           u1 += v.y;
         }
-        float* gsg = a.gstage + ((size_t)p * 8 + (lane >> 2)) * 128 + (grp % GPT) * RW_G + 2 * (lane & 3);
-        __stcg(gsg, u0);
-        __stcg(gsg + 1, u1);
-        // keep bits of (token lane/4, neurons 2(lane%4), +1), gathered into one byte per token
-        const int t = lane >> 2;
-        const bool k0 = t < T && fabsf(act_fn(u0 + b0, a.tw.act)) > a.tw.tau;
-        const bool k1 = t < T && fabsf(act_fn(u1 + b1, a.tw.act)) > a.tw.tau;
-        uint32_t bits = ((k0 ? 1u : 0u) | (k1 ? 2u : 0u)) << (2 * (lane & 3));
-        bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 1);
-        bits |= __shfl_xor_sync(0xFFFFFFFFu, bits, 2);
-        if ((lane & 3) == 0) a.kbits[(size_t)t * NG + grp] = (uint8_t)bits;
-      }
-    }
-    gsq += n_st;
-  }
-  // every gate value and keep bit in, every slice of out zeroed
-  grid_barrier(a.gbar, abort_flag, a.status, bar_ok);
-
-  // ------------------------------------------------------------ R: rows
-  int* tpre = reinterpret_cast<int*>(sm + L.uni);
-  uint4* ums = reinterpret_cast<uint4*>(sm + L.uni + (((P + 1) * 4 + 15) & ~15));
-  int* nid = reinterpret_cast<int*>(ums + P);
-  uint32_t* lmask = reinterpret_cast<uint32_t*>(nid + a.lcap);
-  uint4* lval = reinterpret_cast<uint4*>(lmask + a.lcap);
-  // per (token, tile) keep masks from the keep bits: counts, overflow tokens
-  // ([TwELL] hybrid: a token overflows iff some tile keeps more than C),
-  // then the union of the live (valid, not overflowing) tokens' masks
-  uint4 km[8];
-  if (tid == 0) {
-    misc[50] = 0;
-    misc[51] = 0;
-  }
-  __syncthreads();
-  if (tid < P) {
-    uint32_t ob = 0u;
+        const int tn = lane >> 2, rr = 2 * (lane & 3);
+        float hv[2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      km[i] = i < T ? __ldcg(reinterpret_cast<const uint4*>(a.kbits + (size_t)i * NG) + tid) : make_uint4(0, 0, 0, 0);
-      const int c = __popc(km[i].x) + __popc(km[i].y) + __popc(km[i].z) + __popc(km[i].w);
-      if (c > C) ob |= 1u << i;
-    }
-    if (ob) atomicOr(reinterpret_cast<unsigned*>(&misc[51]), ob);
-  }
-  __syncthreads();
-  if (tid == 0) misc[50] = (int)(((1u << T) - 1u) & ~(uint32_t)misc[51]);
-  __syncthreads();
-  const uint32_t live = (uint32_t)misc[50], obits = (uint32_t)misc[51];
-  if (tid < P) {
-    uint4 u = make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if ((live >> i) & 1u) {
-        u.x |= km[i].x;
-        u.y |= km[i].y;
-        u.z |= km[i].z;
-        u.w |= km[i].w;
-      }
-    ums[tid] = u;
-  }
-  // overflow routing ([TwELL] hybrid): the overflow tokens, in token order,
-  // take the dense channel (phase D below)
-  if (s == 0 && tid == 0) {
-    int o = 0;
-    for (int i = 0; i < 8; ++i)
-      if ((obits >> i) & 1u) a.ovf_list[o++] = i;
-    *a.ovf_count = o;
-  }
-  __syncthreads();
-  // exclusive prefix of the tile union counts; this CTA's rank range
-  if (warp == 0) {
-    int run = 0;
-    for (int p0 = 0; p0 < P; p0 += 32) {
-      const int p = p0 + lane;
-      int c = 0;
-      if (p < P) {
-        const uint4 m = ums[p];
-        c = __popc(m.x) + __popc(m.y) + __popc(m.z) + __popc(m.w);
-      }
-      int inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-        if (lane >= o) inc += n;
-      }
-      if (p < P) tpre[p] = run + inc - c;
-      run += __shfl_sync(0xFFFFFFFFu, inc, 31);
-    }
-    if (lane == 0) tpre[P] = run;
-  }
-  __syncthreads();
-  // the TwELL records of tile s (and s + G, ...) by warps 0-3, the same
-  // emission as the tile kernels'; the rows phase does not wait for them
-  auto emit_tiles = [&]() {
-    if (warp >= 4) return;
-    for (int p = s; p < P; p += G) {
-      float g[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) g[i] = __ldcg(a.gstage + ((size_t)p * 8 + i) * 128 + tid);
-      twell_tile32<8>(a.tw, g, p * 128 + tid, 0, tid, sm + L.emit, 1);
-    }
-  };
-  {
-    const int U = tpre[P];
-    const int r0 = (int)((long long)U * s / G), r1 = (int)((long long)U * (s + 1) / G);
-    if (r0 >= r1) emit_tiles();  // no rows for this CTA
-    for (int c0 = r0; c0 < r1; c0 += a.lcap) {
-      const int c1 = min(r1, c0 + a.lcap), Lc = c1 - c0;
-      const int n_groups = (Lc + RW_G - 1) / RW_G;
-      const int n_st = n_groups * 2;  // per group: its W_up rows, then its W_down rows
-      for (int p = tid; p < P; p += blockDim.x) {
-        if (tpre[p] <= c0 && c0 < tpre[p + 1]) misc[48] = p;
-        if (tpre[p] < c1 && c1 <= tpre[p + 1]) misc[49] = p;
-      }
-      __syncthreads();
-      const int pa = misc[48], pb = misc[49];
-      for (int e = tid; e < (pb - pa + 1) * 128; e += blockDim.x) {
-        const int p = pa + (e >> 7), bit = e & 127;
-        const uint4 m = ums[p];
-        if ((word4(m, bit >> 5) >> (bit & 31)) & 1u) {
-          const int rank = tpre[p] + popc_below(m, bit);
-          if (rank >= c0 && rank < c1) nid[rank - c0] = p * 128 + bit;
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t id = ib_id[cur * 8 + rr + e];
+          float h = 0.f;
+          if ((id >> (24 + tn)) & 1u) {
+            const float v = __uint_as_float(
+                (uint32_t)reinterpret_cast<const uint16_t*>(&ib_val[cur * 8 + rr + e])[tn] << 16);
+            h = v * (e ? u1 : u0);
+          }
+          hv[e] = h;
         }
+        split_hilo(hv[0], hv[1], bh, bl);
       }
-      for (int e = tid; e < Lc; e += blockDim.x) {
-        lmask[e] = 0u;
-        lval[e] = make_uint4(0, 0, 0, 0);
+      {  // W_down stage: y += h·W_down
+        const int k = kr + 1, sl = k & 1;
+        const bool ok = mbar_wait(&full[sl], r_par(k), abort_flag, a.status);
+        down_acc(ring_s + (uint32_t)(sl * SB) + lrow, ok, bh, bl);
+        __syncthreads();
+        if (have_next) issue_item(kr + 3, cur ^ 1);
+        if (!published) publish();  // while the next item's stages are in flight
       }
-      __syncthreads();
-      auto issue_r = [&](int q) {
-        const int n0 = (q >> 1) * RW_G;
-        issue_rows(gsq + q, (q & 1) ? a.W_down : a.W_up, nid + n0, min(RW_G, Lc - n0), 0);
-      };
-      for (int q = 0; q < ns && q < n_st; ++q) issue_r(q);
-      issued_end = gsq + min(ns, n_st);
-      if (c0 == r0) emit_tiles();  // while the first stages are in flight
-      // h's bf16 values v = bf16(sigma(g + b)) of the live tokens' kept
-      // pairs of this chunk's neurons: one thread per (neuron, token)
-      for (int e = tid; e < Lc * 8; e += blockDim.x) {
-        const int r = e >> 3, i = e & 7;
-        const int n = nid[r];
-        if (!((live >> i) & 1u)) continue;
-        if (!((a.kbits[(size_t)i * NG + (n >> 3)] >> (n & 7)) & 1u)) continue;
-        const float gv = __ldcg(a.gstage + ((size_t)(n >> 7) * 8 + i) * 128 + (n & 127)) +
-                         (a.tw.bias ? a.tw.bias[n] : 0.f);
-        reinterpret_cast<uint16_t*>(&lval[r])[i] = __bfloat16_as_ushort(__float2bfloat16_rn(act_fn(gv, a.tw.act)));
-        atomicOr(&lmask[r], 1u << i);
-      }
-      __syncthreads();
-      for (int g = 0; g < n_groups; ++g) {
-        const int n0 = g * RW_G, nn = min(RW_G, Lc - n0);
-        uint32_t bh = 0u, bl = 0u;
-        {  // up stage
-          const int q = 2 * g, gs = gsq + q, slot = gs % ns;
-          const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
-          float cu[4];
-          up_partial(ring_s + (uint32_t)(slot * SB) + lrow, ok, cu);
-          ured[warp * 32 + lane] = make_float2(cu[0], cu[1]);
-          __syncthreads();
-          if (q + ns < n_st) {
-            issue_r(q + ns);
-            issued_end = gs + ns + 1;
-          }
-          const int tn = lane >> 2, rr = 2 * (lane & 3);
-          float u0 = 0.f, u1 = 0.f;
-#pragma unroll
-          for (int w = 0; w < RW_WARPS; ++w) {
-            const float2 v = ured[w * 32 + lane];
-            u0 += v.x;
-            u1 += v.y;
-          }
-          float hv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int r = rr + e, n = n0 + r;
-            float h = 0.f;
-            if (r < nn && ((lmask[n] >> tn) & 1u)) {
-              const float v = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(&lval[n])[tn] << 16);
-              h = v * (e ? u1 : u0);
+      kr += 2;
+      if (!have_next) break;
+      cur ^= 1;
+      have_next = acquire(cur ^ 1);
+    }
+  }
+  // ------------------------------------------------------------- TwELL
+  // ([TwELL] "TwELL 減掉轉換開銷") CTA s writes the records of tiles [e_lo,
+  // e_hi) with warps 4-7, the tile kernels' emission from the staged gate
+  // values, while the reduce copies of y run.  A tile is complete once the
+  // CTAs that gated its groups have published their lists (the last steal
+  // scan usually saw them all).  The emission also flags each token that
+  // keeps more than C neurons of the tile (the hybrid routing: in this kernel
+  // such a token's kept rows were in the row lists like any other's).
+  const int e_lo = (int)(((long long)s * P + G - 1) / G), e_hi = (int)(((long long)(s + 1) * P + G - 1) / G);
+  const bool emitter = warp >= 4 && warp < 8 && e_lo < e_hi;
+  const int et = tid - 128;
+  float eg[8];
+  if (emitter) {
+    if (et == 0) {
+      int good = !*abort_flag;
+      if (good && !all_seen) {
+        // the CTA that gates group g: the v with g0(v) <= g < g1(v)
+        auto gater = [&](int g) {
+          int v = (int)((long long)g * G / NG);
+          while (v + 1 < G && (int)((long long)NG * (v + 1) / G) <= g) ++v;
+          while (v > 0 && (int)((long long)NG * v / G) > g) --v;
+          return v;
+        };
+        const uint64_t t0 = globaltimer();
+        for (int v = gater(e_lo * GPT); v <= gater(e_hi * GPT - 1) && good; ++v) {
+          for (;;) {
+            const uint32_t pv = (uint32_t)ld_acquire_gpu(sc + S.pub(v));
+            if ((pv >> 16) == (epoch & 0xFFFFu) && (pv & 0xFFFFu) != 0u) break;
+            if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+              atomicOr(a.status, DEV_ERR_TIMEOUT);
+              good = 0;
+              break;
             }
-            hv[e] = h;
-          }
-          split_hilo(hv[0], hv[1], bh, bl);
-        }
-        {  // down stage
-          const int q = 2 * g + 1, gs = gsq + q, slot = gs % ns;
-          const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
-          down_acc(ring_s + (uint32_t)(slot * SB) + lrow, ok, bh, bl);
-          __syncthreads();
-          if (q + ns < n_st) {
-            issue_r(q + ns);
-            issued_end = gs + ns + 1;
+            __nanosleep(128);
           }
         }
       }
-      gsq += n_st;
-      __syncthreads();
-      if (*abort_flag) break;
+      misc[DM_EMOK] = good;
+    }
+    named_bar_sync(1, 128);
+    if (misc[DM_EMOK]) {  // the first tile's values, loading while y goes out
+      const float b = a.tw.bias ? __ldg(a.tw.bias + e_lo * 128 + et) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) eg[i] = __ldcg(a.gstage + ((size_t)e_lo * 8 + i) * 128 + et) + b;
     }
   }
 
-  // -------------------------------------------- D: dense channel (overflow)
-  if (obits != 0u && !*abort_flag) {
-    const int n_st = 2 * (g1 - g0);  // per group: its W_gate rows, then its W_up rows
-    auto issue_d1 = [&](int q) {
-      issue_rows(gsq + q, (q & 1) ? a.W_up : a.W_gate, nullptr, RW_G, (g0 + (q >> 1)) * RW_G);
-    };
-    for (int q = 0; q < ns && q < n_st; ++q) issue_d1(q);
-    issued_end = gsq + min(ns, n_st);
-    for (int q = 0; q < n_st; ++q) {
-      const int gs = gsq + q, slot = gs % ns;
-      const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
-      float cu[4];
-      up_partial(ring_s + (uint32_t)(slot * SB) + lrow, ok, cu);
-      float2* ub = ured + (q & 1) * RW_WARPS * 32;  // g partials, then u partials
-      ub[warp * 32 + lane] = make_float2(cu[0], cu[1]);
-      __syncthreads();
-      if (q + ns < n_st) {
-        issue_d1(q + ns);
-        issued_end = gs + ns + 1;
-      }
-      if (q & 1) {
-        // h_tj = bf16(sigma(g + b))·u where kept, for the overflow tokens; 0 otherwise
-        if (warp == 0) {
-          float gv[2] = {0.f, 0.f}, uv[2] = {0.f, 0.f};
-#pragma unroll
-          for (int w = 0; w < RW_WARPS; ++w) {
-            const float2 vg = ured[w * 32 + lane], vu = ured[RW_WARPS * 32 + w * 32 + lane];
-            gv[0] += vg.x;
-            gv[1] += vg.y;
-            uv[0] += vu.x;
-            uv[1] += vu.y;
-          }
-          const int t = lane >> 2, j = (g0 + (q >> 1)) * RW_G + 2 * (lane & 3);
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float gb = gv[e] + (a.tw.bias ? a.tw.bias[j + e] : 0.f);
-            const float act = act_fn(gb, a.tw.act);
-            const bool keep = ((obits >> t) & 1u) && fabsf(act) > a.tw.tau;
-            const float v = __bfloat162float(__float2bfloat16_rn(act));
-            a.hdense[(size_t)t * F + j + e] = keep ? v * uv[e] : 0.f;
-          }
-        }
-        __syncthreads();  // the partials are read before the next group writes them
-      }
-    }
-    gsq += n_st;
-    // every overflow token's h is in
-    grid_barrier(a.gbar, abort_flag, a.status, bar_ok);
-    const int n_st2 = g1 - g0;
-    for (int q = 0; q < ns && q < n_st2; ++q) issue_rows(gsq + q, a.W_down, nullptr, RW_G, (g0 + q) * RW_G);
-    issued_end = gsq + min(ns, n_st2);
-    for (int q = 0; q < n_st2; ++q) {
-      const int gs = gsq + q, slot = gs % ns;
-      // this lane's B fragment: h of token lane/4 at neurons 2(lane%4), +1 of the group
-      const int j = (g0 + q) * RW_G + 2 * (lane & 3);
-      const float2 hv = __ldcg(reinterpret_cast<const float2*>(a.hdense + (size_t)(lane >> 2) * F + j));
-      uint32_t bh, bl;
-      split_hilo(hv.x, hv.y, bh, bl);
-      const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
-      down_acc(ring_s + (uint32_t)(slot * SB) + lrow, ok, bh, bl);
-      __syncthreads();
-      if (q + ns < n_st2) {
-        issue_rows(gs + ns, a.W_down, nullptr, RW_G, (g0 + q + ns) * RW_G);
-        issued_end = gs + ns + 1;
-      }
-    }
-    gsq += n_st2;
-  }
-
-  // drain copies still in flight (only after an abort): the last fill of every slot
+  // ---------------------------------------------------------------- y out
+  // drain copies still in flight (only after an abort): the last x copy and
+  // the last fill of every slot (misc holds the parity of each last phase)
   if (tid == 0 && *abort_flag) {
-    for (int k = 0; k < ns && k < issued_end; ++k) {
-      const int last = issued_end - 1 - k;
+    const uint64_t tx = globaltimer();
+    while (!mbar_try_wait(xbar, (uint32_t)((misc[DM_XLK] - 1) & 1))) {
+      if (globaltimer() - tx > SFFN_WAIT_LIMIT_NS) break;
+    }
+    for (int sl = 0; sl < 3; ++sl) {
+      const int par = misc[DM_LK0 + sl];
+      if (par < 0) continue;
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&full[last % ns], (uint32_t)((last / ns) & 1))) {
+      while (!mbar_try_wait(&full[sl], (uint32_t)par)) {
         if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) break;
       }
     }
   }
   __syncthreads();
-  const bool okall = !*abort_flag;
-
   // partial y -> red[8][d] (rows padded by 4 floats against bank conflicts,
   // over the x block and the ring), then out by bulk reduce-add per token
   const int RP = d + 4;
@@ -554,12 +658,46 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     }
   }
   fence_proxy_async_smem();
-  __syncthreads();
-  if (tid < nvalid && okall) {
+  // every CTA's slice of out is zero (it published its list after zeroing;
+  // the last steal scan may have seen every list already)
+  if (tid < G && !all_seen) {
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+      const uint32_t pv = (uint32_t)ld_acquire_gpu(sc + S.pub(tid));
+      if ((pv >> 16) == (epoch & 0xFFFFu) && (pv & 0xFFFFu) != 0u) break;
+      if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+        atomicOr(a.status, DEV_ERR_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  const bool okall = !__syncthreads_or(*abort_flag);
+  // eight pieces per token row, each CTA starting at a different piece so
+  // that the grid's adds spread over the output's L2 lines
+  if (tid < nvalid * 8 && okall) {
+    const int t = tid >> 3, c = ((tid & 7) + s) & 7, n = d >> 3;
     asm volatile("fence.proxy.async.global;" ::: "memory");  // after the other CTAs' zeroing of out
-    bulk_reduce_add_f32(a.out + (size_t)tid * d, red + tid * RP, (uint32_t)d * 4u);
+    bulk_reduce_add_f32(a.out + (size_t)t * d + c * n, red + t * RP + c * n, (uint32_t)n * 4u);
     bulk_commit();
-    bulk_wait_all();
+    bulk_wait_read();  // the grid's end completes the writes
+  }
+  if (emitter && misc[DM_EMOK]) {
+    TwellParams twb = a.tw;  // the emission gets g + b
+    twb.bias = nullptr;
+    for (int p = e_lo; p < e_hi; ++p) {
+      float g[8];
+      if (p == e_lo) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[i] = eg[i];
+      } else {
+        const float b = a.tw.bias ? __ldg(a.tw.bias + p * 128 + et) : 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[i] = __ldcg(a.gstage + ((size_t)p * 8 + i) * 128 + et) + b;
+      }
+      twell_tile32<8>(twb, g, p * 128 + et, 0, et, sm + L.emit, 1);
+    }
   }
 }
 

@@ -203,12 +203,15 @@ struct sffn_handle {
   int* gtick = nullptr;
   int gr_nslot = 0, gr_smem = 0;
   bool gr_ok = false;
-  // single persistent launch for T <= 8: dense-channel h, grid barrier, launch shape
-  float* hdense = nullptr;
-  uint8_t* kbits = nullptr;
-  unsigned* gbar = nullptr;
-  int dec_nslot = 0, dec_lcap = 0, dec_smem = 0, dec_grid = 0;
+  // single persistent launch for T <= 8: scheduler words, published row lists, launch shape
+  int* dsched = nullptr;
+  int dsched_ints = 0;
+  uint32_t* wl_id = nullptr;
+  uint4* wl_val = nullptr;
+  int dec_maxr = 0, dec_smem = 0, dec_grid = 0;
   bool dec_ok = false;
+  bool last_fused = false;     // the last forward was the single launch: its routing is the ovf flags
+  uint32_t last_epoch = 0;
   // per-kernel timing (sffn_timing_begin/end)
   bool tm_on = false;
   int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
@@ -227,7 +230,7 @@ void free_handle(sffn_handle* h) {
   void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zpart,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->zero_row, h->gstage, h->gtick, h->hdense, h->kbits, h->gbar};
+                  h->zero_row, h->gstage, h->gtick, h->dsched, h->wl_id, h->wl_val};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -399,9 +402,6 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   if (!h->f32 && !h->wina && !h->lowrank) {
     ok = ok && dalloc(&h->gstage, P * 8 * 128 * 4);
     ok = ok && dalloc(&h->gtick, P * 4);
-    ok = ok && dalloc(&h->hdense, 8 * F * 4);
-    ok = ok && dalloc(&h->kbits, F);
-    ok = ok && dalloc(&h->gbar, 16);
   }
   if (!ok) {
     free_handle(h);
@@ -413,7 +413,6 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
   if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, std::max<size_t>(2048, d * 2), st);
   if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
-  if (h->gbar) e = e ? e : cudaMemsetAsync(h->gbar, 0, 16, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * 4, st);
   }
@@ -485,20 +484,31 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem;
       if (h->gr_ok)
         e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->gr_smem);
-      // the single persistent launch: two ring slots, the largest rank list that fits,
-      // and exactly as many CTAs as can be resident at once (its grid barriers need that)
-      int dl = 512;
-      while (dl > 64 && DecodeSmem::make(h->P, h->C, dl, h->d, 2).total > max_smem) dl -= 64;
-      h->dec_nslot = 2;
-      h->dec_lcap = dl;
-      h->dec_smem = DecodeSmem::make(h->P, h->C, dl, h->d, 2).total;
-      h->dec_ok = h->gr_ok && h->rows_ok && h->dec_smem <= max_smem && h->P <= RW_THREADS;
+      // the single persistent launch: one CTA per SM, all resident at once (a CTA
+      // may wait for another's list or zeroed slice of out), lists sized for the
+      // most gate groups one CTA takes
+      const int G = h->n_sm, NG = (int)(F / RW_G), gmax = cdiv(NG, G);
+      h->dec_grid = G;
+      h->dec_maxr = gmax * RW_G;
+      h->dec_smem = DecodeSmem::make(h->C, h->dec_maxr, h->d).total;
+      h->dec_ok = h->gr_ok && h->rows_ok && h->dec_smem <= max_smem && G <= RW_THREADS && F < (1 << 24) &&
+                  h->dec_maxr < (1 << 16);
       if (h->dec_ok && !e) {
         e = cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, h->dec_smem);
         int nb = 0;
         if (!e) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode, RW_THREADS, h->dec_smem);
-        h->dec_grid = nb * h->n_sm;
         h->dec_ok = !e && nb >= 1;
+      }
+      if (h->dec_ok && !e) {
+        h->dsched_ints = decode_sched_ints((int)P, G);
+        bool aok = dalloc(&h->dsched, (size_t)h->dsched_ints * 4);
+        aok = aok && dalloc(&h->wl_id, (size_t)G * h->dec_maxr * 4);
+        aok = aok && dalloc(&h->wl_val, (size_t)G * h->dec_maxr * 16);
+        if (!aok) {
+          free_handle(h);
+          return SFFN_ERR_ALLOC;
+        }
+        e = cudaMemsetAsync(h->dsched, 0, (size_t)h->dsched_ints * 4, st);
       }
     }
   }
@@ -585,21 +595,19 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     da.zero_row = h->zero_row;
     da.tw = tw;
     da.gstage = h->gstage;
-    da.kbits = h->kbits;
-    da.gbar = h->gbar;
-    da.ovf_list = h->ovf_list;
-    da.ovf_count = h->ovf_count;
-    da.hdense = h->hdense;
+    da.sched = h->dsched;
+    da.wl_id = h->wl_id;
+    da.wl_val = h->wl_val;
+    da.maxr = h->dec_maxr;
     da.out = out;
     da.d = d;
-    da.nslot = h->dec_nslot;
-    da.lcap = h->dec_lcap;
     da.status = h->status;
     tmark(h, st, L_DECODE);
     if (launch_pdl(k_decode, dim3(h->dec_grid), dim3(RW_THREADS), (size_t)h->dec_smem, st, 1, da))
       return SFFN_ERR_CUDA;
     h->last_path = SFFN_PATH_ROWS;
     h->last_launches = 1;
+    h->last_fused = true;
     return SFFN_OK;
   }
 
@@ -854,6 +862,8 @@ sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void*
   ++h->epoch;
   if (h->epoch == 0) ++h->epoch;  // 0 marks "never overflowed"
   h->last_T = T;
+  h->last_epoch = h->epoch;
+  h->last_fused = false;
   tmark_begin(h);
   const sffn_status r = h->f32 ? forward_f32(h, x, T, out, st) : forward_bf16(h, x, T, out, st);
   tmark_end(h, st);
@@ -946,7 +956,12 @@ sffn_status sffn_read_status(sffn_handle* h, void* cuda_stream) {
   uint32_t w = 0;
   if (cudaStreamSynchronize(st) != cudaSuccess) return SFFN_ERR_CUDA;
   if (cudaMemcpy(&w, h->status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFFN_ERR_CUDA;
-  if (w) cudaMemset(h->status, 0, 4);
+  if (w) {
+    cudaMemset(h->status, 0, 4);
+    // a CTA that gave up may have left scheduler words of the single-launch
+    // decode kernel set: start the next forward from zero
+    if (h->dsched) cudaMemset(h->dsched, 0, (size_t)h->dsched_ints * 4);
+  }
   if (w & DEV_ERR_TIMEOUT) return SFFN_ERR_TIMEOUT;
   if (w & DEV_ERR_RANGE) return SFFN_ERR_DEVICE;
   return SFFN_OK;
@@ -983,7 +998,16 @@ sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st) {
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   int n = 0;
   if (cudaStreamSynchronize(s) != cudaSuccess) return SFFN_ERR_CUDA;
-  if (cudaMemcpy(&n, h->ovf_count, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFFN_ERR_CUDA;
+  if (h->last_fused) {
+    // the single launch routes implicitly (an overflow token's kept rows are
+    // in the row lists); its record of the routing is the per-token flags
+    std::vector<uint32_t> f(std::max(h->last_T, 1));
+    if (cudaMemcpy(f.data(), h->ovf, (size_t)h->last_T * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return SFFN_ERR_CUDA;
+    for (int t = 0; t < h->last_T; ++t) n += f[t] == h->last_epoch;
+  } else if (cudaMemcpy(&n, h->ovf_count, 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    return SFFN_ERR_CUDA;
+  }
   st->n_overflow = n;
   st->n_launches = h->last_launches;
   st->path = h->last_path;
