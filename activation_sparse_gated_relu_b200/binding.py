@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_debug_twell.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                      ctypes.POINTER(vp), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.sffn_debug_twell.restype = st
+    lib.sffn_debug_keep.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.sffn_debug_keep.restype = st
     lib.sffn_debug_gate.argtypes = [vp, ctypes.POINTER(vp)]
     lib.sffn_debug_gate.restype = st
     lib.sffn_debug_norms.argtypes = [vp, ctypes.POINTER(vp)]
@@ -249,6 +251,12 @@ class SparseFFN:
         return {"count": _view(c.value, (T, P), "<i2"), "idx": _view(i.value, (T, P, C), "<i2"),
                 "val": _view(v.value, (T, P, C), vt[0], vt[1]),
                 "overflow_epoch": _view(o.value, (T,), "<u4")}
+
+    def keep_masks(self, T: int):
+        """The last ROWS-path forward's keep masks, uint32 [T][n_tiles][4]."""
+        k = ctypes.c_void_p()
+        _check(load_library().sffn_debug_keep(self.h, ctypes.byref(k)), "keep_masks")
+        return _view(k.value, (T, self.d_ff // 128, 4), "<u4")
 
     def gate_debug(self, T: int):
         g = ctypes.c_void_p()

@@ -979,6 +979,12 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
   return SFFN_OK;
 }
 
+sffn_status sffn_debug_keep(sffn_handle* h, const uint32_t** keep) {
+  if (!h || !keep) return SFFN_ERR_INVALID_ARG;
+  *keep = h->kmask;
+  return SFFN_OK;
+}
+
 sffn_status sffn_debug_gate(sffn_handle* h, const float** g) {
   if (!h || !g) return SFFN_ERR_INVALID_ARG;
   if (!h->gdebug) return SFFN_ERR_UNSUPPORTED;

@@ -270,11 +270,13 @@ def kernel_work(wl, T: int, path: str, st: dict) -> dict:
         if wl.mode != "wina_topk":
             w["fallback_h"] = {"bytes": dense_in + n_o * F * 4, "flops": 2 * n_o * d * F}
         w["down"] = {"bytes": (F * d * es + n_o * F * 4 + n_o * d * 4) if n_o else 0, "flops": 2 * n_o * F * d}
-        # the single persistent launch (T <= 8) does all of the above; the gate
-        # TwELL and keep masks stay on chip-near L2 between its phases but are
-        # still written and read, so they count like the separate kernels'
-        w["decode_fused"] = {"bytes": sum(w[k]["bytes"] for k in (g, "updown_rows", "fallback_h", "down")) - xb,
-                             "flops": sum(w[k]["flops"] for k in (g, "updown_rows", "fallback_h", "down"))}
+        # the single persistent launch (T <= 8): W_gate once, the W_up and
+        # W_down rows of every token's kept neurons (an overflow token's too:
+        # it has no separate dense channel), x in, y out, the TwELL records
+        # and keep masks written once
+        Ua, nnza = st.get("union_all", U), st.get("nnz_all", nnz)
+        w["decode_fused"] = {"bytes": F * d * es + xb + Ua * 2 * d * es + yb + twell + kmask,
+                             "flops": 2 * T * d * F + 4 * nnza * d}
     else:
         w["router"] = {"bytes": yb + 2 * n_o * d * es, "flops": 0}
         w["tile_h"] = {"bytes": F * d * es + xb + twell + T * F * 4, "flops": 2 * T * d * F}
@@ -337,8 +339,17 @@ def batch_sparsity(ffn, T: int, C: int) -> dict:
     kept_idx, kept_tok = idx[used], tok[used]
     blocks = torch.zeros(((T + 7) // 8, ffn.d_ff), dtype=torch.bool, device=cnt.device)
     blocks[kept_tok // 8, kept_idx] = True
-    return {"union": int(torch.unique(kept_idx).numel()), "nnz": int(kept_idx.numel()),
-            "block_rows": int(blocks.sum()), "n_overflow": int(ovf.sum())}
+    st = {"union": int(torch.unique(kept_idx).numel()), "nnz": int(kept_idx.numel()),
+          "block_rows": int(blocks.sum()), "n_overflow": int(ovf.sum())}
+    # every token's full kept set (overflow tokens too), from the keep masks
+    # of a ROWS-path forward: what the single launch streams
+    st["union_all"], st["nnz_all"] = st["union"], st["nnz"]
+    if ffn.stats().path == 1:
+        km = ffn.keep_masks(T).to(torch.int64) & 0xFFFFFFFF
+        bits = ((km[..., None] >> torch.arange(32, device=km.device)) & 1).bool()  # [T][P][4][32]
+        st["nnz_all"] = int(bits.sum())
+        st["union_all"] = int(bits.any(dim=0).sum())
+    return st
 
 
 def run_ours(args) -> None:

@@ -157,6 +157,12 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
                              const void** val, const uint32_t** overflow, int* n_tiles,
                              int* tile_capacity);
 
+/* Device view of the last forward's keep masks: uint32 [T][n_tiles][4], bit
+ * (32 w + b) of word w set iff the token keeps neuron 128 p + 32 w + b of tile
+ * p, with no capacity limit (an overflow token's full kept set).  Written by
+ * the ROWS path only (undefined after a TILES forward).  Test and bench use. */
+sffn_status sffn_debug_keep(sffn_handle* h, const uint32_t** keep);
+
 /* Device view of the dense fp32 gate g[T][d_ff] of the last forward (only
  * with SFFN_FLAG_DEBUG_GATE; dense gate only).  Test use. */
 sffn_status sffn_debug_gate(sffn_handle* h, const float** g);

@@ -78,8 +78,14 @@ def test_work_model_decode_matches_byte_formula():
     assert f == 2 * 8 * wl.d_model * wl.d_ff + 4 * 12000 * wl.d_model
     w = bench.kernel_work(wl, 8, "rows", st)
     assert set(w) == {"gate", "updown_rows", "fallback_h", "down", "decode_fused"}
-    # the single launch moves the step's bytes plus the keep masks written and read
-    assert w["decode_fused"]["bytes"] == b + 2 * 8 * P * 16
+    # the single launch moves the step's bytes with the TwELL records and keep
+    # masks written once (nothing reads them back inside it)
+    assert w["decode_fused"]["bytes"] == b - twell + 8 * P * 16
+    # an overflow token's kept rows stream with the others in the single launch
+    st2 = dict(st, n_overflow=1, union_all=9000, nnz_all=12500)
+    w2 = bench.kernel_work(wl, 8, "rows", st2)
+    assert w2["decode_fused"]["bytes"] == w["decode_fused"]["bytes"] + (9000 - 8163) * 2 * wl.d_model * 2
+    assert w2["decode_fused"]["flops"] == 2 * 8 * wl.d_model * wl.d_ff + 4 * 12500 * wl.d_model
     # no overflow: the dense channel moves nothing
     assert w["fallback_h"]["bytes"] == 0 and w["down"]["flops"] == 0
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
