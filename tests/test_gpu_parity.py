@@ -227,10 +227,41 @@ def test_decode_single_launch_and_separate_kernels(decode_inputs):
 
 @pytest.mark.parametrize("C", [8, 16])
 def test_decode_single_launch_dense_channel(decode_inputs, C):
-    # small capacities make tokens overflow: the single launch's dense channel
-    # (its third phase, after a second grid barrier) computes their outputs
+    # small capacities make tokens overflow: in the single launch their kept
+    # rows stream with everyone else's (the dense channel's sum without its
+    # zero terms); their TwELL records cap at C and their flags are set
     st = check(decode_inputs, T=8, C=C)
     assert st["overflow"] > 0 and st["launches"] == 1
+
+
+@pytest.mark.parametrize("d_ff,T", [(128, 8), (512, 3), (1024, 1)])
+def test_decode_single_launch_few_gate_groups(d_ff, T):
+    # fewer 8-neuron gate groups than SMs: most CTAs gate nothing, build no
+    # list and only steal; one tile at d_ff = 128
+    inp = synth.make_inputs(small(tokens=T, d_model=512, d_ff=d_ff))
+    st = check(inp, path="rows")
+    assert st["launches"] == 1
+
+
+def test_decode_single_launch_silu_no_bias():
+    inp = synth.make_inputs(small(tokens=7, d_model=1024, d_ff=2048, act="silu", threshold=0.3, bias=None))
+    st = check(inp, path="rows")
+    assert st["launches"] == 1
+
+
+def test_decode_single_launch_repeated_mixed_T(decode_inputs):
+    # the scheduler words carry each forward's epoch: back-to-back forwards of
+    # different sizes through one handle see only their own lists and zeros
+    ffn = make_ffn(decode_inputs, max_tokens=8)
+    res = {}
+    try:
+        for T in (8, 3, 8, 1, 5, 8, 8):
+            if T not in res:
+                res[T] = oracle.forward_inputs(decode_inputs, T=T)
+            st = check(decode_inputs, T=T, ffn=ffn, res=res[T])
+            assert st["launches"] == 1
+    finally:
+        ffn.close()
 
 
 def test_lopa_config():
