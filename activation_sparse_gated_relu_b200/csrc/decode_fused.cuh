@@ -144,7 +144,6 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   const uint32_t hi_off = (lane >> 4) ? 32u * RW_WARPS : 0u;
   const uint32_t xsl = smem_u32(sm + L.xs) + lrow;
 
-  griddep_wait();  // x, out and the workspace belong to the stream order
   // ---------------------------------------------------------------- setup
   // The gate streams through three slots, the two ring slots and the x
   // block: x moves into registers for the gate (the partial y is not live
@@ -161,16 +160,20 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     misc[DM_ABORT] = 0;
     misc[DM_LK0] = misc[DM_LK0 + 1] = misc[DM_LK0 + 2] = -1;
     fence_mbar_init();
-    mbar_expect_tx(xbar, (uint32_t)(nvalid * d * 2));
-    misc[DM_XLK] = 1;
-    for (int t = 0; t < nvalid; ++t) bulk_g2s(sm + L.xs + t * RS, a.x + (size_t)t * d, (uint32_t)d * 2u, xbar);
-    // the gate's first stages go out with x
+    // the gate's first stages: the weights stay unchanged for the handle's
+    // life, so they load before the previous grid on the stream has finished
     for (int q = 0; q < 2 && q < n_g; ++q) {
       mbar_expect_tx(&full[q], (uint32_t)(RW_G * d * 2));
       misc[DM_LK0 + q] = 0;
       for (int r = 0; r < RW_G; ++r)
         bulk_g2s(ring + (size_t)q * SB + r * RS, a.W_gate + (size_t)((g0 + q) * RW_G + r) * d, (uint32_t)d * 2u, &full[q]);
     }
+  }
+  griddep_wait();  // x, out and the workspace belong to the stream order
+  if (tid == 0) {
+    mbar_expect_tx(xbar, (uint32_t)(nvalid * d * 2));
+    misc[DM_XLK] = 1;
+    for (int t = 0; t < nvalid; ++t) bulk_g2s(sm + L.xs + t * RS, a.x + (size_t)t * d, (uint32_t)d * 2u, xbar);
   }
   for (int e = tid; e < (8 - nvalid) * (d >> 3); e += blockDim.x) {
     const int t = nvalid + e / (d >> 3), v = e % (d >> 3);
@@ -577,6 +580,11 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
       have_next = acquire(cur ^ 1);
     }
   }
+  // This CTA streams no more weights: the next forward's launch may begin
+  // (its CTAs take an SM as ours leave and load their first gate stages
+  // while the output copies of this one run).
+  griddep_launch();
+
   // ------------------------------------------------------------- TwELL
   // ([TwELL] "TwELL 減掉轉換開銷") CTA s writes the records of tiles [e_lo,
   // e_hi) with warps 4-7, the tile kernels' emission from the staged gate

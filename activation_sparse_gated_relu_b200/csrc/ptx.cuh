@@ -205,6 +205,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // attribute.  Every kernel calls it before touching data that an earlier
 // kernel writes or reads.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream (launched with programmatic stream
+// serialisation) begin its launch; it still waits in griddep_wait until this
+// grid has completed.
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------- misc
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
