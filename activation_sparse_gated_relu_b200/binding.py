@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_debug_twell.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                      ctypes.POINTER(vp), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.sffn_debug_twell.restype = st
+    lib.sffn_debug_decode_waits.argtypes = [vp, ctypes.c_int, ctypes.c_uint]
+    lib.sffn_debug_decode_waits.restype = st
     lib.sffn_debug_keep.argtypes = [vp, ctypes.POINTER(vp)]
     lib.sffn_debug_keep.restype = st
     lib.sffn_debug_gate.argtypes = [vp, ctypes.POINTER(vp)]
@@ -251,6 +253,11 @@ class SparseFFN:
         return {"count": _view(c.value, (T, P), "<i2"), "idx": _view(i.value, (T, P, C), "<i2"),
                 "val": _view(v.value, (T, P, C), vt[0], vt[1]),
                 "overflow_epoch": _view(o.value, (T,), "<u4")}
+
+    def debug_decode_waits(self, phantom_ctas: int, wait_us: int) -> None:
+        """Test hook: single-launch decode forwards await `phantom_ctas` CTAs
+        that never run, with waits of `wait_us` µs (0, 0 restores)."""
+        _check(load_library().sffn_debug_decode_waits(self.h, phantom_ctas, wait_us), "debug_decode_waits")
 
     def keep_masks(self, T: int):
         """The last ROWS-path forward's keep masks, uint32 [T][n_tiles][4]."""

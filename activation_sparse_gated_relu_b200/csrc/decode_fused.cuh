@@ -70,6 +70,8 @@ struct DecodeArgs {
   float* out;                    // [T][d]
   int d;
   uint32_t* status;
+  unsigned long long wait_ns;    // limit of the waits on other CTAs
+  int phantom;                   // test hook: CTAs counted in the grid that never run (0 or 1)
 };
 
 // Scheduler words, in ints from the start of DecodeArgs::sched.  A list
@@ -132,7 +134,8 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, s = blockIdx.x;
-  const DecodeSched S{P, G};
+  const DecodeSched S{P, G + 1};  // one spare slot: the test hook's CTA that never runs
+  const int GS = G + a.phantom;    // the CTAs whose lists and zeroed slices are awaited
   int* sc = a.sched;
   const int nj = d / RW_DIV;
   const int NG = F / RW_G;
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
         for (;;) {
           int key = -1;
           bool unpub = false;
-          if (tid < G && tid != s) {
+          if (tid < GS && tid != s) {
             const uint32_t pv = (uint32_t)ld_acquire_gpu(sc + S.pub(tid));
             const int len = (int)(pv & 0xFFFFu) - 1;
             if ((pv >> 16) != (epoch & 0xFFFFu) || len < 0) {
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
                 res = 1;
               }
             } else if (n_unpub > 0) {  // lists still being gated: wait for them, bounded
-              if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+              if (globaltimer() - t0 > a.wait_ns) {
                 atomicOr(a.status, DEV_ERR_TIMEOUT);
                 *abort_flag = 1;
                 res = 2;
@@ -613,7 +616,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
           for (;;) {
             const uint32_t pv = (uint32_t)ld_acquire_gpu(sc + S.pub(v));
             if ((pv >> 16) == (epoch & 0xFFFFu) && (pv & 0xFFFFu) != 0u) break;
-            if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+            if (globaltimer() - t0 > a.wait_ns) {
               atomicOr(a.status, DEV_ERR_TIMEOUT);
               good = 0;
               break;
@@ -668,12 +671,12 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   fence_proxy_async_smem();
   // every CTA's slice of out is zero (it published its list after zeroing;
   // the last steal scan may have seen every list already)
-  if (tid < G && !all_seen) {
+  if (tid < GS && !all_seen) {
     const uint64_t t0 = globaltimer();
     for (;;) {
       const uint32_t pv = (uint32_t)ld_acquire_gpu(sc + S.pub(tid));
       if ((pv >> 16) == (epoch & 0xFFFFu) && (pv & 0xFFFFu) != 0u) break;
-      if (globaltimer() - t0 > SFFN_WAIT_LIMIT_NS) {
+      if (globaltimer() - t0 > a.wait_ns) {
         atomicOr(a.status, DEV_ERR_TIMEOUT);
         *abort_flag = 1;
         break;

@@ -210,6 +210,8 @@ struct sffn_handle {
   uint4* wl_val = nullptr;
   int dec_maxr = 0, dec_smem = 0, dec_grid = 0;
   bool dec_ok = false;
+  int dec_phantom = 0;           // test hook (sffn_debug_decode_waits)
+  unsigned long long dec_wait_ns = SFFN_WAIT_LIMIT_NS;
   bool last_fused = false;     // the last forward was the single launch: its routing is the ovf flags
   uint32_t last_epoch = 0;
   // per-kernel timing (sffn_timing_begin/end)
@@ -500,7 +502,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
         h->dec_ok = !e && nb >= 1;
       }
       if (h->dec_ok && !e) {
-        h->dsched_ints = decode_sched_ints((int)P, G);
+        h->dsched_ints = decode_sched_ints((int)P, G + 1);
         bool aok = dalloc(&h->dsched, (size_t)h->dsched_ints * 4);
         aok = aok && dalloc(&h->wl_id, (size_t)G * h->dec_maxr * 4);
         aok = aok && dalloc(&h->wl_val, (size_t)G * h->dec_maxr * 16);
@@ -602,6 +604,8 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     da.out = out;
     da.d = d;
     da.status = h->status;
+    da.wait_ns = h->dec_wait_ns;
+    da.phantom = h->dec_phantom;
     tmark(h, st, L_DECODE);
     if (launch_pdl(k_decode, dim3(h->dec_grid), dim3(RW_THREADS), (size_t)h->dec_smem, st, 1, da))
       return SFFN_ERR_CUDA;
@@ -976,6 +980,13 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
   if (overflow) *overflow = h->ovf;
   if (n_tiles) *n_tiles = h->P;
   if (tile_capacity) *tile_capacity = h->C;
+  return SFFN_OK;
+}
+
+sffn_status sffn_debug_decode_waits(sffn_handle* h, int phantom_ctas, unsigned wait_us) {
+  if (!h || phantom_ctas < 0 || phantom_ctas > 1) return SFFN_ERR_INVALID_ARG;
+  h->dec_phantom = phantom_ctas;
+  h->dec_wait_ns = wait_us ? (unsigned long long)wait_us * 1000ull : SFFN_WAIT_LIMIT_NS;
   return SFFN_OK;
 }
 

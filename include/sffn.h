@@ -157,6 +157,16 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
                              const void** val, const uint32_t** overflow, int* n_tiles,
                              int* tile_capacity);
 
+/* Test hook for the bounded waits of the single-launch decode forward (ROWS
+ * path, T <= 8).  Until called again with (0, 0), those forwards count
+ * `phantom_ctas` (0 or 1) extra CTAs in their grid that never run, so every
+ * wait on them expires, and limit their waits on other CTAs to `wait_us`
+ * microseconds (0: the default of 2 s).  Such a forward's out is not valid
+ * and it sets the status word's timeout (sffn_read_status returns
+ * SFFN_ERR_TIMEOUT and clears the scheduler state); nothing faults or hangs.
+ * Errors: SFFN_ERR_INVALID_ARG for a null handle or phantom_ctas not 0 or 1. */
+sffn_status sffn_debug_decode_waits(sffn_handle* h, int phantom_ctas, unsigned wait_us);
+
 /* Device view of the last forward's keep masks: uint32 [T][n_tiles][4], bit
  * (32 w + b) of word w set iff the token keeps neuron 128 p + 32 w + b of tile
  * p, with no capacity limit (an overflow token's full kept set).  Written by

@@ -249,6 +249,27 @@ def test_decode_single_launch_silu_no_bias():
     assert st["launches"] == 1
 
 
+def test_decode_single_launch_bounded_waits(decode_inputs):
+    # every wait on another CTA is bounded: with a CTA in the grid that never
+    # runs (a list never published, a slice of out never zeroed) the launch
+    # gives up after the limit and reports a timeout, and the handle works
+    # again afterwards
+    from activation_sparse_gated_relu_b200 import SFFN_ERR_TIMEOUT
+    ffn = make_ffn(decode_inputs, max_tokens=8)
+    try:
+        x = to_dev(decode_inputs.x[:8])
+        out = torch.full((8, ffn.d_model), 7.0, dtype=torch.float32, device="cuda")
+        ffn.debug_decode_waits(1, 20000)
+        ffn.forward(x, out)
+        torch.cuda.synchronize()
+        assert ffn.read_status() == SFFN_ERR_TIMEOUT
+        ffn.debug_decode_waits(0, 0)
+        st = check(decode_inputs, T=8, ffn=ffn)
+        assert st["launches"] == 1
+    finally:
+        ffn.close()
+
+
 def test_decode_single_launch_repeated_mixed_T(decode_inputs):
     # the scheduler words carry each forward's epoch: back-to-back forwards of
     # different sizes through one handle see only their own lists and zeros
