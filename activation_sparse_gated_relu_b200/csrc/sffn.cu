@@ -30,6 +30,7 @@
 #include "../../include/sffn.h"
 #include "epilogues.cuh"
 #include "decode_fused.cuh"
+#include "tc_gate_persist.cuh"
 #include "gate_rows.cuh"
 #include "rows_mma.cuh"
 #include "simt.cuh"
@@ -143,6 +144,30 @@ cudaError_t launch_tc(int BN, dim3 grid, cudaStream_t st, const CUtensorMap& a0,
     case 128: return launch_tc_bn<128, Epi>(grid, st, a0, b0, a1, b1, args, ep);
     default: return launch_tc_bn<256, Epi>(grid, st, a0, b0, a1, b1, args, ep);
   }
+}
+
+// The persistent gate for as many 128-neuron x BN-token tiles as there are
+// SMs or more: one CTA per SM walks the tiles (tc_gate_persist.cuh).
+cudaError_t launch_gate_persist(int BN, int n_sm, int n_work, cudaStream_t st, const CUtensorMap& a,
+                                const CUtensorMap& b, const TcArgs& args, const TwellParams& tw) {
+  const dim3 grid(std::min(n_sm, n_work)), block(TP_THREADS);
+  const size_t smem = (size_t)tp_layout(BN, tw.C).total;
+  switch (BN) {
+    case 16: return launch_pdl(k_tc_gate_persist<16>, grid, block, smem, st, 1, a, b, args, tw);
+    case 32: return launch_pdl(k_tc_gate_persist<32>, grid, block, smem, st, 1, a, b, args, tw);
+    case 64: return launch_pdl(k_tc_gate_persist<64>, grid, block, smem, st, 1, a, b, args, tw);
+    case 128: return launch_pdl(k_tc_gate_persist<128>, grid, block, smem, st, 1, a, b, args, tw);
+    default: return launch_pdl(k_tc_gate_persist<256>, grid, block, smem, st, 1, a, b, args, tw);
+  }
+}
+cudaError_t set_gate_persist_attrs(int C) {
+  cudaError_t e = cudaSuccess;
+  e = e ? e : cudaFuncSetAttribute(k_tc_gate_persist<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, tp_layout(16, C).total);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gate_persist<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, tp_layout(32, C).total);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gate_persist<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, tp_layout(64, C).total);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gate_persist<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, tp_layout(128, C).total);
+  e = e ? e : cudaFuncSetAttribute(k_tc_gate_persist<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, tp_layout(256, C).total);
+  return e;
 }
 
 template <class Epi>
@@ -445,6 +470,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   // kernel attributes and A-operand tensor maps
   if (!e && !h->f32) {
     e = e ? e : set_tc_attrs<EpiGateTwell>();
+    e = e ? e : set_gate_persist_attrs(h->C);
     e = e ? e : set_tc_attrs<EpiWina>();
     e = e ? e : set_tc_attrs<EpiLowRankZ>();
     e = e ? e : set_tc_attrs<EpiFallbackH>();
@@ -675,6 +701,10 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
       gr.status = h->status;
       e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS), (size_t)h->gr_smem, st, 1,
                      gr);
+    } else if (P * ntile_tok > h->n_sm && !(D.flags & SFFN_FLAG_SEPARATE)) {
+      // at least a tile per SM: the persistent gate overlaps each tile's
+      // TwELL emission with the next tile's MMAs
+      e = launch_gate_persist(BN, h->n_sm, P * ntile_tok, st, *gateA, *gateB, ga, tw);
     } else {
       e = launch_tc<EpiGateTwell>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, tw);
     }

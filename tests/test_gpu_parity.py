@@ -333,6 +333,20 @@ def test_prefill_sampled_full_size():
     compare_twell(sub, res, wl.tile_capacity, ambiguous(res, "relu_threshold", 0.0, 0, False), False, "bf16")
 
 
+@pytest.mark.parametrize("exact", [False, True])
+def test_persistent_gate_many_tiles(exact):
+    # more 128-neuron x token tiles than SMs: the persistent gate (two TMEM
+    # accumulators, each tile's emission beside the next tile's MMAs); 1200
+    # tokens leave a ragged last token tile.  The separate flag keeps the
+    # one-CTA-per-tile gate, which must agree.
+    inp = synth.make_inputs(small(tokens=1200, d_model=256, d_ff=4096, exact_grid=exact))
+    res = oracle.forward_inputs(inp)
+    a = check(inp, res=res)
+    b = check(inp, res=res, separate=True)
+    if exact:
+        assert a["mismatch"] == 0 and b["mismatch"] == 0
+
+
 def test_prefill_reduced_full_check():
     inp = synth.make_inputs(W["prefill_bf16"], T=384)
     st = check(inp)
