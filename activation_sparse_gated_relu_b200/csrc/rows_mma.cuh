@@ -8,14 +8,16 @@
 // number of rows.  CTA 0 of each block also routes the block's overflow
 // tokens to the dense channel (list, count, gathered rows).
 //
-// Neurons are processed in groups of 8.  A group's 8 W_up rows, then its 8
-// W_down rows, pass through a ring of shared-memory stages, one stage = 8
-// whole rows (8 x d bf16), each row brought by one 1-D bulk copy (8 KB at
-// d = 4096: the copy size at which one SM's bulk-copy traffic reaches the HBM
-// rate, where 2 KB pieces fall about a fifth short).  Rows are padded by 16
-// bytes so that ldmatrix is free of bank conflicts.  The warps issue the 8
-// copies of a stage in parallel, and one CTA barrier per stage releases its
-// slot, which is refilled at once with the stage nslot ahead.
+// Neurons are processed in groups of 8, and groups in pairs (A, B): the W_up
+// rows of A, then of B, then the W_down rows of A and of B pass through a
+// ring of shared-memory stages, one stage = 8 whole rows (8 x d bf16), each
+// row brought by one 1-D bulk copy (8 KB at d = 4096: the copy size at which
+// one SM's bulk-copy traffic reaches the HBM rate, where 2 KB pieces fall
+// about a fifth short).  Rows are padded by 16 bytes so that ldmatrix is free
+// of bank conflicts.  The warps issue the 8 copies of a stage in parallel;
+// one CTA barrier frees both W_up stages of a pair (whose up products share
+// the x fragments) and another both W_down stages, and each freed slot is
+// refilled at once with the stage nslot ahead.
 //
 // Both contractions are warp-level tensor-core MMAs (bf16 inputs, fp32
 // accumulate) on the staged rows:
@@ -91,7 +93,7 @@ struct RowsSmem {
     s.nid = o;   o += lcap * 4;
     s.lmask = o; o += lcap * 4;
     s.lval = o;  o += lcap * 16;
-    s.ured = o;  o += RW_WARPS * 32 * 8;
+    s.ured = o;  o += 2 * RW_WARPS * 32 * 8;  // the partials of a pair of groups
     s.misc = o;  o += 64 * 4;
     s.total = o;
     return s;
@@ -280,7 +282,11 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
   for (int c0 = r0; c0 < r1; c0 += a.lcap) {
     const int c1 = min(r1, c0 + a.lcap), Lc = c1 - c0;
     const int n_groups = (Lc + RW_G - 1) / RW_G;
-    const int n_stages = n_groups * 2;  // per group: its W_up rows, then its W_down rows
+    // groups go in pairs (A, B): stages W_up A, W_up B, W_down A, W_down B, so
+    // that one barrier frees two stages and the up products share x; a
+    // missing last B has no rows
+    const int n_pairs = (n_groups + 1) >> 1;
+    const int n_stages = n_pairs * 4;
     // a. tiles overlapping [c0, c1): pa holds rank c0, pb holds rank c1 - 1
     for (int p = tid; p < P; p += blockDim.x) {
       if (tpre[p] <= c0 && c0 < tpre[p + 1]) misc[48] = p;
@@ -303,17 +309,18 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       lval[e] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    // c. stage q of this chunk (group q / 2; W_up rows if q is even): warp w
-    // (lane 0) copies row w; padding rows of W_down stages copy zeros, of W_up
-    // stages nothing (their u is never used)
+    // c. stage q of this chunk (group 2 (q / 4) + q % 2; W_up rows if q % 4 < 2):
+    // warp w (lane 0) copies row w; padding rows of W_down stages copy zeros,
+    // of W_up stages nothing (their u is never used); an absent group copies
+    // nothing at all
     auto issue_stage = [&](int q) {
       if (q >= n_stages || lane != 0 || warp >= RW_G) return;
       const int gs = sbase + q, slot = gs % ns;
-      const int g = q >> 1;
-      const bool up = (q & 1) == 0;
+      const int g = 2 * (q >> 2) + (q & 1);
+      const bool up = (q & 2) == 0;
       const uint32_t bytes = (uint32_t)d * 2u;
-      const int n0 = g * RW_G, nn = min(RW_G, Lc - n0);
-      const int nrows = up ? nn : RW_G;
+      const int n0 = g * RW_G, nn = max(0, min(RW_G, Lc - n0));
+      const int nrows = up || nn == 0 ? nn : RW_G;
       if (warp == 0) mbar_expect_tx(&full[slot], bytes * (uint32_t)nrows);
       if (warp < nrows) {
         const __nv_bfloat16* src = warp < nn ? (up ? a.W_up : a.W_down) + (size_t)nid[n0 + warp] * d : a.zero_row;
@@ -348,88 +355,105 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     __syncthreads();
     if (sbase == 0) mbar_wait(xbar, 0, abort_flag, a.status);  // the x rows have landed
 
-    // e. consume the stages in order; one barrier per stage releases its slot.
+    // e. consume the stages in order, a pair of groups at a time; one barrier
+    // frees both W_up stages, another both W_down stages.
     // ldmatrix lanes: 0-7 rows 0-7 at column c, 8-15 rows 0-7 at column c + 8,
     // 16-31 the same for the warp's next k step (or output tile)
     const uint32_t lrow = (uint32_t)((lane & 7) * RS + 16 * ((lane >> 3) & 1) + 32 * warp);
     const uint32_t xsl = smem_u32(sm + L.xs) + lrow;
     const uint32_t hi_off = (lane >> 4) ? 32u * RW_WARPS : 0u;  // lanes 16-31: the next k step / tile
-    for (int g = 0; g < n_groups; ++g) {
-      const int n0 = g * RW_G, nn = min(RW_G, Lc - n0);
-      uint32_t bh = 0u, bl = 0u;  // h of the group as the down product's B fragment (hi, lo)
+    auto stage_wait = [&](int q) {
+      const int gs = sbase + q;
+      return mbar_wait(&full[gs % ns], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
+    };
+    auto stage_addr = [&](int q) { return ring_s + (uint32_t)(((sbase + q) % ns) * SB) + lrow; };
+    // h of one group as the down product's B fragment (hi, lo), from the 16
+    // warps' partials at this lane's fragment position (token lane/4, neurons
+    // 2(lane%4) and +1)
+    auto group_h = [&](const float2* ub, int n0, int nn, uint32_t& bh, uint32_t& bl) {
+      const int tn = lane >> 2, r0 = 2 * (lane & 3);
+      float u0 = 0.f, u1 = 0.f;
 #pragma unroll
-      for (int ud = 0; ud < 2; ++ud) {
-        const int q = 2 * g + ud;
-        const int gs = sbase + q, slot = gs % ns;
-        const bool ok = mbar_wait(&full[slot], (uint32_t)((gs / ns) & 1), abort_flag, a.status);
-        const uint32_t sbs = ring_s + (uint32_t)(slot * SB) + lrow;
-        if (ud == 0) {
-          // up: u^T[token][neuron] partial over this warp's k steps
-          float cu[4] = {0.f, 0.f, 0.f, 0.f};
-          if (ok) {
+      for (int w = 0; w < RW_WARPS; ++w) {
+        const float2 v = ub[w * 32 + lane];
+        u0 += v.x;
+        u1 += v.y;
+      }
+      float hv[2];
 #pragma unroll
-            for (int j = 0; j < RW_MAXJ; j += 2) {
-              if (j < nj) {
-                const uint32_t off = 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u);
-                uint32_t x0, x1, x2, x3, b0, b1, b2, b3;
-                ldsm_x4(xsl + off, x0, x1, x2, x3);
-                ldsm_x4(sbs + off, b0, b1, b2, b3);
-                mma_bf16_16816(cu, x0, 0u, x1, 0u, b0, b1);
-                if (j + 1 < nj) mma_bf16_16816(cu, x2, 0u, x3, 0u, b2, b3);
-              }
-            }
+      for (int e = 0; e < 2; ++e) {
+        const int r = r0 + e, n = n0 + r;
+        float h = 0.f;
+        if (r < nn && ((lmask[n] >> tn) & 1u)) {
+          const float v = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(&lval[n])[tn] << 16);
+          h = v * (e ? u1 : u0);
+        }
+        hv[e] = h;
+      }
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(hv[0]), h1 = __float2bfloat16_rn(hv[1]);
+      bh = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      bl = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[0] - __bfloat162float(h0))) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[1] - __bfloat162float(h1))) << 16);
+    };
+    // y^T[d][token] += W_down rows^T · h over a group's 8 neurons
+    auto down_group = [&](uint32_t sbs, uint32_t bh, uint32_t bl) {
+#pragma unroll
+      for (int j = 0; j < RW_MAXJ; j += 2) {
+        if (j < nj) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(sbs + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), a0, a1, a2, a3);
+          mma_bf16_1688(acc[j], a0, a1, bh);
+          mma_bf16_1688(acc[j], a0, a1, bl);
+          if (j + 1 < nj) {
+            mma_bf16_1688(acc[j + 1], a2, a3, bh);
+            mma_bf16_1688(acc[j + 1], a2, a3, bl);
           }
-          ured[warp * 32 + lane] = make_float2(cu[0], cu[1]);
-          __syncthreads();
-          issue_stage(q + ns);  // the W_up slot is free
-          if (q + ns < n_stages) issued_end = sbase + q + ns + 1;
-          // h for (token lane/4, neurons 2(lane%4) and +1): the sum of the 16
-          // warps' partials at this lane's own fragment position
-          const int tn = lane >> 2, r0 = 2 * (lane & 3);
-          float u0 = 0.f, u1 = 0.f;
-#pragma unroll
-          for (int w = 0; w < RW_WARPS; ++w) {
-            const float2 v = ured[w * 32 + lane];
-            u0 += v.x;
-            u1 += v.y;
-          }
-          float hv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int r = r0 + e, n = n0 + r;
-            float h = 0.f;
-            if (r < nn && ((lmask[n] >> tn) & 1u)) {
-              const float v = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(&lval[n])[tn] << 16);
-              h = v * (e ? u1 : u0);
-            }
-            hv[e] = h;
-          }
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(hv[0]), h1 = __float2bfloat16_rn(hv[1]);
-          bh = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-          bl = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[0] - __bfloat162float(h0))) |
-               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[1] - __bfloat162float(h1))) << 16);
-        } else {
-          // down: y^T[d][token] += W_down rows^T · h over the 8 neurons
-          if (ok) {
-#pragma unroll
-            for (int j = 0; j < RW_MAXJ; j += 2) {
-              if (j < nj) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(sbs + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), a0, a1, a2, a3);
-                mma_bf16_1688(acc[j], a0, a1, bh);
-                mma_bf16_1688(acc[j], a0, a1, bl);
-                if (j + 1 < nj) {
-                  mma_bf16_1688(acc[j + 1], a2, a3, bh);
-                  mma_bf16_1688(acc[j + 1], a2, a3, bl);
-                }
-              }
-            }
-          }
-          __syncthreads();
-          issue_stage(q + ns);  // the W_down slot is free
-          if (q + ns < n_stages) issued_end = sbase + q + ns + 1;
         }
       }
+    };
+    for (int pr = 0; pr < n_pairs; ++pr) {
+      const int q0 = 4 * pr;
+      const int nA = RW_G * 2 * pr, nB = nA + RW_G;
+      const int nnA = min(RW_G, Lc - nA), nnB = max(0, min(RW_G, Lc - nB));
+      // up: u^T[token][neuron] partials of both groups over this warp's k steps
+      const bool okA = stage_wait(q0);
+      const bool okB = stage_wait(q0 + 1);
+      float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (okA && okB) {
+        const uint32_t sa = stage_addr(q0), sb = stage_addr(q0 + 1);
+#pragma unroll
+        for (int j = 0; j < RW_MAXJ; j += 2) {
+          if (j < nj) {
+            const uint32_t off = 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u);
+            uint32_t x0, x1, x2, x3, b0, b1, b2, b3;
+            ldsm_x4(xsl + off, x0, x1, x2, x3);
+            ldsm_x4(sa + off, b0, b1, b2, b3);
+            mma_bf16_16816(ca, x0, 0u, x1, 0u, b0, b1);
+            if (j + 1 < nj) mma_bf16_16816(ca, x2, 0u, x3, 0u, b2, b3);
+            if (nnB > 0) {
+              ldsm_x4(sb + off, b0, b1, b2, b3);
+              mma_bf16_16816(cb, x0, 0u, x1, 0u, b0, b1);
+              if (j + 1 < nj) mma_bf16_16816(cb, x2, 0u, x3, 0u, b2, b3);
+            }
+          }
+        }
+      }
+      ured[warp * 32 + lane] = make_float2(ca[0], ca[1]);
+      ured[RW_WARPS * 32 + warp * 32 + lane] = make_float2(cb[0], cb[1]);
+      __syncthreads();
+      issue_stage(q0 + ns);  // both W_up slots are free
+      issue_stage(q0 + 1 + ns);
+      if (q0 + ns < n_stages) issued_end = sbase + min(n_stages, q0 + 2 + ns);
+      uint32_t bhA, blA, bhB = 0u, blB = 0u;
+      group_h(ured, nA, nnA, bhA, blA);
+      if (nnB > 0) group_h(ured + RW_WARPS * 32, nB, nnB, bhB, blB);
+      // down: both groups into the partial y
+      if (stage_wait(q0 + 2)) down_group(stage_addr(q0 + 2), bhA, blA);
+      if (stage_wait(q0 + 3) && nnB > 0) down_group(stage_addr(q0 + 3), bhB, blB);
+      __syncthreads();
+      issue_stage(q0 + 2 + ns);  // both W_down slots are free
+      issue_stage(q0 + 3 + ns);
+      if (q0 + 2 + ns < n_stages) issued_end = sbase + min(n_stages, q0 + 4 + ns);
     }
     sbase += n_stages;
     __syncthreads();
