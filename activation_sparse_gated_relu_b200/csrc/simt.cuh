@@ -282,9 +282,12 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
 
 // ---------------------------------------------------------------- fp32 path
 // The fp32 configuration has no full-precision tensor-core MMA, so its gate
-// is a SIMT tile: 128 threads = the 128 neurons of one tile, 16 tokens, the
-// tokens' x staged in shared memory 256 columns at a time.  The same TwELL
-// (or WINA score) emission as the tensor-core epilogue follows.
+// is a SIMT tile: 128 threads = the 128 neurons of one tile, 16 tokens.  K
+// goes in chunks of 64: the tile's 128 W_gate row pieces and the tokens' x
+// pieces are staged in shared memory by coalesced loads (rows padded to 65
+// floats, so that each thread reads its own row bank-conflict free), then
+// every thread accumulates its neuron's 16 dot products.  The same TwELL (or
+// WINA score) emission as the tensor-core epilogue follows.
 struct GateF32Args {
   const float* x;       // [T][d]
   const float* W_gate;  // [F][d]
@@ -294,28 +297,70 @@ struct GateF32Args {
   WinaParams wp;
 };
 
+constexpr int GF_K = 64;
+
 __global__ void __launch_bounds__(128) k_gate_f32(const GateF32Args a) {
-  __shared__ __align__(16) float xs[16][256];
+  __shared__ float ws[128][GF_K + 1];
+  __shared__ __align__(16) float xs[16][GF_K];
   __shared__ uint32_t masks[2][64];
   griddep_wait();
   const int p = blockIdx.x, t0 = blockIdx.y * 16;
   const int etid = threadIdx.x, j = p * 128 + etid;
   const int T = a.wina ? a.wp.T : a.tw.T;
+  const int d = a.d;
   float g[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) g[i] = 0.f;
-  const float* wrow = a.W_gate + (size_t)j * a.d;
-  for (int k0 = 0; k0 < a.d; k0 += 256) {
-    const int kn = min(256, a.d - k0);
+  const float* wtile = a.W_gate + (size_t)p * 128 * d;
+  for (int k0 = 0; k0 < d; k0 += GF_K) {
+    const int kn = min(GF_K, d - k0);
     __syncthreads();
-    for (int e = etid; e < 16 * 256; e += 128) {
-      const int i = e >> 8, kk = e & 255;
-      const int t = t0 + i;
-      xs[i][kk] = (t < T && kk < kn) ? a.x[(size_t)t * a.d + k0 + kk] : 0.f;
+    // all of a thread's loads go out before its first store (64 W and 8 x
+    // values per thread per chunk): one memory latency per chunk, not 72
+    if ((d & 3) == 0) {
+      float4 wv[16], xv[2];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int e = etid + 128 * q, r = e >> 4, c = 4 * (e & 15);
+        wv[q] = c < kn ? __ldg(reinterpret_cast<const float4*>(wtile + (size_t)r * d + k0 + c))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int e = etid + 128 * q, i = e >> 4, c = 4 * (e & 15), t = t0 + i;
+        xv[q] = (t < T && c < kn) ? __ldg(reinterpret_cast<const float4*>(a.x + (size_t)t * d + k0 + c))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int e = etid + 128 * q, r = e >> 4, c = 4 * (e & 15);
+        ws[r][c] = wv[q].x;
+        ws[r][c + 1] = wv[q].y;
+        ws[r][c + 2] = wv[q].z;
+        ws[r][c + 3] = wv[q].w;
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int e = etid + 128 * q, i = e >> 4, c = 4 * (e & 15);
+        *reinterpret_cast<float4*>(&xs[i][c]) = xv[q];
+      }
+    } else {
+#pragma unroll 8
+      for (int e = etid; e < 128 * GF_K; e += 128) {
+        const int r = e / GF_K, c = e % GF_K;
+        ws[r][c] = c < kn ? wtile[(size_t)r * d + k0 + c] : 0.f;
+      }
+#pragma unroll 8
+      for (int e = etid; e < 16 * GF_K; e += 128) {
+        const int i = e / GF_K, c = e % GF_K;
+        const int t = t0 + i;
+        xs[i][c] = (t < T && c < kn) ? a.x[(size_t)t * d + k0 + c] : 0.f;
+      }
     }
     __syncthreads();
-    for (int kk = 0; kk < kn; ++kk) {
-      const float w = wrow[k0 + kk];
+#pragma unroll 8
+    for (int kk = 0; kk < GF_K; ++kk) {
+      const float w = ws[etid][kk];
 #pragma unroll
       for (int i = 0; i < 16; ++i) g[i] = fmaf(w, xs[i][kk], g[i]);
     }
