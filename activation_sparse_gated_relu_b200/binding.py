@@ -76,6 +76,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_debug_twell.restype = st
     lib.sffn_debug_decode_waits.argtypes = [vp, ctypes.c_int, ctypes.c_uint]
     lib.sffn_debug_decode_waits.restype = st
+    lib.sffn_debug_set_epoch.argtypes = [vp, ctypes.c_uint]
+    lib.sffn_debug_set_epoch.restype = st
     lib.sffn_debug_keep.argtypes = [vp, ctypes.POINTER(vp)]
     lib.sffn_debug_keep.restype = st
     lib.sffn_debug_gate.argtypes = [vp, ctypes.POINTER(vp)]
@@ -258,6 +260,10 @@ class SparseFFN:
         """Test hook: single-launch decode forwards await `phantom_ctas` CTAs
         that never run, with waits of `wait_us` µs (0, 0 restores)."""
         _check(load_library().sffn_debug_decode_waits(self.h, phantom_ctas, wait_us), "debug_decode_waits")
+
+    def debug_set_epoch(self, epoch: int) -> None:
+        """Test hook: the next forward takes epoch `epoch` + 1 (0 skipped)."""
+        _check(load_library().sffn_debug_set_epoch(self.h, epoch), "debug_set_epoch")
 
     def keep_masks(self, T: int):
         """The last ROWS-path forward's keep masks, uint32 [T][n_tiles][4]."""

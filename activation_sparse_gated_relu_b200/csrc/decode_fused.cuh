@@ -21,9 +21,10 @@
 //      stage and a W_down stage each, with x back in the x block; u and h
 //      stay in registers, y accumulates in registers.  The first item's
 //      stages are issued while the last gate stages are still in use, so the
-//      stream does not pause between G and R.  Each list is published (its
-//      length, tagged with the forward's epoch, after a release fence), its
-//      owner takes items in small claims, and a CTA whose own list is
+//      stream does not pause between G and R.  Each list is published as
+//      soon as its gate phase ends (its length, tagged with the forward's
+//      epoch, after a release fence); its owner keeps the first half of its
+//      items and takes the rest in claims of one, and a CTA whose own list is
 //      exhausted steals half of the largest remainder of another CTA's list:
 //      the work of an SM that gated slowly, or whose range keeps more
 //      neurons, spreads over the others.
@@ -60,7 +61,6 @@ struct DecodeArgs {
   const __nv_bfloat16* W_gate;   // [F][d]
   const __nv_bfloat16* W_up;
   const __nv_bfloat16* W_down;
-  const __nv_bfloat16* zero_row; // >= d bf16 zeros
   TwellParams tw;                // T, F, n_tiles, C, bias, tau, act, TwELL outputs, keep masks, epochs
   float* gstage;                 // [n_tiles][8][128] fp32 gate values (before the bias)
   int* sched;                    // [decode_sched_ints(n_tiles, grid)] zero before the first launch
@@ -202,19 +202,25 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     bulk_g2s(slot_at(sl) + warp * RS, a.W_gate + (size_t)((g0 + q) * RW_G + warp) * d, (uint32_t)d * 2u, &full[sl]);
   };
   // rows stage kr: item kr/2's W_up rows (kr even) or W_down rows (kr odd)
-  // from item buffer b into ring slot kr % 2; absent records stream the zero row
+  // from item buffer b into ring slot kr % 2.  Absent records copy nothing:
+  // their slot rows keep stale weights, which the products mask out (a
+  // shared zero row, copied by every CTA at once, made one L2 slice a hot
+  // spot at the end of the rows phase).
   auto r_par = [&](int kr) { return (uint32_t)((g_fills(kr & 1) + (kr >> 1)) & 1); };
   auto issue_item = [&](int kr, int b) {
     if (lane != 0 || warp >= RW_G) return;
     const int sl = kr & 1;
     if (warp == 0) {
-      mbar_expect_tx(&full[sl], (uint32_t)(RW_G * d * 2));
+      int present = 0;
+#pragma unroll
+      for (int r = 0; r < RW_G; ++r) present += ib_id[b * 8 + r] != 0u;
+      mbar_expect_tx(&full[sl], (uint32_t)(present * d * 2));
       misc[DM_LK0 + sl] = (int)r_par(kr);
     }
     const uint32_t id = ib_id[b * 8 + warp];
+    if (id == 0u) return;
     const __nv_bfloat16* W = (kr & 1) ? a.W_down : a.W_up;
-    const __nv_bfloat16* src = id ? W + (size_t)(id & 0xFFFFFFu) * d : a.zero_row;
-    bulk_g2s(ring + (size_t)sl * SB + warp * RS, src, (uint32_t)d * 2u, &full[sl]);
+    bulk_g2s(ring + (size_t)sl * SB + warp * RS, W + (size_t)(id & 0xFFFFFFu) * d, (uint32_t)d * 2u, &full[sl]);
   };
   // up-style product of a staged stage: the warp's partial of
   // u^T[token lane/4][rows 2(lane%4), +1] over its k steps, x from the x block
@@ -372,14 +378,20 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   for (int j = 0; j < RW_MAXJ; ++j)
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
-  // down product of a staged stage of 8 W_down rows with h (bh, bl) into acc
-  auto down_acc = [&](uint32_t sbs, bool ok, uint32_t bh, uint32_t bl) {
+  // down product of a staged stage of 8 W_down rows with h (bh, bl) into
+  // acc; keep (per 16-bit half) clears the rows of absent records, whose
+  // slot rows hold stale data (h is zero there, and 0 * inf would not be)
+  auto down_acc = [&](uint32_t sbs, bool ok, uint32_t bh, uint32_t bl, uint32_t keep) {
     if (!ok) return;
 #pragma unroll
     for (int j = 0; j < RW_MAXJ; j += 2) {
       if (j < nj) {
         uint32_t a0, a1, a2, a3;
         ldsm_x4_t(sbs + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), a0, a1, a2, a3);
+        a0 &= keep;
+        a1 &= keep;
+        a2 &= keep;
+        a3 &= keep;
         mma_bf16_1688(acc[j], a0, a1, bh);
         mma_bf16_1688(acc[j], a0, a1, bl);
         if (j + 1 < nj) {
@@ -395,7 +407,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     misc[DM_RISS] = r_iss;
     misc[DM_CHV] = s;
     misc[DM_CHK] = 0;
-    misc[DM_CHK1] = min(items, max(2, (items + 1) >> 1));
+    misc[DM_CHK1] = min(items, max(1, (items + 1) >> 1));
     misc[DM_VCNT] = cnt;
     misc[DM_OWNMORE] = misc[DM_CHK1] < items;
   }
@@ -404,32 +416,33 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
   // ------------------------------------------------------ own list, steals
   const int cnt_own = misc[DM_CNT], r_issued = misc[DM_RISS];
   const int items_own = (cnt_own + 7) >> 3;
-  const int k_pre = min(items_own, max(2, (items_own + 1) >> 1));  // items the owner keeps outright
+  const int k_pre = min(items_own, max(1, (items_own + 1) >> 1));  // items the owner keeps outright
   const uint32_t epoch = a.tw.epoch;
   // Publication of the own list (its length, tagged with the epoch, after the
   // claim count and a release fence that also covers the records, the gate
-  // values and the zeroed slice of out).  It comes after the first item's
-  // stages are under way, or before the first claim or steal.
-  bool published = false;   // uniform
+  // values and the zeroed slice of out), right away: a CTA that gated late
+  // is the one whose remainder the others wait for.  Measured against
+  // publishing once the first item's stages were under way: 1 us less per
+  // forward at 1, 4 and 8 tokens.
   bool all_seen = false;    // uniform: a steal scan found every list published
-  auto publish = [&]() {
-    if (tid == 0) {
-      sc[S.claim(s)] = k_pre;
-      fence_acq_rel_gpu();
-      atomicExch(sc + S.pub(s), (int)(((epoch & 0xFFFFu) << 16) | (uint32_t)(cnt_own + 1)));
-    }
-    published = true;
-  };
+  if (tid == 0) {
+    sc[S.claim(s)] = k_pre;
+    fence_acq_rel_gpu();
+    atomicExch(sc + S.pub(s), (int)(((epoch & 0xFFFFu) << 16) | (uint32_t)(cnt_own + 1)));
+  }
 
-  // The next item into item buffer `buf` (block-wide; false when no list
-  // anywhere has work left).  The items of the current claim come first
-  // (one barrier); then own items, one per claim; then the largest published
+  // The next item into item buffer `buf` (block-wide).  Returns ACQ_GOT, or
+  // ACQ_NONE when no list anywhere has work left, or (only when `wait` is
+  // false) ACQ_LATER when nothing is stealable yet but some lists are still
+  // being gated: the caller has an item in flight and asks again, waiting,
+  // once that item is done.  The items of the current claim come first (one
+  // barrier); then own items, one per claim; then the largest published
   // remainder, half of it per steal.  Only tid 0 writes the claim state in
   // misc, between barriers.
-  auto acquire = [&](int buf) -> bool {
+  enum { ACQ_NONE = 0, ACQ_GOT = 1, ACQ_LATER = 2 };
+  auto acquire = [&](int buf, bool wait) -> int {
     if (misc[DM_CHK] >= misc[DM_CHK1]) {
-      if (__syncthreads_or(*abort_flag)) return false;
-      if (!published) publish();
+      if (__syncthreads_or(*abort_flag)) return ACQ_NONE;
       if (tid == 0) {
         int got = 0;
         if (misc[DM_OWNMORE]) {
@@ -471,7 +484,7 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
           if (tid == 0) {
             int best = -1;
             for (int w = 0; w < RW_WARPS; ++w) best = max(best, misc[DM_RED + w]);
-            int res = 0;  // 0: look again, 1: claimed, 2: no work left (3: and every list seen)
+            int res = 0;  // 0: look again, 1: claimed, 2: no work left (3: and every list seen), 4: later
             if (best >= 0) {
               const int v = best & 511, vc = vcs[v], it = (vc + 7) >> 3;
               const int m = max(1, (best >> 9) >> 1);
@@ -484,7 +497,9 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
                 res = 1;
               }
             } else if (n_unpub > 0) {  // lists still being gated: wait for them, bounded
-              if (globaltimer() - t0 > a.wait_ns) {
+              if (!wait) {
+                res = 4;
+              } else if (globaltimer() - t0 > a.wait_ns) {
                 atomicOr(a.status, DEV_ERR_TIMEOUT);
                 *abort_flag = 1;
                 res = 2;
@@ -499,9 +514,11 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
           __syncthreads();
           if (misc[DM_RES] != 0) break;
         }
-        if (misc[DM_RES] >= 2) {
-          all_seen = misc[DM_RES] == 3;
-          return false;
+        const int res = misc[DM_RES];
+        if (res == 4) return ACQ_LATER;
+        if (res >= 2) {
+          all_seen = res == 3;
+          return ACQ_NONE;
         }
       }
     }
@@ -524,21 +541,22 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
     }
     __syncthreads();  // the item buffer is complete; every thread has read the claim state
     if (tid == 0) misc[DM_CHK] = k + 1;  // read again only after the loop's next barrier
-    return true;
+    return ACQ_GOT;
   };
 
   // ------------------------------------------------------------ R: rows
   // rows stage 2i is item i's W_up stage, 2i + 1 its W_down stage
-  const bool have_first = acquire(0);
+  const bool have_first = acquire(0, true) == ACQ_GOT;
   if (have_first)
     for (int r = r_issued; r < 2; ++r) issue_item(r, 0);  // those G did not issue
   if (x_slot) mbar_wait(xbar, 1, abort_flag, a.status);  // the second copy of x
   if (have_first) {
     int kr = 0, cur = 0;
     __syncthreads();  // the claim state acquire(0) left
-    bool have_next = acquire(1);
+    int nx = acquire(1, false);
     for (;;) {
-      uint32_t bh, bl;
+      const bool have_next = nx == ACQ_GOT;
+      uint32_t bh, bl, keep;
       {  // W_up stage: u of the item's rows, then h = v·u where the token keeps the row
         const int sl = kr & 1;
         const bool ok = mbar_wait(&full[sl], r_par(kr), abort_flag, a.status);
@@ -556,9 +574,11 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
         }
         const int tn = lane >> 2, rr = 2 * (lane & 3);
         float hv[2];
+        keep = 0u;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const uint32_t id = ib_id[cur * 8 + rr + e];
+          if (id != 0u) keep |= 0xFFFFu << (16 * e);
           float h = 0.f;
           if ((id >> (24 + tn)) & 1u) {
             const float v = __uint_as_float(
@@ -572,15 +592,21 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_decode(const DecodeArgs a) {
       {  // W_down stage: y += h·W_down
         const int k = kr + 1, sl = k & 1;
         const bool ok = mbar_wait(&full[sl], r_par(k), abort_flag, a.status);
-        down_acc(ring_s + (uint32_t)(sl * SB) + lrow, ok, bh, bl);
+        down_acc(ring_s + (uint32_t)(sl * SB) + lrow, ok, bh, bl, keep);
         __syncthreads();
         if (have_next) issue_item(kr + 3, cur ^ 1);
-        if (!published) publish();  // while the next item's stages are in flight
       }
       kr += 2;
-      if (!have_next) break;
+      if (nx == ACQ_LATER) {  // nothing in flight now: wait for a list, then issue its stages
+        nx = acquire(cur ^ 1, true);
+        if (nx == ACQ_GOT) {
+          issue_item(kr, cur ^ 1);
+          issue_item(kr + 1, cur ^ 1);
+        }
+      }
+      if (nx != ACQ_GOT) break;
       cur ^= 1;
-      have_next = acquire(cur ^ 1);
+      nx = acquire(cur ^ 1, false);
     }
   }
   // This CTA streams no more weights: the next forward's launch may begin

@@ -55,7 +55,6 @@ struct RowsArgs {
   const __nv_bfloat16* x;
   const __nv_bfloat16* W_up;
   const __nv_bfloat16* W_down;
-  const __nv_bfloat16* zero_row;   // >= 2 KB of zeros (rows of padding neurons)
   const int16_t* count;
   const int16_t* idx;
   const __nv_bfloat16* val;
@@ -310,9 +309,8 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
     }
     __syncthreads();
     // c. stage q of this chunk (group 2 (q / 4) + q % 2; W_up rows if q % 4 < 2):
-    // warp w (lane 0) copies row w; padding rows of W_down stages copy zeros,
-    // of W_up stages nothing (their u is never used); an absent group copies
-    // nothing at all
+    // warp w (lane 0) copies row w; padding rows copy nothing (their u is
+    // never used, and the down product masks their stale rows out)
     auto issue_stage = [&](int q) {
       if (q >= n_stages || lane != 0 || warp >= RW_G) return;
       const int gs = sbase + q, slot = gs % ns;
@@ -320,12 +318,10 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       const bool up = (q & 2) == 0;
       const uint32_t bytes = (uint32_t)d * 2u;
       const int n0 = g * RW_G, nn = max(0, min(RW_G, Lc - n0));
-      const int nrows = up || nn == 0 ? nn : RW_G;
-      if (warp == 0) mbar_expect_tx(&full[slot], bytes * (uint32_t)nrows);
-      if (warp < nrows) {
-        const __nv_bfloat16* src = warp < nn ? (up ? a.W_up : a.W_down) + (size_t)nid[n0 + warp] * d : a.zero_row;
-        bulk_g2s(ring + (size_t)slot * SB + warp * RS, src, bytes, &full[slot]);
-      }
+      if (warp == 0) mbar_expect_tx(&full[slot], bytes * (uint32_t)nn);
+      if (warp < nn)
+        bulk_g2s(ring + (size_t)slot * SB + warp * RS, (up ? a.W_up : a.W_down) + (size_t)nid[n0 + warp] * d, bytes,
+                 &full[slot]);
     };
     for (int q = 0; q < ns; ++q) issue_stage(q);
     issued_end = sbase + min(ns, n_stages);
@@ -395,13 +391,22 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       bl = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[0] - __bfloat162float(h0))) |
            ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hv[1] - __bfloat162float(h1))) << 16);
     };
-    // y^T[d][token] += W_down rows^T · h over a group's 8 neurons
-    auto down_group = [&](uint32_t sbs, uint32_t bh, uint32_t bl) {
+    // y^T[d][token] += W_down rows^T · h over a group's nn neurons: this
+    // lane's A fragments hold rows 2(lane%4) and +1, and the rows of padding
+    // neurons (stale slot data; h is zero there, and 0 * inf would not be)
+    // are cleared
+    auto down_group = [&](uint32_t sbs, uint32_t bh, uint32_t bl, int nn) {
+      const int r0 = 2 * (lane & 3);
+      const uint32_t keep = (r0 < nn ? 0xFFFFu : 0u) | (r0 + 1 < nn ? 0xFFFF0000u : 0u);
 #pragma unroll
       for (int j = 0; j < RW_MAXJ; j += 2) {
         if (j < nj) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(sbs + 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u), a0, a1, a2, a3);
+          a0 &= keep;
+          a1 &= keep;
+          a2 &= keep;
+          a3 &= keep;
           mma_bf16_1688(acc[j], a0, a1, bh);
           mma_bf16_1688(acc[j], a0, a1, bl);
           if (j + 1 < nj) {
@@ -448,8 +453,8 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       group_h(ured, nA, nnA, bhA, blA);
       if (nnB > 0) group_h(ured + RW_WARPS * 32, nB, nnB, bhB, blB);
       // down: both groups into the partial y
-      if (stage_wait(q0 + 2)) down_group(stage_addr(q0 + 2), bhA, blA);
-      if (stage_wait(q0 + 3) && nnB > 0) down_group(stage_addr(q0 + 3), bhB, blB);
+      if (stage_wait(q0 + 2)) down_group(stage_addr(q0 + 2), bhA, blA, nnA);
+      if (stage_wait(q0 + 3) && nnB > 0) down_group(stage_addr(q0 + 3), bhB, blB, nnB);
       __syncthreads();
       issue_stage(q0 + 2 + ns);  // both W_down slots are free
       issue_stage(q0 + 3 + ns);

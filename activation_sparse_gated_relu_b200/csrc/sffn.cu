@@ -221,7 +221,6 @@ struct sffn_handle {
   int last_T = 0, last_path = 0, last_launches = 0;
   int rows_nslot = 0, rows_lcap = 0, rows_smem = 0;
   bool rows_ok = false;                // the fused row kernel supports this shape
-  __nv_bfloat16* zero_row = nullptr;   // a row of zeros (>= 2 KB): W_down rows of padding neurons
   int gate_stages = 0, down_stages = 0;  // ring depth of the gate and down tile kernels (0: all)
   // row-streaming gate for up to 8 tokens: tile staging, tickets, ring slots, shared memory
   float* gstage = nullptr;
@@ -257,7 +256,7 @@ void free_handle(sffn_handle* h) {
   void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
                   h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zpart,
                   h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->zero_row, h->gstage, h->gtick, h->dsched, h->wl_id, h->wl_val};
+                  h->gstage, h->gtick, h->dsched, h->wl_id, h->wl_val};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   delete h;
@@ -409,7 +408,6 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     ok = ok && dalloc(&h->h_hi, T * F * 2);
     ok = ok && dalloc(&h->h_lo, T * F * 2);
     ok = ok && dalloc(&h->WdT, d * F * 2);
-    ok = ok && dalloc(&h->zero_row, std::max<size_t>(2048, d * 2));
   }
   if (h->wina) {
     ok = ok && dalloc(&h->scores, T * F * 4);
@@ -438,7 +436,6 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
   e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
-  if (h->zero_row) e = e ? e : cudaMemsetAsync(h->zero_row, 0, std::max<size_t>(2048, d * 2), st);
   if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
   if (h->lowrank) {
     e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * 4, st);
@@ -620,7 +617,6 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     da.W_gate = static_cast<const __nv_bfloat16*>(D.W_gate);
     da.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
     da.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
-    da.zero_row = h->zero_row;
     da.tw = tw;
     da.gstage = h->gstage;
     da.sched = h->dsched;
@@ -718,7 +714,6 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     rw.x = static_cast<const __nv_bfloat16*>(x);
     rw.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
     rw.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
-    rw.zero_row = h->zero_row;
     rw.count = h->count;
     rw.idx = h->idx;
     rw.val = static_cast<const __nv_bfloat16*>(h->val);
@@ -895,6 +890,12 @@ sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void*
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   ++h->epoch;
   if (h->epoch == 0) ++h->epoch;  // 0 marks "never overflowed"
+  // the single-launch schedule's words carry the low 16 bits of the epoch:
+  // cleared at the start of every window of 65536 epochs, no word left by an
+  // earlier launch carries the current tag
+  if (h->dsched && ((h->epoch & 0xFFFFu) == 0u || h->epoch == 1u)) {
+    if (cudaMemsetAsync(h->dsched, 0, (size_t)h->dsched_ints * 4, st) != cudaSuccess) return SFFN_ERR_CUDA;
+  }
   h->last_T = T;
   h->last_epoch = h->epoch;
   h->last_fused = false;
@@ -1010,6 +1011,14 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
   if (overflow) *overflow = h->ovf;
   if (n_tiles) *n_tiles = h->P;
   if (tile_capacity) *tile_capacity = h->C;
+  return SFFN_OK;
+}
+
+sffn_status sffn_debug_set_epoch(sffn_handle* h, unsigned epoch) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (h->dsched && cudaMemset(h->dsched, 0, (size_t)h->dsched_ints * 4) != cudaSuccess) return SFFN_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SFFN_ERR_CUDA;
+  h->epoch = epoch;
   return SFFN_OK;
 }
 

@@ -167,6 +167,14 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
  * Errors: SFFN_ERR_INVALID_ARG for a null handle or phantom_ctas not 0 or 1. */
 sffn_status sffn_debug_decode_waits(sffn_handle* h, int phantom_ctas, unsigned wait_us);
 
+/* Test hook: the next forward takes epoch `epoch` + 1 (0 is skipped).  The
+ * single-launch decode forward's scheduler words carry the low 16 bits of the
+ * epoch and are cleared here (synchronously) and at the start of every
+ * window of 65536 epochs, so tests can cross those windows and the 32-bit
+ * wrap.  Errors: SFFN_ERR_INVALID_ARG for a null handle; SFFN_ERR_CUDA if the
+ * clear fails. */
+sffn_status sffn_debug_set_epoch(sffn_handle* h, unsigned epoch);
+
 /* Device view of the last forward's keep masks: uint32 [T][n_tiles][4], bit
  * (32 w + b) of word w set iff the token keeps neuron 128 p + 32 w + b of tile
  * p, with no capacity limit (an overflow token's full kept set).  Written by

@@ -285,6 +285,25 @@ def test_decode_single_launch_repeated_mixed_T(decode_inputs):
         ffn.close()
 
 
+def test_decode_single_launch_across_epoch_windows(decode_inputs):
+    # the scheduler words carry the low 16 bits of the epoch; forwards that
+    # cross a window of 65536 epochs, and the 32-bit wrap (which skips 0),
+    # still see only their own lists
+    ffn = make_ffn(decode_inputs, max_tokens=8)
+    res = {T: oracle.forward_inputs(decode_inputs, T=T) for T in (8, 3)}
+    try:
+        for start, epochs in ((0xFFFD, (0xFFFE, 0xFFFF, 0x10000, 0x10001)),
+                              (0x2FFFE, (0x2FFFF, 0x30000, 0x30001, 0x30002)),
+                              (0xFFFFFFFD, (0xFFFFFFFE, 0xFFFFFFFF, 1, 2))):
+            ffn.debug_set_epoch(start)
+            for T, ep in zip((8, 3, 8, 8), epochs):
+                st = check(decode_inputs, T=T, ffn=ffn, res=res[T])
+                assert st["launches"] == 1
+                assert ffn.stats().epoch == ep
+    finally:
+        ffn.close()
+
+
 def test_lopa_config():
     inp = synth.make_inputs(W["lopa_bf16"])
     st = check(inp)
