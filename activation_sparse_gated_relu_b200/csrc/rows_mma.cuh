@@ -420,31 +420,39 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_rows(const RowsArgs a) {
       const int q0 = 4 * pr;
       const int nA = RW_G * 2 * pr, nB = nA + RW_G;
       const int nnA = min(RW_G, Lc - nA), nnB = max(0, min(RW_G, Lc - nB));
-      // up: u^T[token][neuron] partials of both groups over this warp's k steps
+      // up: u[neuron][token] partials of both groups over this warp's k
+      // steps, the pair's 16 rows as the MMA's M (group A rows 0-7, group B
+      // rows 8-15) and the 8 tokens as its N: no half-empty tiles.  Rows of
+      // padding neurons (and all of B's when the pair has one group) hold
+      // stale data; each D row depends on its own A row only, and group_h
+      // reads none of them.
       const bool okA = stage_wait(q0);
       const bool okB = stage_wait(q0 + 1);
-      float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+      float cu[4] = {0.f, 0.f, 0.f, 0.f};
       if (okA && okB) {
         const uint32_t sa = stage_addr(q0), sb = stage_addr(q0 + 1);
 #pragma unroll
         for (int j = 0; j < RW_MAXJ; j += 2) {
           if (j < nj) {
             const uint32_t off = 32u * RW_WARPS * j + (j + 1 < nj ? hi_off : 0u);
-            uint32_t x0, x1, x2, x3, b0, b1, b2, b3;
+            uint32_t x0, x1, x2, x3, a0, a1, a2, a3, b0, b1, b2, b3;
             ldsm_x4(xsl + off, x0, x1, x2, x3);
-            ldsm_x4(sa + off, b0, b1, b2, b3);
-            mma_bf16_16816(ca, x0, 0u, x1, 0u, b0, b1);
-            if (j + 1 < nj) mma_bf16_16816(ca, x2, 0u, x3, 0u, b2, b3);
-            if (nnB > 0) {
-              ldsm_x4(sb + off, b0, b1, b2, b3);
-              mma_bf16_16816(cb, x0, 0u, x1, 0u, b0, b1);
-              if (j + 1 < nj) mma_bf16_16816(cb, x2, 0u, x3, 0u, b2, b3);
-            }
+            ldsm_x4(sa + off, a0, a1, a2, a3);
+            ldsm_x4(sb + off, b0, b1, b2, b3);
+            mma_bf16_16816(cu, a0, b0, a1, b1, x0, x1);
+            if (j + 1 < nj) mma_bf16_16816(cu, a2, b2, a3, b3, x2, x3);
           }
         }
       }
-      ured[warp * 32 + lane] = make_float2(ca[0], ca[1]);
-      ured[RW_WARPS * 32 + warp * 32 + lane] = make_float2(cb[0], cb[1]);
+      {  // into ured as [group][warp][token][neuron]: group_h's float2 at
+         // (warp, lane) is its token's two neurons 2 (lane % 4) and + 1
+        float* uf = reinterpret_cast<float*>(ured);
+        const int n = lane >> 2, t = 2 * (lane & 3);
+        uf[(warp * 8 + t) * 8 + n] = cu[0];
+        uf[(warp * 8 + t + 1) * 8 + n] = cu[1];
+        uf[RW_WARPS * 64 + (warp * 8 + t) * 8 + n] = cu[2];
+        uf[RW_WARPS * 64 + (warp * 8 + t + 1) * 8 + n] = cu[3];
+      }
       __syncthreads();
       issue_stage(q0 + ns);  // both W_up slots are free
       issue_stage(q0 + 1 + ns);
