@@ -588,11 +588,11 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   int rows_split = rows ? std::max(1, h->n_sm / nblk) : 1;
   // down projection split over d_ff so that its grid covers the SMs.  On the
   // ROWS path it takes the overflow rows only, whose count is on the device:
-  // the split assumes up to four token tiles of them (every token tile of the
-  // grid still launches, and the empty ones cost a wave each; at 4096 tokens
-  // with ~10 % overflow a split of 2 measured 64.7 us against 96.2 us for 9)
+  // the split assumes two token tiles of them (at 4096 tokens with ~10 %
+  // overflow, two tiles of 256, a split of 4 measured 64.7 us, 2 84.3 us and
+  // 9 96.2 us)
   const int m_tiles_down = cdiv(d, 128);
-  const int est_rows_tiles = rows ? std::min(ntile_tok, 4) : ntile_tok;
+  const int est_rows_tiles = rows ? std::min(ntile_tok, 2) : ntile_tok;
   const int kb_down = cdiv(F, 64);
   const int sk_down = std::max(1, std::min(kb_down / 4, h->n_sm / (m_tiles_down * est_rows_tiles)));
 
