@@ -15,21 +15,21 @@
 // one SM's bulk-copy traffic reaches the HBM rate, where 2 KB pieces fall
 // about a fifth short).  Rows are padded by 16 bytes so that ldmatrix is free
 // of bank conflicts.  The warps issue the 8 copies of a stage in parallel;
-// one CTA barrier frees both W_up stages of a pair (whose up products share
-// the x fragments) and another both W_down stages, and each freed slot is
+// one CTA barrier frees both W_up stages of a pair (whose up product is one
+// MMA chain over both) and another both W_down stages, and each freed slot is
 // refilled at once with the stage nslot ahead.
 //
 // Both contractions are warp-level tensor-core MMAs (bf16 inputs, fp32
 // accumulate) on the staged rows:
-//   up:   u^T[8 tokens][8 neurons] = x · W_up rows^T (m16n8k16, tokens as M,
-//         padded to 16 with zero rows; rows as N via ldmatrix) -- warp w takes
-//         every 16th 16-wide k step, whose x fragments it keeps in registers;
-//         the 16 warps' partial sums meet in shared memory and every lane
-//         adds up the 16 partials of its own fragment position;
+//   up:   u[16 neurons][8 tokens] = W_up rows · x^T over a pair of groups
+//         (m16n8k16: the pair's 16 rows as M, the 8 tokens as N, both via
+//         ldmatrix) -- warp w takes every 16th 16-wide k step; the 16 warps'
+//         partial sums meet in shared memory, laid out so that every lane
+//         adds up the 16 partials at its position in the down product's B
+//         fragment (token lane/4, neurons 2 (lane%4) and +1);
 //   h:    h_tj = v_tj·u_tj where (t, j) is kept, else 0, split into
 //         hi = bf16(h) and lo = bf16(h - hi) (so the bf16 MMA operand loses at
-//         most 2^-16 of h); the up output fragment is exactly the B fragment
-//         of the down product, so h never leaves the registers;
+//         most 2^-16 of h), straight into the down product's B fragment;
 //   down: y^T[d][8 tokens] += W_down rows^T (ldmatrix.trans) · (h_hi + h_lo)
 //         (m16n8k8, the 8 neurons as K) -- warp w owns every 16th 16-row
 //         output tile, held in registers for the whole CTA.
