@@ -375,6 +375,7 @@ def run_ours(args) -> None:
 
     wl = synth.WORKLOADS[args.workload]
     T, _, NXB, _ = BENCH_SHAPES[args.workload]
+    T = args.tokens or T
     NS = args.weight_sets
     inp = synth.make_inputs(wl, T=T * NXB)
     dev = lambda t: None if t is None else t.to("cuda")  # noqa: E731
@@ -452,7 +453,9 @@ def run_ours(args) -> None:
     roof = None
     if dom in works and ms_dom > 0:
         roof = roofline_of(works[dom], ms_dom, peaks, peak_src)
-        roof.update({"kernel": dom, "traffic": profiled_traffic(dom, args.workload),
+        # the committed captures are of the workload's own token count
+        traffic = profiled_traffic(dom, args.workload) if T == BENCH_SHAPES[args.workload][0] else None
+        roof.update({"kernel": dom, "traffic": traffic,
                      "ms_per_launch": round(ms_dom, 5)})
         if single:
             roof.update({"ms_per_launch_events": round(per[dom], 5),
@@ -543,6 +546,7 @@ def run_reference(args) -> None:
     import synth
     wl = synth.WORKLOADS[args.workload]
     T, _, NXB, _ = BENCH_SHAPES[args.workload]
+    T = args.tokens or T
     inp = synth.make_inputs(wl, T=T * min(NXB, 4))
     _, nw, elw = oracle_timing(inp, T, 0, steps=max(1, min(args.warmup, 3)))
     per_fwd = elw / nw
@@ -574,9 +578,13 @@ def main(argv=None) -> None:
     ap.add_argument("--weight-sets", type=int, default=None,
                     help="rotating weight copies (fewer only for small profiler captures)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per forward instead of the workload's own (e.g. 1 or 4 for decode_bf16)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.tokens is not None and args.tokens < 1:
+        ap.error("--tokens must be >= 1")
     _, sets, _, steps = BENCH_SHAPES[args.workload]
     if args.steps is None:
         args.steps = steps
