@@ -129,7 +129,12 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
 /* y = FFN(x) for T tokens, asynchronously on `cuda_stream`.  x: [T][d_model]
  * device, operand dtype; out: [T][d_model] fp32 device, fully overwritten.
  * 0 <= T <= max_tokens; T == 0 returns SFFN_OK and launches nothing.  Must not
- * overlap another forward of the same handle. */
+ * overlap another forward of the same handle.  Each call takes the handle's
+ * next epoch, passed to its kernels by value: it tags the forward's overflow
+ * flags and, on the single-launch path, the scheduler words that the CTAs
+ * exchange.  A forward captured into a CUDA graph and replayed would reuse
+ * its epoch and could read a previous replay's scheduler words, so stream
+ * capture of sffn_forward is not supported. */
 sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void* cuda_stream);
 
 /* Same as sffn_forward but x and out are HOST buffers: copies x to the
