@@ -88,6 +88,9 @@ def _create(lib, d):
     (dict(rank=512), B.SFFN_ERR_INVALID_ARG),             # W_gate given with rank > 0
     (dict(mode=1, k=20000), B.SFFN_ERR_INVALID_ARG),      # k > d_ff
     (dict(mode=1, k=100, tile_capacity=32), B.SFFN_ERR_UNSUPPORTED),  # WINA needs C = 128
+    (dict(mode=1, k=-1, tile_capacity=128), B.SFFN_ERR_INVALID_ARG),  # k < 0
+    (dict(flags=1 << 7), B.SFFN_ERR_INVALID_ARG),         # an undefined flag bit
+    (dict(dtype=B.SFFN_FP32, d_ff=16384), B.SFFN_ERR_UNSUPPORTED),  # fp32 rows kernel: d_ff <= 8192
 ])
 def test_create_rejects_bad_descriptors(lib, kw, want):
     s, h = _create(lib, _desc(**kw))
@@ -102,6 +105,9 @@ def test_create_lowrank_rules(lib):
     assert _create(lib, _desc(**{**ok, "rank": 100}))[0] == B.SFFN_ERR_UNSUPPORTED
     assert _create(lib, _desc(**{**ok, "dtype": B.SFFN_FP32}))[0] == B.SFFN_ERR_UNSUPPORTED
     assert _create(lib, _desc(**{**ok, "B": None}))[0] == B.SFFN_ERR_INVALID_ARG
+    assert _create(lib, _desc(**{**ok, "rank": 4160}))[0] == B.SFFN_ERR_UNSUPPORTED
+    # the dense debug gate exists for the dense gate only
+    assert _create(lib, _desc(**{**ok, "flags": B.SFFN_FLAG_DEBUG_GATE}))[0] == B.SFFN_ERR_UNSUPPORTED
 
 
 def test_null_arguments(lib):
@@ -114,6 +120,8 @@ def test_null_arguments(lib):
     assert lib.sffn_forward_host(None, None, 1, None, None) == B.SFFN_ERR_INVALID_ARG
     assert lib.sffn_read_status(None, None) == B.SFFN_ERR_INVALID_ARG
     assert lib.sffn_get_stats(None, None, None) == B.SFFN_ERR_INVALID_ARG
+    assert lib.sffn_debug_set_epoch(None, 5) == B.SFFN_ERR_INVALID_ARG
+    assert lib.sffn_debug_decode_waits(None, 0, 0) == B.SFFN_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="a GPU is present")
