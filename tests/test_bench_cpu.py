@@ -121,3 +121,18 @@ def test_reference_arm_tiny_workload(capsys):
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["steps"] == 2 and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["config"]["tokens_per_step"] == 64
+
+
+def test_tokens_option():
+    import json
+    with pytest.raises(SystemExit):
+        bench.main(["--tokens", "0"])
+    # the reference arm takes the override like the GPU arm does
+    import io
+    import contextlib
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "tiny_fp32", "--tokens", "16", "--steps", "2",
+                    "--warmup", "3"])
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["config"]["tokens_per_step"] == 16 and "tokens=16" in line["config"]["workload"]
