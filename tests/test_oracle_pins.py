@@ -261,6 +261,22 @@ def test_wina_reductions():
     assert np.all(eq.keep.sum(axis=1) == 40)
 
 
+def test_lowrank_z_is_rounded_to_the_operand_dtype():
+    # reading 4: z = round(x·A) before z·B.  Here x·A = 1 + 2^-8, halfway
+    # between the bf16 neighbours 1 and 1 + 2^-7; round-to-nearest-even gives 1
+    # in bf16, while fp32 holds 1 + 2^-8 exactly
+    x = np.array([[1.0, 2.0 ** -8]])
+    A = np.array([[1.0], [1.0]])
+    B = np.array([[1.0, -3.0]])
+    import oracle.ffn as F  # looked up at call time, as the oracle's forward does
+    g, z = F.gate_lowrank(x, A, B, None, "bf16")
+    assert z[0, 0] == 1.0
+    assert np.array_equal(g, [[1.0, -3.0]])
+    g32, z32 = F.gate_lowrank(x, A, B, None, "fp32")
+    assert z32[0, 0] == 1.0 + 2.0 ** -8
+    assert np.array_equal(g32, [[1.0 + 2.0 ** -8, -3.0 - 3.0 * 2.0 ** -8]])
+
+
 def test_wina_norms_closed_form():
     Wd = np.zeros((128, 4)); Wd[:, 0] = 3.0; Wd[:, 1] = 4.0
     assert np.all(oracle.wina_norms(Wd) == 5.0)
@@ -301,7 +317,7 @@ def test_lognormal_nnz_recipe():
 # mutations: plant mistakes in the oracle and check that the pins catch them
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("mutation", ["no_bias", "no_value_round", "transposed_down",
-                                      "nonstrict", "silu_sign", "topk_tie_high"])
+                                      "nonstrict", "silu_sign", "topk_tie_high", "no_z_round"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     import oracle.ffn as F
     if mutation == "no_bias":
@@ -329,10 +345,16 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
                 keep[t, order[:k]] = True
             return keep
         monkeypatch.setattr(F, "keep_topk", bad_topk)
+    elif mutation == "no_z_round":
+        def no_round(x, A, B, bias, dtype):
+            z = x @ A
+            g = z @ B
+            return (g + bias[None, :] if bias is not None else g), z
+        monkeypatch.setattr(F, "gate_lowrank", no_round)
     failures = 0
     for test in (test_hand_worked_threshold, test_hand_worked_wina_relu,
                  lambda: test_bruteforce_rational(0, 128, 4, 3, 0.0),
-                 test_wina_reductions):
+                 test_wina_reductions, test_lowrank_z_is_rounded_to_the_operand_dtype):
         try:
             test()
         except AssertionError:
