@@ -261,6 +261,23 @@ def test_wina_reductions():
     assert np.all(eq.keep.sum(axis=1) == 40)
 
 
+def test_threshold_tests_the_unrounded_activation():
+    # reading 2: keep iff |sigma(g)| > tau on the unrounded activation, strict.
+    # a = 1 + 2^-10 with tau = 1: kept, although its stored bf16 value is
+    # 1.0 = tau (2^-10 is below half a bf16 ulp at 1); a = 1 exactly is not
+    F, dm = 128, 2
+    x = np.array([[1.0, 2.0 ** -10], [1.0, 0.0]])
+    Wg = np.zeros((F, dm)); Wu = np.zeros((F, dm)); Wd = np.zeros((F, dm))
+    b = np.full(F, -1.0)
+    Wg[5] = [1.0, 1.0]; b[5] = 0.0; Wu[5] = [2.0, 0.0]; Wd[5] = [1.0, 3.0]
+    res = oracle.forward(x, Wu, Wd, W_gate=Wg, bias=b, dtype="bf16", threshold=1.0, C=8)
+    assert res.keep[0, 5] and not res.keep[1, 5]
+    assert res.keep.sum() == 1 and res.v[0, 5] == 1.0
+    # h = v·u = 1·2, y = h·W_down[5] = [2, 6]; token 1 keeps nothing
+    np.testing.assert_array_equal(res.y, [[2.0, 6.0], [0.0, 0.0]])
+    assert res.count.tolist() == [[1], [0]]
+
+
 def test_lowrank_z_is_rounded_to_the_operand_dtype():
     # reading 4: z = round(x·A) before z·B.  Here x·A = 1 + 2^-8, halfway
     # between the bf16 neighbours 1 and 1 + 2^-7; round-to-nearest-even gives 1
@@ -317,7 +334,8 @@ def test_lognormal_nnz_recipe():
 # mutations: plant mistakes in the oracle and check that the pins catch them
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("mutation", ["no_bias", "no_value_round", "transposed_down",
-                                      "nonstrict", "silu_sign", "topk_tie_high", "no_z_round"])
+                                      "nonstrict", "silu_sign", "topk_tie_high", "no_z_round",
+                                      "keep_on_rounded"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     import oracle.ffn as F
     if mutation == "no_bias":
@@ -345,6 +363,8 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
                 keep[t, order[:k]] = True
             return keep
         monkeypatch.setattr(F, "keep_topk", bad_topk)
+    elif mutation == "keep_on_rounded":
+        monkeypatch.setattr(F, "keep_threshold", lambda a, tau: np.abs(F.round_bf16(a)) > tau)
     elif mutation == "no_z_round":
         def no_round(x, A, B, bias, dtype):
             z = x @ A
@@ -354,7 +374,8 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     failures = 0
     for test in (test_hand_worked_threshold, test_hand_worked_wina_relu,
                  lambda: test_bruteforce_rational(0, 128, 4, 3, 0.0),
-                 test_wina_reductions, test_lowrank_z_is_rounded_to_the_operand_dtype):
+                 test_wina_reductions, test_lowrank_z_is_rounded_to_the_operand_dtype,
+                 test_threshold_tests_the_unrounded_activation):
         try:
             test()
         except AssertionError:
