@@ -299,6 +299,16 @@ def test_wina_norms_closed_form():
     assert np.all(oracle.wina_norms(Wd) == 5.0)
 
 
+def test_wina_norms_are_fp32_rounded():
+    # reading 5: n_j is the fp64 norm rounded to fp32; ||(1, 1)|| = sqrt(2)
+    # is not an fp32 number, and its fp32 rounding is 1.41421353816986083984375
+    import oracle.ffn as F  # looked up at call time, as the oracle's forward does
+    Wd = np.zeros((128, 2)); Wd[:, :] = 1.0
+    n = F.wina_norms(Wd)
+    assert np.all(n == 1.41421353816986083984375)
+    assert n[0] != math.sqrt(2.0)
+
+
 # ----------------------------------------------------------------------------
 # closed-form sparsity of the synthetic recipes
 # ----------------------------------------------------------------------------
@@ -335,7 +345,7 @@ def test_lognormal_nnz_recipe():
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("mutation", ["no_bias", "no_value_round", "transposed_down",
                                       "nonstrict", "silu_sign", "topk_tie_high", "no_z_round",
-                                      "keep_on_rounded"])
+                                      "keep_on_rounded", "norms_unrounded"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     import oracle.ffn as F
     if mutation == "no_bias":
@@ -363,6 +373,8 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
                 keep[t, order[:k]] = True
             return keep
         monkeypatch.setattr(F, "keep_topk", bad_topk)
+    elif mutation == "norms_unrounded":
+        monkeypatch.setattr(F, "wina_norms", lambda W: np.sqrt(np.sum(W * W, axis=1)))
     elif mutation == "keep_on_rounded":
         monkeypatch.setattr(F, "keep_threshold", lambda a, tau: np.abs(F.round_bf16(a)) > tau)
     elif mutation == "no_z_round":
@@ -375,7 +387,7 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     for test in (test_hand_worked_threshold, test_hand_worked_wina_relu,
                  lambda: test_bruteforce_rational(0, 128, 4, 3, 0.0),
                  test_wina_reductions, test_lowrank_z_is_rounded_to_the_operand_dtype,
-                 test_threshold_tests_the_unrounded_activation):
+                 test_threshold_tests_the_unrounded_activation, test_wina_norms_are_fp32_rounded):
         try:
             test()
         except AssertionError:
