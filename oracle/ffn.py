@@ -333,22 +333,3 @@ def forward_inputs(inp, T: Optional[int] = None) -> OracleResult:
                    A=f64(inp.A), B=f64(inp.B), bias=f64(inp.bias), dtype=wl.dtype,
                    mode=wl.mode, act=wl.act, threshold=wl.threshold, k=wl.k,
                    C=wl.tile_capacity)
-
-
-# ----------------------------------------------------------------------------
-# what the method must move (the byte model of the roofline)
-# ----------------------------------------------------------------------------
-def algorithmic_bytes(res: OracleResult, d: int, F: int, rank: int, esize: int,
-                      wina: bool = False) -> dict:
-    """Bytes a forward must move: the gate weights in full, each W_up and W_down
-    row that some token keeps (once), x, out (fp32), the TwELL write and read,
-    and the WINA norms.  Dense work the method avoids, L2 re-reads and scratch
-    are not counted."""
-    T = res.keep.shape[0]
-    union = int(res.keep.any(axis=0).sum())
-    gate = (F * d if rank == 0 else d * rank + rank * F) * esize
-    rows = union * 2 * d * esize
-    P, C = res.idx.shape[1], res.idx.shape[2]
-    twell = T * P * (2 + C * (2 + esize))
-    total = gate + rows + T * d * esize + T * d * 4 + 2 * twell + (F * 4 if wina else 0)
-    return {"union": union, "gate": gate, "rows": rows, "twell": twell, "total": total}

@@ -261,6 +261,34 @@ def test_wina_reductions():
     assert np.all(eq.keep.sum(axis=1) == 40)
 
 
+def _ulp_close(got: float, want: Fraction, n_ulp: int) -> bool:
+    """|got - want| <= n_ulp fp64 ulps of want, compared in exact rationals."""
+    if want == 0:
+        return got == 0.0
+    ulp = Fraction(math.ulp(float(want)))
+    return abs(Fraction(got) - want) <= n_ulp * ulp
+
+
+def test_silu_hand_worked_values():
+    # SiLU(g) = g/(1 + e^-g) at points worked by hand from e's decimal
+    # expansion (tests/golden/silu.json), to 2 ulp of fp64
+    cases = json.load(open(os.path.join(GOLDEN, "silu.json")))["cases"]
+    g = np.array([c["g"] for c in cases])
+    import oracle.ffn as F  # looked up at call time, as the oracle's forward does
+    got = F.activate(g, "silu")
+    for c, gv in zip(cases, got):
+        assert _ulp_close(float(gv), Fraction(c["silu"]), 2), (c, gv)
+
+
+def test_silu_odd_part_identity():
+    # SiLU(g) - SiLU(-g) = g·(sigma(g) + sigma(-g)) - 0 = g for every g,
+    # since sigma(g) + sigma(-g) = 1
+    import oracle.ffn as F  # looked up at call time, as the oracle's forward does
+    g = np.linspace(-20.0, 20.0, 4001)
+    d = F.activate(g, "silu") - F.activate(-g, "silu")
+    assert np.all(np.abs(d - g) <= 4 * np.finfo(np.float64).eps * np.maximum(np.abs(g), 1))
+
+
 def test_threshold_tests_the_unrounded_activation():
     # reading 2: keep iff |sigma(g)| > tau on the unrounded activation, strict.
     # a = 1 + 2^-10 with tau = 1: kept, although its stored bf16 value is
@@ -345,7 +373,7 @@ def test_lognormal_nnz_recipe():
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("mutation", ["no_bias", "no_value_round", "transposed_down",
                                       "nonstrict", "silu_sign", "topk_tie_high", "no_z_round",
-                                      "keep_on_rounded", "norms_unrounded"])
+                                      "keep_on_rounded", "norms_unrounded", "silu_is_sigmoid"])
 def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     import oracle.ffn as F
     if mutation == "no_bias":
@@ -377,6 +405,10 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
         monkeypatch.setattr(F, "wina_norms", lambda W: np.sqrt(np.sum(W * W, axis=1)))
     elif mutation == "keep_on_rounded":
         monkeypatch.setattr(F, "keep_threshold", lambda a, tau: np.abs(F.round_bf16(a)) > tau)
+    elif mutation == "silu_is_sigmoid":
+        orig_act = F.activate
+        monkeypatch.setattr(F, "activate",
+                            lambda g, act: 1 / (1 + np.exp(-g)) if act == "silu" else orig_act(g, act))
     elif mutation == "no_z_round":
         def no_round(x, A, B, bias, dtype):
             z = x @ A
@@ -387,9 +419,22 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutation):
     for test in (test_hand_worked_threshold, test_hand_worked_wina_relu,
                  lambda: test_bruteforce_rational(0, 128, 4, 3, 0.0),
                  test_wina_reductions, test_lowrank_z_is_rounded_to_the_operand_dtype,
-                 test_threshold_tests_the_unrounded_activation, test_wina_norms_are_fp32_rounded):
+                 test_threshold_tests_the_unrounded_activation, test_wina_norms_are_fp32_rounded,
+                 test_silu_hand_worked_values, test_silu_odd_part_identity):
         try:
             test()
         except AssertionError:
             failures += 1
     assert failures > 0, mutation
+
+
+def test_silu_goldens_alone_catch_sigmoid_for_silu(monkeypatch):
+    # the hand-worked values and the odd-part identity each reject a SiLU
+    # replaced by the plain logistic sigmoid, without any other pin's help
+    import oracle.ffn as F
+    orig_act = F.activate
+    monkeypatch.setattr(F, "activate",
+                        lambda g, act: 1 / (1 + np.exp(-g)) if act == "silu" else orig_act(g, act))
+    for test in (test_silu_hand_worked_values, test_silu_odd_part_identity):
+        with pytest.raises(AssertionError):
+            test()
