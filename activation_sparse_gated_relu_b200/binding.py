@@ -176,6 +176,24 @@ def _view(ptr: int, shape, typestr: str, torch_dtype=None):
     return t.clone()
 
 
+def _check_tensor(t, name: str, dtype, shape, cuda: bool) -> None:
+    """The C ABI sees only a pointer: the dtype, shape, device and layout of
+    every tensor are checked here, before the call."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if t.is_cuda != cuda:
+        raise ValueError(f"{name} must be a {'CUDA' if cuda else 'host (CPU)'} tensor")
+    if t.numel() and t.data_ptr() % 16:
+        raise ValueError(f"{name} must start on a 16-byte boundary")
+
+
 _DTYPE = {"bf16": SFFN_BF16, "fp32": SFFN_FP32}
 _MODE = {"relu_threshold": SFFN_MODE_RELU_THRESHOLD, "wina_topk": SFFN_MODE_WINA_TOPK}
 _ACT = {"relu": SFFN_ACT_RELU, "silu": SFFN_ACT_SILU}
@@ -194,12 +212,29 @@ class SparseFFN:
                  k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
                  debug_gate: bool = False, separate: bool = False, stream: Optional[int] = None):
         import torch
+        self.h = None
         self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias) if t is not None]
         dt = W_up.dtype
         if dt not in (torch.bfloat16, torch.float32):
             raise TypeError("operands must be bf16 or fp32")
+        if W_up.dim() != 2:
+            raise ValueError("W_up must be [d_ff][d_model]")
         self.dtype = "bf16" if dt == torch.bfloat16 else "fp32"
+        self._torch_dtype = dt
         F, d = W_up.shape
+        _check_tensor(W_up, "W_up", dt, (F, d), True)
+        _check_tensor(W_down, "W_down", dt, (F, d), True)
+        if (W_gate is None) == (A is None):
+            raise ValueError("give either W_gate (dense gate) or A and B (low-rank gate)")
+        if W_gate is not None:
+            _check_tensor(W_gate, "W_gate", dt, (F, d), True)
+        else:
+            if B is None or A.dim() != 2:
+                raise ValueError("the low-rank gate needs A [d_model][rank] and B [rank][d_ff]")
+            _check_tensor(A, "A", dt, (d, A.shape[1]), True)
+            _check_tensor(B, "B", dt, (A.shape[1], F), True)
+        if bias is not None:
+            _check_tensor(bias, "bias", torch.float32, (F,), True)
         self.d_model, self.d_ff, self.max_tokens = d, F, max_tokens
         desc = sffn_desc()
         desc.d_model, desc.d_ff, desc.max_tokens = d, F, max_tokens
@@ -223,9 +258,23 @@ class SparseFFN:
         import torch
         return torch.cuda.current_stream().cuda_stream if stream is None else int(stream)
 
+    def _check_io(self, x, out, cuda: bool) -> int:
+        import torch
+        if not isinstance(x, torch.Tensor) or x.dim() != 2:
+            raise ValueError("x must be a [T][d_model] tensor")
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T = {T} exceeds max_tokens = {self.max_tokens}")
+        _check_tensor(x, "x", self._torch_dtype, (T, self.d_model), cuda)
+        if out is not None:
+            _check_tensor(out, "out", torch.float32, (T, self.d_model), cuda)
+            if cuda and out.device != x.device:
+                raise ValueError("x and out must be on the same device")
+        return T
+
     def forward(self, x, out=None, stream: Optional[int] = None):
         import torch
-        T = x.shape[0]
+        T = self._check_io(x, out, cuda=True)
         if out is None:
             out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
         sffn_forward(self.h, x.data_ptr(), T, out.data_ptr(), self._stream(stream))
@@ -235,7 +284,7 @@ class SparseFFN:
 
     def forward_host(self, x_host, out_host=None, stream: Optional[int] = None):
         import torch
-        T = x_host.shape[0]
+        T = self._check_io(x_host, out_host, cuda=False)
         if out_host is None:
             out_host = torch.empty((T, self.d_model), dtype=torch.float32, pin_memory=True)
         sffn_forward_host(self.h, x_host.data_ptr(), T, out_host.data_ptr(), self._stream(stream))

@@ -23,6 +23,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -1095,6 +1096,9 @@ namespace {
 
 constexpr int kNaMaxT = 64, kNaMaxD = 4096, kNaMaxR = 1024, kNaMaxF = 16384;
 constexpr int kNaTickets = kNaMaxR / 128;
+// Scratch held per GPU: the fp32 split partials of z, (1024/128 row tiles) x
+// 4 splits x 64 tokens x 128 rows x 4 B = 1 MiB; z itself, 64 x 1024 x 2 B =
+// 128 KiB; the tickets and the status word: 1,179,696 bytes in all (~1.2 MB).
 
 static __device__ __align__(256) float g_na_zpart[(kNaMaxR / 128) * Z_MAX_SPLITS * kNaMaxT * 128];
 static __device__ __align__(256) __nv_bfloat16 g_na_z[kNaMaxT * kNaMaxR];
@@ -1111,6 +1115,8 @@ struct NaScratch {
 constexpr int kNaMaxDevices = 64;
 NaScratch g_na_dev[kNaMaxDevices];
 std::mutex g_na_mu;
+// test hook (sffn_debug_noalloc_waits): hold time of the calls' kernels, ns
+std::atomic<unsigned long long> g_na_hold_ns{0};
 
 // Device addresses of the scratch arrays for the current device (looked up
 // once per device; the host-side names of the arrays are not device addresses).
@@ -1181,11 +1187,13 @@ extern "C" sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_mo
   if (!make_map(&mAt, A_t, d_model, rank, 128) || !make_map(&mx, x, d_model, T, BN) ||
       !make_map(&mBt, B_t, rank, d_ff, 128) || !make_map(&mz, sc->z, rank, T, BN))
     return SFFN_ERR_CUDA;
+  const unsigned long long hold = g_na_hold_ns.load();
   TcArgs za{};
   za.n_phase = 1;
   za.kb_total[0] = cdiv(d_model, 64);
   za.n_rows = T;
   za.status = sc->status;
+  za.hold_ns = hold;
   ZParams zp{T, rank, sk, sc->zpart, sc->z, sc->tickets};
   if (launch_tc<EpiLowRankZ>(BN, dim3(mt, ntile, sk), st, mAt, mx, mAt, mx, za, zp) != cudaSuccess)
     return SFFN_ERR_CUDA;
@@ -1194,6 +1202,7 @@ extern "C" sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_mo
   ga.kb_total[0] = cdiv(rank, 64);
   ga.n_rows = T;
   ga.status = sc->status;
+  ga.hold_ns = hold;
   TwellParams tw;
   tw.bias = gate_bias;
   tw.tau = threshold;
@@ -1212,5 +1221,35 @@ extern "C" sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_mo
   tw.gdebug = nullptr;
   if (launch_tc<EpiGateTwell>(BN, dim3(P, ntile, 1), st, mBt, mz, mBt, mz, ga, tw) != cudaSuccess)
     return SFFN_ERR_CUDA;
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_lowrank_twell_noalloc_status(void* cuda_stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_NO_DEVICE;
+  }
+  NaScratch* sc = nullptr;
+  sffn_status ss = na_setup(dev, &sc);
+  if (ss != SFFN_OK) return ss;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint32_t w = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemcpy(&w, sc->status, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_CUDA;
+  }
+  if (w && cudaMemset(sc->status, 0, sizeof(w)) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_CUDA;
+  }
+  if (w & DEV_ERR_TIMEOUT) return SFFN_ERR_TIMEOUT;
+  if (w & DEV_ERR_RANGE) return SFFN_ERR_DEVICE;
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_debug_noalloc_waits(unsigned wait_us) {
+  g_na_hold_ns.store((unsigned long long)wait_us * 1000ull);
   return SFFN_OK;
 }

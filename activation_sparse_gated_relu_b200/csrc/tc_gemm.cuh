@@ -48,6 +48,9 @@ struct TcArgs {
   float4* zero_out;     // if set, the CTAs zero zero_n4 float4 here (after the grid dependency)
   long long zero_n4;
   int stages;           // ring stages in use (0: all that fit); fewer bound the bytes in flight
+  unsigned long long hold_ns;  // test hook (0: off): before issuing any copy the producer waits
+                               // this long on a barrier that nothing signals, then records a
+                               // timeout and the CTA returns without output
 };
 
 template <class E, class = void>
@@ -143,6 +146,17 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       // ------------------------------------------------------- TMA producer
       int it = 0;
       bool ok = true;
+      if (args.hold_ns) {
+        // no copy is in flight yet: the wait runs out, the MMA warp sees the
+        // abort flag, and the epilogue writes nothing
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&full[0], 0)) {
+          if (globaltimer() - t0 > args.hold_ns) break;
+        }
+        *abort_flag = 1;
+        atomicOr(args.status, DEV_ERR_TIMEOUT);
+        ok = false;
+      }
       for (int ph = 0; ph < args.n_phase && ok; ++ph) {
         const CUtensorMap* ma = ph == 0 ? &mA0 : &mA1;
         const CUtensorMap* mb = ph == 0 ? &mB0 : &mB1;

@@ -234,16 +234,34 @@ sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], 
  * Limits: T <= 64, d_model <= 4096 (multiple of 8), rank <= 1024 (multiple of
  * 64), d_ff <= 16384 (multiple of 128); larger sizes return
  * SFFN_ERR_UNSUPPORTED before anything runs.  Scratch lives in fixed device
- * arrays inside this library (about 400 KB per GPU, held until the process
- * exits); the first call on a device looks their addresses up, so make that
- * call before any stream capture.  Every call shares that scratch and clears
- * what must start at zero, so calls that overlap on the GPU (two streams, two
- * threads) race and must be serialised by the caller.  Asynchronous on
- * cuda_stream; no allocation, no host synchronisation. */
+ * arrays inside this library (1,179,696 bytes, about 1.2 MB, per GPU, held
+ * until the process exits); the first call on a device looks their addresses
+ * up, so make that call before any stream capture.  Every call shares that
+ * scratch and clears what must start at zero, so calls that overlap on the
+ * GPU (two streams, two threads) race and must be serialised by the caller.
+ * Asynchronous on cuda_stream; no allocation, no host synchronisation.
+ * Device-side errors (a bounded wait that expired) go to a status word that
+ * all calls on the device share; sffn_lowrank_twell_noalloc_status reads it.
+ * A call whose kernels recorded an error leaves its outputs undefined. */
 sffn_status sffn_lowrank_twell_noalloc(const void* x, int T, int d_model, const void* A_t, int rank,
                                        const void* B_t, int d_ff, const float* gate_bias, int act,
                                        float threshold, int tile_capacity, int16_t* count, int16_t* idx,
                                        void* val, uint32_t* overflow, void* cuda_stream);
+
+/* Status of the allocation-free calls on the current device: synchronises
+ * `cuda_stream`, then returns and clears the device status word that those
+ * calls' kernels share (SFFN_OK, SFFN_ERR_TIMEOUT or SFFN_ERR_DEVICE).  Errors
+ * of every call since the last read accumulate in it.  SFFN_ERR_CUDA if the
+ * synchronisation or the read fails. */
+sffn_status sffn_lowrank_twell_noalloc_status(void* cuda_stream);
+
+/* Test hook for the allocation-free calls' bounded waits.  While wait_us is
+ * not 0, their kernels wait wait_us microseconds on a barrier that nothing
+ * signals before they issue any copy, then record a timeout and return
+ * without writing outputs (sffn_lowrank_twell_noalloc_status then returns
+ * SFFN_ERR_TIMEOUT); nothing faults or hangs.  0 turns the hook off.
+ * Process-wide; always SFFN_OK. */
+sffn_status sffn_debug_noalloc_waits(unsigned wait_us);
 
 /* Library version string. */
 const char* sffn_version(void);

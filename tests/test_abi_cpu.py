@@ -134,3 +134,45 @@ def test_binding_raises_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(ImportError):
         B.load_library(str(tmp_path / "missing.so"))
+
+
+def _handle_stub(dtype: str = "bf16", d_model: int = 64, max_tokens: int = 8):
+    """A SparseFFN whose argument checks run without a device: the checks use
+    only the descriptor-level attributes, and every bad call below must raise
+    before the library is reached (a null handle would be rejected there)."""
+    import torch
+    f = B.SparseFFN.__new__(B.SparseFFN)
+    f.h = None
+    f.dtype = dtype
+    f._torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+    f.d_model, f.d_ff, f.max_tokens = d_model, 256, max_tokens
+    return f
+
+
+def test_binding_rejects_mismatched_activations():
+    import torch
+    f = _handle_stub()
+    x = torch.zeros((4, 64), dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="x must be torch.bfloat16"):
+        f.forward(x.float())                           # fp32 x on a bf16 handle
+    with pytest.raises(ValueError, match="shape"):
+        f.forward(torch.zeros((4, 32), dtype=torch.bfloat16))   # wrong d_model
+    with pytest.raises(ValueError, match="contiguous"):
+        f.forward(torch.zeros((64, 4), dtype=torch.bfloat16).t())  # a transposed view
+    with pytest.raises(ValueError, match="CUDA"):
+        f.forward(x)                                   # host tensor on the device entry point
+    with pytest.raises(ValueError, match="max_tokens"):
+        f.forward(torch.zeros((9, 64), dtype=torch.bfloat16))
+    with pytest.raises(TypeError, match="out must be torch.float32"):
+        f.forward_host(x, torch.zeros((4, 64), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out must have shape"):
+        f.forward_host(x, torch.zeros((3, 64), dtype=torch.float32))
+
+
+def test_binding_rejects_host_or_misshaped_weights():
+    import torch
+    W = torch.zeros((256, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.SparseFFN(W, W, W_gate=W)                   # host weights
+    with pytest.raises(ValueError, match="W_gate or A and B"):
+        B.SparseFFN(W, W)                             # no gate at all
