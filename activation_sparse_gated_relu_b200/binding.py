@@ -219,13 +219,13 @@ class SparseFFN:
             raise TypeError("operands must be bf16 or fp32")
         if W_up.dim() != 2:
             raise ValueError("W_up must be [d_ff][d_model]")
+        if (W_gate is None) == (A is None):
+            raise ValueError("give either W_gate (dense gate) or A and B (low-rank gate)")
         self.dtype = "bf16" if dt == torch.bfloat16 else "fp32"
         self._torch_dtype = dt
         F, d = W_up.shape
         _check_tensor(W_up, "W_up", dt, (F, d), True)
         _check_tensor(W_down, "W_down", dt, (F, d), True)
-        if (W_gate is None) == (A is None):
-            raise ValueError("give either W_gate (dense gate) or A and B (low-rank gate)")
         if W_gate is not None:
             _check_tensor(W_gate, "W_gate", dt, (F, d), True)
         else:
