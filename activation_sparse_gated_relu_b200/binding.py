@@ -82,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_debug_keep.restype = st
     lib.sffn_debug_gate.argtypes = [vp, ctypes.POINTER(vp)]
     lib.sffn_debug_gate.restype = st
+    lib.sffn_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.sffn_workspace_bytes.restype = st
     lib.sffn_debug_norms.argtypes = [vp, ctypes.POINTER(vp)]
     lib.sffn_debug_norms.restype = st
     lib.sffn_get_stats.argtypes = [vp, vp, ctypes.POINTER(sffn_stats)]
@@ -324,6 +326,12 @@ class SparseFFN:
         g = ctypes.c_void_p()
         _check(load_library().sffn_debug_gate(self.h, ctypes.byref(g)), "gate_debug")
         return _view(g.value, (T, self.d_ff), "<f4")
+
+    def workspace_bytes(self) -> int:
+        """Bytes of device memory the handle allocated (one workspace)."""
+        n = ctypes.c_size_t()
+        _check(load_library().sffn_workspace_bytes(self.h, ctypes.byref(n)), "workspace_bytes")
+        return int(n.value)
 
     def norms(self):
         n = ctypes.c_void_p()

@@ -217,6 +217,9 @@ struct sffn_handle {
   uint32_t* status = nullptr;
   void* xstage = nullptr;
   float* ostage = nullptr;
+  void* arena = nullptr;         // the one device allocation all of the above live in
+  size_t arena_bytes = 0;
+  bool dense_bufs = false;       // xo, h_hi, h_lo and W_down^T exist (paths other than the single launch)
   // A-operand tensor maps (box 64 x 128)
   CUtensorMap tmWgate, tmWup, tmWdT, tmAt, tmBt;
   int last_T = 0, last_path = 0, last_launches = 0;
@@ -235,6 +238,7 @@ struct sffn_handle {
   uint4* wl_val = nullptr;
   int dec_maxr = 0, dec_smem = 0, dec_grid = 0;
   bool dec_ok = false;
+  bool dec_pdl = true;           // the single launch also asks for programmatic dependent launch
   int dec_phantom = 0;           // test hook (sffn_debug_decode_waits)
   unsigned long long dec_wait_ns = SFFN_WAIT_LIMIT_NS;
   bool last_fused = false;     // the last forward was the single launch: its routing is the ovf flags
@@ -254,14 +258,23 @@ void timing_free(sffn_handle* h);
 void free_handle(sffn_handle* h) {
   if (!h) return;
   timing_free(h);
-  void* ptrs[] = {h->count, h->idx, h->val, h->ovf, h->kmask, h->ovf_list, h->ovf_count,
-                  h->xo, h->h_hi, h->h_lo, h->scores, h->vdense, h->norms, h->z, h->zo, h->zpart,
-                  h->tickets, h->At, h->Bt, h->WdT, h->gdebug, h->status, h->xstage, h->ostage,
-                  h->gstage, h->gtick, h->dsched, h->wl_id, h->wl_val};
-  for (void* p : ptrs)
-    if (p) cudaFree(p);
+  if (h->arena) cudaFree(h->arena);
   delete h;
 }
+
+// Carves the handle's workspace out of one device allocation: run once with
+// base == nullptr to size it, then again with the allocation's base.  Every
+// buffer starts on a 256-byte boundary (TMA and 16-byte vector accesses).
+struct Arena {
+  uint8_t* base = nullptr;
+  size_t size = 0;
+  template <typename T>
+  void take(T** p, size_t bytes) {
+    size = (size + 255) & ~size_t(255);
+    *p = base ? reinterpret_cast<T*>(base + size) : nullptr;
+    size += bytes ? bytes : 16;
+  }
+};
 
 template <typename T>
 bool dalloc(T** p, size_t bytes) {
@@ -393,80 +406,14 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   h->wina = desc->mode == SFFN_MODE_WINA_TOPK;
   h->lowrank = desc->rank > 0;
   const size_t T = (size_t)h->maxT, d = (size_t)h->d, F = (size_t)h->F, P = (size_t)h->P, C = (size_t)h->C;
-  bool ok = true;
-  ok = ok && dalloc(&h->count, T * P * 2);
-  ok = ok && dalloc(&h->idx, T * P * C * 2);
-  ok = ok && dalloc(&h->val, T * P * C * h->esize);
-  ok = ok && dalloc(&h->ovf, T * 4);
-  ok = ok && dalloc(&h->kmask, T * P * 16);
-  ok = ok && dalloc(&h->ovf_list, T * 4);
-  ok = ok && dalloc(&h->ovf_count, 16);
-  ok = ok && dalloc(&h->status, 16);
-  ok = ok && dalloc(&h->xstage, T * d * h->esize);
-  ok = ok && dalloc(&h->ostage, T * d * 4);
-  if (!h->f32) {
-    ok = ok && dalloc(&h->xo, T * d * 2);
-    ok = ok && dalloc(&h->h_hi, T * F * 2);
-    ok = ok && dalloc(&h->h_lo, T * F * 2);
-    ok = ok && dalloc(&h->WdT, d * F * 2);
-  }
-  if (h->wina) {
-    ok = ok && dalloc(&h->scores, T * F * 4);
-    ok = ok && dalloc(&h->vdense, T * F * h->esize);
-    ok = ok && dalloc(&h->norms, F * 4);
-  }
-  if (h->lowrank) {
-    const size_t R = (size_t)h->R;
-    ok = ok && dalloc(&h->z, T * R * 2);
-    ok = ok && dalloc(&h->zo, T * R * 2);
-    ok = ok && dalloc(&h->zpart, (R / 128 + 1) * Z_MAX_SPLITS * (size_t)pick_bn((int)std::min<size_t>(T, 256)) * 128 * 4);
-    ok = ok && dalloc(&h->tickets, (R / 128 + 1) * 4);
-    ok = ok && dalloc(&h->At, R * d * 2);
-    ok = ok && dalloc(&h->Bt, F * R * 2);
-  }
-  if (desc->flags & SFFN_FLAG_DEBUG_GATE) ok = ok && dalloc(&h->gdebug, T * F * 4);
-  if (!h->f32 && !h->wina && !h->lowrank) {
-    ok = ok && dalloc(&h->gstage, P * 8 * 128 * 4);
-    ok = ok && dalloc(&h->gtick, P * 4);
-  }
-  if (!ok) {
-    free_handle(h);
-    return SFFN_ERR_ALLOC;
-  }
+  const size_t R = (size_t)h->R;
   cudaError_t e = cudaSuccess;
-  e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
-  e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
-  e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
-  if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
-  if (h->lowrank) {
-    e = e ? e : cudaMemsetAsync(h->tickets, 0, ((size_t)h->R / 128 + 1) * 4, st);
-  }
-  // create-time derived data
-  const dim3 tb(32, 8);
-  if (!e && !h->f32) {
-    k_transpose_bf16<<<dim3(cdiv(d, 32), cdiv(F, 32)), tb, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(desc->W_down), h->WdT, (int)F, (int)d);
-    e = cudaGetLastError();
-  }
-  if (!e && h->lowrank) {
-    const int R = h->R;
-    k_transpose_bf16<<<dim3(cdiv(R, 32), cdiv(d, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->A),
-                                                                    h->At, (int)d, R);
-    k_transpose_bf16<<<dim3(cdiv(F, 32), cdiv(R, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->B),
-                                                                    h->Bt, R, (int)F);
-    e = cudaGetLastError();
-  }
-  if (!e && h->wina) {
-    if (h->f32)
-      k_row_norms<float><<<cdiv(F, 8), 256, 0, st>>>(static_cast<const float*>(desc->W_down), (int)F, (int)d,
-                                                      h->norms);
-    else
-      k_row_norms<__nv_bfloat16><<<cdiv(F, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->W_down),
-                                                             (int)F, (int)d, h->norms);
-    e = cudaGetLastError();
-  }
-  // kernel attributes and A-operand tensor maps
-  if (!e && !h->f32) {
+  int max_smem = 0;
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const bool dense_gate_bf16 = !h->f32 && !h->wina && !h->lowrank;
+
+  // ------------------------------------------- kernel attributes and shapes
+  if (!h->f32) {
     e = e ? e : set_tc_attrs<EpiGateTwell>();
     e = e ? e : set_gate_persist_attrs(h->C);
     e = e ? e : set_tc_attrs<EpiWina>();
@@ -474,21 +421,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     e = e ? e : set_tc_attrs<EpiFallbackH>();
     e = e ? e : set_tc_attrs<EpiTwellH>();
     e = e ? e : set_tc_attrs<EpiDownOut>();
-    bool mok = true;
-    if (!h->lowrank) mok = mok && make_map(&h->tmWgate, desc->W_gate, h->d, h->F, 128);
-    mok = mok && make_map(&h->tmWup, desc->W_up, h->d, h->F, 128);
-    mok = mok && make_map(&h->tmWdT, h->WdT, h->F, h->d, 128);
-    if (h->lowrank) {
-      mok = mok && make_map(&h->tmAt, h->At, h->d, h->R, 128);
-      mok = mok && make_map(&h->tmBt, h->Bt, h->R, h->F, 128);
-    }
-    if (!mok) {
-      free_handle(h);
-      return SFFN_ERR_CUDA;
-    }
     // fused up x down: ring slots and list capacity from the shared memory budget
-    int max_smem = 0;
-    cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     int lcap = 512, ns = RW_NSMAX;
     auto fits = [&](int l, int n) { return RowsSmem::make(h->P, l, h->d, n).total <= max_smem; };
     while (ns > 2 && !fits(lcap, ns)) --ns;
@@ -502,8 +435,8 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
                  h->P <= RW_THREADS &&
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
-    // row-streaming gate: the same staged-row layout, as many ring slots as fit
-    if (h->gstage) {
+    if (dense_gate_bf16) {
+      // row-streaming gate: the same staged-row layout, two ring slots
       const int gns = 2;
       h->gr_nslot = gns;
       h->gr_smem = GateRowsSmem::make(h->d, gns).total;
@@ -525,17 +458,6 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
         if (!e) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode, RW_THREADS, h->dec_smem);
         h->dec_ok = !e && nb >= 1;
       }
-      if (h->dec_ok && !e) {
-        h->dsched_ints = decode_sched_ints((int)P, G + 1);
-        bool aok = dalloc(&h->dsched, (size_t)h->dsched_ints * 4);
-        aok = aok && dalloc(&h->wl_id, (size_t)G * h->dec_maxr * 4);
-        aok = aok && dalloc(&h->wl_val, (size_t)G * h->dec_maxr * 16);
-        if (!aok) {
-          free_handle(h);
-          return SFFN_ERR_ALLOC;
-        }
-        e = cudaMemsetAsync(h->dsched, 0, (size_t)h->dsched_ints * 4, st);
-      }
     }
   }
   if (!e && h->wina) {
@@ -549,9 +471,121 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     e = e ? e : cudaFuncSetAttribute(k_fallback_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)((d + F) * 4));
   }
+  if (e) {
+    cudaGetLastError();
+    free_handle(h);
+    return SFFN_ERR_CUDA;
+  }
+  // Every forward of a handle whose token count never exceeds 8 takes the
+  // single decode launch (ROWS path, no SFFN_FLAG_SEPARATE), which reads
+  // W_down by rows and keeps h in registers: such a handle holds neither the
+  // transposed W_down nor the h and overflow-row buffers of the other paths.
+  h->dense_bufs = !h->f32 && !(h->dec_ok && h->maxT <= 8 && !(desc->flags & SFFN_FLAG_SEPARATE) &&
+                               desc->path != SFFN_PATH_TILES);
+
+  // ------------------------------------------ workspace: one allocation
+  Arena ar;
+  auto plan = [&](Arena& a) {
+    a.take(&h->count, T * P * 2);
+    a.take(&h->idx, T * P * C * 2);
+    a.take(&h->val, T * P * C * h->esize);
+    a.take(&h->ovf, T * 4);
+    a.take(&h->kmask, T * P * 16);
+    a.take(&h->ovf_list, T * 4);
+    a.take(&h->ovf_count, 16);
+    a.take(&h->status, 16);
+    a.take(&h->xstage, T * d * h->esize);
+    a.take(&h->ostage, T * d * 4);
+    if (h->dense_bufs) {
+      a.take(&h->xo, T * d * 2);
+      a.take(&h->h_hi, T * F * 2);
+      a.take(&h->h_lo, T * F * 2);
+      a.take(&h->WdT, d * F * 2);
+    }
+    if (h->wina) {
+      a.take(&h->scores, T * F * 4);
+      a.take(&h->vdense, T * F * h->esize);
+      a.take(&h->norms, F * 4);
+    }
+    if (h->lowrank) {
+      a.take(&h->z, T * R * 2);
+      a.take(&h->zo, T * R * 2);
+      a.take(&h->zpart, (R / 128 + 1) * Z_MAX_SPLITS * (size_t)pick_bn((int)std::min<size_t>(T, 256)) * 128 * 4);
+      a.take(&h->tickets, (R / 128 + 1) * 4);
+      a.take(&h->At, R * d * 2);
+      a.take(&h->Bt, F * R * 2);
+    }
+    if (desc->flags & SFFN_FLAG_DEBUG_GATE) a.take(&h->gdebug, T * F * 4);
+    if (dense_gate_bf16) {
+      a.take(&h->gstage, P * 8 * 128 * 4);
+      a.take(&h->gtick, P * 4);
+    }
+    if (h->dec_ok) {
+      h->dsched_ints = decode_sched_ints((int)P, h->dec_grid + 1);
+      a.take(&h->dsched, (size_t)h->dsched_ints * 4);
+      a.take(&h->wl_id, (size_t)h->dec_grid * h->dec_maxr * 4);
+      a.take(&h->wl_val, (size_t)h->dec_grid * h->dec_maxr * 16);
+    }
+  };
+  plan(ar);                      // sizes
+  if (!dalloc(&h->arena, ar.size)) {
+    free_handle(h);
+    return SFFN_ERR_ALLOC;
+  }
+  h->arena_bytes = ar.size;
+  ar.base = static_cast<uint8_t*>(h->arena);
+  ar.size = 0;
+  plan(ar);                      // addresses
+
+  e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
+  e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
+  e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
+  if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
+  if (h->lowrank) e = e ? e : cudaMemsetAsync(h->tickets, 0, (R / 128 + 1) * 4, st);
+  if (h->dsched) e = e ? e : cudaMemsetAsync(h->dsched, 0, (size_t)h->dsched_ints * 4, st);
+  // create-time derived data
+  const dim3 tb(32, 8);
+  if (!e && h->WdT) {
+    k_transpose_bf16<<<dim3(cdiv(d, 32), cdiv(F, 32)), tb, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(desc->W_down), h->WdT, (int)F, (int)d);
+    e = cudaGetLastError();
+  }
+  if (!e && h->lowrank) {
+    k_transpose_bf16<<<dim3(cdiv(R, 32), cdiv(d, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->A),
+                                                                    h->At, (int)d, (int)R);
+    k_transpose_bf16<<<dim3(cdiv(F, 32), cdiv(R, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->B),
+                                                                    h->Bt, (int)R, (int)F);
+    e = cudaGetLastError();
+  }
+  if (!e && h->wina) {
+    if (h->f32)
+      k_row_norms<float><<<cdiv(F, 8), 256, 0, st>>>(static_cast<const float*>(desc->W_down), (int)F, (int)d,
+                                                      h->norms);
+    else
+      k_row_norms<__nv_bfloat16><<<cdiv(F, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->W_down),
+                                                             (int)F, (int)d, h->norms);
+    e = cudaGetLastError();
+  }
+  // A-operand tensor maps
+  if (!e && !h->f32) {
+    bool mok = true;
+    if (!h->lowrank) mok = mok && make_map(&h->tmWgate, desc->W_gate, h->d, h->F, 128);
+    mok = mok && make_map(&h->tmWup, desc->W_up, h->d, h->F, 128);
+    if (h->WdT) mok = mok && make_map(&h->tmWdT, h->WdT, h->F, h->d, 128);
+    if (h->lowrank) {
+      mok = mok && make_map(&h->tmAt, h->At, h->d, h->R, 128);
+      mok = mok && make_map(&h->tmBt, h->Bt, h->R, h->F, 128);
+    }
+    if (!mok) {
+      cudaStreamSynchronize(st);
+      free_handle(h);
+      return SFFN_ERR_CUDA;
+    }
+  }
   if (!e) e = cudaStreamSynchronize(st);
   if (e) {
     cudaGetLastError();
+    cudaStreamSynchronize(st);
     free_handle(h);
     return SFFN_ERR_CUDA;
   }
@@ -566,6 +600,42 @@ sffn_status sffn_destroy(sffn_handle* h) {
   return SFFN_OK;
 }
 
+// The single decode launch's CTAs wait on one another (row lists, zeroed
+// slices of out), so all of them must be resident at once.  It is launched
+// cooperatively: when the grid cannot be co-resident (an SM-limited MPS
+// client, a green context, SMs held by another persistent kernel) the driver
+// fails the launch up front, or holds it until the whole grid fits, instead of
+// the resident CTAs waiting out their limits.  Programmatic dependent launch
+// is requested beside it; if the driver refuses the pair, the launch is
+// repeated, and later ones made, without it.
+static cudaError_t launch_decode(sffn_handle* h, const DecodeArgs& da, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(h->dec_grid);
+  cfg.blockDim = dim3(RW_THREADS);
+  cfg.dynamicSmemBytes = (size_t)h->dec_smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeCooperative;
+  at[n].val.cooperative = 1;
+  ++n;
+  if (h->dec_pdl) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode, da);
+  if (e == cudaSuccess) return e;
+  cudaGetLastError();
+  if (h->dec_pdl && e != cudaErrorCooperativeLaunchTooLarge) {
+    h->dec_pdl = false;
+    return launch_decode(h, da, st);
+  }
+  return e;
+}
+
 static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out, cudaStream_t st) {
   const sffn_desc& D = h->desc;
   const int d = h->d, F = h->F, P = h->P;
@@ -573,13 +643,6 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   const uint32_t epoch = h->epoch;
   const int BN = pick_bn(T);
   const int ntile_tok = cdiv(T, BN);
-  CUtensorMap mx, mxo, mhi, mlo, mz, mzo;
-  bool mok = make_map(&mx, x, d, T, BN) && make_map(&mxo, h->xo, d, h->maxT, BN) &&
-             make_map(&mhi, h->h_hi, F, h->maxT, BN) && make_map(&mlo, h->h_lo, F, h->maxT, BN);
-  if (h->lowrank)
-    mok = mok && make_map(&mz, h->z, h->R, h->maxT, BN) && make_map(&mzo, h->zo, h->R, h->maxT, BN);
-  if (!mok) return SFFN_ERR_CUDA;
-
   int path = D.path;
   if (path == SFFN_PATH_AUTO) path = (h->rows_ok && (T <= 8 || T > 256)) ? SFFN_PATH_ROWS : SFFN_PATH_TILES;
   if (h->wina) path = SFFN_PATH_TILES;  // the top-k kernel writes no per-token keep masks
@@ -634,13 +697,21 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     da.wait_ns = h->dec_wait_ns;
     da.phantom = h->dec_phantom;
     tmark(h, st, L_DECODE);
-    if (launch_pdl(k_decode, dim3(h->dec_grid), dim3(RW_THREADS), (size_t)h->dec_smem, st, 1, da))
-      return SFFN_ERR_CUDA;
+    if (launch_decode(h, da, st)) return SFFN_ERR_CUDA;
     h->last_path = SFFN_PATH_ROWS;
     h->last_launches = 1;
     h->last_fused = true;
     return SFFN_OK;
   }
+
+  // the other paths: tensor maps of x and of the workspace rows they use
+  if (!h->dense_bufs) return SFFN_ERR_UNSUPPORTED;  // unreachable: such handles always take the single launch
+  CUtensorMap mx, mxo, mhi, mlo, mz, mzo;
+  bool mok = make_map(&mx, x, d, T, BN) && make_map(&mxo, h->xo, d, h->maxT, BN) &&
+             make_map(&mhi, h->h_hi, F, h->maxT, BN) && make_map(&mlo, h->h_lo, F, h->maxT, BN);
+  if (h->lowrank)
+    mok = mok && make_map(&mz, h->z, h->R, h->maxT, BN) && make_map(&mzo, h->zo, h->R, h->maxT, BN);
+  if (!mok) return SFFN_ERR_CUDA;
 
   // ---------------------------------------------------------------- gate
   const CUtensorMap* gateA = &h->tmWgate;
@@ -1044,6 +1115,12 @@ sffn_status sffn_debug_gate(sffn_handle* h, const float** g) {
   if (!h || !g) return SFFN_ERR_INVALID_ARG;
   if (!h->gdebug) return SFFN_ERR_UNSUPPORTED;
   *g = h->gdebug;
+  return SFFN_OK;
+}
+
+sffn_status sffn_workspace_bytes(const sffn_handle* h, size_t* bytes) {
+  if (!h || !bytes) return SFFN_ERR_INVALID_ARG;
+  *bytes = h->arena_bytes;
   return SFFN_OK;
 }
 

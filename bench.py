@@ -352,31 +352,17 @@ def batch_sparsity(ffn, T: int, C: int) -> dict:
     return st
 
 
-def run_ours(args) -> None:
+def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, traffic_key) -> dict:
+    """Time `steps` forwards of workload `wl` at T tokens (after `warmup`):
+    NS rotating weight copies and NXB x batches resident in HBM, CUDA events
+    around the whole region, barrier and max over ranks.  Returns the line's
+    device-side fields (no e2e, no CPU baseline) plus the handles' objects
+    for the caller's end-to-end pass."""
     import torch
 
     import synth
-    from activation_sparse_gated_relu_b200 import SFFN_OK, SparseFFN, load_library
-    from activation_sparse_gated_relu_b200.build import build
+    from activation_sparse_gated_relu_b200 import SFFN_OK, SparseFFN
 
-    rank, local, world = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    if rank == 0:
-        build()
-    barrier(world)
-    load_library()
-
-    wl = synth.WORKLOADS[args.workload]
-    T, _, NXB, _ = BENCH_SHAPES[args.workload]
-    T = args.tokens or T
-    NS = args.weight_sets
     inp = synth.make_inputs(wl, T=T * NXB)
     dev = lambda t: None if t is None else t.to("cuda")  # noqa: E731
     sets = []
@@ -394,7 +380,7 @@ def run_ours(args) -> None:
     def step(i):
         sets[i % NS][1].forward(xb[i % NXB], outs[i % NS])
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
     for _, ffn in sets:
@@ -405,14 +391,14 @@ def run_ours(args) -> None:
     # per-kernel events on every TIMING_STRIDE-th forward of each handle: enough
     # launches to average, few enough not to perturb the timed region
     for _, ffn in sets:
-        ffn.timing_begin(args.steps // NS // TIMING_STRIDE + 2, TIMING_STRIDE)
+        ffn.timing_begin(steps // NS // TIMING_STRIDE + 2, TIMING_STRIDE)
     clocks = ClockSampler(torch.cuda.current_device())
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     ev0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -427,7 +413,7 @@ def run_ours(args) -> None:
             a[1] += n
     for _, ffn in sets:
         assert ffn.read_status() == SFFN_OK
-    tot_ms, tot_units = aggregate(elapsed, float(T * args.steps), world)
+    tot_ms, tot_units = aggregate(elapsed, float(T * steps), world)
 
     # ---------------------------------- algorithmic work of the batches
     ffn0 = sets[0][1]
@@ -448,15 +434,13 @@ def run_ours(args) -> None:
     # launches overlap prologue and tail by programmatic dependent launch; the
     # per-launch events, which break that overlap for the forwards they
     # bracket, are reported beside it as ms_per_launch_events)
-    single = len(kernels) == 1 and ffn0.stats().n_launches == 1
-    ms_dom = tot_ms / args.steps if single else per.get(dom, 0.0)
+    single = len(kernels) == 1 and launches_per_fwd == 1
+    ms_dom = tot_ms / steps if single else per.get(dom, 0.0)
     roof = None
     if dom in works and ms_dom > 0:
         roof = roofline_of(works[dom], ms_dom, peaks, peak_src)
-        # the committed captures are of the workload's own token count
-        traffic = profiled_traffic(dom, args.workload) if T == BENCH_SHAPES[args.workload][0] else None
-        roof.update({"kernel": dom, "traffic": traffic,
-                     "ms_per_launch": round(ms_dom, 5)})
+        traffic = profiled_traffic(dom, traffic_key) if traffic_key else None
+        roof.update({"kernel": dom, "traffic": traffic, "ms_per_launch": round(ms_dom, 5)})
         if single:
             roof.update({"ms_per_launch_events": round(per[dom], 5),
                          "launch_time": "timed-region events / launches (one launch per forward)"})
@@ -469,6 +453,60 @@ def run_ours(args) -> None:
             r = roofline_of(works[k], per[k], peaks, peak_src)
             e.update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
         kern_out[k] = e
+    step_s = tot_ms * 1e-3 / steps
+    return {
+        "value": round(tot_units / (tot_ms * 1e-3), 1), "ms_per_step": round(tot_ms / steps, 5),
+        "steps": steps, "warmup": warmup,
+        "hbm_gbs_step": round(bytes_step * world / step_s / 1e9, 1),
+        "hbm_frac_step": round(bytes_step * world / step_s / 1e9 / peaks["hbm_gbs"], 4),
+        "tflops_step": round(flops_step * world / step_s / 1e12, 2),
+        "tensor_frac_step": round(flops_step * world / step_s / 1e12
+                                  / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
+        "sparsity": {k: round(v, 1) for k, v in st.items()},
+        "path": path, "algorithmic_bytes_per_step": bytes_step, "algorithmic_flops_per_step": flops_step,
+        "roofline": roof, "kernels": kern_out, "gpu_launches": launches_per_fwd * steps, "clocks": clk,
+        "_sets": sets, "_inp": inp, "_NXB": NXB,
+    }
+
+
+# the other configurations, measured after the headline in the same default
+# run: (workload, tokens per forward)
+EXTRA_WORKLOADS = [("decode_bf16", 1), ("decode_bf16", 4), ("lopa_bf16", 32), ("wina_bf16", 32),
+                   ("prefill_bf16", 4096), ("tiny_fp32", 64)]
+EXTRA_MIN_STEPS = 200
+EXTRA_MAX_S = 2.0
+
+
+def run_ours(args) -> None:
+    import torch
+
+    import synth
+    from activation_sparse_gated_relu_b200 import load_library
+    from activation_sparse_gated_relu_b200.build import build
+
+    rank, local, world = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if rank == 0:
+        build()
+    barrier(world)
+    load_library()
+
+    wl = synth.WORKLOADS[args.workload]
+    T, _, NXB, _ = BENCH_SHAPES[args.workload]
+    T = args.tokens or T
+    NS = args.weight_sets
+    # the committed captures are of the workload's own token count
+    tkey = args.workload if T == BENCH_SHAPES[args.workload][0] else None
+    m = measure(wl, T, NS, NXB, args.steps, args.warmup, world, tkey)
+    sets, inp = m.pop("_sets"), m.pop("_inp")
+    m.pop("_NXB")
 
     # ------------------------------------------------------ end to end
     e2e = None
@@ -478,6 +516,7 @@ def run_ours(args) -> None:
         oh = torch.empty((T, wl.d_model), dtype=torch.float32).pin_memory()
         for i in range(3):
             sets[i % NS][1].forward_host(xh[i % NXB], oh)
+        stream = torch.cuda.current_stream()
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -492,6 +531,10 @@ def run_ours(args) -> None:
         e2e = {"value": round(e2e_units / (e2e_ms * 1e-3), 1), "unit": UNIT,
                "h2d_bytes_per_step": T * wl.d_model * es, "d2h_bytes_per_step": T * wl.d_model * 4,
                "api": "sffn_forward_host (pinned host x in, host y out, stream synchronised per step)"}
+    for _, ffn in sets:
+        ffn.close()
+    del sets
+    torch.cuda.empty_cache()
 
     # --------------------------------------------------- CPU baseline
     cpu = None
@@ -502,33 +545,47 @@ def run_ours(args) -> None:
                "sample": f"{n} fp64 oracle forwards of {T}-token batches of the same workload "
                          f"({el:.1f} s; operands decoded to fp64 once, before timing)"}
 
+    # ------------------------- the other configurations (one GPU only)
+    workloads = None
+    if world == 1 and not args.no_workloads and args.workload == DEFAULT_WORKLOAD and not args.tokens:
+        workloads = {}
+        for name, Tw in EXTRA_WORKLOADS:
+            wlx = synth.WORKLOADS[name]
+            _, NSx, NXBx, _ = BENCH_SHAPES[name]
+            # a bounded run: at least EXTRA_MIN_STEPS forwards, about
+            # EXTRA_MAX_S seconds at most, from a short probe of the step time
+            probe = measure(wlx, Tw, NSx, NXBx, 10, max(args.warmup, 3), world, None)
+            for _, f in probe.pop("_sets"):
+                f.close()
+            ksteps = max(EXTRA_MIN_STEPS, min(5000, int(EXTRA_MAX_S / (probe["ms_per_step"] * 1e-3))))
+            ksteps -= ksteps % NSx
+            key = name if Tw == BENCH_SHAPES[name][0] else None
+            r = measure(wlx, Tw, NSx, NXBx, ksteps, max(args.warmup, 3), world, key)
+            for _, f in r.pop("_sets"):
+                f.close()
+            r.pop("_inp"), r.pop("_NXB")
+            torch.cuda.empty_cache()
+            r["config"] = config_dict(wlx, Tw, NSx, NXBx)
+            r["dtype"] = "f32" if wlx.dtype == "fp32" else "bf16"
+            r["unit"] = UNIT
+            workloads[f"{name}@T={Tw}"] = r
+
     if rank == 0:
-        value = tot_units / (tot_ms * 1e-3)
-        step_s = tot_ms * 1e-3 / args.steps
         line = {
-            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_ms / args.steps, 5),
+            "metric": METRIC, "value": m["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if wl.dtype == "fp32" else "bf16",
             "data": "synthetic (seeded Gaussian x and N(0,1/fan_in) weights)",
             "config": config_dict(wl, T, NS, NXB),
-            "hbm_gbs_step": round(bytes_step * world / step_s / 1e9, 1),
-            "hbm_frac_step": round(bytes_step * world / step_s / 1e9 / peaks["hbm_gbs"], 4),
-            "tflops_step": round(flops_step * world / step_s / 1e12, 2),
-            "sparsity": {k: round(v, 1) for k, v in st.items()},
-            "path": path,
-            "algorithmic_bytes_per_step": bytes_step,
-            "algorithmic_flops_per_step": flops_step,
-            "roofline": roof,
-            "kernels": kern_out,
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": launches_per_fwd * args.steps,
-            "clocks": clk,
         }
+        for k in ("hbm_gbs_step", "hbm_frac_step", "tflops_step", "tensor_frac_step", "sparsity", "path",
+                  "algorithmic_bytes_per_step", "algorithmic_flops_per_step", "roofline", "kernels"):
+            line[k] = m[k]
+        line.update({"cpu_baseline": cpu, "e2e": e2e, "gpu_launches": m["gpu_launches"], "clocks": m["clocks"]})
+        if workloads is not None:
+            line["workloads"] = workloads
         print(json.dumps(line), flush=True)
-    for _, ffn in sets:
-        ffn.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -575,6 +632,8 @@ def main(argv=None) -> None:
     ap.add_argument("--workload", choices=sorted(BENCH_SHAPES), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other configurations measured after the default workload")
     ap.add_argument("--weight-sets", type=int, default=None,
                     help="rotating weight copies (fewer only for small profiler captures)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")

@@ -190,6 +190,12 @@ sffn_status sffn_debug_keep(sffn_handle* h, const uint32_t** keep);
  * with SFFN_FLAG_DEBUG_GATE; dense gate only).  Test use. */
 sffn_status sffn_debug_gate(sffn_handle* h, const float** g);
 
+/* Bytes of device memory the handle allocated (its whole workspace, one
+ * allocation: TwELL, routing, scratch, status and the create-time derived
+ * data).  A handle whose max_tokens is at most 8 and whose forwards all take
+ * the single decode launch holds no transposed W_down and no h buffers. */
+sffn_status sffn_workspace_bytes(const sffn_handle* h, size_t* bytes);
+
 /* Device view of the WINA norms n_j (fp32 [d_ff]), wina-topk mode only. */
 sffn_status sffn_debug_norms(sffn_handle* h, const float** norms);
 

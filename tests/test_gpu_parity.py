@@ -270,6 +270,66 @@ def test_decode_single_launch_bounded_waits(decode_inputs):
         ffn.close()
 
 
+def test_decode_handle_holds_no_dense_channel_copies(decode_inputs):
+    # a handle for at most 8 tokens takes the single launch on every forward:
+    # it holds neither the transposed W_down (117 MB at these sizes) nor the
+    # h buffers, and its device memory is its one workspace allocation
+    from activation_sparse_gated_relu_b200 import SparseFFN
+    inp = decode_inputs
+    dev = {k: to_dev(getattr(inp, k)) for k in ("W_gate", "W_up", "W_down", "bias")}
+
+    def make(max_tokens):
+        return SparseFFN(dev["W_up"], dev["W_down"], W_gate=dev["W_gate"], bias=dev["bias"],
+                         tile_capacity=32, max_tokens=max_tokens)
+
+    make(8).close()          # loads the kernels once, outside the measurement
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    ffn = make(8)
+    try:
+        torch.cuda.synchronize()
+        grew = free0 - torch.cuda.mem_get_info()[0]
+        ws = ffn.workspace_bytes()
+        assert ws < (4 << 20), ws
+        assert grew <= ws + (5 << 20), (grew, ws)
+        check(inp, T=8, ffn=ffn)
+    finally:
+        ffn.close()
+    # room for 9 tokens: other paths can run, so the handle keeps W_down^T
+    big = make(9)
+    try:
+        assert big.workspace_bytes() > inp.wl.d_model * inp.wl.d_ff * 2
+        check(inp, T=8, ffn=big)
+    finally:
+        big.close()
+
+
+def test_decode_two_handles_concurrently_on_two_streams(decode_inputs):
+    # two handles' single launches issued on two streams at once: each grid
+    # is co-resident by its cooperative launch (the driver runs them one
+    # after the other when both cannot fit), and both match the oracle
+    ffn_a = make_ffn(decode_inputs, max_tokens=8)
+    ffn_b = make_ffn(decode_inputs, max_tokens=8)
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    xa, xb = to_dev(decode_inputs.x[:8]), to_dev(decode_inputs.x[5:8])
+    oa = torch.full((8, ffn_a.d_model), float("nan"), dtype=torch.float32, device="cuda")
+    ob = torch.full((3, ffn_b.d_model), float("nan"), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    try:
+        for _ in range(25):
+            ffn_a.forward(xa, oa, stream=sa.cuda_stream)
+            ffn_b.forward(xb, ob, stream=sb.cuda_stream)
+        torch.cuda.synchronize()
+        assert ffn_a.read_status(sa.cuda_stream) == SFFN_OK
+        assert ffn_b.read_status(sb.cuda_stream) == SFFN_OK
+        ra = oracle.forward_inputs(decode_inputs, T=8)
+        assert rel_err(oa.double().cpu().numpy(), ra.y) <= 2e-3
+        assert rel_err(ob.double().cpu().numpy(), ra.y[5:8]) <= 2e-3
+    finally:
+        ffn_a.close()
+        ffn_b.close()
+
+
 def test_decode_single_launch_repeated_mixed_T(decode_inputs):
     # the scheduler words carry each forward's epoch: back-to-back forwards of
     # different sizes through one handle see only their own lists and zeros
