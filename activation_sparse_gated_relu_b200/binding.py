@@ -22,6 +22,7 @@ SFFN_ACT_RELU, SFFN_ACT_SILU = 0, 1
 SFFN_PATH_AUTO, SFFN_PATH_ROWS, SFFN_PATH_TILES = 0, 1, 2
 SFFN_FLAG_DEBUG_GATE = 1
 SFFN_FLAG_SEPARATE = 2
+SFFN_FLAG_COOPERATIVE = 4
 
 
 class sffn_desc(ctypes.Structure):
@@ -37,7 +38,7 @@ class sffn_desc(ctypes.Structure):
 
 class sffn_stats(ctypes.Structure):
     _fields_ = [("n_overflow", ctypes.c_int), ("n_launches", ctypes.c_int), ("path", ctypes.c_int),
-                ("epoch", ctypes.c_uint)]
+                ("epoch", ctypes.c_uint), ("launch_attrs", ctypes.c_uint)]
 
 
 class SffnError(RuntimeError):
@@ -212,7 +213,8 @@ class SparseFFN:
     def __init__(self, W_up, W_down, *, W_gate=None, A=None, B=None, bias=None,
                  mode: str = "relu_threshold", act: str = "relu", threshold: float = 0.0,
                  k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
-                 debug_gate: bool = False, separate: bool = False, stream: Optional[int] = None):
+                 debug_gate: bool = False, separate: bool = False, cooperative: bool = False,
+                 stream: Optional[int] = None):
         import torch
         self.h = None
         self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias) if t is not None]
@@ -248,7 +250,8 @@ class SparseFFN:
         desc.k = int(k)
         desc.tile_capacity = int(tile_capacity)
         desc.path = _PATH[path]
-        desc.flags = (SFFN_FLAG_DEBUG_GATE if debug_gate else 0) | (SFFN_FLAG_SEPARATE if separate else 0)
+        desc.flags = ((SFFN_FLAG_DEBUG_GATE if debug_gate else 0) | (SFFN_FLAG_SEPARATE if separate else 0)
+                      | (SFFN_FLAG_COOPERATIVE if cooperative else 0))
         ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         desc.W_gate, desc.A, desc.B = ptr(W_gate), ptr(A), ptr(B)
         desc.W_up, desc.W_down, desc.gate_bias = ptr(W_up), ptr(W_down), ptr(bias)

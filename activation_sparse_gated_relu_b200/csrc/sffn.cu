@@ -239,6 +239,7 @@ struct sffn_handle {
   int dec_maxr = 0, dec_smem = 0, dec_grid = 0;
   bool dec_ok = false;
   bool dec_pdl = true;           // the single launch also asks for programmatic dependent launch
+  unsigned last_attrs = 0;       // attributes of the last single launch (sffn_stats.launch_attrs)
   int dec_phantom = 0;           // test hook (sffn_debug_decode_waits)
   unsigned long long dec_wait_ns = SFFN_WAIT_LIMIT_NS;
   bool last_fused = false;     // the last forward was the single launch: its routing is the ovf flags
@@ -349,7 +350,7 @@ sffn_status validate(const sffn_desc* d) {
   if (d->rank > 0 && (d->dtype != SFFN_BF16 || d->rank % 64 != 0 || d->rank > 4096)) return SFFN_ERR_UNSUPPORTED;
   if (d->dtype == SFFN_FP32 && d->d_ff > 8192) return SFFN_ERR_UNSUPPORTED;
   if ((d->flags & SFFN_FLAG_DEBUG_GATE) && d->rank > 0) return SFFN_ERR_UNSUPPORTED;
-  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE)) return SFFN_ERR_INVALID_ARG;
+  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE | SFFN_FLAG_COOPERATIVE)) return SFFN_ERR_INVALID_ARG;
   return SFFN_OK;
 }
 
@@ -601,13 +602,17 @@ sffn_status sffn_destroy(sffn_handle* h) {
 }
 
 // The single decode launch's CTAs wait on one another (row lists, zeroed
-// slices of out), so all of them must be resident at once.  It is launched
-// cooperatively: when the grid cannot be co-resident (an SM-limited MPS
-// client, a green context, SMs held by another persistent kernel) the driver
-// fails the launch up front, or holds it until the whole grid fits, instead of
-// the resident CTAs waiting out their limits.  Programmatic dependent launch
-// is requested beside it; if the driver refuses the pair, the launch is
-// repeated, and later ones made, without it.
+// slices of out), so all of them must be resident at once: one CTA per SM,
+// checked against the occupancy at create time.  With SFFN_FLAG_COOPERATIVE
+// it is launched cooperatively, so that when the grid cannot be co-resident
+// (an SM-limited MPS client, a green context, SMs held by another persistent
+// kernel) the driver holds the launch until the whole grid fits or fails it
+// up front, instead of the resident CTAs waiting out their limits.  That
+// costs about 4 us per forward (the grid cannot start while the previous
+// forward's CTAs hold SMs), so it is not the default.  Programmatic
+// dependent launch is requested; if the driver refuses it beside the
+// cooperative attribute, the launch is repeated, and later ones made,
+// without it.
 static cudaError_t launch_decode(sffn_handle* h, const DecodeArgs& da, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(h->dec_grid);
@@ -616,9 +621,12 @@ static cudaError_t launch_decode(sffn_handle* h, const DecodeArgs& da, cudaStrea
   cfg.stream = st;
   cudaLaunchAttribute at[2];
   int n = 0;
-  at[n].id = cudaLaunchAttributeCooperative;
-  at[n].val.cooperative = 1;
-  ++n;
+  const bool coop = (h->desc.flags & SFFN_FLAG_COOPERATIVE) != 0;
+  if (coop) {
+    at[n].id = cudaLaunchAttributeCooperative;
+    at[n].val.cooperative = 1;
+    ++n;
+  }
   if (h->dec_pdl) {
     at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[n].val.programmaticStreamSerializationAllowed = 1;
@@ -627,9 +635,12 @@ static cudaError_t launch_decode(sffn_handle* h, const DecodeArgs& da, cudaStrea
   cfg.attrs = at;
   cfg.numAttrs = n;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode, da);
-  if (e == cudaSuccess) return e;
+  if (e == cudaSuccess) {
+    h->last_attrs = (coop ? 1u : 0u) | (h->dec_pdl ? 2u : 0u);
+    return e;
+  }
   cudaGetLastError();
-  if (h->dec_pdl && e != cudaErrorCooperativeLaunchTooLarge) {
+  if (coop && h->dec_pdl && e != cudaErrorCooperativeLaunchTooLarge) {
     h->dec_pdl = false;
     return launch_decode(h, da, st);
   }
@@ -1150,6 +1161,7 @@ sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st) {
   st->n_launches = h->last_launches;
   st->path = h->last_path;
   st->epoch = h->epoch;
+  st->launch_attrs = h->last_fused ? h->last_attrs : 0u;
   return SFFN_OK;
 }
 

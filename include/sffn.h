@@ -95,6 +95,8 @@ typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sff
 #define SFFN_FLAG_DEBUG_GATE 1u   /* keep the dense fp32 gate g[T][d_ff] of the last forward */
 #define SFFN_FLAG_SEPARATE 2u     /* T <= 8: separate gate, up x down and dense-channel launches
                                      instead of the single persistent launch (diagnostics, tests) */
+#define SFFN_FLAG_COOPERATIVE 4u  /* launch the single persistent forward with the cooperative
+                                     attribute (see sffn_forward) */
 
 typedef struct sffn_desc {
   int d_model;          /* d: multiple of 8, 8..4096 (ROWS path needs d <= 4096)   */
@@ -134,7 +136,20 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
  * flags and, on the single-launch path, the scheduler words that the CTAs
  * exchange.  A forward captured into a CUDA graph and replayed would reuse
  * its epoch and could read a previous replay's scheduler words, so stream
- * capture of sffn_forward is not supported. */
+ * capture of sffn_forward is not supported.
+ *
+ * The single persistent launch (T <= 8, ROWS path) has one CTA per SM and its
+ * CTAs wait on one another, so it needs all of them resident at once.  That
+ * holds when the forward has the GPU's SMs to itself or shares them with
+ * ordinary kernels; it need not hold for an MPS client limited to part of the
+ * SMs, a green context, or a concurrent persistent kernel that never yields
+ * its SMs.  There every wait is bounded: the forward gives up after 2 s,
+ * writes no valid out and records SFFN_ERR_TIMEOUT (sffn_read_status), and
+ * nothing hangs.  Callers in such settings set SFFN_FLAG_COOPERATIVE: the
+ * launch is then cooperative, so the driver holds it until the whole grid
+ * fits, or refuses it (SFFN_ERR_CUDA) when it never can.  It costs about
+ * 4 us per forward on B200, because a cooperative grid cannot start while
+ * the previous forward's CTAs still hold SMs. */
 sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void* cuda_stream);
 
 /* Same as sffn_forward but x and out are HOST buffers: copies x to the
@@ -207,6 +222,8 @@ typedef struct sffn_stats {
   int n_launches;
   int path;             /* the sffn_path actually taken (ROWS or TILES) */
   unsigned epoch;       /* overflow[t] == epoch marks the last forward's overflow tokens */
+  unsigned launch_attrs; /* the last single persistent launch: bit 0 cooperative, bit 1
+                            programmatic dependent launch (0 if none was made) */
 } sffn_stats;
 sffn_status sffn_get_stats(sffn_handle* h, void* cuda_stream, sffn_stats* st);
 

@@ -304,12 +304,13 @@ def test_decode_handle_holds_no_dense_channel_copies(decode_inputs):
         big.close()
 
 
-def test_decode_two_handles_concurrently_on_two_streams(decode_inputs):
-    # two handles' single launches issued on two streams at once: each grid
-    # is co-resident by its cooperative launch (the driver runs them one
-    # after the other when both cannot fit), and both match the oracle
-    ffn_a = make_ffn(decode_inputs, max_tokens=8)
-    ffn_b = make_ffn(decode_inputs, max_tokens=8)
+@pytest.mark.parametrize("cooperative", [False, True])
+def test_decode_two_handles_concurrently_on_two_streams(decode_inputs, cooperative):
+    # two handles' single launches issued on two streams at once, with and
+    # without the cooperative attribute: both grids run whole (one after the
+    # other: each fills every SM) and both match the oracle
+    ffn_a = make_ffn(decode_inputs, max_tokens=8, cooperative=cooperative)
+    ffn_b = make_ffn(decode_inputs, max_tokens=8, cooperative=cooperative)
     sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
     xa, xb = to_dev(decode_inputs.x[:8]), to_dev(decode_inputs.x[5:8])
     oa = torch.full((8, ffn_a.d_model), float("nan"), dtype=torch.float32, device="cuda")
@@ -322,6 +323,7 @@ def test_decode_two_handles_concurrently_on_two_streams(decode_inputs):
         torch.cuda.synchronize()
         assert ffn_a.read_status(sa.cuda_stream) == SFFN_OK
         assert ffn_b.read_status(sb.cuda_stream) == SFFN_OK
+        assert ffn_a.stats(sa.cuda_stream).launch_attrs & 1 == (1 if cooperative else 0)
         ra = oracle.forward_inputs(decode_inputs, T=8)
         assert rel_err(oa.double().cpu().numpy(), ra.y) <= 2e-3
         assert rel_err(ob.double().cpu().numpy(), ra.y[5:8]) <= 2e-3
