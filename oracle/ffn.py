@@ -158,6 +158,51 @@ def keep_topk(s: np.ndarray, k: int) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
+# WINA variants ([WINA] sections 3.1 to 3.3)
+# ----------------------------------------------------------------------------
+def wina_full_h_scores(a: np.ndarray, u: np.ndarray, norms: np.ndarray) -> np.ndarray:
+    """s[t, j] = |a[t, j]·u[t, j]|·n_j: the score of section 3.1 with the
+    hidden value taken as the full gated product h = sigma(g)·u (unrounded),
+    which needs the up projection of every neuron."""
+    return np.abs(a * u) * norms[None, :]
+
+
+def input_col_norms(W_gate: np.ndarray, W_up: np.ndarray) -> np.ndarray:
+    """c_i = ||column i of the stacked [W_gate; W_up]||_2 in fp64, rounded to
+    fp32: x feeds the gate and the up projection, so the layer that consumes
+    x_i is the stacked [2 d_ff][d] matrix, and its column i is the "weight
+    column" of section 3.1 for input coordinate i."""
+    return round_fp32(np.sqrt(np.sum(W_gate * W_gate, axis=0) + np.sum(W_up * W_up, axis=0)))
+
+
+def input_scores(x: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """s[t, i] = |x[t, i]|·c_i rounded once to fp32 (the precision the
+    selection is decided in on both sides: x and c are exact in fp64, so the
+    rounded product is unique)."""
+    return round_fp32(np.abs(x) * c[None, :])
+
+
+def select_input(x: np.ndarray, keep_in: np.ndarray) -> np.ndarray:
+    """x with the input coordinates that are not kept set to zero."""
+    return np.where(keep_in, x, 0.0)
+
+
+def orthogonal_basis(W_gate: np.ndarray, W_up: np.ndarray) -> np.ndarray:
+    """V of the SVD [W_gate; W_up] = U·S·V^T (section 3.3: the weight is
+    right-multiplied by V, which makes its columns orthogonal, U·S).  A
+    library SVD is the step."""
+    _, _, Vt = np.linalg.svd(np.concatenate([W_gate, W_up], axis=0), full_matrices=False)
+    return Vt.T.copy()
+
+
+def rotate(M: np.ndarray, V: np.ndarray, dtype: str) -> np.ndarray:
+    """M·V rounded to the operand dtype: a neuron-major weight [n][d] times V
+    gives the orthogonalised weight; an activation batch [T][d] times V gives
+    the rotated input V^T x_t of each token (so that W V V^T x = W x)."""
+    return round_operand(M @ V, dtype)
+
+
+# ----------------------------------------------------------------------------
 # TwELL ([TwELL] "TwELL 減掉轉換開銷")
 # ----------------------------------------------------------------------------
 def twell_pack(keep: np.ndarray, v: np.ndarray, C: int, tile: int = TILE):
@@ -272,20 +317,45 @@ class OracleResult:
     scores: Optional[np.ndarray] = None
     norms: Optional[np.ndarray] = None
     z: Optional[np.ndarray] = None
+    x_used: Optional[np.ndarray] = None   # [T][d] the input both projections saw
+    x_keep: Optional[np.ndarray] = None   # [T][d] input coordinates kept (input-side WINA)
 
 
 def forward(x: np.ndarray, W_up: np.ndarray, W_down: np.ndarray, *,
             W_gate: Optional[np.ndarray] = None, A: Optional[np.ndarray] = None,
             B: Optional[np.ndarray] = None, bias: Optional[np.ndarray] = None,
             dtype: str = "bf16", mode: str = "relu_threshold", act: str = "relu",
-            threshold: float = 0.0, k: int = 0, C: int = 32) -> OracleResult:
+            threshold: float = 0.0, k: int = 0, C: int = 32,
+            input_k: Optional[int] = None, V: Optional[np.ndarray] = None) -> OracleResult:
     """The activation-sparse gated FFN forward, step by step, in fp64.
 
     All array arguments are float64 decodes of the operands (exact).  Steps:
-    gate -> activation -> stored value -> selection -> TwELL pack/overflow ->
-    up on kept rows -> product -> down on kept rows.
+    [rotation] -> [input selection] -> gate -> activation -> stored value ->
+    selection -> TwELL pack/overflow -> up on kept rows -> product -> down on
+    kept rows.
+
+    WINA variants ([WINA] sections 3.1 to 3.3): ``mode="wina_full_h"`` scores
+    the full gated product |sigma(g)·u| instead of |sigma(g)|; ``input_k``
+    keeps, per token, the input_k input coordinates with the largest
+    |x_i|·c_i (c = column norms of [W_gate; W_up]) and zeroes the others
+    before both projections (dense gate only); ``V`` orthogonalises: the gate
+    and up weights become round(W·V) and each token's input round(x·V), which
+    leaves W·x unchanged up to those roundings.
     """
     x = np.asarray(x, dtype=np.float64)
+    x_in = None
+    if V is not None:
+        if W_gate is None:
+            raise ValueError("the orthogonalisation needs the dense gate")
+        W_gate = rotate(W_gate, V, dtype)
+        W_up = rotate(W_up, V, dtype)
+        x = rotate(x, V, dtype)
+    if input_k is not None:
+        if W_gate is None:
+            raise ValueError("input-side selection needs the dense gate")
+        c = input_col_norms(W_gate, W_up)
+        x_in = keep_topk(input_scores(x, c), input_k)
+        x = select_input(x, x_in)
     z = None
     if W_gate is not None:
         g = gate_dense(x, W_gate, bias)
@@ -306,12 +376,22 @@ def forward(x: np.ndarray, W_up: np.ndarray, W_down: np.ndarray, *,
         # device's float32 rounding of the activation and of the product
         slope = np.abs(_silu_slope(g)) if act == "silu" else 1.0
         band = (slope * band + np.ldexp(np.abs(a), -21)) * norms[None, :]
+    elif mode == "wina_full_h":
+        norms = wina_norms(W_down)
+        u_all = x @ W_up.T
+        scores = wina_full_h_scores(a, u_all, norms)
+        keep = keep_topk(scores, k)
+        # the score moves with the device's gate error (through sigma'), its
+        # up-projection error (the same band on W_up) and fp32 roundings
+        slope = np.abs(_silu_slope(g)) if act == "silu" else 1.0
+        band = (slope * band * np.abs(u_all) + np.abs(a) * gate_band(x, W_up)
+                + np.ldexp(np.abs(a * u_all), -20)) * norms[None, :]
     else:
         raise ValueError(mode)
     count, idx, val, overflow = twell_pack(keep, v, C)
     y = sparse_up_down(x, W_up, W_down, keep, v)
     return OracleResult(y, g, a, v, keep, count, idx, val, overflow, band,
-                        scores=scores, norms=norms, z=z)
+                        scores=scores, norms=norms, z=z, x_used=x, x_keep=x_in)
 
 
 def _silu_slope(g: np.ndarray) -> np.ndarray:
@@ -332,4 +412,5 @@ def forward_inputs(inp, T: Optional[int] = None) -> OracleResult:
     return forward(x, f64(inp.W_up), f64(inp.W_down), W_gate=f64(inp.W_gate),
                    A=f64(inp.A), B=f64(inp.B), bias=f64(inp.bias), dtype=wl.dtype,
                    mode=wl.mode, act=wl.act, threshold=wl.threshold, k=wl.k,
-                   C=wl.tile_capacity)
+                   C=wl.tile_capacity, input_k=getattr(wl, "input_k", None),
+                   V=f64(getattr(inp, "V", None)))
