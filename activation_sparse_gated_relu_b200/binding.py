@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, "libsffn.so")
 SFFN_OK, SFFN_ERR_INVALID_ARG, SFFN_ERR_UNSUPPORTED, SFFN_ERR_ALLOC, SFFN_ERR_CUDA, \
     SFFN_ERR_TIMEOUT, SFFN_ERR_DEVICE, SFFN_ERR_NO_DEVICE = range(8)
 SFFN_BF16, SFFN_FP32 = 0, 1
-SFFN_MODE_RELU_THRESHOLD, SFFN_MODE_WINA_TOPK = 0, 1
+SFFN_MODE_RELU_THRESHOLD, SFFN_MODE_WINA_TOPK, SFFN_MODE_WINA_FULL_H = 0, 1, 2
 SFFN_ACT_RELU, SFFN_ACT_SILU = 0, 1
 SFFN_PATH_AUTO, SFFN_PATH_ROWS, SFFN_PATH_TILES = 0, 1, 2
 SFFN_FLAG_DEBUG_GATE = 1
@@ -33,6 +33,7 @@ class sffn_desc(ctypes.Structure):
         ("tile_capacity", ctypes.c_int), ("path", ctypes.c_int), ("flags", ctypes.c_uint),
         ("W_gate", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
         ("W_up", ctypes.c_void_p), ("W_down", ctypes.c_void_p), ("gate_bias", ctypes.c_void_p),
+        ("input_k", ctypes.c_int), ("V", ctypes.c_void_p),
     ]
 
 
@@ -198,7 +199,8 @@ def _check_tensor(t, name: str, dtype, shape, cuda: bool) -> None:
 
 
 _DTYPE = {"bf16": SFFN_BF16, "fp32": SFFN_FP32}
-_MODE = {"relu_threshold": SFFN_MODE_RELU_THRESHOLD, "wina_topk": SFFN_MODE_WINA_TOPK}
+_MODE = {"relu_threshold": SFFN_MODE_RELU_THRESHOLD, "wina_topk": SFFN_MODE_WINA_TOPK,
+         "wina_full_h": SFFN_MODE_WINA_FULL_H}
 _ACT = {"relu": SFFN_ACT_RELU, "silu": SFFN_ACT_SILU}
 _PATH = {"auto": SFFN_PATH_AUTO, "rows": SFFN_PATH_ROWS, "tiles": SFFN_PATH_TILES}
 
@@ -214,10 +216,10 @@ class SparseFFN:
                  mode: str = "relu_threshold", act: str = "relu", threshold: float = 0.0,
                  k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
                  debug_gate: bool = False, separate: bool = False, cooperative: bool = False,
-                 stream: Optional[int] = None):
+                 input_k: int = 0, V=None, stream: Optional[int] = None):
         import torch
         self.h = None
-        self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias) if t is not None]
+        self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias, V) if t is not None]
         dt = W_up.dtype
         if dt not in (torch.bfloat16, torch.float32):
             raise TypeError("operands must be bf16 or fp32")
@@ -239,6 +241,8 @@ class SparseFFN:
             _check_tensor(B, "B", dt, (A.shape[1], F), True)
         if bias is not None:
             _check_tensor(bias, "bias", torch.float32, (F,), True)
+        if V is not None:
+            _check_tensor(V, "V", dt, (d, d), True)
         self.d_model, self.d_ff, self.max_tokens = d, F, max_tokens
         desc = sffn_desc()
         desc.d_model, desc.d_ff, desc.max_tokens = d, F, max_tokens
@@ -255,6 +259,8 @@ class SparseFFN:
         ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         desc.W_gate, desc.A, desc.B = ptr(W_gate), ptr(A), ptr(B)
         desc.W_up, desc.W_down, desc.gate_bias = ptr(W_up), ptr(W_down), ptr(bias)
+        desc.input_k = int(input_k or 0)
+        desc.V = ptr(V)
         self.desc = desc
         self.h = sffn_create(desc, self._stream(stream))
 

@@ -251,6 +251,99 @@ struct EpiWina {
   }
 };
 
+// ------------------------------------------------------- WINA, full-h score
+// [WINA] section 3.1 with the hidden value taken as the whole gated product:
+// the tile kernel runs two phases into two accumulators, g = W_gate·x (col 0)
+// and u = W_up·x (col BN), for every neuron of the tile.  Per (token, neuron):
+// a = sigma(g + b), v = round(a) (the TwELL value), s = |a·u|·n_j (the score
+// of the unrounded product) and h = v·u (fp32, what the down projection adds
+// for a kept neuron).
+struct WinaFullHParams {
+  const float* bias;
+  int act, T, F;
+  const float* norms;
+  __nv_bfloat16* vdense;  // [T][F]
+  float* scores;          // [T][F]
+  float* hfull;           // [T][F]
+};
+
+struct EpiWinaFullH {
+  static constexpr int N_ACC = 2;
+  using Params = WinaFullHParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int j = m0 + etid;
+    const float b = o.bias ? o.bias[j] : 0.0f;
+    const float n = o.norms[j];
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.T) break;
+      float g[16], u[16];
+      tmem_ld16(tmem + c, g);
+      tmem_ld16(tmem + BN + c, u);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = n0 + c + i;
+        if (t < o.T) {
+          const float a = act_fn(g[i] + b, o.act);
+          const __nv_bfloat16 v = __float2bfloat16_rn(a);
+          const size_t off = (size_t)t * o.F + j;
+          o.vdense[off] = v;
+          o.scores[off] = fabsf(a * u[i]) * n;
+          o.hfull[off] = __bfloat162float(v) * u[i];
+        }
+      }
+    }
+  }
+};
+
+// -------------------------------------------------- plain bf16 store of D
+// D[128 rows][BN cols] rounded to bf16 and stored row-major: out[r][c] at
+// r·ld + c (transpose = 0) or out[c][r] at c·ld + r (transpose = 1), rows
+// below `rows` and columns below `cols` only.  Used for the orthogonalising
+// rotations ([WINA] section 3.3): W' = W·V (rows = neurons) and x' = x·V
+// (computed as V^T·x^T, rows = input coordinates, stored transposed).
+struct StoreParams {
+  __nv_bfloat16* out;
+  long long ld;
+  int rows, cols, transpose;
+};
+
+struct EpiStoreBf16 {
+  static constexpr int N_ACC = 1;
+  using Params = StoreParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int r = m0 + etid;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.cols) break;
+      float v[16];
+      tmem_ld16(tmem + c, v);
+      if (r < o.rows) {
+        if (o.transpose) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n0 + c + i < o.cols) o.out[(size_t)(n0 + c + i) * o.ld + r] = __float2bfloat16_rn(v[i]);
+        } else {
+          __align__(16) __nv_bfloat16 pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = __float2bfloat16_rn(v[i]);
+          __nv_bfloat16* dst = o.out + (size_t)r * o.ld + n0 + c;
+          if (n0 + c + 16 <= o.cols && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+            reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(pk)[0];
+            reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(pk)[1];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n0 + c + i < o.cols) dst[i] = pk[i];
+          }
+        }
+      }
+    }
+  }
+};
+
 // ------------------------------------------------------- low-rank gate: z
 // z = round_bf16(x·A).  The tile's rows are rank coordinates r, its columns
 // tokens.  With a split K every CTA stores its fp32 partial in its split's

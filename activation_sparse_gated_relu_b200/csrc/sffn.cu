@@ -46,10 +46,10 @@ namespace {
 constexpr int kNumSMsFallback = 148;
 constexpr int kMaxMarks = 12;
 enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
-                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_COUNT };
+                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_ROTATE_X, L_INPUT_SELECT, L_COUNT };
 const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
                                           "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
-                                          "fallback_f32", "decode_fused"};
+                                          "fallback_f32", "decode_fused", "rotate_x", "input_select"};
 constexpr int kMaxTokensLimit = 16384;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -191,6 +191,10 @@ struct sffn_handle {
   int dev = 0, n_sm = kNumSMsFallback;
   int d = 0, F = 0, P = 0, R = 0, C = 0, maxT = 0, esize = 2;
   bool f32 = false, wina = false, lowrank = false;
+  bool fullh = false;            // WINA with the full-h score (wina is set too)
+  // effective gate and up weights: the caller's, or their orthogonalised copies
+  const __nv_bfloat16* Wg = nullptr;
+  const __nv_bfloat16* Wu = nullptr;
   uint32_t epoch = 0;
   // workspace
   int16_t* count = nullptr;
@@ -217,6 +221,15 @@ struct sffn_handle {
   uint32_t* status = nullptr;
   void* xstage = nullptr;
   float* ostage = nullptr;
+  float* hfull = nullptr;        // full-h WINA: h = v·u [T][F]
+  float* colnorm = nullptr;      // input-side WINA: column norms of [W_gate; W_up] [d]
+  double* colacc = nullptr;      // their fp64 sums (create time)
+  __nv_bfloat16* xsel = nullptr; // input-side WINA: the selected x [T][d]
+  __nv_bfloat16* Vt = nullptr;   // orthogonalisation: V^T [d][d]
+  __nv_bfloat16* Wg_rot = nullptr;  // W_gate·V [F][d]
+  __nv_bfloat16* Wu_rot = nullptr;  // W_up·V [F][d]
+  __nv_bfloat16* xrot = nullptr;    // x·V [T][d]
+  CUtensorMap tmVt;              // V^T rows as the A operand of x·V
   void* arena = nullptr;         // the one device allocation all of the above live in
   size_t arena_bytes = 0;
   bool dense_bufs = false;       // xo, h_hi, h_lo and W_down^T exist (paths other than the single launch)
@@ -328,14 +341,17 @@ sffn_status validate(const sffn_desc* d) {
   if (!d) return SFFN_ERR_INVALID_ARG;
   if (d->d_model <= 0 || d->d_ff <= 0 || d->max_tokens <= 0 || d->rank < 0) return SFFN_ERR_INVALID_ARG;
   if (d->dtype != SFFN_BF16 && d->dtype != SFFN_FP32) return SFFN_ERR_INVALID_ARG;
-  if (d->mode != SFFN_MODE_RELU_THRESHOLD && d->mode != SFFN_MODE_WINA_TOPK) return SFFN_ERR_INVALID_ARG;
+  if (d->mode != SFFN_MODE_RELU_THRESHOLD && d->mode != SFFN_MODE_WINA_TOPK && d->mode != SFFN_MODE_WINA_FULL_H)
+    return SFFN_ERR_INVALID_ARG;
   if (d->act != SFFN_ACT_RELU && d->act != SFFN_ACT_SILU) return SFFN_ERR_INVALID_ARG;
   if (d->path < SFFN_PATH_AUTO || d->path > SFFN_PATH_TILES) return SFFN_ERR_INVALID_ARG;
   const int C = d->tile_capacity;
   if (C != 8 && C != 16 && C != 32 && C != 64 && C != 128) return SFFN_ERR_INVALID_ARG;
   if (d->mode == SFFN_MODE_RELU_THRESHOLD && (!(d->threshold >= 0.0f) || !std::isfinite(d->threshold)))
     return SFFN_ERR_INVALID_ARG;
-  if (d->mode == SFFN_MODE_WINA_TOPK && (d->k < 0 || d->k > d->d_ff)) return SFFN_ERR_INVALID_ARG;
+  if (d->mode != SFFN_MODE_RELU_THRESHOLD && (d->k < 0 || d->k > d->d_ff)) return SFFN_ERR_INVALID_ARG;
+  if (d->input_k < 0 || d->input_k > d->d_model) return SFFN_ERR_INVALID_ARG;
+  if (d->V && !aligned16(d->V)) return SFFN_ERR_INVALID_ARG;
   if (!d->W_up || !d->W_down) return SFFN_ERR_INVALID_ARG;
   if (d->rank == 0 && (!d->W_gate || d->A || d->B)) return SFFN_ERR_INVALID_ARG;
   if (d->rank > 0 && (d->W_gate || !d->A || !d->B)) return SFFN_ERR_INVALID_ARG;
@@ -346,7 +362,11 @@ sffn_status validate(const sffn_desc* d) {
   if (d->d_ff % 128 != 0 || d->d_ff > 32767) return SFFN_ERR_UNSUPPORTED;
   if (d->max_tokens > kMaxTokensLimit) return SFFN_ERR_UNSUPPORTED;
   if (d->d_model > 4096) return SFFN_ERR_UNSUPPORTED;
-  if (d->mode == SFFN_MODE_WINA_TOPK && C != 128) return SFFN_ERR_UNSUPPORTED;
+  if (d->mode != SFFN_MODE_RELU_THRESHOLD && C != 128) return SFFN_ERR_UNSUPPORTED;
+  // the WINA variants of the full-h score, the input side and the
+  // orthogonalisation: dense gate, bf16 operands
+  if ((d->mode == SFFN_MODE_WINA_FULL_H || d->input_k > 0 || d->V) && (d->rank > 0 || d->dtype != SFFN_BF16))
+    return SFFN_ERR_UNSUPPORTED;
   if (d->rank > 0 && (d->dtype != SFFN_BF16 || d->rank % 64 != 0 || d->rank > 4096)) return SFFN_ERR_UNSUPPORTED;
   if (d->dtype == SFFN_FP32 && d->d_ff > 8192) return SFFN_ERR_UNSUPPORTED;
   if ((d->flags & SFFN_FLAG_DEBUG_GATE) && d->rank > 0) return SFFN_ERR_UNSUPPORTED;
@@ -404,7 +424,10 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   h->maxT = desc->max_tokens;
   h->f32 = desc->dtype == SFFN_FP32;
   h->esize = h->f32 ? 4 : 2;
-  h->wina = desc->mode == SFFN_MODE_WINA_TOPK;
+  h->wina = desc->mode == SFFN_MODE_WINA_TOPK || desc->mode == SFFN_MODE_WINA_FULL_H;
+  h->fullh = desc->mode == SFFN_MODE_WINA_FULL_H;
+  h->Wg = static_cast<const __nv_bfloat16*>(desc->W_gate);
+  h->Wu = static_cast<const __nv_bfloat16*>(desc->W_up);
   h->lowrank = desc->rank > 0;
   const size_t T = (size_t)h->maxT, d = (size_t)h->d, F = (size_t)h->F, P = (size_t)h->P, C = (size_t)h->C;
   const size_t R = (size_t)h->R;
@@ -422,6 +445,8 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     e = e ? e : set_tc_attrs<EpiFallbackH>();
     e = e ? e : set_tc_attrs<EpiTwellH>();
     e = e ? e : set_tc_attrs<EpiDownOut>();
+    e = e ? e : set_tc_attrs<EpiWinaFullH>();
+    e = e ? e : set_tc_attrs<EpiStoreBf16>();
     // fused up x down: ring slots and list capacity from the shared memory budget
     int lcap = 512, ns = RW_NSMAX;
     auto fits = [&](int l, int n) { return RowsSmem::make(h->P, l, h->d, n).total <= max_smem; };
@@ -465,6 +490,9 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     const int tk_smem = topk_smem_bytes((int)F, (int)P, (int)C);
     e = cudaFuncSetAttribute(k_wina_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, tk_smem);
   }
+  if (!e && desc->input_k > 0)
+    e = cudaFuncSetAttribute(k_input_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             input_select_smem_bytes((int)d));
   if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, router_smem_bytes((int)T));
   if (!e && h->f32) {
     e = cudaFuncSetAttribute(k_rows_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -507,6 +535,18 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       a.take(&h->scores, T * F * 4);
       a.take(&h->vdense, T * F * h->esize);
       a.take(&h->norms, F * 4);
+    }
+    if (h->fullh) a.take(&h->hfull, T * F * 4);
+    if (desc->input_k > 0) {
+      a.take(&h->colnorm, d * 4);
+      a.take(&h->colacc, d * 8);
+      a.take(&h->xsel, T * d * 2);
+    }
+    if (desc->V) {
+      a.take(&h->Vt, d * d * 2);
+      a.take(&h->Wg_rot, F * d * 2);
+      a.take(&h->Wu_rot, F * d * 2);
+      a.take(&h->xrot, T * d * 2);
     }
     if (h->lowrank) {
       a.take(&h->z, T * R * 2);
@@ -567,11 +607,49 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
                                                              (int)F, (int)d, h->norms);
     e = cudaGetLastError();
   }
+  // [WINA] section 3.3: the gate and up weights right-multiplied by V,
+  // rounded to bf16 (D[neuron][n] = sum_k W[neuron][k]·V^T[n][k] on the
+  // tile kernel); the forwards then use these copies
+  if (!e && desc->V) {
+    k_transpose_bf16<<<dim3(cdiv(d, 32), cdiv(d, 32)), tb, 0, st>>>(static_cast<const __nv_bfloat16*>(desc->V),
+                                                                    h->Vt, (int)d, (int)d);
+    e = cudaGetLastError();
+    CUtensorMap mW, mV;
+    const int BNr = 256;
+    if (!e && !make_map(&mV, h->Vt, d, d, BNr)) e = cudaErrorInvalidValue;
+    for (int which = 0; which < 2 && !e; ++which) {
+      const void* Wsrc = which == 0 ? desc->W_gate : desc->W_up;
+      __nv_bfloat16* Wdst = which == 0 ? h->Wg_rot : h->Wu_rot;
+      if (!make_map(&mW, Wsrc, d, F, 128)) {
+        e = cudaErrorInvalidValue;
+        break;
+      }
+      TcArgs ra{};
+      ra.n_phase = 1;
+      ra.kb_total[0] = cdiv(d, 64);
+      ra.n_rows = (int)d;
+      ra.status = h->status;
+      StoreParams sp{Wdst, (long long)d, (int)F, (int)d, 0};
+      e = launch_tc<EpiStoreBf16>(BNr, dim3(P, cdiv(d, BNr), 1), st, mW, mV, mW, mV, ra, sp);
+    }
+    h->Wg = h->Wg_rot;
+    h->Wu = h->Wu_rot;
+  }
+  // input-side WINA: column norms of the (orthogonalised) [W_gate; W_up]
+  if (!e && desc->input_k > 0) {
+    e = cudaMemsetAsync(h->colacc, 0, d * 8, st);
+    if (!e) {
+      k_col_sumsq<<<dim3(cdiv(d, 256), 64), 256, 0, st>>>(h->Wg, h->Wu, (int)F, (int)d, h->colacc);
+      k_col_norms_finish<<<cdiv(d, 256), 256, 0, st>>>(h->colacc, (int)d, h->colnorm);
+      e = cudaGetLastError();
+    }
+  }
   // A-operand tensor maps
   if (!e && !h->f32) {
     bool mok = true;
-    if (!h->lowrank) mok = mok && make_map(&h->tmWgate, desc->W_gate, h->d, h->F, 128);
-    mok = mok && make_map(&h->tmWup, desc->W_up, h->d, h->F, 128);
+    if (!h->lowrank) mok = mok && make_map(&h->tmWgate, h->Wg, h->d, h->F, 128);
+    mok = mok && make_map(&h->tmWup, h->Wu, h->d, h->F, 128);
+    if (h->Vt) mok = mok && make_map(&h->tmVt, h->Vt, h->d, h->d, 128);
     if (h->WdT) mok = mok && make_map(&h->tmWdT, h->WdT, h->F, h->d, 128);
     if (h->lowrank) {
       mok = mok && make_map(&h->tmAt, h->At, h->d, h->R, 128);
@@ -654,6 +732,35 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   const uint32_t epoch = h->epoch;
   const int BN = pick_bn(T);
   const int ntile_tok = cdiv(T, BN);
+
+  // [WINA] section 3.3: each token's input rotated by the same V as the
+  // weights, x' = bf16(x·V), computed as V^T·x^T on the tile kernel and
+  // stored transposed
+  if (h->Vt) {
+    CUtensorMap mx0;
+    if (!make_map(&mx0, x, d, T, BN)) return SFFN_ERR_CUDA;
+    TcArgs ra{};
+    ra.n_phase = 1;
+    ra.kb_total[0] = cdiv(d, 64);
+    ra.n_rows = T;
+    ra.status = h->status;
+    StoreParams sp{h->xrot, (long long)d, d, T, 1};
+    tmark(h, st, L_ROTATE_X);
+    if (launch_tc<EpiStoreBf16>(BN, dim3(cdiv(d, 128), ntile_tok, 1), st, h->tmVt, mx0, h->tmVt, mx0, ra, sp))
+      return SFFN_ERR_CUDA;
+    ++launches;
+    x = h->xrot;
+  }
+  // [WINA] section 3.1 on the input side: keep the input_k coordinates of
+  // largest |x_i|·c_i per token, zero the rest; both projections see the result
+  if (h->xsel) {
+    InputSelectArgs ia{static_cast<const __nv_bfloat16*>(x), h->colnorm, h->xsel, T, d, D.input_k};
+    tmark(h, st, L_INPUT_SELECT);
+    if (launch_pdl(k_input_select, dim3(T), dim3(1024), (size_t)input_select_smem_bytes(d), st, 1, ia))
+      return SFFN_ERR_CUDA;
+    ++launches;
+    x = h->xsel;
+  }
   int path = D.path;
   if (path == SFFN_PATH_AUTO) path = (h->rows_ok && (T <= 8 || T > 256)) ? SFFN_PATH_ROWS : SFFN_PATH_TILES;
   if (h->wina) path = SFFN_PATH_TILES;  // the top-k kernel writes no per-token keep masks
@@ -693,8 +800,8 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   if (rows && T <= 8 && h->dec_ok && !(D.flags & SFFN_FLAG_SEPARATE)) {
     DecodeArgs da{};
     da.x = static_cast<const __nv_bfloat16*>(x);
-    da.W_gate = static_cast<const __nv_bfloat16*>(D.W_gate);
-    da.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
+    da.W_gate = h->Wg;
+    da.W_up = h->Wu;
     da.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
     da.tw = tw;
     da.gstage = h->gstage;
@@ -710,7 +817,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     tmark(h, st, L_DECODE);
     if (launch_decode(h, da, st)) return SFFN_ERR_CUDA;
     h->last_path = SFFN_PATH_ROWS;
-    h->last_launches = 1;
+    h->last_launches = launches + 1;
     h->last_fused = true;
     return SFFN_OK;
   }
@@ -757,12 +864,27 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     ga.zero_n4 = (long long)T * d / 4;
   }
   if (h->wina) {
-    WinaParams wp{D.gate_bias, D.act, T, F, h->norms, h->vdense, 0, h->scores};
     tmark(h, st, L_GATE);
-    e = launch_tc<EpiWina>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, wp);
+    if (h->fullh) {
+      // g and u of every neuron in one tile kernel (two accumulators)
+      TcArgs fa = ga;
+      fa.n_phase = 2;
+      fa.kb_total[1] = cdiv(d, 64);
+      WinaFullHParams fp{D.gate_bias, D.act, T, F, h->norms, static_cast<__nv_bfloat16*>(h->vdense), h->scores,
+                         h->hfull};
+      e = launch_tc<EpiWinaFullH>(BN, dim3(P, ntile_tok, 1), st, h->tmWgate, mx, h->tmWup, mx, fa, fp);
+    } else {
+      WinaParams wp{D.gate_bias, D.act, T, F, h->norms, h->vdense, 0, h->scores};
+      e = launch_tc<EpiWina>(BN, dim3(P, ntile_tok, 1), st, *gateA, *gateB, *gateA, *gateB, ga, wp);
+    }
     ++launches;
     if (e) return SFFN_ERR_CUDA;
     TopkArgs ta{h->scores, h->vdense, 0, T, F, D.k, P, h->C, h->count, h->idx, h->val, h->ovf, epoch};
+    if (h->fullh) {  // the top-k also writes the down projection's masked h rows
+      ta.hfull = h->hfull;
+      ta.h_hi = h->h_hi;
+      ta.h_lo = h->h_lo;
+    }
     tmark(h, st, L_WINA_TOPK);
     ++launches;
     if (launch_pdl(k_wina_topk, dim3(T), dim3(1024), (size_t)topk_smem_bytes(F, P, h->C), st, 1, ta))
@@ -773,7 +895,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
       // up to 8 tokens: stream whole W_gate rows over every SM
       GateRowsArgs gr{};
       gr.x = static_cast<const __nv_bfloat16*>(x);
-      gr.W_gate = static_cast<const __nv_bfloat16*>(D.W_gate);
+      gr.W_gate = h->Wg;
       gr.tw = tw;
       gr.gstage = h->gstage;
       gr.tick = h->gtick;
@@ -799,7 +921,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   if (rows) {
     RowsArgs rw{};
     rw.x = static_cast<const __nv_bfloat16*>(x);
-    rw.W_up = static_cast<const __nv_bfloat16*>(D.W_up);
+    rw.W_up = h->Wu;
     rw.W_down = static_cast<const __nv_bfloat16*>(D.W_down);
     rw.count = h->count;
     rw.idx = h->idx;
@@ -828,7 +950,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     ++launches;
     if (launch_pdl(k_rows, dim3(rows_split, nblk, 1), dim3(RW_THREADS), (size_t)h->rows_smem, st, 1, rw))
       return SFFN_ERR_CUDA;
-  } else {
+  } else if (!h->fullh) {  // (full-h: the top-k kernel wrote h)
     TcArgs ua{};
     ua.n_phase = 1;
     ua.kb_total[0] = cdiv(d, 64);

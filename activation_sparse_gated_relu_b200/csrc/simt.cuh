@@ -124,11 +124,74 @@ struct TopkArgs {
   void* val;
   uint32_t* ovf;
   uint32_t epoch;
+  const float* hfull;    // full-h variant: [T][F] h = v·u; the kept entries go to
+  __nv_bfloat16* h_hi;   // h_hi/h_lo [T][F] (hi + lo split), the others are zeroed
+  __nv_bfloat16* h_lo;   // (null: TwELL only)
 };
 
 // keys, histograms, tie prefix (padded to 16 bytes), per-warp staged records
 __host__ __device__ inline int topk_smem_bytes(int F, int n_tiles, int C) {
   return F * 4 + 32 * 256 * 4 + ((n_tiles + 3) & ~3) * 4 + 32 * 3 * C * 2;
+}
+
+// The k-th largest of n non-negative fp32 bit patterns in shared memory, by a
+// 4-pass 8-bit radix select (1024 threads, per-warp histograms hist[32][256]).
+// Returns K, the k-th largest pattern, and *rem, how many entries equal to K
+// belong to the k largest (ties are then broken by the caller, by index).
+// Needs 0 < k < n.
+__device__ __forceinline__ uint32_t radix_select_kth(const uint32_t* keys, int n, int k, uint32_t* hist,
+                                                     int* wtot, int* wpre, uint32_t* sel, int* rem_out) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t prefix = 0, mask = 0;
+  int rem = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int e = tid; e < 32 * 256; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    for (int j = tid; j < n; j += blockDim.x) {
+      const uint32_t key = keys[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key >> shift) & 255u)], 1u);
+    }
+    __syncthreads();
+    // bins in descending order: four threads per bin (thread group g = bin
+    // 255 - g) add the 32 per-warp counts, then a scan over the groups gives
+    // every bin the number of keys in higher bins
+    const int g = tid >> 2, part = tid & 3, bin = 255 - g;
+    int c = 0;
+    for (int w2 = part; w2 < 32; w2 += 4) c += (int)hist[w2 * 256 + bin];
+    c += __shfl_xor_sync(0xFFFFFFFFu, c, 1);
+    c += __shfl_xor_sync(0xFFFFFFFFu, c, 2);
+    int inc = c;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      const int nn = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+      if (lane >= o) inc += nn;
+    }
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = wtot[lane];
+      int vi = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nn = __shfl_up_sync(0xFFFFFFFFu, vi, o);
+        if (lane >= o) vi += nn;
+      }
+      wpre[lane] = vi - v;
+    }
+    __syncthreads();
+    const int ex = wpre[warp] + inc - c;
+    if (part == 0 && ex < rem && ex + c >= rem) {
+      sel[0] = (uint32_t)bin;
+      sel[1] = (uint32_t)(rem - ex);
+    }
+    __syncthreads();
+    prefix |= sel[0] << shift;
+    mask |= 255u << shift;
+    rem = (int)sel[1];
+    __syncthreads();
+  }
+  *rem_out = rem;
+  return prefix;
 }
 
 __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
@@ -148,55 +211,11 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
     *reinterpret_cast<uint4*>(&tk_keys[j]) = *reinterpret_cast<const uint4*>(&sc[j]);
   const int k = a.k;
   const bool keep_all = k >= a.F, keep_none = k <= 0;
-  uint32_t prefix = 0, mask = 0;
   int rem = k;
+  uint32_t prefix = 0;
   if (!keep_all && !keep_none) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int e = tid; e < 32 * 256; e += blockDim.x) hist[e] = 0;
-      __syncthreads();
-      for (int j = tid; j < a.F; j += blockDim.x) {
-        const uint32_t key = tk_keys[j];
-        if ((key & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key >> shift) & 255u)], 1u);
-      }
-      __syncthreads();
-      // bins in descending order: four threads per bin (thread group g = bin
-      // 255 - g) add the 32 per-warp counts, then a scan over the groups gives
-      // every bin the number of keys in higher bins
-      const int g = tid >> 2, part = tid & 3, bin = 255 - g;
-      int c = 0;
-      for (int w2 = part; w2 < 32; w2 += 4) c += (int)hist[w2 * 256 + bin];
-      c += __shfl_xor_sync(0xFFFFFFFFu, c, 1);
-      c += __shfl_xor_sync(0xFFFFFFFFu, c, 2);
-      int inc = c;
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-        if (lane >= o) inc += n;
-      }
-      if (lane == 31) wtot[warp] = inc;
-      __syncthreads();
-      if (warp == 0) {
-        const int v = wtot[lane];
-        int vi = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int n = __shfl_up_sync(0xFFFFFFFFu, vi, o);
-          if (lane >= o) vi += n;
-        }
-        wpre[lane] = vi - v;
-      }
-      __syncthreads();
-      const int ex = wpre[warp] + inc - c;
-      if (part == 0 && ex < rem && ex + c >= rem) {
-        sel[0] = (uint32_t)bin;
-        sel[1] = (uint32_t)(rem - ex);
-      }
-      __syncthreads();
-      prefix |= sel[0] << shift;
-      mask |= 255u << shift;
-      rem = (int)sel[1];
-      __syncthreads();
-    }
+    __syncthreads();
+    prefix = radix_select_kth(tk_keys, a.F, k, hist, wtot, wpre, sel, &rem);
   }
   // tie prefix over tiles: number of keys equal to K in lower tiles
   const uint32_t K = prefix;
@@ -261,6 +280,13 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
           rval[slot] = reinterpret_cast<const uint16_t*>(a.vdense)[(size_t)t * a.F + j];
       }
       run += __popc(kb);
+      if (a.hfull) {  // full-h variant: the down projection's h row, zero where not kept
+        const size_t off = (size_t)t * a.F + j;
+        const float hv = keep ? a.hfull[off] : 0.0f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+        a.h_hi[off] = hi;
+        a.h_lo[off] = __float2bfloat16_rn(hv - __bfloat162float(hi));
+      }
     }
     __syncwarp();
     const int ni = a.C >> 3, nvv = a.C * vb / 16;  // 16-byte vectors of idx and of values
@@ -278,6 +304,83 @@ __global__ void __launch_bounds__(1024) k_wina_topk(const TopkArgs a) {
     }
     __syncwarp();
   }
+}
+
+// ------------------------------------------------- WINA on the input side
+// [WINA] section 3.1 applied to the layer that consumes x, the stacked
+// [W_gate; W_up]: per token keep the k input coordinates with the largest
+// s_i = |x_i|·c_i (c = the stacked matrix's column norms; the product
+// rounded once to fp32, equal scores to the smaller index) and zero the rest.
+// One CTA (1024 threads) per token; d <= 4 x 1024.
+struct InputSelectArgs {
+  const __nv_bfloat16* x;   // [T][d]
+  const float* colnorm;     // [d]
+  __nv_bfloat16* xsel;      // [T][d]
+  int T, d, k;
+};
+
+__host__ __device__ inline int input_select_smem_bytes(int d) { return d * 4 + 32 * 256 * 4; }
+
+__global__ void __launch_bounds__(1024) k_input_select(const InputSelectArgs a) {
+  extern __shared__ uint32_t is_keys[];   // [d] keys, [32][256] histograms
+  uint32_t* hist = is_keys + a.d;
+  __shared__ int wtot[33], wpre[32];
+  __shared__ uint32_t sel[4];
+  griddep_wait();
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const __nv_bfloat16* xr = a.x + (size_t)t * a.d;
+  for (int i = tid; i < a.d; i += blockDim.x)
+    is_keys[i] = __float_as_uint(fabsf(__bfloat162float(xr[i])) * a.colnorm[i]);
+  __syncthreads();
+  const int k = a.k;
+  int rem = k;
+  uint32_t K = 0;
+  const bool keep_all = k >= a.d;
+  if (!keep_all && k > 0) K = radix_select_kth(is_keys, a.d, k, hist, wtot, wpre, sel, &rem);
+  // ties at K: the rem lowest indices.  Thread tid owns the contiguous
+  // coordinates [4 tid, 4 tid + 4): a block scan of its tie count ranks them
+  const int i0 = 4 * tid;
+  int eq = 0;
+  for (int q = 0; q < 4; ++q) eq += (i0 + q < a.d && is_keys[i0 + q] == K) ? 1 : 0;
+  int tot;
+  int rank = block_scan_excl(eq, wtot, &tot);
+  __nv_bfloat16* out = a.xsel + (size_t)t * a.d;
+  for (int q = 0; q < 4; ++q) {
+    const int i = i0 + q;
+    if (i >= a.d) break;
+    const uint32_t key = is_keys[i];
+    bool keep = keep_all;
+    if (!keep_all && k > 0) {
+      keep = key > K;
+      if (key == K) keep = rank++ < rem;
+    }
+    out[i] = keep ? xr[i] : __float2bfloat16_rn(0.0f);
+  }
+}
+
+// Column norms of the stacked [W_gate; W_up] (create time): c_i = sqrt of the
+// sum over both matrices' rows of W[j][i]^2, accumulated in fp64 and rounded
+// to fp32.  One thread per column (consecutive threads read consecutive
+// columns of a row), rows split across gridDim.y with fp64 atomics into
+// acc[d], then k_col_norms_finish rounds.
+__global__ void k_col_sumsq(const __nv_bfloat16* __restrict__ Wg, const __nv_bfloat16* __restrict__ Wu, int F,
+                            int d, double* acc) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d) return;
+  const int per = (2 * F + gridDim.y - 1) / gridDim.y;
+  const int r0 = blockIdx.y * per, r1 = min(2 * F, r0 + per);
+  double s = 0.0;
+  for (int r = r0; r < r1; ++r) {
+    const __nv_bfloat16* W = r < F ? Wg : Wu;
+    const double v = (double)__bfloat162float(W[(size_t)(r < F ? r : r - F) * d + i]);
+    s += v * v;
+  }
+  atomicAdd(&acc[i], s);
+}
+
+__global__ void k_col_norms_finish(const double* acc, int d, float* c) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < d) c[i] = (float)sqrt(acc[i]);
 }
 
 // ---------------------------------------------------------------- fp32 path

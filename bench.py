@@ -49,6 +49,8 @@ BENCH_SHAPES = {
     "wina_bf16": (32, 2, 16, 1000),
     "prefill_bf16": (4096, 4, 3, 300),
     "tiny_fp32": (64, 1, 4, 1000),
+    "wina_fullh_bf16": (32, 2, 16, 1000),
+    "wina_input_bf16": (32, 2, 16, 1000),
 }
 SPARSITY = {
     "decode_bf16": "relu gate bias -1.2816 (~90% zeros)",
@@ -56,6 +58,8 @@ SPARSITY = {
     "wina_bf16": "silu gate, WINA top-k k=5018 (65% dropped)",
     "prefill_bf16": "relu gate, heavy-tailed per-token nnz (mean ~99 dropped of 8192)",
     "tiny_fp32": "relu gate bias -1.2816 (~90% zeros)",
+    "wina_fullh_bf16": "silu gate, WINA full-h top-k |a*u|*||w_down|| k=5018 (65% dropped)",
+    "wina_input_bf16": "silu gate, orthogonal rotation V, input-side top-2048 of 4096, WINA top-k k=5018",
 }
 TIMING_STRIDE = 8
 REF_BUDGET_S = 90.0
@@ -73,6 +77,8 @@ KERNEL_SOURCES = {
     "gate_f32": ["simt.cuh", "epilogues.cuh", "ptx.cuh"],
     "rows_f32": ["simt.cuh", "ptx.cuh"],
     "fallback_f32": ["simt.cuh", "ptx.cuh"],
+    "rotate_x": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
+    "input_select": ["simt.cuh", "ptx.cuh"],
 }
 
 
@@ -201,14 +207,14 @@ def oracle_timing(inp, T: int, budget_s: float, steps: int = 0):
     f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
     wl = inp.wl
     W = dict(W_up=f(inp.W_up), W_down=f(inp.W_down), W_gate=f(inp.W_gate), A=f(inp.A), B=f(inp.B),
-             bias=f(inp.bias))
+             bias=f(inp.bias), V=f(inp.V))
     xs = f(inp.x)
     n, tokens, t0 = 0, 0, time.perf_counter()
     while True:
         x = xs[(n * T) % xs.shape[0]:][:T]
         oracle.forward(np.ascontiguousarray(x), W["W_up"], W["W_down"], W_gate=W["W_gate"], A=W["A"],
                        B=W["B"], bias=W["bias"], dtype=wl.dtype, mode=wl.mode, act=wl.act,
-                       threshold=wl.threshold, k=wl.k, C=wl.tile_capacity)
+                       threshold=wl.threshold, k=wl.k, C=wl.tile_capacity, input_k=wl.input_k, V=W["V"])
         n += 1
         tokens += x.shape[0]
         el = time.perf_counter() - t0
@@ -250,6 +256,10 @@ def kernel_work(wl, T: int, path: str, st: dict) -> dict:
     n_o, U, nnz = st["n_overflow"], st["union"], st["nnz"]
     fp32 = wl.dtype == "fp32"
     w = {}
+    if wl.rotation != "none":
+        w["rotate_x"] = {"bytes": d * d * es + 2 * xb, "flops": 2 * T * d * d}
+    if wl.input_k:
+        w["input_select"] = {"bytes": 2 * xb + d * 4, "flops": 0}
     g = "gate_f32" if fp32 else "gate"
     if R:
         w["gate_lowrank_z"] = {"bytes": d * R * es + xb + T * R * es, "flops": 2 * T * d * R}
@@ -257,6 +267,10 @@ def kernel_work(wl, T: int, path: str, st: dict) -> dict:
     elif wl.mode == "wina_topk":
         w[g] = {"bytes": F * d * es + xb + T * F * (es + 4) + F * 4, "flops": 2 * T * d * F}
         w["wina_topk"] = {"bytes": T * F * (es + 4) + twell, "flops": 0}
+    elif wl.mode == "wina_full_h":
+        # g and u of every neuron: W_gate and W_up in full; v, score and h out
+        w[g] = {"bytes": 2 * F * d * es + xb + T * F * (es + 8) + F * 4, "flops": 4 * T * d * F}
+        w["wina_topk"] = {"bytes": T * F * (es + 8) + twell + T * F * 4, "flops": 0}
     else:
         w[g] = {"bytes": F * d * es + xb + twell + (0 if fp32 else kmask), "flops": 2 * T * d * F}
     sparse = {"bytes": U * 2 * d * es + xb + yb + twell, "flops": 4 * nnz * d}
@@ -279,8 +293,9 @@ def kernel_work(wl, T: int, path: str, st: dict) -> dict:
                              "flops": 2 * T * d * F + 4 * nnza * d}
     else:
         w["router"] = {"bytes": yb + 2 * n_o * d * es, "flops": 0}
-        w["tile_h"] = {"bytes": F * d * es + xb + twell + T * F * 4, "flops": 2 * T * d * F}
-        if wl.mode != "wina_topk":
+        if wl.mode != "wina_full_h":
+            w["tile_h"] = {"bytes": F * d * es + xb + twell + T * F * 4, "flops": 2 * T * d * F}
+        if wl.mode == "relu_threshold":
             w["fallback_h"] = {"bytes": dense_in + n_o * F * 4, "flops": 2 * n_o * d * F}
         w["down"] = {"bytes": F * d * es + T * F * 4 + yb, "flops": 2 * T * F * d}
     return w
@@ -299,6 +314,12 @@ def step_work(wl, T: int, st: dict) -> tuple[int, int]:
     if n_o:
         byts += 2 * F * d * es
     flops = gate_f + 4 * st["nnz"] * d + 4 * n_o * d * F
+    if wl.mode == "wina_full_h":       # W_up read in full (not the union), u of every neuron
+        byts += (F - st["union"]) * d * es
+        flops += 2 * T * d * F - 2 * st["nnz"] * d
+    if wl.rotation != "none":          # V read once per forward; x·V
+        byts += d * d * es
+        flops += 2 * T * d * d
     return int(byts), int(flops)
 
 
@@ -370,7 +391,8 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
         ws = {k: dev(getattr(inp, k)) for k in ("W_gate", "A", "B", "W_up", "W_down", "bias")}
         ffn = SparseFFN(ws["W_up"], ws["W_down"], W_gate=ws["W_gate"], A=ws["A"], B=ws["B"], bias=ws["bias"],
                         mode=wl.mode, act=wl.act, threshold=wl.threshold, k=wl.k,
-                        tile_capacity=wl.tile_capacity, max_tokens=T)
+                        tile_capacity=wl.tile_capacity, max_tokens=T, input_k=wl.input_k or 0,
+                        V=dev(inp.V))
         sets.append((ws, ffn))
     xall = dev(inp.x)
     xb = [xall[i * T:(i + 1) * T].contiguous() for i in range(NXB)]
@@ -472,7 +494,7 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
 # the other configurations, measured after the headline in the same default
 # run: (workload, tokens per forward)
 EXTRA_WORKLOADS = [("decode_bf16", 1), ("decode_bf16", 4), ("lopa_bf16", 32), ("wina_bf16", 32),
-                   ("prefill_bf16", 4096), ("tiny_fp32", 64)]
+                   ("prefill_bf16", 4096), ("tiny_fp32", 64), ("wina_fullh_bf16", 32), ("wina_input_bf16", 32)]
 EXTRA_MIN_STEPS = 200
 EXTRA_MAX_S = 2.0
 

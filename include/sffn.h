@@ -76,7 +76,17 @@ typedef enum {
 } sffn_status;
 
 typedef enum { SFFN_BF16 = 0, SFFN_FP32 = 1 } sffn_dtype;
-typedef enum { SFFN_MODE_RELU_THRESHOLD = 0, SFFN_MODE_WINA_TOPK = 1 } sffn_mode;
+/* Selection of the kept neurons.
+ *   RELU_THRESHOLD: keep iff |sigma(g)| > threshold;
+ *   WINA_TOPK     : per token the k largest |sigma(g_j)|·||W_down[j,:]||_2 (WINA
+ *                   framework explainer, section 3.1, hidden value = the gate
+ *                   activation: only the kept neurons' W_up rows are read);
+ *   WINA_FULL_H   : per token the k largest |sigma(g_j)·u_j|·||W_down[j,:]||_2,
+ *                   the same score with the hidden value taken as the full
+ *                   gated product: the up projection of every neuron is
+ *                   computed (W_up read in full), the down projection is sparse.
+ *                   Dense gate, bf16, tile_capacity 128. */
+typedef enum { SFFN_MODE_RELU_THRESHOLD = 0, SFFN_MODE_WINA_TOPK = 1, SFFN_MODE_WINA_FULL_H = 2 } sffn_mode;
 typedef enum { SFFN_ACT_RELU = 0, SFFN_ACT_SILU = 1 } sffn_act;
 
 /* How the kept (token, neuron) pairs of non-overflow tokens are computed.
@@ -117,6 +127,21 @@ typedef struct sffn_desc {
   const void* W_up;     /* [d_ff][d_model]                                         */
   const void* W_down;   /* [d_ff][d_model]                                         */
   const float* gate_bias; /* [d_ff] fp32 or NULL                                   */
+  /* WINA on the input side (WINA explainer, section 3.1, applied to the layer
+   * that consumes x, the stacked [W_gate; W_up]): per token keep the input_k
+   * coordinates of largest |x_i|·c_i, c_i = ||column i of [W_gate; W_up]||_2
+   * (fp64, rounded to fp32; the product rounded to fp32, equal scores to the
+   * smaller index), zero the others, and run both projections on the result.
+   * 0 = off; 1..d_model.  Dense gate, bf16. */
+  int input_k;
+  /* Orthogonalisation (WINA explainer, section 3.3): V [d_model][d_model] bf16,
+   * the right singular vectors of [W_gate; W_up] (any V is accepted; the SVD
+   * itself is the caller's).  At create time the handle stores W_gate·V and
+   * W_up·V rounded to bf16 (2·d_ff·d_model·2 bytes), and every forward first
+   * rotates its tokens, x' = bf16(x·V), so that W V V^T x = W x; the input-side
+   * selection then acts on x' with the rotated column norms (the singular
+   * values when V comes from the SVD).  NULL = off.  Dense gate, bf16. */
+  const void* V;
 } sffn_desc;
 
 typedef struct sffn_handle sffn_handle;

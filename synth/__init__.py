@@ -53,7 +53,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-TID_X, TID_WGATE, TID_WUP, TID_WDOWN, TID_A, TID_B, TID_BIAS, TID_NNZ, TID_APAT = range(9)
+TID_X, TID_WGATE, TID_WUP, TID_WDOWN, TID_A, TID_B, TID_BIAS, TID_NNZ, TID_APAT, TID_V = range(10)
 
 
 @dataclass(frozen=True)
@@ -77,6 +77,8 @@ class Workload:
     nnz_cap_frac: float = 0.45
     exact_grid: bool = False
     seed: int = 0
+    input_k: Optional[int] = None  # input-side WINA: input coordinates kept per token
+    rotation: str = "none"         # "none", "signed_perm" or "orthogonal": a V [d][d] to orthogonalise with
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -90,6 +92,12 @@ WORKLOADS = {
                              x_kind="lognormal_nnz", bias=None),
     "wina_bf16": Workload("wina_bf16", 4096, 14336, 32, mode="wina_topk", act="silu",
                           bias=None, k=5018, tile_capacity=128),
+    # WINA variants: the full-h score, and input-side selection (half of the
+    # input coordinates) after an orthogonal rotation, on the WINA shapes
+    "wina_fullh_bf16": Workload("wina_fullh_bf16", 4096, 14336, 32, mode="wina_full_h", act="silu",
+                                bias=None, k=5018, tile_capacity=128),
+    "wina_input_bf16": Workload("wina_input_bf16", 4096, 14336, 32, mode="wina_topk", act="silu",
+                                bias=None, k=5018, tile_capacity=128, input_k=2048, rotation="orthogonal"),
 }
 
 
@@ -137,6 +145,24 @@ class Inputs:
     bias: Optional[torch.Tensor]          # fp32 [d_ff] or None
     nnz_target: Optional[np.ndarray] = None
     extra: dict = field(default_factory=dict)
+    V: Optional[torch.Tensor] = None      # [d][d] orthogonalising rotation, or None
+
+
+def rotation_matrix(kind: str, d: int, seed: int, dtype: str) -> torch.Tensor:
+    """A seeded d x d rotation to orthogonalise with (an input of the method,
+    like the weights): "signed_perm" is a permutation with random signs
+    (exact in any dtype); "orthogonal" is the Q factor of a Gaussian matrix,
+    rounded to the operand dtype (orthogonal up to that rounding)."""
+    rng = _rng(seed, TID_V)
+    if kind == "signed_perm":
+        V = np.zeros((d, d), dtype=np.float32)
+        V[np.arange(d), rng.permutation(d)] = rng.choice(np.array([-1.0, 1.0], dtype=np.float32), d)
+    elif kind == "orthogonal":
+        q, r = np.linalg.qr(rng.standard_normal((d, d)))
+        V = (q * np.sign(np.diag(r))[None, :]).astype(np.float32)
+    else:
+        raise ValueError(kind)
+    return _to_dtype(V, dtype)
 
 
 def token_scales(wl: Workload, T: Optional[int] = None) -> tuple[np.ndarray, np.ndarray]:
@@ -213,7 +239,8 @@ def make_inputs(wl: Workload, T: Optional[int] = None, weights_only: bool = Fals
         if eg:
             b = round(b * 2.0 ** 14) / 2.0 ** 14
         bias = torch.full((F,), b, dtype=torch.float32)
-    return Inputs(wl, x, W_gate, A, B, W_up, W_down, bias, nnz)
+    V = rotation_matrix(wl.rotation, d, seed, wl.dtype) if wl.rotation != "none" else None
+    return Inputs(wl, x, W_gate, A, B, W_up, W_down, bias, nnz, V=V)
 
 
 def to_f64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:

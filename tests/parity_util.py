@@ -28,7 +28,8 @@ def make_ffn(inp: synth.Inputs, max_tokens: int, path: str = "auto", C: Optional
                      B=to_dev(inp.B), bias=to_dev(inp.bias), mode=wl.mode, act=wl.act,
                      threshold=wl.threshold, k=wl.k,
                      tile_capacity=wl.tile_capacity if C is None else C, max_tokens=max_tokens,
-                     path=path, debug_gate=debug_gate, separate=separate, cooperative=cooperative)
+                     path=path, debug_gate=debug_gate, separate=separate, cooperative=cooperative,
+                     input_k=wl.input_k or 0, V=to_dev(inp.V))
 
 
 @dataclass
@@ -139,7 +140,8 @@ def check(inp: synth.Inputs, T: Optional[int] = None, path: str = "auto", C: Opt
         res = oracle.forward(synth.to_f64(x), synth.to_f64(inp.W_up), synth.to_f64(inp.W_down),
                              W_gate=synth.to_f64(inp.W_gate), A=synth.to_f64(inp.A), B=synth.to_f64(inp.B),
                              bias=synth.to_f64(inp.bias), dtype=wl.dtype, mode=wl.mode, act=wl.act,
-                             threshold=wl.threshold, k=wl.k, C=C)
+                             threshold=wl.threshold, k=wl.k, C=C, input_k=wl.input_k,
+                             V=synth.to_f64(inp.V))
     own = ffn is None
     if own:
         ffn = make_ffn(inp, max_tokens=T, path=path, C=C, separate=separate)

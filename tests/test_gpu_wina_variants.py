@@ -1,0 +1,154 @@
+"""GPU parity of the WINA variants (WINA framework explainer, sections 3.1
+to 3.3) through the C ABI against the fp64 oracle: the full-h score
+(|sigma(g)·u|·||W_down row||), input-side selection (|x_i|·||column i of
+[W_gate; W_up]||) and the orthogonalising rotation by V.
+
+Exact cases (exact-grid operands, a signed-permutation V, which is exact in
+bf16) must match bit for bit.  On Gaussian inputs the kept sets must match
+outside the decision band; with a general orthogonal V the device and the
+oracle round W·V and x·V independently (fp32 against fp64 sums before the
+bf16 rounding), so a few kept decisions may differ there and y is held to the
+parity tolerance.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from activation_sparse_gated_relu_b200 import SFFN_PATH_ROWS, SFFN_PATH_TILES
+
+from parity_util import check, make_ffn, rel_err, run_gpu, to_dev
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+
+def small(**kw):
+    base = dict(name="small", d_model=256, d_ff=512, tokens=32, tile_capacity=32)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+# ----------------------------------------------------------------- full-h
+def test_fullh_config():
+    inp = synth.make_inputs(W["wina_fullh_bf16"])
+    st = check(inp)
+    assert st["path"] == SFFN_PATH_TILES
+
+
+@pytest.mark.parametrize("T", [1, 9, 32])
+def test_fullh_small_relu(T):
+    wl = small(tokens=T, mode="wina_full_h", act="relu", bias=-0.5, k=150, tile_capacity=128)
+    check(synth.make_inputs(wl))
+
+
+def test_fullh_keeps_exactly_k_and_differs_from_gate_only():
+    wl = small(tokens=16, mode="wina_full_h", act="silu", bias=None, k=100, tile_capacity=128)
+    inp = synth.make_inputs(wl)
+    ffn = make_ffn(inp, max_tokens=16)
+    try:
+        g = run_gpu(ffn, inp.x)
+    finally:
+        ffn.close()
+    assert np.all(g.count.sum(axis=1) == 100)
+    gate_only = oracle.forward_inputs(synth.make_inputs(wl.with_(mode="wina_topk")))
+    full = oracle.forward_inputs(inp)
+    assert (gate_only.keep != full.keep).any()     # the variants select differently
+
+
+def test_fullh_k_edges():
+    for k in (0, 512):
+        wl = small(tokens=8, mode="wina_full_h", act="silu", bias=None, k=k, tile_capacity=128)
+        check(synth.make_inputs(wl))
+
+
+# ------------------------------------------------------------- input side
+@pytest.mark.parametrize("T,path", [(8, "auto"), (8, "tiles"), (32, "auto")])
+def test_input_side_exact_grid_bit_exact(T, path):
+    wl = small(tokens=T, exact_grid=True, input_k=100)
+    st = check(synth.make_inputs(wl), path=path)
+    assert st["mismatch"] == 0
+
+
+@pytest.mark.parametrize("T", [8, 32])
+def test_input_side_with_signed_permutation_bit_exact(T):
+    # a signed permutation is exact in bf16: W·V, x·V, the column norms and
+    # the selection are exact, so everything matches bit for bit
+    wl = small(tokens=T, exact_grid=True, input_k=64, rotation="signed_perm")
+    st = check(synth.make_inputs(wl))
+    assert st["mismatch"] == 0
+
+
+def test_input_side_decode_gaussian():
+    wl = W["decode_bf16"].with_(input_k=2048)
+    inp = synth.make_inputs(wl)
+    st = check(inp, T=8)
+    assert st["launches"] == 2          # input selection, then the single launch
+    assert st["path"] == SFFN_PATH_ROWS
+
+
+def test_input_side_k_edges():
+    # k_in = d keeps every coordinate: the plain forward
+    wl = small(tokens=8, input_k=256, exact_grid=True)
+    inp = synth.make_inputs(wl)
+    st = check(inp)
+    plain = check(synth.make_inputs(wl.with_(input_k=None)))
+    assert st["mismatch"] == plain["mismatch"] == 0
+    wl1 = small(tokens=8, input_k=1)
+    check(synth.make_inputs(wl1))
+
+
+# ------------------------------------------------------- orthogonalisation
+def _compare_rotated(inp, T):
+    wl = inp.wl
+    res = oracle.forward_inputs(inp, T=T)
+    ffn = make_ffn(inp, max_tokens=T)
+    try:
+        g = run_gpu(ffn, inp.x[:T])
+    finally:
+        ffn.close()
+    err = rel_err(g.y, res.y)
+    assert err <= 2e-3, err
+    # kept sets: per token; exactly k in WINA modes
+    Pn = res.count.shape[1]
+    gk = np.zeros_like(res.keep)
+    for t in range(T):
+        for p in range(Pn):
+            n = min(int(g.count[t, p]), g.idx.shape[2])
+            gk[t, g.idx[t, p, :n].astype(np.int64)] = True
+    agree = float(np.mean(gk == res.keep))
+    assert agree >= 0.999, agree
+    if wl.mode != "relu_threshold":
+        assert np.all(g.count.sum(axis=1) == wl.k)
+    return err, agree
+
+
+def test_rotation_orthogonal_small():
+    wl = small(tokens=16, mode="wina_topk", act="silu", bias=None, k=150, tile_capacity=128,
+               rotation="orthogonal", input_k=128)
+    _compare_rotated(synth.make_inputs(wl), 16)
+
+
+def test_rotation_without_input_selection_keeps_y():
+    # V only (every input coordinate kept): y is the unrotated forward's up to
+    # the bf16 roundings of W·V and x·V
+    wl = small(tokens=8, rotation="orthogonal")
+    inp = synth.make_inputs(wl)
+    ffn = make_ffn(inp, max_tokens=8)
+    try:
+        g = run_gpu(ffn, inp.x)
+    finally:
+        ffn.close()
+    plain = oracle.forward_inputs(synth.make_inputs(wl.with_(rotation="none")))
+    rot = oracle.forward_inputs(inp)
+    assert rel_err(g.y, rot.y) <= 2e-3
+    assert rel_err(rot.y, plain.y) <= 0.05      # the rotation itself only rounds
+
+
+def test_wina_input_config():
+    inp = synth.make_inputs(W["wina_input_bf16"])
+    _compare_rotated(inp, 32)
