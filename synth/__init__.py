@@ -10,7 +10,7 @@ Every tensor is drawn from ``numpy.random.default_rng([seed, tensor_id])``
 operand dtype (bf16 by round-to-nearest-even through torch, or kept in fp32).
 
 Tensor ids: x = 0, W_gate = 1, W_up = 2, W_down = 3, A = 4, B = 5, bias = 6,
-nnz draw = 7, exact-grid sparsity pattern of A = 8.
+nnz draw = 7, exact-grid sparsity pattern of A = 8, rotation V = 9.
 
 Weight scales follow N(0, 1/fan_in): fan_in = d for W_gate, W_up and A, r for
 B, and d_ff for W_down (the down projection sums over the d_ff neurons).  All
@@ -36,6 +36,11 @@ produce, stood in for by Gaussian draws):
   P(g_tj > 0) = min(nnz_t/d_ff, 0.45).  C = 8, so heavy tokens overflow.
 * ``wina_bf16``: d=4096, d_ff=14336, T=32, SiLU, no bias, keep the top
   k = round(0.35·14336) = 5018 neurons per token, C = 128.
+* ``wina_fullh_bf16``: the same shapes and k, scored on the full gated
+  product |sigma(g)·u|.
+* ``wina_input_bf16``: the same shapes and k, after an orthogonal rotation V
+  (a randomly signed and permuted Hadamard matrix over 64) and input-side
+  selection of 2048 of the 4096 rotated input coordinates per token.
 
 The optional ``exact_grid`` flag quantises every operand to a coarse dyadic
 grid (x to multiples of 2^-4, weights to k·2^-e with |k| <= 255, the bias to
@@ -78,7 +83,7 @@ class Workload:
     exact_grid: bool = False
     seed: int = 0
     input_k: Optional[int] = None  # input-side WINA: input coordinates kept per token
-    rotation: str = "none"         # "none", "signed_perm" or "orthogonal": a V [d][d] to orthogonalise with
+    rotation: str = "none"         # "none", "signed_perm", "hadamard" or "orthogonal": a V [d][d]
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -97,7 +102,7 @@ WORKLOADS = {
     "wina_fullh_bf16": Workload("wina_fullh_bf16", 4096, 14336, 32, mode="wina_full_h", act="silu",
                                 bias=None, k=5018, tile_capacity=128),
     "wina_input_bf16": Workload("wina_input_bf16", 4096, 14336, 32, mode="wina_topk", act="silu",
-                                bias=None, k=5018, tile_capacity=128, input_k=2048, rotation="orthogonal"),
+                                bias=None, k=5018, tile_capacity=128, input_k=2048, rotation="hadamard"),
 }
 
 
@@ -160,6 +165,18 @@ def rotation_matrix(kind: str, d: int, seed: int, dtype: str) -> torch.Tensor:
     elif kind == "orthogonal":
         q, r = np.linalg.qr(rng.standard_normal((d, d)))
         V = (q * np.sign(np.diag(r))[None, :]).astype(np.float32)
+    elif kind == "hadamard":
+        # Sylvester's Hadamard matrix over sqrt(d), with its columns permuted
+        # and signed at random: orthogonal, entries +-2^-m for d = 4^m, so x·V
+        # and W·V of grid operands are exact fp32 sums
+        m = int(round(math.log(d, 4)))
+        if 4 ** m != d:
+            raise ValueError("the Hadamard rotation needs d = 4^m")
+        H = np.ones((1, 1), dtype=np.float32)
+        while H.shape[0] < d:
+            H = np.block([[H, H], [H, -H]])
+        V = (H / np.float32(2 ** m))[:, rng.permutation(d)] * rng.choice(
+            np.array([-1.0, 1.0], dtype=np.float32), d)[None, :]
     else:
         raise ValueError(kind)
     return _to_dtype(V, dtype)

@@ -150,5 +150,44 @@ def test_rotation_without_input_selection_keeps_y():
 
 
 def test_wina_input_config():
-    inp = synth.make_inputs(W["wina_input_bf16"])
-    _compare_rotated(inp, 32)
+    # the Hadamard V (entries +-2^-6) on exact-grid operands: x·V and W·V
+    # are exact fp32 sums, so both sides round the same values to bf16 and the
+    # input selection matches exactly; the SiLU top-k follows under its band
+    wl = W["wina_input_bf16"].with_(exact_grid=True)
+    check(synth.make_inputs(wl))
+
+
+def test_wina_input_config_gaussian():
+    # the bench's own operands (Gaussian x and weights): x·V is rounded to
+    # bf16 where the device's fp32 sum and the oracle's fp64 sum may straddle
+    # a rounding midpoint, which can swap an input coordinate at the selection
+    # boundary of a token.  Such tokens are found from the oracle's own sums
+    # and held to a valid selection (exactly k kept), the others to the
+    # parity tolerance
+    wl = W["wina_input_bf16"]
+    inp = synth.make_inputs(wl)
+    T = wl.tokens
+    f = synth.to_f64
+    x, V = f(inp.x), f(inp.V)
+    Wg_r, Wu_r = oracle.rotate(f(inp.W_gate), V, "bf16"), oracle.rotate(f(inp.W_up), V, "bf16")
+    xr = oracle.rotate(x, V, "bf16")
+    # the oracle's forward with V does exactly these rotations first
+    res = oracle.forward(xr, Wu_r, f(inp.W_down), W_gate=Wg_r, dtype="bf16", mode=wl.mode, act=wl.act,
+                         k=wl.k, C=wl.tile_capacity, input_k=wl.input_k)
+    exact = x @ V
+    err = np.ldexp(np.abs(x) @ np.abs(V), -14)      # bound on the device's fp32 sum error
+    half = np.abs(oracle.round_bf16(np.abs(xr) * (1 + 2.0 ** -7)) - np.abs(xr)) / 2
+    may_flip = np.abs(np.abs(exact - xr) - half) <= err     # within err of a midpoint
+    sc = oracle.input_scores(xr, oracle.input_col_norms(Wg_r, Wu_r))
+    kth = np.sort(sc, axis=1)[:, ::-1][:, wl.input_k - 1][:, None]
+    near = np.abs(sc - kth) <= 2.0 ** -6 * kth
+    amb_tok = (may_flip & near).any(axis=1)
+    assert amb_tok.sum() <= T // 4, amb_tok.sum()
+    ffn = make_ffn(inp, max_tokens=T)
+    try:
+        g = run_gpu(ffn, inp.x)
+    finally:
+        ffn.close()
+    ok = ~amb_tok
+    assert rel_err(g.y[ok], res.y[ok]) <= 2e-3
+    assert np.all(g.count.sum(axis=1) == wl.k)
