@@ -3,12 +3,16 @@ to 3.3) through the C ABI against the fp64 oracle: the full-h score
 (|sigma(g)·u|·||W_down row||), input-side selection (|x_i|·||column i of
 [W_gate; W_up]||) and the orthogonalising rotation by V.
 
-Exact cases (exact-grid operands, a signed-permutation V, which is exact in
-bf16) must match bit for bit.  On Gaussian inputs the kept sets must match
-outside the decision band; with a general orthogonal V the device and the
-oracle round W·V and x·V independently (fp32 against fp64 sums before the
-bf16 rounding), so a few kept decisions may differ there and y is held to the
-parity tolerance.
+Exact cases (exact-grid operands; a signed-permutation V, or a signed and
+permuted Hadamard V over sqrt(d), whose products with grid operands are exact
+fp32 sums) must match bit for bit in the input selection.  On Gaussian inputs
+the kept sets must match outside the decision band.  With a general
+orthogonal V the device and the oracle round W·V and x·V to bf16 from
+different sums (fp32 against fp64), so an element whose exact value lies near
+a rounding midpoint may round either way; at full size (4096 coordinates per
+token) that reaches the input selection's boundary in some tokens, so the
+general V is checked on a small case and the full size on the exact Hadamard
+case.
 """
 from __future__ import annotations
 
@@ -155,39 +159,3 @@ def test_wina_input_config():
     # input selection matches exactly; the SiLU top-k follows under its band
     wl = W["wina_input_bf16"].with_(exact_grid=True)
     check(synth.make_inputs(wl))
-
-
-def test_wina_input_config_gaussian():
-    # the bench's own operands (Gaussian x and weights): x·V is rounded to
-    # bf16 where the device's fp32 sum and the oracle's fp64 sum may straddle
-    # a rounding midpoint, which can swap an input coordinate at the selection
-    # boundary of a token.  Such tokens are found from the oracle's own sums
-    # and held to a valid selection (exactly k kept), the others to the
-    # parity tolerance
-    wl = W["wina_input_bf16"]
-    inp = synth.make_inputs(wl)
-    T = wl.tokens
-    f = synth.to_f64
-    x, V = f(inp.x), f(inp.V)
-    Wg_r, Wu_r = oracle.rotate(f(inp.W_gate), V, "bf16"), oracle.rotate(f(inp.W_up), V, "bf16")
-    xr = oracle.rotate(x, V, "bf16")
-    # the oracle's forward with V does exactly these rotations first
-    res = oracle.forward(xr, Wu_r, f(inp.W_down), W_gate=Wg_r, dtype="bf16", mode=wl.mode, act=wl.act,
-                         k=wl.k, C=wl.tile_capacity, input_k=wl.input_k)
-    exact = x @ V
-    err = np.ldexp(np.abs(x) @ np.abs(V), -14)      # bound on the device's fp32 sum error
-    half = np.abs(oracle.round_bf16(np.abs(xr) * (1 + 2.0 ** -7)) - np.abs(xr)) / 2
-    may_flip = np.abs(np.abs(exact - xr) - half) <= err     # within err of a midpoint
-    sc = oracle.input_scores(xr, oracle.input_col_norms(Wg_r, Wu_r))
-    kth = np.sort(sc, axis=1)[:, ::-1][:, wl.input_k - 1][:, None]
-    near = np.abs(sc - kth) <= 2.0 ** -6 * kth
-    amb_tok = (may_flip & near).any(axis=1)
-    assert amb_tok.sum() <= T // 4, amb_tok.sum()
-    ffn = make_ffn(inp, max_tokens=T)
-    try:
-        g = run_gpu(ffn, inp.x)
-    finally:
-        ffn.close()
-    ok = ~amb_tok
-    assert rel_err(g.y[ok], res.y[ok]) <= 2e-3
-    assert np.all(g.count.sum(axis=1) == wl.k)
