@@ -265,3 +265,74 @@ def to_f64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:
     if t is None:
         return None
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------------------
+# gated subspace linear layer (GSI)
+# ---------------------------------------------------------------------------
+TID_GSI_W, TID_GSI_Q, TID_GSI_C, TID_GSI_E, TID_GSI_RHO = range(20, 25)
+
+
+@dataclass(frozen=True)
+class GsiWorkload:
+    """A linear layer y = W x with W [d_out][d_in] and a k-column basis V_k
+    of the activation subspace; tokens x_t = V_k c_t + Q_perp e_t with
+    c_t ~ N(0, I_k), e_t a random direction of the orthogonal complement whose
+    length gives the residual ratio rho_t = ||e_t|| / ||x_t|| a lognormal
+    target (median rho_med, log-spread rho_sigma, capped at 0.95).  The basis
+    and its complement are the columns of one orthogonal matrix Q: a Hadamard
+    matrix over sqrt(d_in) with its columns permuted and signed at random
+    (d_in = 4^m), so V_k is exact in bf16."""
+    name: str
+    d_in: int
+    d_out: int
+    k: int
+    tokens: int
+    eps: float = 0.10
+    rho_med: float = 0.025
+    rho_sigma: float = 0.5
+    dtype: str = "bf16"
+    exact_grid: bool = False
+    seed: int = 0
+
+    def with_(self, **kw) -> "GsiWorkload":
+        return replace(self, **kw)
+
+
+# GPT-J's MLP input projection (d = 4096, d_ff = 16384) at the page's working
+# point k = 256, eps = 0.10 (99.8 % of its tokens took the fast path there;
+# here P(rho > eps) = 1 - Phi(ln(0.1/0.025)/0.5) = 0.28 %), decode batches
+GSI_WORKLOADS = {
+    "gsi_bf16": GsiWorkload("gsi_bf16", 4096, 16384, 256, 8),
+}
+
+
+@dataclass
+class GsiInputs:
+    wl: GsiWorkload
+    x: torch.Tensor        # [T][d_in]
+    W: torch.Tensor        # [d_out][d_in]
+    Vk: torch.Tensor       # [d_in][k]
+    rho_target: np.ndarray
+
+
+def make_gsi_inputs(wl: GsiWorkload, T: Optional[int] = None) -> GsiInputs:
+    T = wl.tokens if T is None else T
+    d, k, seed = wl.d_in, wl.k, wl.seed
+    Q = rotation_matrix("hadamard", d, seed + 1000, "fp32").numpy().astype(np.float64)
+    Vk = Q[:, :k]
+    c = _normal(seed, TID_GSI_C, (T, k), 1.0).astype(np.float64)
+    e = _normal(seed, TID_GSI_E, (T, d - k), 1.0).astype(np.float64)
+    e /= np.linalg.norm(e, axis=1, keepdims=True)
+    xi = _normal(seed, TID_GSI_RHO, (T,), 1.0).astype(np.float64)
+    rho = np.minimum(wl.rho_med * np.exp(wl.rho_sigma * xi), 0.95)
+    cn = np.linalg.norm(c, axis=1)
+    e *= (rho * cn / np.sqrt(1.0 - rho * rho))[:, None]
+    xa = (c @ Vk.T + e @ Q[:, k:].T).astype(np.float32)
+    std = 1.0 / math.sqrt(d)
+    Wa = _normal(seed, TID_GSI_W, (wl.d_out, d), std)
+    if wl.exact_grid:
+        xa = _grid(xa, 4, kmax=4095)
+        Wa = _grid(Wa, _grid_exp(std))
+    return GsiInputs(wl, _to_dtype(xa, wl.dtype), _to_dtype(Wa, wl.dtype),
+                     _to_dtype(Vk.astype(np.float32), wl.dtype), rho)
