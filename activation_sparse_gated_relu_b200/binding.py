@@ -37,6 +37,12 @@ class sffn_desc(ctypes.Structure):
     ]
 
 
+class sffn_gsi_desc(ctypes.Structure):
+    _fields_ = [("d_in", ctypes.c_int), ("d_out", ctypes.c_int), ("k", ctypes.c_int),
+                ("max_tokens", ctypes.c_int), ("eps", ctypes.c_float), ("W", ctypes.c_void_p),
+                ("Vk", ctypes.c_void_p)]
+
+
 class sffn_stats(ctypes.Structure):
     _fields_ = [("n_overflow", ctypes.c_int), ("n_launches", ctypes.c_int), ("path", ctypes.c_int),
                 ("epoch", ctypes.c_uint), ("launch_attrs", ctypes.c_uint)]
@@ -95,6 +101,22 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_timing_end.argtypes = [vp, ip, vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ip),
                                     ctypes.POINTER(ip)]
     lib.sffn_timing_end.restype = st
+    lib.sffn_gsi_create.argtypes = [ctypes.POINTER(sffn_gsi_desc), vp, ctypes.POINTER(vp)]
+    lib.sffn_gsi_create.restype = st
+    lib.sffn_gsi_forward.argtypes = [vp, vp, ip, vp, vp]
+    lib.sffn_gsi_forward.restype = st
+    lib.sffn_gsi_destroy.argtypes = [vp]
+    lib.sffn_gsi_destroy.restype = st
+    lib.sffn_gsi_stats.argtypes = [vp, vp, ctypes.POINTER(ip)]
+    lib.sffn_gsi_stats.restype = st
+    lib.sffn_gsi_debug.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                   ctypes.POINTER(vp)]
+    lib.sffn_gsi_debug.restype = st
+    lib.sffn_gsi_timing_begin.argtypes = [vp, ip, ip]
+    lib.sffn_gsi_timing_begin.restype = st
+    lib.sffn_gsi_timing_end.argtypes = [vp, ip, vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ip),
+                                        ctypes.POINTER(ip)]
+    lib.sffn_gsi_timing_end.restype = st
     lib.sffn_version.argtypes = []
     lib.sffn_version.restype = ctypes.c_char_p
     _lib = lib
@@ -147,15 +169,15 @@ def sffn_timing_begin(h, max_forwards: int, stride: int = 1) -> None:
     _check(load_library().sffn_timing_begin(h, int(max_forwards), int(stride)), "sffn_timing_begin")
 
 
-def sffn_timing_end(h) -> dict:
+def sffn_timing_end(h, fn: str = "sffn_timing_end") -> dict:
     """{label: (total_ms, launches)} over the forwards timed since sffn_timing_begin."""
-    n_max = 16
+    n_max = 24
     names = (ctypes.c_char * 32 * n_max)()
     ms = (ctypes.c_float * n_max)()
     cnt = (ctypes.c_int * n_max)()
     n = ctypes.c_int()
-    _check(load_library().sffn_timing_end(h, n_max, ctypes.cast(names, ctypes.c_void_p), ms, cnt,
-                                          ctypes.byref(n)), "sffn_timing_end")
+    _check(getattr(load_library(), fn)(h, n_max, ctypes.cast(names, ctypes.c_void_p), ms, cnt,
+                                       ctypes.byref(n)), fn)
     return {names[i].value.decode(): (float(ms[i]), int(cnt[i])) for i in range(min(n.value, n_max))}
 
 
@@ -362,6 +384,83 @@ class SparseFFN:
     def close(self) -> None:
         if getattr(self, "h", None) is not None and self.h.value:
             sffn_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class GsiLinear:
+    """Gated subspace linear layer over device tensors: y = M·bf16(V_k^T x)
+    for tokens whose residual ratio is below eps, y = W x for the others.
+    W is [d_out][d_in] bf16, V_k is [d_in][k] bf16 (orthonormal columns)."""
+
+    def __init__(self, W, Vk, eps: float, max_tokens: int = 8, stream: Optional[int] = None):
+        import torch
+        self.h = None
+        if W.dim() != 2 or Vk.dim() != 2:
+            raise ValueError("W must be [d_out][d_in] and Vk [d_in][k]")
+        d_out, d_in = W.shape
+        k = Vk.shape[1]
+        _check_tensor(W, "W", torch.bfloat16, (d_out, d_in), True)
+        _check_tensor(Vk, "Vk", torch.bfloat16, (d_in, k), True)
+        self._keep = [W, Vk]
+        self.d_in, self.d_out, self.k, self.max_tokens = d_in, d_out, k, max_tokens
+        desc = sffn_gsi_desc()
+        desc.d_in, desc.d_out, desc.k, desc.max_tokens = d_in, d_out, k, max_tokens
+        desc.eps = float(eps)
+        desc.W, desc.Vk = W.data_ptr(), Vk.data_ptr()
+        h = ctypes.c_void_p()
+        _check(load_library().sffn_gsi_create(ctypes.byref(desc), ctypes.c_void_p(SparseFFN._stream(stream)),
+                                              ctypes.byref(h)), "sffn_gsi_create")
+        self.h = h
+
+    def forward(self, x, y=None, stream: Optional[int] = None):
+        import torch
+        if not isinstance(x, torch.Tensor) or x.dim() != 2:
+            raise ValueError("x must be a [T][d_in] tensor")
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T = {T} exceeds max_tokens = {self.max_tokens}")
+        _check_tensor(x, "x", torch.bfloat16, (T, self.d_in), True)
+        if y is None:
+            y = torch.empty((T, self.d_out), dtype=torch.float32, device=x.device)
+        _check_tensor(y, "y", torch.float32, (T, self.d_out), True)
+        _check(load_library().sffn_gsi_forward(self.h, ctypes.c_void_p(x.data_ptr()), T,
+                                               ctypes.c_void_p(y.data_ptr()),
+                                               ctypes.c_void_p(SparseFFN._stream(stream))), "sffn_gsi_forward")
+        return y
+
+    __call__ = forward
+
+    def n_slow(self, stream: Optional[int] = None) -> int:
+        n = ctypes.c_int()
+        _check(load_library().sffn_gsi_stats(self.h, ctypes.c_void_p(SparseFFN._stream(stream)), ctypes.byref(n)),
+               "sffn_gsi_stats")
+        return int(n.value)
+
+    def debug(self, T: int) -> dict:
+        import torch
+        vp = ctypes.c_void_p
+        g, rn2, xn2, M = vp(), vp(), vp(), vp()
+        _check(load_library().sffn_gsi_debug(self.h, ctypes.byref(g), ctypes.byref(rn2), ctypes.byref(xn2),
+                                             ctypes.byref(M)), "sffn_gsi_debug")
+        return {"g": _view(g.value, (T, self.k), "<f4"), "rn2": _view(rn2.value, (T,), "<f4"),
+                "xn2": _view(xn2.value, (T,), "<f4"),
+                "M": _view(M.value, (self.d_out, self.k), "<u2", torch.bfloat16)}
+
+    def timing_begin(self, max_forwards: int, stride: int = 1) -> None:
+        _check(load_library().sffn_gsi_timing_begin(self.h, int(max_forwards), int(stride)), "sffn_gsi_timing_begin")
+
+    def timing_end(self) -> dict:
+        return sffn_timing_end(self.h, "sffn_gsi_timing_end")
+
+    def close(self) -> None:
+        if getattr(self, "h", None) is not None and self.h.value:
+            _check(load_library().sffn_gsi_destroy(self.h), "sffn_gsi_destroy")
             self.h = None
 
     def __del__(self):

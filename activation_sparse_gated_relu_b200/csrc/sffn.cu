@@ -33,6 +33,7 @@
 #include "decode_fused.cuh"
 #include "tc_gate_persist.cuh"
 #include "gate_rows.cuh"
+#include "gsi.cuh"
 #include "rows_mma.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -46,10 +47,12 @@ namespace {
 constexpr int kNumSMsFallback = 148;
 constexpr int kMaxMarks = 12;
 enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
-                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_ROTATE_X, L_INPUT_SELECT, L_COUNT };
+                   L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_ROTATE_X, L_INPUT_SELECT,
+                   L_GSI_PROJECT, L_GSI_RESID, L_GSI_OUT, L_COUNT };
 const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
                                           "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
-                                          "fallback_f32", "decode_fused", "rotate_x", "input_select"};
+                                          "fallback_f32", "decode_fused", "rotate_x", "input_select",
+                                          "gsi_project", "gsi_resid", "gsi_out"};
 constexpr int kMaxTokensLimit = 16384;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -186,7 +189,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
-struct sffn_handle {
+// Per-kernel device timing (sffn_timing_begin / sffn_gsi_timing_begin): CUDA
+// events recorded on the launching stream before each kernel of every
+// stride-th forward and after its last one.
+struct KTiming {
+  bool tm_on = false;
+  int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
+  std::vector<cudaEvent_t> tm_ev;   // [tm_max][kMaxMarks + 1]
+  std::vector<int> tm_lab;          // [tm_max][kMaxMarks]
+  std::vector<int> tm_nk;           // [tm_max]
+};
+
+struct sffn_handle : KTiming {
   sffn_desc desc;
   int dev = 0, n_sm = kNumSMsFallback;
   int d = 0, F = 0, P = 0, R = 0, C = 0, maxT = 0, esize = 2;
@@ -257,17 +271,11 @@ struct sffn_handle {
   unsigned long long dec_wait_ns = SFFN_WAIT_LIMIT_NS;
   bool last_fused = false;     // the last forward was the single launch: its routing is the ovf flags
   uint32_t last_epoch = 0;
-  // per-kernel timing (sffn_timing_begin/end)
-  bool tm_on = false;
-  int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
-  std::vector<cudaEvent_t> tm_ev;   // [tm_max][kMaxMarks + 1]
-  std::vector<int> tm_lab;          // [tm_max][kMaxMarks]
-  std::vector<int> tm_nk;           // [tm_max]
 };
 
 namespace {
 
-void timing_free(sffn_handle* h);
+void timing_free(KTiming* h);
 
 void free_handle(sffn_handle* h) {
   if (!h) return;
@@ -302,7 +310,7 @@ bool dalloc(T** p, size_t bytes) {
   return true;
 }
 
-void tmark(sffn_handle* h, cudaStream_t st, int label) {
+void tmark(KTiming* h, cudaStream_t st, int label) {
   if (!h->tm_on || h->tm_cur < 0) return;
   const int f = h->tm_cur, i = h->tm_nk[f];
   if (i >= kMaxMarks) return;
@@ -311,7 +319,7 @@ void tmark(sffn_handle* h, cudaStream_t st, int label) {
   h->tm_nk[f] = i + 1;
 }
 
-void tmark_begin(sffn_handle* h) {
+void tmark_begin(KTiming* h) {
   h->tm_cur = -1;
   if (h->tm_on && (h->tm_seen++ % h->tm_stride) == 0 && h->tm_n < h->tm_max) {
     h->tm_cur = h->tm_n++;
@@ -319,14 +327,14 @@ void tmark_begin(sffn_handle* h) {
   }
 }
 
-void tmark_end(sffn_handle* h, cudaStream_t st) {
+void tmark_end(KTiming* h, cudaStream_t st) {
   if (!h->tm_on || h->tm_cur < 0) return;
   const int f = h->tm_cur;
   cudaEventRecord(h->tm_ev[(size_t)f * (kMaxMarks + 1) + h->tm_nk[f]], st);
   h->tm_cur = -1;
 }
 
-void timing_free(sffn_handle* h) {
+void timing_free(KTiming* h) {
   for (cudaEvent_t e : h->tm_ev)
     if (e) cudaEventDestroy(e);
   h->tm_ev.clear();
@@ -1114,7 +1122,7 @@ sffn_status sffn_forward(sffn_handle* h, const void* x, int T, float* out, void*
   return r;
 }
 
-sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards, int stride) {
+static sffn_status timing_begin_impl(KTiming* h, int max_forwards, int stride) {
   if (!h || max_forwards <= 0 || max_forwards > 100000 || stride <= 0) return SFFN_ERR_INVALID_ARG;
   timing_free(h);
   h->tm_stride = stride;
@@ -1136,8 +1144,8 @@ sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards, int stride) {
   return SFFN_OK;
 }
 
-sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], float* total_ms, int* launches,
-                            int* n_kernels) {
+static sffn_status timing_end_impl(KTiming* h, int max_kernels, char (*names)[32], float* total_ms,
+                                   int* launches, int* n_kernels) {
   if (!h || !h->tm_on) return SFFN_ERR_INVALID_ARG;
   double acc[L_COUNT] = {0};
   int cnt[L_COUNT] = {0};
@@ -1177,6 +1185,15 @@ sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], 
   timing_free(h);
   cudaGetLastError();
   return rs;
+}
+
+sffn_status sffn_timing_begin(sffn_handle* h, int max_forwards, int stride) {
+  return timing_begin_impl(h, max_forwards, stride);
+}
+
+sffn_status sffn_timing_end(sffn_handle* h, int max_kernels, char (*names)[32], float* total_ms, int* launches,
+                            int* n_kernels) {
+  return timing_end_impl(h, max_kernels, names, total_ms, launches, n_kernels);
 }
 
 sffn_status sffn_forward_host(sffn_handle* h, const void* x_host, int T, float* out_host, void* cuda_stream) {
@@ -1463,4 +1480,201 @@ extern "C" sffn_status sffn_lowrank_twell_noalloc_status(void* cuda_stream) {
 extern "C" sffn_status sffn_debug_noalloc_waits(unsigned wait_us) {
   g_na_hold_ns.store((unsigned long long)wait_us * 1000ull);
   return SFFN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Gated subspace linear layer ("Gated Subspace Inference for Transformer
+// Acceleration", sections 2.1 and 2.2): y = M·bf16(V_k^T x) for tokens whose
+// residual ratio ||x - V_k V_k^T x|| / ||x|| is below eps, y = W x for the
+// others, with M = bf16(W V_k) made at create time.
+struct sffn_gsi_handle : KTiming {
+  sffn_gsi_desc desc;
+  int dev = 0, n_sm = kNumSMsFallback;
+  void* arena = nullptr;
+  size_t arena_bytes = 0;
+  __nv_bfloat16* Vkt = nullptr;   // [k][d_in]
+  __nv_bfloat16* M = nullptr;     // [d_out][k]
+  float* g = nullptr;             // [maxT][k]
+  float* rn2 = nullptr;           // [maxT]
+  float* xn2 = nullptr;           // [maxT]
+  int* n_slow = nullptr;          // [4]
+  uint32_t* status = nullptr;     // [4]
+  int smem_proj = 0, smem_resid = 0, smem_out = 0, grid = 0;
+  int last_T = 0;
+};
+
+namespace {
+
+sffn_status gsi_validate(const sffn_gsi_desc* d) {
+  if (!d || !d->W || !d->Vk) return SFFN_ERR_INVALID_ARG;
+  if (d->d_in <= 0 || d->d_out <= 0 || d->k <= 0 || d->max_tokens <= 0) return SFFN_ERR_INVALID_ARG;
+  if (!(d->eps >= 0.0f) || std::isnan(d->eps)) return SFFN_ERR_INVALID_ARG;
+  if (!aligned16(d->W) || !aligned16(d->Vk)) return SFFN_ERR_INVALID_ARG;
+  if (d->k > d->d_in) return SFFN_ERR_INVALID_ARG;
+  if (d->d_in % 8 || d->k % 8 || d->d_in > 8192 || d->k > 512 || d->max_tokens > 64) return SFFN_ERR_UNSUPPORTED;
+  return SFFN_OK;
+}
+
+void gsi_free(sffn_gsi_handle* h) {
+  if (!h) return;
+  timing_free(h);
+  if (h->arena) cudaFree(h->arena);
+  delete h;
+}
+
+}  // namespace
+
+extern "C" sffn_status sffn_gsi_create(const sffn_gsi_desc* desc, void* cuda_stream, sffn_gsi_handle** out) {
+  if (!out) return SFFN_ERR_INVALID_ARG;
+  *out = nullptr;
+  sffn_status vs = gsi_validate(desc);
+  if (vs != SFFN_OK) return vs;
+  int dev = 0, major = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_NO_DEVICE;
+  }
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10) return SFFN_ERR_NO_DEVICE;
+  if (!get_encode()) return SFFN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  sffn_gsi_handle* h = new (std::nothrow) sffn_gsi_handle();
+  if (!h) return SFFN_ERR_ALLOC;
+  h->desc = *desc;
+  h->dev = dev;
+  h->n_sm = nsm > 0 ? nsm : kNumSMsFallback;
+  const size_t di = desc->d_in, dout = desc->d_out, k = desc->k, T = desc->max_tokens;
+  Arena ar;
+  auto plan = [&](Arena& a) {
+    a.take(&h->Vkt, k * di * 2);
+    a.take(&h->M, dout * k * 2);
+    a.take(&h->g, T * k * 4);
+    a.take(&h->rn2, T * 4);
+    a.take(&h->xn2, T * 4);
+    a.take(&h->n_slow, 16);
+    a.take(&h->status, 16);
+  };
+  plan(ar);
+  if (!dalloc(&h->arena, ar.size)) {
+    gsi_free(h);
+    return SFFN_ERR_ALLOC;
+  }
+  h->arena_bytes = ar.size;
+  ar.base = static_cast<uint8_t*>(h->arena);
+  ar.size = 0;
+  plan(ar);
+  h->grid = h->n_sm;
+  h->smem_proj = GSI_TC * (int)di * 2;
+  h->smem_resid = GSI_TC * (int)k * 4;
+  h->smem_out = GsiOutSmem::make((int)T, (int)k, (int)di).total;
+  cudaError_t e = cudaMemsetAsync(h->status, 0, 16, st);
+  e = e ? e : cudaMemsetAsync(h->n_slow, 0, 16, st);
+  e = e ? e : cudaFuncSetAttribute(k_gsi_project, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_proj);
+  e = e ? e : cudaFuncSetAttribute(k_gsi_resid, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_resid);
+  e = e ? e : cudaFuncSetAttribute(k_gsi_out, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_out);
+  e = e ? e : set_tc_attrs<EpiStoreBf16>();
+  // V_k^T, then the cached image M = bf16(W V_k): D[o][j] = sum_i W[o][i] V_k^T[j][i]
+  if (!e) {
+    k_transpose_bf16<<<dim3(cdiv(k, 32), cdiv(di, 32)), dim3(32, 8), 0, st>>>(
+        static_cast<const __nv_bfloat16*>(desc->Vk), h->Vkt, (int)di, (int)k);
+    e = cudaGetLastError();
+  }
+  if (!e) {
+    CUtensorMap mW, mV;
+    const int BNr = 256;
+    if (!make_map(&mW, desc->W, (long long)di, (long long)dout, 128) ||
+        !make_map(&mV, h->Vkt, (long long)di, (long long)k, BNr)) {
+      e = cudaErrorInvalidValue;
+    } else {
+      TcArgs ra{};
+      ra.n_phase = 1;
+      ra.kb_total[0] = cdiv(di, 64);
+      ra.n_rows = (int)k;
+      ra.status = h->status;
+      StoreParams sp{h->M, (long long)k, (int)dout, (int)k, 0};
+      e = launch_tc<EpiStoreBf16>(BNr, dim3(cdiv(dout, 128), cdiv(k, BNr), 1), st, mW, mV, mW, mV, ra, sp);
+    }
+  }
+  if (!e) e = cudaStreamSynchronize(st);
+  if (e) {
+    cudaGetLastError();
+    cudaStreamSynchronize(st);
+    gsi_free(h);
+    return SFFN_ERR_CUDA;
+  }
+  *out = h;
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_gsi_forward(sffn_gsi_handle* h, const void* x, int T, float* y, void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (T < 0 || T > h->desc.max_tokens) return SFFN_ERR_INVALID_ARG;
+  if (T == 0) return SFFN_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  GsiArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.Vkt = h->Vkt;
+  a.Vk = static_cast<const __nv_bfloat16*>(h->desc.Vk);
+  a.M = h->M;
+  a.W = static_cast<const __nv_bfloat16*>(h->desc.W);
+  a.g = h->g;
+  a.rn2 = h->rn2;
+  a.xn2 = h->xn2;
+  a.n_slow = h->n_slow;
+  a.y = y;
+  a.T = T;
+  a.d_in = h->desc.d_in;
+  a.d_out = h->desc.d_out;
+  a.k = h->desc.k;
+  a.eps2 = h->desc.eps * h->desc.eps;
+  h->last_T = T;
+  tmark_begin(h);
+  const int gp = std::max(1, std::min(h->grid, cdiv(a.k, GSI_THREADS / 32)));
+  tmark(h, st, L_GSI_PROJECT);
+  if (launch_pdl(k_gsi_project, dim3(gp), dim3(GSI_THREADS), (size_t)h->smem_proj, st, 1, a)) return SFFN_ERR_CUDA;
+  tmark(h, st, L_GSI_RESID);
+  if (launch_pdl(k_gsi_resid, dim3(h->grid), dim3(GSI_THREADS), (size_t)h->smem_resid, st, 1, a))
+    return SFFN_ERR_CUDA;
+  tmark(h, st, L_GSI_OUT);
+  if (launch_pdl(k_gsi_out, dim3(h->grid), dim3(GSI_THREADS), (size_t)h->smem_out, st, 1, a)) return SFFN_ERR_CUDA;
+  tmark_end(h, st);
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_gsi_destroy(sffn_gsi_handle* h) {
+  if (!h) return SFFN_OK;
+  cudaDeviceSynchronize();
+  gsi_free(h);
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_gsi_stats(sffn_gsi_handle* h, void* cuda_stream, int* n_slow) {
+  if (!h || !n_slow) return SFFN_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess ||
+      cudaMemcpy(n_slow, h->n_slow, 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_CUDA;
+  }
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_gsi_debug(sffn_gsi_handle* h, const float** g, const float** rn2, const float** xn2,
+                                      const void** M) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (g) *g = h->g;
+  if (rn2) *rn2 = h->rn2;
+  if (xn2) *xn2 = h->xn2;
+  if (M) *M = h->M;
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_gsi_timing_begin(sffn_gsi_handle* h, int max_forwards, int stride) {
+  return timing_begin_impl(h, max_forwards, stride);
+}
+
+extern "C" sffn_status sffn_gsi_timing_end(sffn_gsi_handle* h, int max_kernels, char (*names)[32], float* total_ms,
+                                           int* launches, int* n_kernels) {
+  return timing_end_impl(h, max_kernels, names, total_ms, launches, n_kernels);
 }

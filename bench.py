@@ -51,6 +51,7 @@ BENCH_SHAPES = {
     "tiny_fp32": (64, 1, 4, 1000),
     "wina_fullh_bf16": (32, 2, 16, 1000),
     "wina_input_bf16": (32, 2, 16, 1000),
+    "gsi_bf16": (8, 12, 16, 2000),
 }
 SPARSITY = {
     "decode_bf16": "relu gate bias -1.2816 (~90% zeros)",
@@ -61,6 +62,7 @@ SPARSITY = {
     "wina_fullh_bf16": "silu gate, WINA full-h top-k |a*u|*||w_down|| k=5018 (65% dropped)",
     "wina_input_bf16": "silu gate, orthogonal rotation V, input-side top-2048 of 4096, WINA top-k k=5018",
 }
+GSI_WORKLOADS = ("gsi_bf16",)
 TIMING_STRIDE = 8
 REF_BUDGET_S = 90.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
@@ -79,6 +81,9 @@ KERNEL_SOURCES = {
     "fallback_f32": ["simt.cuh", "ptx.cuh"],
     "rotate_x": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "input_select": ["simt.cuh", "ptx.cuh"],
+    "gsi_project": ["gsi.cuh", "ptx.cuh"],
+    "gsi_resid": ["gsi.cuh", "ptx.cuh"],
+    "gsi_out": ["gsi.cuh", "ptx.cuh"],
 }
 
 
@@ -491,10 +496,120 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
     }
 
 
+def gsi_work(wl, T: int, n_slow: float, any_slow: float) -> dict:
+    """Algorithmic bytes of the GSI forward's kernels (bf16 operands): the
+    basis twice (V_k^T rows for g, V_k rows for r), the cached image M, W only
+    when some token of the batch is slow (any_slow = the fraction of batches
+    with one), x, g and y.  FLOPs: 2 k d_in per token twice, 2 k d_out per
+    token and 2 d_in d_out per slow token."""
+    di, do, k = wl.d_in, wl.d_out, wl.k
+    xb = T * di * 2
+    return {
+        "gsi_project": {"bytes": k * di * 2 + xb + T * k * 4, "flops": 2 * T * k * di},
+        "gsi_resid": {"bytes": di * k * 2 + xb + T * k * 4, "flops": 2 * T * k * di},
+        "gsi_out": {"bytes": do * k * 2 + any_slow * do * di * 2 + T * k * 4 + T * do * 4,
+                    "flops": 2 * T * k * do + 2 * n_slow * di * do},
+    }
+
+
+def measure_gsi(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int) -> dict:
+    """The same protocol as `measure` for the gated subspace linear layer."""
+    import torch
+
+    import synth
+    from activation_sparse_gated_relu_b200 import GsiLinear
+
+    inp = synth.make_gsi_inputs(wl, T=T * NXB)
+    Vk = inp.Vk.to("cuda")
+    layers = []
+    for s in range(NS):
+        W = inp.W.to("cuda") if s == 0 else layers[0][0].clone()
+        Vs = Vk if s == 0 else Vk.clone()
+        layers.append((W, Vs, GsiLinear(W, Vs, wl.eps, max_tokens=T)))
+    xall = inp.x.to("cuda")
+    xb = [xall[i * T:(i + 1) * T].contiguous() for i in range(NXB)]
+    outs = [torch.empty((T, wl.d_out), dtype=torch.float32, device="cuda") for _ in range(NS)]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        layers[i % NS][2].forward(xb[i % NXB], outs[i % NS])
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    for _, _, lay in layers:
+        lay.timing_begin(steps // NS // TIMING_STRIDE + 2, TIMING_STRIDE)
+    clocks = ClockSampler(torch.cuda.current_device())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0.record(stream)
+    for i in range(steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed = ev0.elapsed_time(ev1)
+    kernels = {}
+    for _, _, lay in layers:
+        for name, (ms, n) in lay.timing_end().items():
+            a = kernels.setdefault(name, [0.0, 0])
+            a[0] += ms
+            a[1] += n
+    tot_ms, tot_units = aggregate(elapsed, float(T * steps), world)
+    slow = []
+    for b in range(NXB):
+        layers[0][2].forward(xb[b], outs[0])
+        slow.append(layers[0][2].n_slow())
+    n_slow = sum(slow) / NXB
+    any_slow = sum(1 for v in slow if v) / NXB
+    works = gsi_work(wl, T, n_slow, any_slow)
+    for _, _, lay in layers:
+        lay.close()
+    peaks, peak_src = load_peaks()
+    per = {k: (v[0] / v[1] if v[1] else 0.0) for k, v in kernels.items()}
+    dom = max(per, key=lambda k: kernels[k][0]) if per else None
+    roof = None
+    if dom in works and per[dom] > 0:
+        roof = roofline_of(works[dom], per[dom], peaks, peak_src)
+        roof.update({"kernel": dom, "traffic": None, "ms_per_launch": round(per[dom], 5)})
+    total_kernel_ms = sum(v[0] for v in kernels.values())
+    kern_out = {}
+    for k in kernels:
+        e = {"ms_per_launch": round(per[k], 5), "launches": kernels[k][1],
+             "share": round(kernels[k][0] / total_kernel_ms, 4) if total_kernel_ms else None}
+        if k in works and per[k] > 0:
+            r = roofline_of(works[k], per[k], peaks, peak_src)
+            e.update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
+        kern_out[k] = e
+    bytes_step = sum(w["bytes"] for w in works.values())
+    step_s = tot_ms * 1e-3 / steps
+    dense_bytes = wl.d_out * wl.d_in * 2
+    return {
+        "value": round(tot_units / (tot_ms * 1e-3), 1), "ms_per_step": round(tot_ms / steps, 5),
+        "steps": steps, "warmup": warmup,
+        "hbm_gbs_step": round(bytes_step * world / step_s / 1e9, 1),
+        "hbm_frac_step": round(bytes_step * world / step_s / 1e9 / peaks["hbm_gbs"], 4),
+        "algorithmic_bytes_per_step": int(bytes_step),
+        "slow_tokens_per_step": n_slow, "batches_with_a_slow_token": any_slow,
+        "weight_read_ratio_vs_dense": round(dense_bytes / bytes_step, 2),
+        "roofline": roof, "kernels": kern_out, "gpu_launches": 3 * steps, "clocks": clk,
+        "config": {"workload": f"{wl.name}: linear d_in={wl.d_in} -> d_out={wl.d_out}, basis k={wl.k}, "
+                               f"eps={wl.eps}, tokens={T} bf16, residual ratio lognormal(median "
+                               f"{wl.rho_med}, sigma {wl.rho_sigma})",
+                   "tokens_per_step": T,
+                   "l2": f"inputs larger than L2: {NS} rotating weight sets (each: W, V_k, M) and {NXB} x batches"},
+        "dtype": "bf16", "unit": UNIT,
+    }
+
+
 # the other configurations, measured after the headline in the same default
 # run: (workload, tokens per forward)
 EXTRA_WORKLOADS = [("decode_bf16", 1), ("decode_bf16", 4), ("lopa_bf16", 32), ("wina_bf16", 32),
-                   ("prefill_bf16", 4096), ("tiny_fp32", 64), ("wina_fullh_bf16", 32), ("wina_input_bf16", 32)]
+                   ("prefill_bf16", 4096), ("tiny_fp32", 64), ("wina_fullh_bf16", 32), ("wina_input_bf16", 32),
+                   ("gsi_bf16", 8)]
 EXTRA_MIN_STEPS = 200
 EXTRA_MAX_S = 2.0
 
@@ -520,6 +635,24 @@ def run_ours(args) -> None:
     barrier(world)
     load_library()
 
+    if args.workload in GSI_WORKLOADS:
+        T, _, NXB, _ = BENCH_SHAPES[args.workload]
+        T = args.tokens or T
+        m = measure_gsi(synth.GSI_WORKLOADS[args.workload], T, args.weight_sets, NXB, args.steps, args.warmup,
+                        world)
+        if rank == 0:
+            line = {"metric": METRIC, "value": m.pop("value"), "unit": UNIT, "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.pop("ms_per_step"),
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                    "data": "synthetic (seeded low-rank activations and N(0,1/d_in) weights)",
+                    "config": m.pop("config")}
+            m.pop("steps"), m.pop("warmup"), m.pop("unit"), m.pop("dtype")
+            line.update(m)
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     wl = synth.WORKLOADS[args.workload]
     T, _, NXB, _ = BENCH_SHAPES[args.workload]
     T = args.tokens or T
@@ -572,8 +705,16 @@ def run_ours(args) -> None:
     if world == 1 and not args.no_workloads and args.workload == DEFAULT_WORKLOAD and not args.tokens:
         workloads = {}
         for name, Tw in EXTRA_WORKLOADS:
-            wlx = synth.WORKLOADS[name]
             _, NSx, NXBx, _ = BENCH_SHAPES[name]
+            if name in GSI_WORKLOADS:
+                wlg = synth.GSI_WORKLOADS[name]
+                probe = measure_gsi(wlg, Tw, NSx, NXBx, 24, max(args.warmup, 3), world)
+                ksteps = max(EXTRA_MIN_STEPS, min(5000, int(EXTRA_MAX_S / (probe["ms_per_step"] * 1e-3))))
+                ksteps -= ksteps % NSx
+                workloads[f"{name}@T={Tw}"] = measure_gsi(wlg, Tw, NSx, NXBx, ksteps, max(args.warmup, 3), world)
+                torch.cuda.empty_cache()
+                continue
+            wlx = synth.WORKLOADS[name]
             # a bounded run: at least EXTRA_MIN_STEPS forwards, about
             # EXTRA_MAX_S seconds at most, from a short probe of the step time
             probe = measure(wlx, Tw, NSx, NXBx, 10, max(args.warmup, 3), world, None)
@@ -623,6 +764,9 @@ def run_reference(args) -> None:
     if rank != 0:
         return
     import synth
+    if args.workload in GSI_WORKLOADS:
+        run_reference_gsi(args)
+        return
     wl = synth.WORKLOADS[args.workload]
     T, _, NXB, _ = BENCH_SHAPES[args.workload]
     T = args.tokens or T
@@ -642,6 +786,35 @@ def run_reference(args) -> None:
         "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_gsi(args) -> None:
+    """The reference arm for the GSI workload: oracle.gsi.forward on the host."""
+    import numpy as np
+
+    import oracle.gsi
+    import synth
+    wl = synth.GSI_WORKLOADS[args.workload]
+    T = args.tokens or BENCH_SHAPES[args.workload][0]
+    inp = synth.make_gsi_inputs(wl, T=T * 4)
+    x, W, Vk = (t.double().numpy() for t in (inp.x, inp.W, inp.Vk))
+    n, t0 = 0, time.perf_counter()
+    while n < max(1, args.steps):
+        oracle.gsi.forward(np.ascontiguousarray(x[(n * T) % x.shape[0]:][:T]), W, Vk, wl.eps, wl.dtype)
+        n += 1
+        if time.perf_counter() - t0 > REF_BUDGET_S:
+            break
+    el = time.perf_counter() - t0
+    v = n * T / el
+    line = {"metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": 1, "steps": n,
+            "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: d_in={wl.d_in} d_out={wl.d_out} k={wl.k} eps={wl.eps} tokens={T}"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": f"{n} fp64 oracle GSI forwards of {T} tokens"},
+            "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 

@@ -311,6 +311,64 @@ sffn_status sffn_lowrank_twell_noalloc_status(void* cuda_stream);
  * Process-wide; always SFFN_OK. */
 sffn_status sffn_debug_noalloc_waits(unsigned wait_us);
 
+/* ------------------------------------------------------------------------
+ * Gated subspace linear layer (GSI).  Source: "Gated Subspace Inference for
+ * Transformer Acceleration" (technical summary), section 2.1 (core
+ * decomposition) and section 2.2 (gated residual pass-through).  For a linear
+ * layer y = W x and an orthonormal basis V_k of the activation subspace:
+ *
+ *     g = V_k^T x,   r = x - V_k g,   M = W V_k  (cached at create time),
+ *     y = M·bf16(g)   if ||r||^2 < eps^2·||x||^2   (fast path: reads only M)
+ *     y = W x         otherwise                   (slow path: reads W)
+ *
+ * so a token on the fast path is off by at most ||W||_2·eps·||x|| (the
+ * page's Theorem 4) and a token on the slow path is exact.
+ *
+ * Layouts (device pointers, 16-byte aligned, row-major): W [d_out][d_in] bf16
+ * (PyTorch Linear weight), V_k [d_in][k] bf16 (orthonormal columns: the
+ * caller's calibrated basis), x [T][d_in] bf16, y [T][d_out] fp32.  M is
+ * stored as bf16(W V_k), and g is rounded to bf16 for the fast path; the
+ * residual and the norms use the fp32 g.  The test is strict (rho = eps takes
+ * the slow path) and x = 0 takes the slow path.
+ * Limits: d_in % 8 == 0 and <= 8192; k % 8 == 0, k <= 512 and k <= d_in;
+ * max_tokens <= 64 (decode batches); otherwise SFFN_ERR_UNSUPPORTED.
+ * Ownership as for sffn_create: W and V_k are borrowed for the handle's life;
+ * the handle owns M (d_out·k·2 bytes), V_k^T and its workspace. */
+typedef struct sffn_gsi_desc {
+  int d_in, d_out, k, max_tokens;
+  float eps;            /* residual-ratio threshold (>= 0; 0: every token slow) */
+  const void* W;        /* [d_out][d_in] bf16 */
+  const void* Vk;       /* [d_in][k] bf16    */
+} sffn_gsi_desc;
+
+typedef struct sffn_gsi_handle sffn_gsi_handle;
+
+/* Validate, allocate, transpose V_k and compute M on `cuda_stream`, then
+ * synchronise it.  On error *out is NULL and nothing stays allocated. */
+sffn_status sffn_gsi_create(const sffn_gsi_desc* desc, void* cuda_stream, sffn_gsi_handle** out);
+
+/* y = GSI(x) for T tokens (0 <= T <= max_tokens; 0: nothing launched),
+ * asynchronously on `cuda_stream`: three kernels (projection, residual norms,
+ * routed output).  y is fully overwritten.  One forward at a time per handle. */
+sffn_status sffn_gsi_forward(sffn_gsi_handle* h, const void* x, int T, float* y, void* cuda_stream);
+
+sffn_status sffn_gsi_destroy(sffn_gsi_handle* h);
+
+/* Number of tokens of the last forward that took the slow path (synchronises
+ * the stream). */
+sffn_status sffn_gsi_stats(sffn_gsi_handle* h, void* cuda_stream, int* n_slow);
+
+/* Device views of the last forward (valid until the next forward or destroy):
+ * g fp32 [T][k], sum of r^2 and of x^2 per token fp32 [T], and the cached
+ * image M bf16 [d_out][k].  Test use. */
+sffn_status sffn_gsi_debug(sffn_gsi_handle* h, const float** g, const float** rn2, const float** xn2,
+                           const void** M);
+
+/* Per-kernel device timing of the GSI forward, as sffn_timing_begin/end. */
+sffn_status sffn_gsi_timing_begin(sffn_gsi_handle* h, int max_forwards, int stride);
+sffn_status sffn_gsi_timing_end(sffn_gsi_handle* h, int max_kernels, char (*names)[32], float* total_ms,
+                                int* launches, int* n_kernels);
+
 /* Library version string. */
 const char* sffn_version(void);
 

@@ -176,3 +176,23 @@ def test_binding_rejects_host_or_misshaped_weights():
         B.SparseFFN(W, W, W_gate=W)                   # host weights
     with pytest.raises(ValueError, match="give either W_gate"):
         B.SparseFFN(W, W)                             # no gate at all
+
+
+def test_gsi_create_rejects_bad_descriptors(lib):
+    fake = 0x7F0000000000
+    def desc(**kw):
+        d = B.sffn_gsi_desc()
+        d.d_in, d.d_out, d.k, d.max_tokens, d.eps, d.W, d.Vk = 4096, 16384, 256, 8, 0.1, fake, fake
+        for k, v in kw.items():
+            setattr(d, k, v)
+        return d
+    h = ctypes.c_void_p()
+    for kw, want in [({"d_in": 4100}, B.SFFN_ERR_UNSUPPORTED), ({"k": 513}, B.SFFN_ERR_UNSUPPORTED),
+                     ({"max_tokens": 65}, B.SFFN_ERR_UNSUPPORTED), ({"k": 0}, B.SFFN_ERR_INVALID_ARG),
+                     ({"eps": -1.0}, B.SFFN_ERR_INVALID_ARG), ({"W": None}, B.SFFN_ERR_INVALID_ARG),
+                     ({"W": fake + 8}, B.SFFN_ERR_INVALID_ARG), ({"d_in": 64, "k": 128}, B.SFFN_ERR_INVALID_ARG)]:
+        d = desc(**kw)
+        assert lib.sffn_gsi_create(ctypes.byref(d), None, ctypes.byref(h)) == want, kw
+        assert not h.value
+    assert lib.sffn_gsi_create(ctypes.byref(desc()), None, ctypes.byref(h)) == B.SFFN_ERR_NO_DEVICE
+    assert lib.sffn_gsi_destroy(None) == B.SFFN_OK
