@@ -109,7 +109,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_gsi_destroy.restype = st
     lib.sffn_gsi_stats.argtypes = [vp, vp, ctypes.POINTER(ip)]
     lib.sffn_gsi_stats.restype = st
-    lib.sffn_gsi_debug.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+    lib.sffn_gsi_debug.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(ip),
                                    ctypes.POINTER(vp)]
     lib.sffn_gsi_debug.restype = st
     lib.sffn_gsi_timing_begin.argtypes = [vp, ip, ip]
@@ -445,11 +445,12 @@ class GsiLinear:
     def debug(self, T: int) -> dict:
         import torch
         vp = ctypes.c_void_p
-        g, rn2, xn2, M = vp(), vp(), vp(), vp()
-        _check(load_library().sffn_gsi_debug(self.h, ctypes.byref(g), ctypes.byref(rn2), ctypes.byref(xn2),
+        g, part, M = vp(), vp(), vp()
+        n = ctypes.c_int()
+        _check(load_library().sffn_gsi_debug(self.h, ctypes.byref(g), ctypes.byref(part), ctypes.byref(n),
                                              ctypes.byref(M)), "sffn_gsi_debug")
-        return {"g": _view(g.value, (T, self.k), "<f4"), "rn2": _view(rn2.value, (T,), "<f4"),
-                "xn2": _view(xn2.value, (T,), "<f4"),
+        p = _view(part.value, (n.value, self.max_tokens, 2), "<f4")[:, :T, :]
+        return {"g": _view(g.value, (T, self.k), "<f4"), "rn2": p[:, :, 0].sum(0), "xn2": p[:, :, 1].sum(0),
                 "M": _view(M.value, (self.d_out, self.k), "<u2", torch.bfloat16)}
 
     def timing_begin(self, max_forwards: int, stride: int = 1) -> None:

@@ -1494,12 +1494,13 @@ struct sffn_gsi_handle : KTiming {
   size_t arena_bytes = 0;
   __nv_bfloat16* Vkt = nullptr;   // [k][d_in]
   __nv_bfloat16* M = nullptr;     // [d_out][k]
-  float* g = nullptr;             // [maxT][k]
-  float* rn2 = nullptr;           // [maxT]
-  float* xn2 = nullptr;           // [maxT]
+  float* g[2] = {nullptr, nullptr};   // [maxT][k], alternate forwards (one is cleared for the next)
+  float* part = nullptr;          // [grid_resid][maxT][2]
   int* n_slow = nullptr;          // [4]
   uint32_t* status = nullptr;     // [4]
-  int smem_proj = 0, smem_resid = 0, smem_out = 0, grid = 0;
+  int smem_proj = 0, smem_resid = 0, smem_out = 0;
+  int grid_proj = 0, grid_resid = 0, grid_out = 0;
+  int parity = 0;
   int last_T = 0;
 };
 
@@ -1546,12 +1547,15 @@ extern "C" sffn_status sffn_gsi_create(const sffn_gsi_desc* desc, void* cuda_str
   h->n_sm = nsm > 0 ? nsm : kNumSMsFallback;
   const size_t di = desc->d_in, dout = desc->d_out, k = desc->k, T = desc->max_tokens;
   Arena ar;
+  h->grid_proj = cdiv(di, GSI_PROJ_ROWS);
+  h->grid_resid = cdiv(di, GSI_RESID_ROWS);
+  h->grid_out = h->n_sm;
   auto plan = [&](Arena& a) {
     a.take(&h->Vkt, k * di * 2);
     a.take(&h->M, dout * k * 2);
-    a.take(&h->g, T * k * 4);
-    a.take(&h->rn2, T * 4);
-    a.take(&h->xn2, T * 4);
+    a.take(&h->g[0], T * k * 4);
+    a.take(&h->g[1], T * k * 4);
+    a.take(&h->part, (size_t)h->grid_resid * T * 2 * 4);
     a.take(&h->n_slow, 16);
     a.take(&h->status, 16);
   };
@@ -1564,12 +1568,13 @@ extern "C" sffn_status sffn_gsi_create(const sffn_gsi_desc* desc, void* cuda_str
   ar.base = static_cast<uint8_t*>(h->arena);
   ar.size = 0;
   plan(ar);
-  h->grid = h->n_sm;
-  h->smem_proj = GSI_TC * (int)di * 2;
+  h->smem_proj = (GSI_THREADS / ((int)k / 2)) * GSI_TC * (int)k * 4;
   h->smem_resid = GSI_TC * (int)k * 4;
   h->smem_out = GsiOutSmem::make((int)T, (int)k, (int)di).total;
   cudaError_t e = cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->n_slow, 0, 16, st);
+  e = e ? e : cudaMemsetAsync(h->g[0], 0, T * k * 4, st);
+  e = e ? e : cudaMemsetAsync(h->g[1], 0, T * k * 4, st);
   e = e ? e : cudaFuncSetAttribute(k_gsi_project, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_proj);
   e = e ? e : cudaFuncSetAttribute(k_gsi_resid, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_resid);
   e = e ? e : cudaFuncSetAttribute(k_gsi_out, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem_out);
@@ -1615,31 +1620,34 @@ extern "C" sffn_status sffn_gsi_forward(sffn_gsi_handle* h, const void* x, int T
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   GsiArgs a{};
   a.x = static_cast<const __nv_bfloat16*>(x);
-  a.Vkt = h->Vkt;
   a.Vk = static_cast<const __nv_bfloat16*>(h->desc.Vk);
   a.M = h->M;
   a.W = static_cast<const __nv_bfloat16*>(h->desc.W);
-  a.g = h->g;
-  a.rn2 = h->rn2;
-  a.xn2 = h->xn2;
+  a.g = h->g[h->parity];
+  a.g_next = h->g[h->parity ^ 1];
+  a.part = h->part;
   a.n_slow = h->n_slow;
   a.y = y;
   a.T = T;
   a.d_in = h->desc.d_in;
   a.d_out = h->desc.d_out;
   a.k = h->desc.k;
+  a.maxT = h->desc.max_tokens;
+  a.grid_resid = h->grid_resid;
   a.eps2 = h->desc.eps * h->desc.eps;
   h->last_T = T;
   tmark_begin(h);
-  const int gp = std::max(1, std::min(h->grid, cdiv(a.k, GSI_THREADS / 32)));
   tmark(h, st, L_GSI_PROJECT);
-  if (launch_pdl(k_gsi_project, dim3(gp), dim3(GSI_THREADS), (size_t)h->smem_proj, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_gsi_project, dim3(h->grid_proj), dim3(GSI_THREADS), (size_t)h->smem_proj, st, 1, a))
+    return SFFN_ERR_CUDA;
   tmark(h, st, L_GSI_RESID);
-  if (launch_pdl(k_gsi_resid, dim3(h->grid), dim3(GSI_THREADS), (size_t)h->smem_resid, st, 1, a))
+  if (launch_pdl(k_gsi_resid, dim3(h->grid_resid), dim3(GSI_THREADS), (size_t)h->smem_resid, st, 1, a))
     return SFFN_ERR_CUDA;
   tmark(h, st, L_GSI_OUT);
-  if (launch_pdl(k_gsi_out, dim3(h->grid), dim3(GSI_THREADS), (size_t)h->smem_out, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_gsi_out, dim3(h->grid_out), dim3(GSI_THREADS), (size_t)h->smem_out, st, 1, a))
+    return SFFN_ERR_CUDA;
   tmark_end(h, st);
+  h->parity ^= 1;   // the launches went out: the next forward sums into the other buffer
   return SFFN_OK;
 }
 
@@ -1660,12 +1668,12 @@ extern "C" sffn_status sffn_gsi_stats(sffn_gsi_handle* h, void* cuda_stream, int
   return SFFN_OK;
 }
 
-extern "C" sffn_status sffn_gsi_debug(sffn_gsi_handle* h, const float** g, const float** rn2, const float** xn2,
+extern "C" sffn_status sffn_gsi_debug(sffn_gsi_handle* h, const float** g, const float** part, int* n_part,
                                       const void** M) {
   if (!h) return SFFN_ERR_INVALID_ARG;
-  if (g) *g = h->g;
-  if (rn2) *rn2 = h->rn2;
-  if (xn2) *xn2 = h->xn2;
+  if (g) *g = h->g[h->parity ^ 1];   // the last forward's buffer
+  if (part) *part = h->part;
+  if (n_part) *n_part = h->grid_resid;
   if (M) *M = h->M;
   return SFFN_OK;
 }

@@ -359,9 +359,10 @@ sffn_status sffn_gsi_destroy(sffn_gsi_handle* h);
 sffn_status sffn_gsi_stats(sffn_gsi_handle* h, void* cuda_stream, int* n_slow);
 
 /* Device views of the last forward (valid until the next forward or destroy):
- * g fp32 [T][k], sum of r^2 and of x^2 per token fp32 [T], and the cached
- * image M bf16 [d_out][k].  Test use. */
-sffn_status sffn_gsi_debug(sffn_gsi_handle* h, const float** g, const float** rn2, const float** xn2,
+ * g fp32 [T][k]; the per-CTA partial sums of r^2 and x^2, fp32
+ * [n_part][T][2] (a token's ||r||^2 and ||x||^2 are their sums over the
+ * n_part CTAs); and the cached image M bf16 [d_out][k].  Test use. */
+sffn_status sffn_gsi_debug(sffn_gsi_handle* h, const float** g, const float** part, int* n_part,
                            const void** M);
 
 /* Per-kernel device timing of the GSI forward, as sffn_timing_begin/end. */
