@@ -336,3 +336,67 @@ def make_gsi_inputs(wl: GsiWorkload, T: Optional[int] = None) -> GsiInputs:
         Wa = _grid(Wa, _grid_exp(std))
     return GsiInputs(wl, _to_dtype(xa, wl.dtype), _to_dtype(Wa, wl.dtype),
                      _to_dtype(Vk.astype(np.float32), wl.dtype), rho)
+
+
+# ---------------------------------------------------------------------------
+# mixture of LoPA-gated sparse experts
+# ---------------------------------------------------------------------------
+TID_MOE_WR = 30
+
+
+@dataclass(frozen=True)
+class MoeWorkload:
+    """E experts, each the low-rank-gated sparse FFN of ``lopa_bf16``'s
+    recipe (its own seeded weights), a router W_r ~ N(0, 1/d) [E][d] and
+    x ~ N(0, 1): the router logits are about N(0, 1), so tokens spread over
+    the experts at random."""
+    name: str
+    d_model: int
+    d_ff: int
+    rank: int
+    experts: int
+    top_k: int
+    tokens: int
+    bias: Optional[float] = -1.2816
+    threshold: float = 0.0
+    tile_capacity: int = 32
+    exact_grid: bool = False
+    seed: int = 0
+
+    def with_(self, **kw) -> "MoeWorkload":
+        return replace(self, **kw)
+
+    def expert_workload(self, e: int) -> Workload:
+        return Workload(f"{self.name}.e{e}", self.d_model, self.d_ff, self.tokens, rank=self.rank,
+                        bias=self.bias, threshold=self.threshold, tile_capacity=self.tile_capacity,
+                        exact_grid=self.exact_grid, seed=self.seed * 1009 + 17 + e)
+
+
+# Mixtral's layout (8 experts, 2 per token) on the decode shapes, LoPA gate
+# rank d/8, about 90 % zeros per expert
+MOE_WORKLOADS = {
+    "moe_lopa_bf16": MoeWorkload("moe_lopa_bf16", 4096, 14336, 512, 8, 2, 8),
+}
+
+
+@dataclass
+class MoeInputs:
+    wl: MoeWorkload
+    x: torch.Tensor                 # [T][d]
+    W_r: torch.Tensor               # [E][d]
+    experts: list                   # per expert: dict(A, B, W_up, W_down, bias)
+
+
+def make_moe_inputs(wl: MoeWorkload, T: Optional[int] = None) -> MoeInputs:
+    T = wl.tokens if T is None else T
+    xa = _normal(wl.seed, TID_X, (T, wl.d_model), 1.0)
+    std = 1.0 / math.sqrt(wl.d_model)
+    Wr = _normal(wl.seed, TID_MOE_WR, (wl.experts, wl.d_model), std)
+    if wl.exact_grid:
+        xa = _grid(xa, 4)
+        Wr = _grid(Wr, _grid_exp(std))
+    ex = []
+    for e in range(wl.experts):
+        inp = make_inputs(wl.expert_workload(e), weights_only=True)
+        ex.append({"A": inp.A, "B": inp.B, "W_up": inp.W_up, "W_down": inp.W_down, "bias": inp.bias})
+    return MoeInputs(wl, _to_dtype(xa, "bf16"), _to_dtype(Wr, "bf16"), ex)
