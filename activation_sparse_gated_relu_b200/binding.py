@@ -43,6 +43,15 @@ class sffn_gsi_desc(ctypes.Structure):
                 ("Vk", ctypes.c_void_p)]
 
 
+class sffn_moe_desc(ctypes.Structure):
+    _fields_ = [("n_experts", ctypes.c_int), ("top_k", ctypes.c_int), ("d_model", ctypes.c_int),
+                ("d_ff", ctypes.c_int), ("rank", ctypes.c_int), ("max_tokens", ctypes.c_int),
+                ("tile_capacity", ctypes.c_int), ("threshold", ctypes.c_float), ("W_router", ctypes.c_void_p),
+                ("A", ctypes.POINTER(ctypes.c_void_p)), ("B", ctypes.POINTER(ctypes.c_void_p)),
+                ("W_up", ctypes.POINTER(ctypes.c_void_p)), ("W_down", ctypes.POINTER(ctypes.c_void_p)),
+                ("gate_bias", ctypes.POINTER(ctypes.c_void_p))]
+
+
 class sffn_stats(ctypes.Structure):
     _fields_ = [("n_overflow", ctypes.c_int), ("n_launches", ctypes.c_int), ("path", ctypes.c_int),
                 ("epoch", ctypes.c_uint), ("launch_attrs", ctypes.c_uint)]
@@ -117,6 +126,23 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_gsi_timing_end.argtypes = [vp, ip, vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ip),
                                         ctypes.POINTER(ip)]
     lib.sffn_gsi_timing_end.restype = st
+    lib.sffn_moe_create.argtypes = [ctypes.POINTER(sffn_moe_desc), vp, ctypes.POINTER(vp)]
+    lib.sffn_moe_create.restype = st
+    lib.sffn_moe_forward.argtypes = [vp, vp, ip, vp, vp]
+    lib.sffn_moe_forward.restype = st
+    lib.sffn_moe_destroy.argtypes = [vp]
+    lib.sffn_moe_destroy.restype = st
+    lib.sffn_moe_expert.argtypes = [vp, ip, ctypes.POINTER(vp)]
+    lib.sffn_moe_expert.restype = st
+    lib.sffn_moe_debug.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp)]
+    lib.sffn_moe_debug.restype = st
+    lib.sffn_moe_read_status.argtypes = [vp, vp]
+    lib.sffn_moe_read_status.restype = st
+    lib.sffn_moe_timing_begin.argtypes = [vp, ip, ip]
+    lib.sffn_moe_timing_begin.restype = st
+    lib.sffn_moe_timing_end.argtypes = [vp, ip, vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ip),
+                                        ctypes.POINTER(ip)]
+    lib.sffn_moe_timing_end.restype = st
     lib.sffn_version.argtypes = []
     lib.sffn_version.restype = ctypes.c_char_p
     _lib = lib
@@ -462,6 +488,108 @@ class GsiLinear:
     def close(self) -> None:
         if getattr(self, "h", None) is not None and self.h.value:
             _check(load_library().sffn_gsi_destroy(self.h), "sffn_gsi_destroy")
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class MoeFFN:
+    """Mixture of LoPA-gated sparse experts over device tensors.
+
+    experts: a list of dicts with A [d][rank], B [rank][d_ff], W_up and W_down
+    [d_ff][d] (bf16) and bias [d_ff] fp32 (<= 0) or None; W_router [E][d]."""
+
+    def __init__(self, W_router, experts: list, top_k: int, *, threshold: float = 0.0,
+                 tile_capacity: int = 32, max_tokens: int = 8, stream: Optional[int] = None):
+        import torch
+        self.h = None
+        E = len(experts)
+        if E == 0:
+            raise ValueError("at least one expert")
+        F, d = experts[0]["W_up"].shape
+        r = experts[0]["A"].shape[1]
+        _check_tensor(W_router, "W_router", torch.bfloat16, (E, d), True)
+        for e, ex in enumerate(experts):
+            _check_tensor(ex["A"], f"A[{e}]", torch.bfloat16, (d, r), True)
+            _check_tensor(ex["B"], f"B[{e}]", torch.bfloat16, (r, F), True)
+            _check_tensor(ex["W_up"], f"W_up[{e}]", torch.bfloat16, (F, d), True)
+            _check_tensor(ex["W_down"], f"W_down[{e}]", torch.bfloat16, (F, d), True)
+            if ex.get("bias") is not None:
+                _check_tensor(ex["bias"], f"bias[{e}]", torch.float32, (F,), True)
+        self._keep = [W_router] + [t for ex in experts for t in ex.values() if t is not None]
+        self.d_model, self.d_ff, self.n_experts, self.top_k, self.max_tokens = d, F, E, top_k, max_tokens
+        arr = lambda key: (ctypes.c_void_p * E)(*[  # noqa: E731
+            (ex[key].data_ptr() if ex.get(key) is not None else None) for ex in experts])
+        self._arrays = {k: arr(k) for k in ("A", "B", "W_up", "W_down", "bias")}
+        desc = sffn_moe_desc()
+        desc.n_experts, desc.top_k, desc.d_model, desc.d_ff, desc.rank = E, top_k, d, F, r
+        desc.max_tokens, desc.tile_capacity, desc.threshold = max_tokens, tile_capacity, float(threshold)
+        desc.W_router = W_router.data_ptr()
+        cast = lambda a: ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))  # noqa: E731
+        desc.A, desc.B = cast(self._arrays["A"]), cast(self._arrays["B"])
+        desc.W_up, desc.W_down = cast(self._arrays["W_up"]), cast(self._arrays["W_down"])
+        desc.gate_bias = cast(self._arrays["bias"]) if all(ex.get("bias") is not None for ex in experts) else None
+        h = ctypes.c_void_p()
+        _check(load_library().sffn_moe_create(ctypes.byref(desc), ctypes.c_void_p(SparseFFN._stream(stream)),
+                                              ctypes.byref(h)), "sffn_moe_create")
+        self.h = h
+
+    def forward(self, x, out=None, stream: Optional[int] = None):
+        import torch
+        if not isinstance(x, torch.Tensor) or x.dim() != 2:
+            raise ValueError("x must be a [T][d_model] tensor")
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T = {T} exceeds max_tokens = {self.max_tokens}")
+        _check_tensor(x, "x", torch.bfloat16, (T, self.d_model), True)
+        if out is None:
+            out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
+        _check_tensor(out, "out", torch.float32, (T, self.d_model), True)
+        _check(load_library().sffn_moe_forward(self.h, ctypes.c_void_p(x.data_ptr()), T,
+                                               ctypes.c_void_p(out.data_ptr()),
+                                               ctypes.c_void_p(SparseFFN._stream(stream))), "sffn_moe_forward")
+        return out
+
+    __call__ = forward
+
+    def routing(self, T: int) -> dict:
+        vp = ctypes.c_void_p
+        sel, w, lg = vp(), vp(), vp()
+        _check(load_library().sffn_moe_debug(self.h, ctypes.byref(sel), ctypes.byref(w), ctypes.byref(lg)),
+               "sffn_moe_debug")
+        return {"sel": _view(sel.value, (T, self.top_k), "<i4"), "w": _view(w.value, (T, self.top_k), "<f4"),
+                "logits": _view(lg.value, (T, self.n_experts), "<f4")}
+
+    def expert_twell(self, e: int, T: int) -> dict:
+        """Copies of expert e's TwELL records for its last block of T rows."""
+        import torch
+        eh = ctypes.c_void_p()
+        _check(load_library().sffn_moe_expert(self.h, int(e), ctypes.byref(eh)), "sffn_moe_expert")
+        view = SparseFFN.__new__(SparseFFN)      # a non-owning view: the MoE handle owns the expert
+        view.h, view.dtype, view._torch_dtype = None, "bf16", torch.bfloat16
+        view.d_model, view.d_ff, view.max_tokens = self.d_model, self.d_ff, self.max_tokens
+        view.h = eh
+        try:
+            return view.twell(T)
+        finally:
+            view.h = None
+
+    def read_status(self, stream: Optional[int] = None) -> int:
+        return load_library().sffn_moe_read_status(self.h, ctypes.c_void_p(SparseFFN._stream(stream)))
+
+    def timing_begin(self, max_forwards: int, stride: int = 1) -> None:
+        _check(load_library().sffn_moe_timing_begin(self.h, int(max_forwards), int(stride)), "sffn_moe_timing_begin")
+
+    def timing_end(self) -> dict:
+        return sffn_timing_end(self.h, "sffn_moe_timing_end")
+
+    def close(self) -> None:
+        if getattr(self, "h", None) is not None and self.h.value:
+            _check(load_library().sffn_moe_destroy(self.h), "sffn_moe_destroy")
             self.h = None
 
     def __del__(self):

@@ -34,6 +34,7 @@
 #include "tc_gate_persist.cuh"
 #include "gate_rows.cuh"
 #include "gsi.cuh"
+#include "moe.cuh"
 #include "rows_mma.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -48,11 +49,11 @@ constexpr int kNumSMsFallback = 148;
 constexpr int kMaxMarks = 12;
 enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
                    L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_ROTATE_X, L_INPUT_SELECT,
-                   L_GSI_PROJECT, L_GSI_RESID, L_GSI_OUT, L_COUNT };
+                   L_GSI_PROJECT, L_GSI_RESID, L_GSI_OUT, L_MOE_ROUTE, L_MOE_COMBINE, L_COUNT };
 const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
                                           "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
                                           "fallback_f32", "decode_fused", "rotate_x", "input_select",
-                                          "gsi_project", "gsi_resid", "gsi_out"};
+                                          "gsi_project", "gsi_resid", "gsi_out", "moe_route", "moe_combine"};
 constexpr int kMaxTokensLimit = 16384;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1685,4 +1686,246 @@ extern "C" sffn_status sffn_gsi_timing_begin(sffn_gsi_handle* h, int max_forward
 extern "C" sffn_status sffn_gsi_timing_end(sffn_gsi_handle* h, int max_kernels, char (*names)[32], float* total_ms,
                                            int* launches, int* n_kernels) {
   return timing_end_impl(h, max_kernels, names, total_ms, launches, n_kernels);
+}
+
+// ---------------------------------------------------------------------------
+// Mixture of LoPA-gated sparse experts (see moe.cuh): a router launch, every
+// expert's own sparse forward on its block of T rows (x where the token is
+// routed to it, zero elsewhere), a combine launch.
+struct sffn_moe_handle : KTiming {
+  int E = 0, top_k = 0, d = 0, F = 0, maxT = 0;
+  const void* Wr = nullptr;
+  std::vector<sffn_handle*> experts;
+  void* arena = nullptr;
+  __nv_bfloat16* xe = nullptr;    // [E][maxT][d]
+  float* ye = nullptr;            // [E][maxT][d]
+  int* sel = nullptr;             // [maxT][top_k]
+  float* w = nullptr;             // [maxT][top_k]
+  float* logits = nullptr;        // [maxT][E]
+  int last_T = 0;
+};
+
+namespace {
+void moe_free(sffn_moe_handle* h) {
+  if (!h) return;
+  for (sffn_handle* e : h->experts) sffn_destroy(e);
+  timing_free(h);
+  if (h->arena) cudaFree(h->arena);
+  delete h;
+}
+}  // namespace
+
+extern "C" sffn_status sffn_moe_create(const sffn_moe_desc* md, void* cuda_stream, sffn_moe_handle** out) {
+  if (!out) return SFFN_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!md || !md->W_router || !md->A || !md->B || !md->W_up || !md->W_down) return SFFN_ERR_INVALID_ARG;
+  if (md->n_experts < 1 || md->top_k < 1 || md->top_k > md->n_experts) return SFFN_ERR_INVALID_ARG;
+  if (md->n_experts > MOE_MAX_E || md->top_k > MOE_MAX_K) return SFFN_ERR_UNSUPPORTED;
+  if (md->rank <= 0 || md->d_model <= 0 || md->max_tokens <= 0) return SFFN_ERR_INVALID_ARG;
+  if (!aligned16(md->W_router)) return SFFN_ERR_INVALID_ARG;
+  if (md->d_model % 8 || md->max_tokens > 1024) return SFFN_ERR_UNSUPPORTED;
+  // unrouted rows are zero: they must keep nothing, so the gate bias is <= 0
+  for (int e = 0; e < md->n_experts; ++e) {
+    sffn_desc d{};
+    d.d_model = md->d_model;
+    d.d_ff = md->d_ff;
+    d.max_tokens = md->max_tokens;
+    d.rank = md->rank;
+    d.dtype = SFFN_BF16;
+    d.mode = SFFN_MODE_RELU_THRESHOLD;
+    d.act = SFFN_ACT_RELU;
+    d.threshold = md->threshold;
+    d.tile_capacity = md->tile_capacity;
+    d.A = md->A[e];
+    d.B = md->B[e];
+    d.W_up = md->W_up[e];
+    d.W_down = md->W_down[e];
+    d.gate_bias = md->gate_bias ? md->gate_bias[e] : nullptr;
+    const sffn_status vs = validate(&d);
+    if (vs != SFFN_OK) return vs;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SFFN_ERR_NO_DEVICE;
+  }
+  int major = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major != 10) return SFFN_ERR_NO_DEVICE;
+  sffn_moe_handle* h = new (std::nothrow) sffn_moe_handle();
+  if (!h) return SFFN_ERR_ALLOC;
+  h->E = md->n_experts;
+  h->top_k = md->top_k;
+  h->d = md->d_model;
+  h->F = md->d_ff;
+  h->maxT = md->max_tokens;
+  h->Wr = md->W_router;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (md->gate_bias) {   // a positive bias would keep neurons of the zero rows: checked on the host copy
+    std::vector<float> b((size_t)md->d_ff);
+    for (int e = 0; e < md->n_experts; ++e) {
+      if (!md->gate_bias[e]) continue;
+      if (cudaMemcpy(b.data(), md->gate_bias[e], b.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        moe_free(h);
+        return SFFN_ERR_CUDA;
+      }
+      for (float v : b)
+        if (!(v <= 0.0f)) {
+          moe_free(h);
+          return SFFN_ERR_UNSUPPORTED;
+        }
+    }
+  }
+  for (int e = 0; e < h->E; ++e) {
+    sffn_desc d{};
+    d.d_model = md->d_model;
+    d.d_ff = md->d_ff;
+    d.max_tokens = md->max_tokens;
+    d.rank = md->rank;
+    d.dtype = SFFN_BF16;
+    d.mode = SFFN_MODE_RELU_THRESHOLD;
+    d.act = SFFN_ACT_RELU;
+    d.threshold = md->threshold;
+    d.tile_capacity = md->tile_capacity;
+    d.A = md->A[e];
+    d.B = md->B[e];
+    d.W_up = md->W_up[e];
+    d.W_down = md->W_down[e];
+    d.gate_bias = md->gate_bias ? md->gate_bias[e] : nullptr;
+    sffn_handle* eh = nullptr;
+    const sffn_status cs = sffn_create(&d, cuda_stream, &eh);
+    if (cs != SFFN_OK) {
+      moe_free(h);
+      return cs;
+    }
+    h->experts.push_back(eh);
+  }
+  const size_t E = h->E, T = h->maxT, dd = h->d, K = h->top_k;
+  Arena ar;
+  auto plan = [&](Arena& a) {
+    a.take(&h->xe, E * T * dd * 2);
+    a.take(&h->ye, E * T * dd * 4);
+    a.take(&h->sel, T * K * 4);
+    a.take(&h->w, T * K * 4);
+    a.take(&h->logits, T * E * 4);
+  };
+  plan(ar);
+  if (!dalloc(&h->arena, ar.size)) {
+    moe_free(h);
+    return SFFN_ERR_ALLOC;
+  }
+  ar.base = static_cast<uint8_t*>(h->arena);
+  ar.size = 0;
+  plan(ar);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    moe_free(h);
+    return SFFN_ERR_CUDA;
+  }
+  *out = h;
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_moe_forward(sffn_moe_handle* h, const void* x, int T, float* out, void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (T < 0 || T > h->maxT) return SFFN_ERR_INVALID_ARG;
+  if (T == 0) return SFFN_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  h->last_T = T;
+  tmark_begin(h);
+  MoeRouteArgs ra{static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(h->Wr), h->xe,
+                  h->sel, h->w, h->logits, T, h->d, h->E, h->top_k};
+  tmark(h, st, L_MOE_ROUTE);
+  if (launch_pdl(k_moe_route, dim3(T), dim3(256), 0, st, 1, ra)) return SFFN_ERR_CUDA;
+  tmark_end(h, st);
+  for (int e = 0; e < h->E; ++e) {
+    const sffn_status s = sffn_forward(h->experts[e], h->xe + (size_t)e * T * h->d, T,
+                                       h->ye + (size_t)e * T * h->d, cuda_stream);
+    if (s != SFFN_OK) return s;
+  }
+  tmark_begin(h);
+  MoeCombineArgs ca{h->ye, h->sel, h->w, out, T, h->d, h->top_k};
+  tmark(h, st, L_MOE_COMBINE);
+  if (launch_pdl(k_moe_combine, dim3(std::max(1, cdiv(h->d / 4, 256)), T), dim3(256), 0, st, 1, ca))
+    return SFFN_ERR_CUDA;
+  tmark_end(h, st);
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_moe_destroy(sffn_moe_handle* h) {
+  if (!h) return SFFN_OK;
+  cudaDeviceSynchronize();
+  moe_free(h);
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_moe_expert(sffn_moe_handle* h, int e, sffn_handle** expert) {
+  if (!h || !expert || e < 0 || e >= h->E) return SFFN_ERR_INVALID_ARG;
+  *expert = h->experts[e];
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_moe_debug(sffn_moe_handle* h, const int** sel, const float** w, const float** logits) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (sel) *sel = h->sel;
+  if (w) *w = h->w;
+  if (logits) *logits = h->logits;
+  return SFFN_OK;
+}
+
+extern "C" sffn_status sffn_moe_read_status(sffn_moe_handle* h, void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  sffn_status worst = SFFN_OK;
+  for (sffn_handle* e : h->experts) {
+    const sffn_status s = sffn_read_status(e, cuda_stream);
+    if (s != SFFN_OK && worst == SFFN_OK) worst = s;
+  }
+  return worst;
+}
+
+extern "C" sffn_status sffn_moe_timing_begin(sffn_moe_handle* h, int max_forwards, int stride) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  sffn_status s = timing_begin_impl(h, 2 * max_forwards, stride);
+  for (size_t e = 0; e < h->experts.size() && s == SFFN_OK; ++e) s = timing_begin_impl(h->experts[e], max_forwards, stride);
+  return s;
+}
+
+extern "C" sffn_status sffn_moe_timing_end(sffn_moe_handle* h, int max_kernels, char (*names)[32], float* total_ms,
+                                           int* launches, int* n_kernels) {
+  // the router and combine launches, then every expert's kernels, added by label
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  std::vector<std::vector<char>> nm;
+  std::vector<float> ms;
+  std::vector<int> ln;
+  auto collect = [&](KTiming* t) -> sffn_status {
+    char tn[L_COUNT][32];
+    float tm[L_COUNT];
+    int tl[L_COUNT], n = 0;
+    const sffn_status s = timing_end_impl(t, L_COUNT, tn, tm, tl, &n);
+    if (s != SFFN_OK) return s;
+    for (int i = 0; i < std::min(n, (int)L_COUNT); ++i) {
+      size_t j = 0;
+      while (j < nm.size() && std::strcmp(nm[j].data(), tn[i]) != 0) ++j;
+      if (j == nm.size()) {
+        nm.emplace_back(tn[i], tn[i] + 32);
+        ms.push_back(0.f);
+        ln.push_back(0);
+      }
+      ms[j] += tm[i];
+      ln[j] += tl[i];
+    }
+    return SFFN_OK;
+  };
+  sffn_status s = collect(h);
+  for (size_t e = 0; e < h->experts.size() && s == SFFN_OK; ++e) s = collect(h->experts[e]);
+  const int n = (int)nm.size();
+  for (int i = 0; i < std::min(n, max_kernels); ++i) {
+    if (names) std::memcpy(names[i], nm[i].data(), 32);
+    if (total_ms) total_ms[i] = ms[i];
+    if (launches) launches[i] = ln[i];
+  }
+  if (n_kernels) *n_kernels = n;
+  return s;
 }

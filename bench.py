@@ -52,6 +52,7 @@ BENCH_SHAPES = {
     "wina_fullh_bf16": (32, 2, 16, 1000),
     "wina_input_bf16": (32, 2, 16, 1000),
     "gsi_bf16": (8, 12, 16, 2000),
+    "moe_lopa_bf16": (8, 1, 16, 400),
 }
 SPARSITY = {
     "decode_bf16": "relu gate bias -1.2816 (~90% zeros)",
@@ -63,6 +64,7 @@ SPARSITY = {
     "wina_input_bf16": "silu gate, orthogonal rotation V, input-side top-2048 of 4096, WINA top-k k=5018",
 }
 GSI_WORKLOADS = ("gsi_bf16",)
+MOE_WORKLOADS = ("moe_lopa_bf16",)
 TIMING_STRIDE = 8
 REF_BUDGET_S = 90.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
@@ -84,6 +86,8 @@ KERNEL_SOURCES = {
     "gsi_project": ["gsi.cuh", "ptx.cuh"],
     "gsi_resid": ["gsi.cuh", "ptx.cuh"],
     "gsi_out": ["gsi.cuh", "ptx.cuh"],
+    "moe_route": ["moe.cuh", "ptx.cuh"],
+    "moe_combine": ["moe.cuh", "ptx.cuh"],
 }
 
 
@@ -605,11 +609,92 @@ def measure_gsi(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: i
     }
 
 
+def measure_moe(wl, T: int, NXB: int, steps: int, warmup: int, world: int) -> dict:
+    """The same protocol as `measure` for the mixture of LoPA-gated experts
+    (one weight set: the E experts' weights are far larger than L2)."""
+    import torch
+
+    import synth
+    from activation_sparse_gated_relu_b200 import SFFN_OK, MoeFFN
+
+    inp = synth.make_moe_inputs(wl, T=T * NXB)
+    dev = lambda t: None if t is None else t.to("cuda")  # noqa: E731
+    ex = [{k: dev(v) for k, v in e.items()} for e in inp.experts]
+    moe = MoeFFN(dev(inp.W_r), ex, wl.top_k, threshold=wl.threshold, tile_capacity=wl.tile_capacity,
+                 max_tokens=T)
+    xall = dev(inp.x)
+    xb = [xall[i * T:(i + 1) * T].contiguous() for i in range(NXB)]
+    out = torch.empty((T, wl.d_model), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        moe.forward(xb[i % NXB], out)
+    torch.cuda.synchronize()
+    assert moe.read_status() == SFFN_OK
+    moe.timing_begin(steps // TIMING_STRIDE + 2, TIMING_STRIDE)
+    clocks = ClockSampler(torch.cuda.current_device())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0.record(stream)
+    for i in range(steps):
+        moe.forward(xb[i % NXB], out)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    elapsed = ev0.elapsed_time(ev1)
+    kernels = {k: list(v) for k, v in moe.timing_end().items()}
+    assert moe.read_status() == SFFN_OK
+    tot_ms, tot_units = aggregate(elapsed, float(T * steps), world)
+    # realised work: every expert reads its low-rank gate, then the W_up and
+    # W_down rows its routed tokens keep (zero rows keep nothing)
+    d, F, r, E = wl.d_model, wl.d_ff, wl.rank, wl.experts
+    rows = []
+    for b in range(NXB):
+        moe.forward(xb[b], out)
+        u = 0
+        for e in range(E):
+            tw = moe.expert_twell(e, T)
+            n = torch.minimum(tw["count"].long(), torch.tensor(wl.tile_capacity, device="cuda"))
+            used = torch.arange(wl.tile_capacity, device="cuda")[None, None, :] < n[:, :, None]
+            u += int(torch.unique(tw["idx"].long()[used]).numel())
+        rows.append(u)
+    moe.close()
+    union = sum(rows) / NXB
+    bytes_step = E * d * 2 + E * (d * r + r * F) * 2 + union * 2 * d * 2 + T * d * 2 + T * d * 4
+    peaks, peak_src = load_peaks()
+    step_s = tot_ms * 1e-3 / steps
+    per = {k: (v[0] / v[1] if v[1] else 0.0) for k, v in kernels.items()}
+    total_kernel_ms = sum(v[0] for v in kernels.values())
+    kern_out = {k: {"ms_per_launch": round(per[k], 5), "launches": kernels[k][1],
+                    "share": round(kernels[k][0] / total_kernel_ms, 4) if total_kernel_ms else None}
+                for k in kernels}
+    dom = max(per, key=lambda k: kernels[k][0]) if per else None
+    return {
+        "value": round(tot_units / (tot_ms * 1e-3), 1), "ms_per_step": round(tot_ms / steps, 5),
+        "steps": steps, "warmup": warmup,
+        "hbm_gbs_step": round(bytes_step * world / step_s / 1e9, 1),
+        "hbm_frac_step": round(bytes_step * world / step_s / 1e9 / peaks["hbm_gbs"], 4),
+        "algorithmic_bytes_per_step": int(bytes_step), "expert_rows_kept_per_step": union,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(bytes_step / step_s / 1e9, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(bytes_step / step_s / 1e9 / peaks["hbm_gbs"], 4), "traffic": None,
+                     "scope": "whole forward (router, every expert's kernels, combine)"},
+        "kernels": kern_out, "clocks": clk,
+        "config": {"workload": f"{wl.name}: {E} experts, top-{wl.top_k}, d_model={d} d_ff={F} rank={r} "
+                               f"tokens={T} bf16, relu gate bias {wl.bias} (~90% zeros per expert)",
+                   "tokens_per_step": T,
+                   "l2": f"inputs larger than L2: {E} experts' weights ({E * (2 * F * d + d * r + r * F) * 2 / 1e9:.2f} GB)"},
+        "dtype": "bf16", "unit": UNIT,
+    }
+
+
 # the other configurations, measured after the headline in the same default
 # run: (workload, tokens per forward)
 EXTRA_WORKLOADS = [("decode_bf16", 1), ("decode_bf16", 4), ("lopa_bf16", 32), ("wina_bf16", 32),
                    ("prefill_bf16", 4096), ("tiny_fp32", 64), ("wina_fullh_bf16", 32), ("wina_input_bf16", 32),
-                   ("gsi_bf16", 8)]
+                   ("gsi_bf16", 8), ("moe_lopa_bf16", 8)]
 EXTRA_MIN_STEPS = 200
 EXTRA_MAX_S = 2.0
 
@@ -635,16 +720,19 @@ def run_ours(args) -> None:
     barrier(world)
     load_library()
 
-    if args.workload in GSI_WORKLOADS:
+    if args.workload in GSI_WORKLOADS or args.workload in MOE_WORKLOADS:
         T, _, NXB, _ = BENCH_SHAPES[args.workload]
         T = args.tokens or T
-        m = measure_gsi(synth.GSI_WORKLOADS[args.workload], T, args.weight_sets, NXB, args.steps, args.warmup,
-                        world)
+        if args.workload in GSI_WORKLOADS:
+            m = measure_gsi(synth.GSI_WORKLOADS[args.workload], T, args.weight_sets, NXB, args.steps,
+                            args.warmup, world)
+        else:
+            m = measure_moe(synth.MOE_WORKLOADS[args.workload], T, NXB, args.steps, args.warmup, world)
         if rank == 0:
             line = {"metric": METRIC, "value": m.pop("value"), "unit": UNIT, "n_gpus": world,
                     "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.pop("ms_per_step"),
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                    "data": "synthetic (seeded low-rank activations and N(0,1/d_in) weights)",
+                    "data": "synthetic (seeded Gaussian or low-rank activations, N(0,1/fan_in) weights)",
                     "config": m.pop("config")}
             m.pop("steps"), m.pop("warmup"), m.pop("unit"), m.pop("dtype")
             line.update(m)
@@ -706,6 +794,13 @@ def run_ours(args) -> None:
         workloads = {}
         for name, Tw in EXTRA_WORKLOADS:
             _, NSx, NXBx, _ = BENCH_SHAPES[name]
+            if name in MOE_WORKLOADS:
+                wlm = synth.MOE_WORKLOADS[name]
+                probe = measure_moe(wlm, Tw, NXBx, 16, max(args.warmup, 3), world)
+                ksteps = max(EXTRA_MIN_STEPS, min(2000, int(EXTRA_MAX_S / (probe["ms_per_step"] * 1e-3))))
+                workloads[f"{name}@T={Tw}"] = measure_moe(wlm, Tw, NXBx, ksteps, max(args.warmup, 3), world)
+                torch.cuda.empty_cache()
+                continue
             if name in GSI_WORKLOADS:
                 wlg = synth.GSI_WORKLOADS[name]
                 probe = measure_gsi(wlg, Tw, NSx, NXBx, 24, max(args.warmup, 3), world)
@@ -764,8 +859,8 @@ def run_reference(args) -> None:
     if rank != 0:
         return
     import synth
-    if args.workload in GSI_WORKLOADS:
-        run_reference_gsi(args)
+    if args.workload in GSI_WORKLOADS or args.workload in MOE_WORKLOADS:
+        run_reference_other(args)
         return
     wl = synth.WORKLOADS[args.workload]
     T, _, NXB, _ = BENCH_SHAPES[args.workload]
@@ -789,19 +884,33 @@ def run_reference(args) -> None:
     print(json.dumps(line), flush=True)
 
 
-def run_reference_gsi(args) -> None:
-    """The reference arm for the GSI workload: oracle.gsi.forward on the host."""
+def run_reference_other(args) -> None:
+    """The reference arm for the GSI and MoE workloads: their fp64 oracles on
+    the host, one forward of the workload's token batch per step."""
     import numpy as np
 
     import oracle.gsi
+    import oracle.moe
     import synth
-    wl = synth.GSI_WORKLOADS[args.workload]
     T = args.tokens or BENCH_SHAPES[args.workload][0]
-    inp = synth.make_gsi_inputs(wl, T=T * 4)
-    x, W, Vk = (t.double().numpy() for t in (inp.x, inp.W, inp.Vk))
+    if args.workload in GSI_WORKLOADS:
+        wl = synth.GSI_WORKLOADS[args.workload]
+        inp = synth.make_gsi_inputs(wl, T=T * 4)
+        x, W, Vk = (t.double().numpy() for t in (inp.x, inp.W, inp.Vk))
+        run = lambda xt: oracle.gsi.forward(xt, W, Vk, wl.eps, wl.dtype)  # noqa: E731
+        desc = f"{wl.name}: d_in={wl.d_in} d_out={wl.d_out} k={wl.k} eps={wl.eps} tokens={T}"
+    else:
+        wl = synth.MOE_WORKLOADS[args.workload]
+        inp = synth.make_moe_inputs(wl, T=T * 4)
+        x = inp.x.double().numpy()
+        Wr = inp.W_r.double().numpy()
+        ex = [{k: (None if v is None else v.double().numpy()) for k, v in e.items()} for e in inp.experts]
+        run = lambda xt: oracle.moe.forward(xt, Wr, ex, wl.top_k, threshold=wl.threshold,  # noqa: E731
+                                            C=wl.tile_capacity)
+        desc = f"{wl.name}: {wl.experts} experts top-{wl.top_k} d_model={wl.d_model} d_ff={wl.d_ff} tokens={T}"
     n, t0 = 0, time.perf_counter()
     while n < max(1, args.steps):
-        oracle.gsi.forward(np.ascontiguousarray(x[(n * T) % x.shape[0]:][:T]), W, Vk, wl.eps, wl.dtype)
+        run(np.ascontiguousarray(x[(n * T) % x.shape[0]:][:T]))
         n += 1
         if time.perf_counter() - t0 > REF_BUDGET_S:
             break
@@ -810,10 +919,9 @@ def run_reference_gsi(args) -> None:
     line = {"metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": 1, "steps": n,
             "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: d_in={wl.d_in} d_out={wl.d_out} k={wl.k} eps={wl.eps} tokens={T}"},
-            "impl": "reference",
+            "config": {"workload": desc}, "impl": "reference",
             "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                             "sample": f"{n} fp64 oracle GSI forwards of {T} tokens"},
+                             "sample": f"{n} fp64 oracle forwards of {T} tokens"},
             "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

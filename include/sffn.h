@@ -370,6 +370,69 @@ sffn_status sffn_gsi_timing_begin(sffn_gsi_handle* h, int max_forwards, int stri
 sffn_status sffn_gsi_timing_end(sffn_gsi_handle* h, int max_kernels, char (*names)[32], float* total_ms,
                                 int* launches, int* n_kernels);
 
+/* ------------------------------------------------------------------------
+ * Mixture of LoPA-gated sparse experts.  Source: "Meta FAIR and Inria's LoPA
+ * Gating Hits 3.31x Real GPU Speedup for LLM Inference", section "Model
+ * Casting and Quality at 90% Sparsity" (LoPA gating carries over to MoE
+ * layers whose experts share the gated FFN structure) and section "How LoPA
+ * Gating Restructures FFN Computation" (the low-rank gate).  The page gives
+ * no routing rule; this library takes Mixtral's:
+ *
+ *     l[t][e] = <W_r[e], x_t>;  S_t = the top_k experts by l (ties to the
+ *     smaller index);  w[t][e] = softmax of l[t][S_t];
+ *     y_t = sum_{e in S_t} w[t][e] · FFN_e(x_t),
+ *
+ * each FFN_e the relu-threshold forward of sffn_forward with a low-rank gate
+ * (A_e, B_e), its own W_up, W_down and bias.  A forward is a router launch,
+ * each expert's sparse forward on a block of T rows (x_t where t is routed to
+ * the expert, zero elsewhere: a zero row keeps no neuron, so the gate biases
+ * must be <= 0, checked at create time) and a combine launch.
+ *
+ * Layouts as for sffn_desc; W_router [n_experts][d_model] bf16; the per-expert
+ * pointer arrays are HOST arrays of n_experts device pointers (copied).
+ * Limits: n_experts <= 64, top_k <= 8, max_tokens <= 1024. */
+typedef struct sffn_moe_desc {
+  int n_experts, top_k;
+  int d_model, d_ff, rank, max_tokens, tile_capacity;
+  float threshold;
+  const void* W_router;
+  const void* const* A;             /* [n_experts] -> [d_model][rank]   */
+  const void* const* B;             /* [n_experts] -> [rank][d_ff]      */
+  const void* const* W_up;          /* [n_experts] -> [d_ff][d_model]   */
+  const void* const* W_down;        /* [n_experts] -> [d_ff][d_model]   */
+  const float* const* gate_bias;    /* [n_experts] -> [d_ff], or NULL   */
+} sffn_moe_desc;
+
+typedef struct sffn_moe_handle sffn_moe_handle;
+
+/* Create one sparse-FFN handle per expert and the routing workspace.
+ * SFFN_ERR_UNSUPPORTED for a positive gate bias (see above). */
+sffn_status sffn_moe_create(const sffn_moe_desc* desc, void* cuda_stream, sffn_moe_handle** out);
+
+/* y = MoE(x) for T tokens (device x [T][d_model] bf16, out [T][d_model]
+ * fp32), asynchronously on cuda_stream; no host synchronisation. */
+sffn_status sffn_moe_forward(sffn_moe_handle* h, const void* x, int T, float* out, void* cuda_stream);
+
+sffn_status sffn_moe_destroy(sffn_moe_handle* h);
+
+/* The handle of expert e (owned by the MoE handle): its TwELL and stats views
+ * describe its last block of T rows. */
+sffn_status sffn_moe_expert(sffn_moe_handle* h, int e, sffn_handle** expert);
+
+/* Device views of the last forward's routing: sel int32 [T][top_k], weights
+ * fp32 [T][top_k] and logits fp32 [T][n_experts].  Test use. */
+sffn_status sffn_moe_debug(sffn_moe_handle* h, const int** sel, const float** w, const float** logits);
+
+/* Synchronise and return (and clear) the first device-side error any expert
+ * recorded (as sffn_read_status). */
+sffn_status sffn_moe_read_status(sffn_moe_handle* h, void* cuda_stream);
+
+/* Per-kernel device timing of the MoE forward (router, combine and every
+ * expert's kernels, added by label), as sffn_timing_begin/end. */
+sffn_status sffn_moe_timing_begin(sffn_moe_handle* h, int max_forwards, int stride);
+sffn_status sffn_moe_timing_end(sffn_moe_handle* h, int max_kernels, char (*names)[32], float* total_ms,
+                                int* launches, int* n_kernels);
+
 /* Library version string. */
 const char* sffn_version(void);
 
