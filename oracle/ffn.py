@@ -95,6 +95,10 @@ def round_fp32(a: np.ndarray) -> np.ndarray:
 
 
 def round_operand(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Round to the operand dtype: "bf16", "fp32", or "fp64" (no rounding: the
+    exact-arithmetic variant the finite-difference pins of the backward use)."""
+    if dtype == "fp64":
+        return np.asarray(a, dtype=np.float64)
     return round_bf16(a) if dtype == "bf16" else round_fp32(a)
 
 
