@@ -23,6 +23,7 @@ SFFN_PATH_AUTO, SFFN_PATH_ROWS, SFFN_PATH_TILES = 0, 1, 2
 SFFN_FLAG_DEBUG_GATE = 1
 SFFN_FLAG_SEPARATE = 2
 SFFN_FLAG_COOPERATIVE = 4
+SFFN_FLAG_BACKWARD = 8
 
 
 class sffn_desc(ctypes.Structure):
@@ -99,6 +100,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.sffn_debug_keep.restype = st
     lib.sffn_debug_gate.argtypes = [vp, ctypes.POINTER(vp)]
     lib.sffn_debug_gate.restype = st
+    lib.sffn_backward.argtypes = [vp, vp, vp, ip, vp, vp, vp, vp, vp, vp]
+    lib.sffn_backward.restype = st
     lib.sffn_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
     lib.sffn_workspace_bytes.restype = st
     lib.sffn_debug_norms.argtypes = [vp, ctypes.POINTER(vp)]
@@ -264,7 +267,7 @@ class SparseFFN:
                  mode: str = "relu_threshold", act: str = "relu", threshold: float = 0.0,
                  k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
                  debug_gate: bool = False, separate: bool = False, cooperative: bool = False,
-                 input_k: int = 0, V=None, stream: Optional[int] = None):
+                 input_k: int = 0, V=None, backward: bool = False, stream: Optional[int] = None):
         import torch
         self.h = None
         self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias, V) if t is not None]
@@ -303,7 +306,7 @@ class SparseFFN:
         desc.tile_capacity = int(tile_capacity)
         desc.path = _PATH[path]
         desc.flags = ((SFFN_FLAG_DEBUG_GATE if debug_gate else 0) | (SFFN_FLAG_SEPARATE if separate else 0)
-                      | (SFFN_FLAG_COOPERATIVE if cooperative else 0))
+                      | (SFFN_FLAG_COOPERATIVE if cooperative else 0) | (SFFN_FLAG_BACKWARD if backward else 0))
         ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         desc.W_gate, desc.A, desc.B = ptr(W_gate), ptr(A), ptr(B)
         desc.W_up, desc.W_down, desc.gate_bias = ptr(W_up), ptr(W_down), ptr(bias)
@@ -340,6 +343,31 @@ class SparseFFN:
         return out
 
     __call__ = forward
+
+    def backward(self, x, dy, *, dx=None, dW_gate=None, dW_up=None, dW_down=None, d_bias=None,
+                 with_bias: bool = True, stream: Optional[int] = None) -> dict:
+        """Gradients of the last forward for upstream dy (fp32 [T][d_model]):
+        {dx, dW_gate, dW_up, dW_down, d_bias} as fp32 device tensors."""
+        import torch
+        T = self._check_io(x, None, cuda=True)
+        _check_tensor(dy, "dy", torch.float32, (T, self.d_model), True)
+        z = lambda shape: torch.empty(shape, dtype=torch.float32, device=x.device)  # noqa: E731
+        dx = z((T, self.d_model)) if dx is None else dx
+        dW_gate = z((self.d_ff, self.d_model)) if dW_gate is None else dW_gate
+        dW_up = z((self.d_ff, self.d_model)) if dW_up is None else dW_up
+        dW_down = z((self.d_ff, self.d_model)) if dW_down is None else dW_down
+        if with_bias and d_bias is None:
+            d_bias = z((self.d_ff,))
+        for name, t, shape in (("dx", dx, (T, self.d_model)), ("dW_gate", dW_gate, (self.d_ff, self.d_model)),
+                               ("dW_up", dW_up, (self.d_ff, self.d_model)),
+                               ("dW_down", dW_down, (self.d_ff, self.d_model))):
+            _check_tensor(t, name, torch.float32, shape, True)
+        if d_bias is not None:
+            _check_tensor(d_bias, "d_bias", torch.float32, (self.d_ff,), True)
+        p = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else None)  # noqa: E731
+        _check(load_library().sffn_backward(self.h, p(x), p(dy), T, p(dx), p(dW_gate), p(dW_up), p(dW_down),
+                                            p(d_bias), ctypes.c_void_p(self._stream(stream))), "sffn_backward")
+        return {"dx": dx, "dW_gate": dW_gate, "dW_up": dW_up, "dW_down": dW_down, "d_bias": d_bias}
 
     def forward_host(self, x_host, out_host=None, stream: Optional[int] = None):
         import torch

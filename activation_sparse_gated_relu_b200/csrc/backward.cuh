@@ -1,0 +1,380 @@
+// Backward pass of the activation-sparse gated FFN (relu-threshold selection,
+// dense gate): training over the sparse format ("Sparser, Faster, Lighter
+// Transformer Language Models", news article, section "Hybrid 應對非均勻稀疏").
+// With the forward's selection held fixed and the rounding of the stored
+// value passed straight through, for upstream dy:
+//     dh = dy W_down^T (kept), du = dh·v, dg = dh·u·sigma'(g),
+//     dW_down = h^T dy, dW_up = du^T x, dW_gate = dg^T x, db = sum_t dg,
+//     dx = du W_up + dg W_gate.
+// Only the kept (token, neuron) pairs are touched.  They come from the
+// forward's keep masks (kmask [T][P][4] words: every token's full kept set,
+// overflow tokens included), in two orders:
+//   token-major (CSR): pair p of token t sits at rowptr[t] + its rank among
+//     the token's kept neurons (ascending);
+//   neuron-major (CSC): for neuron j, the CSR positions of its pairs in token
+//     order.
+// Kernels, in launch order:
+//   k_bwd_rows     per token: kept count, per-word rank prefix; zeroes dx of
+//                  tokens split over several chunks
+//   k_bwd_scan     (one CTA) CSR offsets and the chunk table: each token's kept
+//                  list cut into chunks of BW_CH pairs
+//   k_bwd_token    persistent: CTAs take chunks from a counter; per chunk
+//                  the token's x and dy rows in shared memory, the chunk's
+//                  neurons listed, warp = neuron: g, u, dh (three row dot
+//                  products), then du, dg, h per pair (stored in CSR order)
+//                  and du·W_up[j] + dg·W_gate[j] into the warp's dx row;
+//                  the warps' rows summed into dx (added when the token has
+//                  several chunks)
+//   k_bwd_colcount thread = neuron: pairs per neuron; k_bwd_scan2 offsets
+//   k_bwd_colfill  thread = neuron: the CSR positions of its pairs
+//   k_bwd_neuron   CTA = neuron: dW_gate, dW_up and dW_down rows and db
+//                  from its pairs (x and dy rows gathered), no atomics
+#pragma once
+
+#include "epilogues.cuh"
+#include "ptx.cuh"
+#include "simt.cuh"
+
+namespace sffn {
+
+constexpr int BW_THREADS = 256;
+constexpr int BW_CH = 256;           // kept pairs per chunk of the token pass
+
+struct BwdArgs {
+  const __nv_bfloat16* x;       // [T][d]
+  const float* dy;              // [T][d]
+  const __nv_bfloat16* W_gate;  // [F][d]
+  const __nv_bfloat16* W_up;    // [F][d]
+  const __nv_bfloat16* W_down;  // [F][d]
+  const float* bias;            // [F] or null
+  const uint32_t* kmask;        // [T][n_words]
+  int T, d, F, n_words;         // n_words = F / 32
+  int act;
+  int* wordpre;                 // [T][n_words] exclusive rank prefix within the token
+  int* nnz;                     // [T]
+  int* rowptr;                  // [T + 1]
+  int2* chunks;                 // [max_chunks] (token, first rank)
+  int* n_chunks;                // [1]
+  int* counter;                 // [1] chunk counter of k_bwd_token
+  float* du;                    // [pairs]
+  float* dg;                    // [pairs]
+  float* hv;                    // [pairs]
+  int* colcnt;                  // [F]
+  int* colptr;                  // [F + 1]
+  int* cscpos;                  // [pairs] CSR position of the pair
+  int* csctok;                  // [pairs] its token
+  float* dx;                    // [T][d]
+  float* dW_gate;               // [F][d]
+  float* dW_up;                 // [F][d]
+  float* dW_down;               // [F][d]
+  float* db;                    // [F] or null
+};
+
+// Exclusive scan of a[0..n) into out[0..n], out[n] = total (one CTA of 1024).
+__device__ __forceinline__ void cta_scan_excl(const int* a, int n, int* out, int* tmp) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
+  int s = 0;
+  for (int i = i0; i < i1; ++i) s += a[i];
+  int tot;
+  int run = block_scan_excl(s, tmp, &tot);
+  for (int i = i0; i < i1; ++i) {
+    const int v = a[i];
+    out[i] = run;
+    run += v;
+  }
+  if (threadIdx.x == 0) out[n] = tot;
+}
+
+__global__ void __launch_bounds__(BW_THREADS) k_bwd_rows(const BwdArgs a) {
+  __shared__ int tmp[33];
+  griddep_wait();
+  const int t = blockIdx.x;
+  const uint32_t* km = a.kmask + (size_t)t * a.n_words;
+  const int per = (a.n_words + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * per, w1 = min(a.n_words, w0 + per);
+  int s = 0;
+  for (int w = w0; w < w1; ++w) s += __popc(km[w]);
+  int tot;
+  int run = block_scan_excl(s, tmp, &tot);
+  for (int w = w0; w < w1; ++w) {
+    a.wordpre[(size_t)t * a.n_words + w] = run;
+    run += __popc(km[w]);
+  }
+  if (threadIdx.x == 0) a.nnz[t] = tot;
+  if (tot > BW_CH)   // several chunks add into dx
+    for (int i = threadIdx.x; i < a.d; i += blockDim.x) a.dx[(size_t)t * a.d + i] = 0.0f;
+}
+
+__global__ void __launch_bounds__(1024) k_bwd_scan(const BwdArgs a) {
+  __shared__ int tmp[33];
+  griddep_wait();
+  cta_scan_excl(a.nnz, a.T, a.rowptr, tmp);
+  __syncthreads();
+  // chunk table: token t owns ceil(nnz_t / BW_CH) chunks (at least one, so
+  // that a token that keeps nothing still gets dx = 0)
+  const int per = (a.T + blockDim.x - 1) / blockDim.x;
+  const int t0 = threadIdx.x * per, t1 = min(a.T, t0 + per);
+  int s = 0;
+  for (int t = t0; t < t1; ++t) s += max(1, (a.nnz[t] + BW_CH - 1) / BW_CH);
+  int tot;
+  int run = block_scan_excl(s, tmp, &tot);
+  for (int t = t0; t < t1; ++t) {
+    const int nc = max(1, (a.nnz[t] + BW_CH - 1) / BW_CH);
+    for (int c = 0; c < nc; ++c) a.chunks[run + c] = make_int2(t, c * BW_CH);
+    run += nc;
+  }
+  if (threadIdx.x == 0) {
+    *a.n_chunks = tot;
+    *a.counter = 0;
+  }
+}
+
+// x and dy of the chunk's token, the chunk's neurons, per-warp dx rows
+struct BwdTokenSmem {
+  int x, dy, list, dxw, total;
+  __host__ __device__ static BwdTokenSmem make(int d) {
+    BwdTokenSmem s;
+    int o = 0;
+    s.x = o;    o += d * 2;
+    s.dy = o;   o += d * 4;
+    s.list = o; o += BW_CH * 4;
+    s.dxw = o;  o += (BW_THREADS / 32) * d * 4;
+    s.total = o + 16;
+    return s;
+  }
+};
+
+__global__ void __launch_bounds__(BW_THREADS) k_bwd_token(const BwdArgs a) {
+  extern __shared__ __align__(16) uint8_t bw_s[];
+  const BwdTokenSmem L = BwdTokenSmem::make(a.d);
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(bw_s + L.x);
+  float* dys = reinterpret_cast<float*>(bw_s + L.dy);
+  int* list = reinterpret_cast<int*>(bw_s + L.list);
+  float* dxw = reinterpret_cast<float*>(bw_s + L.dxw);
+  __shared__ int s_chunk;
+  griddep_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = BW_THREADS / 32;
+  const int dv = a.d / 8;
+  const int nch = *a.n_chunks;
+  int cur_t = -1;
+  for (;;) {
+    __syncthreads();
+    if (threadIdx.x == 0) s_chunk = atomicAdd(a.counter, 1);
+    __syncthreads();
+    const int c = s_chunk;
+    if (c >= nch) break;
+    const int2 ch = a.chunks[c];
+    const int t = ch.x, r0 = ch.y;
+    const int nz = a.nnz[t];
+    const int n = min(BW_CH, nz - r0);
+    if (t != cur_t) {   // stage the token's x and dy rows
+      for (int v = threadIdx.x; v < dv; v += blockDim.x) {
+        reinterpret_cast<uint4*>(xs)[v] = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d)[v];
+        reinterpret_cast<float4*>(dys)[2 * v] = reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d)[2 * v];
+        reinterpret_cast<float4*>(dys)[2 * v + 1] =
+            reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d)[2 * v + 1];
+      }
+      cur_t = t;
+    }
+    // the chunk's neurons: the kept ones of rank r0 .. r0 + n - 1
+    const uint32_t* km = a.kmask + (size_t)t * a.n_words;
+    const int* wp = a.wordpre + (size_t)t * a.n_words;
+    for (int w = threadIdx.x; w < a.n_words; w += blockDim.x) {
+      uint32_t m = km[w];
+      int rk = wp[w];
+      if (rk >= r0 + n || rk + __popc(m) <= r0) continue;
+      while (m) {
+        const int b = __ffs(m) - 1;
+        m &= m - 1u;
+        if (rk >= r0 && rk < r0 + n) list[rk - r0] = w * 32 + b;
+        ++rk;
+      }
+    }
+    for (int i = threadIdx.x; i < nwarp * a.d; i += blockDim.x) dxw[i] = 0.0f;
+    __syncthreads();
+    float* myacc = dxw + warp * a.d;
+    for (int q = warp; q < n; q += nwarp) {
+      const int j = list[q];
+      const uint4* rg = reinterpret_cast<const uint4*>(a.W_gate + (size_t)j * a.d);
+      const uint4* ru = reinterpret_cast<const uint4*>(a.W_up + (size_t)j * a.d);
+      const uint4* rd = reinterpret_cast<const uint4*>(a.W_down + (size_t)j * a.d);
+      float sg = 0.f, su = 0.f, sd = 0.f;
+      for (int v = lane; v < dv; v += 32) {
+        const uint4 pg = __ldg(rg + v), pu = __ldg(ru + v), pd = __ldg(rd + v);
+        const uint4 px = reinterpret_cast<const uint4*>(xs)[v];
+        const float4 y0 = reinterpret_cast<const float4*>(dys)[2 * v];
+        const float4 y1 = reinterpret_cast<const float4*>(dys)[2 * v + 1];
+        const float yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+        const uint32_t gg[4] = {pg.x, pg.y, pg.z, pg.w}, uu[4] = {pu.x, pu.y, pu.z, pu.w};
+        const uint32_t dd[4] = {pd.x, pd.y, pd.z, pd.w}, xx[4] = {px.x, px.y, px.z, px.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xx[e]));
+          const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gg[e]));
+          const float2 fu = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
+          const float2 fd = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dd[e]));
+          sg += fg.x * fx.x + fg.y * fx.y;
+          su += fu.x * fx.x + fu.y * fx.y;
+          sd += fd.x * yy[2 * e] + fd.y * yy[2 * e + 1];
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sg += __shfl_xor_sync(0xFFFFFFFFu, sg, o);
+        su += __shfl_xor_sync(0xFFFFFFFFu, su, o);
+        sd += __shfl_xor_sync(0xFFFFFFFFu, sd, o);
+      }
+      const float g = sg + (a.bias ? a.bias[j] : 0.0f);
+      const float act = act_fn(g, a.act);
+      const float v = __bfloat162float(__float2bfloat16_rn(act));
+      // sigma'(g): 1 for ReLU on a kept neuron (the forward kept it, so g >
+      // threshold >= 0), s(1 + g(1 - s)) for SiLU
+      float slope = 1.0f;
+      if (a.act == ACT_SILU) {
+        const float sgm = 1.0f / (1.0f + expf(-g));
+        slope = sgm * (1.0f + g * (1.0f - sgm));
+      }
+      const float du = sd * v, dg = sd * su * slope;
+      if (lane == 0) {
+        const int pos = a.rowptr[t] + r0 + q;
+        a.du[pos] = du;
+        a.dg[pos] = dg;
+        a.hv[pos] = v * su;
+      }
+      // dx row of this warp: du·W_up[j] + dg·W_gate[j] (the rows are in L1)
+      for (int v8 = lane; v8 < dv; v8 += 32) {
+        const uint4 pu = __ldg(ru + v8), pg = __ldg(rg + v8);
+        const uint32_t uu[4] = {pu.x, pu.y, pu.z, pu.w}, gg[4] = {pg.x, pg.y, pg.z, pg.w};
+        float4* acc = reinterpret_cast<float4*>(myacc + 8 * v8);
+        float4 a0 = acc[0], a1 = acc[1];
+        float r[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fu = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
+          const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gg[e]));
+          r[2 * e] = du * fu.x + dg * fg.x;
+          r[2 * e + 1] = du * fu.y + dg * fg.y;
+        }
+        a0.x += r[0]; a0.y += r[1]; a0.z += r[2]; a0.w += r[3];
+        a1.x += r[4]; a1.y += r[5]; a1.z += r[6]; a1.w += r[7];
+        acc[0] = a0;
+        acc[1] = a1;
+      }
+    }
+    __syncthreads();
+    const bool split = nz > BW_CH;
+    for (int i = threadIdx.x; i < a.d; i += blockDim.x) {
+      float s = 0.0f;
+      for (int w = 0; w < nwarp; ++w) s += dxw[w * a.d + i];
+      float* dst = a.dx + (size_t)t * a.d + i;
+      if (split)
+        atomicAdd(dst, s);
+      else
+        *dst = s;
+    }
+  }
+}
+
+__global__ void k_bwd_colcount(const BwdArgs a) {
+  griddep_wait();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= a.F) return;
+  const int w = j >> 5;
+  const uint32_t bit = 1u << (j & 31);
+  int c = 0;
+  for (int t = 0; t < a.T; ++t) c += (a.kmask[(size_t)t * a.n_words + w] & bit) ? 1 : 0;
+  a.colcnt[j] = c;
+}
+
+__global__ void __launch_bounds__(1024) k_bwd_scan2(const BwdArgs a) {
+  __shared__ int tmp[33];
+  griddep_wait();
+  cta_scan_excl(a.colcnt, a.F, a.colptr, tmp);
+}
+
+__global__ void k_bwd_colfill(const BwdArgs a) {
+  griddep_wait();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= a.F) return;
+  const int w = j >> 5, b = j & 31;
+  const uint32_t bit = 1u << b, below = bit - 1u;
+  int k = a.colptr[j];
+  for (int t = 0; t < a.T; ++t) {
+    const uint32_t m = a.kmask[(size_t)t * a.n_words + w];
+    if (m & bit) {
+      a.cscpos[k] = a.rowptr[t] + a.wordpre[(size_t)t * a.n_words + w] + __popc(m & below);
+      a.csctok[k] = t;
+      ++k;
+    }
+  }
+}
+
+// dW rows of neuron j (blockIdx.x): thread = 8 consecutive columns per
+// 16-byte piece (d / 8 pieces over the CTA); pairs four at a time, their x
+// and dy pieces loaded before use.
+__global__ void __launch_bounds__(BW_THREADS) k_bwd_neuron(const BwdArgs a) {
+  griddep_wait();
+  const int j = blockIdx.x;
+  const int p0 = a.colptr[j], p1 = a.colptr[j + 1];
+  const int dv = a.d / 8;
+  for (int v = threadIdx.x; v < dv; v += blockDim.x) {
+    float ag[8], au[8], ad[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ag[e] = au[e] = ad[e] = 0.0f;
+    for (int p = p0; p < p1; p += 4) {
+      uint4 xq[4];
+      float4 y0[4], y1[4];
+      float cu[4], cg[4], ch[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (p + q < p1) {
+          const int t = a.csctok[p + q], pos = a.cscpos[p + q];
+          cu[q] = a.du[pos];
+          cg[q] = a.dg[pos];
+          ch[q] = a.hv[pos];
+          xq[q] = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d)[v];
+          y0[q] = reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d)[2 * v];
+          y1[q] = reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d)[2 * v + 1];
+        } else {
+          cu[q] = cg[q] = ch[q] = 0.0f;
+          xq[q] = make_uint4(0, 0, 0, 0);
+          y0[q] = y1[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t xx[4] = {xq[q].x, xq[q].y, xq[q].z, xq[q].w};
+        const float yy[8] = {y0[q].x, y0[q].y, y0[q].z, y0[q].w, y1[q].x, y1[q].y, y1[q].z, y1[q].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xx[e]));
+          ag[2 * e] += cg[q] * fx.x;
+          ag[2 * e + 1] += cg[q] * fx.y;
+          au[2 * e] += cu[q] * fx.x;
+          au[2 * e + 1] += cu[q] * fx.y;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ad[e] += ch[q] * yy[e];
+      }
+    }
+    float4* og = reinterpret_cast<float4*>(a.dW_gate + (size_t)j * a.d) + 2 * v;
+    float4* ou = reinterpret_cast<float4*>(a.dW_up + (size_t)j * a.d) + 2 * v;
+    float4* od = reinterpret_cast<float4*>(a.dW_down + (size_t)j * a.d) + 2 * v;
+    og[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
+    og[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+    ou[0] = make_float4(au[0], au[1], au[2], au[3]);
+    ou[1] = make_float4(au[4], au[5], au[6], au[7]);
+    od[0] = make_float4(ad[0], ad[1], ad[2], ad[3]);
+    od[1] = make_float4(ad[4], ad[5], ad[6], ad[7]);
+  }
+  if (a.db && threadIdx.x < 32) {
+    float s = 0.0f;
+    for (int p = p0 + threadIdx.x; p < p1; p += 32) s += a.dg[a.cscpos[p]];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    if (threadIdx.x == 0) a.db[j] = s;
+  }
+}
+
+}  // namespace sffn

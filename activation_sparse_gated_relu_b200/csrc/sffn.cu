@@ -35,6 +35,7 @@
 #include "gate_rows.cuh"
 #include "gsi.cuh"
 #include "moe.cuh"
+#include "backward.cuh"
 #include "rows_mma.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -49,11 +50,13 @@ constexpr int kNumSMsFallback = 148;
 constexpr int kMaxMarks = 12;
 enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
                    L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_ROTATE_X, L_INPUT_SELECT,
-                   L_GSI_PROJECT, L_GSI_RESID, L_GSI_OUT, L_MOE_ROUTE, L_MOE_COMBINE, L_COUNT };
+                   L_GSI_PROJECT, L_GSI_RESID, L_GSI_OUT, L_MOE_ROUTE, L_MOE_COMBINE,
+                   L_BWD_INDEX, L_BWD_TOKEN, L_BWD_NEURON, L_COUNT };
 const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
                                           "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
                                           "fallback_f32", "decode_fused", "rotate_x", "input_select",
-                                          "gsi_project", "gsi_resid", "gsi_out", "moe_route", "moe_combine"};
+                                          "gsi_project", "gsi_resid", "gsi_out", "moe_route", "moe_combine",
+                                          "bwd_index", "bwd_token", "bwd_neuron"};
 constexpr int kMaxTokensLimit = 16384;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -245,6 +248,21 @@ struct sffn_handle : KTiming {
   __nv_bfloat16* Wu_rot = nullptr;  // W_up·V [F][d]
   __nv_bfloat16* xrot = nullptr;    // x·V [T][d]
   CUtensorMap tmVt;              // V^T rows as the A operand of x·V
+  // backward workspace (SFFN_FLAG_BACKWARD)
+  int* bw_wordpre = nullptr;
+  int* bw_nnz = nullptr;
+  int* bw_rowptr = nullptr;
+  int2* bw_chunks = nullptr;
+  int* bw_nchunks = nullptr;
+  int* bw_counter = nullptr;
+  float* bw_du = nullptr;
+  float* bw_dg = nullptr;
+  float* bw_h = nullptr;
+  int* bw_colcnt = nullptr;
+  int* bw_colptr = nullptr;
+  int* bw_cscpos = nullptr;
+  int* bw_csctok = nullptr;
+  int bw_smem = 0;
   void* arena = nullptr;         // the one device allocation all of the above live in
   size_t arena_bytes = 0;
   bool dense_bufs = false;       // xo, h_hi, h_lo and W_down^T exist (paths other than the single launch)
@@ -379,7 +397,12 @@ sffn_status validate(const sffn_desc* d) {
   if (d->rank > 0 && (d->dtype != SFFN_BF16 || d->rank % 64 != 0 || d->rank > 4096)) return SFFN_ERR_UNSUPPORTED;
   if (d->dtype == SFFN_FP32 && d->d_ff > 8192) return SFFN_ERR_UNSUPPORTED;
   if ((d->flags & SFFN_FLAG_DEBUG_GATE) && d->rank > 0) return SFFN_ERR_UNSUPPORTED;
-  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE | SFFN_FLAG_COOPERATIVE)) return SFFN_ERR_INVALID_ARG;
+  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE | SFFN_FLAG_COOPERATIVE | SFFN_FLAG_BACKWARD))
+    return SFFN_ERR_INVALID_ARG;
+  // the backward: threshold selection, dense gate, bf16, the plain input
+  if ((d->flags & SFFN_FLAG_BACKWARD) && (d->mode != SFFN_MODE_RELU_THRESHOLD || d->rank > 0 ||
+                                          d->dtype != SFFN_BF16 || d->input_k > 0 || d->V))
+    return SFFN_ERR_UNSUPPORTED;
   return SFFN_OK;
 }
 
@@ -502,6 +525,10 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   if (!e && desc->input_k > 0)
     e = cudaFuncSetAttribute(k_input_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              input_select_smem_bytes((int)d));
+  if (!e && (desc->flags & SFFN_FLAG_BACKWARD)) {
+    h->bw_smem = BwdTokenSmem::make((int)d).total;
+    e = cudaFuncSetAttribute(k_bwd_token, cudaFuncAttributeMaxDynamicSharedMemorySize, h->bw_smem);
+  }
   if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, router_smem_bytes((int)T));
   if (!e && h->f32) {
     e = cudaFuncSetAttribute(k_rows_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -569,6 +596,22 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     if (dense_gate_bf16) {
       a.take(&h->gstage, P * 8 * 128 * 4);
       a.take(&h->gtick, P * 4);
+    }
+    if (desc->flags & SFFN_FLAG_BACKWARD) {
+      const size_t W32 = F / 32, pairs = T * F;
+      a.take(&h->bw_wordpre, T * W32 * 4);
+      a.take(&h->bw_nnz, T * 4);
+      a.take(&h->bw_rowptr, (T + 1) * 4);
+      a.take(&h->bw_chunks, (T + pairs / BW_CH + 1) * 8);
+      a.take(&h->bw_nchunks, 16);
+      a.take(&h->bw_counter, 16);
+      a.take(&h->bw_du, pairs * 4);
+      a.take(&h->bw_dg, pairs * 4);
+      a.take(&h->bw_h, pairs * 4);
+      a.take(&h->bw_colcnt, F * 4);
+      a.take(&h->bw_colptr, (F + 1) * 4);
+      a.take(&h->bw_cscpos, pairs * 4);
+      a.take(&h->bw_csctok, pairs * 4);
     }
     if (h->dec_ok) {
       h->dsched_ints = decode_sched_ints((int)P, h->dec_grid + 1);
@@ -1928,4 +1971,69 @@ extern "C" sffn_status sffn_moe_timing_end(sffn_moe_handle* h, int max_kernels, 
   }
   if (n_kernels) *n_kernels = n;
   return s;
+}
+
+// ---------------------------------------------------------------------------
+// Backward of the last forward (see backward.cuh).
+extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float* dy, int T, float* dx,
+                                     float* dW_gate, float* dW_up, float* dW_down, float* d_bias,
+                                     void* cuda_stream) {
+  if (!h) return SFFN_ERR_INVALID_ARG;
+  if (!(h->desc.flags & SFFN_FLAG_BACKWARD)) return SFFN_ERR_UNSUPPORTED;
+  if (T < 0 || T > h->maxT) return SFFN_ERR_INVALID_ARG;
+  if (T == 0) return SFFN_OK;
+  if (!x || !dy || !dx || !dW_gate || !dW_up || !dW_down) return SFFN_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, dy, dx, dW_gate, dW_up, dW_down};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SFFN_ERR_INVALID_ARG;
+  if (d_bias && (reinterpret_cast<uintptr_t>(d_bias) & 3u)) return SFFN_ERR_INVALID_ARG;
+  // the keep masks of the last forward: it must have been a ROWS-path forward of these T tokens
+  if (h->last_T != T || h->last_path != SFFN_PATH_ROWS) return SFFN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  BwdArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.dy = dy;
+  a.W_gate = h->Wg;
+  a.W_up = h->Wu;
+  a.W_down = static_cast<const __nv_bfloat16*>(h->desc.W_down);
+  a.bias = h->desc.gate_bias;
+  a.kmask = h->kmask;
+  a.T = T;
+  a.d = h->d;
+  a.F = h->F;
+  a.n_words = h->F / 32;
+  a.act = h->desc.act;
+  a.wordpre = h->bw_wordpre;
+  a.nnz = h->bw_nnz;
+  a.rowptr = h->bw_rowptr;
+  a.chunks = h->bw_chunks;
+  a.n_chunks = h->bw_nchunks;
+  a.counter = h->bw_counter;
+  a.du = h->bw_du;
+  a.dg = h->bw_dg;
+  a.hv = h->bw_h;
+  a.colcnt = h->bw_colcnt;
+  a.colptr = h->bw_colptr;
+  a.cscpos = h->bw_cscpos;
+  a.csctok = h->bw_csctok;
+  a.dx = dx;
+  a.dW_gate = dW_gate;
+  a.dW_up = dW_up;
+  a.dW_down = dW_down;
+  a.db = d_bias;
+  tmark_begin(h);
+  tmark(h, st, L_BWD_INDEX);
+  if (launch_pdl(k_bwd_rows, dim3(T), dim3(BW_THREADS), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_bwd_scan, dim3(1), dim3(1024), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  tmark(h, st, L_BWD_TOKEN);
+  if (launch_pdl(k_bwd_token, dim3(2 * h->n_sm), dim3(BW_THREADS), (size_t)h->bw_smem, st, 1, a))
+    return SFFN_ERR_CUDA;
+  tmark(h, st, L_BWD_INDEX);
+  if (launch_pdl(k_bwd_colcount, dim3(cdiv(h->F, 256)), dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_bwd_scan2, dim3(1), dim3(1024), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_bwd_colfill, dim3(cdiv(h->F, 256)), dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  tmark(h, st, L_BWD_NEURON);
+  if (launch_pdl(k_bwd_neuron, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  tmark_end(h, st);
+  return SFFN_OK;
 }

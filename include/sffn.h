@@ -107,6 +107,8 @@ typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sff
                                      instead of the single persistent launch (diagnostics, tests) */
 #define SFFN_FLAG_COOPERATIVE 4u  /* launch the single persistent forward with the cooperative
                                      attribute (see sffn_forward) */
+#define SFFN_FLAG_BACKWARD 8u     /* allocate the workspace of sffn_backward (relu-threshold
+                                     mode, dense gate, bf16, no input_k or V) */
 
 typedef struct sffn_desc {
   int d_model;          /* d: multiple of 8, 8..4096 (ROWS path needs d <= 4096)   */
@@ -229,6 +231,27 @@ sffn_status sffn_debug_keep(sffn_handle* h, const uint32_t** keep);
 /* Device view of the dense fp32 gate g[T][d_ff] of the last forward (only
  * with SFFN_FLAG_DEBUG_GATE; dense gate only).  Test use. */
 sffn_status sffn_debug_gate(sffn_handle* h, const float** g);
+
+/* Backward of the last forward: given that forward's x (device, [T][d_model]
+ * bf16) and the upstream gradient dy = dL/dy (device, [T][d_model] fp32),
+ * write dx [T][d_model], dW_gate, dW_up and dW_down [d_ff][d_model] (neuron-
+ * major like the weights) and, if d_bias is not NULL, d_bias [d_ff], all fp32
+ * device buffers, fully overwritten.  Source: "Sparser, Faster, Lighter
+ * Transformer Language Models" (news article), section "Hybrid 應對非均勻稀疏"
+ * (training over the sparse format).  The selection of the forward is held
+ * fixed (its keep masks, every token's full kept set) and the rounding of the
+ * stored value passes the gradient through:
+ *     dh = dy W_down^T on kept pairs, du = dh·v, dg = dh·u·sigma'(g),
+ *     dW_down = h^T dy, dW_up = du^T x, dW_gate = dg^T x, d_bias = sum_t dg,
+ *     dx = du W_up + dg W_gate.
+ * Only kept pairs are computed: a token pass (x and dy rows staged, the
+ * kept rows of W_gate, W_up and W_down streamed; dx) and a neuron pass (the
+ * dW rows and d_bias from each neuron's pairs, x and dy rows gathered).
+ * Requires SFFN_FLAG_BACKWARD at create time (workspace 20·max_tokens·d_ff
+ * bytes plus small arrays) and a last forward on the ROWS path with the same
+ * T (else SFFN_ERR_INVALID_ARG).  Asynchronous on cuda_stream. */
+sffn_status sffn_backward(sffn_handle* h, const void* x, const float* dy, int T, float* dx, float* dW_gate,
+                          float* dW_up, float* dW_down, float* d_bias, void* cuda_stream);
 
 /* Bytes of device memory the handle allocated (its whole workspace, one
  * allocation: TwELL, routing, scratch, status and the create-time derived

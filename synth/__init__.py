@@ -400,3 +400,15 @@ def make_moe_inputs(wl: MoeWorkload, T: Optional[int] = None) -> MoeInputs:
         inp = make_inputs(wl.expert_workload(e), weights_only=True)
         ex.append({"A": inp.A, "B": inp.B, "W_up": inp.W_up, "W_down": inp.W_down, "bias": inp.bias})
     return MoeInputs(wl, _to_dtype(xa, "bf16"), _to_dtype(Wr, "bf16"), ex)
+
+
+# ---------------------------------------------------------------------------
+# upstream gradient for the backward pass
+# ---------------------------------------------------------------------------
+TID_DY = 40
+
+
+def upstream_grad(wl: Workload, T: Optional[int] = None) -> torch.Tensor:
+    """dy = dL/dy [T][d_model] fp32 ~ N(0, 1), seeded by the workload."""
+    T = wl.tokens if T is None else T
+    return torch.from_numpy(_normal(wl.seed, TID_DY, (T, wl.d_model), 1.0))

@@ -22,14 +22,15 @@ def to_dev(t: Optional[torch.Tensor]):
 
 
 def make_ffn(inp: synth.Inputs, max_tokens: int, path: str = "auto", C: Optional[int] = None,
-             debug_gate: bool = False, separate: bool = False, cooperative: bool = False) -> SparseFFN:
+             debug_gate: bool = False, separate: bool = False, cooperative: bool = False,
+             backward: bool = False) -> SparseFFN:
     wl = inp.wl
     return SparseFFN(to_dev(inp.W_up), to_dev(inp.W_down), W_gate=to_dev(inp.W_gate), A=to_dev(inp.A),
                      B=to_dev(inp.B), bias=to_dev(inp.bias), mode=wl.mode, act=wl.act,
                      threshold=wl.threshold, k=wl.k,
                      tile_capacity=wl.tile_capacity if C is None else C, max_tokens=max_tokens,
                      path=path, debug_gate=debug_gate, separate=separate, cooperative=cooperative,
-                     input_k=wl.input_k or 0, V=to_dev(inp.V))
+                     input_k=wl.input_k or 0, V=to_dev(inp.V), backward=backward)
 
 
 @dataclass
