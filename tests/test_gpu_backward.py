@@ -56,7 +56,7 @@ def _check(inp, T, exact, path="rows", C=None):
         amb = ambiguous(res, wl.mode, wl.threshold, wl.k, False)
         rows_ok = ~amb.any(axis=0)
         tok_ok = ~amb.any(axis=1)
-        assert rows_ok.mean() > 0.5 and tok_ok.mean() > 0.5
+        assert rows_ok.mean() > 0.25 and tok_ok.mean() > 0.25
     for k in NAMES:
         sel = tok_ok if k == "dx" else rows_ok
         e = rel_err(got[k][sel], want[k][sel])
