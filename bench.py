@@ -53,6 +53,7 @@ BENCH_SHAPES = {
     "wina_input_bf16": (32, 2, 16, 1000),
     "gsi_bf16": (8, 12, 16, 2000),
     "moe_lopa_bf16": (8, 1, 16, 400),
+    "train_prefill_bf16": (4096, 2, 3, 100),
 }
 SPARSITY = {
     "decode_bf16": "relu gate bias -1.2816 (~90% zeros)",
@@ -88,6 +89,9 @@ KERNEL_SOURCES = {
     "gsi_out": ["gsi.cuh", "ptx.cuh"],
     "moe_route": ["moe.cuh", "ptx.cuh"],
     "moe_combine": ["moe.cuh", "ptx.cuh"],
+    "bwd_index": ["backward.cuh", "simt.cuh", "ptx.cuh"],
+    "bwd_token": ["backward.cuh", "epilogues.cuh", "ptx.cuh"],
+    "bwd_neuron": ["backward.cuh", "ptx.cuh"],
 }
 
 
@@ -382,7 +386,23 @@ def batch_sparsity(ffn, T: int, C: int) -> dict:
     return st
 
 
-def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, traffic_key) -> dict:
+def backward_work(wl, T: int, st: dict) -> dict:
+    """Algorithmic bytes and FLOPs of the backward's kernels: the kept rows
+    of W_gate, W_up and W_down read once, x and dy read, dx and the three dW
+    arrays (fp32) written, three fp32 values per kept pair written and read;
+    per kept pair 3 dot products and 2 updates of d in the token pass, 3
+    updates of d in the neuron pass."""
+    d, F = wl.d_model, wl.d_ff
+    U, nnz = st.get("union_all", st["union"]), st.get("nnz_all", st["nnz"])
+    return {
+        "bwd_index": {"bytes": T * F // 8 * 3 + nnz * 8, "flops": 0},
+        "bwd_token": {"bytes": U * 3 * d * 2 + T * d * (2 + 4 + 4) + nnz * 12, "flops": 10 * nnz * d},
+        "bwd_neuron": {"bytes": 3 * F * d * 4 + F * 4 + nnz * 12, "flops": 6 * nnz * d},
+    }
+
+
+def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, traffic_key,
+            train: bool = False) -> dict:
     """Time `steps` forwards of workload `wl` at T tokens (after `warmup`):
     NS rotating weight copies and NXB x batches resident in HBM, CUDA events
     around the whole region, barrier and max over ranks.  Returns the line's
@@ -401,15 +421,23 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
         ffn = SparseFFN(ws["W_up"], ws["W_down"], W_gate=ws["W_gate"], A=ws["A"], B=ws["B"], bias=ws["bias"],
                         mode=wl.mode, act=wl.act, threshold=wl.threshold, k=wl.k,
                         tile_capacity=wl.tile_capacity, max_tokens=T, input_k=wl.input_k or 0,
-                        V=dev(inp.V))
+                        V=dev(inp.V), backward=train)
         sets.append((ws, ffn))
     xall = dev(inp.x)
     xb = [xall[i * T:(i + 1) * T].contiguous() for i in range(NXB)]
     outs = [torch.empty((T, wl.d_model), dtype=torch.float32, device="cuda") for _ in range(NS)]
     stream = torch.cuda.current_stream()
+    if train:   # one training step: the forward, then the backward for a fixed upstream gradient
+        dys = dev(synth.upstream_grad(wl, T).contiguous())
+        gbuf = {k: torch.empty(shape, dtype=torch.float32, device="cuda") for k, shape in (
+            ("dx", (T, wl.d_model)), ("dW_gate", (wl.d_ff, wl.d_model)), ("dW_up", (wl.d_ff, wl.d_model)),
+            ("dW_down", (wl.d_ff, wl.d_model)), ("d_bias", (wl.d_ff,)))}
 
     def step(i):
-        sets[i % NS][1].forward(xb[i % NXB], outs[i % NS])
+        f = sets[i % NS][1]
+        f.forward(xb[i % NXB], outs[i % NS])
+        if train:
+            f.backward(xb[i % NXB], dys, **gbuf)
 
     for i in range(warmup):
         step(i)
@@ -456,6 +484,11 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
     path = "rows" if ffn0.stats().path == 1 else "tiles"
     works = kernel_work(wl, T, path, st)
     bytes_step, flops_step = step_work(wl, T, st)
+    if train:
+        bw = backward_work(wl, T, st)
+        works.update(bw)
+        bytes_step += sum(v["bytes"] for v in bw.values())
+        flops_step += sum(v["flops"] for v in bw.values())
 
     peaks, peak_src = load_peaks()
     per = {k: (v[0] / v[1] if v[1] else 0.0) for k, v in kernels.items()}
@@ -465,7 +498,7 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
     # launches overlap prologue and tail by programmatic dependent launch; the
     # per-launch events, which break that overlap for the forwards they
     # bracket, are reported beside it as ms_per_launch_events)
-    single = len(kernels) == 1 and launches_per_fwd == 1
+    single = len(kernels) == 1 and launches_per_fwd == 1 and not train
     ms_dom = tot_ms / steps if single else per.get(dom, 0.0)
     roof = None
     if dom in works and ms_dom > 0:
@@ -694,7 +727,7 @@ def measure_moe(wl, T: int, NXB: int, steps: int, warmup: int, world: int) -> di
 # run: (workload, tokens per forward)
 EXTRA_WORKLOADS = [("decode_bf16", 1), ("decode_bf16", 4), ("lopa_bf16", 32), ("wina_bf16", 32),
                    ("prefill_bf16", 4096), ("tiny_fp32", 64), ("wina_fullh_bf16", 32), ("wina_input_bf16", 32),
-                   ("gsi_bf16", 8), ("moe_lopa_bf16", 8)]
+                   ("gsi_bf16", 8), ("moe_lopa_bf16", 8), ("train_prefill_bf16", 4096)]
 EXTRA_MIN_STEPS = 200
 EXTRA_MAX_S = 2.0
 
@@ -720,6 +753,26 @@ def run_ours(args) -> None:
     barrier(world)
     load_library()
 
+    if args.workload == "train_prefill_bf16":
+        T = args.tokens or BENCH_SHAPES[args.workload][0]
+        _, NSt, NXBt, _ = BENCH_SHAPES[args.workload]
+        m = measure(synth.WORKLOADS["prefill_bf16"], T, NSt, NXBt, args.steps, args.warmup, world, None, train=True)
+        for _, f in m.pop("_sets"):
+            f.close()
+        m.pop("_inp"), m.pop("_NXB")
+        if rank == 0:
+            line = {"metric": METRIC + " (training step: forward + sparse backward)", "value": m.pop("value"),
+                    "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": m.pop("ms_per_step"), "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                    "config": config_dict(synth.WORKLOADS["prefill_bf16"], T, NSt, NXBt)}
+            m.pop("steps"), m.pop("warmup")
+            line.update(m)
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if args.workload in GSI_WORKLOADS or args.workload in MOE_WORKLOADS:
         T, _, NXB, _ = BENCH_SHAPES[args.workload]
         T = args.tokens or T
@@ -809,16 +862,17 @@ def run_ours(args) -> None:
                 workloads[f"{name}@T={Tw}"] = measure_gsi(wlg, Tw, NSx, NXBx, ksteps, max(args.warmup, 3), world)
                 torch.cuda.empty_cache()
                 continue
-            wlx = synth.WORKLOADS[name]
+            train = name == "train_prefill_bf16"
+            wlx = synth.WORKLOADS["prefill_bf16" if train else name]
             # a bounded run: at least EXTRA_MIN_STEPS forwards, about
             # EXTRA_MAX_S seconds at most, from a short probe of the step time
-            probe = measure(wlx, Tw, NSx, NXBx, 10, max(args.warmup, 3), world, None)
+            probe = measure(wlx, Tw, NSx, NXBx, 10, max(args.warmup, 3), world, None, train=train)
             for _, f in probe.pop("_sets"):
                 f.close()
             ksteps = max(EXTRA_MIN_STEPS, min(5000, int(EXTRA_MAX_S / (probe["ms_per_step"] * 1e-3))))
             ksteps -= ksteps % NSx
             key = name if Tw == BENCH_SHAPES[name][0] else None
-            r = measure(wlx, Tw, NSx, NXBx, ksteps, max(args.warmup, 3), world, key)
+            r = measure(wlx, Tw, NSx, NXBx, ksteps, max(args.warmup, 3), world, None if train else key, train=train)
             for _, f in r.pop("_sets"):
                 f.close()
             r.pop("_inp"), r.pop("_NXB")
