@@ -198,6 +198,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // stride-th forward and after its last one.
 struct KTiming {
   bool tm_on = false;
+  bool tm_prev = false;             // the last tmark_begin opened a record
   int tm_max = 0, tm_n = 0, tm_cur = -1, tm_stride = 1, tm_seen = 0;
   std::vector<cudaEvent_t> tm_ev;   // [tm_max][kMaxMarks + 1]
   std::vector<int> tm_lab;          // [tm_max][kMaxMarks]
@@ -341,6 +342,18 @@ void tmark(KTiming* h, cudaStream_t st, int label) {
 void tmark_begin(KTiming* h) {
   h->tm_cur = -1;
   if (h->tm_on && (h->tm_seen++ % h->tm_stride) == 0 && h->tm_n < h->tm_max) {
+    h->tm_cur = h->tm_n++;
+    h->tm_nk[h->tm_cur] = 0;
+  }
+  h->tm_prev = h->tm_cur >= 0;
+}
+
+// A record for a pass that follows a forward (the backward, a MoE combine):
+// opened exactly when the forward's own record was, so the stride counts
+// forwards only.
+void tmark_follow(KTiming* h) {
+  h->tm_cur = -1;
+  if (h->tm_on && h->tm_prev && h->tm_n < h->tm_max) {
     h->tm_cur = h->tm_n++;
     h->tm_nk[h->tm_cur] = 0;
   }
@@ -1888,7 +1901,7 @@ extern "C" sffn_status sffn_moe_forward(sffn_moe_handle* h, const void* x, int T
                                        h->ye + (size_t)e * T * h->d, cuda_stream);
     if (s != SFFN_OK) return s;
   }
-  tmark_begin(h);
+  tmark_follow(h);
   MoeCombineArgs ca{h->ye, h->sel, h->w, out, T, h->d, h->top_k};
   tmark(h, st, L_MOE_COMBINE);
   if (launch_pdl(k_moe_combine, dim3(std::max(1, cdiv(h->d / 4, 256)), T), dim3(256), 0, st, 1, ca))
@@ -2021,7 +2034,7 @@ extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float*
   a.dW_up = dW_up;
   a.dW_down = dW_down;
   a.db = d_bias;
-  tmark_begin(h);
+  tmark_follow(h);
   tmark(h, st, L_BWD_INDEX);
   if (launch_pdl(k_bwd_rows, dim3(T), dim3(BW_THREADS), 0, st, 1, a)) return SFFN_ERR_CUDA;
   if (launch_pdl(k_bwd_scan, dim3(1), dim3(1024), 0, st, 1, a)) return SFFN_ERR_CUDA;

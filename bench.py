@@ -449,8 +449,8 @@ def measure(wl, T: int, NS: int, NXB: int, steps: int, warmup: int, world: int, 
     # ------------------------------------------------------- timed region
     # per-kernel events on every TIMING_STRIDE-th forward of each handle: enough
     # launches to average, few enough not to perturb the timed region
-    for _, ffn in sets:
-        ffn.timing_begin(steps // NS // TIMING_STRIDE + 2, TIMING_STRIDE)
+    for _, ffn in sets:   # (a training step records the forward and the backward)
+        ffn.timing_begin((2 if train else 1) * (steps // NS // TIMING_STRIDE + 2), TIMING_STRIDE)
     clocks = ClockSampler(torch.cuda.current_device())
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
