@@ -25,8 +25,9 @@
 //                  and du·W_up[j] + dg·W_gate[j] into the warp's dx row;
 //                  the warps' rows summed into dx (added when the token has
 //                  several chunks)
-//   k_bwd_colcount thread = neuron: pairs per neuron; k_bwd_scan2 offsets
-//   k_bwd_colfill  thread = neuron: the CSR positions of its pairs
+//   k_bwd_colcount thread = (chunk of 64 tokens, neuron): pairs counted;
+//                  k_bwd_scan2 turns the counts into offsets
+//   k_bwd_colfill  thread = (chunk, neuron): the CSR positions of its pairs
 //   k_bwd_neuron   CTA = neuron: dW_gate, dW_up and dW_down rows and db
 //                  from its pairs (x and dy rows gathered), no atomics
 #pragma once
@@ -59,7 +60,7 @@ struct BwdArgs {
   float* du;                    // [pairs]
   float* dg;                    // [pairs]
   float* hv;                    // [pairs]
-  int* colcnt;                  // [F]
+  int* colcnt;                  // [T / BW_TCH][F] pairs per (token chunk, neuron), then their offsets
   int* colptr;                  // [F + 1]
   int* cscpos;                  // [pairs] CSR position of the pair
   int* csctok;                  // [pairs] its token
@@ -276,32 +277,70 @@ __global__ void __launch_bounds__(BW_THREADS) k_bwd_token(const BwdArgs a) {
   }
 }
 
+// The column index, in parallel over (token chunk, neuron): thread = one
+// neuron over BW_TCH consecutive tokens.  k_bwd_colcount writes the count
+// of each (chunk, neuron); k_bwd_scan2 turns them into offsets (chunks in
+// token order inside each neuron, neurons one after another); k_bwd_colfill
+// writes each chunk's pairs at its offset, so every neuron's list is in token
+// order, the same on every run (k_bwd_colprefix and k_bwd_scan2 between them).
+constexpr int BW_TCH = 64;
+
 __global__ void k_bwd_colcount(const BwdArgs a) {
   griddep_wait();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x, tc = blockIdx.y;
   if (j >= a.F) return;
   const int w = j >> 5;
   const uint32_t bit = 1u << (j & 31);
+  const int t0 = tc * BW_TCH, t1 = min(a.T, t0 + BW_TCH);
   int c = 0;
-  for (int t = 0; t < a.T; ++t) c += (a.kmask[(size_t)t * a.n_words + w] & bit) ? 1 : 0;
-  a.colcnt[j] = c;
+  for (int t = t0; t < t1; ++t) c += (__ldg(a.kmask + (size_t)t * a.n_words + w) & bit) ? 1 : 0;
+  a.colcnt[(size_t)tc * a.F + j] = c;
 }
 
+// per neuron (thread): its chunks' counts turned into exclusive prefixes in
+// place, the total into colptr[j]
+__global__ void k_bwd_colprefix(const BwdArgs a) {
+  griddep_wait();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= a.F) return;
+  const int nch = (a.T + BW_TCH - 1) / BW_TCH;
+  int run = 0;
+  for (int c = 0; c < nch; ++c) {
+    const int v = a.colcnt[(size_t)c * a.F + j];
+    a.colcnt[(size_t)c * a.F + j] = run;
+    run += v;
+  }
+  a.colptr[j] = run;
+}
+
+// colptr: exclusive scan of the neurons' totals, in place (one CTA)
 __global__ void __launch_bounds__(1024) k_bwd_scan2(const BwdArgs a) {
   __shared__ int tmp[33];
   griddep_wait();
-  cta_scan_excl(a.colcnt, a.F, a.colptr, tmp);
+  const int per = (a.F + blockDim.x - 1) / blockDim.x;
+  const int i0 = threadIdx.x * per, i1 = min(a.F, i0 + per);
+  int sum = 0;
+  for (int i = i0; i < i1; ++i) sum += a.colptr[i];
+  int tot;
+  int run = block_scan_excl(sum, tmp, &tot);
+  for (int i = i0; i < i1; ++i) {
+    const int v = a.colptr[i];
+    a.colptr[i] = run;
+    run += v;
+  }
+  if (threadIdx.x == 0) a.colptr[a.F] = tot;
 }
 
 __global__ void k_bwd_colfill(const BwdArgs a) {
   griddep_wait();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x, tc = blockIdx.y;
   if (j >= a.F) return;
   const int w = j >> 5, b = j & 31;
   const uint32_t bit = 1u << b, below = bit - 1u;
-  int k = a.colptr[j];
-  for (int t = 0; t < a.T; ++t) {
-    const uint32_t m = a.kmask[(size_t)t * a.n_words + w];
+  const int t0 = tc * BW_TCH, t1 = min(a.T, t0 + BW_TCH);
+  int k = a.colptr[j] + a.colcnt[(size_t)tc * a.F + j];
+  for (int t = t0; t < t1; ++t) {
+    const uint32_t m = __ldg(a.kmask + (size_t)t * a.n_words + w);
     if (m & bit) {
       a.cscpos[k] = a.rowptr[t] + a.wordpre[(size_t)t * a.n_words + w] + __popc(m & below);
       a.csctok[k] = t;

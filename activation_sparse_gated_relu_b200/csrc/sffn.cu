@@ -621,7 +621,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       a.take(&h->bw_du, pairs * 4);
       a.take(&h->bw_dg, pairs * 4);
       a.take(&h->bw_h, pairs * 4);
-      a.take(&h->bw_colcnt, F * 4);
+      a.take(&h->bw_colcnt, ((T + BW_TCH - 1) / BW_TCH) * F * 4);
       a.take(&h->bw_colptr, (F + 1) * 4);
       a.take(&h->bw_cscpos, pairs * 4);
       a.take(&h->bw_csctok, pairs * 4);
@@ -2042,9 +2042,11 @@ extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float*
   if (launch_pdl(k_bwd_token, dim3(2 * h->n_sm), dim3(BW_THREADS), (size_t)h->bw_smem, st, 1, a))
     return SFFN_ERR_CUDA;
   tmark(h, st, L_BWD_INDEX);
-  if (launch_pdl(k_bwd_colcount, dim3(cdiv(h->F, 256)), dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  const dim3 gcol(cdiv(h->F, 256), cdiv(T, BW_TCH));
+  if (launch_pdl(k_bwd_colcount, gcol, dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_bwd_colprefix, dim3(cdiv(h->F, 256)), dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
   if (launch_pdl(k_bwd_scan2, dim3(1), dim3(1024), 0, st, 1, a)) return SFFN_ERR_CUDA;
-  if (launch_pdl(k_bwd_colfill, dim3(cdiv(h->F, 256)), dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  if (launch_pdl(k_bwd_colfill, gcol, dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
   tmark(h, st, L_BWD_NEURON);
   if (launch_pdl(k_bwd_neuron, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a)) return SFFN_ERR_CUDA;
   tmark_end(h, st);
