@@ -195,29 +195,44 @@ __global__ void __launch_bounds__(BW_THREADS) k_bwd_token(const BwdArgs a) {
     for (int i = threadIdx.x; i < nwarp * a.d; i += blockDim.x) dxw[i] = 0.0f;
     __syncthreads();
     float* myacc = dxw + warp * a.d;
+    constexpr int PB = 8;   // 16-byte pieces per lane loaded at once (d <= 2048 in one batch)
     for (int q = warp; q < n; q += nwarp) {
       const int j = list[q];
       const uint4* rg = reinterpret_cast<const uint4*>(a.W_gate + (size_t)j * a.d);
       const uint4* ru = reinterpret_cast<const uint4*>(a.W_up + (size_t)j * a.d);
       const uint4* rd = reinterpret_cast<const uint4*>(a.W_down + (size_t)j * a.d);
       float sg = 0.f, su = 0.f, sd = 0.f;
-      for (int v = lane; v < dv; v += 32) {
-        const uint4 pg = __ldg(rg + v), pu = __ldg(ru + v), pd = __ldg(rd + v);
-        const uint4 px = reinterpret_cast<const uint4*>(xs)[v];
-        const float4 y0 = reinterpret_cast<const float4*>(dys)[2 * v];
-        const float4 y1 = reinterpret_cast<const float4*>(dys)[2 * v + 1];
-        const float yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-        const uint32_t gg[4] = {pg.x, pg.y, pg.z, pg.w}, uu[4] = {pu.x, pu.y, pu.z, pu.w};
-        const uint32_t dd[4] = {pd.x, pd.y, pd.z, pd.w}, xx[4] = {px.x, px.y, px.z, px.w};
+      uint4 pg[PB], pu[PB];
+      for (int vb = 0; vb < dv; vb += 32 * PB) {
+        uint4 pd[PB];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xx[e]));
-          const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gg[e]));
-          const float2 fu = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
-          const float2 fd = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dd[e]));
-          sg += fg.x * fx.x + fg.y * fx.y;
-          su += fu.x * fx.x + fu.y * fx.y;
-          sd += fd.x * yy[2 * e] + fd.y * yy[2 * e + 1];
+        for (int i = 0; i < PB; ++i) {   // every piece's loads go out before the first use
+          const int v = vb + lane + 32 * i;
+          const bool in = v < dv;
+          pg[i] = in ? __ldg(rg + v) : make_uint4(0, 0, 0, 0);
+          pu[i] = in ? __ldg(ru + v) : make_uint4(0, 0, 0, 0);
+          pd[i] = in ? __ldg(rd + v) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < PB; ++i) {
+          const int v = vb + lane + 32 * i;
+          if (v >= dv) break;
+          const uint4 px = reinterpret_cast<const uint4*>(xs)[v];
+          const float4 y0 = reinterpret_cast<const float4*>(dys)[2 * v];
+          const float4 y1 = reinterpret_cast<const float4*>(dys)[2 * v + 1];
+          const float yy[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+          const uint32_t gg[4] = {pg[i].x, pg[i].y, pg[i].z, pg[i].w}, uu[4] = {pu[i].x, pu[i].y, pu[i].z, pu[i].w};
+          const uint32_t dd[4] = {pd[i].x, pd[i].y, pd[i].z, pd[i].w}, xx[4] = {px.x, px.y, px.z, px.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xx[e]));
+            const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gg[e]));
+            const float2 fu = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
+            const float2 fd = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dd[e]));
+            sg += fg.x * fx.x + fg.y * fx.y;
+            su += fu.x * fx.x + fu.y * fx.y;
+            sd += fd.x * yy[2 * e] + fd.y * yy[2 * e + 1];
+          }
         }
       }
 #pragma unroll
@@ -243,24 +258,31 @@ __global__ void __launch_bounds__(BW_THREADS) k_bwd_token(const BwdArgs a) {
         a.dg[pos] = dg;
         a.hv[pos] = v * su;
       }
-      // dx row of this warp: du·W_up[j] + dg·W_gate[j] (the rows are in L1)
-      for (int v8 = lane; v8 < dv; v8 += 32) {
-        const uint4 pu = __ldg(ru + v8), pg = __ldg(rg + v8);
-        const uint32_t uu[4] = {pu.x, pu.y, pu.z, pu.w}, gg[4] = {pg.x, pg.y, pg.z, pg.w};
-        float4* acc = reinterpret_cast<float4*>(myacc + 8 * v8);
-        float4 a0 = acc[0], a1 = acc[1];
-        float r[8];
+      // dx row of this warp: du·W_up[j] + dg·W_gate[j]; the last batch's
+      // pieces are still in registers, earlier batches (d > 2048) reload
+      for (int vb = 0; vb < dv; vb += 32 * PB) {
+        const bool last = vb + 32 * PB >= dv;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 fu = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
-          const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gg[e]));
-          r[2 * e] = du * fu.x + dg * fg.x;
-          r[2 * e + 1] = du * fu.y + dg * fg.y;
+        for (int i = 0; i < PB; ++i) {
+          const int v8 = vb + lane + 32 * i;
+          if (v8 >= dv) break;
+          const uint4 qu = last ? pu[i] : __ldg(ru + v8), qg = last ? pg[i] : __ldg(rg + v8);
+          const uint32_t uu[4] = {qu.x, qu.y, qu.z, qu.w}, gg[4] = {qg.x, qg.y, qg.z, qg.w};
+          float4* acc = reinterpret_cast<float4*>(myacc + 8 * v8);
+          float4 a0 = acc[0], a1 = acc[1];
+          float r[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fu = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uu[e]));
+            const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gg[e]));
+            r[2 * e] = du * fu.x + dg * fg.x;
+            r[2 * e + 1] = du * fu.y + dg * fg.y;
+          }
+          a0.x += r[0]; a0.y += r[1]; a0.z += r[2]; a0.w += r[3];
+          a1.x += r[4]; a1.y += r[5]; a1.z += r[6]; a1.w += r[7];
+          acc[0] = a0;
+          acc[1] = a1;
         }
-        a0.x += r[0]; a0.y += r[1]; a0.z += r[2]; a0.w += r[3];
-        a1.x += r[4]; a1.y += r[5]; a1.z += r[6]; a1.w += r[7];
-        acc[0] = a0;
-        acc[1] = a1;
       }
     }
     __syncthreads();
@@ -349,70 +371,103 @@ __global__ void k_bwd_colfill(const BwdArgs a) {
   }
 }
 
-// dW rows of neuron j (blockIdx.x): thread = 8 consecutive columns per
-// 16-byte piece (d / 8 pieces over the CTA); pairs four at a time, their x
-// and dy pieces loaded before use.
+// dW rows of neuron j (blockIdx.x): its pairs' tokens and values staged in
+// shared memory BW_NB at a time, then thread = 8 consecutive columns per
+// 16-byte piece (d / 8 pieces over the CTA), eight pairs' x and dy pieces
+// loaded before use.
+constexpr int BW_NB = 256;
+
 __global__ void __launch_bounds__(BW_THREADS) k_bwd_neuron(const BwdArgs a) {
+  __shared__ int s_tok[BW_NB];
+  __shared__ float s_du[BW_NB], s_dg[BW_NB], s_h[BW_NB];
+  __shared__ float s_red[BW_THREADS / 32];
   griddep_wait();
   const int j = blockIdx.x;
   const int p0 = a.colptr[j], p1 = a.colptr[j + 1];
   const int dv = a.d / 8;
-  for (int v = threadIdx.x; v < dv; v += blockDim.x) {
-    float ag[8], au[8], ad[8];
+  constexpr int MAXV = 2;   // pieces per thread: d <= 2 x 8 x 256 = 4096
+  float ag[MAXV][8], au[MAXV][8], ad[MAXV][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ag[e] = au[e] = ad[e] = 0.0f;
-    for (int p = p0; p < p1; p += 4) {
-      uint4 xq[4];
-      float4 y0[4], y1[4];
-      float cu[4], cg[4], ch[4];
+  for (int m = 0; m < MAXV; ++m)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (p + q < p1) {
-          const int t = a.csctok[p + q], pos = a.cscpos[p + q];
-          cu[q] = a.du[pos];
-          cg[q] = a.dg[pos];
-          ch[q] = a.hv[pos];
-          xq[q] = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d)[v];
-          y0[q] = reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d)[2 * v];
-          y1[q] = reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d)[2 * v + 1];
-        } else {
-          cu[q] = cg[q] = ch[q] = 0.0f;
-          xq[q] = make_uint4(0, 0, 0, 0);
-          y0[q] = y1[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < 8; ++e) ag[m][e] = au[m][e] = ad[m][e] = 0.0f;
+  float dbs = 0.0f;
+  for (int pb = p0; pb < p1; pb += BW_NB) {
+    const int nb = min(BW_NB, p1 - pb);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+      const int pos = a.cscpos[pb + i];
+      s_tok[i] = a.csctok[pb + i];
+      s_du[i] = a.du[pos];
+      s_dg[i] = a.dg[pos];
+      s_h[i] = a.hv[pos];
+      dbs += a.dg[pos];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int v = threadIdx.x + m * BW_THREADS;
+      if (v >= dv) break;
+      for (int i0 = 0; i0 < nb; i0 += 8) {
+        uint4 xq[8];
+        float4 y0[8], y1[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (i0 + q < nb) {
+            const int t = s_tok[i0 + q];
+            xq[q] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + v);
+            y0[q] = __ldg(reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d) + 2 * v);
+            y1[q] = __ldg(reinterpret_cast<const float4*>(a.dy + (size_t)t * a.d) + 2 * v + 1);
+          } else {
+            xq[q] = make_uint4(0, 0, 0, 0);
+            y0[q] = y1[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
-      }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t xx[4] = {xq[q].x, xq[q].y, xq[q].z, xq[q].w};
-        const float yy[8] = {y0[q].x, y0[q].y, y0[q].z, y0[q].w, y1[q].x, y1[q].y, y1[q].z, y1[q].w};
+        for (int q = 0; q < 8; ++q) {
+          const float cu = i0 + q < nb ? s_du[i0 + q] : 0.0f;
+          const float cg = i0 + q < nb ? s_dg[i0 + q] : 0.0f;
+          const float ch = i0 + q < nb ? s_h[i0 + q] : 0.0f;
+          const uint32_t xx[4] = {xq[q].x, xq[q].y, xq[q].z, xq[q].w};
+          const float yy[8] = {y0[q].x, y0[q].y, y0[q].z, y0[q].w, y1[q].x, y1[q].y, y1[q].z, y1[q].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xx[e]));
-          ag[2 * e] += cg[q] * fx.x;
-          ag[2 * e + 1] += cg[q] * fx.y;
-          au[2 * e] += cu[q] * fx.x;
-          au[2 * e + 1] += cu[q] * fx.y;
+          for (int e = 0; e < 4; ++e) {
+            const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xx[e]));
+            ag[m][2 * e] += cg * fx.x;
+            ag[m][2 * e + 1] += cg * fx.y;
+            au[m][2 * e] += cu * fx.x;
+            au[m][2 * e + 1] += cu * fx.y;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ad[m][e] += ch * yy[e];
         }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ad[e] += ch[q] * yy[e];
       }
     }
+  }
+#pragma unroll
+  for (int m = 0; m < MAXV; ++m) {
+    const int v = threadIdx.x + m * BW_THREADS;
+    if (v >= dv) break;
     float4* og = reinterpret_cast<float4*>(a.dW_gate + (size_t)j * a.d) + 2 * v;
     float4* ou = reinterpret_cast<float4*>(a.dW_up + (size_t)j * a.d) + 2 * v;
     float4* od = reinterpret_cast<float4*>(a.dW_down + (size_t)j * a.d) + 2 * v;
-    og[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
-    og[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
-    ou[0] = make_float4(au[0], au[1], au[2], au[3]);
-    ou[1] = make_float4(au[4], au[5], au[6], au[7]);
-    od[0] = make_float4(ad[0], ad[1], ad[2], ad[3]);
-    od[1] = make_float4(ad[4], ad[5], ad[6], ad[7]);
+    og[0] = make_float4(ag[m][0], ag[m][1], ag[m][2], ag[m][3]);
+    og[1] = make_float4(ag[m][4], ag[m][5], ag[m][6], ag[m][7]);
+    ou[0] = make_float4(au[m][0], au[m][1], au[m][2], au[m][3]);
+    ou[1] = make_float4(au[m][4], au[m][5], au[m][6], au[m][7]);
+    od[0] = make_float4(ad[m][0], ad[m][1], ad[m][2], ad[m][3]);
+    od[1] = make_float4(ad[m][4], ad[m][5], ad[m][6], ad[m][7]);
   }
-  if (a.db && threadIdx.x < 32) {
-    float s = 0.0f;
-    for (int p = p0 + threadIdx.x; p < p1; p += 32) s += a.dg[a.cscpos[p]];
+  if (a.db) {   // d_bias[j] = sum of dg over the pairs, in pair order within each thread's share
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    if (threadIdx.x == 0) a.db[j] = s;
+    for (int o = 16; o > 0; o >>= 1) dbs += __shfl_xor_sync(0xFFFFFFFFu, dbs, o);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = dbs;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.0f;
+      for (int w = 0; w < BW_THREADS / 32; ++w) s += s_red[w];
+      a.db[j] = s;
+    }
   }
 }
 

@@ -27,7 +27,8 @@ namespace sffn {
 
 constexpr int GSI_TC = 8;          // tokens per chunk
 constexpr int GSI_THREADS = 256;   // 8 warps
-constexpr int GSI_ROWS = 8;        // rows a warp loads at once in k_gsi_out
+constexpr int GSI_ROWS = 6;        // rows a warp loads at once in k_gsi_out (register budget of 512 threads)
+constexpr int GSI_OUT_THREADS = 512;   // 16 warps: a whole batch of rows in flight per SM
 
 struct GsiArgs {
   const __nv_bfloat16* x;      // [T][d_in]
@@ -85,7 +86,7 @@ __device__ __forceinline__ void row_range(int rows, int& r0, int& r1) {
 // per row, 256 / (k / 2) groups take interleaved rows, all of a thread's row
 // loads go out before their use, the groups' sums meet in shared memory and
 // the CTA adds its partial g into g (red.add).
-constexpr int GSI_PROJ_ROWS = 64;
+constexpr int GSI_PROJ_ROWS = 32;
 
 __global__ void __launch_bounds__(GSI_THREADS) k_gsi_project(const GsiArgs a) {
   __shared__ float xs[GSI_TC][GSI_PROJ_ROWS];
@@ -242,7 +243,7 @@ struct GsiOutSmem {
   }
 };
 
-__global__ void __launch_bounds__(GSI_THREADS) k_gsi_out(const GsiArgs a) {
+__global__ void __launch_bounds__(GSI_OUT_THREADS) k_gsi_out(const GsiArgs a) {
   extern __shared__ __align__(16) uint8_t gsi_o[];
   const GsiOutSmem L = GsiOutSmem::make(a.T, a.k, a.d_in);
   __nv_bfloat16* ghat = reinterpret_cast<__nv_bfloat16*>(gsi_o + L.ghat);
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(GSI_THREADS) k_gsi_out(const GsiArgs a) {
   int* slow = reinterpret_cast<int*>(gsi_o + L.slow);
   int* nslow = slow + a.T;
   griddep_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = GSI_THREADS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = GSI_OUT_THREADS / 32;
   // routes: warp w adds the partial norms of tokens w, w + 8, ...
   for (int t = warp; t < a.T; t += nwarp) {
     float r2 = 0.0f, x2 = 0.0f;

@@ -1701,7 +1701,7 @@ extern "C" sffn_status sffn_gsi_forward(sffn_gsi_handle* h, const void* x, int T
   if (launch_pdl(k_gsi_resid, dim3(h->grid_resid), dim3(GSI_THREADS), (size_t)h->smem_resid, st, 1, a))
     return SFFN_ERR_CUDA;
   tmark(h, st, L_GSI_OUT);
-  if (launch_pdl(k_gsi_out, dim3(h->grid_out), dim3(GSI_THREADS), (size_t)h->smem_out, st, 1, a))
+  if (launch_pdl(k_gsi_out, dim3(h->grid_out), dim3(GSI_OUT_THREADS), (size_t)h->smem_out, st, 1, a))
     return SFFN_ERR_CUDA;
   tmark_end(h, st);
   h->parity ^= 1;   // the launches went out: the next forward sums into the other buffer
