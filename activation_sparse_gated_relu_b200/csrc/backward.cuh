@@ -377,6 +377,7 @@ __global__ void k_bwd_colfill(const BwdArgs a) {
 // loaded before use.
 constexpr int BW_NB = 256;
 
+template <int MAXV>   // 16-byte pieces per thread: d <= MAXV x 8 x 256
 __global__ void __launch_bounds__(BW_THREADS) k_bwd_neuron(const BwdArgs a) {
   __shared__ int s_tok[BW_NB];
   __shared__ float s_du[BW_NB], s_dg[BW_NB], s_h[BW_NB];
@@ -385,7 +386,6 @@ __global__ void __launch_bounds__(BW_THREADS) k_bwd_neuron(const BwdArgs a) {
   const int j = blockIdx.x;
   const int p0 = a.colptr[j], p1 = a.colptr[j + 1];
   const int dv = a.d / 8;
-  constexpr int MAXV = 2;   // pieces per thread: d <= 2 x 8 x 256 = 4096
   float ag[MAXV][8], au[MAXV][8], ad[MAXV][8];
 #pragma unroll
   for (int m = 0; m < MAXV; ++m)

@@ -2048,7 +2048,11 @@ extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float*
   if (launch_pdl(k_bwd_scan2, dim3(1), dim3(1024), 0, st, 1, a)) return SFFN_ERR_CUDA;
   if (launch_pdl(k_bwd_colfill, gcol, dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
   tmark(h, st, L_BWD_NEURON);
-  if (launch_pdl(k_bwd_neuron, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a)) return SFFN_ERR_CUDA;
+  // one 16-byte piece per thread up to d = 2048 (fewer registers, more CTAs per SM), two up to 4096
+  const cudaError_t en = h->d <= 8 * BW_THREADS
+                             ? launch_pdl(k_bwd_neuron<1>, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a)
+                             : launch_pdl(k_bwd_neuron<2>, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a);
+  if (en) return SFFN_ERR_CUDA;
   tmark_end(h, st);
   return SFFN_OK;
 }
