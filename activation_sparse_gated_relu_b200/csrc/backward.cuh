@@ -378,7 +378,7 @@ __global__ void k_bwd_colfill(const BwdArgs a) {
 constexpr int BW_NB = 256;
 
 template <int MAXV>   // 16-byte pieces per thread: d <= MAXV x 8 x 256
-__global__ void __launch_bounds__(BW_THREADS) k_bwd_neuron(const BwdArgs a) {
+__global__ void __launch_bounds__(BW_THREADS, 2) k_bwd_neuron(const BwdArgs a) {
   __shared__ int s_tok[BW_NB];
   __shared__ float s_du[BW_NB], s_dg[BW_NB], s_h[BW_NB];
   __shared__ float s_red[BW_THREADS / 32];
