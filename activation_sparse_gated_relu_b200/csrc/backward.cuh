@@ -373,9 +373,10 @@ __global__ void k_bwd_colfill(const BwdArgs a) {
 
 // dW rows of neuron j (blockIdx.x): its pairs' tokens and values staged in
 // shared memory BW_NB at a time, then thread = 8 consecutive columns per
-// 16-byte piece (d / 8 pieces over the CTA), eight pairs' x and dy pieces
-// loaded before use.
+// 16-byte piece (d / 8 pieces over the CTA), BW_PB pairs' x and dy pieces
+// loaded before use (two CTAs per SM).
 constexpr int BW_NB = 256;
+constexpr int BW_PB = 4;   // pairs whose x and dy pieces are loaded at once
 
 template <int MAXV>   // 16-byte pieces per thread: d <= MAXV x 8 x 256
 __global__ void __launch_bounds__(BW_THREADS, 2) k_bwd_neuron(const BwdArgs a) {
@@ -408,11 +409,11 @@ __global__ void __launch_bounds__(BW_THREADS, 2) k_bwd_neuron(const BwdArgs a) {
     for (int m = 0; m < MAXV; ++m) {
       const int v = threadIdx.x + m * BW_THREADS;
       if (v >= dv) break;
-      for (int i0 = 0; i0 < nb; i0 += 8) {
-        uint4 xq[8];
-        float4 y0[8], y1[8];
+      for (int i0 = 0; i0 < nb; i0 += BW_PB) {
+        uint4 xq[BW_PB];
+        float4 y0[BW_PB], y1[BW_PB];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < BW_PB; ++q) {
           if (i0 + q < nb) {
             const int t = s_tok[i0 + q];
             xq[q] = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d) + v);
@@ -424,7 +425,7 @@ __global__ void __launch_bounds__(BW_THREADS, 2) k_bwd_neuron(const BwdArgs a) {
           }
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < BW_PB; ++q) {
           const float cu = i0 + q < nb ? s_du[i0 + q] : 0.0f;
           const float cg = i0 + q < nb ? s_dg[i0 + q] : 0.0f;
           const float ch = i0 + q < nb ? s_h[i0 + q] : 0.0f;
