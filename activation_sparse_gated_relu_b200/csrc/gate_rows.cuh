@@ -19,6 +19,10 @@
 // whose ticket completes the tile reads the whole tile back.  That CTA emits
 // TwELL exactly as the tile-kernel epilogue does: counts, ascending indices,
 // bf16 values, pads, keep masks and overflow epochs.
+//
+// The low-rank gate ([LoPA]) runs it twice at up to 8 tokens: first over the
+// rows of A^T with x, storing z = bf16(x·A) instead of emitting TwELL, then
+// over the rows of B^T (rank-long rows) with z, emitting TwELL.
 #pragma once
 
 #include "epilogues.cuh"
@@ -37,6 +41,8 @@ struct GateRowsArgs {
   int d;
   int nslot;                   // ring slots (<= RW_NSMAX)
   uint32_t* status;
+  __nv_bfloat16* zout;         // if set: store bf16(g) [T][F] (no bias) instead of emitting TwELL
+                               // (the low-rank gate's z = bf16(x·A) with W_gate = A^T)
 };
 
 struct GateRowsSmem {
@@ -172,7 +178,13 @@ __global__ void __launch_bounds__(RW_THREADS, 1) k_gate_rows(const GateRowsArgs 
           float g[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) g[i] = i < 8 ? __ldcg(a.gstage + ((size_t)p * 8 + i) * 128 + tid) : 0.f;
-          twell_tile32(a.tw, g, p * 128 + tid, 0, tid, tw_stage, 1);
+          if (a.zout) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (i < T) a.zout[(size_t)i * F + p * 128 + tid] = __float2bfloat16_rn(g[i]);
+          } else {
+            twell_tile32(a.tw, g, p * 128 + tid, 0, tid, tw_stage, 1);
+          }
           if (tid == 0) a.tick[p] = 0;
         }
         named_bar_sync(2, 128);  // done_flag is read by all four warps before it is rewritten

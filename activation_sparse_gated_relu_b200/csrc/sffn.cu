@@ -480,6 +480,9 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   int max_smem = 0;
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const bool dense_gate_bf16 = !h->f32 && !h->wina && !h->lowrank;
+  // the low-rank gate streams rows too at up to 8 tokens: z over A^T's rank
+  // rows (length d), then the gate over B^T's neuron rows (length rank)
+  const bool lowrank_rows = !h->f32 && !h->wina && h->lowrank && h->R % RW_DIV == 0 && h->R <= RW_MAXJ * RW_DIV;
 
   // ------------------------------------------- kernel attributes and shapes
   if (!h->f32) {
@@ -506,6 +509,14 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
                  h->P <= RW_THREADS &&
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
+    if (lowrank_rows) {
+      const int gns = 2;
+      h->gr_nslot = gns;
+      h->gr_smem = GateRowsSmem::make(std::max(h->d, h->R), gns).total;
+      h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem;
+      if (h->gr_ok)
+        e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->gr_smem);
+    }
     if (dense_gate_bf16) {
       // row-streaming gate: the same staged-row layout, two ring slots
       const int gns = 2;
@@ -606,9 +617,10 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       a.take(&h->Bt, F * R * 2);
     }
     if (desc->flags & SFFN_FLAG_DEBUG_GATE) a.take(&h->gdebug, T * F * 4);
-    if (dense_gate_bf16) {
-      a.take(&h->gstage, P * 8 * 128 * 4);
-      a.take(&h->gtick, P * 4);
+    if (dense_gate_bf16 || lowrank_rows) {
+      const size_t tiles = std::max(P, R / 128);   // the gate's tiles, or z's (low rank)
+      a.take(&h->gstage, tiles * 8 * 128 * 4);
+      a.take(&h->gtick, tiles * 4);
     }
     if (desc->flags & SFFN_FLAG_BACKWARD) {
       const size_t W32 = F / 32, pairs = T * F;
@@ -646,7 +658,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   e = e ? e : cudaMemsetAsync(h->ovf, 0, T * 4, st);
   e = e ? e : cudaMemsetAsync(h->status, 0, 16, st);
   e = e ? e : cudaMemsetAsync(h->ovf_count, 0, 16, st);
-  if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, P * 4, st);
+  if (h->gtick) e = e ? e : cudaMemsetAsync(h->gtick, 0, std::max(P, R / 128) * 4, st);
   if (h->lowrank) e = e ? e : cudaMemsetAsync(h->tickets, 0, (R / 128 + 1) * 4, st);
   if (h->dsched) e = e ? e : cudaMemsetAsync(h->dsched, 0, (size_t)h->dsched_ints * 4, st);
   // create-time derived data
@@ -900,7 +912,27 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   const CUtensorMap* gateA = &h->tmWgate;
   const CUtensorMap* gateB = &mx;
   int gate_kb = cdiv(d, 64);
-  if (h->lowrank) {
+  const bool lr_rows = h->lowrank && h->gr_ok && T <= 8;
+  if (lr_rows) {
+    // up to 8 tokens: z = bf16(x·A) by streaming the rank rows of A^T
+    GateRowsArgs zr{};
+    zr.x = static_cast<const __nv_bfloat16*>(x);
+    zr.W_gate = h->At;
+    zr.tw.T = T;
+    zr.tw.F = h->R;
+    zr.tw.n_tiles = h->R / 128;
+    zr.gstage = h->gstage;
+    zr.tick = h->gtick;
+    zr.d = d;
+    zr.nslot = h->gr_nslot;
+    zr.status = h->status;
+    zr.zout = h->z;
+    tmark(h, st, L_GATE_Z);
+    e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, h->R / RW_G)), dim3(RW_THREADS), (size_t)h->gr_smem, st, 1,
+                   zr);
+    ++launches;
+    if (e) return SFFN_ERR_CUDA;
+  } else if (h->lowrank) {
     // z = bf16(x·A): rows are rank coordinates, split over d
     const int mt = cdiv(h->R, 128);
     const int sk = z_splits(d, mt, ntile_tok, h->n_sm);
@@ -959,14 +991,14 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     if (h->gr_ok && T <= 8) {
       // up to 8 tokens: stream whole W_gate rows over every SM
       GateRowsArgs gr{};
-      gr.x = static_cast<const __nv_bfloat16*>(x);
-      gr.W_gate = h->Wg;
+      gr.x = lr_rows ? h->z : static_cast<const __nv_bfloat16*>(x);
+      gr.W_gate = lr_rows ? h->Bt : h->Wg;   // B^T: one rank-long row per neuron
       gr.tw = tw;
       gr.gstage = h->gstage;
       gr.tick = h->gtick;
       gr.zero_out = ga.zero_out;
       gr.zero_n4 = ga.zero_n4;
-      gr.d = d;
+      gr.d = lr_rows ? h->R : d;
       gr.nslot = h->gr_nslot;
       gr.status = h->status;
       e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS), (size_t)h->gr_smem, st, 1,
