@@ -277,6 +277,7 @@ struct sffn_handle : KTiming {
   float* gstage = nullptr;
   int* gtick = nullptr;
   int gr_nslot = 0, gr_smem = 0;
+  int gr_nslot_lr = 0, gr_smem_lr = 0;   // the low-rank gate's pass over B^T rows
   bool gr_ok = false;
   // single persistent launch for T <= 8: scheduler words, published row lists, launch shape
   int* dsched = nullptr;
@@ -510,12 +511,19 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
     if (lowrank_rows) {
-      const int gns = 2;
-      h->gr_nslot = gns;
-      h->gr_smem = GateRowsSmem::make(std::max(h->d, h->R), gns).total;
-      h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem;
+      // z streams d-long rows through two slots; the gate's rank-long rows
+      // are short, so as many slots as fit keep more bytes in flight
+      h->gr_nslot = 2;
+      h->gr_smem = GateRowsSmem::make(h->d, 2).total;
+      int gs = RW_NSMAX;
+      while (gs > 2 && GateRowsSmem::make(h->R, gs).total > max_smem) --gs;
+      h->gr_nslot_lr = gs;
+      h->gr_smem_lr = GateRowsSmem::make(h->R, gs).total;
+      h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem &&
+                 h->gr_smem_lr <= max_smem;
       if (h->gr_ok)
-        e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->gr_smem);
+        e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         std::max(h->gr_smem, h->gr_smem_lr));
     }
     if (dense_gate_bf16) {
       // row-streaming gate: the same staged-row layout, two ring slots
@@ -999,10 +1007,10 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
       gr.zero_out = ga.zero_out;
       gr.zero_n4 = ga.zero_n4;
       gr.d = lr_rows ? h->R : d;
-      gr.nslot = h->gr_nslot;
+      gr.nslot = lr_rows ? h->gr_nslot_lr : h->gr_nslot;
       gr.status = h->status;
-      e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS), (size_t)h->gr_smem, st, 1,
-                     gr);
+      e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS),
+                     (size_t)(lr_rows ? h->gr_smem_lr : h->gr_smem), st, 1, gr);
     } else if (P * ntile_tok > h->n_sm && !(D.flags & SFFN_FLAG_SEPARATE)) {
       // at least a tile per SM: the persistent gate overlaps each tile's
       // TwELL emission with the next tile's MMAs
