@@ -20,9 +20,9 @@
 // TwELL exactly as the tile-kernel epilogue does: counts, ascending indices,
 // bf16 values, pads, keep masks and overflow epochs.
 //
-// The low-rank gate ([LoPA]) runs it twice at up to 8 tokens: first over the
-// rows of A^T with x, storing z = bf16(x·A) instead of emitting TwELL, then
-// over the rows of B^T (rank-long rows) with z, emitting TwELL.
+// The low-rank gate ([LoPA]) runs it at up to 8 tokens over the rank rows of
+// A^T with x, storing z = bf16(x·A) instead of emitting TwELL (the gate over
+// B then runs on the tile kernel).
 #pragma once
 
 #include "epilogues.cuh"

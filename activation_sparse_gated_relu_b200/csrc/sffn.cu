@@ -277,7 +277,6 @@ struct sffn_handle : KTiming {
   float* gstage = nullptr;
   int* gtick = nullptr;
   int gr_nslot = 0, gr_smem = 0;
-  int gr_nslot_lr = 0, gr_smem_lr = 0;   // the low-rank gate's pass over B^T rows
   bool gr_ok = false;
   // single persistent launch for T <= 8: scheduler words, published row lists, launch shape
   int* dsched = nullptr;
@@ -481,9 +480,9 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   int max_smem = 0;
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const bool dense_gate_bf16 = !h->f32 && !h->wina && !h->lowrank;
-  // the low-rank gate streams rows too at up to 8 tokens: z over A^T's rank
-  // rows (length d), then the gate over B^T's neuron rows (length rank)
-  const bool lowrank_rows = !h->f32 && !h->wina && h->lowrank && h->R % RW_DIV == 0 && h->R <= RW_MAXJ * RW_DIV;
+  // the low-rank gate's z = bf16(x·A) streams the rank rows of A^T at up to
+  // 8 tokens
+  const bool lowrank_rows = !h->f32 && !h->wina && h->lowrank && h->R % 128 == 0;
 
   // ------------------------------------------- kernel attributes and shapes
   if (!h->f32) {
@@ -511,19 +510,12 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
                  h->rows_smem <= max_smem;
     e = e ? e : cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->rows_smem);
     if (lowrank_rows) {
-      // z streams d-long rows through two slots; the gate's rank-long rows
-      // are short, so as many slots as fit keep more bytes in flight
+      // z = bf16(x·A) streams the d-long rank rows of A^T through two slots
       h->gr_nslot = 2;
       h->gr_smem = GateRowsSmem::make(h->d, 2).total;
-      int gs = RW_NSMAX;
-      while (gs > 2 && GateRowsSmem::make(h->R, gs).total > max_smem) --gs;
-      h->gr_nslot_lr = gs;
-      h->gr_smem_lr = GateRowsSmem::make(h->R, gs).total;
-      h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem &&
-                 h->gr_smem_lr <= max_smem;
+      h->gr_ok = h->d % RW_DIV == 0 && h->d <= RW_MAXJ * RW_DIV && h->gr_smem <= max_smem;
       if (h->gr_ok)
-        e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         std::max(h->gr_smem, h->gr_smem_lr));
+        e = e ? e : cudaFuncSetAttribute(k_gate_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, h->gr_smem);
     }
     if (dense_gate_bf16) {
       // row-streaming gate: the same staged-row layout, two ring slots
@@ -917,10 +909,10 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   if (!mok) return SFFN_ERR_CUDA;
 
   // ---------------------------------------------------------------- gate
+  const bool lr_rows = h->lowrank && h->gr_ok && T <= 8;
   const CUtensorMap* gateA = &h->tmWgate;
   const CUtensorMap* gateB = &mx;
   int gate_kb = cdiv(d, 64);
-  const bool lr_rows = h->lowrank && h->gr_ok && T <= 8;
   if (lr_rows) {
     // up to 8 tokens: z = bf16(x·A) by streaming the rank rows of A^T
     GateRowsArgs zr{};
@@ -940,6 +932,12 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
                    zr);
     ++launches;
     if (e) return SFFN_ERR_CUDA;
+    // the gate over B (15 MB at d = 4096, d_ff = 14336, rank 512) stays on
+    // the tile kernel: streaming B^T's short rows measured slower (21.8 vs
+    // 16.4 us per launch at 8 tokens), the row kernel's fixed cost dominating
+    gateA = &h->tmBt;
+    gateB = &mz;
+    gate_kb = cdiv(h->R, 64);
   } else if (h->lowrank) {
     // z = bf16(x·A): rows are rank coordinates, split over d
     const int mt = cdiv(h->R, 128);
@@ -996,21 +994,21 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
       return SFFN_ERR_CUDA;
   } else {
     tmark(h, st, L_GATE);
-    if (h->gr_ok && T <= 8) {
+    if (h->gr_ok && T <= 8 && !h->lowrank) {
       // up to 8 tokens: stream whole W_gate rows over every SM
       GateRowsArgs gr{};
-      gr.x = lr_rows ? h->z : static_cast<const __nv_bfloat16*>(x);
-      gr.W_gate = lr_rows ? h->Bt : h->Wg;   // B^T: one rank-long row per neuron
+      gr.x = static_cast<const __nv_bfloat16*>(x);
+      gr.W_gate = h->Wg;
       gr.tw = tw;
       gr.gstage = h->gstage;
       gr.tick = h->gtick;
       gr.zero_out = ga.zero_out;
       gr.zero_n4 = ga.zero_n4;
-      gr.d = lr_rows ? h->R : d;
-      gr.nslot = lr_rows ? h->gr_nslot_lr : h->gr_nslot;
+      gr.d = d;
+      gr.nslot = h->gr_nslot;
       gr.status = h->status;
-      e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS),
-                     (size_t)(lr_rows ? h->gr_smem_lr : h->gr_smem), st, 1, gr);
+      e = launch_pdl(k_gate_rows, dim3(std::min(h->n_sm, F / RW_G)), dim3(RW_THREADS), (size_t)h->gr_smem, st, 1,
+                     gr);
     } else if (P * ntile_tok > h->n_sm && !(D.flags & SFFN_FLAG_SEPARATE)) {
       // at least a tile per SM: the persistent gate overlaps each tile's
       // TwELL emission with the next tile's MMAs

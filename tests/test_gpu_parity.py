@@ -436,9 +436,8 @@ def test_prefill_reduced_full_check():
 
 @pytest.mark.parametrize("T", [1, 5, 8])
 def test_lopa_row_gate_exact_grid(T):
-    # up to 8 tokens with a rank that is a multiple of 256 the low-rank gate
-    # streams rows: z over the rank rows of A^T, then the gate over the
-    # rank-long rows of B^T; on grid inputs every value is exact
+    # up to 8 tokens with a rank that is a multiple of 128 the low-rank
+    # gate's z streams the rank rows of A^T; on grid inputs every value is exact
     inp = synth.make_inputs(W["lopa_bf16"].with_(exact_grid=True, tokens=T, d_model=1024, d_ff=2048, rank=256))
     st = check(inp, path="rows")
     assert st["mismatch"] == 0 and st["path"] == SFFN_PATH_ROWS
