@@ -35,6 +35,7 @@
 #include "epilogues.cuh"
 #include "ptx.cuh"
 #include "simt.cuh"
+#include "tc_gemm.cuh"
 
 namespace sffn {
 
@@ -69,6 +70,14 @@ struct BwdArgs {
   float* dW_up;                 // [F][d]
   float* dW_down;               // [F][d]
   float* db;                    // [F] or null
+  // hybrid routing: the forward's overflow tokens ("heavy") take the dense
+  // tensor-core channel instead of the sparse passes
+  const uint32_t* ovf;          // [T] overflow epochs of the forward
+  uint32_t epoch;               // the forward's epoch
+  int* heavy;                   // [T] 1 for a heavy token
+  int* hlist;                   // [T] heavy tokens in token order
+  int* n_heavy;                 // [1]
+  float* dbh;                   // [F] heavy tokens' d_bias contributions (added by the neuron pass)
 };
 
 // Exclusive scan of a[0..n) into out[0..n], out[n] = total (one CTA of 1024).
@@ -102,8 +111,12 @@ __global__ void __launch_bounds__(BW_THREADS) k_bwd_rows(const BwdArgs a) {
     a.wordpre[(size_t)t * a.n_words + w] = run;
     run += __popc(km[w]);
   }
-  if (threadIdx.x == 0) a.nnz[t] = tot;
-  if (tot > BW_CH)   // several chunks add into dx
+  const bool hv = a.ovf && a.ovf[t] == a.epoch;
+  if (threadIdx.x == 0) {
+    a.nnz[t] = hv ? 0 : tot;   // a heavy token's pairs go to the dense channel
+    if (a.heavy) a.heavy[t] = hv ? 1 : 0;
+  }
+  if (!hv && tot > BW_CH)    // several chunks add into dx
     for (int i = threadIdx.x; i < a.d; i += blockDim.x) a.dx[(size_t)t * a.d + i] = 0.0f;
 }
 
@@ -116,14 +129,25 @@ __global__ void __launch_bounds__(1024) k_bwd_scan(const BwdArgs a) {
   // that a token that keeps nothing still gets dx = 0)
   const int per = (a.T + blockDim.x - 1) / blockDim.x;
   const int t0 = threadIdx.x * per, t1 = min(a.T, t0 + per);
+  auto is_heavy = [&](int t) { return a.heavy && a.heavy[t]; };
   int s = 0;
-  for (int t = t0; t < t1; ++t) s += max(1, (a.nnz[t] + BW_CH - 1) / BW_CH);
+  for (int t = t0; t < t1; ++t) s += is_heavy(t) ? 0 : max(1, (a.nnz[t] + BW_CH - 1) / BW_CH);
   int tot;
   int run = block_scan_excl(s, tmp, &tot);
   for (int t = t0; t < t1; ++t) {
-    const int nc = max(1, (a.nnz[t] + BW_CH - 1) / BW_CH);
+    const int nc = is_heavy(t) ? 0 : max(1, (a.nnz[t] + BW_CH - 1) / BW_CH);
     for (int c = 0; c < nc; ++c) a.chunks[run + c] = make_int2(t, c * BW_CH);
     run += nc;
+  }
+  __syncthreads();
+  if (a.hlist) {   // the heavy tokens in token order
+    int hs = 0;
+    for (int t = t0; t < t1; ++t) hs += is_heavy(t) ? 1 : 0;
+    int htot;
+    int hr = block_scan_excl(hs, tmp, &htot);
+    for (int t = t0; t < t1; ++t)
+      if (is_heavy(t)) a.hlist[hr++] = t;
+    if (threadIdx.x == 0) *a.n_heavy = htot;
   }
   if (threadIdx.x == 0) {
     *a.n_chunks = tot;
@@ -315,7 +339,8 @@ __global__ void k_bwd_colcount(const BwdArgs a) {
   const uint32_t bit = 1u << (j & 31);
   const int t0 = tc * BW_TCH, t1 = min(a.T, t0 + BW_TCH);
   int c = 0;
-  for (int t = t0; t < t1; ++t) c += (__ldg(a.kmask + (size_t)t * a.n_words + w) & bit) ? 1 : 0;
+  for (int t = t0; t < t1; ++t)
+    c += (!(a.heavy && a.heavy[t]) && (__ldg(a.kmask + (size_t)t * a.n_words + w) & bit)) ? 1 : 0;
   a.colcnt[(size_t)tc * a.F + j] = c;
 }
 
@@ -363,7 +388,7 @@ __global__ void k_bwd_colfill(const BwdArgs a) {
   int k = a.colptr[j] + a.colcnt[(size_t)tc * a.F + j];
   for (int t = t0; t < t1; ++t) {
     const uint32_t m = __ldg(a.kmask + (size_t)t * a.n_words + w);
-    if (m & bit) {
+    if ((m & bit) && !(a.heavy && a.heavy[t])) {
       a.cscpos[k] = a.rowptr[t] + a.wordpre[(size_t)t * a.n_words + w] + __popc(m & below);
       a.csctok[k] = t;
       ++k;
@@ -467,9 +492,232 @@ __global__ void __launch_bounds__(BW_THREADS, 2) k_bwd_neuron(const BwdArgs a) {
     if (threadIdx.x == 0) {
       float s = 0.0f;
       for (int w = 0; w < BW_THREADS / 32; ++w) s += s_red[w];
-      a.db[j] = s;
+      a.db[j] = s + (a.dbh ? a.dbh[j] : 0.0f);
     }
   }
 }
+
+// ------------------------------------------------ dense channel (heavy tokens)
+// Heavy token o (hlist[o]) in the dense buffers; NP = max_tokens rounded up
+// to 64 (the K padding of the GEMMs over tokens).
+struct HeavyPrepArgs {
+  const __nv_bfloat16* x;       // [T][d]
+  const float* dy;              // [T][d]
+  const int* hlist;
+  const int* n_heavy;
+  __nv_bfloat16* xh;            // [NP][d]   x rows of the heavy tokens
+  __nv_bfloat16* dyh_hi;        // [NP][d]   dy rows, split hi + lo
+  __nv_bfloat16* dyh_lo;
+  __nv_bfloat16* xhT;           // [d][NP]   transposed, zero past n_heavy up to a multiple of 64
+  __nv_bfloat16* dyhT_hi;       // [d][NP]
+  __nv_bfloat16* dyhT_lo;
+  float* dbh;                   // [F] zeroed here
+  int d, F, NP;
+};
+
+// grid (d / 32, NP / 32), block (32, 8): a 32 x 32 tile of (heavy token,
+// column), read by token rows and written transposed through shared memory
+__global__ void k_bwd_heavy_prep(const HeavyPrepArgs a) {
+  __shared__ float tx[32][33], ty[32][33];
+  griddep_wait();
+  const int nh = *a.n_heavy;
+  const int npad = (nh + 63) & ~63;
+  const int i0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int j = threadIdx.y * 32 + threadIdx.x; j < a.F; j += 256) a.dbh[j] = 0.0f;
+  if (o0 >= npad) return;
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int o = o0 + r, i = i0 + threadIdx.x;
+    float xv = 0.f, yv = 0.f;
+    if (o < nh && i < a.d) {
+      const int t = a.hlist[o];
+      xv = __bfloat162float(a.x[(size_t)t * a.d + i]);
+      yv = a.dy[(size_t)t * a.d + i];
+      const __nv_bfloat16 yh = __float2bfloat16_rn(yv);
+      a.xh[(size_t)o * a.d + i] = a.x[(size_t)t * a.d + i];
+      a.dyh_hi[(size_t)o * a.d + i] = yh;
+      a.dyh_lo[(size_t)o * a.d + i] = __float2bfloat16_rn(yv - __bfloat162float(yh));
+    }
+    tx[r][threadIdx.x] = xv;
+    ty[r][threadIdx.x] = yv;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int i = i0 + r, o = o0 + threadIdx.x;
+    if (i < a.d && o < npad) {
+      const float yv = ty[threadIdx.x][r];
+      const __nv_bfloat16 yh = __float2bfloat16_rn(yv);
+      a.xhT[(size_t)i * a.NP + o] = __float2bfloat16_rn(tx[threadIdx.x][r]);
+      a.dyhT_hi[(size_t)i * a.NP + o] = yh;
+      a.dyhT_lo[(size_t)i * a.NP + o] = __float2bfloat16_rn(yv - __bfloat162float(yh));
+    }
+  }
+}
+
+// g and u of the heavy tokens, every neuron: two accumulators (W_gate, then
+// W_up, against the heavy x rows); stored fp32 [NP][F]
+struct GuParams {
+  float* g;
+  float* u;
+  const int* n_rows_dev;
+  int F;
+};
+
+struct EpiStoreGU {
+  static constexpr int N_ACC = 2;
+  using Params = GuParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int n = *o.n_rows_dev, j = m0 + etid;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= n) break;
+      float g[16], u[16];
+      tmem_ld16(tmem + c, g);
+      tmem_ld16(tmem + BN + c, u);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = n0 + c + i;
+        if (r < n) {
+          o.g[(size_t)r * o.F + j] = g[i];
+          o.u[(size_t)r * o.F + j] = u[i];
+        }
+      }
+    }
+  }
+};
+
+// dh = dy W_down^T for the heavy tokens (dy split hi + lo, one accumulator);
+// the epilogue forms the pair values: with the keep bit of the forward,
+// v = bf16(sigma(g + b)), du = dh·v, dg = dh·u·sigma'(g), h = v·u (zero where
+// not kept).  Written hi + lo: token-major [NP][F] (du, dg: the dx GEMMs'
+// B operands) and neuron-major [F][NP] (du, dg, h: the dW GEMMs' A operands,
+// zero in the K padding past the last heavy token).  d_bias sums go to dbh.
+struct BwdDhParams {
+  const float* g;
+  const float* u;
+  const float* bias;
+  const uint32_t* kmask;
+  int n_words;
+  const int* hlist;
+  const int* n_rows_dev;
+  int F, NP, act;
+  __nv_bfloat16 *du_hi, *du_lo, *dg_hi, *dg_lo;          // [NP][F]
+  __nv_bfloat16 *duT_hi, *duT_lo, *dgT_hi, *dgT_lo;      // [F][NP]
+  __nv_bfloat16 *hT_hi, *hT_lo;                          // [F][NP]
+  float* dbh;                                            // [F]
+};
+
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(v);
+  lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+struct EpiBwdDh {
+  static constexpr int N_ACC = 1;
+  static constexpr bool DUAL_B = true;   // dy hi + lo
+  using Params = BwdDhParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int n = *o.n_rows_dev, npad = (n + 63) & ~63, j = m0 + etid;
+    const float b = o.bias ? o.bias[j] : 0.0f;
+    const int w = j >> 5;
+    const uint32_t bit = 1u << (j & 31);
+    float dbs = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= npad) break;
+      float dh[16];
+      tmem_ld16(tmem + c, dh);
+      __align__(16) __nv_bfloat16 Tdu_h[16], Tdu_l[16], Tdg_h[16], Tdg_l[16], Th_h[16], Th_l[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = n0 + c + i;
+        float du = 0.f, dg = 0.f, hv = 0.f;
+        if (r < n) {
+          const int t = o.hlist[r];
+          if (o.kmask[(size_t)t * o.n_words + w] & bit) {
+            const float gg = o.g[(size_t)r * o.F + j] + b;
+            const float uu = o.u[(size_t)r * o.F + j];
+            const float v = __bfloat162float(__float2bfloat16_rn(act_fn(gg, o.act)));
+            float slope = 1.0f;
+            if (o.act == ACT_SILU) {
+              const float sg = 1.0f / (1.0f + expf(-gg));
+              slope = sg * (1.0f + gg * (1.0f - sg));
+            }
+            du = dh[i] * v;
+            dg = dh[i] * uu * slope;
+            hv = v * uu;
+          }
+          __nv_bfloat16 hi, lo;
+          split_bf16(du, hi, lo);
+          o.du_hi[(size_t)r * o.F + j] = hi;
+          o.du_lo[(size_t)r * o.F + j] = lo;
+          split_bf16(dg, hi, lo);
+          o.dg_hi[(size_t)r * o.F + j] = hi;
+          o.dg_lo[(size_t)r * o.F + j] = lo;
+          dbs += dg;
+        }
+        split_bf16(du, Tdu_h[i], Tdu_l[i]);
+        split_bf16(dg, Tdg_h[i], Tdg_l[i]);
+        split_bf16(hv, Th_h[i], Th_l[i]);
+      }
+      // neuron-major: 16 consecutive tokens of row j, two 16-byte stores each
+      const size_t off = (size_t)j * o.NP + n0 + c;
+      __nv_bfloat16* dst[6] = {o.duT_hi, o.duT_lo, o.dgT_hi, o.dgT_lo, o.hT_hi, o.hT_lo};
+      const __nv_bfloat16* src[6] = {Tdu_h, Tdu_l, Tdg_h, Tdg_l, Th_h, Th_l};
+#pragma unroll
+      for (int q = 0; q < 6; ++q) {
+        reinterpret_cast<uint4*>(dst[q] + off)[0] = reinterpret_cast<const uint4*>(src[q])[0];
+        reinterpret_cast<uint4*>(dst[q] + off)[1] = reinterpret_cast<const uint4*>(src[q])[1];
+      }
+    }
+    if (dbs != 0.0f) atomicAdd(&o.dbh[j], dbs);
+  }
+};
+
+// D[rows][cols] added into dst (fp32, row-major, ld), rows below `rows` and
+// columns below `cols`: the heavy tokens' share of dW_gate, dW_up, dW_down
+struct AddParams {
+  float* dst;
+  long long ld;
+  int rows, cols;
+};
+
+template <bool DUAL>
+struct EpiAddF32T {
+  static constexpr int N_ACC = 1;
+  static constexpr bool DUAL_B = DUAL;     // B split hi + lo ...
+  static constexpr bool DUAL_ALL = DUAL;   // ... in both phases (A hi, then A lo)
+  using Params = AddParams;
+  template <int BN>
+  __device__ static void run(const Params& o, uint32_t tmem, int m0, int n0, int, int etid, uint8_t*) {
+    const int r = m0 + etid;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 16) {
+      if (n0 + c >= o.cols) break;
+      float v[16];
+      tmem_ld16(tmem + c, v);
+      if (r < o.rows) {
+        float* dst = o.dst + (size_t)r * o.ld + n0 + c;
+        if (n0 + c + 16 <= o.cols) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float4 p = reinterpret_cast<float4*>(dst)[q];
+            p.x += v[4 * q];
+            p.y += v[4 * q + 1];
+            p.z += v[4 * q + 2];
+            p.w += v[4 * q + 3];
+            reinterpret_cast<float4*>(dst)[q] = p;
+          }
+        } else {
+          for (int i = 0; i < 16 && n0 + c + i < o.cols; ++i) dst[i] += v[i];
+        }
+      }
+    }
+  }
+};
+using EpiAddF32 = EpiAddF32T<false>;
+using EpiAddF32Dual = EpiAddF32T<true>;
 
 }  // namespace sffn

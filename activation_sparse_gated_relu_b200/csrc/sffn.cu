@@ -51,12 +51,12 @@ constexpr int kMaxMarks = 12;
 enum KernelLabel { L_GATE_Z, L_GATE, L_WINA_TOPK, L_ROUTER, L_UPDOWN_ROWS, L_TILE_H, L_FALLBACK_H, L_DOWN,
                    L_GATE_F32, L_ROWS_F32, L_FALLBACK_F32, L_DECODE, L_ROTATE_X, L_INPUT_SELECT,
                    L_GSI_PROJECT, L_GSI_RESID, L_GSI_OUT, L_MOE_ROUTE, L_MOE_COMBINE,
-                   L_BWD_INDEX, L_BWD_TOKEN, L_BWD_NEURON, L_COUNT };
+                   L_BWD_INDEX, L_BWD_TOKEN, L_BWD_NEURON, L_BWD_DENSE, L_COUNT };
 const char* const kLabelNames[L_COUNT] = {"gate_lowrank_z", "gate", "wina_topk", "router", "updown_rows",
                                           "tile_h", "fallback_h", "down", "gate_f32", "rows_f32",
                                           "fallback_f32", "decode_fused", "rotate_x", "input_select",
                                           "gsi_project", "gsi_resid", "gsi_out", "moe_route", "moe_combine",
-                                          "bwd_index", "bwd_token", "bwd_neuron"};
+                                          "bwd_index", "bwd_token", "bwd_neuron", "bwd_dense"};
 constexpr int kMaxTokensLimit = 16384;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -264,6 +264,22 @@ struct sffn_handle : KTiming {
   int* bw_cscpos = nullptr;
   int* bw_csctok = nullptr;
   int bw_smem = 0;
+  // the dense channel of the heavy (overflow) tokens; NP = max_tokens rounded up to 64
+  int bw_NP = 0;
+  int* bw_heavy = nullptr;
+  int* bw_hlist = nullptr;
+  int* bw_nheavy = nullptr;
+  float* bw_dbh = nullptr;
+  __nv_bfloat16 *bw_xh = nullptr, *bw_dyh_hi = nullptr, *bw_dyh_lo = nullptr;       // [NP][d]
+  __nv_bfloat16 *bw_xhT = nullptr, *bw_dyhT_hi = nullptr, *bw_dyhT_lo = nullptr;    // [d][NP]
+  float *bw_g = nullptr, *bw_u = nullptr;                                            // [NP][F]
+  __nv_bfloat16 *bw_du_hi = nullptr, *bw_du_lo = nullptr, *bw_dg_hi = nullptr, *bw_dg_lo = nullptr;  // [NP][F]
+  __nv_bfloat16 *bw_duT_hi = nullptr, *bw_duT_lo = nullptr, *bw_dgT_hi = nullptr, *bw_dgT_lo = nullptr;
+  __nv_bfloat16 *bw_hT_hi = nullptr, *bw_hT_lo = nullptr;                            // [F][NP]
+  __nv_bfloat16 *bw_WuT = nullptr, *bw_WgT = nullptr;                                // [d][F]
+  CUtensorMap bm_Wd, bm_WuT, bm_WgT, bm_duT_hi, bm_duT_lo, bm_dgT_hi, bm_dgT_lo, bm_hT_hi, bm_hT_lo;  // A (128 rows)
+  CUtensorMap bm_xh, bm_dyh_hi, bm_dyh_lo, bm_du_hi, bm_du_lo, bm_dg_hi, bm_dg_lo, bm_xhT, bm_dyhT_hi,
+      bm_dyhT_lo;                                                                    // B (256 rows)
   void* arena = nullptr;         // the one device allocation all of the above live in
   size_t arena_bytes = 0;
   bool dense_bufs = false;       // xo, h_hi, h_lo and W_down^T exist (paths other than the single launch)
@@ -552,6 +568,10 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   if (!e && (desc->flags & SFFN_FLAG_BACKWARD)) {
     h->bw_smem = BwdTokenSmem::make((int)d).total;
     e = cudaFuncSetAttribute(k_bwd_token, cudaFuncAttributeMaxDynamicSharedMemorySize, h->bw_smem);
+    e = e ? e : set_tc_attrs<EpiStoreGU>();
+    e = e ? e : set_tc_attrs<EpiBwdDh>();
+    e = e ? e : set_tc_attrs<EpiAddF32>();
+    e = e ? e : set_tc_attrs<EpiAddF32Dual>();
   }
   if (!e) e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize, router_smem_bytes((int)T));
   if (!e && h->f32) {
@@ -637,6 +657,32 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       a.take(&h->bw_colptr, (F + 1) * 4);
       a.take(&h->bw_cscpos, pairs * 4);
       a.take(&h->bw_csctok, pairs * 4);
+      const size_t NP = (T + 63) / 64 * 64;
+      h->bw_NP = (int)NP;
+      a.take(&h->bw_heavy, T * 4);
+      a.take(&h->bw_hlist, T * 4);
+      a.take(&h->bw_nheavy, 16);
+      a.take(&h->bw_dbh, F * 4);
+      a.take(&h->bw_xh, NP * d * 2);
+      a.take(&h->bw_dyh_hi, NP * d * 2);
+      a.take(&h->bw_dyh_lo, NP * d * 2);
+      a.take(&h->bw_xhT, d * NP * 2);
+      a.take(&h->bw_dyhT_hi, d * NP * 2);
+      a.take(&h->bw_dyhT_lo, d * NP * 2);
+      a.take(&h->bw_g, NP * F * 4);
+      a.take(&h->bw_u, NP * F * 4);
+      a.take(&h->bw_du_hi, NP * F * 2);
+      a.take(&h->bw_du_lo, NP * F * 2);
+      a.take(&h->bw_dg_hi, NP * F * 2);
+      a.take(&h->bw_dg_lo, NP * F * 2);
+      a.take(&h->bw_duT_hi, F * NP * 2);
+      a.take(&h->bw_duT_lo, F * NP * 2);
+      a.take(&h->bw_dgT_hi, F * NP * 2);
+      a.take(&h->bw_dgT_lo, F * NP * 2);
+      a.take(&h->bw_hT_hi, F * NP * 2);
+      a.take(&h->bw_hT_lo, F * NP * 2);
+      a.take(&h->bw_WuT, d * F * 2);
+      a.take(&h->bw_WgT, d * F * 2);
     }
     if (h->dec_ok) {
       h->dsched_ints = decode_sched_ints((int)P, h->dec_grid + 1);
@@ -720,6 +766,25 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       k_col_norms_finish<<<cdiv(d, 256), 256, 0, st>>>(h->colacc, (int)d, h->colnorm);
       e = cudaGetLastError();
     }
+  }
+  // the backward's dense channel: W_up^T and W_gate^T (the A operands of dx)
+  // and the tensor maps of its buffers
+  if (!e && h->bw_WuT) {
+    k_transpose_bf16<<<dim3(cdiv(d, 32), cdiv(F, 32)), tb, 0, st>>>(h->Wu, h->bw_WuT, (int)F, (int)d);
+    k_transpose_bf16<<<dim3(cdiv(d, 32), cdiv(F, 32)), tb, 0, st>>>(h->Wg, h->bw_WgT, (int)F, (int)d);
+    e = cudaGetLastError();
+    const long long NP = h->bw_NP;
+    bool mk = make_map(&h->bm_Wd, desc->W_down, d, F, 128) && make_map(&h->bm_WuT, h->bw_WuT, F, d, 128) &&
+              make_map(&h->bm_WgT, h->bw_WgT, F, d, 128) && make_map(&h->bm_duT_hi, h->bw_duT_hi, NP, F, 128) &&
+              make_map(&h->bm_duT_lo, h->bw_duT_lo, NP, F, 128) && make_map(&h->bm_dgT_hi, h->bw_dgT_hi, NP, F, 128) &&
+              make_map(&h->bm_dgT_lo, h->bw_dgT_lo, NP, F, 128) && make_map(&h->bm_hT_hi, h->bw_hT_hi, NP, F, 128) &&
+              make_map(&h->bm_hT_lo, h->bw_hT_lo, NP, F, 128) && make_map(&h->bm_xh, h->bw_xh, d, NP, 256) &&
+              make_map(&h->bm_dyh_hi, h->bw_dyh_hi, d, NP, 256) && make_map(&h->bm_dyh_lo, h->bw_dyh_lo, d, NP, 256) &&
+              make_map(&h->bm_du_hi, h->bw_du_hi, F, NP, 256) && make_map(&h->bm_du_lo, h->bw_du_lo, F, NP, 256) &&
+              make_map(&h->bm_dg_hi, h->bw_dg_hi, F, NP, 256) && make_map(&h->bm_dg_lo, h->bw_dg_lo, F, NP, 256) &&
+              make_map(&h->bm_xhT, h->bw_xhT, NP, d, 256) && make_map(&h->bm_dyhT_hi, h->bw_dyhT_hi, NP, d, 256) &&
+              make_map(&h->bm_dyhT_lo, h->bw_dyhT_lo, NP, d, 256);
+    if (!e && !mk) e = cudaErrorInvalidValue;
   }
   // A-operand tensor maps
   if (!e && !h->f32) {
@@ -2072,6 +2137,13 @@ extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float*
   a.dW_up = dW_up;
   a.dW_down = dW_down;
   a.db = d_bias;
+  a.ovf = h->ovf;
+  a.epoch = h->last_epoch;
+  a.heavy = h->bw_heavy;
+  a.hlist = h->bw_hlist;
+  a.n_heavy = h->bw_nheavy;
+  a.dbh = d_bias ? h->bw_dbh : nullptr;
+  const int NP = h->bw_NP, d = h->d, F = h->F, P = h->P;
   tmark_follow(h);
   tmark(h, st, L_BWD_INDEX);
   if (launch_pdl(k_bwd_rows, dim3(T), dim3(BW_THREADS), 0, st, 1, a)) return SFFN_ERR_CUDA;
@@ -2079,6 +2151,51 @@ extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float*
   tmark(h, st, L_BWD_TOKEN);
   if (launch_pdl(k_bwd_token, dim3(2 * h->n_sm), dim3(BW_THREADS), (size_t)h->bw_smem, st, 1, a))
     return SFFN_ERR_CUDA;
+  // dense channel of the heavy tokens ([TwELL] hybrid routing): their x and
+  // dy rows gathered (and transposed), g and u over every neuron, dh with the
+  // pair values, dx = du W_up + dg W_gate on the tensor cores
+  {
+    tmark(h, st, L_BWD_DENSE);
+    HeavyPrepArgs pa{a.x, dy, h->bw_hlist, h->bw_nheavy, h->bw_xh, h->bw_dyh_hi, h->bw_dyh_lo, h->bw_xhT,
+                     h->bw_dyhT_hi, h->bw_dyhT_lo, h->bw_dbh, d, F, NP};
+    if (launch_pdl(k_bwd_heavy_prep, dim3(cdiv(d, 32), NP / 32), dim3(32, 8), 0, st, 1, pa)) return SFFN_ERR_CUDA;
+    const int BN = 256, ntok = cdiv(NP, BN);
+    TcArgs ga{};
+    ga.n_phase = 2;
+    ga.kb_total[0] = ga.kb_total[1] = cdiv(d, 64);
+    ga.n_rows = T;
+    ga.n_rows_dev = h->bw_nheavy;
+    ga.status = h->status;
+    GuParams gp{h->bw_g, h->bw_u, h->bw_nheavy, F};
+    if (launch_tc<EpiStoreGU>(BN, dim3(P, ntok, 1), st, h->tmWgate, h->bm_xh, h->tmWup, h->bm_xh, ga, gp))
+      return SFFN_ERR_CUDA;
+    TcArgs da{};
+    da.n_phase = 1;
+    da.kb_total[0] = cdiv(d, 64);
+    da.n_rows = T;
+    da.n_rows_dev = h->bw_nheavy;
+    da.status = h->status;
+    BwdDhParams dp{h->bw_g, h->bw_u, h->desc.gate_bias, h->kmask, F / 32, h->bw_hlist, h->bw_nheavy, F, NP,
+                   h->desc.act, h->bw_du_hi, h->bw_du_lo, h->bw_dg_hi, h->bw_dg_lo, h->bw_duT_hi, h->bw_duT_lo,
+                   h->bw_dgT_hi, h->bw_dgT_lo, h->bw_hT_hi, h->bw_hT_lo, h->bw_dbh};
+    if (launch_tc<EpiBwdDh>(BN, dim3(P, ntok, 1), st, h->bm_Wd, h->bm_dyh_hi, h->bm_Wd, h->bm_dyh_lo, da, dp))
+      return SFFN_ERR_CUDA;
+    // dx rows of the heavy tokens: W_up^T (du hi + lo), then W_gate^T (dg hi + lo) added
+    TcArgs xa{};
+    xa.n_phase = 1;
+    xa.kb_total[0] = cdiv(F, 64);
+    xa.n_rows = T;
+    xa.n_rows_dev = h->bw_nheavy;
+    xa.status = h->status;
+    OutParams op{dx, d, h->bw_nheavy, T, h->bw_hlist, 0};
+    if (launch_tc<EpiDownOut>(BN, dim3(cdiv(d, 128), ntok, 1), st, h->bm_WuT, h->bm_du_hi, h->bm_WuT, h->bm_du_lo,
+                              xa, op))
+      return SFFN_ERR_CUDA;
+    op.atomic = 1;
+    if (launch_tc<EpiDownOut>(BN, dim3(cdiv(d, 128), ntok, 1), st, h->bm_WgT, h->bm_dg_hi, h->bm_WgT, h->bm_dg_lo,
+                              xa, op))
+      return SFFN_ERR_CUDA;
+  }
   tmark(h, st, L_BWD_INDEX);
   const dim3 gcol(cdiv(h->F, 256), cdiv(T, BW_TCH));
   if (launch_pdl(k_bwd_colcount, gcol, dim3(256), 0, st, 1, a)) return SFFN_ERR_CUDA;
@@ -2091,6 +2208,28 @@ extern "C" sffn_status sffn_backward(sffn_handle* h, const void* x, const float*
                              ? launch_pdl(k_bwd_neuron<1>, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a)
                              : launch_pdl(k_bwd_neuron<2>, dim3(h->F), dim3(BW_THREADS), 0, st, 1, a);
   if (en) return SFFN_ERR_CUDA;
+  // the heavy tokens' dW rows, added: K = the heavy tokens (device count),
+  // A = the neuron-major pair values (hi, then lo), B = x^T or dy^T (hi + lo)
+  {
+    tmark(h, st, L_BWD_DENSE);
+    const int BN = 256;
+    TcArgs wa{};
+    wa.n_phase = 2;
+    wa.acc_same = 1;
+    wa.kb_dev = h->bw_nheavy;
+    wa.n_rows = d;
+    wa.status = h->status;
+    const dim3 gw(P, cdiv(d, BN), 1);
+    AddParams ap{dW_up, (long long)d, F, d};
+    if (launch_tc<EpiAddF32>(BN, gw, st, h->bm_duT_hi, h->bm_xhT, h->bm_duT_lo, h->bm_xhT, wa, ap))
+      return SFFN_ERR_CUDA;
+    ap.dst = dW_gate;
+    if (launch_tc<EpiAddF32>(BN, gw, st, h->bm_dgT_hi, h->bm_xhT, h->bm_dgT_lo, h->bm_xhT, wa, ap))
+      return SFFN_ERR_CUDA;
+    ap.dst = dW_down;
+    if (launch_tc<EpiAddF32Dual>(BN, gw, st, h->bm_hT_hi, h->bm_dyhT_hi, h->bm_hT_lo, h->bm_dyhT_lo, wa, ap))
+      return SFFN_ERR_CUDA;
+  }
   tmark_end(h, st);
   return SFFN_OK;
 }

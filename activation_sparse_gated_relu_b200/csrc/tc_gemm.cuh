@@ -48,6 +48,8 @@ struct TcArgs {
   float4* zero_out;     // if set, the CTAs zero zero_n4 float4 here (after the grid dependency)
   long long zero_n4;
   int stages;           // ring stages in use (0: all that fit); fewer bound the bytes in flight
+  const int* kb_dev;    // if set, every phase's K is *kb_dev rows (64-wide blocks rounded up), read
+                        // from the device after the grid dependency (a count an earlier kernel wrote)
   unsigned long long hold_ns;  // test hook (0: off): before issuing any copy the producer waits
                                // this long on a barrier that nothing signals, then records a
                                // timeout and the CTA returns without output
@@ -60,6 +62,16 @@ struct epi_dual_b {
 template <class E>
 struct epi_dual_b<E, decltype(void(E::DUAL_B))> {
   static constexpr bool value = E::DUAL_B;
+};
+// DUAL_ALL: every phase multiplies its A by the same pair (B0 + B1) (without
+// it, a phase after the first reads its single B from mB1)
+template <class E, class = void>
+struct epi_dual_all {
+  static constexpr bool value = false;
+};
+template <class E>
+struct epi_dual_all<E, decltype(void(E::DUAL_ALL))> {
+  static constexpr bool value = E::DUAL_ALL;
 };
 template <class E, class = void>
 struct epi_smem {
@@ -140,6 +152,11 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
   griddep_wait();  // inputs and outputs may belong to earlier kernels on the stream
 
   const int S = gridDim.z, sk = blockIdx.z;
+  int kb_tot[2] = {args.kb_total[0], args.kb_total[1]};
+  if (args.kb_dev) {
+    const int kd = (*args.kb_dev + TC_BK - 1) / TC_BK;
+    kb_tot[0] = kb_tot[1] = kd;
+  }
 
   if (warp == 4) {
     if (lane == 0) {
@@ -159,9 +176,9 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       }
       for (int ph = 0; ph < args.n_phase && ok; ++ph) {
         const CUtensorMap* ma = ph == 0 ? &mA0 : &mA1;
-        const CUtensorMap* mb = ph == 0 ? &mB0 : &mB1;
-        const int kb0 = (int)((long long)args.kb_total[ph] * sk / S);
-        const int kb1 = (int)((long long)args.kb_total[ph] * (sk + 1) / S);
+        const CUtensorMap* mb = (ph == 0 || epi_dual_all<Epi>::value) ? &mB0 : &mB1;
+        const int kb0 = (int)((long long)kb_tot[ph] * sk / S);
+        const int kb1 = (int)((long long)kb_tot[ph] * (sk + 1) / S);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES, f = it / STAGES;
           if (f > 0 && !mbar_wait(&empty[s], (f - 1) & 1, abort_flag, args.status)) {
@@ -193,8 +210,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
       bool ok = true;
       for (int ph = 0; ph < args.n_phase && ok; ++ph) {
         const uint32_t dcol = args.acc_same ? 0u : (uint32_t)(ph * BN);
-        const int kb0 = (int)((long long)args.kb_total[ph] * sk / S);
-        const int kb1 = (int)((long long)args.kb_total[ph] * (sk + 1) / S);
+        const int kb0 = (int)((long long)kb_tot[ph] * sk / S);
+        const int kb1 = (int)((long long)kb_tot[ph] * (sk + 1) / S);
         bool first = (ph == 0) || !args.acc_same;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES, f = it / STAGES;
@@ -234,7 +251,11 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUten
         args.zero_out[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
-    if (mbar_wait(accf, 0, abort_flag, args.status) && !*abort_flag) {
+    // a CTA whose K range is empty (a device-side K of 0) has no accumulator to read
+    bool any_k = false;
+    for (int ph = 0; ph < args.n_phase; ++ph)
+      any_k |= (long long)kb_tot[ph] * (sk + 1) / S > (long long)kb_tot[ph] * sk / S;
+    if (mbar_wait(accf, 0, abort_flag, args.status) && !*abort_flag && any_k) {
       tc_fence_after();
       Epi::template run<BN>(ep, tlane, m0, n0, sk, threadIdx.x, scratch);
     }

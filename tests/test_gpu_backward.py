@@ -70,6 +70,16 @@ def test_backward_exact_grid_small(T):
     _check(inp, T, exact=True)
 
 
+@pytest.mark.parametrize("C", [8, 16])
+def test_backward_heavy_tokens_exact_grid(C):
+    # a small tile capacity makes most tokens overflow: their gradients take
+    # the dense tensor-core channel, the others the sparse passes
+    inp = synth.make_inputs(synth.Workload("small", 256, 512, 32, tile_capacity=C, exact_grid=True))
+    res = oracle.forward_inputs(inp, T=32)
+    assert res.overflow.any() and (C == 8 or not res.overflow.all())
+    _check(inp, 32, exact=True, C=C)
+
+
 def test_backward_silu_threshold_gaussian():
     inp = synth.make_inputs(synth.Workload("small", 512, 1024, 40, tile_capacity=16, act="silu",
                                            threshold=0.3, bias=None))
@@ -77,7 +87,7 @@ def test_backward_silu_threshold_gaussian():
 
 
 def test_backward_after_single_launch_decode():
-    inp = synth.make_inputs(W["decode_bf16"].with_(d_model=1024, d_ff=4096))
+    inp = synth.make_inputs(W["decode_bf16"].with_(d_model=1024, d_ff=4096, tile_capacity=8))
     _check(inp, 8, exact=False)
 
 
