@@ -77,6 +77,7 @@ KERNEL_SOURCES = {
     "down": ["tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "updown_rows": ["rows_mma.cuh", "ptx.cuh"],
     "decode_fused": ["decode_fused.cuh", "rows_mma.cuh", "epilogues.cuh", "ptx.cuh"],
+    "tile_fused": ["tile_fused.cuh", "tc_gemm.cuh", "epilogues.cuh", "ptx.cuh"],
     "router": ["simt.cuh", "ptx.cuh"],
     "wina_topk": ["simt.cuh", "ptx.cuh"],
     "gate_f32": ["simt.cuh", "epilogues.cuh", "ptx.cuh"],
@@ -305,6 +306,13 @@ def kernel_work(wl, T: int, path: str, st: dict) -> dict:
         w["decode_fused"] = {"bytes": F * d * es + xb + Ua * 2 * d * es + yb + twell + kmask,
                              "flops": 2 * T * d * F + 4 * nnza * d}
     else:
+        # the single tile launch (up to 32 tokens, threshold selection): the
+        # gate's weights, the W_up and W_down rows of the kept neurons' union,
+        # x in, y out, the TwELL records written
+        if wl.mode == "relu_threshold":
+            gw = (d * R + R * F) * es if R else F * d * es
+            w["tile_fused"] = {"bytes": gw + U * 2 * d * es + xb + yb + twell,
+                               "flops": (2 * T * (d * R + R * F) if R else 2 * T * d * F) + 4 * T * F * d}
         w["router"] = {"bytes": yb + 2 * n_o * d * es, "flops": 0}
         if wl.mode != "wina_full_h":
             w["tile_h"] = {"bytes": F * d * es + xb + twell + T * F * 4, "flops": 2 * T * d * F}

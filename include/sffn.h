@@ -97,16 +97,23 @@ typedef enum { SFFN_ACT_RELU = 0, SFFN_ACT_SILU = 1 } sffn_act;
  *          dense channel) runs as one persistent launch;
  *   TILES: tensor-core up and down over every 128-neuron tile that some token
  *          keeps, with the non-kept entries of h zeroed (best when the union
- *          of kept neurons covers most tiles: WINA, T in 16..256).
+ *          of kept neurons covers most tiles: WINA, T in 16..256).  At
+ *          T <= 32 in relu-threshold mode with the low-rank gate (with the
+ *          dense gate: SFFN_FLAG_TILE_SINGLE) the whole forward runs as one
+ *          persistent launch;
  *   AUTO : ROWS for T <= 8 or T > 256 in relu-threshold mode, TILES otherwise. */
 typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sffn_path;
 
 /* desc.flags */
 #define SFFN_FLAG_DEBUG_GATE 1u   /* keep the dense fp32 gate g[T][d_ff] of the last forward */
-#define SFFN_FLAG_SEPARATE 2u     /* T <= 8: separate gate, up x down and dense-channel launches
-                                     instead of the single persistent launch (diagnostics, tests) */
+#define SFFN_FLAG_SEPARATE 2u     /* separate gate, up x down and dense-channel launches instead
+                                     of a single persistent launch (ROWS at T <= 8, TILES at
+                                     T <= 32): diagnostics, tests */
 #define SFFN_FLAG_COOPERATIVE 4u  /* launch the single persistent forward with the cooperative
                                      attribute (see sffn_forward) */
+#define SFFN_FLAG_TILE_SINGLE 16u /* dense gate, TILES path at T <= 32: the single persistent
+                                     launch (the default with the low-rank gate only; with the
+                                     dense gate the separate launches measured faster) */
 #define SFFN_FLAG_BACKWARD 8u     /* allocate the workspace of sffn_backward (relu-threshold
                                      mode, dense gate, bf16, no input_k or V) */
 
@@ -165,8 +172,9 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
  * its epoch and could read a previous replay's scheduler words, so stream
  * capture of sffn_forward is not supported.
  *
- * The single persistent launch (T <= 8, ROWS path) has one CTA per SM and its
- * CTAs wait on one another, so it needs all of them resident at once.  That
+ * The single persistent launches (ROWS path at T <= 8, TILES path at T <= 32
+ * in relu-threshold mode, see sffn_path) have one CTA per SM and their CTAs wait on one
+ * another, so each needs all of them resident at once.  That
  * holds when the forward has the GPU's SMs to itself or shares them with
  * ordinary kernels; it need not hold for an MPS client limited to part of the
  * SMs, a green context, or a concurrent persistent kernel that never yields
@@ -204,8 +212,9 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
                              const void** val, const uint32_t** overflow, int* n_tiles,
                              int* tile_capacity);
 
-/* Test hook for the bounded waits of the single-launch decode forward (ROWS
- * path, T <= 8).  Until called again with (0, 0), those forwards count
+/* Test hook for the bounded waits of the single-launch forwards (ROWS path at
+ * T <= 8, TILES path at T <= 32).  Until called again with (0, 0), those
+ * forwards count
  * `phantom_ctas` (0 or 1) extra CTAs in their grid that never run, so every
  * wait on them expires, and limit their waits on other CTAs to `wait_us`
  * microseconds (0: the default of 2 s).  Such a forward's out is not valid
@@ -213,6 +222,18 @@ sffn_status sffn_debug_twell(sffn_handle* h, const int16_t** count, const int16_
  * SFFN_ERR_TIMEOUT and clears the scheduler state); nothing faults or hangs.
  * Errors: SFFN_ERR_INVALID_ARG for a null handle or phantom_ctas not 0 or 1. */
 sffn_status sffn_debug_decode_waits(sffn_handle* h, int phantom_ctas, unsigned wait_us);
+
+/* The job lists of the TILES path's single launch (up to 32 tokens) for a
+ * layer of d_model x d_ff (rank > 0: the low-rank gate) on n_cta CTAs, as the
+ * handle builds them; host only, no device needed.  jobs receives n_jobs
+ * records of 4 ints {type | finisher << 4 | count << 8, tile, k0 | k1 << 16,
+ * id} (type 0 a z range, 1 a tile's gate and first up range, 2 a later up
+ * range, 3 a down range; K in 64-wide blocks), off the n_cta + 1 offsets of
+ * each CTA's list.  Test use: it lets the lists' coverage and wait order be
+ * checked without a GPU.  Errors: SFFN_ERR_INVALID_ARG for sizes out of
+ * range or buffers too small (*n_jobs then holds the count needed). */
+sffn_status sffn_debug_tile_schedule(int d_model, int d_ff, int rank, int n_cta, int* jobs, int max_jobs,
+                                     int* off, int* n_jobs);
 
 /* Test hook: the next forward takes epoch `epoch` + 1 (0 is skipped).  The
  * single-launch decode forward's scheduler words carry the low 16 bits of the

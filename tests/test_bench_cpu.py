@@ -107,7 +107,7 @@ def test_work_model_prefill_gate_is_tensor_bound():
 
 def test_work_model_tile_path_kernels():
     import synth
-    for name, extra in (("lopa_bf16", {"gate_lowrank_z", "fallback_h"}), ("wina_bf16", {"wina_topk"})):
+    for name, extra in (("lopa_bf16", {"gate_lowrank_z", "fallback_h", "tile_fused"}), ("wina_bf16", {"wina_topk"})):
         wl = synth.WORKLOADS[name]
         st = {"union": 14000, "nnz": 32 * 1400, "block_rows": 4 * 14000, "n_overflow": 1}
         w = bench.kernel_work(wl, 32, "tiles", st)
