@@ -24,7 +24,6 @@ SFFN_FLAG_DEBUG_GATE = 1
 SFFN_FLAG_SEPARATE = 2
 SFFN_FLAG_COOPERATIVE = 4
 SFFN_FLAG_BACKWARD = 8
-SFFN_FLAG_TILE_SINGLE = 16
 
 
 class sffn_desc(ctypes.Structure):
@@ -270,8 +269,7 @@ class SparseFFN:
                  mode: str = "relu_threshold", act: str = "relu", threshold: float = 0.0,
                  k: int = 0, tile_capacity: int = 32, max_tokens: int = 8, path: str = "auto",
                  debug_gate: bool = False, separate: bool = False, cooperative: bool = False,
-                 input_k: int = 0, V=None, backward: bool = False, tile_single: bool = False,
-                 stream: Optional[int] = None):
+                 input_k: int = 0, V=None, backward: bool = False, stream: Optional[int] = None):
         import torch
         self.h = None
         self._keep = [t for t in (W_up, W_down, W_gate, A, B, bias, V) if t is not None]
@@ -310,8 +308,7 @@ class SparseFFN:
         desc.tile_capacity = int(tile_capacity)
         desc.path = _PATH[path]
         desc.flags = ((SFFN_FLAG_DEBUG_GATE if debug_gate else 0) | (SFFN_FLAG_SEPARATE if separate else 0)
-                      | (SFFN_FLAG_COOPERATIVE if cooperative else 0) | (SFFN_FLAG_BACKWARD if backward else 0)
-                      | (SFFN_FLAG_TILE_SINGLE if tile_single else 0))
+                      | (SFFN_FLAG_COOPERATIVE if cooperative else 0) | (SFFN_FLAG_BACKWARD if backward else 0))
         ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         desc.W_gate, desc.A, desc.B = ptr(W_gate), ptr(A), ptr(B)
         desc.W_up, desc.W_down, desc.gate_bias = ptr(W_up), ptr(W_down), ptr(bias)

@@ -113,6 +113,8 @@ int z_splits(int d, int m_tiles, int tok_tiles, int n_sm) {
 //     by its z blocks so that phases 0 and 1 together are even;
 //   phase 2: the stream [down of output tile 0] ... [down of output tile
 //     Md-1] cut into n_chunks runs of equal length.
+// A tile here is the kernel's unit, a pair of 128-row tiles (P, Rt and Md
+// count pairs).
 // Phase-1 cuts are moved so that the run holding the end of a tile's gate
 // also holds at least kMinPiece blocks of its up range (the MAIN job), and so
 // that no gate or up piece shorter than kMinPiece is cut off (2 for down).
@@ -128,14 +130,14 @@ struct TfSchedule {
 };
 
 TfSchedule tf_schedule(int n_chunks, int kd, int kg, int P, int Rt, int Md, int Kf) {
-  constexpr int kMinPiece = 4, kZPiece = 8;
+  constexpr int kMinPiece = 2, kZPiece = 8;
   struct Item {
     int type, tile;
     long long s, e;
   };
   TfSchedule S;
   // phase 0: z pieces, piece i of nz to chunk i * n_chunks / nz
-  const int zper = Rt ? std::max(1, cdiv(kd, kZPiece)) : 0, nz = Rt * zper;
+  const int zper = Rt ? std::min(TF_ZMAXP, std::max(1, cdiv(kd, kZPiece))) : 0, nz = Rt * zper;
   std::vector<std::vector<int4>> zjobs(n_chunks);
   std::vector<long long> zload(n_chunks, 0);
   for (int i = 0; i < nz; ++i) {
@@ -251,7 +253,7 @@ TfSchedule tf_schedule(int n_chunks, int kd, int kg, int P, int Rt, int Md, int 
     }
   }
   S.off[n_chunks] = (int)S.jobs.size();
-  if (zper > 0xFF) S.ok = false;
+  if (zper > TF_ZMAXP) S.ok = false;
   for (int p = 0; p < P; ++p)
     if (main_job[p] < 0) S.ok = false;
   S.n_help = hp;
@@ -474,6 +476,7 @@ struct sffn_handle : KTiming {
   int tf_seq = 0;                // the last launch's sequence number
   bool tf_ok = false;
   bool tf_pdl = true;
+  CUtensorMap tf_mgate, tf_mAt, tf_mup, tf_mdT;  // its weight maps (box 64 x 256)
 };
 
 namespace {
@@ -593,8 +596,7 @@ sffn_status validate(const sffn_desc* d) {
   if (d->rank > 0 && (d->dtype != SFFN_BF16 || d->rank % 64 != 0 || d->rank > 4096)) return SFFN_ERR_UNSUPPORTED;
   if (d->dtype == SFFN_FP32 && d->d_ff > 8192) return SFFN_ERR_UNSUPPORTED;
   if ((d->flags & SFFN_FLAG_DEBUG_GATE) && d->rank > 0) return SFFN_ERR_UNSUPPORTED;
-  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE | SFFN_FLAG_COOPERATIVE | SFFN_FLAG_BACKWARD |
-                   SFFN_FLAG_TILE_SINGLE))
+  if (d->flags & ~(SFFN_FLAG_DEBUG_GATE | SFFN_FLAG_SEPARATE | SFFN_FLAG_COOPERATIVE | SFFN_FLAG_BACKWARD))
     return SFFN_ERR_INVALID_ARG;
   // the backward: threshold selection, dense gate, bf16, the plain input
   if ((d->flags & SFFN_FLAG_BACKWARD) && (d->mode != SFFN_MODE_RELU_THRESHOLD || d->rank > 0 ||
@@ -766,18 +768,20 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
   TfSchedule tf_s0, tf_s1;
   if (h->dense_bufs && !h->wina) {
     const TfLayout TL = tf_layout(h->C);
-    const int kd = cdiv(d, 64), kg = h->lowrank ? cdiv(R, 64) : kd, Rt = h->lowrank ? cdiv(R, 128) : 0;
+    // (jobs work on pairs of 128-row tiles)
+    const int kd = cdiv(d, 64), kg = h->lowrank ? cdiv(R, 64) : kd, Rt = h->lowrank ? cdiv(R, 256) : 0;
+    const int P2 = cdiv(P, 2), Md2 = cdiv(d, 256);
     h->tf_grid = h->n_sm;
     h->tf_chunks = h->n_sm;
     h->tf_smem = TL.total;
-    tf_s0 = tf_schedule(h->tf_grid, kd, kg, (int)P, Rt, cdiv(d, 128), (int)(F / 64));
-    tf_s1 = tf_schedule(h->tf_grid + 1, kd, kg, (int)P, Rt, cdiv(d, 128), (int)(F / 64));
+    tf_s0 = tf_schedule(h->tf_grid, kd, kg, P2, Rt, Md2, (int)(F / 64));
+    tf_s1 = tf_schedule(h->tf_grid + 1, kd, kg, P2, Rt, Md2, (int)(F / 64));
     h->tf_ok = tf_s0.ok && tf_s1.ok && TL.stages >= 4 && TL.total <= max_smem;
     if (h->tf_ok) {
       h->tf_max_jobs = (int)std::max(tf_s0.jobs.size(), tf_s1.jobs.size());
       h->tf_max_help = std::max(tf_s0.n_help, tf_s1.n_help);
       h->tf_max_zp = std::max(tf_s0.n_zp, tf_s1.n_zp);
-      h->tf_flag_ints = h->tf_max_zp + Rt + h->tf_max_help + (int)P + h->tf_grid + 1;
+      h->tf_flag_ints = h->tf_max_zp + Rt + h->tf_max_help + P2 + h->tf_grid + 1;
       e = cudaFuncSetAttribute(k_tile_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, h->tf_smem);
       int nb = 0;
       if (!e) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tile_fused, TC_THREADS, h->tf_smem);
@@ -1002,6 +1006,13 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
     mok = mok && make_map(&h->tmWup, h->Wu, h->d, h->F, 128);
     if (h->Vt) mok = mok && make_map(&h->tmVt, h->Vt, h->d, h->d, 128);
     if (h->WdT) mok = mok && make_map(&h->tmWdT, h->WdT, h->F, h->d, 128);
+    if (h->tf_ok) {
+      mok = mok && make_map(&h->tf_mgate, h->lowrank ? static_cast<const void*>(h->Bt) : h->Wg, h->lowrank ? h->R : h->d,
+                            h->F, TF_ROWS);
+      mok = mok && make_map(&h->tf_mup, h->Wu, h->d, h->F, TF_ROWS);
+      mok = mok && make_map(&h->tf_mdT, h->WdT, h->F, h->d, TF_ROWS);
+      if (h->lowrank) mok = mok && make_map(&h->tf_mAt, h->At, h->d, h->R, TF_ROWS);
+    }
     if (h->lowrank) {
       mok = mok && make_map(&h->tmAt, h->At, h->d, h->R, 128);
       mok = mok && make_map(&h->tmBt, h->Bt, h->R, h->F, 128);
@@ -1117,8 +1128,8 @@ static cudaError_t launch_tile_fused(sffn_handle* h, const TfArgs& ta, cudaStrea
 // Uploads the job lists of the fused tile launch for n_chunks runs (the grid,
 // or the grid plus the test hook's CTA that never runs).  Synchronous.
 static bool tf_upload(sffn_handle* h, int n_chunks) {
-  const int kd = cdiv(h->d, 64), kg = h->lowrank ? cdiv(h->R, 64) : kd, Rt = h->lowrank ? cdiv(h->R, 128) : 0;
-  const TfSchedule S = tf_schedule(n_chunks, kd, kg, h->P, Rt, cdiv(h->d, 128), h->F / 64);
+  const int kd = cdiv(h->d, 64), kg = h->lowrank ? cdiv(h->R, 64) : kd, Rt = h->lowrank ? cdiv(h->R, 256) : 0;
+  const TfSchedule S = tf_schedule(n_chunks, kd, kg, cdiv(h->P, 2), Rt, cdiv(h->d, 256), h->F / 64);
   if (!S.ok || (int)S.jobs.size() > h->tf_max_jobs || S.n_help > h->tf_max_help || S.n_zp > h->tf_max_zp)
     return false;
   if (cudaDeviceSynchronize() != cudaSuccess ||
@@ -1229,27 +1240,20 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   }
 
   // ----------------------------- tile path: one persistent launch at T <= 32
-  // (the default with the low-rank gate, where it measured 94.8 against the
-  // separate launches' 94.2 us at 32 tokens, d 4096, d_ff 14336, rank 512, in
-  // one launch instead of five; with the dense gate the separate launches
-  // measured 102 against its 136 us, so there it runs on request only)
-  if (!rows && !h->wina && T <= TF_BN && h->tf_ok && !(D.flags & SFFN_FLAG_SEPARATE) &&
-      (h->lowrank || (D.flags & SFFN_FLAG_TILE_SINGLE))) {
+  // (at 32 tokens, d 4096, d_ff 14336: 89.2 against the separate launches'
+  // 94.2 us with the low-rank gate of rank 512, 86.2 against 102.2 us with
+  // the dense gate)
+  if (!rows && !h->wina && T <= TF_BN && h->tf_ok && !(D.flags & SFFN_FLAG_SEPARATE)) {
     TfArgs ta{};
     bool mok = make_map(&ta.mx, x, d, T, TF_BN) && make_map(&ta.mhi, h->h_hi, F, h->maxT, TF_BN) &&
                make_map(&ta.mlo, h->h_lo, F, h->maxT, TF_BN);
-    if (h->lowrank) {
-      mok = mok && make_map(&ta.mz, h->z, h->R, h->maxT, TF_BN);
-      ta.mgate = h->tmBt;
-      ta.mAt = h->tmAt;
-    } else {
-      ta.mz = ta.mx;  // unused
-      ta.mgate = h->tmWgate;
-      ta.mAt = h->tmWgate;  // unused
-    }
+    if (h->lowrank) mok = mok && make_map(&ta.mz, h->z, h->R, h->maxT, TF_BN);
+    else ta.mz = ta.mx;  // unused
     if (!mok) return SFFN_ERR_CUDA;
-    ta.mup = h->tmWup;
-    ta.mdT = h->tmWdT;
+    ta.mgate = h->tf_mgate;
+    ta.mAt = h->lowrank ? h->tf_mAt : h->tf_mgate;  // (unused with the dense gate)
+    ta.mup = h->tf_mup;
+    ta.mdT = h->tf_mdT;
     ta.jobs = h->tf_jobs;
     ta.job_off = h->tf_off;
     ta.tw = tw;
@@ -1260,7 +1264,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     ta.z = h->z;
     ta.h_hi = h->h_hi;
     ta.h_lo = h->h_lo;
-    const int Rt = h->lowrank ? cdiv(h->R, 128) : 0;
+    const int Rt = h->lowrank ? cdiv(h->R, 256) : 0;
     ta.f_zp = h->tf_flags;
     ta.f_z = ta.f_zp + h->tf_max_zp;
     ta.f_up = ta.f_z + Rt;
@@ -1746,8 +1750,8 @@ sffn_status sffn_debug_tile_schedule(int d_model, int d_ff, int rank, int n_cta,
   if (d_model <= 0 || d_model > 4096 || d_model % 8 || d_ff <= 0 || d_ff % 128 || d_ff > 32767 || rank < 0 ||
       rank % 64 || rank > 4096 || n_cta <= 0 || n_cta > 4096 || !n_jobs)
     return SFFN_ERR_INVALID_ARG;
-  const int kd = cdiv(d_model, 64), kg = rank ? rank / 64 : kd, Rt = rank ? cdiv(rank, 128) : 0;
-  const TfSchedule S = tf_schedule(n_cta, kd, kg, d_ff / 128, Rt, cdiv(d_model, 128), d_ff / 64);
+  const int kd = cdiv(d_model, 64), kg = rank ? rank / 64 : kd, Rt = rank ? cdiv(rank, 256) : 0;
+  const TfSchedule S = tf_schedule(n_cta, kd, kg, cdiv(d_ff / 128, 2), Rt, cdiv(d_model, 256), d_ff / 64);
   if (!S.ok) return SFFN_ERR_UNSUPPORTED;
   *n_jobs = (int)S.jobs.size();
   if (!jobs || !off || max_jobs < (int)S.jobs.size()) return SFFN_ERR_INVALID_ARG;

@@ -5,7 +5,12 @@
 // At 32 tokens nearly every neuron is kept by some token, so the up and down
 // projections stream W_up and W_down^T whole through the tensor cores and the
 // sparsity is applied as a mask on h.  One CTA per SM walks a static list of
-// jobs, built on the host, over one TMA ring and four TMEM accumulators:
+// jobs, built on the host, over one TMA ring and four TMEM accumulator slots.
+// Every job works on a pair of 128-row tiles (256 neurons, rank coordinates
+// or output columns): a ring stage holds one 256-row weight box and one B
+// tile (32 tokens) that both halves multiply, so the small B tiles cost half
+// as much per weight byte as with one tile per stage.  "Tile" below means
+// such a pair.
 //
 //   phase 0 (low-rank gate), the K blocks of z = x·A cut into pieces of a
 //   few blocks, each the first job of its CTA (spread over the grid):
@@ -60,21 +65,26 @@
 namespace sffn {
 
 constexpr int TF_BN = 32;                                  // tokens: one token tile
-constexpr int TF_NACC = 4;                                 // TMEM accumulator slots of TF_BN columns
+constexpr int TF_PAIR = 2;                                 // 128-row tiles per job tile
+constexpr int TF_ROWS = TF_PAIR * TC_BM;                   // 256 weight rows per stage
+constexpr int TF_A_BYTES = TF_PAIR * TC_A_BYTES;           // one 64 x 256 weight box (32 KB)
 constexpr int TF_B_BYTES = TF_BN * TC_BK * 2;              // one B tile (4 KB)
-constexpr int TF_STAGE_BYTES = TC_A_BYTES + 2 * TF_B_BYTES;  // A + two B tiles (24 KB)
-constexpr int TF_MAX_STAGES = 8;
-constexpr int TF_TILE_FLOATS = TF_BN * 128;                // a partial accumulator [32 tokens][128 rows]
+constexpr int TF_STAGE_BYTES = TF_A_BYTES + 2 * TF_B_BYTES;  // weights + up to two B tiles (40 KB)
+constexpr int TF_MAX_STAGES = 6;
+constexpr int TF_NSLOT = 4;                                // TMEM accumulator slots
+constexpr int TF_SLOT_COLS = TF_PAIR * 64;                 // a slot: per half 32 (or 64: hi | lo) columns
+constexpr int TF_TILE_FLOATS = TF_PAIR * TF_BN * 128;      // a partial accumulator [2][32 tokens][128 rows]
+constexpr int TF_ZMAXP = 8;                                // z pieces per rank pair at most
 
 enum : int { TFJ_Z = 0, TFJ_MAIN = 1, TFJ_HELP = 2, TFJ_DOWN = 3, TFJ_GHELP = 4 };
 
 // Job record (int4): x = type | fin << 4 | count << 8 | gcount << 16 (Z:
 // count = pieces of its coordinates, fin = this piece adds them up; MAIN:
-// count = up helpers, gcount = gate helpers), y = tile (rank tile, neuron
-// tile or output-column tile), z = k0 | k1 << 16 (K blocks; MAIN: its gate
-// range is [k0, gate end), its up range [0, k1)), w = id (Z: its piece slot,
-// consecutive in K order within a rank tile; MAIN: its first helper slot,
-// the gate helpers' slots before the up helpers'; HELP, GHELP: its slot).
+// count = up helpers, gcount = gate helpers), y = tile pair (rank, neuron or
+// output-column tiles 2y and 2y + 1), z = k0 | k1 << 16 (K blocks; MAIN: its
+// gate range is [k0, gate end), its up range [0, k1)), w = id (Z: its piece
+// slot, consecutive in K order within a rank pair; MAIN: its first helper
+// slot, the gate helpers' slots before the up helpers'; HELP, GHELP: its slot).
 __host__ __device__ inline int4 tf_job(int type, int fin, int count, int gcount, int tile, int k0, int k1, int id) {
   return make_int4(type | (fin << 4) | (count << 8) | (gcount << 16), tile, k0 | (k1 << 16), id);
 }
@@ -98,23 +108,23 @@ struct TfArgs {
   CUtensorMap mz;      // z [maxT][R] (low rank)
   CUtensorMap mhi;     // h_hi [maxT][F]
   CUtensorMap mlo;     // h_lo [maxT][F]
-  CUtensorMap mgate;   // the gate's A: W_gate [F][d], or B^T [F][R]
-  CUtensorMap mAt;     // A^T [R][d] (low rank)
-  CUtensorMap mup;     // W_up [F][d]
-  CUtensorMap mdT;     // W_down^T [d][F]
+  CUtensorMap mgate;   // the gate's A: W_gate [F][d], or B^T [F][R]; box 64 x 256
+  CUtensorMap mAt;     // A^T [R][d] (low rank); box 64 x 256
+  CUtensorMap mup;     // W_up [F][d]; box 64 x 256
+  CUtensorMap mdT;     // W_down^T [d][F]; box 64 x 256
   const int4* jobs;
   const int* job_off;  // [n_chunks + 1]: CTA c runs jobs [job_off[c], job_off[c + 1])
   TwellParams tw;      // T, F, n_tiles, C, tau, act, TwELL outputs, overflow epoch (bias null)
   const float* bias;   // [F] or null: added to the gate before the emission
-  float* zpart;        // [z pieces][32][128]
-  float* upart;        // [helper slots][32][128]
+  float* zpart;        // [z pieces][2][32][128]
+  float* upart;        // [helper slots][2][32][128]
   __nv_bfloat16* z;    // [maxT][R]
   __nv_bfloat16* h_hi; // [maxT][F]
   __nv_bfloat16* h_lo;
   int* f_zp;           // [z pieces]  = seq once the piece's partial sum is stored
-  int* f_z;            // [R / 128]   = seq once z of those coordinates is stored
+  int* f_z;            // [R / 256]   = seq once z of those coordinates is stored
   int* f_up;           // [helper slots] = seq once the helper's partial is stored
-  int* f_h;            // [F / 128]   = seq once h of the tile is stored
+  int* f_h;            // [F / 256]   = seq once h of the tile pair is stored
   int* f_zero;         // [n_chunks]  = seq once the CTA's slice of out is zeroed
   float* out;          // [T][d]
   int d, R, maxT, kb_gate, lowrank, n_chunks;
@@ -128,7 +138,7 @@ enum : int { TFA_GATE = 0, TFA_AT = 1, TFA_UP = 2, TFA_DT = 3 };  // the A opera
 struct TfSeg {
   int amap;  // TFA_*
   int arow, k0, k1;
-  int kind;  // B operand: 0 x; 1 z (flag f_z[kb / 2]); 2 the h pair (flag f_h[kb / 2])
+  int kind;  // B operand: 0 x; 1 z (flag f_z[kb / 4]); 2 the h pair (flag f_h[kb / 4])
 };
 
 __device__ __forceinline__ int tf_type(const int4& j) { return j.x & 15; }
@@ -136,12 +146,13 @@ __device__ __forceinline__ int tf_nseg(const int4& j) { return tf_type(j) == TFJ
 __device__ __forceinline__ TfSeg tf_seg(const TfArgs& a, const int4& j, int s) {
   const int t = j.y, k0 = j.z & 0xFFFF, k1 = (int)((unsigned)j.z >> 16);
   switch (tf_type(j)) {
-    case TFJ_Z: return TfSeg{TFA_AT, t * 128, k0, k1, 0};
+    case TFJ_Z: return TfSeg{TFA_AT, t * TF_ROWS, k0, k1, 0};
     case TFJ_MAIN:  // the up range first: the gate's B operand (z) may be published later
-      return s == 0 ? TfSeg{TFA_UP, t * 128, 0, k1, 0} : TfSeg{TFA_GATE, t * 128, k0, a.kb_gate, a.lowrank ? 1 : 0};
-    case TFJ_GHELP: return TfSeg{TFA_GATE, t * 128, k0, k1, a.lowrank ? 1 : 0};
-    case TFJ_HELP: return TfSeg{TFA_UP, t * 128, k0, k1, 0};
-    default: return TfSeg{TFA_DT, t * 128, k0, k1, 2};
+      return s == 0 ? TfSeg{TFA_UP, t * TF_ROWS, 0, k1, 0}
+                    : TfSeg{TFA_GATE, t * TF_ROWS, k0, a.kb_gate, a.lowrank ? 1 : 0};
+    case TFJ_GHELP: return TfSeg{TFA_GATE, t * TF_ROWS, k0, k1, a.lowrank ? 1 : 0};
+    case TFJ_HELP: return TfSeg{TFA_UP, t * TF_ROWS, k0, k1, 0};
+    default: return TfSeg{TFA_DT, t * TF_ROWS, k0, k1, 2};
   }
 }
 
@@ -252,8 +263,9 @@ __device__ __forceinline__ bool tf_flag_wait(const int* f, int seq, volatile int
 }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_constant__ TfArgs a) {
-  constexpr uint32_t NCOLS = tmem_cols_for(TF_NACC * TF_BN);
-  constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, TF_BN);
+  constexpr uint32_t NCOLS = tmem_cols_for(TF_NSLOT * TF_SLOT_COLS);
+  constexpr uint32_t IDESC = idesc_bf16_f32(TC_BM, TF_BN);        // B: 32 token rows
+  constexpr uint32_t IDESC2 = idesc_bf16_f32(TC_BM, 2 * TF_BN);   // B: the h pair, hi rows then lo rows
   const TfLayout L = tf_layout(a.tw.C);
   const int STAGES = L.stages;
 
@@ -261,9 +273,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + TF_MAX_STAGES;
-  uint64_t* accfull = empty + TF_MAX_STAGES;  // [TF_NACC]
-  uint64_t* accfree = accfull + TF_NACC;      // [TF_NACC]
-  uint64_t* mma_done = accfree + TF_NACC;
+  uint64_t* accfull = empty + TF_MAX_STAGES;  // [TF_NSLOT]
+  uint64_t* accfree = accfull + TF_NSLOT;     // [TF_NSLOT]
+  uint64_t* mma_done = accfree + TF_NSLOT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* scratch = smem + L.scratch;
@@ -279,7 +291,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < TF_NACC; ++b) {
+    for (int b = 0; b < TF_NSLOT; ++b) {
       mbar_init(&accfull[b], 1);
       mbar_init(&accfree[b], 1);
     }
@@ -299,8 +311,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
   if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------------- TMA producer
-      // Two cursors over the same block sequence: A (weights) loads run ahead
-      // as ring stages free up; each B load follows once its operand is
+      // Two cursors over the same block sequence: weight boxes run ahead as
+      // ring stages free up; each B load follows once its operand is
       // published.  A stage's barrier expects both.
       tma_prefetch_desc(&a.mgate);
       tma_prefetch_desc(&a.mup);
@@ -313,7 +325,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
       auto stage = [&](int i) { return smem + (size_t)(i % STAGES) * TF_STAGE_BYTES; };
       auto issue_a = [&](int i) {
         uint64_t* bar = &full[i % STAGES];
-        mbar_expect_tx(bar, (uint32_t)(TC_A_BYTES + (ia.seg.kind == 2 ? 2 : 1) * TF_B_BYTES));
+        mbar_expect_tx(bar, (uint32_t)(TF_A_BYTES + (ia.seg.kind == 2 ? 2 : 1) * TF_B_BYTES));
         const int c0 = ia.kb * TC_BK, c1 = ia.seg.arow;
         switch (ia.seg.amap) {  // (one call per map: the maps stay kernel parameters)
           case TFA_GATE: tma_load_2d(stage(i), &a.mgate, bar, c0, c1); break;
@@ -324,13 +336,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
       };
       auto issue_b = [&](int i) {
         uint64_t* bar = &full[i % STAGES];
-        uint8_t* sb = stage(i) + TC_A_BYTES;
+        uint8_t* sb = stage(i) + TF_A_BYTES;
         const int c0 = ib.kb * TC_BK;
         if (ib.seg.kind == 0) {
           tma_load_2d(sb, &a.mx, bar, c0, 0);
         } else if (ib.seg.kind == 1) {
           tma_load_2d(sb, &a.mz, bar, c0, 0);
-        } else {
+        } else {  // hi rows then lo rows: one 64-row B operand
           tma_load_2d(sb, &a.mhi, bar, c0, 0);
           tma_load_2d(sb + TF_B_BYTES, &a.mlo, bar, c0, 0);
         }
@@ -341,8 +353,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
         ia.next(a);
       }
       griddep_wait();
-      // tiles [hz_lo, hz_hi) of the B operand kind hz_kind are known to be
-      // published; flags are read eight at a time (independent loads, one
+      // tile pairs [hz_lo, hz_hi) of the B operand kind hz_kind are known to
+      // be published; flags are read eight at a time (independent loads, one
       // acquire fence), since a down range walks many tiles
       int hz_kind = -1, hz_lo = 0, hz_hi = 0;
       bool abort = false;
@@ -351,10 +363,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
         bool prog = false;
         while (bi < ai) {
           if (!abort && ib.seg.kind != 0) {
-            const int tile = ib.kb >> 1;
+            const int tile = ib.kb >> 2;  // 4 K blocks of 64 per 256-row pair
             if (ib.seg.kind != hz_kind || tile < hz_lo || tile >= hz_hi) {
               const int* f = ib.seg.kind == 1 ? a.f_z : a.f_h;
-              const int last = (ib.seg.k1 - 1) >> 1;
+              const int last = (ib.seg.k1 - 1) >> 2;
               int fv[8];
 #pragma unroll
               for (int q = 0; q < 8; ++q) fv[q] = tile + q <= last ? ld_relaxed_gpu(f + tile + q) : 0;
@@ -414,20 +426,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
   } else if (warp == 5) {
     if (lane == 0) {
       // --------------------------------------------------------- MMA issuer
+      // Per stage, both 128-row halves of the weight box against the stage's
+      // B tile, into the two halves of the segment's accumulator slot.
       int i = 0, c = 0;
       bool ok = true;
       for (int jj = j0; jj < j1 && ok; ++jj) {
         const int4 job = __ldg(a.jobs + jj);
         for (int sg = 0; sg < tf_nseg(job) && ok; ++sg, ++c) {
           const TfSeg seg = tf_seg(a, job, sg);
-          const int slot = c % TF_NACC, use = c / TF_NACC;
+          const int slot = c % TF_NSLOT, use = c / TF_NSLOT;
           if (use > 0 && !tf_mbar_wait(&accfree[slot], (uint32_t)((use - 1) & 1), abort_flag, a.status, a.wait_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t dcol = tmem + (uint32_t)(slot * TF_BN);
-          const bool dual = seg.kind == 2;
+          const uint32_t dcol = tmem + (uint32_t)(slot * TF_SLOT_COLS);
+          const uint32_t idesc = seg.kind == 2 ? IDESC2 : IDESC;
           for (int kb = seg.k0; kb < seg.k1; ++kb, ++i) {
             const int s = i % STAGES;
             if (!tf_mbar_wait(&full[s], (uint32_t)((i / STAGES) & 1), abort_flag, a.status, a.wait_ns)) {
@@ -436,13 +450,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
             }
             tc_fence_after();
             uint8_t* st = smem + (size_t)s * TF_STAGE_BYTES;
-            const uint64_t ad = sdesc_k_sw128(smem_u32(st));
-            const uint64_t bd = sdesc_k_sw128(smem_u32(st + TC_A_BYTES));
-            const uint64_t bd1 = sdesc_k_sw128(smem_u32(st + TC_A_BYTES + TF_B_BYTES));
+            const uint64_t bd = sdesc_k_sw128(smem_u32(st + TF_A_BYTES));
 #pragma unroll
-            for (int k = 0; k < TC_BK / 16; ++k) {
-              tc_mma(dcol, ad + 2u * k, bd + 2u * k, IDESC, (kb == seg.k0 && k == 0) ? 0u : 1u);
-              if (dual) tc_mma(dcol, ad + 2u * k, bd1 + 2u * k, IDESC, 1u);
+            for (int h = 0; h < TF_PAIR; ++h) {
+              const uint64_t ad = sdesc_k_sw128(smem_u32(st + h * TC_A_BYTES));
+#pragma unroll
+              for (int k = 0; k < TC_BK / 16; ++k)
+                tc_mma(dcol + (uint32_t)(h * 64), ad + 2u * k, bd + 2u * k, idesc, (kb == seg.k0 && k == 0) ? 0u : 1u);
             }
             tc_commit(&empty[s]);
           }
@@ -481,21 +495,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
     }
     int c = 0;
     bool zero_seen = false;
-    // accumulator c: wait, read its 32 columns, hand the slot back to the MMAs
-    // (one thread waits; the barrier's reduction gives all 128 the same outcome)
-    auto take = [&](float* v) -> bool {
-      const int slot = c % TF_NACC, use = c / TF_NACC;
-      ++c;
+    // accumulator slot of segment c: wait for it (one thread waits; the
+    // barrier's reduction gives all 128 the outcome) ...
+    auto take = [&](int cs) -> bool {
+      const int slot = cs % TF_NSLOT, use = cs / TF_NSLOT;
       bool ok = true;
       if (etid == 0) ok = tf_mbar_wait(&accfull[slot], (uint32_t)(use & 1), abort_flag, a.status, a.wait_ns);
       if (!named_bar_and(1, 128, ok)) return false;
       tc_fence_after();
-      tmem_ld16(tl + (uint32_t)(slot * TF_BN), v);
-      tmem_ld16(tl + (uint32_t)(slot * TF_BN + 16), v + 16);
+      return true;
+    };
+    // ... read half h (32 columns, or 64: hi | lo) ...
+    auto ld_half = [&](int cs, int h, float* v, bool pair64) {
+      const uint32_t col = tl + (uint32_t)((cs % TF_NSLOT) * TF_SLOT_COLS + h * 64);
+      tmem_ld16(col, v);
+      tmem_ld16(col + 16, v + 16);
+      if (pair64) {  // the lo half's product, added to the hi half's
+        float w[TF_BN];
+        tmem_ld16(col + 32, w);
+        tmem_ld16(col + 48, w + 16);
+#pragma unroll
+        for (int t = 0; t < TF_BN; ++t) v[t] += w[t];
+      }
+    };
+    // ... and hand the slot back to the MMAs
+    auto release = [&](int cs) {
       tc_fence_before();
       named_bar_sync(1, 128);
-      if (etid == 0) mbar_arrive(&accfree[slot]);
-      return true;
+      if (etid == 0) mbar_arrive(&accfree[cs % TF_NSLOT]);
     };
     // wait for the flags f[0 .. n) of other CTAs, one thread per flag (the
     // loads in parallel); the barrier's reduction gives all 128 the outcome
@@ -506,114 +533,150 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
       fence_acq_rel_gpu();
       return ok;
     };
-    // a partial accumulator, stored for another CTA, then published
-    auto publish_part = [&](float* base, const float* v, int* flag) {
-#pragma unroll
-      for (int t = 0; t < TF_BN; ++t) __stcg(base + t * 128 + etid, v[t]);
+    auto publish = [&](int* flag) {
       __threadfence();
       named_bar_sync(1, 128);
       if (etid == 0) st_release_gpu(flag, seq);
     };
+    // partial sum [2][32][128] of slot q: element (h, t) of this thread
+    auto part = [&](float* base, int q, int h, int t) { return base + ((size_t)q * TF_PAIR + h) * (TF_BN * 128) + t * 128 + etid; };
 
     for (int jj = j0; jj < j1; ++jj) {
       const int4 job = __ldg(a.jobs + jj);
       const int type = tf_type(job), tile = job.y, id = job.w;
       const int count = (job.x >> 8) & 0xFF, gcount = (job.x >> 16) & 0xFF;
-      float v[TF_BN];
-      if (!take(v)) break;
+      const int cs = c;
+      c += tf_nseg(job);
       if (type == TFJ_Z) {
+        // every piece stores its partial sum; the last K range's piece then
+        // adds all of them in K order (its own last): z = bf16(sum)
+        if (!take(cs)) break;
+#pragma unroll
+        for (int h = 0; h < TF_PAIR; ++h) {
+          float v[TF_BN];
+          ld_half(cs, h, v, false);
+#pragma unroll
+          for (int t = 0; t < TF_BN; ++t) __stcg(part(a.zpart, id, h, t), v[t]);
+        }
+        release(cs);
         if (!((job.x >> 4) & 1)) {
-          publish_part(a.zpart + (size_t)id * TF_TILE_FLOATS, v, a.f_zp + id);
+          publish(a.f_zp + id);
         } else {
-          // the last K range: the other pieces' partial sums in K order, then
-          // this one's; z = bf16(sum)
           const int first = id - count + 1;
+          __threadfence();  // (its own partial, read back below by other threads' loads)
           if (count > 1 && !wait_flags(a.f_zp + first, count - 1)) break;
-          float zs[TF_BN];
 #pragma unroll
-          for (int t = 0; t < TF_BN; ++t) zs[t] = 0.f;
-          for (int q = first; q < id; ++q) {
-            const float* p = a.zpart + (size_t)q * TF_TILE_FLOATS;
-            float pv[TF_BN];  // the loads first, in flight together
+          for (int h = 0; h < TF_PAIR; ++h) {
+            const int r = (tile * TF_PAIR + h) * 128 + etid;
+#pragma unroll 1
+            for (int t0 = 0; t0 < TF_BN; t0 += 8) {
+              // eight tokens of every piece, all loads in flight together
+              float pv[TF_ZMAXP][8];
 #pragma unroll
-            for (int t = 0; t < TF_BN; ++t) pv[t] = __ldcg(p + t * 128 + etid);
+              for (int q = 0; q < TF_ZMAXP; ++q)
 #pragma unroll
-            for (int t = 0; t < TF_BN; ++t) zs[t] += pv[t];
-          }
-          const int r = tile * 128 + etid;
-          if (r < a.R) {
+                for (int t = 0; t < 8; ++t) pv[q][t] = q < count ? __ldcg(part(a.zpart, first + q, h, t0 + t)) : 0.f;
 #pragma unroll
-            for (int t = 0; t < TF_BN; ++t)
-              if (t < rows) a.z[(size_t)t * a.R + r] = __float2bfloat16_rn(t < T ? zs[t] + v[t] : 0.f);
+              for (int t = 0; t < 8; ++t) {
+                float zs = 0.f;
+#pragma unroll
+                for (int q = 0; q < TF_ZMAXP; ++q)
+                  if (q < count) zs += pv[q][t];
+                const int tt = t0 + t;
+                if (r < a.R && tt < rows) a.z[(size_t)tt * a.R + r] = __float2bfloat16_rn(tt < T ? zs : 0.f);
+              }
+            }
           }
           fence_proxy_async_global();  // read by other CTAs' TMA loads
-          __threadfence();
-          named_bar_sync(1, 128);
-          if (etid == 0) st_release_gpu(a.f_z + tile, seq);
+          publish(a.f_z + tile);
         }
       } else if (type == TFJ_MAIN) {
-        // v holds this job's up range: u = it plus the later K ranges'
-        // partial sums, in K order
-        const float bj = a.bias ? __ldg(a.bias + tile * 128 + etid) : 0.f;
+        // slot cs: this job's up range; slot cs + 1: its gate range.  Per
+        // half: g = the earlier K ranges' partial sums, then the gate range,
+        // then the bias, in K order; the TwELL emission; u = the up range
+        // plus the later K ranges' partial sums; h = v·u as hi + lo
         if (count > 0 && !wait_flags(a.f_up + id + gcount, count)) break;
-        for (int q = gcount; q < gcount + count; ++q) {
-          const float* p = a.upart + (size_t)(id + q) * TF_TILE_FLOATS;
+        if (gcount > 0 && !wait_flags(a.f_up + id, gcount)) break;
+        if (!take(cs + 1)) break;  // (the gate range comes after the up range)
+        for (int h = 0; h < TF_PAIR; ++h) {
+          const int p = tile * TF_PAIR + h;     // the 128-neuron tile
+          if (p >= a.tw.n_tiles) break;         // (uniform: the pair's second tile may not exist)
+          const int j = p * 128 + etid;
+          const float bj = a.bias ? __ldg(a.bias + j) : 0.f;
+          float g[TF_BN];
 #pragma unroll
-          for (int t = 0; t < TF_BN; ++t) v[t] += __ldcg(p + t * 128 + etid);
-        }
-        // the gate: the earlier K ranges' partial sums, in K order, then this
-        // job's accumulator, then the bias; the TwELL emission (the kept
-        // values stay staged)
-        float g[TF_BN];
-        if (!take(g)) break;
-        if (gcount > 0) {
-          if (!wait_flags(a.f_up + id, gcount)) break;
-          float gs[TF_BN];
-#pragma unroll
-          for (int t = 0; t < TF_BN; ++t) gs[t] = 0.f;
+          for (int t = 0; t < TF_BN; ++t) g[t] = 0.f;
           for (int q = 0; q < gcount; ++q) {
-            const float* p = a.upart + (size_t)(id + q) * TF_TILE_FLOATS;
+            float pv[TF_BN];
 #pragma unroll
-            for (int t = 0; t < TF_BN; ++t) gs[t] += __ldcg(p + t * 128 + etid);
+            for (int t = 0; t < TF_BN; ++t) pv[t] = __ldcg(part(a.upart, id + q, h, t));
+#pragma unroll
+            for (int t = 0; t < TF_BN; ++t) g[t] += pv[t];
           }
+          {
+            float gv[TF_BN];
+            ld_half(cs + 1, h, gv, false);
 #pragma unroll
-          for (int t = 0; t < TF_BN; ++t) g[t] = gs[t] + g[t];
+            for (int t = 0; t < TF_BN; ++t) g[t] = (gcount > 0 ? g[t] + gv[t] : gv[t]) + bj;
+          }
+          twell_tile32<TF_BN>(a.tw, g, j, 0, etid, scratch, 1);  // (a.tw.bias is null)
+          float u[TF_BN];
+          ld_half(cs, h, u, false);
+          for (int q = gcount; q < gcount + count; ++q) {
+            float pv[TF_BN];
+#pragma unroll
+            for (int t = 0; t < TF_BN; ++t) pv[t] = __ldcg(part(a.upart, id + q, h, t));
+#pragma unroll
+            for (int t = 0; t < TF_BN; ++t) u[t] += pv[t];
+          }
+          const uint32_t* masks = reinterpret_cast<const uint32_t*>(scratch);                 // [32][4]
+          const uint16_t* vals = reinterpret_cast<const uint16_t*>(scratch + TF_BN * 4 * 4);  // [32][TW32_VP]
+          const int wq = etid >> 5, bit = etid & 31;
+#pragma unroll
+          for (int t = 0; t < TF_BN; ++t) {
+            if (t >= rows) break;
+            float hv = 0.f;
+            if (t < T && ((masks[t * 4 + wq] >> bit) & 1u))
+              hv = __uint_as_float((uint32_t)vals[t * TW32_VP + etid] << 16) * u[t];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
+            a.h_hi[(size_t)t * a.tw.F + j] = hi;
+            a.h_lo[(size_t)t * a.tw.F + j] = lo;
+          }
         }
-#pragma unroll
-        for (int t = 0; t < TF_BN; ++t) g[t] += bj;
-        twell_tile32<TF_BN>(a.tw, g, tile * 128 + etid, 0, etid, scratch, 1);  // (a.tw.bias is null)
-        const float* u = v;
-        const uint32_t* masks = reinterpret_cast<const uint32_t*>(scratch);                 // [32][4]
-        const uint16_t* vals = reinterpret_cast<const uint16_t*>(scratch + TF_BN * 4 * 4);  // [32][TW32_VP]
-        const int wq = etid >> 5, bit = etid & 31;
-        const size_t col = (size_t)tile * 128 + etid;
-#pragma unroll
-        for (int t = 0; t < TF_BN; ++t) {
-          if (t >= rows) break;
-          float hv = 0.f;
-          if (t < T && ((masks[t * 4 + wq] >> bit) & 1u))
-            hv = __uint_as_float((uint32_t)vals[t * TW32_VP + etid] << 16) * u[t];
-          const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
-          a.h_hi[(size_t)t * a.tw.F + col] = hi;
-          a.h_lo[(size_t)t * a.tw.F + col] = lo;
-        }
+        release(cs);
+        release(cs + 1);
         fence_proxy_async_global();  // read by other CTAs' TMA loads
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (etid == 0) st_release_gpu(a.f_h + tile, seq);
+        publish(a.f_h + tile);
       } else if (type == TFJ_HELP || type == TFJ_GHELP) {
-        publish_part(a.upart + (size_t)id * TF_TILE_FLOATS, v, a.f_up + id);
+        if (!take(cs)) break;
+#pragma unroll
+        for (int h = 0; h < TF_PAIR; ++h) {
+          float v[TF_BN];
+          ld_half(cs, h, v, false);
+#pragma unroll
+          for (int t = 0; t < TF_BN; ++t) __stcg(part(a.upart, id, h, t), v[t]);
+        }
+        release(cs);
+        publish(a.f_up + id);
       } else {
+        if (!take(cs)) break;
+        float y[TF_PAIR][TF_BN];
+#pragma unroll
+        for (int h = 0; h < TF_PAIR; ++h) ld_half(cs, h, y[h], true);
+        release(cs);
         if (!zero_seen) {  // every CTA's slice of out is zeroed
           if (!wait_flags(a.f_zero, a.n_chunks)) break;
           zero_seen = true;
         }
-        const int colo = tile * 128 + etid;
-        if (colo < a.d) {
 #pragma unroll
-          for (int t = 0; t < TF_BN; ++t)
-            if (t < T) atomicAdd(a.out + (size_t)t * a.d + colo, v[t]);
+        for (int h = 0; h < TF_PAIR; ++h) {
+          const int colo = (tile * TF_PAIR + h) * 128 + etid;
+          if (colo < a.d) {
+#pragma unroll
+            for (int t = 0; t < TF_BN; ++t)
+              if (t < T) atomicAdd(a.out + (size_t)t * a.d + colo, y[h][t]);
+          }
         }
       }
     }

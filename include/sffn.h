@@ -98,9 +98,8 @@ typedef enum { SFFN_ACT_RELU = 0, SFFN_ACT_SILU = 1 } sffn_act;
  *   TILES: tensor-core up and down over every 128-neuron tile that some token
  *          keeps, with the non-kept entries of h zeroed (best when the union
  *          of kept neurons covers most tiles: WINA, T in 16..256).  At
- *          T <= 32 in relu-threshold mode with the low-rank gate (with the
- *          dense gate: SFFN_FLAG_TILE_SINGLE) the whole forward runs as one
- *          persistent launch;
+ *          T <= 32 in relu-threshold mode (dense or low-rank gate) the
+ *          whole forward runs as one persistent launch;
  *   AUTO : ROWS for T <= 8 or T > 256 in relu-threshold mode, TILES otherwise. */
 typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sffn_path;
 
@@ -111,9 +110,6 @@ typedef enum { SFFN_PATH_AUTO = 0, SFFN_PATH_ROWS = 1, SFFN_PATH_TILES = 2 } sff
                                      T <= 32): diagnostics, tests */
 #define SFFN_FLAG_COOPERATIVE 4u  /* launch the single persistent forward with the cooperative
                                      attribute (see sffn_forward) */
-#define SFFN_FLAG_TILE_SINGLE 16u /* dense gate, TILES path at T <= 32: the single persistent
-                                     launch (the default with the low-rank gate only; with the
-                                     dense gate the separate launches measured faster) */
 #define SFFN_FLAG_BACKWARD 8u     /* allocate the workspace of sffn_backward (relu-threshold
                                      mode, dense gate, bf16, no input_k or V) */
 

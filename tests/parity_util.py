@@ -23,14 +23,14 @@ def to_dev(t: Optional[torch.Tensor]):
 
 def make_ffn(inp: synth.Inputs, max_tokens: int, path: str = "auto", C: Optional[int] = None,
              debug_gate: bool = False, separate: bool = False, cooperative: bool = False,
-             backward: bool = False, tile_single: bool = False) -> SparseFFN:
+             backward: bool = False) -> SparseFFN:
     wl = inp.wl
     return SparseFFN(to_dev(inp.W_up), to_dev(inp.W_down), W_gate=to_dev(inp.W_gate), A=to_dev(inp.A),
                      B=to_dev(inp.B), bias=to_dev(inp.bias), mode=wl.mode, act=wl.act,
                      threshold=wl.threshold, k=wl.k,
                      tile_capacity=wl.tile_capacity if C is None else C, max_tokens=max_tokens,
                      path=path, debug_gate=debug_gate, separate=separate, cooperative=cooperative,
-                     input_k=wl.input_k or 0, V=to_dev(inp.V), backward=backward, tile_single=tile_single)
+                     input_k=wl.input_k or 0, V=to_dev(inp.V), backward=backward)
 
 
 @dataclass
@@ -132,7 +132,7 @@ def compare_twell(g: GpuRun, res: oracle.OracleResult, C: int, amb: np.ndarray, 
 
 def check(inp: synth.Inputs, T: Optional[int] = None, path: str = "auto", C: Optional[int] = None,
           res: Optional[oracle.OracleResult] = None, ffn: Optional[SparseFFN] = None,
-          separate: bool = False, tile_single: bool = False) -> dict:
+          separate: bool = False) -> dict:
     wl = inp.wl
     x = inp.x if T is None else inp.x[:T]
     T = x.shape[0]
@@ -145,7 +145,7 @@ def check(inp: synth.Inputs, T: Optional[int] = None, path: str = "auto", C: Opt
                              V=synth.to_f64(inp.V))
     own = ffn is None
     if own:
-        ffn = make_ffn(inp, max_tokens=T, path=path, C=C, separate=separate, tile_single=tile_single)
+        ffn = make_ffn(inp, max_tokens=T, path=path, C=C, separate=separate)
     try:
         g = run_gpu(ffn, x)
     finally:

@@ -61,7 +61,8 @@ SHAPES = [
 @pytest.mark.parametrize("d,F,R,n", SHAPES)
 def test_lists_cover_every_block_once(lib, d, F, R, n):
     lists = schedule(lib, d, F, R, n)
-    kd, P, Rt, Md, Kf = -(-d // 64), F // 128, -(-R // 128), -(-d // 128), F // 64
+    # the kernel's unit is a pair of 128-row tiles
+    kd, P, Rt, Md, Kf = -(-d // 64), -(-(F // 128) // 2), -(-R // 256), -(-d // 256), F // 64
     jobs = [j for L in lists for j in L]
     # z: the pieces of each rank tile, slots consecutive in K order, the last
     # one adds them up
@@ -98,7 +99,7 @@ def test_lists_cover_every_block_once(lib, d, F, R, n):
     # the z pieces are short and spread over the CTAs
     if R:
         zl = [sum(j["k1"] - j["k0"] for j in L if j["type"] == Z) for L in lists]
-        assert max(zl) <= max(8, -(-Rt * kd // n) + 8)
+        assert max(zl) <= max(8, -(-Rt * kd // n) + 8) and max(j["count"] for L in lists for j in L if j["type"] == Z) <= 8
 
 
 @pytest.mark.parametrize("d,F,R,n", SHAPES)
@@ -109,7 +110,7 @@ def test_waits_resolve(lib, d, F, R, n):
     helpers, a DOWN the MAINs of its K range.  Every CTA's zeroing of out
     comes first in its list."""
     lists = schedule(lib, d, F, R, n)
-    Rt = -(-R // 128)
+    Rt = -(-R // 256)
     done_z, done_zt, done_help, done_main = set(), set(), set(), set()
     pos = [0] * n
     progress = True
@@ -137,7 +138,7 @@ def test_waits_resolve(lib, d, F, R, n):
                 elif j["type"] == HELP:
                     done_help.add(j["id"])
                 else:
-                    need = set(range(j["k0"] // 2, (j["k1"] + 1) // 2))
+                    need = set(range(j["k0"] // 4, (j["k1"] + 3) // 4))  # 4 blocks of 64 per pair
                     if not need <= done_main:
                         break
                 pos[c] += 1
