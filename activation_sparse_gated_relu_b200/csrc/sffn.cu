@@ -145,7 +145,7 @@ TfSchedule tf_schedule(int n_chunks, int kd, int kg, int P, int Rt, int Md, int 
     const int k0 = (int)((long long)kd * q / zper), k1 = (int)((long long)kd * (q + 1) / zper);
     const int c = (int)((long long)i * n_chunks / nz);
     if (k1 <= k0) S.ok = false;
-    zjobs[c].push_back(tf_job(TFJ_Z, q == zper - 1 ? 1 : 0, zper, 0, r, k0, k1, i));
+    zjobs[c].push_back(tf_job(TFJ_Z, q >= zper - std::min(TF_ZPARTS, zper) ? 1 : 0, zper, q, r, k0, k1, i));
     zload[c] += k1 - k0;
   }
   S.n_zp = nz;
@@ -781,7 +781,7 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       h->tf_max_jobs = (int)std::max(tf_s0.jobs.size(), tf_s1.jobs.size());
       h->tf_max_help = std::max(tf_s0.n_help, tf_s1.n_help);
       h->tf_max_zp = std::max(tf_s0.n_zp, tf_s1.n_zp);
-      h->tf_flag_ints = h->tf_max_zp + Rt + h->tf_max_help + P2 + h->tf_grid + 1;
+      h->tf_flag_ints = h->tf_max_zp + Rt * TF_ZPARTS + h->tf_max_help + P2 + h->tf_grid + 1;
       e = cudaFuncSetAttribute(k_tile_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, h->tf_smem);
       int nb = 0;
       if (!e) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tile_fused, TC_THREADS, h->tf_smem);
@@ -1240,8 +1240,8 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
   }
 
   // ----------------------------- tile path: one persistent launch at T <= 32
-  // (at 32 tokens, d 4096, d_ff 14336: 89.2 against the separate launches'
-  // 94.2 us with the low-rank gate of rank 512, 86.2 against 102.2 us with
+  // (at 32 tokens, d 4096, d_ff 14336: 77.0 against the separate launches'
+  // 94.2 us with the low-rank gate of rank 512, 86.7 against 102.2 us with
   // the dense gate)
   if (!rows && !h->wina && T <= TF_BN && h->tf_ok && !(D.flags & SFFN_FLAG_SEPARATE)) {
     TfArgs ta{};
@@ -1267,7 +1267,7 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     const int Rt = h->lowrank ? cdiv(h->R, 256) : 0;
     ta.f_zp = h->tf_flags;
     ta.f_z = ta.f_zp + h->tf_max_zp;
-    ta.f_up = ta.f_z + Rt;
+    ta.f_up = ta.f_z + Rt * TF_ZPARTS;
     ta.f_h = ta.f_up + h->tf_max_help;
     ta.f_zero = ta.f_h + P;
     ta.out = out;

@@ -78,9 +78,10 @@ constexpr int TF_ZMAXP = 8;                                // z pieces per rank 
 
 enum : int { TFJ_Z = 0, TFJ_MAIN = 1, TFJ_HELP = 2, TFJ_DOWN = 3, TFJ_GHELP = 4 };
 
-// Job record (int4): x = type | fin << 4 | count << 8 | gcount << 16 (Z:
-// count = pieces of its coordinates, fin = this piece adds them up; MAIN:
-// count = up helpers, gcount = gate helpers), y = tile pair (rank, neuron or
+// Job record (int4): x = type | fin << 4 | count << 8 | gcount << 16.  Z:
+// count = pieces of its rank pair, gcount = this piece's index q among them,
+// fin = it finishes some of the pair's four parts.  MAIN: count = up
+// helpers, gcount = gate helpers.  y = tile pair (rank, neuron or
 // output-column tiles 2y and 2y + 1), z = k0 | k1 << 16 (K blocks; MAIN: its
 // gate range is [k0, gate end), its up range [0, k1)), w = id (Z: its piece
 // slot, consecutive in K order within a rank pair; MAIN: its first helper
@@ -88,6 +89,10 @@ enum : int { TFJ_Z = 0, TFJ_MAIN = 1, TFJ_HELP = 2, TFJ_DOWN = 3, TFJ_GHELP = 4 
 __host__ __device__ inline int4 tf_job(int type, int fin, int count, int gcount, int tile, int k0, int k1, int id) {
   return make_int4(type | (fin << 4) | (count << 8) | (gcount << 16), tile, k0 | (k1 << 16), id);
 }
+// z of a rank pair is finished in four parts (half h = part / 2, tokens
+// 16 (part % 2) .. + 15) by the pair's last min(4, pieces) pieces, part p by
+// finisher p % that count; its flags f_z[4 pair + part]
+constexpr int TF_ZPARTS = 4;
 
 struct TfLayout {
   int stages, bars, scratch, total;
@@ -122,7 +127,7 @@ struct TfArgs {
   __nv_bfloat16* h_hi; // [maxT][F]
   __nv_bfloat16* h_lo;
   int* f_zp;           // [z pieces]  = seq once the piece's partial sum is stored
-  int* f_z;            // [R / 256]   = seq once z of those coordinates is stored
+  int* f_z;            // [R / 256][4] = seq once that part of z is stored
   int* f_up;           // [helper slots] = seq once the helper's partial is stored
   int* f_h;            // [F / 256]   = seq once h of the tile pair is stored
   int* f_zero;         // [n_chunks]  = seq once the CTA's slice of out is zeroed
@@ -138,7 +143,7 @@ enum : int { TFA_GATE = 0, TFA_AT = 1, TFA_UP = 2, TFA_DT = 3 };  // the A opera
 struct TfSeg {
   int amap;  // TFA_*
   int arow, k0, k1;
-  int kind;  // B operand: 0 x; 1 z (flag f_z[kb / 4]); 2 the h pair (flag f_h[kb / 4])
+  int kind;  // B operand: 0 x; 1 z (flags f_z[4 (kb / 4) ..]); 2 the h pair (flag f_h[kb / 4])
 };
 
 __device__ __forceinline__ int tf_type(const int4& j) { return j.x & 15; }
@@ -365,15 +370,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
           if (!abort && ib.seg.kind != 0) {
             const int tile = ib.kb >> 2;  // 4 K blocks of 64 per 256-row pair
             if (ib.seg.kind != hz_kind || tile < hz_lo || tile >= hz_hi) {
-              const int* f = ib.seg.kind == 1 ? a.f_z : a.f_h;
-              const int last = (ib.seg.k1 - 1) >> 2;
+              // flags of up to 8 pairs of h, or 2 pairs of z (four parts each)
+              const int per = ib.seg.kind == 1 ? TF_ZPARTS : 1;
+              const int* f = ib.seg.kind == 1 ? a.f_z + tile * TF_ZPARTS : a.f_h + tile;
+              const int nf = min(8, (((ib.seg.k1 - 1) >> 2) - tile + 1) * per);
               int fv[8];
 #pragma unroll
-              for (int q = 0; q < 8; ++q) fv[q] = tile + q <= last ? ld_relaxed_gpu(f + tile + q) : 0;
-              int n = 0;
+              for (int q = 0; q < 8; ++q) fv[q] = q < nf ? ld_relaxed_gpu(f + q) : 0;
+              int nq = 0;
 #pragma unroll
               for (int q = 0; q < 8; ++q)
-                if (n == q && fv[q] == seq) ++n;
+                if (nq == q && fv[q] == seq) ++nq;
+              const int n = nq / per;  // whole pairs
               if (n == 0) break;
               fence_acq_rel_gpu();          // acquire what those flags' releases published
               fence_proxy_async_global();   // written by generic stores, read by TMA
@@ -548,8 +556,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
       const int cs = c;
       c += tf_nseg(job);
       if (type == TFJ_Z) {
-        // every piece stores its partial sum; the last K range's piece then
-        // adds all of them in K order (its own last): z = bf16(sum)
+        // (the z jobs open the list: every piece stores and publishes its
+        // partial sum before any of them waits, see below)
         if (!take(cs)) break;
 #pragma unroll
         for (int h = 0; h < TF_PAIR; ++h) {
@@ -559,37 +567,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tile_fused(const __grid_const
           for (int t = 0; t < TF_BN; ++t) __stcg(part(a.zpart, id, h, t), v[t]);
         }
         release(cs);
-        if (!((job.x >> 4) & 1)) {
-          publish(a.f_zp + id);
-        } else {
-          const int first = id - count + 1;
-          __threadfence();  // (its own partial, read back below by other threads' loads)
-          if (count > 1 && !wait_flags(a.f_zp + first, count - 1)) break;
-#pragma unroll
-          for (int h = 0; h < TF_PAIR; ++h) {
-            const int r = (tile * TF_PAIR + h) * 128 + etid;
+        publish(a.f_zp + id);
+        const bool last_z = jj + 1 == j1 || tf_type(__ldg(a.jobs + jj + 1)) != TFJ_Z;
+        bool ok = true;
+        for (int jf = j0; last_z && jf <= jj && ok; ++jf) {
+          // the finishers among this list's z pieces: every piece's partial
+          // sum of the rank pair, in K order, for their parts of z
+          const int4 zj = __ldg(a.jobs + jf);
+          if (!((zj.x >> 4) & 1)) continue;
+          const int zq = (zj.x >> 16) & 0xFF, zc = (zj.x >> 8) & 0xFF, zt = zj.y;
+          const int first = zj.w - zq, nfin = min(TF_ZPARTS, zc), f = zq - (zc - nfin);
+          ok = wait_flags(a.f_zp + first, zc);
+          for (int pt = f; pt < TF_ZPARTS && ok; pt += nfin) {
+            const int h = pt >> 1, r = (zt * TF_PAIR + h) * 128 + etid;
 #pragma unroll 1
-            for (int t0 = 0; t0 < TF_BN; t0 += 8) {
+            for (int t0 = (pt & 1) * 16; t0 < (pt & 1) * 16 + 16; t0 += 8) {
               // eight tokens of every piece, all loads in flight together
               float pv[TF_ZMAXP][8];
 #pragma unroll
-              for (int q = 0; q < TF_ZMAXP; ++q)
+              for (int qq = 0; qq < TF_ZMAXP; ++qq)
 #pragma unroll
-                for (int t = 0; t < 8; ++t) pv[q][t] = q < count ? __ldcg(part(a.zpart, first + q, h, t0 + t)) : 0.f;
+                for (int t = 0; t < 8; ++t) pv[qq][t] = qq < zc ? __ldcg(part(a.zpart, first + qq, h, t0 + t)) : 0.f;
 #pragma unroll
               for (int t = 0; t < 8; ++t) {
                 float zs = 0.f;
 #pragma unroll
-                for (int q = 0; q < TF_ZMAXP; ++q)
-                  if (q < count) zs += pv[q][t];
+                for (int qq = 0; qq < TF_ZMAXP; ++qq)
+                  if (qq < zc) zs += pv[qq][t];
                 const int tt = t0 + t;
                 if (r < a.R && tt < rows) a.z[(size_t)tt * a.R + r] = __float2bfloat16_rn(tt < T ? zs : 0.f);
               }
             }
+            fence_proxy_async_global();  // read by other CTAs' TMA loads
+            publish(a.f_z + zt * TF_ZPARTS + pt);
           }
-          fence_proxy_async_global();  // read by other CTAs' TMA loads
-          publish(a.f_z + tile);
         }
+        if (!ok) break;
       } else if (type == TFJ_MAIN) {
         // slot cs: this job's up range; slot cs + 1: its gate range.  Per
         // half: g = the earlier K ranges' partial sums, then the gate range,

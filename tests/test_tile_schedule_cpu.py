@@ -64,14 +64,16 @@ def test_lists_cover_every_block_once(lib, d, F, R, n):
     # the kernel's unit is a pair of 128-row tiles
     kd, P, Rt, Md, Kf = -(-d // 64), -(-(F // 128) // 2), -(-R // 256), -(-d // 256), F // 64
     jobs = [j for L in lists for j in L]
-    # z: the pieces of each rank tile, slots consecutive in K order, the last
-    # one adds them up
+    # z: the pieces of each rank pair, slots consecutive in K order, each
+    # knowing its index; the last min(4, pieces) finish the pair's parts
     for r in range(Rt):
         zs = sorted((j for j in jobs if j["type"] == Z and j["tile"] == r), key=lambda j: j["k0"])
         cover([(j["k0"], j["k1"]) for j in zs], kd)
         assert all(j["count"] == len(zs) for j in zs)
         assert [j["id"] for j in zs] == list(range(zs[0]["id"], zs[0]["id"] + len(zs)))
-        assert [j["fin"] for j in zs] == [0] * (len(zs) - 1) + [1]
+        assert [j["gcount"] for j in zs] == list(range(len(zs)))
+        nfin = min(4, len(zs))
+        assert [j["fin"] for j in zs] == [0] * (len(zs) - nfin) + [1] * nfin
     assert not any(j["type"] == Z for j in jobs) if R == 0 else True
     # each tile: one MAIN holding the end of the gate and the start of the up
     # range; gate helpers before it, up helpers after it, slots consecutive
@@ -105,13 +107,19 @@ def test_lists_cover_every_block_once(lib, d, F, R, n):
 @pytest.mark.parametrize("d,F,R,n", SHAPES)
 def test_waits_resolve(lib, d, F, R, n):
     """Each CTA finishes its jobs in order; a job finishes once what the kernel
-    makes it wait for has finished: a z adder the other pieces of its rank
-    tile, a gate piece (MAIN, GHELP) every z tile (low rank), a MAIN its
-    helpers, a DOWN the MAINs of its K range.  Every CTA's zeroing of out
-    comes first in its list."""
+    makes it wait for has finished: a z finisher every piece of its rank pair
+    (the z pieces, first in every list, publish their partial sums before
+    any of them waits), a gate piece (MAIN, GHELP) every part of z (low
+    rank), a MAIN its helpers, a DOWN the MAINs of its K range.  Every CTA's
+    zeroing of out comes first in its list."""
     lists = schedule(lib, d, F, R, n)
     Rt = -(-R // 256)
     done_z, done_zt, done_help, done_main = set(), set(), set(), set()
+    fin_done = {}
+    for L in lists:
+        for j in L:
+            if j["type"] == Z:
+                done_z.add(j["id"])
     pos = [0] * n
     progress = True
     while progress:
@@ -120,11 +128,13 @@ def test_waits_resolve(lib, d, F, R, n):
             while pos[c] < len(lists[c]):
                 j = lists[c][pos[c]]
                 if j["type"] == Z:
-                    if j["fin"] and not all(q in done_z for q in range(j["id"] - j["count"] + 1, j["id"])):
-                        break
-                    done_z.add(j["id"])
+                    first = j["id"] - j["gcount"]
                     if j["fin"]:
-                        done_zt.add(j["tile"])
+                        if not all(q in done_z for q in range(first, first + j["count"])):
+                            break
+                        fin_done.setdefault(j["tile"], set()).add(j["id"])
+                        if len(fin_done[j["tile"]]) == min(4, j["count"]):
+                            done_zt.add(j["tile"])
                 elif j["type"] == MAIN:
                     if R and len(done_zt) < Rt:
                         break
