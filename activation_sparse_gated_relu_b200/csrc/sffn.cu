@@ -472,6 +472,7 @@ struct sffn_handle : KTiming {
   float* tf_zpart = nullptr;
   int* tf_flags = nullptr;
   int tf_flag_ints = 0, tf_max_jobs = 0, tf_max_zp = 0, tf_max_help = 0;
+  int tf_off_z = 0, tf_off_up = 0, tf_off_h = 0, tf_off_zero = 0;  // flag arrays in tf_flags (ints)
   int tf_smem = 0, tf_grid = 0, tf_chunks = 0;
   int tf_seq = 0;                // the last launch's sequence number
   bool tf_ok = false;
@@ -781,7 +782,12 @@ sffn_status sffn_create(const sffn_desc* desc, void* cuda_stream, sffn_handle** 
       h->tf_max_jobs = (int)std::max(tf_s0.jobs.size(), tf_s1.jobs.size());
       h->tf_max_help = std::max(tf_s0.n_help, tf_s1.n_help);
       h->tf_max_zp = std::max(tf_s0.n_zp, tf_s1.n_zp);
-      h->tf_flag_ints = h->tf_max_zp + Rt * TF_ZPARTS + h->tf_max_help + P2 + h->tf_grid + 1;
+      // flags: z pieces, z parts, helper slots, tile pairs, CTAs (with the hook's extra one)
+      h->tf_off_z = h->tf_max_zp;
+      h->tf_off_up = h->tf_off_z + Rt * TF_ZPARTS;
+      h->tf_off_h = h->tf_off_up + h->tf_max_help;
+      h->tf_off_zero = h->tf_off_h + P2;
+      h->tf_flag_ints = h->tf_off_zero + h->tf_grid + 1;
       e = cudaFuncSetAttribute(k_tile_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, h->tf_smem);
       int nb = 0;
       if (!e) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tile_fused, TC_THREADS, h->tf_smem);
@@ -1264,12 +1270,11 @@ static sffn_status forward_bf16(sffn_handle* h, const void* x, int T, float* out
     ta.z = h->z;
     ta.h_hi = h->h_hi;
     ta.h_lo = h->h_lo;
-    const int Rt = h->lowrank ? cdiv(h->R, 256) : 0;
     ta.f_zp = h->tf_flags;
-    ta.f_z = ta.f_zp + h->tf_max_zp;
-    ta.f_up = ta.f_z + Rt * TF_ZPARTS;
-    ta.f_h = ta.f_up + h->tf_max_help;
-    ta.f_zero = ta.f_h + P;
+    ta.f_z = h->tf_flags + h->tf_off_z;
+    ta.f_up = h->tf_flags + h->tf_off_up;
+    ta.f_h = h->tf_flags + h->tf_off_h;
+    ta.f_zero = h->tf_flags + h->tf_off_zero;
     ta.out = out;
     ta.d = d;
     ta.R = h->R;
