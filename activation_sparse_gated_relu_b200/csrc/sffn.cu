@@ -2216,12 +2216,23 @@ struct sffn_moe_handle : KTiming {
   float* w = nullptr;             // [maxT][top_k]
   float* logits = nullptr;        // [maxT][E]
   int last_T = 0;
+  // the experts' forwards run side by side: expert e on stream e % kMoeStreams,
+  // forked after the router and joined before the combine
+  std::vector<cudaStream_t> es;
+  cudaEvent_t ev_fork = nullptr;
+  std::vector<cudaEvent_t> ev_join;
 };
 
 namespace {
+constexpr int kMoeStreams = 8;
 void moe_free(sffn_moe_handle* h) {
   if (!h) return;
   for (sffn_handle* e : h->experts) sffn_destroy(e);
+  for (cudaStream_t s : h->es)
+    if (s) cudaStreamDestroy(s);
+  for (cudaEvent_t ev : h->ev_join)
+    if (ev) cudaEventDestroy(ev);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   timing_free(h);
   if (h->arena) cudaFree(h->arena);
   delete h;
@@ -2314,6 +2325,23 @@ extern "C" sffn_status sffn_moe_create(const sffn_moe_desc* md, void* cuda_strea
     }
     h->experts.push_back(eh);
   }
+  {
+    const int ns = std::min(h->E, kMoeStreams);
+    bool ok = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < ns && ok; ++i) {
+      cudaStream_t s = nullptr;
+      cudaEvent_t ev = nullptr;
+      ok = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) == cudaSuccess;
+      if (ok) h->es.push_back(s);
+      ok = ok && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess;
+      if (ok) h->ev_join.push_back(ev);
+    }
+    if (!ok) {
+      cudaGetLastError();
+      moe_free(h);
+      return SFFN_ERR_CUDA;
+    }
+  }
   const size_t E = h->E, T = h->maxT, dd = h->d, K = h->top_k;
   Arena ar;
   auto plan = [&](Arena& a) {
@@ -2353,11 +2381,20 @@ extern "C" sffn_status sffn_moe_forward(sffn_moe_handle* h, const void* x, int T
   tmark(h, st, L_MOE_ROUTE);
   if (launch_pdl(k_moe_route, dim3(T), dim3(256), 0, st, 1, ra)) return SFFN_ERR_CUDA;
   tmark_end(h, st);
+  // the experts side by side: each stream waits for the router, the
+  // combine waits for every stream
+  const int ns = (int)h->es.size();
+  if (cudaEventRecord(h->ev_fork, st) != cudaSuccess) return SFFN_ERR_CUDA;
+  for (int i = 0; i < ns; ++i)
+    if (cudaStreamWaitEvent(h->es[i], h->ev_fork, 0) != cudaSuccess) return SFFN_ERR_CUDA;
   for (int e = 0; e < h->E; ++e) {
     const sffn_status s = sffn_forward(h->experts[e], h->xe + (size_t)e * T * h->d, T,
-                                       h->ye + (size_t)e * T * h->d, cuda_stream);
+                                       h->ye + (size_t)e * T * h->d, h->es[e % ns]);
     if (s != SFFN_OK) return s;
   }
+  for (int i = 0; i < ns; ++i)
+    if (cudaEventRecord(h->ev_join[i], h->es[i]) != cudaSuccess || cudaStreamWaitEvent(st, h->ev_join[i], 0) != cudaSuccess)
+      return SFFN_ERR_CUDA;
   tmark_follow(h);
   MoeCombineArgs ca{h->ye, h->sel, h->w, out, T, h->d, h->top_k};
   tmark(h, st, L_MOE_COMBINE);

@@ -450,7 +450,11 @@ typedef struct sffn_moe_handle sffn_moe_handle;
 sffn_status sffn_moe_create(const sffn_moe_desc* desc, void* cuda_stream, sffn_moe_handle** out);
 
 /* y = MoE(x) for T tokens (device x [T][d_model] bf16, out [T][d_model]
- * fp32), asynchronously on cuda_stream; no host synchronisation. */
+ * fp32), asynchronously on cuda_stream; no host synchronisation.  The
+ * experts' forwards run side by side on up to eight streams of the handle,
+ * which wait for the router on cuda_stream and which cuda_stream waits for
+ * before the combine; work queued on cuda_stream after the call is ordered
+ * after all of it. */
 sffn_status sffn_moe_forward(sffn_moe_handle* h, const void* x, int T, float* out, void* cuda_stream);
 
 sffn_status sffn_moe_destroy(sffn_moe_handle* h);
