@@ -2387,14 +2387,17 @@ extern "C" sffn_status sffn_moe_forward(sffn_moe_handle* h, const void* x, int T
   if (cudaEventRecord(h->ev_fork, st) != cudaSuccess) return SFFN_ERR_CUDA;
   for (int i = 0; i < ns; ++i)
     if (cudaStreamWaitEvent(h->es[i], h->ev_fork, 0) != cudaSuccess) return SFFN_ERR_CUDA;
-  for (int e = 0; e < h->E; ++e) {
-    const sffn_status s = sffn_forward(h->experts[e], h->xe + (size_t)e * T * h->d, T,
-                                       h->ye + (size_t)e * T * h->d, h->es[e % ns]);
-    if (s != SFFN_OK) return s;
-  }
+  sffn_status res = SFFN_OK;
+  for (int e = 0; e < h->E && res == SFFN_OK; ++e)
+    res = sffn_forward(h->experts[e], h->xe + (size_t)e * T * h->d, T, h->ye + (size_t)e * T * h->d,
+                       h->es[e % ns]);
+  // joined even after a failed expert, so that the experts already queued
+  // stay ordered before the caller's later work on its stream
   for (int i = 0; i < ns; ++i)
-    if (cudaEventRecord(h->ev_join[i], h->es[i]) != cudaSuccess || cudaStreamWaitEvent(st, h->ev_join[i], 0) != cudaSuccess)
-      return SFFN_ERR_CUDA;
+    if ((cudaEventRecord(h->ev_join[i], h->es[i]) != cudaSuccess ||
+         cudaStreamWaitEvent(st, h->ev_join[i], 0) != cudaSuccess) && res == SFFN_OK)
+      res = SFFN_ERR_CUDA;
+  if (res != SFFN_OK) return res;
   tmark_follow(h);
   MoeCombineArgs ca{h->ye, h->sel, h->w, out, T, h->d, h->top_k};
   tmark(h, st, L_MOE_COMBINE);
