@@ -13,13 +13,15 @@
 // such a pair.
 //
 //   phase 0 (low-rank gate), the K blocks of z = x·A cut into pieces of a
-//   few blocks, each the first job of its CTA (spread over the grid):
-//     Z     a K range of z for 128 rank coordinates, a partial sum stored
-//           and published; the piece of the last K range adds the others'
-//           partial sums and its own in K order, rounds z to bf16 and
-//           publishes it
+//   few blocks, the first jobs of their CTAs (spread over the grid):
+//     Z     a K range of z for 256 rank coordinates, a partial sum stored
+//           and published.  Once every Z piece of its CTA has published,
+//           each of the pair's last min(4, pieces) pieces adds all pieces'
+//           partial sums in K order for its share of the pair's four parts
+//           (a half of the rank coordinates x 16 tokens), rounds them to
+//           bf16 and publishes each part
 //   phase 1, a stream of 64-wide K blocks cut into one equal run per CTA:
-//     MAIN  one 128-neuron tile: the first K range of u = x·W_up^T, then
+//     MAIN  one tile (256 neurons): the first K range of u = x·W_up^T, then
 //           the last K range of the gate GEMM (over W_gate, or over B with z
 //           as the operand; last, so that z has long been published).  The
 //           gate's earlier ranges come from GHELP jobs of the previous CTAs,
@@ -31,8 +33,8 @@
 //     GHELP an earlier K range of one tile's gate, a partial sum
 //     HELP  a later K range of one tile's u, a partial sum
 //   phase 2, the down projection's K blocks cut the same way:
-//     DOWN  a K range of y^T = W_down^T · h^T for 128 output columns, added
-//           into out at L2
+//     DOWN  a K range of y^T = W_down^T · h^T for 256 output columns, added
+//           into out at L2 (after every CTA has zeroed its slice of out)
 //
 // Overflow tokens: the emission holds every kept value of the tile, not only
 // the first C, and u is computed for every token, so a token whose record
