@@ -60,7 +60,10 @@ SHAPES = [
 
 @pytest.mark.parametrize("d,F,R,n", SHAPES)
 def test_lists_cover_every_block_once(lib, d, F, R, n):
-    lists = schedule(lib, d, F, R, n)
+    check_cover(schedule(lib, d, F, R, n), d, F, R, n)
+
+
+def check_cover(lists, d, F, R, n):
     # the kernel's unit is a pair of 128-row tiles
     kd, P, Rt, Md, Kf = -(-d // 64), -(-(F // 128) // 2), -(-R // 256), -(-d // 256), F // 64
     jobs = [j for L in lists for j in L]
@@ -106,13 +109,16 @@ def test_lists_cover_every_block_once(lib, d, F, R, n):
 
 @pytest.mark.parametrize("d,F,R,n", SHAPES)
 def test_waits_resolve(lib, d, F, R, n):
+    check_waits(schedule(lib, d, F, R, n), R, n)
+
+
+def check_waits(lists, R, n):
     """Each CTA finishes its jobs in order; a job finishes once what the kernel
     makes it wait for has finished: a z finisher every piece of its rank pair
     (the z pieces, first in every list, publish their partial sums before
     any of them waits), a gate piece (MAIN, GHELP) every part of z (low
     rank), a MAIN its helpers, a DOWN the MAINs of its K range.  Every CTA's
     zeroing of out comes first in its list."""
-    lists = schedule(lib, d, F, R, n)
     Rt = -(-R // 256)
     done_z, done_zt, done_help, done_main = set(), set(), set(), set()
     fin_done = {}
@@ -173,3 +179,19 @@ def test_rejects_bad_sizes(lib):
     nj = ctypes.c_int(0)
     for args in [(0, 1024, 0, 4), (4096, 1000, 0, 4), (4096, 1024, 65, 4), (4096, 1024, 0, 0), (4100, 1024, 0, 4)]:
         assert lib.sffn_debug_tile_schedule(*args, None, 0, None, ctypes.byref(nj)) == B.SFFN_ERR_INVALID_ARG
+
+
+def test_random_shapes(lib):
+    """Seeded sizes across the accepted range (d a multiple of 8 up to 4096,
+    d_ff a multiple of 128, rank 0 or a multiple of 64, 1 to 160 CTAs): the
+    builder accepts each, every block is covered once and the waits resolve."""
+    import random
+    rng = random.Random(20241203)
+    for _ in range(150):
+        d = 8 * rng.randint(1, 512)
+        F = 128 * rng.randint(1, 224)
+        R = rng.choice([0, 0, 64 * rng.randint(1, 16)])
+        n = rng.choice([1, 2, 3, 7, 32, 64, 100, 132, 148, 149, 160])
+        lists = schedule(lib, d, F, R, n)
+        check_cover(lists, d, F, R, n)
+        check_waits(lists, R, n)
